@@ -1,0 +1,27 @@
+"""Compile the fp64 CPU oracle (plain C, OpenMP) into oracle/liboracle.so.
+
+Test infrastructure: the library it builds is loaded only by the tests, the smoke
+check and the CPU-baseline leg of the benchmark.
+"""
+import os
+import subprocess
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "retnet_oracle.c")
+LIB = os.path.join(HERE, "liboracle.so")
+
+
+def build(force: bool = False) -> str:
+    """Build liboracle.so if it is missing or older than its source; return its path."""
+    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
+        return LIB
+    # -O2 without -ffast-math: IEEE fp64 arithmetic in the order the source states.
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-Wall", "-Wextra",
+           SRC, "-o", LIB + ".tmp", "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(LIB + ".tmp", LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    print(build(force=True))
