@@ -1,0 +1,394 @@
+#!/usr/bin/env python
+"""Benchmark of the retention hot path on B200, one JSON line on stdout.
+
+Step: one chunkwise retention forward (xPos, QK^T/sqrt(d), D~) over one batch of the
+workload "chunkwise forward bf16: batch 8, d_model 1024, h 8, d_k = d_v = 128, seq 2048,
+chunk 64", raw output in bf16, through the C interface.  value = tokens/s of the whole job.
+Inputs rotate over 4 resident sets (4 x 134 MB > the 126 MB L2), so no step re-reads the
+previous step's operands from L2.
+
+Alongside the step (1 GPU only), the same line carries: the decode step on the workload
+"batch 64, h 16, d_k 256, d_v 512, fp32 state" (state GB/s), and, where enabled, the
+long-sequence and MSR workloads.  --impl reference times the fp64 CPU oracle instead.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own batch (weak scaling);
+the path has no exchange step, so the only collectives are the barrier and the max of the
+timed durations.
+"""
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+MAIN = dict(workload="chunkwise_fwd_bf16_b8_L2048_h8_dk128_dv128_B64", batch=8, seqlen=2048, heads=8, d_k=128,
+            d_v=128, chunk=64)
+DECODE = dict(workload="decode_step_b64_h16_dk256_dv512_fp32state", batch=64, heads=16, d_k=256, d_v=512)
+LONG = dict(workload="chunkwise_fwd_bf16_b2_L8192_h16_dk256_dv512", batch=2, seqlen=8192, heads=16, d_k=256, d_v=512)
+MSR = dict(workload="msr_fwd_bf16_b4_L4096_h8_dk256_dv256_B256", batch=4, seqlen=4096, heads=8, d_k=256, d_v=256,
+           chunk=256)
+FLAGS = 1 | 2 | 4  # XPOS | SCALE_SQRT_D | NORM_D
+N_SETS = 4
+
+
+def flops_per_token_head(dk, dv, B):
+    """Algorithmic FLOPs: causal inner-chunk QK^T and PV, cross-chunk Q R, state update K^T V."""
+    return (dk + dv) * (B + 1) + 4 * dk * dv
+
+
+def bytes_per_token_head(dk, dv, elt=2):
+    """Algorithmic HBM bytes: read q, k, v, write o, each once."""
+    return elt * (2 * dk + 2 * dv)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sust=d.get("bf16_tflops_sustained"),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, source="fallback")
+
+
+# ---- clocks during the timed region ----------------------------------------------------------
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML every 10 ms (read-only)."""
+
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, index):
+        self.samples = []
+        self.ok = False
+        self.marks = []
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                rs = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+
+    def mark(self):
+        self.marks.append(time.perf_counter())
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self, t0, t1):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        win = [s for s in self.samples if t0 <= s[0] <= t1]
+        window = "timed region"
+        if len(win) < 3:  # the timed region is shorter than a few samples: use the whole run
+            win = self.samples
+            window = "whole benchmark run (timed region shorter than the sampling interval)"
+        if not win:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        reasons = sorted({name for _, _, r in win for name, bit in self.REASONS.items() if r & bit})
+        return {"sm_mhz": statistics.median(m for _, m, _ in win), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(win), "window": window}
+
+
+# ---- distributed plumbing --------------------------------------------------------------------
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(x, world, device):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---- our arm -------------------------------------------------------------------------------
+
+def make_main_inputs(cfg, device, rank):
+    import torch
+
+    import synth_inputs as si
+    sets = []
+    for i in range(N_SETS):
+        q, k, v = si.qkv(cfg["batch"], cfg["seqlen"], cfg["heads"], cfg["d_k"], cfg["d_v"], 2 + 100 * rank + i,
+                         "bf16")
+        o = torch.empty(cfg["batch"], cfg["seqlen"], cfg["heads"], cfg["d_v"], dtype=torch.bfloat16, device=device)
+        sets.append((q.to(device), k.to(device), v.to(device), o))
+    return sets
+
+
+def run_chunkwise(rn, s, cfg, gamma, theta, stream):
+    q, k, v, o = s
+    rn.retnet_retention_chunkwise(q, k, v, o, gamma, theta, 0, FLAGS, cfg["chunk"], stream=stream)
+
+
+def time_steps(fn, steps, stream):
+    import torch
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(steps):
+        fn(i)
+    end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end) / 1e3  # seconds
+
+
+def bench_decode(rn, device, stream, steps, warmup, peaks):
+    import torch
+
+    import synth_inputs as si
+    c = DECODE
+    b, h, dk, dv = c["batch"], c["heads"], c["d_k"], c["d_v"]
+    S = si.decode_state(b, h, dk, dv, 4).to(device)
+    toks = []
+    for t in range(16):
+        q, k, v = si.decode_token(b, h, dk, dv, 4, t)
+        toks.append((q.to(device), k.to(device), v.to(device)))
+    o = torch.empty(b, h, dv, device=device)
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+
+    def step(i):
+        q, k, v = toks[i % len(toks)]
+        rn.retnet_retention_step(q, k, v, o, S, g, th, i, FLAGS, None, stream)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    secs = time_steps(step, steps, stream)
+    per = secs / steps
+    state_bytes = 2 * b * h * dk * dv * 4
+    io_bytes = b * h * (2 * dk + dv) * 2 + b * h * dv * 4
+    gbs = (state_bytes + io_bytes) / per / 1e9
+    return {"workload": c["workload"], "steps": steps, "us_per_step": per * 1e6,
+            "bytes_per_step": state_bytes + io_bytes, "gbs": gbs, "frac_of_measured_hbm": gbs / peaks["hbm"],
+            "frac_of_8tbs": gbs / 8000.0, "gpu_launches": steps}
+
+
+def oracle_sample(cfg, budget_s):
+    """Size a bounded sample of the workload for the fp64 oracle: whole batch rows (all heads)."""
+    import oracle
+    import synth_inputs as si
+    threads = oracle.num_threads(0)
+    b, L, h, dk, dv = cfg["batch"], cfg["seqlen"], cfg["heads"], cfg["d_k"], cfg["d_v"]
+    q, k, v = si.qkv(1, L, h, dk, dv, 2, "bf16")
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+    t0 = time.perf_counter()
+    oracle.recurrent(q[:, :, :1], k[:, :, :1], v[:, :, :1], g[:1], th, 0, FLAGS)  # one (row, head) pair
+    one = time.perf_counter() - t0
+    rows = int(min(b, max(1, round(budget_s * threads / (one * h)))))
+    q, k, v = si.qkv(rows, L, h, dk, dv, 2, "bf16")
+    desc = (f"{rows} of {b} batch rows (all {h} heads, L={L}, d_k={dk}, d_v={dv}) through the fp64 "
+            f"recurrent-form oracle, OpenMP over (row, head) pairs")
+    return dict(q=q, k=k, v=v, g=g, th=th, rows=rows, L=L, threads=threads, desc=desc)
+
+
+def run_oracle(smp):
+    import oracle
+    t0 = time.perf_counter()
+    oracle.recurrent(smp["q"], smp["k"], smp["v"], smp["g"], smp["th"], 0, FLAGS)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(cfg, budget_s=15.0):
+    """The oracle as it stands, timed on this host's cores on a bounded sample of the workload."""
+    smp = oracle_sample(cfg, budget_s)
+    secs = run_oracle(smp)
+    return {"value": smp["rows"] * smp["L"] / secs, "unit": "tokens/s", "cores": smp["threads"], "kind": "oracle",
+            "sample": smp["desc"], "seconds": secs}
+
+
+def main_ours(args):
+    import torch
+
+    import linear_attention_sequence_chunkwise_b200 as rn
+    import synth_inputs as si
+    world, rank, local = dist_env()
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    device = torch.device("cuda", torch.cuda.current_device())
+    rn.load()
+    peaks = load_peaks()
+    cfg = MAIN
+    b, L, h, dk, dv, B = cfg["batch"], cfg["seqlen"], cfg["heads"], cfg["d_k"], cfg["d_v"], cfg["chunk"]
+    gamma, theta = si.gamma_schedule(h), si.theta_schedule(dk)
+    sets = make_main_inputs(cfg, device, rank)
+    stream = torch.cuda.current_stream()
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+
+    def step(i):
+        run_chunkwise(rn, sets[i % N_SETS], cfg, gamma, theta, stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    t_wall0 = time.perf_counter()
+    secs = time_steps(step, args.steps, stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.perf_counter()
+    barrier(world)
+    secs_max = max_over_ranks(secs, world, device)
+    clk = clocks.summary(t_wall0, t_wall1)
+
+    tokens = b * L * world * args.steps
+    value = tokens / secs_max
+    per_launch = secs / args.steps
+    alg_bytes = b * L * h * bytes_per_token_head(dk, dv)
+    alg_flops = b * L * h * flops_per_token_head(dk, dv, B)
+    achieved_gbs = alg_bytes / per_launch / 1e9
+    tflops = alg_flops / per_launch / 1e12
+    line = {
+        "metric": "retention fwd tokens/s + TFLOP/s (% bf16 peak); decode-step state GB/s",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": secs_max / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": args.dtype_label, "input_dtype": "bf16", "data": "synthetic",
+        "config": {"workload": cfg["workload"], "batch_per_gpu": b, "global_batch": b * world, "seq_len": L,
+                   "heads": h, "d_k": dk, "d_v": dv, "chunk": B, "flags": "xpos|sqrt_d|norm_d",
+                   "out_dtype": "bf16", "l2": f"inputs rotate over {N_SETS} resident sets "
+                                             f"({N_SETS * alg_bytes / 1e6:.0f} MB > 126 MB L2)",
+                   "parallelism": f"dp{world}"},
+        "tflops": tflops, "frac_bf16_peak": tflops * 1e12 / (peaks["bf16"] * 1e12),
+        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm"], "unit": "GB/s",
+                     "frac": achieved_gbs / peaks["hbm"], "traffic": args.traffic,
+                     "peak_source": peaks["source"], "algorithmic_bytes_per_launch": alg_bytes,
+                     "launch_us": per_launch * 1e6},
+        "gpu_launches": args.steps,
+        "clocks": clk,
+    }
+    # e2e: host buffers in pinned memory, copies inside the timed region, through the same C call
+    e2e_steps = max(3, min(args.steps, 50))
+    hq = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in sets[0][:3]]
+    for hx, dx in zip(hq, sets[0][:3]):
+        hx.copy_(dx.cpu())
+    ho = torch.empty(sets[0][3].shape, dtype=torch.bfloat16, pin_memory=True)
+    dq, dk_, dv_, do = sets[0]
+
+    def e2e_step(i):
+        dq.copy_(hq[0], non_blocking=True)
+        dk_.copy_(hq[1], non_blocking=True)
+        dv_.copy_(hq[2], non_blocking=True)
+        run_chunkwise(rn, (dq, dk_, dv_, do), cfg, gamma, theta, stream)
+        ho.copy_(do, non_blocking=True)
+
+    e2e_step(0)
+    torch.cuda.synchronize()
+    barrier(world)
+    e_secs = time_steps(e2e_step, e2e_steps, stream)
+    barrier(world)
+    e_secs = max_over_ranks(e_secs, world, device)
+    line["e2e"] = {"value": b * L * world * e2e_steps / e_secs, "unit": "tokens/s",
+                   "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in hq),
+                   "d2h_bytes_per_step": ho.numel() * ho.element_size(), "steps": e2e_steps}
+    if world == 1 and "decode" in args.sections:
+        line["decode"] = bench_decode(rn, device, stream, args.decode_steps, 3, peaks)
+    clocks.stop()
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main_reference(args):
+    """The oracle on the host cores, on the same workload, metric and unit as our arm."""
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return  # rank 0 alone runs and prints
+    cfg = MAIN
+    smp = oracle_sample(cfg, max(0.5, args.cpu_seconds / max(1, args.steps)))
+    for _ in range(args.warmup):
+        run_oracle(smp)
+    secs = sum(run_oracle(smp) for _ in range(args.steps))
+    value = smp["rows"] * smp["L"] * args.steps / secs
+    line = {"metric": "retention fwd tokens/s + TFLOP/s (% bf16 peak); decode-step state GB/s", "impl": "reference",
+            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg["workload"], "batch": cfg["batch"], "seq_len": cfg["seqlen"],
+                       "heads": cfg["heads"], "d_k": cfg["d_k"], "d_v": cfg["d_v"], "chunk": cfg["chunk"],
+                       "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": smp["threads"], "kind": "oracle",
+                             "sample": "each step: " + smp["desc"]},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--sections", default="main,decode")
+    ap.add_argument("--decode-steps", type=int, default=200)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="ncu dram bytes per launch of the chunkwise kernel, when known for this build")
+    ap.add_argument("--dtype-label", default="f32")
+    a = ap.parse_args(argv)
+    if a.warmup < 3 and a.impl == "ours":
+        a.warmup = 3
+    return a
+
+
+if __name__ == "__main__":
+    args = parse_args()
+    if args.impl == "reference":
+        main_reference(args)
+    else:
+        main_ours(args)

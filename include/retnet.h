@@ -1,0 +1,174 @@
+/*
+ * retnet.h -- C interface of the B200 (sm_100a) RetNet multi-scale retention library
+ * (libretnet.so).
+ *
+ * What it computes.  Retention as defined in "阅读笔记：RetNet" (mzeromiko blog, reading
+ * notes on arXiv 2307.08621):
+ *   - §2.2 Recurrent Mode:   S_n = gamma S_{n-1} + K_n^T V_n,  o_n = Q_n S_n
+ *   - §2.3 Parallel Mode:    O = (Q K^T (.) D) V,  D_nm = gamma^(n-m) for n >= m, else 0,
+ *                            Q = (X W_Q) (.) Theta, K = (X W_K) (.) conj(Theta), Theta_n = e^{in.theta}
+ *   - §2.4 Chunkwise Recurrent Mode: per chunk i of B tokens,
+ *                            R_i = K_[i]^T (V_[i] (.) zeta) + gamma^B R_{i-1},  zeta_r = gamma^(B-1-r)
+ *                            O_[i] = (Q_[i] K_[i]^T (.) D) V_[i] + (Q_[i] R_{i-1}) (.) xi,  xi_r = gamma^(r+1)
+ *   - §三.2 MSR: per-head gamma, Y = GroupNorm_h(heads), out = swish(G) (.) Y
+ *   - §三.3 Normalization: QK^T / sqrt(d), D~ (rows of D divided by the root of their sum),
+ *                          R~ (rows of the score matrix divided by max(|row sum|, 1))
+ *
+ * Readings where the page is silent (the library and its tests follow these):
+ *   - xPos on real tensors: elements (2j, 2j+1) of a head vector are one complex number;
+ *     q and k of the token at absolute position p are both turned by the angle p*theta[j].
+ *     Their real dot product is then Re[(q e^{in.theta})(k e^{im.theta})^dagger], a function
+ *     of n-m only.
+ *   - Positions are 0-based absolute: token t of a call is at p = pos0 + t.  D~ divides row p
+ *     by c_p = sqrt(sum_{j=0..p} gamma^j), the number of decayed tokens seen so far.
+ *   - Chunk rows r are 0-based: xi_r = gamma^(r+1), zeta_r = gamma^(b'-1-r) with b' the
+ *     chunk's actual length (the tail chunk may be shorter than B).
+ *   - The recurrent step updates the state with token n before reading it (D_nn = 1).
+ *   - GroupNorm: groups are heads, biased variance over d_v, eps inside the root, unit affine;
+ *     swish(g) = g * sigmoid(g).
+ *
+ * Layout ("BLHD", dense, row-major, no strides):
+ *   q, k : [batch][seqlen][heads][d_k]     v, o : [batch][seqlen][heads][d_v]
+ *   state: [batch][heads][d_k][d_v] fp32   z    : [batch][heads][d_k] fp32 (key-sum state)
+ *   MSR y, g, out: [tokens][heads][d_v]
+ *
+ * Ownership and memory.  The caller owns every buffer.  Tensor arguments (q, k, v, o, state,
+ * z, y, g, out) are DEVICE pointers on the current CUDA device.  gamma and theta are HOST
+ * pointers, read before the call returns (their values travel to the kernels as launch
+ * parameters).  The library allocates no device memory, frees nothing, and keeps no
+ * per-call state.
+ *
+ * Asynchrony.  Every compute call enqueues its kernels on `stream` (a cudaStream_t; NULL is
+ * the legacy default stream) and returns without synchronising.  Outputs are valid once the
+ * stream reaches that point.
+ *
+ * Errors.  Arguments are checked on the host before any launch; a bad argument returns a
+ * status and enqueues nothing.  A failed launch returns RETNET_ERR_CUDA.  No exception
+ * crosses this interface and no kernel traps.  Devices other than sm_100 return
+ * RETNET_ERR_UNSUPPORTED.
+ *
+ * Precision.  fp32 inputs are computed in fp32 on the CUDA cores.  bf16 inputs of the
+ * chunkwise call, for the shapes listed at retnet_retention_chunkwise, run on the tensor
+ * cores (tcgen05) with fp16 operands and fp32 accumulation: bf16 q, k, v convert to fp16
+ * exactly, the rotated q, k, the masked scores and the chunk state are rounded to fp16 once
+ * each.  fp16 has three more mantissa bits than bf16 and a smaller range, so finite results
+ * need |q|, |k|, |v| < 32768, |q.k| < 32768 * sqrt(d_k) and state entries < 65504.
+ */
+#ifndef RETNET_H
+#define RETNET_H
+
+#include <stdint.h>
+
+/* Exported symbols of libretnet.so (the library is built with hidden default visibility). */
+#if defined(__GNUC__)
+#define RETNET_API __attribute__((visibility("default")))
+#else
+#define RETNET_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    RETNET_OK = 0,
+    RETNET_ERR_NULL_PTR = 1,    /* a required pointer is NULL */
+    RETNET_ERR_BAD_SHAPE = 2,   /* a size is <= 0 (or < 0 where 0 is allowed), or over a limit */
+    RETNET_ERR_BAD_DTYPE = 3,   /* dtype value not in retnet_dtype_t, or combination unsupported */
+    RETNET_ERR_BAD_PARAM = 4,   /* gamma not in (0,1), chunk <= 0, odd d_k with XPOS, eps < 0,
+                                   negative position, unknown flag bits, non-finite theta */
+    RETNET_ERR_UNSUPPORTED = 5, /* e.g. NORM_R on a step call without z, or not an sm_100 device */
+    RETNET_ERR_CUDA = 6         /* a CUDA runtime/driver call or a launch failed */
+} retnet_status_t;
+
+typedef enum { RETNET_F32 = 0, RETNET_BF16 = 1 } retnet_dtype_t;
+
+/* Normalisation / position flags (bitwise OR). */
+enum {
+    RETNET_F_XPOS = 1u,         /* xPos rotation of q and k (§2.3 Theta) */
+    RETNET_F_SCALE_SQRT_D = 2u, /* QK^T / sqrt(d_k) (§三.3) */
+    RETNET_F_NORM_D = 4u,       /* D~ row normalisation (§三.3) */
+    RETNET_F_NORM_R = 8u        /* R~ normalisation by max(|row sum|, 1) (§三.3) */
+};
+
+typedef struct {
+    int64_t batch, seqlen, heads, d_k, d_v;
+} retnet_dims_t;
+
+/* Limits checked on the host (RETNET_ERR_BAD_SHAPE beyond them). */
+#define RETNET_MAX_HEADS 256
+#define RETNET_MAX_DK 512
+#define RETNET_MAX_DV 1024
+
+/*
+ * Parallel form (§2.3 with §三.3): o = ((Q K^T) * s (.) D~) V / max(|row sum|, 1), the flags
+ * choosing which factors apply.  A fresh sequence whose first token sits at absolute
+ * position pos0 >= 0 (pos0 moves the rotation and the D~ row counts; no earlier tokens
+ * contribute).  q, k, v: in_dtype; o: out_dtype.  gamma: host float[heads] in (0,1);
+ * theta: host float[d_k/2] (may be NULL without RETNET_F_XPOS).  seqlen may be 0 (no work).
+ * Cost is O(seqlen^2) per (batch, head).
+ */
+RETNET_API retnet_status_t retnet_retention_parallel(const void* q, const void* k, const void* v, void* o,
+                                          retnet_dims_t dims, retnet_dtype_t in_dtype,
+                                          retnet_dtype_t out_dtype, const float* gamma,
+                                          const float* theta, int64_t pos0, uint32_t flags,
+                                          void* stream);
+
+/*
+ * Chunkwise recurrent form (§2.4) with chunk length `chunk` (> 0); the result equals the
+ * parallel form's up to rounding, and continues from a carried state.
+ *   state_in : device fp32 [batch][heads][d_k][d_v], the state S before the first token
+ *              (the recurrent S_{pos0-1}); NULL means zeros.
+ *   state_out: device fp32, same shape; receives the state after the last token; may be NULL;
+ *              may alias state_in.
+ *   z_in/z_out: device fp32 [batch][heads][d_k], the key-sum state (gamma z + k) that the
+ *              R~ row sum needs across calls; read/written only with RETNET_F_NORM_R; NULL
+ *              means zeros / not written.
+ * Kernels: bf16 q, k, v with d_k in {64, 128, 256}, d_v a multiple of 64 (<= 512) and
+ * chunk in {64, 128, 256, 512} run on the tcgen05 tensor-core kernel; every other case runs
+ * on the fp32 CUDA-core kernel.
+ */
+RETNET_API retnet_status_t retnet_retention_chunkwise(const void* q, const void* k, const void* v, void* o,
+                                           retnet_dims_t dims, retnet_dtype_t in_dtype,
+                                           retnet_dtype_t out_dtype, const float* gamma,
+                                           const float* theta, int64_t pos0, uint32_t flags,
+                                           int64_t chunk, const float* state_in, float* state_out,
+                                           const float* z_in, float* z_out, void* stream);
+
+/*
+ * One recurrent decode step (§2.2) for a whole batch: for the token at absolute position
+ * pos >= 0, S <- gamma S + k^T v in place, then o = (q S) * s / c_pos / max(|s/c_pos q.z|, 1)
+ * as the flags ask (z <- gamma z + k in place with RETNET_F_NORM_R, which requires z).
+ *   q, k: [batch][heads][d_k] in_dtype;  v: [batch][heads][d_v] in_dtype;
+ *   o: [batch][heads][d_v] out_dtype;  state: device fp32 [batch][heads][d_k][d_v], in/out.
+ * The state is read once and written once per call (the call is HBM-bound).  o must not
+ * overlap the state.
+ */
+RETNET_API retnet_status_t retnet_retention_step(const void* q, const void* k, const void* v, void* o,
+                                      int64_t batch, int64_t heads, int64_t d_k, int64_t d_v,
+                                      retnet_dtype_t in_dtype, retnet_dtype_t out_dtype,
+                                      float* state, float* z, const float* gamma,
+                                      const float* theta, int64_t pos, uint32_t flags,
+                                      void* stream);
+
+/*
+ * MSR epilogue (§三.2): for every (token, head) row of d_v values of y, GroupNorm with the
+ * biased variance and eps >= 0 inside the root, unit affine, then multiply by swish(g).
+ *   y, g: [tokens][heads][d_v] in_dtype;  out: same shape, out_dtype (may alias y when the
+ *   dtypes match).  tokens may be 0.  d_v must be a multiple of 8 and <= RETNET_MAX_DV.
+ */
+RETNET_API retnet_status_t retnet_msr_epilogue(const void* y, const void* g, void* out, int64_t tokens,
+                                    int64_t heads, int64_t d_v, float eps, retnet_dtype_t in_dtype,
+                                    retnet_dtype_t out_dtype, void* stream);
+
+/* Static, NUL-terminated description of a status code (never NULL). */
+RETNET_API const char* retnet_status_string(retnet_status_t status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+RETNET_API int retnet_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RETNET_H */

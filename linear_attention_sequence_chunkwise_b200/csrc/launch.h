@@ -1,0 +1,55 @@
+// launch.h -- host-side launchers behind the C interface (internal to libretnet.so).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace retnet {
+
+// Arguments of one chunkwise / parallel retention call, after host validation.
+struct RetentionCall {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  Dims dims;
+  retnet_dtype_t in_dtype, out_dtype;
+  int64_t pos0;
+  uint32_t flags;
+  int64_t chunk;  // == seqlen (or more) for the parallel form
+  bool has_state;  // false for the parallel form: no state is read or written
+  const float* state_in;
+  float* state_out;
+  const float* z_in;
+  float* z_out;
+};
+
+// fp32 CUDA-core kernel: the parallel form (chunk >= seqlen, no state) and the chunkwise
+// form for any shape.
+cudaError_t launch_simt_retention(const RetentionCall& c, const HeadParams& hp, cudaStream_t s);
+
+// tcgen05 tensor-core chunkwise kernel for bf16 inputs; `supported` says whether the shape
+// is one it handles (then it launches and returns the launch status).
+bool tc_chunkwise_supported(const RetentionCall& c);
+cudaError_t launch_tc_chunkwise(const RetentionCall& c, const HeadParams& hp, cudaStream_t s);
+
+struct StepCall {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  int64_t batch, heads, d_k, d_v;
+  retnet_dtype_t in_dtype, out_dtype;
+  float* state;
+  float* z;
+  int64_t pos;
+  uint32_t flags;
+};
+cudaError_t launch_step(const StepCall& c, const HeadParams& hp, cudaStream_t s);
+
+cudaError_t launch_msr_epilogue(const void* y, const void* g, void* out, int64_t tokens, int64_t heads,
+                                int64_t d_v, float eps, retnet_dtype_t in_dtype, retnet_dtype_t out_dtype,
+                                cudaStream_t s);
+
+}  // namespace retnet

@@ -1,0 +1,170 @@
+// retnet_abi.cu -- the extern "C" entry points of libretnet.so (declared in include/retnet.h).
+//
+// Each entry point checks its arguments on the host, fills the per-head parameter block
+// (gamma, log2 gamma, theta) from the caller's host arrays, and enqueues the kernels on the
+// caller's stream.  Nothing is allocated; no state survives the call.
+#include <math.h>
+
+#include "launch.h"
+
+using namespace retnet;
+
+namespace {
+
+constexpr uint32_t kAllFlags = RETNET_F_XPOS | RETNET_F_SCALE_SQRT_D | RETNET_F_NORM_D | RETNET_F_NORM_R;
+
+bool valid_dtype(retnet_dtype_t t) { return t == RETNET_F32 || t == RETNET_BF16; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// The current device must be an sm_100 part (B200); the kernels are built for sm_100a only.
+retnet_status_t check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return RETNET_ERR_CUDA;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return RETNET_ERR_CUDA;
+  if (major != 10 || minor != 0) return RETNET_ERR_UNSUPPORTED;
+  return RETNET_OK;
+}
+
+// gamma in (0, 1) per head; theta finite per pair when XPOS is set.
+retnet_status_t fill_params(HeadParams* hp, const float* gamma, const float* theta, int64_t heads, int64_t d_k,
+                            uint32_t flags) {
+  if (!gamma) return RETNET_ERR_NULL_PTR;
+  if ((flags & RETNET_F_XPOS) && !theta) return RETNET_ERR_NULL_PTR;
+  for (int64_t h = 0; h < heads; ++h) {
+    const float g = gamma[h];
+    if (!(g > 0.f && g < 1.f)) return RETNET_ERR_BAD_PARAM;
+    hp->gamma[h] = g;
+    hp->log2g[h] = static_cast<float>(log2(static_cast<double>(g)));
+  }
+  const int64_t pairs = d_k / 2;
+  for (int64_t j = 0; j < pairs; ++j) {
+    float t = (flags & RETNET_F_XPOS) ? theta[j] : 0.f;
+    if (!isfinite(t)) return RETNET_ERR_BAD_PARAM;
+    hp->theta[j] = t;
+  }
+  return RETNET_OK;
+}
+
+retnet_status_t check_common(const retnet_dims_t& d, retnet_dtype_t in_dtype, retnet_dtype_t out_dtype,
+                             int64_t pos0, uint32_t flags, bool allow_zero_len) {
+  if (!valid_dtype(in_dtype) || !valid_dtype(out_dtype)) return RETNET_ERR_BAD_DTYPE;
+  if (d.batch <= 0 || d.heads <= 0 || d.d_k <= 0 || d.d_v <= 0) return RETNET_ERR_BAD_SHAPE;
+  if (d.seqlen < 0 || (!allow_zero_len && d.seqlen == 0)) return RETNET_ERR_BAD_SHAPE;
+  if (d.heads > RETNET_MAX_HEADS || d.d_k > RETNET_MAX_DK || d.d_v > RETNET_MAX_DV) return RETNET_ERR_BAD_SHAPE;
+  if (d.batch > 65535 || d.heads > 65535) return RETNET_ERR_BAD_SHAPE;  // grid y/z limits
+  if (flags & ~kAllFlags) return RETNET_ERR_BAD_PARAM;
+  if ((flags & RETNET_F_XPOS) && (d.d_k & 1)) return RETNET_ERR_BAD_PARAM;
+  if (pos0 < 0) return RETNET_ERR_BAD_PARAM;
+  return RETNET_OK;
+}
+
+retnet_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? RETNET_OK : RETNET_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* retnet_status_string(retnet_status_t status) {
+  switch (status) {
+    case RETNET_OK: return "ok";
+    case RETNET_ERR_NULL_PTR: return "a required pointer is NULL";
+    case RETNET_ERR_BAD_SHAPE: return "bad shape (non-positive size or over a limit)";
+    case RETNET_ERR_BAD_DTYPE: return "bad or unsupported dtype";
+    case RETNET_ERR_BAD_PARAM: return "bad parameter (gamma, theta, chunk, eps, position, flags or alignment)";
+    case RETNET_ERR_UNSUPPORTED: return "unsupported (device is not sm_100, or option needs a missing buffer)";
+    case RETNET_ERR_CUDA: return "CUDA call or kernel launch failed";
+  }
+  return "unknown status";
+}
+
+int retnet_version(void) { return 100; }
+
+retnet_status_t retnet_retention_parallel(const void* q, const void* k, const void* v, void* o, retnet_dims_t dims,
+                                          retnet_dtype_t in_dtype, retnet_dtype_t out_dtype, const float* gamma,
+                                          const float* theta, int64_t pos0, uint32_t flags, void* stream) {
+  retnet_status_t st = check_common(dims, in_dtype, out_dtype, pos0, flags, true);
+  if (st != RETNET_OK) return st;
+  if (dims.seqlen > 0 && (!q || !k || !v || !o)) return RETNET_ERR_NULL_PTR;
+  HeadParams hp;
+  if ((st = fill_params(&hp, gamma, theta, dims.heads, dims.d_k, flags)) != RETNET_OK) return st;
+  if (dims.seqlen == 0) return RETNET_OK;
+  if ((st = check_device()) != RETNET_OK) return st;
+  RetentionCall c{q, k, v, o, Dims{dims.batch, dims.seqlen, dims.heads, dims.d_k, dims.d_v}, in_dtype, out_dtype,
+                  pos0, flags, dims.seqlen, false, nullptr, nullptr, nullptr, nullptr};
+  return from_cuda(launch_simt_retention(c, hp, static_cast<cudaStream_t>(stream)));
+}
+
+retnet_status_t retnet_retention_chunkwise(const void* q, const void* k, const void* v, void* o, retnet_dims_t dims,
+                                           retnet_dtype_t in_dtype, retnet_dtype_t out_dtype, const float* gamma,
+                                           const float* theta, int64_t pos0, uint32_t flags, int64_t chunk,
+                                           const float* state_in, float* state_out, const float* z_in,
+                                           float* z_out, void* stream) {
+  retnet_status_t st = check_common(dims, in_dtype, out_dtype, pos0, flags, true);
+  if (st != RETNET_OK) return st;
+  if (chunk <= 0) return RETNET_ERR_BAD_PARAM;
+  if (dims.seqlen > 0 && (!q || !k || !v || !o)) return RETNET_ERR_NULL_PTR;
+  HeadParams hp;
+  if ((st = fill_params(&hp, gamma, theta, dims.heads, dims.d_k, flags)) != RETNET_OK) return st;
+  if ((st = check_device()) != RETNET_OK) return st;
+  RetentionCall c{q, k, v, o, Dims{dims.batch, dims.seqlen, dims.heads, dims.d_k, dims.d_v}, in_dtype, out_dtype,
+                  pos0, flags, chunk, true, state_in, state_out, z_in, z_out};
+  if (dims.seqlen == 0) {
+    // No tokens: the state passes through unchanged.
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t sbytes = sizeof(float) * (size_t)(dims.batch * dims.heads * dims.d_k * dims.d_v);
+    const size_t zbytes = sizeof(float) * (size_t)(dims.batch * dims.heads * dims.d_k);
+    if (state_out && state_out != state_in) {
+      cudaError_t e = state_in ? cudaMemcpyAsync(state_out, state_in, sbytes, cudaMemcpyDeviceToDevice, s)
+                               : cudaMemsetAsync(state_out, 0, sbytes, s);
+      if (e != cudaSuccess) return RETNET_ERR_CUDA;
+    }
+    if ((flags & RETNET_F_NORM_R) && z_out && z_out != z_in) {
+      cudaError_t e = z_in ? cudaMemcpyAsync(z_out, z_in, zbytes, cudaMemcpyDeviceToDevice, s)
+                           : cudaMemsetAsync(z_out, 0, zbytes, s);
+      if (e != cudaSuccess) return RETNET_ERR_CUDA;
+    }
+    return RETNET_OK;
+  }
+  if (tc_chunkwise_supported(c)) return from_cuda(launch_tc_chunkwise(c, hp, static_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_simt_retention(c, hp, static_cast<cudaStream_t>(stream)));
+}
+
+retnet_status_t retnet_retention_step(const void* q, const void* k, const void* v, void* o, int64_t batch,
+                                      int64_t heads, int64_t d_k, int64_t d_v, retnet_dtype_t in_dtype,
+                                      retnet_dtype_t out_dtype, float* state, float* z, const float* gamma,
+                                      const float* theta, int64_t pos, uint32_t flags, void* stream) {
+  retnet_dims_t d{batch, 1, heads, d_k, d_v};
+  retnet_status_t st = check_common(d, in_dtype, out_dtype, pos, flags, false);
+  if (st != RETNET_OK) return st;
+  if (batch * heads > 0x7fffffffLL) return RETNET_ERR_BAD_SHAPE;
+  if (!q || !k || !v || !o || !state) return RETNET_ERR_NULL_PTR;
+  if ((flags & RETNET_F_NORM_R) && !z) return RETNET_ERR_UNSUPPORTED;
+  if (!aligned16(state)) return RETNET_ERR_BAD_PARAM;
+  HeadParams hp;
+  if ((st = fill_params(&hp, gamma, theta, heads, d_k, flags)) != RETNET_OK) return st;
+  if ((st = check_device()) != RETNET_OK) return st;
+  StepCall c{q, k, v, o, batch, heads, d_k, d_v, in_dtype, out_dtype, state, z, pos, flags};
+  return from_cuda(launch_step(c, hp, static_cast<cudaStream_t>(stream)));
+}
+
+retnet_status_t retnet_msr_epilogue(const void* y, const void* g, void* out, int64_t tokens, int64_t heads,
+                                    int64_t d_v, float eps, retnet_dtype_t in_dtype, retnet_dtype_t out_dtype,
+                                    void* stream) {
+  if (!valid_dtype(in_dtype) || !valid_dtype(out_dtype)) return RETNET_ERR_BAD_DTYPE;
+  if (tokens < 0 || heads <= 0 || d_v <= 0 || d_v > RETNET_MAX_DV || (d_v % 8) != 0) return RETNET_ERR_BAD_SHAPE;
+  if (!(eps >= 0.f) || !isfinite(eps)) return RETNET_ERR_BAD_PARAM;
+  if (!y || !g || !out) return RETNET_ERR_NULL_PTR;
+  if (!aligned16(y) || !aligned16(g) || !aligned16(out)) return RETNET_ERR_BAD_PARAM;
+  if ((tokens * heads + 7) / 8 > 0x7fffffffLL) return RETNET_ERR_BAD_SHAPE;
+  if (tokens == 0) return RETNET_OK;
+  retnet_status_t st = check_device();
+  if (st != RETNET_OK) return st;
+  return from_cuda(launch_msr_epilogue(y, g, out, tokens, heads, d_v, eps, in_dtype, out_dtype,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

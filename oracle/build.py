@@ -16,10 +16,11 @@ def build(force: bool = False) -> str:
     if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
         return LIB
     # -O2 without -ffast-math: IEEE fp64 arithmetic in the order the source states.
+    tmp = f"{LIB}.{os.getpid()}.tmp"
     cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-Wall", "-Wextra",
-           SRC, "-o", LIB + ".tmp", "-lm"]
+           SRC, "-o", tmp, "-lm"]
     subprocess.run(cmd, check=True)
-    os.replace(LIB + ".tmp", LIB)
+    os.replace(tmp, LIB)
     return LIB
 
 

@@ -1,0 +1,139 @@
+"""Host-side checks of the C interface (no GPU needed, no compute calls).
+
+The library must load here, export every function include/retnet.h declares, and reject
+bad arguments with the documented status before it touches a device.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import linear_attention_sequence_chunkwise_b200 as rn
+from linear_attention_sequence_chunkwise_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "retnet.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    _build.build()
+    return rn.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"RETNET_API\s+[\w\s\*]+?\b(retnet_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_interface():
+    names = declared_functions()
+    assert set(names) == set(rn.EXPORTS), names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", _build.LIB], capture_output=True, text=True, check=True)
+    exported = set(re.findall(r"\bT (retnet_\w+)", out.stdout))
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(lib, name)
+
+
+def test_header_compiles_as_c():
+    src = '#include "retnet.h"\nint main(void){ retnet_dims_t d = {1,2,3,4,5}; return (int)d.batch - 1; }\n'
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), "-x", "c", "-",
+                        "-fsyntax-only"], input=src, text=True, capture_output=True)
+    assert r.returncode == 0, r.stderr
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        s = rn.retnet_status_string(code)
+        assert isinstance(s, str) and len(s) > 0
+    assert rn.retnet_status_string(99) == "unknown status"
+    assert lib.retnet_version() >= 100
+
+
+# Fake, never-dereferenced device addresses: every call below must fail validation first.
+FAKE = 0x10000
+
+
+def _gamma(h, val=0.9):
+    return np.full(h, val, dtype=np.float32)
+
+
+def _par(lib, dims, gamma, theta=None, flags=0, q=FAKE, in_dt=0, out_dt=0, pos0=0):
+    g = np.ascontiguousarray(gamma, dtype=np.float32)
+    th = None if theta is None else np.ascontiguousarray(theta, dtype=np.float32)
+    return lib.retnet_retention_parallel(q, FAKE, FAKE, FAKE, rn.Dims(*dims), in_dt, out_dt,
+                                         g.ctypes.data_as(rn._fp), None if th is None else th.ctypes.data_as(rn._fp),
+                                         pos0, flags, None)
+
+
+def test_parallel_validation(lib):
+    ok = (1, 8, 2, 4, 4)
+    assert _par(lib, ok, _gamma(2), q=0) == 1                            # NULL q
+    assert _par(lib, (0, 8, 2, 4, 4), _gamma(2)) == 2                    # batch 0
+    assert _par(lib, (1, 8, 2, 0, 4), _gamma(2)) == 2                    # d_k 0
+    assert _par(lib, (1, 8, 2, 4, 2000), _gamma(2)) == 2                 # d_v over the limit
+    assert _par(lib, (1, 8, 300, 4, 4), _gamma(300)) == 2                # heads over the limit
+    assert _par(lib, ok, _gamma(2), in_dt=7) == 3                        # bad dtype
+    assert _par(lib, ok, _gamma(2, 1.0)) == 4                            # gamma = 1
+    assert _par(lib, ok, _gamma(2, 0.0)) == 4                            # gamma = 0
+    assert _par(lib, ok, np.array([0.9, np.nan], np.float32)) == 4       # gamma NaN
+    assert _par(lib, ok, _gamma(2), flags=16) == 4                       # unknown flag bit
+    assert _par(lib, (1, 8, 2, 5, 4), _gamma(2), np.ones(2), flags=rn.F_XPOS) == 4  # odd d_k with xPos
+    assert _par(lib, ok, _gamma(2), None, flags=rn.F_XPOS) == 1          # xPos without theta
+    assert _par(lib, ok, _gamma(2), np.array([1.0, np.inf]), flags=rn.F_XPOS) == 4  # theta inf
+    assert _par(lib, ok, _gamma(2), pos0=-1) == 4                        # negative position
+    assert _par(lib, (1, 0, 2, 4, 4), _gamma(2)) == 0                    # empty sequence: no work
+
+
+def test_chunkwise_and_step_validation(lib):
+    g = _gamma(2)
+    gp = g.ctypes.data_as(rn._fp)
+    d = rn.Dims(1, 8, 2, 4, 4)
+    # chunk <= 0
+    assert lib.retnet_retention_chunkwise(FAKE, FAKE, FAKE, FAKE, d, 0, 0, gp, None, 0, 0, 0, None, None, None,
+                                          None, None) == 4
+    # NULL o
+    assert lib.retnet_retention_chunkwise(FAKE, FAKE, FAKE, None, d, 0, 0, gp, None, 0, 0, 16, None, None, None,
+                                          None, None) == 1
+    # step: NORM_R without z
+    assert lib.retnet_retention_step(FAKE, FAKE, FAKE, FAKE, 1, 2, 4, 4, 0, 0, FAKE, None, gp, None, 0,
+                                     rn.F_NORM_R, None) == 5
+    # step: misaligned state
+    assert lib.retnet_retention_step(FAKE, FAKE, FAKE, FAKE, 1, 2, 4, 4, 0, 0, FAKE + 4, None, gp, None, 0, 0,
+                                     None) == 4
+    # step: NULL state
+    assert lib.retnet_retention_step(FAKE, FAKE, FAKE, FAKE, 1, 2, 4, 4, 0, 0, None, None, gp, None, 0, 0,
+                                     None) == 1
+    # step: negative position
+    assert lib.retnet_retention_step(FAKE, FAKE, FAKE, FAKE, 1, 2, 4, 4, 0, 0, FAKE, None, gp, None, -3, 0,
+                                     None) == 4
+
+
+def test_epilogue_validation(lib):
+    f = lib.retnet_msr_epilogue
+    assert f(FAKE, FAKE, FAKE, 4, 2, 12, 1e-5, 0, 0, None) == 2          # d_v not a multiple of 8
+    assert f(FAKE, FAKE, FAKE, 4, 2, 16, -1.0, 0, 0, None) == 4          # eps < 0
+    assert f(FAKE, FAKE, FAKE, 4, 2, 16, float("nan"), 0, 0, None) == 4  # eps NaN
+    assert f(None, FAKE, FAKE, 4, 2, 16, 1e-5, 0, 0, None) == 1          # NULL y
+    assert f(FAKE + 2, FAKE, FAKE, 4, 2, 16, 1e-5, 0, 0, None) == 4      # misaligned
+    assert f(FAKE, FAKE, FAKE, 4, 2, 16, 1e-5, 5, 0, None) == 3          # bad dtype
+    assert f(FAKE, FAKE, FAKE, 0, 2, 16, 1e-5, 0, 0, None) == 0          # no tokens: no work
+
+
+def test_binding_raises_without_library(tmp_path):
+    import importlib
+    mod = importlib.import_module("linear_attention_sequence_chunkwise_b200")
+    saved = mod._lib
+    try:
+        mod._lib = None
+        with pytest.raises(RuntimeError, match="not found"):
+            mod.load(str(tmp_path / "missing.so"))
+    finally:
+        mod._lib = saved
