@@ -261,6 +261,8 @@ def main_ours(args):
     cfg = MAIN
     b, L, h, dk, dv, B = cfg["batch"], cfg["seqlen"], cfg["heads"], cfg["d_k"], cfg["d_v"], cfg["chunk"]
     gamma, theta = si.gamma_schedule(h), si.theta_schedule(dk)
+    path = rn.retnet_chunkwise_kernel((b, L, h, dk), dv, rn.BF16, FLAGS, B, gamma)
+    dtype_label = "f16" if path == 1 else "f32"  # arithmetic type of the kernel that runs
     sets = make_main_inputs(cfg, device, rank)
     stream = torch.cuda.current_stream()
     clocks = ClockSampler(torch.cuda.current_device())
@@ -293,7 +295,9 @@ def main_ours(args):
         "metric": "retention fwd tokens/s + TFLOP/s (% bf16 peak); decode-step state GB/s",
         "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": secs_max / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": args.dtype_label, "input_dtype": "bf16", "data": "synthetic",
+        "vs_baseline": None, "dtype": dtype_label, "input_dtype": "bf16",
+        "kernel": "tcgen05 tensor-core chunkwise" if path == 1 else "fp32 CUDA-core chunkwise",
+        "data": "synthetic",
         "config": {"workload": cfg["workload"], "batch_per_gpu": b, "global_batch": b * world, "seq_len": L,
                    "heads": h, "d_k": dk, "d_v": dv, "chunk": B, "flags": "xpos|sqrt_d|norm_d",
                    "out_dtype": "bf16", "l2": f"inputs rotate over {N_SETS} resident sets "
@@ -379,7 +383,6 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu dram bytes per launch of the chunkwise kernel, when known for this build")
-    ap.add_argument("--dtype-label", default="f32")
     a = ap.parse_args(argv)
     if a.warmup < 3 and a.impl == "ours":
         a.warmup = 3

@@ -161,6 +161,24 @@ RETNET_API retnet_status_t retnet_msr_epilogue(const void* y, const void* g, voi
                                     int64_t heads, int64_t d_v, float eps, retnet_dtype_t in_dtype,
                                     retnet_dtype_t out_dtype, void* stream);
 
+/*
+ * Which kernel retnet_retention_chunkwise runs for these arguments (host-only decision, no
+ * device access): 1 = the tcgen05 tensor-core kernel, 0 = the fp32 CUDA-core kernel,
+ * negative = the arguments would be rejected (the negated status).  Device pointers that
+ * are not 16-byte aligned also send a call to the CUDA-core kernel; this query assumes
+ * aligned buffers.  gamma: host float[heads].
+ */
+RETNET_API int retnet_chunkwise_kernel(retnet_dims_t dims, retnet_dtype_t in_dtype, uint32_t flags, int64_t chunk,
+                                       const float* gamma);
+
+/*
+ * Number of bounded waits that gave up inside the tensor-core kernel since the last clear
+ * (a kernel that hits one abandons its output, releases what it holds and returns rather
+ * than hang).  Synchronises with the device.  With clear != 0 the count is reset to 0.
+ * Returns RETNET_OK or RETNET_ERR_CUDA; *count receives the value before any clear.
+ */
+RETNET_API retnet_status_t retnet_debug_wait_timeouts(unsigned int* count, int clear);
+
 /* Static, NUL-terminated description of a status code (never NULL). */
 RETNET_API const char* retnet_status_string(retnet_status_t status);
 

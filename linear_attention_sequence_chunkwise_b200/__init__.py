@@ -31,7 +31,8 @@ BF16 = 1
 STATUS = {0: "RETNET_OK", 1: "RETNET_ERR_NULL_PTR", 2: "RETNET_ERR_BAD_SHAPE", 3: "RETNET_ERR_BAD_DTYPE",
           4: "RETNET_ERR_BAD_PARAM", 5: "RETNET_ERR_UNSUPPORTED", 6: "RETNET_ERR_CUDA"}
 EXPORTS = ("retnet_retention_parallel", "retnet_retention_chunkwise", "retnet_retention_step",
-           "retnet_msr_epilogue", "retnet_status_string", "retnet_version")
+           "retnet_msr_epilogue", "retnet_chunkwise_kernel", "retnet_debug_wait_timeouts", "retnet_status_string",
+           "retnet_version")
 
 
 class RetnetError(RuntimeError):
@@ -72,6 +73,10 @@ def load(path: str = None):
     for name in ("retnet_retention_parallel", "retnet_retention_chunkwise", "retnet_retention_step",
                  "retnet_msr_epilogue"):
         getattr(lib, name).restype = _i32
+    lib.retnet_chunkwise_kernel.argtypes = [Dims, _i32, _u32, _i64, _fp]
+    lib.retnet_chunkwise_kernel.restype = _i32
+    lib.retnet_debug_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint), _i32]
+    lib.retnet_debug_wait_timeouts.restype = _i32
     lib.retnet_status_string.argtypes = [_i32]
     lib.retnet_status_string.restype = ctypes.c_char_p
     lib.retnet_version.argtypes = []
@@ -209,6 +214,21 @@ def retnet_msr_epilogue(y, g, out, heads, eps=1e-5, stream=None):
     tokens = total // (heads * dv)
     _check(load().retnet_msr_epilogue(_ptr(y), _ptr(g), _ptr(out), tokens, heads, dv, float(eps), _dtype_code(y),
                                       _dtype_code(out), _stream(stream)))
+
+
+def retnet_chunkwise_kernel(shape_qk, d_v, in_dtype, flags, chunk, gamma):
+    """1 if a chunkwise call of this shape runs on the tensor-core kernel, 0 for the CUDA-core
+    kernel, negative (-status) if it would be rejected.  shape_qk = (batch, L, heads, d_k)."""
+    b, L, h, dk = shape_qk
+    g = _host_f32(gamma, h)
+    return load().retnet_chunkwise_kernel(Dims(b, L, h, dk, d_v), int(in_dtype), int(flags), int(chunk), _fptr(g))
+
+
+def retnet_debug_wait_timeouts(clear=True):
+    """Bounded waits that gave up in the tensor-core kernel since the last clear (synchronises)."""
+    c = ctypes.c_uint(0)
+    _check(load().retnet_debug_wait_timeouts(ctypes.byref(c), 1 if clear else 0))
+    return c.value
 
 
 # ---- allocating conveniences (torch.empty for the outputs, then the calls above) ----------

@@ -1,12 +1,625 @@
-// chunkwise_tc.cu -- tcgen05 tensor-core chunkwise retention kernel (bf16 inputs).
+// chunkwise_tc.cu -- tcgen05 tensor-core kernel for the chunkwise recurrent form of retention
+// ("阅读笔记：RetNet" (mzeromiko blog) §2.4 Chunkwise Recurrent Mode, with the §2.3 xPos
+// rotation and the §三.3 QK^T/sqrt(d) and D~ normalisations), bf16 inputs.
+//
+// One CTA owns one (batch, head, 64-wide slice of d_v) and walks the chunks of B = T tokens
+// in order, carrying its slice of the chunk state R (d_k x 64, fp32) in tensor memory.
+//
+// Scaled operands.  With xi_r = gamma^(r+1) and zeta_c = gamma^(b'-1-c) (b' the chunk's
+// length), the kernel stages Qx = xi (.) rot(q) and Kz = zeta (.) rot(k) in fp16.  Then
+//   Qx Kz^T = gamma^(b' + r - c) (Q K^T)         ->  P = (Qx Kz^T) * gamma^(-b') (.) causal mask
+//   Qx R_{i-1} = (Q R_{i-1}) (.) xi                   (the cross-chunk term, as written)
+//   Kz^T V = K^T (V (.) zeta)                         (the state increment, as written)
+// so O = P V + Qx R_{i-1} accumulates in one TMEM tile and R_i = gamma^b' R_{i-1} + Kz^T V.
+// All fp16 operands stay in the normal range when gamma^B >= 2^-12; the host sends other
+// heads/chunk sizes to the CUDA-core kernel.
+//
+// Warp roles (320 threads):
+//   warps 0-3  TMEM warpgroup: S -> P (mask, rescale, fp16 to smem); state update
+//              (R_i from TMEM -> fp16 copy in smem for the next cross term, gamma^b' R_i back
+//              to TMEM as the base of the next accumulation); epilogue (row scales, store O).
+//   warps 4-7  converters: in place over each TMA-staged chunk, rotate q and k by the xPos
+//              angle (pairs (2j, 2j+1)), scale by xi / zeta, convert bf16 -> fp16 (V exact).
+//   warp 8     TMA producer (Q, K, V tiles, 128-byte swizzle, no multicast).
+//   warp 9     TMEM allocator and single-thread tcgen05.mma issuer.
+// Every mbarrier wait is bounded in time; a wait that gives up counts a timeout, and every
+// role then leaves its loop, drains what it issued and the CTA frees its TMEM and returns.
 #include "launch.h"
+#include "sm100_ptx.cuh"
 
 namespace retnet {
 
-bool tc_chunkwise_supported(const RetentionCall&) { return false; }
+namespace {
+using namespace sm100;
 
-cudaError_t launch_tc_chunkwise(const RetentionCall&, const HeadParams&, cudaStream_t) {
-  return cudaErrorNotSupported;
+constexpr int kThreads = 320;
+constexpr int kWarpConv0 = 4;
+constexpr int kWarpTma = 8;
+constexpr int kWarpMma = 9;
+constexpr int kDVS = 64;  // d_v slice per CTA
+
+struct TcArgs {
+  void* o;
+  const float* state_in;
+  float* state_out;
+  int L;
+  int heads;
+  int dv;
+  int n_chunks;
+  int64_t pos0;
+  uint32_t flags;
+};
+
+template <int DK, int T>
+struct Cfg {
+  static constexpr int QBYTES = T * DK * 2;  // one fp16 Qx or Kz tile
+  static constexpr int VBYTES = T * kDVS * 2;
+  static constexpr int STAGE = 2 * QBYTES + VBYTES;
+  static constexpr int PBYTES = T * T * 2;
+  static constexpr int RBYTES = DK * kDVS * 2;
+  static constexpr int NBARS = 4 * 3 + 10;
+  static constexpr int TABBYTES = 2 * (DK / 2) * 8;  // double-buffered per-chunk rotation base
+  static constexpr int FIXED = PBYTES + RBYTES + TABBYTES + NBARS * 8 + 16;
+  static constexpr int BUDGET = 227 * 1024 - 1024;
+  static constexpr int NS_FIT = (BUDGET - FIXED) / STAGE;
+  static constexpr int NS = NS_FIT > 4 ? 4 : NS_FIT;
+  static constexpr int SMEM = NS * STAGE + FIXED + 1024;
+  static constexpr int RBLK = DK > 128 ? 2 : 1;    // 128-row blocks of the state
+  static constexpr int MR = DK >= 128 ? 128 : 64;  // M of the state-update MMA
+  static constexpr int COL_O = 0;
+  static constexpr int COL_S = kDVS;
+  static constexpr int COL_R = kDVS + T;
+  static constexpr int USED = kDVS + T + RBLK * kDVS;
+  static constexpr int TMEM_COLS = USED <= 128 ? 128 : (USED <= 256 ? 256 : 512);
+  static_assert(NS >= 1, "tile does not fit in shared memory");
+  static_assert(USED <= 512, "accumulators do not fit in tensor memory");
+};
+
+// Barrier slots.
+enum : int {
+  B_TMA_FULL = 0,     // [4]
+  B_CONV_FULL = 4,    // [4]
+  B_STAGE_EMPTY = 8,  // [4]
+  B_S_FULL = 12,
+  B_S_FREE,
+  B_P_FULL,
+  B_R_DONE,
+  B_R_READY,
+  B_O_FULL,
+  B_O_FREE,
+  B_DRAIN,
+  B_TAB0,  // [2]: per-chunk rotation base table written (converters)
+};
+
+__device__ __forceinline__ float2 cmul(float2 a, float2 b) {
+  return make_float2(a.x * b.x - a.y * b.y, a.x * b.y + a.y * b.x);
+}
+
+template <int DK, int T, typename Tout>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_chunkwise_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, TcArgs a, HeadParams hp) {
+  using C = Cfg<DK, T>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_addr(smem_raw);
+  const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (sbase - raw_addr);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int dvb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const float log2g = hp.log2g[h];
+  const int n = a.n_chunks;
+  // P and the fp16 state copy carry a fixed 1/sqrt(d_k) so that their fp16 magnitudes stay small;
+  // the epilogue multiplies it back out.
+  const float sd = rsqrtf(static_cast<float>(DK));
+
+  const uint32_t sP = sbase + C::NS * C::STAGE;
+  const uint32_t sR = sP + C::PBYTES;
+  float2* tab = reinterpret_cast<float2*>(gbase + C::NS * C::STAGE + C::PBYTES + C::RBYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + C::NS * C::STAGE + C::PBYTES + C::RBYTES + C::TABBYTES);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::NBARS);
+  auto bar = [&](int i) { return smem_addr(bars + i); };
+  auto sQ = [&](int s) { return sbase + s * C::STAGE; };
+  auto sK = [&](int s) { return sbase + s * C::STAGE + C::QBYTES; };
+  auto sV = [&](int s) { return sbase + s * C::STAGE + 2 * C::QBYTES; };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 4; ++s) {
+      mbar_init(bar(B_TMA_FULL + s), 1);
+      mbar_init(bar(B_CONV_FULL + s), 128);
+      mbar_init(bar(B_STAGE_EMPTY + s), 1);
+    }
+    mbar_init(bar(B_S_FULL), 1);
+    mbar_init(bar(B_S_FREE), 128);
+    mbar_init(bar(B_P_FULL), 128);
+    mbar_init(bar(B_R_DONE), 1);
+    mbar_init(bar(B_R_READY), 128);
+    mbar_init(bar(B_O_FULL), 1);
+    mbar_init(bar(B_O_FREE), 128);
+    mbar_init(bar(B_DRAIN), 1);
+    mbar_init(bar(B_TAB0), 128);
+    mbar_init(bar(B_TAB0 + 1), 128);
+    fence_mbar_init();
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(smem_addr(tmem_holder), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == kWarpTma && lane == 0) {
+    prefetch_tensormap(&tm_q);
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == kWarpTma) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int issued[4] = {0, 0, 0, 0};
+      for (int i = 0; i < n; ++i) {
+        const int s = i % C::NS;
+        if (i >= C::NS && !mbar_wait(bar(B_STAGE_EMPTY + s), ((i / C::NS) - 1) & 1)) break;
+        mbar_arrive_expect_tx(bar(B_TMA_FULL + s), C::STAGE);
+        const int t0 = i * T;
+#pragma unroll
+        for (int bx = 0; bx < DK / 64; ++bx) {
+          tma_load_4d(sQ(s) + bx * T * 128, &tm_q, bar(B_TMA_FULL + s), bx * 64, h, t0, b);
+          tma_load_4d(sK(s) + bx * T * 128, &tm_k, bar(B_TMA_FULL + s), bx * 64, h, t0, b);
+        }
+        tma_load_4d(sV(s), &tm_v, bar(B_TMA_FULL + s), dvb * kDVS, h, t0, b);
+        issued[s]++;
+      }
+      // Every load this thread issued must have landed before the CTA may exit.
+      for (int s = 0; s < C::NS; ++s)
+        if (issued[s] > 0) mbar_wait(bar(B_TMA_FULL + s), (issued[s] - 1) & 1);
+    }
+  } else if (warp == kWarpMma) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t ID_S = idesc_f16_f32(T, T, 0, 0);
+      constexpr uint32_t ID_X = idesc_f16_f32(T, kDVS, 0, 1);
+      constexpr uint32_t ID_R = idesc_f16_f32(C::MR, kDVS, 1, 1);
+      const uint32_t tO = tmem + C::COL_O, tS = tmem + C::COL_S, tR = tmem + C::COL_R;
+      bool ok = true;
+      for (int i = 0; i < n && ok; ++i) {
+        const int s = i % C::NS;
+        ok = mbar_wait(bar(B_CONV_FULL + s), (i / C::NS) & 1);
+        if (ok && i > 0) ok = mbar_wait(bar(B_S_FREE), (i - 1) & 1);
+        if (!ok) break;
+        tc_fence_after();
+        // S'' = Qx Kz^T  (M = T rows r, N = T columns c, K = d_k)
+#pragma unroll
+        for (int kk = 0; kk < DK / 16; ++kk) {
+          const uint32_t off = (kk / 4) * T * 128 + (kk % 4) * 32;
+          mma_f16_ss(tS, sdesc_sw128(sQ(s) + off, 16, 1024), sdesc_sw128(sK(s) + off, 16, 1024), ID_S, kk > 0);
+        }
+        mma_commit(bar(B_S_FULL));
+        ok = mbar_wait(bar(B_R_READY), i & 1);
+        if (ok && i > 0) ok = mbar_wait(bar(B_O_FREE), (i - 1) & 1);
+        if (!ok) break;
+        tc_fence_after();
+        // O = Qx R16  (cross-chunk term; K = d_k)
+#pragma unroll
+        for (int kk = 0; kk < DK / 16; ++kk) {
+          const uint32_t off = (kk / 4) * T * 128 + (kk % 4) * 32;
+          mma_f16_ss(tO, sdesc_sw128(sQ(s) + off, 16, 1024), sdesc_sw128(sR + kk * 2048, DK * 128, 1024), ID_X,
+                     kk > 0);
+        }
+        // R += Kz^T V  (state increment; M = d_k rows in blocks of 128, K = T tokens)
+#pragma unroll
+        for (int blk = 0; blk < C::RBLK; ++blk) {
+#pragma unroll
+          for (int ks = 0; ks < T / 16; ++ks) {
+            mma_f16_ss(tR + blk * kDVS, sdesc_sw128(sK(s) + blk * 2 * T * 128 + ks * 2048, T * 128, 1024),
+                       sdesc_sw128(sV(s) + ks * 2048, T * 128, 1024), ID_R, 1);
+          }
+        }
+        mma_commit(bar(B_R_DONE));
+        ok = mbar_wait(bar(B_P_FULL), i & 1);
+        if (!ok) break;
+        tc_fence_after();
+        // O += P V  (inner-chunk term; K = T tokens)
+#pragma unroll
+        for (int kk = 0; kk < T / 16; ++kk) {
+          const uint32_t off = (kk / 4) * T * 128 + (kk % 4) * 32;
+          mma_f16_ss(tO, sdesc_sw128(sP + off, 16, 1024), sdesc_sw128(sV(s) + kk * 2048, T * 128, 1024), ID_X, 1);
+        }
+        mma_commit(bar(B_O_FULL));
+        mma_commit(bar(B_STAGE_EMPTY + s));
+      }
+      // Drain: every MMA issued above completes before TMEM is released.
+      mma_commit(bar(B_DRAIN));
+      mbar_wait(bar(B_DRAIN), 0);
+    }
+  } else if (warp >= kWarpConv0) {
+    // ------------------------------------------------------------------ converters
+    const int lt = threadIdx.x - 32 * kWarpConv0;  // 0..127
+    const int cj = lt & 7;                          // 16-byte chunk within a 128-byte row
+    const int row0 = lt >> 3;                       // rows row0 + 16 k
+    const bool xpos = (a.flags & RETNET_F_XPOS) != 0;
+    // Per-thread rotation constants for its pairs j = 32 bx + 4 cj + jj:
+    //   W_j = e^{i row0 theta_j},  Z_j = e^{i 16 theta_j}.
+    float2 W[DK / 64][4], Z[DK / 64][4];
+#pragma unroll
+    for (int bx = 0; bx < DK / 64; ++bx)
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const float th = hp.theta[bx * 32 + cj * 4 + jj];
+        float s, c;
+        sincosf(static_cast<float>(row0) * th, &s, &c);
+        W[bx][jj] = make_float2(c, s);
+        sincosf(16.f * th, &s, &c);
+        Z[bx][jj] = make_float2(c, s);
+      }
+    bool ok = true;
+    for (int i = 0; i < n && ok; ++i) {
+      const int s = i % C::NS;
+      const int t0 = i * T;
+      const int bl = min(T, a.L - t0);
+      float2* base = tab + (i & 1) * (DK / 2);
+      if (xpos) {
+        for (int j = lt; j < DK / 2; j += 128) {
+          float sn, cs;
+          xpos_sincos(a.pos0 + t0, hp.theta[j], &sn, &cs);
+          base[j] = make_float2(cs, sn);
+        }
+      }
+      // The table buffer (i & 1) is complete once all 128 converters arrived; a thread that
+      // rewrites it two chunks later has passed this wait, so every read of it is done.
+      mbar_arrive(bar(B_TAB0 + (i & 1)));
+      ok = mbar_wait(bar(B_TAB0 + (i & 1)), (i >> 1) & 1);
+      if (ok) ok = mbar_wait(bar(B_TMA_FULL + s), (i / C::NS) & 1);
+      if (!ok) break;
+      // Row scales xi_r = gamma^(r+1), zeta_r = gamma^(b'-1-r) for r = row0 + 16 k.
+      const float xi0 = decay_pow(log2g, row0 + 1), zeta0 = exp2f(static_cast<float>(bl - 1 - row0) * log2g);
+      const float xstep = decay_pow(log2g, 16), zstep = exp2f(-16.f * log2g);
+#pragma unroll
+      for (int bx = 0; bx < DK / 64; ++bx) {
+        float2 F[4];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) F[jj] = xpos ? cmul(base[bx * 32 + cj * 4 + jj], W[bx][jj]) : make_float2(1.f, 0.f);
+        float xi = xi0, zeta = zeta0;
+#pragma unroll 2
+        for (int k = 0; k < T / 16; ++k) {
+          const int r = row0 + 16 * k;
+          const uint32_t aq = sQ(s) + bx * T * 128 + sw128(r, cj);
+          const uint32_t ak = sK(s) + bx * T * 128 + sw128(r, cj);
+          uint32_t q4[4], k4[4];
+          ld_shared_v4(aq, q4[0], q4[1], q4[2], q4[3]);
+          ld_shared_v4(ak, k4[0], k4[1], k4[2], k4[3]);
+          uint32_t qo[4], ko[4];
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) {
+            const float q0 = __uint_as_float(q4[jj] << 16), q1 = __uint_as_float(q4[jj] & 0xffff0000u);
+            const float k0 = __uint_as_float(k4[jj] << 16), k1 = __uint_as_float(k4[jj] & 0xffff0000u);
+            const float c = F[jj].x, sn = F[jj].y;
+            qo[jj] = pack_f16x2(xi * (q0 * c - q1 * sn), xi * (q0 * sn + q1 * c));
+            ko[jj] = pack_f16x2(zeta * (k0 * c - k1 * sn), zeta * (k0 * sn + k1 * c));
+            F[jj] = cmul(F[jj], Z[bx][jj]);
+          }
+          st_shared_v4(aq, qo[0], qo[1], qo[2], qo[3]);
+          st_shared_v4(ak, ko[0], ko[1], ko[2], ko[3]);
+          xi *= xstep;
+          zeta *= zstep;
+        }
+      }
+      // V: bf16 -> fp16 (exact for values in the fp16 range).
+#pragma unroll
+      for (int k = 0; k < T / 16; ++k) {
+        const int r = row0 + 16 * k;
+        const uint32_t av = sV(s) + sw128(r, cj);
+        uint32_t v4[4], vo[4];
+        ld_shared_v4(av, v4[0], v4[1], v4[2], v4[3]);
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj)
+          vo[jj] = pack_f16x2(__uint_as_float(v4[jj] << 16), __uint_as_float(v4[jj] & 0xffff0000u));
+        st_shared_v4(av, vo[0], vo[1], vo[2], vo[3]);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bar(B_CONV_FULL + s));
+    }
+  } else {
+    // ------------------------------------------------------------------ TMEM warpgroup
+    const uint32_t lane_off = static_cast<uint32_t>(32 * warp) << 16;
+    const int my_row = (T == 128) ? 32 * warp + lane : (lane < 16 ? 16 * warp + lane : -1);
+    // State rows (d_k) held by this thread's TMEM lane in each 128-row block.
+    auto state_row = [&](int blk) -> int {
+      if (DK == 64) return lane < 16 ? 16 * warp + lane : -1;
+      return blk * 128 + 32 * warp + lane;
+    };
+    const int64_t bh = static_cast<int64_t>(b) * a.heads + h;
+    const size_t srow = static_cast<size_t>(a.dv);
+    float* sbase_g_out = a.state_out ? a.state_out + static_cast<size_t>(bh) * DK * a.dv + dvb * kDVS : nullptr;
+    const float* sbase_g_in = a.state_in ? a.state_in + static_cast<size_t>(bh) * DK * a.dv + dvb * kDVS : nullptr;
+
+    // Write R (64 fp32 of one state row) as fp16 into the cross-term operand (MN-major,
+    // rows = d_k, 128 B = 64 d_v per row, 128-byte swizzle).
+    auto put_r16 = [&](int dk, const float* rv) {
+#pragma unroll
+      for (int c8 = 0; c8 < 8; ++c8)
+        st_shared_v4(sR + sw128(dk, c8), pack_f16x2(sd * rv[8 * c8 + 0], sd * rv[8 * c8 + 1]),
+                     pack_f16x2(sd * rv[8 * c8 + 2], sd * rv[8 * c8 + 3]),
+                     pack_f16x2(sd * rv[8 * c8 + 4], sd * rv[8 * c8 + 5]),
+                     pack_f16x2(sd * rv[8 * c8 + 6], sd * rv[8 * c8 + 7]));
+    };
+
+    // Initial state: master = gamma^(b'_0) R_in, fp16 copy = R_in.
+    {
+      const int bl0 = min(T, a.L);
+      const float g0 = decay_pow(log2g, bl0);
+#pragma unroll 1
+      for (int blk = 0; blk < C::RBLK; ++blk) {
+        const int dk = state_row(blk);
+        float rv[kDVS];
+#pragma unroll
+        for (int c = 0; c < kDVS; ++c) rv[c] = 0.f;
+        if (dk >= 0 && sbase_g_in) {
+#pragma unroll
+          for (int c4 = 0; c4 < kDVS / 4; ++c4) {
+            const float4 x = *reinterpret_cast<const float4*>(sbase_g_in + dk * srow + 4 * c4);
+            rv[4 * c4] = x.x; rv[4 * c4 + 1] = x.y; rv[4 * c4 + 2] = x.z; rv[4 * c4 + 3] = x.w;
+          }
+        }
+        if (dk >= 0) put_r16(dk, rv);
+#pragma unroll
+        for (int c16 = 0; c16 < kDVS / 16; ++c16) {
+          uint32_t u[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) u[e] = __float_as_uint(g0 * rv[16 * c16 + e]);
+          tmem_st16(tmem + C::COL_R + blk * kDVS + 16 * c16 + lane_off, u);
+        }
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(B_R_READY));
+    }
+
+    bool ok = true;
+    for (int i = 0; i < n && ok; ++i) {
+      const int t0 = i * T;
+      const int bl = min(T, a.L - t0);
+      const bool last = (i == n - 1);
+      // (1) P = S'' gamma^(-b') on and below the diagonal, fp16, into the K-major A tile.
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL), i & 1));
+      if (!ok) break;
+      tc_fence_after();
+      {
+        const float ginv = exp2f(-static_cast<float>(bl) * log2g) * sd;
+#pragma unroll
+        for (int half = 0; half < T / 64; ++half) {
+          uint32_t u[4][16];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) tmem_ld16(tmem + C::COL_S + half * 64 + 16 * q + lane_off, u[q]);
+          tmem_wait_ld();
+          if (my_row >= 0) {
+#pragma unroll
+            for (int c8 = 0; c8 < 8; ++c8) {
+              uint32_t pk[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int c0 = half * 64 + 8 * c8 + 2 * e;
+                const float p0 = (c0 <= my_row) ? __uint_as_float(u[c8 / 2][(8 * c8 + 2 * e) % 16]) * ginv : 0.f;
+                const float p1 = (c0 + 1 <= my_row) ? __uint_as_float(u[c8 / 2][(8 * c8 + 2 * e + 1) % 16]) * ginv : 0.f;
+                pk[e] = pack_f16x2(p0, p1);
+              }
+              st_shared_v4(sP + half * T * 128 + sw128(my_row, c8), pk[0], pk[1], pk[2], pk[3]);
+            }
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(B_S_FREE));
+      mbar_arrive(bar(B_P_FULL));
+
+      // (2) State: R_i (TMEM, after the increment) -> fp16 copy; gamma^(b'_{i+1}) R_i -> TMEM.
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_R_DONE), i & 1));
+      if (!ok) break;
+      tc_fence_after();
+      {
+        const int bln = last ? 0 : min(T, a.L - t0 - T);
+        const float gn = decay_pow(log2g, bln);
+#pragma unroll 1
+        for (int blk = 0; blk < C::RBLK; ++blk) {
+          const int dk = state_row(blk);
+          uint32_t u[4][16];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) tmem_ld16(tmem + C::COL_R + blk * kDVS + 16 * q + lane_off, u[q]);
+          tmem_wait_ld();
+          float rv[kDVS];
+#pragma unroll
+          for (int c = 0; c < kDVS; ++c) rv[c] = __uint_as_float(u[c / 16][c % 16]);
+          if (!last) {
+            if (dk >= 0) put_r16(dk, rv);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint32_t w16[16];
+#pragma unroll
+              for (int e = 0; e < 16; ++e) w16[e] = __float_as_uint(gn * rv[16 * q + e]);
+              tmem_st16(tmem + C::COL_R + blk * kDVS + 16 * q + lane_off, w16);
+            }
+          } else if (dk >= 0 && sbase_g_out) {
+#pragma unroll
+            for (int c4 = 0; c4 < kDVS / 4; ++c4)
+              *reinterpret_cast<float4*>(sbase_g_out + dk * srow + 4 * c4) =
+                  make_float4(rv[4 * c4], rv[4 * c4 + 1], rv[4 * c4 + 2], rv[4 * c4 + 3]);
+          }
+        }
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(bar(B_R_READY));
+      }
+
+      // (3) Epilogue: o = O * s / c_p, stored as the output dtype.
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_O_FULL), i & 1));
+      if (!ok) break;
+      tc_fence_after();
+      {
+        uint32_t u[4][16];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tmem_ld16(tmem + C::COL_O + 16 * q + lane_off, u[q]);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar(B_O_FREE));
+        if (my_row >= 0 && my_row < bl) {
+          const float f = row_factor(hp.gamma[h], DK, a.pos0 + t0 + my_row, a.flags) / sd;
+          const int64_t orow = ((static_cast<int64_t>(b) * a.L + t0 + my_row) * a.heads + h) * a.dv + dvb * kDVS;
+          Tout* dst = static_cast<Tout*>(a.o) + orow;
+          if constexpr (sizeof(Tout) == 2) {
+#pragma unroll
+            for (int c8 = 0; c8 < 8; ++c8) {
+              uint32_t pk[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                __nv_bfloat162 v2 = __floats2bfloat162_rn(f * __uint_as_float(u[c8 / 2][(8 * c8 + 2 * e) % 16]),
+                                                          f * __uint_as_float(u[c8 / 2][(8 * c8 + 2 * e + 1) % 16]));
+                pk[e] = *reinterpret_cast<uint32_t*>(&v2);
+              }
+              *reinterpret_cast<uint4*>(dst + 8 * c8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+          } else {
+#pragma unroll
+            for (int c4 = 0; c4 < 16; ++c4)
+              *reinterpret_cast<float4*>(dst + 4 * c4) =
+                  make_float4(f * __uint_as_float(u[c4 / 4][(4 * c4) % 16]), f * __uint_as_float(u[c4 / 4][(4 * c4 + 1) % 16]),
+                              f * __uint_as_float(u[c4 / 4][(4 * c4 + 2) % 16]), f * __uint_as_float(u[c4 / 4][(4 * c4 + 3) % 16]));
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ---- host side -------------------------------------------------------------------------------
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;  // resolved once from the driver; no CUDA context state
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 4-D map over a BLHD bf16 tensor [b][L][h][d] with a (64, 1, T, 1) box, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, int64_t b, int64_t L, int64_t h, int64_t d, int T) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(h), static_cast<cuuint64_t>(L),
+                        static_cast<cuuint64_t>(b)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(d * 2), static_cast<cuuint64_t>(h * d * 2),
+                           static_cast<cuuint64_t>(L * h * d * 2)};
+  cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(T), 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int DK, int T, typename Tout>
+cudaError_t launch_cfg(const RetentionCall& c, const HeadParams& hp, cudaStream_t s) {
+  using Cf = Cfg<DK, T>;
+  CUtensorMap mq, mk, mv;
+  const Dims& d = c.dims;
+  if (!make_map(&mq, c.q, d.batch, d.seqlen, d.heads, d.d_k, T) ||
+      !make_map(&mk, c.k, d.batch, d.seqlen, d.heads, d.d_k, T) ||
+      !make_map(&mv, c.v, d.batch, d.seqlen, d.heads, d.d_v, T))
+    return cudaErrorInvalidValue;
+  TcArgs a;
+  a.o = c.o;
+  a.state_in = c.state_in;
+  a.state_out = c.state_out;
+  a.L = static_cast<int>(d.seqlen);
+  a.heads = static_cast<int>(d.heads);
+  a.dv = static_cast<int>(d.d_v);
+  a.n_chunks = static_cast<int>((d.seqlen + T - 1) / T);
+  a.pos0 = c.pos0;
+  a.flags = c.flags;
+  auto kern = tc_chunkwise_kernel<DK, T, Tout>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM);
+  if (e != cudaSuccess) return e;
+  dim3 grid(static_cast<unsigned>(d.d_v / kDVS), static_cast<unsigned>(d.heads), static_cast<unsigned>(d.batch));
+  kern<<<grid, kThreads, Cf::SMEM, s>>>(mq, mk, mv, a, hp);
+  return cudaGetLastError();
+}
+
+template <int DK, typename Tout>
+cudaError_t launch_dk(const RetentionCall& c, const HeadParams& hp, cudaStream_t s) {
+  if (c.chunk == 64) return launch_cfg<DK, 64, Tout>(c, hp, s);
+  return launch_cfg<DK, 128, Tout>(c, hp, s);
+}
+
+template <typename Tout>
+cudaError_t launch_out(const RetentionCall& c, const HeadParams& hp, cudaStream_t s) {
+  switch (c.dims.d_k) {
+    case 64: return launch_dk<64, Tout>(c, hp, s);
+    case 128: return launch_dk<128, Tout>(c, hp, s);
+    default: return launch_dk<256, Tout>(c, hp, s);
+  }
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+bool tc_chunkwise_supported(const RetentionCall& c) {
+  const Dims& d = c.dims;
+  if (c.in_dtype != RETNET_BF16) return false;
+  if (c.flags & RETNET_F_NORM_R) return false;
+  if (d.d_k != 64 && d.d_k != 128 && d.d_k != 256) return false;
+  if (d.d_v % kDVS != 0) return false;
+  if (c.chunk != 64 && c.chunk != 128) return false;
+  if (d.seqlen < 1 || d.seqlen > (1LL << 30) || d.heads > 65535 || d.batch > 65535) return false;
+  if (!aligned16(c.q) || !aligned16(c.k) || !aligned16(c.v) || !aligned16(c.o)) return false;
+  if ((c.state_in && !aligned16(c.state_in)) || (c.state_out && !aligned16(c.state_out))) return false;
+  if (c.state_in && c.state_out && c.state_in != c.state_out) {
+    // distinct buffers are fine; overlapping but unequal ones are not supported here
+    const char* a0 = reinterpret_cast<const char*>(c.state_in);
+    const char* b0 = reinterpret_cast<const char*>(c.state_out);
+    const size_t bytes = sizeof(float) * static_cast<size_t>(d.batch * d.heads * d.d_k * d.d_v);
+    if (a0 < b0 + bytes && b0 < a0 + bytes) return false;
+  }
+  return true;
+}
+
+bool tc_driver_ready() { return encode_fn() != nullptr; }
+
+// Host-side part of the scaled-operand condition: every head keeps gamma^B >= 2^-12.
+bool tc_chunkwise_heads_ok(const RetentionCall& c, const HeadParams& hp) {
+  for (int64_t h = 0; h < c.dims.heads; ++h)
+    if (static_cast<double>(hp.log2g[h]) * static_cast<double>(c.chunk) < -12.0) return false;
+  return true;
+}
+
+cudaError_t tc_wait_timeouts(unsigned int* count, bool clear) {
+  cudaError_t e = cudaMemcpyFromSymbol(count, sm100::g_wait_timeouts, sizeof(unsigned int));
+  if (e != cudaSuccess || !clear || *count == 0) return e;
+  const unsigned int zero = 0;
+  return cudaMemcpyToSymbol(sm100::g_wait_timeouts, &zero, sizeof(unsigned int));
+}
+
+cudaError_t launch_tc_chunkwise(const RetentionCall& c, const HeadParams& hp, cudaStream_t s) {
+  if (c.out_dtype == RETNET_F32) return launch_out<float>(c, hp, s);
+  return launch_out<__nv_bfloat16>(c, hp, s);
 }
 
 }  // namespace retnet

@@ -30,9 +30,14 @@ struct RetentionCall {
 cudaError_t launch_simt_retention(const RetentionCall& c, const HeadParams& hp, cudaStream_t s);
 
 // tcgen05 tensor-core chunkwise kernel for bf16 inputs; `supported` says whether the shape
-// is one it handles (then it launches and returns the launch status).
+// and buffers are ones it handles, `heads_ok` whether every head keeps gamma^chunk >= 2^-12.
 bool tc_chunkwise_supported(const RetentionCall& c);
+bool tc_chunkwise_heads_ok(const RetentionCall& c, const HeadParams& hp);
+// The driver entry point that encodes TMA tensor maps could be resolved.
+bool tc_driver_ready();
 cudaError_t launch_tc_chunkwise(const RetentionCall& c, const HeadParams& hp, cudaStream_t s);
+// Reads (and optionally clears) the count of bounded waits that gave up in the tensor-core kernel.
+cudaError_t tc_wait_timeouts(unsigned int* count, bool clear);
 
 struct StepCall {
   const void* q;

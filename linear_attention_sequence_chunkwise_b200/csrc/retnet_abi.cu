@@ -129,8 +129,33 @@ retnet_status_t retnet_retention_chunkwise(const void* q, const void* k, const v
     }
     return RETNET_OK;
   }
-  if (tc_chunkwise_supported(c)) return from_cuda(launch_tc_chunkwise(c, hp, static_cast<cudaStream_t>(stream)));
+  if (tc_chunkwise_supported(c) && tc_chunkwise_heads_ok(c, hp)) {
+    if (!tc_driver_ready()) return RETNET_ERR_CUDA;
+    return from_cuda(launch_tc_chunkwise(c, hp, static_cast<cudaStream_t>(stream)));
+  }
   return from_cuda(launch_simt_retention(c, hp, static_cast<cudaStream_t>(stream)));
+}
+
+int retnet_chunkwise_kernel(retnet_dims_t dims, retnet_dtype_t in_dtype, uint32_t flags, int64_t chunk,
+                            const float* gamma) {
+  retnet_status_t st = check_common(dims, in_dtype, RETNET_F32, 0, flags, true);
+  if (st != RETNET_OK) return -static_cast<int>(st);
+  if (chunk <= 0) return -static_cast<int>(RETNET_ERR_BAD_PARAM);
+  HeadParams hp;
+  // theta is not read without XPOS, and its values do not affect the choice of kernel.
+  st = fill_params(&hp, gamma, nullptr, dims.heads, dims.d_k, flags & ~static_cast<uint32_t>(RETNET_F_XPOS));
+  if (st != RETNET_OK) return -static_cast<int>(st);
+  alignas(16) static const uint32_t kAligned[4] = {0, 0, 0, 0};
+  RetentionCall c{kAligned, kAligned, kAligned, const_cast<uint32_t*>(kAligned),
+                  Dims{dims.batch, dims.seqlen, dims.heads, dims.d_k, dims.d_v}, in_dtype, RETNET_F32, 0, flags,
+                  chunk, true, nullptr, nullptr, nullptr, nullptr};
+  return (tc_chunkwise_supported(c) && tc_chunkwise_heads_ok(c, hp)) ? 1 : 0;
+}
+
+retnet_status_t retnet_debug_wait_timeouts(unsigned int* count, int clear) {
+  if (!count) return RETNET_ERR_NULL_PTR;
+  if (cudaDeviceSynchronize() != cudaSuccess) return RETNET_ERR_CUDA;
+  return from_cuda(tc_wait_timeouts(count, clear != 0));
 }
 
 retnet_status_t retnet_retention_step(const void* q, const void* k, const void* v, void* o, int64_t batch,

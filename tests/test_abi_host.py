@@ -137,3 +137,20 @@ def test_binding_raises_without_library(tmp_path):
             mod.load(str(tmp_path / "missing.so"))
     finally:
         mod._lib = saved
+
+
+def test_chunkwise_kernel_choice(lib):
+    g8 = np.array([1.0 - 2.0 ** (-5 - i) for i in range(8)], np.float32)
+    f = rn.F_XPOS | rn.F_SCALE_SQRT_D | rn.F_NORM_D
+    assert rn.retnet_chunkwise_kernel((8, 2048, 8, 128), 128, rn.BF16, f, 64, g8) == 1
+    assert rn.retnet_chunkwise_kernel((2, 8192, 8, 256), 512, rn.BF16, f, 128, g8) == 1
+    assert rn.retnet_chunkwise_kernel((1, 64, 8, 64), 64, rn.BF16, f, 128, g8) == 1
+    assert rn.retnet_chunkwise_kernel((1, 64, 8, 128), 128, rn.F32, f, 64, g8) == 0      # fp32 inputs
+    assert rn.retnet_chunkwise_kernel((1, 64, 8, 128), 128, rn.BF16, f | rn.F_NORM_R, 64, g8) == 0
+    assert rn.retnet_chunkwise_kernel((1, 64, 8, 96), 128, rn.BF16, f, 64, g8) == 0      # d_k 96
+    assert rn.retnet_chunkwise_kernel((1, 64, 8, 128), 96, rn.BF16, f, 64, g8) == 0      # d_v 96
+    assert rn.retnet_chunkwise_kernel((1, 64, 8, 128), 128, rn.BF16, f, 32, g8) == 0     # chunk 32
+    # gamma^B < 2^-12 for some head: the scaled tensor-core form does not apply
+    assert rn.retnet_chunkwise_kernel((1, 64, 2, 128), 128, rn.BF16, f, 128, np.array([0.9, 0.99], np.float32)) == 0
+    assert rn.retnet_chunkwise_kernel((1, 64, 2, 128), 128, rn.BF16, f, 0, g8) == -4
+    assert rn.retnet_chunkwise_kernel((1, 64, 2, 128), 128, 9, f, 64, g8) == -3

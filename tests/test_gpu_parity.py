@@ -11,7 +11,7 @@ import torch
 import linear_attention_sequence_chunkwise_b200 as rn
 import oracle
 import synth_inputs as si
-from gpu_util import TOL_BF16, TOL_F32, bf16_round, dev, err, require_gpu
+from gpu_util import TOL_BF16, TOL_F32, dev, err, err_bf16_out, require_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -90,7 +90,7 @@ def test_chunkwise_bf16_inputs_cuda_core_shapes():
     assert err(o, ref) <= TOL_F32  # exact inputs, fp32 arithmetic
     ob = torch.empty(b, L, h, dv, device="cuda", dtype=torch.bfloat16)
     rn.retnet_retention_chunkwise(dev(q), dev(k), dev(v), ob, g, th, 0, oracle.F_ALL, B)
-    assert err(ob, bf16_round(ref)) <= TOL_BF16
+    assert err_bf16_out(ob, ref) <= TOL_BF16
 
 
 @pytest.mark.parametrize("dv", [48, 42, 520])
@@ -152,7 +152,7 @@ def test_msr_epilogue(dtype, dv):
     assert err(out, ref) <= TOL_F32
     outb = torch.empty(tokens, h * dv, device="cuda", dtype=torch.bfloat16)
     rn.retnet_msr_epilogue(dev(y), dev(gt), outb, h, 1e-5)
-    assert err(outb, bf16_round(ref)) <= TOL_BF16
+    assert err_bf16_out(outb, ref) <= TOL_BF16
 
 
 def test_causality_bitwise():
@@ -183,7 +183,8 @@ def test_degenerate_sizes():
     zo = torch.empty_like(z0)
     e = torch.empty(1, 0, 1, 4, device="cuda")
     ev = torch.empty(1, 0, 1, 8, device="cuda")
-    rn.retnet_retention_chunkwise(e, e, ev, ev.clone(), g, None, 0, oracle.F_ALL, 16, S0, So, z0, zo)
+    nox = oracle.F_SCALE_SQRT_D | oracle.F_NORM_D | oracle.F_NORM_R
+    rn.retnet_retention_chunkwise(e, e, ev, ev.clone(), g, None, 0, nox, 16, S0, So, z0, zo)
     torch.cuda.synchronize()
     assert torch.equal(So, S0) and torch.equal(zo, z0)
     # seqlen 1, d_k = d_v = 1, no rotation

@@ -1,0 +1,122 @@
+"""Parity of the tcgen05 tensor-core chunkwise kernel (bf16 inputs) against the fp64 oracle.
+
+Bar: max|err|/rms(oracle) <= 1e-2 on the raw output (the bf16-input tolerance); the
+state hand-off is held to the same bar.  Every case asserts first that the call takes
+the tensor-core kernel, and last that no bounded wait inside it gave up.
+"""
+import numpy as np
+import pytest
+import torch
+
+import linear_attention_sequence_chunkwise_b200 as rn
+import oracle
+import synth_inputs as si
+from gpu_util import TOL_BF16, dev, err, err_bf16_out, require_gpu
+
+pytestmark = pytest.mark.gpu
+FLAGS = rn.F_XPOS | rn.F_SCALE_SQRT_D | rn.F_NORM_D
+
+
+@pytest.fixture(autouse=True)
+def _gpu(cuda_lib):
+    require_gpu()
+    rn.retnet_debug_wait_timeouts(clear=True)
+    yield
+    assert rn.retnet_debug_wait_timeouts(clear=True) == 0
+
+
+def run_tc(q, k, v, g, th, B, flags=FLAGS, pos0=0, state_in=None, want_state=False, out_dtype=torch.float32):
+    b, L, h, dk = q.shape
+    dv = v.shape[-1]
+    assert rn.retnet_chunkwise_kernel((b, L, h, dk), dv, rn.BF16, flags, B, g) == 1
+    o = torch.empty(b, L, h, dv, device="cuda", dtype=out_dtype)
+    so = torch.empty(b, h, dk, dv, device="cuda") if want_state else None
+    rn.retnet_retention_chunkwise(dev(q), dev(k), dev(v), o, g, th, pos0, flags, B,
+                                  None if state_in is None else dev(state_in), so)
+    torch.cuda.synchronize()
+    return o, so
+
+
+@pytest.mark.parametrize("dk,dv,B,L", [(128, 128, 64, 300), (128, 192, 128, 300), (64, 64, 64, 130),
+                                       (64, 128, 128, 257), (256, 128, 64, 200), (256, 64, 128, 129),
+                                       (128, 64, 64, 1), (128, 64, 64, 64), (128, 64, 128, 128)])
+def test_tc_matches_oracle(dk, dv, B, L):
+    b, h = 2, 3
+    q, k, v = si.qkv(b, L, h, dk, dv, 60 + dk + B, "bf16")
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+    ref, Sref, _ = oracle.recurrent(q, k, v, g, th, 0, FLAGS)
+    o, so = run_tc(q, k, v, g, th, B, want_state=True)
+    e = err(o, ref)
+    print(f"dk={dk} dv={dv} B={B} L={L}: max|err|/rms = {e:.3e}")
+    assert e <= TOL_BF16
+    assert err(so, Sref) <= TOL_BF16
+
+
+@pytest.mark.parametrize("flags", [0, rn.F_XPOS, rn.F_SCALE_SQRT_D, rn.F_NORM_D, FLAGS])
+def test_tc_flag_combinations(flags):
+    b, L, h, dk, dv, B = 1, 200, 4, 128, 64, 64
+    q, k, v = si.qkv(b, L, h, dk, dv, 70, "bf16")
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+    ref = oracle.parallel(q, k, v, g, th, 0, flags)
+    o, _ = run_tc(q, k, v, g, th, B, flags=flags)
+    assert err(o, ref) <= TOL_BF16
+
+
+def test_tc_state_in_and_position():
+    b, L, h, dk, dv, B = 2, 190, 2, 128, 128, 64
+    q, k, v = si.qkv(b, L, h, dk, dv, 71, "bf16")
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+    S0 = si.decode_state(b, h, dk, dv, 72, std=0.3)
+    pos0 = 777
+    ref, Sref, _ = oracle.recurrent(q, k, v, g, th, pos0, FLAGS, S0)
+    o, so = run_tc(q, k, v, g, th, B, pos0=pos0, state_in=S0, want_state=True)
+    assert err(o, ref) <= TOL_BF16
+    assert err(so, Sref) <= TOL_BF16
+
+
+def test_tc_bf16_output():
+    b, L, h, dk, dv, B = 2, 256, 2, 128, 128, 128
+    q, k, v = si.qkv(b, L, h, dk, dv, 73, "bf16")
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+    ref = oracle.parallel(q, k, v, g, th, 0, FLAGS)
+    o, _ = run_tc(q, k, v, g, th, B, out_dtype=torch.bfloat16)
+    assert err_bf16_out(o, ref) <= TOL_BF16
+
+
+def test_tc_causality_bitwise():
+    b, L, h, dk, dv, B, m = 1, 300, 2, 128, 64, 64, 150
+    q, k, v = si.qkv(b, L, h, dk, dv, 74, "bf16")
+    q2, k2, v2 = q.clone(), k.clone(), v.clone()
+    q2[:, m:] = -q2[:, m:]; k2[:, m:] *= 2; v2[:, m:] += 1
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+    o1, _ = run_tc(q, k, v, g, th, B)
+    o2, _ = run_tc(q2, k2, v2, g, th, B)
+    assert torch.equal(o1[:, :m].cpu(), o2[:, :m].cpu())
+    assert not torch.equal(o1[:, m:].cpu(), o2[:, m:].cpu())
+
+
+def test_tc_prefill_then_decode_matches_parallel():
+    b, L, P, h, dk, dv = 2, 160, 128, 2, 128, 64
+    q, k, v = si.qkv(b, L, h, dk, dv, 75, "bf16")
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+    ref = oracle.parallel(q, k, v, g, th, 0, FLAGS)
+    o1, S = run_tc(q[:, :P].contiguous(), k[:, :P].contiguous(), v[:, :P].contiguous(), g, th, 64,
+                   want_state=True)
+    outs = [o1]
+    for t in range(P, L):
+        ot = torch.empty(b, 1, h, dv, device="cuda")
+        rn.retnet_retention_step(dev(q[:, t]), dev(k[:, t]), dev(v[:, t]), ot.view(b, h, dv), S, g, th, t, FLAGS)
+        outs.append(ot)
+    assert err(torch.cat(outs, 1), ref) <= TOL_BF16
+
+
+def test_tc_chunkwise_workload_full_size():
+    """The benchmark workload in full: batch 8, h 8, d_k = d_v = 128, L 2048, B 64, every output."""
+    b, L, h, dk, dv, B = 8, 2048, 8, 128, 128, 64
+    q, k, v = si.qkv(b, L, h, dk, dv, 2, "bf16")
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+    o, _ = run_tc(q, k, v, g, th, B)
+    ref, _, _ = oracle.recurrent(q, k, v, g, th, 0, FLAGS)
+    e = err(o, ref)
+    print(f"full workload max|err|/rms = {e:.3e}")
+    assert e <= TOL_BF16
