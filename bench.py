@@ -312,7 +312,9 @@ def main_ours(args):
         "clocks": clk,
     }
     # e2e: host buffers in pinned memory, copies inside the timed region, through the same C call
-    e2e_steps = max(3, min(args.steps, 50))
+    if "e2e" not in args.sections:
+        line["e2e"] = None
+    e2e_steps = max(3, min(args.steps, 50)) if "e2e" in args.sections else 0
     hq = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in sets[0][:3]]
     for hx, dx in zip(hq, sets[0][:3]):
         hx.copy_(dx.cpu())
@@ -326,15 +328,16 @@ def main_ours(args):
         run_chunkwise(rn, (dq, dk_, dv_, do), cfg, gamma, theta, stream)
         ho.copy_(do, non_blocking=True)
 
-    e2e_step(0)
-    torch.cuda.synchronize()
-    barrier(world)
-    e_secs = time_steps(e2e_step, e2e_steps, stream)
-    barrier(world)
-    e_secs = max_over_ranks(e_secs, world, device)
-    line["e2e"] = {"value": b * L * world * e2e_steps / e_secs, "unit": "tokens/s",
-                   "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in hq),
-                   "d2h_bytes_per_step": ho.numel() * ho.element_size(), "steps": e2e_steps}
+    if e2e_steps:
+        e2e_step(0)
+        torch.cuda.synchronize()
+        barrier(world)
+        e_secs = time_steps(e2e_step, e2e_steps, stream)
+        barrier(world)
+        e_secs = max_over_ranks(e_secs, world, device)
+        line["e2e"] = {"value": b * L * world * e2e_steps / e_secs, "unit": "tokens/s",
+                       "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in hq),
+                       "d2h_bytes_per_step": ho.numel() * ho.element_size(), "steps": e2e_steps}
     if world == 1 and "decode" in args.sections:
         line["decode"] = bench_decode(rn, device, stream, args.decode_steps, 3, peaks)
     clocks.stop()
@@ -377,7 +380,8 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--sections", default="main,decode")
+    ap.add_argument("--sections", default="e2e,decode",
+                    help="comma list of extra legs to run beside the timed step: e2e, decode")
     ap.add_argument("--decode-steps", type=int, default=200)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

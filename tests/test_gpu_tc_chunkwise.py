@@ -120,3 +120,17 @@ def test_tc_chunkwise_workload_full_size():
     e = err(o, ref)
     print(f"full workload max|err|/rms = {e:.3e}")
     assert e <= TOL_BF16
+
+
+def test_serial_kernel_variant_in_subprocess():
+    """RETNET_TC_KERNEL=serial routes every tensor-core call to the serial kernel; it must
+    pass the same parity cases as the pipelined kernel."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, RETNET_TC_KERNEL="serial")
+    here = os.path.dirname(os.path.abspath(__file__))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider", "-m", "gpu",
+                        "-k", "tc_matches_oracle or tc_state_in or tc_flag", os.path.join(here, "test_gpu_tc_chunkwise.py")],
+                       env=env, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
