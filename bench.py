@@ -49,6 +49,21 @@ def bytes_per_token_head(dk, dv, elt=2):
     return elt * (2 * dk + 2 * dv)
 
 
+def ncu_traffic(name):
+    """DRAM bytes per launch from the committed ncu record, if the kernel's sources still hash
+    to the profiled version (else None: the counters no longer describe this build)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        rec = json.load(open(path))[name]
+        h = hashlib.sha256()
+        for f in rec["sources"]:
+            h.update(open(os.path.join(ROOT, f), "rb").read())
+        return rec["dram_bytes_per_launch"] if h.hexdigest()[:16] == rec["hash"] else None
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -204,7 +219,10 @@ def bench_decode(rn, device, stream, steps, warmup, peaks):
     gbs = (state_bytes + io_bytes) / per / 1e9
     return {"workload": c["workload"], "steps": steps, "us_per_step": per * 1e6,
             "bytes_per_step": state_bytes + io_bytes, "gbs": gbs, "frac_of_measured_hbm": gbs / peaks["hbm"],
-            "frac_of_8tbs": gbs / 8000.0, "gpu_launches": steps}
+            "frac_of_8tbs": gbs / 8000.0, "gpu_launches": steps,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm"], "traffic": ncu_traffic("decode_step"),
+                         "peak_source": peaks["source"]}}
 
 
 def oracle_sample(cfg, budget_s):
@@ -305,7 +323,7 @@ def main_ours(args):
                    "parallelism": f"dp{world}"},
         "tflops": tflops, "frac_bf16_peak": tflops * 1e12 / (peaks["bf16"] * 1e12),
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm"], "unit": "GB/s",
-                     "frac": achieved_gbs / peaks["hbm"], "traffic": args.traffic,
+                     "frac": achieved_gbs / peaks["hbm"], "traffic": ncu_traffic("chunkwise_tc") if path == 1 else None,
                      "peak_source": peaks["source"], "algorithmic_bytes_per_launch": alg_bytes,
                      "launch_us": per_launch * 1e6},
         "gpu_launches": args.steps,
@@ -385,8 +403,6 @@ def parse_args(argv=None):
     ap.add_argument("--decode-steps", type=int, default=200)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--traffic", type=float, default=None,
-                    help="ncu dram bytes per launch of the chunkwise kernel, when known for this build")
     a = ap.parse_args(argv)
     if a.warmup < 3 and a.impl == "ours":
         a.warmup = 3

@@ -52,7 +52,8 @@
  * cores (tcgen05) with fp16 operands and fp32 accumulation: bf16 q, k, v convert to fp16
  * exactly, the rotated q, k, the masked scores and the chunk state are rounded to fp16 once
  * each.  fp16 has three more mantissa bits than bf16 and a smaller range, so finite results
- * need |q|, |k|, |v| < 32768, |q.k| < 32768 * sqrt(d_k) and state entries < 65504.
+ * need |q|, |k|, |v| < 32768, |q.k| / sqrt(d_k) < 65504 and state entries below
+ * 65504 * sqrt(d_k).
  */
 #ifndef RETNET_H
 #define RETNET_H
