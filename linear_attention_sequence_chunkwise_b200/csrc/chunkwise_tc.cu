@@ -51,6 +51,7 @@ struct TcArgs {
   int n_chunks;
   int64_t pos0;
   uint32_t flags;
+  int nb;  // sub-blocks of T rows per chunk (pipelined kernel)
 };
 
 template <int DK, int T>
@@ -557,24 +558,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ============================================================================================
-// Pipelined kernel.  Same arithmetic as the kernel above; the work is split so that no role
-// waits on another within a chunk:
-//   warps 0-3        P/epilogue group: S -> P for chunk j, then the epilogue of chunk j-1.
-//   next 4*RBLK warps state group: the chunk state R lives in registers (one d_k row of the
-//                    64-wide slice per thread); per chunk it adds the increment Kz^T V from TMEM,
-//                    R_j = gamma^b' R_{j-1} + dR_j, and writes the fp16 copy the next chunk's
-//                    cross term reads.
-//   4 warps          converters (as above);   1 warp TMA;   1 warp MMA issuer.
-// TMEM holds two S tiles, two O tiles and two increment tiles, so consecutive chunks overlap;
-// the MMA issuer runs one chunk ahead: it issues S_{j+1} and dR_{j+1} before the cross and
-// P V products of chunk j, which wait for the state and for P_j.
+// Pipelined kernel.  The work of a chunk of B = nb * T tokens is split into units
+// (u, w): row block u (T query rows) against column block w <= u (T key/value rows).
+// Sub-block-local scaled operands: rows r and columns c are local to their T-row block and
+//   Qx_u = gamma^(r+1) (.) rot(q),   Kz_w = gamma^(T-1-c) (.) rot(k)   (fp16),
+// so that, with S'' = Qx_u Kz_w^T = gamma^(T+r-c) (Q K^T),
+//   P_{u,w} = S'' * gamma^((u-w-1) T)      (causal mask on the diagonal block only),
+//   O_u = sum_{w<=u} P_{u,w} V_w,   X_u = Qx_u R16 (the chunk-start state),
+//   o = (O_u + gamma^(u T) X_u) * s / c_p            (X goes straight into O when nb = 1),
+//   R_i = gamma^b' R_{i-1} + sum_w gamma^(b'-(w+1)T) Kz_w^T V_w   (taken in Horner form).
+// fp16 operands stay in range when gamma^T >= 2^-12.  Roles:
+//   warps 0-3        P/epilogue group: S -> P for each unit; epilogue of each finished row block.
+//   next 4*RBLK warps state group: the chunk state R in registers (one d_k row of the 64-wide
+//                    d_v slice per thread); Horner update per column block of the last row block;
+//                    fp16 copy of R for the next chunk's cross terms.
+//   4 warps          converters: rotate/scale/convert each unit's Q, K, V tiles in place.
+//   1 warp TMA, 1 warp MMA issuer (one unit ahead: S and dR of unit k+1 before X/PV of unit k).
 // ============================================================================================
 
 template <int DK, int T>
-struct Cfg2 {
+struct Cfg3 {
   static constexpr int RBLK = DK > 128 ? 2 : 1;
   static constexpr int MR = DK >= 128 ? 128 : 64;
-  static constexpr int WARPS_S = 4 * RBLK;            // state group warps
+  static constexpr int WARPS_S = 4 * RBLK;
   static constexpr int WARP_S0 = 4;
   static constexpr int WARP_CONV0 = WARP_S0 + WARPS_S;
   static constexpr int WARP_TMA = WARP_CONV0 + 4;
@@ -585,19 +591,21 @@ struct Cfg2 {
   static constexpr int STAGE = 2 * QBYTES + VBYTES;
   static constexpr int PBYTES = T * T * 2;
   static constexpr int RBYTES = DK * kDVS * 2;
-  // TMEM: O[2], S[SBUF], dR[2] x RBLK (64 columns each for the 64-wide slice)
-  static constexpr int SBUF = (2 * kDVS + 2 * T + 2 * RBLK * kDVS) <= 512 ? 2 : 1;
+  // TMEM: O[2], X[2] (64 columns each), S[SBUF] (T columns), dR[DRBUF] (RBLK x 64 columns).
+  static constexpr int SBUF = (4 * kDVS + 2 * T + RBLK * kDVS <= 512) ? 2 : 1;
+  static constexpr int DRBUF = (4 * kDVS + SBUF * T + 2 * RBLK * kDVS <= 512) ? 2 : 1;
   static constexpr int COL_O = 0;
-  static constexpr int COL_S = 2 * kDVS;
-  static constexpr int COL_DR = 2 * kDVS + SBUF * T;
-  static constexpr int USED = COL_DR + 2 * RBLK * kDVS;
+  static constexpr int COL_X = 2 * kDVS;
+  static constexpr int COL_S = 4 * kDVS;
+  static constexpr int COL_DR = 4 * kDVS + SBUF * T;
+  static constexpr int USED = COL_DR + DRBUF * RBLK * kDVS;
   static constexpr int TMEM_COLS = USED <= 128 ? 128 : (USED <= 256 ? 256 : 512);
-  // shared memory: stages, P[PBUF], R16[RBUF], rotation table, barriers
-  static constexpr int NBARS = 3 * 4 + 2 * 10 + 1;
-  static constexpr int TABBYTES = 2 * (DK / 2) * 8;
+  // shared memory: stages, P[PBUF], R16[RBUF], rotation tables (Q and K, double-buffered), barriers
+  static constexpr int NBARS = 3 * 4 + 2 * 10 + 2;
+  static constexpr int TABBYTES = 2 * 2 * (DK / 2) * 8;
   static constexpr int BUDGET = 227 * 1024 - 1024;
   static constexpr int TAIL = TABBYTES + NBARS * 8 + 16;
-  static constexpr int PBUF = (2 * STAGE + 2 * PBYTES + 2 * RBYTES + TAIL <= BUDGET) ? 2 : 1;
+  static constexpr int PBUF = (2 * STAGE + 2 * PBYTES + RBYTES + TAIL <= BUDGET) ? 2 : 1;
   static constexpr int RBUF = (2 * STAGE + PBUF * PBYTES + 2 * RBYTES + TAIL <= BUDGET) ? 2 : 1;
   static constexpr int FIXED = PBUF * PBYTES + RBUF * RBYTES + TAIL;
   static constexpr int NS_FIT = (BUDGET - FIXED) / STAGE;
@@ -606,40 +614,31 @@ struct Cfg2 {
   static constexpr bool FITS = NS >= 2 && USED <= 512;
 };
 
-// Barrier slots of the pipelined kernel (pairs are [chunk parity]).
+// Barrier slots of the pipelined kernel ([2] = indexed by buffer).
 enum : int {
-  Q_TMA_FULL = 0,      // [4]
-  Q_CONV_FULL = 4,     // [4]
-  Q_STAGE_EMPTY = 8,   // [4]
-  Q_S_FULL = 12,       // [2]
-  Q_S_FREE = 14,       // [2]
-  Q_P_FULL = 16,       // [2]
-  Q_P_FREE = 18,       // [2]
-  Q_DR_FULL = 20,      // [2]
-  Q_DR_FREE = 22,      // [2]
-  Q_R16_FULL = 24,     // [2]
-  Q_R16_FREE = 26,     // [2]
-  Q_O_FULL = 28,       // [2]
-  Q_O_FREE = 30,       // [2]
+  Q_TMA_FULL = 0,      // [4] stage landed (TMA transaction count)
+  Q_CONV_FULL = 4,     // [4] stage converted (128 converters)
+  Q_STAGE_EMPTY = 8,   // [4] stage consumed (MMA commit)
+  Q_S_FULL = 12,       // [2] S'' of a unit in TMEM (commit)
+  Q_S_FREE = 14,       // [2] S read by the P group
+  Q_P_FULL = 16,       // [2] P in shared memory
+  Q_P_FREE = 18,       // [2] P consumed by the P V product (commit)
+  Q_DR_FULL = 20,      // [2] state increment Kz^T V in TMEM (commit)
+  Q_DR_FREE = 22,      // [2] increment read by the state group
+  Q_R16_FULL = 24,     // [2] fp16 chunk-start state written (state group)
+  Q_R16_FREE = 26,     // [2] every cross term of that chunk done (commit)
+  Q_O_FULL = 28,       // [2] O (and X) of a row block complete (commit)
+  Q_O_FREE = 30,       // [2] O/X read by the epilogue
   Q_DRAIN = 32,
-  Q_TAB = 33           // [2]
+  Q_TAB = 33           // [2] rotation tables written (converters)
 };
 
-__device__ __forceinline__ uint64_t f2_bits(float2 v) { return *reinterpret_cast<uint64_t*>(&v); }
-__device__ __forceinline__ float2 bits_f2(uint64_t u) { return *reinterpret_cast<float2*>(&u); }
-// Packed fp32 pair arithmetic (two lanes per instruction on sm_100).
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
-  uint64_t r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)), "l"(f2_bits(c)));
-  return bits_f2(r);
-}
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
-  uint64_t r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)));
-  return bits_f2(r);
+__device__ __forceinline__ float2 cpow_mul(float2 base, float2 step, int n) {
+  for (int i = 0; i < n; ++i) base = cmul(base, step);
+  return base;
 }
 
-// s / c_p of the normalisations (fp32; relative error a few ulp): see row_factor in common.cuh.
+// s / c_p of the normalisations in fp32 (see row_factor in common.cuh; relative error a few ulp).
 __device__ __forceinline__ float row_factor_f32(float gamma, float sqrt_dk_inv, int64_t p, uint32_t flags) {
   float f = (flags & RETNET_F_SCALE_SQRT_D) ? sqrt_dk_inv : 1.f;
   if (flags & RETNET_F_NORM_D) {
@@ -650,11 +649,165 @@ __device__ __forceinline__ float row_factor_f32(float gamma, float sqrt_dk_inv, 
   return f;
 }
 
+// Walks the units of the whole sequence in the order every role processes them:
+// for chunk i, for row block u < nbw_i, for column block w <= u  (nbw_i = ceil(b'_i / T)).
+template <int T>
+struct UnitIter {
+  int L, nb;         // sequence length, sub-blocks per full chunk
+  int i, u, w;       // current unit
+  int nbw, bl;       // sub-blocks and length of chunk i
+  int k;             // unit sequence number
+  int rb;            // row-block sequence number (for O/X buffers)
+  int dr;            // sequence number of state-increment units (u == nbw - 1)
+  __device__ void start(int L_, int nb_) {
+    L = L_;
+    nb = nb_;
+    i = 0; u = 0; w = 0; k = 0; rb = 0; dr = 0;
+    set_chunk();
+  }
+  __device__ void set_chunk() {
+    bl = min(nb * T, L - i * nb * T);
+    nbw = (bl + T - 1) / T;
+  }
+  __device__ bool valid() const { return i * nb * T < L; }
+  __device__ bool last_row() const { return u == nbw - 1; }  // this unit carries a state increment
+  __device__ bool rb_done() const { return w == u; }         // last unit of its row block
+  __device__ int t0() const { return i * nb * T; }          // chunk start (token)
+  __device__ void next() {
+    if (last_row()) ++dr;
+    ++k;
+    if (w < u) { ++w; return; }
+    ++rb;
+    w = 0;
+    if (u + 1 < nbw) { ++u; return; }
+    u = 0;
+    ++i;
+    if (valid()) set_chunk();
+  }
+};
+
+// Converter role of the pipelined kernel: like Converter, with the sub-block-local row scales
+// and separate rotation bases for the unit's query rows (block u) and key rows (block w).
+template <int DK, int T>
+struct UnitConverter {
+  static constexpr int CS = DK / 8;    // 16-byte column slots across the DK/64 boxes
+  static constexpr int RS = 128 / CS;  // row step of one thread
+  static constexpr int NR = T / RS;    // rows per thread
+  float2 W[4], Z[4];                   // e^{i r0 theta_j}, e^{i RS theta_j} for the thread's pairs
+  float2 cur, stepT, stepB;            // table producer (lt < DK/2): chunk base, e^{iT theta}, e^{iB theta}
+  int cs, r0, lt, cur_chunk;
+
+  __device__ void init(int lt_, int nb, const HeadParams& hp) {
+    lt = lt_;
+    cs = lt % CS;
+    r0 = lt / CS;
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const float th = hp.theta[4 * cs + jj];
+      float sn, c;
+      sincosf(static_cast<float>(r0) * th, &sn, &c);
+      W[jj] = make_float2(c, sn);
+      sincosf(static_cast<float>(RS) * th, &sn, &c);
+      Z[jj] = make_float2(c, sn);
+    }
+    cur = stepT = stepB = make_float2(1.f, 0.f);
+    cur_chunk = -1;
+    if (lt < DK / 2) {
+      float sn, c;
+      xpos_sincos(T, hp.theta[lt], &sn, &c);
+      stepT = make_float2(c, sn);
+      xpos_sincos(static_cast<int64_t>(nb) * T, hp.theta[lt], &sn, &c);
+      stepB = make_float2(c, sn);
+    }
+  }
+
+  // Rotation bases e^{i p theta_j} of the unit's query rows (p = pos0 + t0 + uT) and key rows
+  // (p = pos0 + t0 + wT), j = lt.  The chunk base advances by an fp32 complex product and is
+  // recomputed from the fp64-reduced angle every 64 chunks (drift below ~1e-5 rad).
+  __device__ void put_bases(float2* tq, float2* tk, int chunk, int u, int w, int t0, int64_t pos0,
+                            const HeadParams& hp) {
+    if (lt >= DK / 2) return;
+    if (chunk != cur_chunk) {
+      if ((chunk & 63) == 0 || cur_chunk < 0) {
+        float sn, c;
+        xpos_sincos(pos0 + t0, hp.theta[lt], &sn, &c);
+        cur = make_float2(c, sn);
+      } else {
+        cur = cmul(cur, stepB);
+      }
+      cur_chunk = chunk;
+    }
+    tq[lt] = cpow_mul(cur, stepT, u);
+    tk[lt] = cpow_mul(cur, stepT, w);
+  }
+
+  // In place: q -> gamma^(r+1) rot(q), k -> gamma^(T-1-r) rot(k) as fp16 (r local); v -> fp16.
+  __device__ void convert(uint32_t sq, uint32_t sk, uint32_t sv, const float2* bq, const float2* bk, bool xpos,
+                          float log2g) const {
+    const uint32_t box = (cs / 8) * T * 128;
+    const uint32_t chunk = cs % 8;
+    const float xstep = decay_pow(log2g, RS), zstep = exp2f(-static_cast<float>(RS) * log2g);
+    float xi = decay_pow(log2g, r0 + 1);
+    float zeta = decay_pow(log2g, T - 1 - r0);
+    float2 Fq[4], Fk[4];
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      Fq[jj] = xpos ? cmul(bq[4 * cs + jj], W[jj]) : make_float2(1.f, 0.f);
+      Fk[jj] = xpos ? cmul(bk[4 * cs + jj], W[jj]) : make_float2(1.f, 0.f);
+    }
+    static_assert(NR % 4 == 0, "rows per thread must be a multiple of 4");
+#pragma unroll 1
+    for (int kg = 0; kg < NR; kg += 4) {
+      uint32_t q4[4][4], k4[4][4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t off = box + sw128(r0 + RS * (kg + k), chunk);
+        ld_shared_v4(sq + off, q4[k][0], q4[k][1], q4[k][2], q4[k][3]);
+        ld_shared_v4(sk + off, k4[k][0], k4[k][1], k4[k][2], k4[k][3]);
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        uint32_t qo[4], ko[4];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const float q0 = __uint_as_float(q4[k][jj] << 16), q1 = __uint_as_float(q4[k][jj] & 0xffff0000u);
+          const float k0 = __uint_as_float(k4[k][jj] << 16), k1 = __uint_as_float(k4[k][jj] & 0xffff0000u);
+          const float cq = Fq[jj].x, sq_ = Fq[jj].y, ck = Fk[jj].x, sk_ = Fk[jj].y;
+          qo[jj] = pack_f16x2(xi * (q0 * cq - q1 * sq_), xi * (q0 * sq_ + q1 * cq));
+          ko[jj] = pack_f16x2(zeta * (k0 * ck - k1 * sk_), zeta * (k0 * sk_ + k1 * ck));
+          Fq[jj] = cmul(Fq[jj], Z[jj]);
+          Fk[jj] = cmul(Fk[jj], Z[jj]);
+        }
+        const uint32_t off = box + sw128(r0 + RS * (kg + k), chunk);
+        st_shared_v4(sq + off, qo[0], qo[1], qo[2], qo[3]);
+        st_shared_v4(sk + off, ko[0], ko[1], ko[2], ko[3]);
+        xi *= xstep;
+        zeta *= zstep;
+      }
+    }
+#pragma unroll 1
+    for (int kg = 0; kg < T / 16; kg += 4) {
+      uint32_t v4[4][4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        ld_shared_v4(sv + sw128(lt / 8 + 16 * (kg + k), lt % 8), v4[k][0], v4[k][1], v4[k][2], v4[k][3]);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        uint32_t vo[4];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj)
+          vo[jj] = pack_f16x2(__uint_as_float(v4[k][jj] << 16), __uint_as_float(v4[k][jj] & 0xffff0000u));
+        st_shared_v4(sv + sw128(lt / 8 + 16 * (kg + k), lt % 8), vo[0], vo[1], vo[2], vo[3]);
+      }
+    }
+  }
+};
+
 template <int DK, int T, typename Tout>
-__global__ void __launch_bounds__(Cfg2<DK, T>::THREADS, 1)
+__global__ void __launch_bounds__(Cfg3<DK, T>::THREADS, 1)
     tc_chunkwise_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v, TcArgs a, HeadParams hp) {
-  using C = Cfg2<DK, T>;
+  using C = Cfg3<DK, T>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_addr(smem_raw);
   const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
@@ -663,7 +816,7 @@ __global__ void __launch_bounds__(Cfg2<DK, T>::THREADS, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int dvb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const float log2g = hp.log2g[h];
-  const int n = a.n_chunks;
+  const int nb = a.nb;
   const float sd = rsqrtf(static_cast<float>(DK));  // carried by P and the fp16 state copy
 
   const uint32_t sP0 = sbase + C::NS * C::STAGE;
@@ -676,8 +829,8 @@ __global__ void __launch_bounds__(Cfg2<DK, T>::THREADS, 1)
   auto sQ = [&](int s) { return sbase + s * C::STAGE; };
   auto sK = [&](int s) { return sbase + s * C::STAGE + C::QBYTES; };
   auto sV = [&](int s) { return sbase + s * C::STAGE + 2 * C::QBYTES; };
-  auto sP = [&](int j) { return sP0 + (j % C::PBUF) * C::PBYTES; };
-  auto sR = [&](int j) { return sR0 + (j % C::RBUF) * C::RBYTES; };
+  auto sP = [&](int k) { return sP0 + (k % C::PBUF) * C::PBYTES; };
+  auto sR = [&](int i) { return sR0 + (i % C::RBUF) * C::RBYTES; };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < 4; ++s) {
@@ -719,19 +872,21 @@ __global__ void __launch_bounds__(Cfg2<DK, T>::THREADS, 1)
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int issued[4] = {0, 0, 0, 0};
-      for (int i = 0; i < n; ++i) {
-        const int s = i % C::NS;
-        if (i >= C::NS && !mbar_wait(bar(Q_STAGE_EMPTY + s), ((i / C::NS) - 1) & 1)) break;
+      UnitIter<T> it;
+      for (it.start(a.L, nb); it.valid(); it.next()) {
+        const int s = it.k % C::NS;
+        if (it.k >= C::NS && !mbar_wait(bar(Q_STAGE_EMPTY + s), ((it.k / C::NS) - 1) & 1)) break;
         mbar_arrive_expect_tx(bar(Q_TMA_FULL + s), C::STAGE);
-        const int t0 = i * T;
+        const int tq = it.t0() + it.u * T, tk = it.t0() + it.w * T;
 #pragma unroll
         for (int bx = 0; bx < DK / 64; ++bx) {
-          tma_load_4d(sQ(s) + bx * T * 128, &tm_q, bar(Q_TMA_FULL + s), bx * 64, h, t0, b);
-          tma_load_4d(sK(s) + bx * T * 128, &tm_k, bar(Q_TMA_FULL + s), bx * 64, h, t0, b);
+          tma_load_4d(sQ(s) + bx * T * 128, &tm_q, bar(Q_TMA_FULL + s), bx * 64, h, tq, b);
+          tma_load_4d(sK(s) + bx * T * 128, &tm_k, bar(Q_TMA_FULL + s), bx * 64, h, tk, b);
         }
-        tma_load_4d(sV(s), &tm_v, bar(Q_TMA_FULL + s), dvb * kDVS, h, t0, b);
+        tma_load_4d(sV(s), &tm_v, bar(Q_TMA_FULL + s), dvb * kDVS, h, tk, b);
         issued[s]++;
       }
+      // Every load this thread issued must have landed before the CTA may exit.
       for (int s = 0; s < C::NS; ++s)
         if (issued[s] > 0) mbar_wait(bar(Q_TMA_FULL + s), (issued[s] - 1) & 1);
     }
@@ -741,91 +896,105 @@ __global__ void __launch_bounds__(Cfg2<DK, T>::THREADS, 1)
       constexpr uint32_t ID_S = idesc_f16_f32(T, T, 0, 0);
       constexpr uint32_t ID_X = idesc_f16_f32(T, kDVS, 0, 1);
       constexpr uint32_t ID_R = idesc_f16_f32(C::MR, kDVS, 1, 1);
-      bool ok = true;
-      // S_j and dR_j: need chunk j converted and its S / dR buffers released.
-      // Descriptors are built once per operand tile and advanced per MMA by a constant: the
-      // start-address field (address >> 4, bits 0-13) never carries, since every operand lies
-      // below 256 KB of shared memory.  K-major tiles advance 32 B per K step inside a
-      // 128-byte row and T*128 B per 64-wide box; MN-major tiles advance 2048 B per 16 rows.
+      // Descriptors are built once per operand tile and advanced by constants (the start
+      // address field never carries: every operand lies below 256 KB of shared memory).
       auto kstep = [](int kk) -> uint64_t { return static_cast<uint64_t>(((kk / 4) * T * 128 + (kk % 4) * 32) >> 4); };
-      auto front = [&](int j) -> bool {
-        const int s = j % C::NS;
-        if (!mbar_wait(bar(Q_CONV_FULL + s), (j / C::NS) & 1)) return false;
-        if (j >= C::SBUF && !mbar_wait(bar(Q_S_FREE + (j % C::SBUF)), ((j - C::SBUF) / C::SBUF) & 1)) return false;
-        if (j >= 2 && !mbar_wait(bar(Q_DR_FREE + (j & 1)), ((j - 2) >> 1) & 1)) return false;
+      // S'' of the unit and, for the last row block, the state increment Kz_w^T V_w.
+      auto front = [&](const UnitIter<T>& f) -> bool {
+        const int s = f.k % C::NS;
+        if (!mbar_wait(bar(Q_CONV_FULL + s), (f.k / C::NS) & 1)) return false;
+        if (f.k >= C::SBUF && !mbar_wait(bar(Q_S_FREE + (f.k % C::SBUF)), ((f.k - C::SBUF) / C::SBUF) & 1)) return false;
+        if (f.last_row() && f.dr >= C::DRBUF &&
+            !mbar_wait(bar(Q_DR_FREE + (f.dr % C::DRBUF)), ((f.dr - C::DRBUF) / C::DRBUF) & 1))
+          return false;
         tc_fence_after();
-        const uint32_t tS = tmem + C::COL_S + (j % C::SBUF) * T;
+        const uint32_t tS = tmem + C::COL_S + (f.k % C::SBUF) * T;
         const uint64_t dq = sdesc_sw128(sQ(s), 16, 1024), dk = sdesc_sw128(sK(s), 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk) mma_f16_ss(tS, dq + kstep(kk), dk + kstep(kk), ID_S, kk > 0);
-        mma_commit(bar(Q_S_FULL + (j % C::SBUF)));
-        const uint32_t tD = tmem + C::COL_DR + (j & 1) * C::RBLK * kDVS;
-        const uint64_t dkm = sdesc_sw128(sK(s), T * 128, 1024), dv = sdesc_sw128(sV(s), T * 128, 1024);
+        mma_commit(bar(Q_S_FULL + (f.k % C::SBUF)));
+        if (f.last_row()) {
+          const uint32_t tD = tmem + C::COL_DR + (f.dr % C::DRBUF) * C::RBLK * kDVS;
+          const uint64_t dkm = sdesc_sw128(sK(s), T * 128, 1024), dv = sdesc_sw128(sV(s), T * 128, 1024);
 #pragma unroll
-        for (int blk = 0; blk < C::RBLK; ++blk)
+          for (int blk = 0; blk < C::RBLK; ++blk)
 #pragma unroll
-          for (int ks = 0; ks < T / 16; ++ks)
-            mma_f16_ss(tD + blk * kDVS, dkm + static_cast<uint64_t>((blk * 2 * T * 128 + ks * 2048) >> 4),
-                       dv + static_cast<uint64_t>((ks * 2048) >> 4), ID_R, ks > 0);
-        mma_commit(bar(Q_DR_FULL + (j & 1)));
+            for (int ks = 0; ks < T / 16; ++ks)
+              mma_f16_ss(tD + blk * kDVS, dkm + static_cast<uint64_t>((blk * 2 * T * 128 + ks * 2048) >> 4),
+                         dv + static_cast<uint64_t>((ks * 2048) >> 4), ID_R, ks > 0);
+          mma_commit(bar(Q_DR_FULL + (f.dr % C::DRBUF)));
+        }
         return true;
       };
-      // cross_j and P_j V_j into O_j: need the entering state R_{j-1}, O buffer and P_j.
-      auto back = [&](int j) -> bool {
-        const int s = j % C::NS;
-        if (!mbar_wait(bar(Q_R16_FULL + (j % C::RBUF)), (j / C::RBUF) & 1)) return false;
-        if (j >= 2 && !mbar_wait(bar(Q_O_FREE + (j & 1)), ((j - 2) >> 1) & 1)) return false;
-        tc_fence_after();
-        const uint32_t tO = tmem + C::COL_O + (j & 1) * kDVS;
-        const uint64_t dq = sdesc_sw128(sQ(s), 16, 1024), dr = sdesc_sw128(sR(j), DK * 128, 1024);
+      // Cross term of the row block (first unit only) and P V into O.
+      auto back = [&](const UnitIter<T>& q) -> bool {
+        const int s = q.k % C::NS;
+        const uint32_t tO = tmem + C::COL_O + (q.rb & 1) * kDVS;
+        if (q.w == 0) {
+          if (!mbar_wait(bar(Q_R16_FULL + (q.i % C::RBUF)), (q.i / C::RBUF) & 1)) return false;
+          if (q.rb >= 2 && !mbar_wait(bar(Q_O_FREE + (q.rb & 1)), ((q.rb - 2) >> 1) & 1)) return false;
+          tc_fence_after();
+          const uint32_t tX = (nb > 1) ? tmem + C::COL_X + (q.rb & 1) * kDVS : tO;
+          const uint64_t dq = sdesc_sw128(sQ(s), 16, 1024), dr = sdesc_sw128(sR(q.i), DK * 128, 1024);
 #pragma unroll
-        for (int kk = 0; kk < DK / 16; ++kk)
-          mma_f16_ss(tO, dq + kstep(kk), dr + static_cast<uint64_t>((kk * 2048) >> 4), ID_X, kk > 0);
-        mma_commit(bar(Q_R16_FREE + (j % C::RBUF)));
-        if (!mbar_wait(bar(Q_P_FULL + (j % C::PBUF)), (j / C::PBUF) & 1)) return false;
+          for (int kk = 0; kk < DK / 16; ++kk)
+            mma_f16_ss(tX, dq + kstep(kk), dr + static_cast<uint64_t>((kk * 2048) >> 4), ID_X, kk > 0);
+          if (q.last_row()) mma_commit(bar(Q_R16_FREE + (q.i % C::RBUF)));
+        }
+        if (!mbar_wait(bar(Q_P_FULL + (q.k % C::PBUF)), (q.k / C::PBUF) & 1)) return false;
         tc_fence_after();
-        const uint64_t dp = sdesc_sw128(sP(j), 16, 1024), dv = sdesc_sw128(sV(s), T * 128, 1024);
+        const uint64_t dp = sdesc_sw128(sP(q.k), 16, 1024), dv = sdesc_sw128(sV(s), T * 128, 1024);
+        const uint32_t acc0 = (q.w > 0 || nb == 1) ? 1u : 0u;
 #pragma unroll
         for (int kk = 0; kk < T / 16; ++kk)
-          mma_f16_ss(tO, dp + kstep(kk), dv + static_cast<uint64_t>((kk * 2048) >> 4), ID_X, 1);
-        mma_commit(bar(Q_O_FULL + (j & 1)));
-        mma_commit(bar(Q_P_FREE + (j % C::PBUF)));
+          mma_f16_ss(tO, dp + kstep(kk), dv + static_cast<uint64_t>((kk * 2048) >> 4), ID_X, kk > 0 ? 1u : acc0);
+        mma_commit(bar(Q_P_FREE + (q.k % C::PBUF)));
+        if (q.rb_done()) mma_commit(bar(Q_O_FULL + (q.rb & 1)));
         mma_commit(bar(Q_STAGE_EMPTY + s));
         return true;
       };
-      ok = front(0);
-      for (int j = 0; j < n && ok; ++j) {
-        if (j + 1 < n) ok = front(j + 1);
-        if (ok) ok = back(j);
+      UnitIter<T> f, q;
+      f.start(a.L, nb);
+      q.start(a.L, nb);
+      bool ok = front(f);
+      f.next();
+      while (ok && q.valid()) {
+        if (f.valid()) {
+          ok = front(f);
+          f.next();
+        }
+        if (ok) ok = back(q);
+        q.next();
       }
       mma_commit(bar(Q_DRAIN));
       mbar_wait(bar(Q_DRAIN), 0);
     }
   } else if (warp >= C::WARP_CONV0) {
     // ------------------------------------------------------------------ converters
-    Converter<DK, T> cv;
-    cv.init(threadIdx.x - 32 * C::WARP_CONV0, hp);
+    UnitConverter<DK, T> cv;
+    cv.init(threadIdx.x - 32 * C::WARP_CONV0, nb, hp);
     const bool xpos = (a.flags & RETNET_F_XPOS) != 0;
     bool ok = true;
-    for (int i = 0; i < n && ok; ++i) {
-      const int s = i % C::NS;
-      const int bl = min(T, a.L - i * T);
-      float2* base = tab + (i & 1) * (DK / 2);
-      if (xpos) cv.put_base(base, i, a.pos0, hp);
-      // The table buffer (i & 1) is complete once all 128 converters arrived; a thread that
-      // rewrites it two chunks later has passed this wait, so every read of it is done.
-      mbar_arrive(bar(Q_TAB + (i & 1)));
-      ok = mbar_wait(bar(Q_TAB + (i & 1)), (i >> 1) & 1);
-      if (ok) ok = mbar_wait(bar(Q_TMA_FULL + s), (i / C::NS) & 1);
+    UnitIter<T> it;
+    for (it.start(a.L, nb); ok && it.valid(); it.next()) {
+      const int s = it.k % C::NS;
+      float2* tq = tab + (it.k & 1) * DK;
+      float2* tk = tq + DK / 2;
+      if (xpos) cv.put_bases(tq, tk, it.i, it.u, it.w, it.t0(), a.pos0, hp);
+      // Table buffer (k & 1) is complete once all 128 converters arrived; a thread that
+      // rewrites it two units later has passed this wait, so every read of it is done.
+      mbar_arrive(bar(Q_TAB + (it.k & 1)));
+      ok = mbar_wait(bar(Q_TAB + (it.k & 1)), (it.k >> 1) & 1);
+      if (ok) ok = mbar_wait(bar(Q_TMA_FULL + s), (it.k / C::NS) & 1);
       if (!ok) break;
-      cv.convert(sQ(s), sK(s), sV(s), base, xpos, log2g, bl);
+      cv.convert(sQ(s), sK(s), sV(s), tq, tk, xpos, log2g);
       fence_proxy_async_smem();
       mbar_arrive(bar(Q_CONV_FULL + s));
     }
   } else if (warp >= C::WARP_S0) {
     // ------------------------------------------------------------------ state group
-    const int ws = warp - C::WARP_S0;           // 0 .. 4*RBLK-1
-    const int blk = ws / 4;                     // 128-row block of the state
+    const int ws = warp - C::WARP_S0;
+    const int blk = ws / 4;
     const uint32_t lane_off = static_cast<uint32_t>(32 * (warp % 4)) << 16;
     const int dk = (DK == 64) ? (lane < 16 ? 16 * (warp % 4) + lane : -1) : blk * 128 + 32 * (warp % 4) + lane;
     const int64_t bh = static_cast<int64_t>(b) * a.heads + h;
@@ -854,29 +1023,38 @@ __global__ void __launch_bounds__(Cfg2<DK, T>::THREADS, 1)
     fence_proxy_async_smem();
     mbar_arrive(bar(Q_R16_FULL + 0));
     bool ok = true;
-    for (int i = 0; i < n && ok; ++i) {
-      const int bl = min(T, a.L - i * T);
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(Q_DR_FULL + (i & 1)), (i >> 1) & 1));
+    UnitIter<T> it;
+    for (it.start(a.L, nb); ok && it.valid(); it.next()) {
+      if (!it.last_row()) continue;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(Q_DR_FULL + (it.dr % C::DRBUF)), (it.dr / C::DRBUF) & 1));
       if (!ok) break;
       tc_fence_after();
       uint32_t u[4][16];
-      const uint32_t tD = tmem + C::COL_DR + (i & 1) * C::RBLK * kDVS + blk * kDVS + lane_off;
+      const uint32_t tD = tmem + C::COL_DR + (it.dr % C::DRBUF) * C::RBLK * kDVS + blk * kDVS + lane_off;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) tmem_ld16(tD + 16 * q, u[q]);
+      for (int q4 = 0; q4 < 4; ++q4) tmem_ld16(tD + 16 * q4, u[q4]);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(bar(Q_DR_FREE + (i & 1)));
-      const float g = decay_pow(log2g, bl);
+      mbar_arrive(bar(Q_DR_FREE + (it.dr % C::DRBUF)));
+      // Horner form of R_i = gamma^b' R_{i-1} + sum_w gamma^(b'-(w+1)T) dR_w:
+      //   w = 0: R = gamma^(b'-(nbw-1)T) R + hh dR_0;  w > 0: R = gamma^T R + hh dR_w,
+      //   hh = gamma^(b' - nbw T) (1 for a full chunk).
+      const float g = (it.w == 0) ? exp2f(static_cast<float>(it.bl - (it.nbw - 1) * T) * log2g)
+                                  : decay_pow(log2g, T);
+      const float hh = exp2f(static_cast<float>(it.bl - it.nbw * T) * log2g);
 #pragma unroll
-      for (int c = 0; c < kDVS; ++c) R[c] = fmaf(g, R[c], __uint_as_float(u[c / 16][c % 16]));
-      if (i + 1 < n) {
-        // R16 buffer for chunk i+1 was last read by the cross term of chunk i+1-RBUF.
-        const int prev = i + 1 - C::RBUF;
-        if (prev >= 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(Q_R16_FREE + (prev % C::RBUF)), (prev / C::RBUF) & 1));
+      for (int c = 0; c < kDVS; ++c) R[c] = fmaf(g, R[c], hh * __uint_as_float(u[c / 16][c % 16]));
+      if (it.w + 1 < it.nbw) continue;  // chunk not finished
+      const int nxt = it.i + 1;
+      if (nxt * nb * T < a.L) {
+        // R16 buffer of chunk nxt was last read by the cross terms of chunk nxt - RBUF.
+        const int prev = nxt - C::RBUF;
+        if (prev >= 0)
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(Q_R16_FREE + (prev % C::RBUF)), (prev / C::RBUF) & 1));
         if (!ok) break;
-        put_r16(sR(i + 1));
+        put_r16(sR(nxt));
         fence_proxy_async_smem();
-        mbar_arrive(bar(Q_R16_FULL + ((i + 1) % C::RBUF)));
+        mbar_arrive(bar(Q_R16_FULL + (nxt % C::RBUF)));
       } else if (dk >= 0 && a.state_out) {
         float* dst = a.state_out + static_cast<size_t>(bh) * DK * a.dv + dvb * kDVS + dk * srow;
 #pragma unroll
@@ -889,63 +1067,79 @@ __global__ void __launch_bounds__(Cfg2<DK, T>::THREADS, 1)
     const uint32_t lane_off = static_cast<uint32_t>(32 * warp) << 16;
     const int my_row = (T == 128) ? 32 * warp + lane : (lane < 16 ? 16 * warp + lane : -1);
     const float gam = hp.gamma[h];
-    auto epilogue = [&](int j) -> bool {
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(Q_O_FULL + (j & 1)), (j >> 1) & 1))) return false;
+    // Epilogue of row block (chunk i, block u), O/X buffer rb & 1.
+    auto epilogue = [&](int rb, int i, int u, int bl) -> bool {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(Q_O_FULL + (rb & 1)), (rb >> 1) & 1))) return false;
       tc_fence_after();
-      uint32_t u[4][16];
+      const int rows = min(T, bl - u * T);
+      const bool live = my_row >= 0 && my_row < rows;
+      const int t = i * nb * T + u * T + (my_row < 0 ? 0 : my_row);
+      const float f = row_factor_f32(gam, sd, a.pos0 + t, a.flags) / sd;
+      const float gx = (nb > 1) ? exp2f(static_cast<float>(u * T) * log2g) : 0.f;
+      Tout* dst = static_cast<Tout*>(a.o) + ((static_cast<int64_t>(b) * a.L + t) * a.heads + h) * a.dv + dvb * kDVS;
+      // 16 columns at a time: O (and X) from TMEM, o = (O + gamma^(uT) X) * s / c_p, 16-byte stores.
+#pragma unroll 1
+      for (int q = 0; q < 4; ++q) {
+        uint32_t uo[16], ux[16];
+        tmem_ld16(tmem + C::COL_O + (rb & 1) * kDVS + 16 * q + lane_off, uo);
+        if (nb > 1) tmem_ld16(tmem + C::COL_X + (rb & 1) * kDVS + 16 * q + lane_off, ux);
+        tmem_wait_ld();
+        if (q == 3) {
+          tc_fence_before();
+          mbar_arrive(bar(Q_O_FREE + (rb & 1)));
+        }
+        if (live) {
+          float ov[16];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) tmem_ld16(tmem + C::COL_O + (j & 1) * kDVS + 16 * q + lane_off, u[q]);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar(Q_O_FREE + (j & 1)));
-      const int t0 = j * T;
-      const int bl = min(T, a.L - t0);
-      if (my_row >= 0 && my_row < bl) {
-        const float f = row_factor_f32(gam, sd, a.pos0 + t0 + my_row, a.flags) / sd;
-        const int64_t orow = ((static_cast<int64_t>(b) * a.L + t0 + my_row) * a.heads + h) * a.dv + dvb * kDVS;
-        Tout* dst = static_cast<Tout*>(a.o) + orow;
-        if constexpr (sizeof(Tout) == 2) {
-#pragma unroll
-          for (int c8 = 0; c8 < 8; ++c8) {
-            uint32_t pk[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              __nv_bfloat162 v2 = __floats2bfloat162_rn(f * __uint_as_float(u[c8 / 2][(8 * c8 + 2 * e) % 16]),
-                                                        f * __uint_as_float(u[c8 / 2][(8 * c8 + 2 * e + 1) % 16]));
-              pk[e] = *reinterpret_cast<uint32_t*>(&v2);
-            }
-            *reinterpret_cast<uint4*>(dst + 8 * c8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          for (int c = 0; c < 16; ++c) {
+            float x = __uint_as_float(uo[c]);
+            if (nb > 1) x = fmaf(gx, __uint_as_float(ux[c]), x);
+            ov[c] = f * x;
           }
-        } else {
+          if constexpr (sizeof(Tout) == 2) {
 #pragma unroll
-          for (int c4 = 0; c4 < 16; ++c4)
-            *reinterpret_cast<float4*>(dst + 4 * c4) =
-                make_float4(f * __uint_as_float(u[c4 / 4][(4 * c4) % 16]), f * __uint_as_float(u[c4 / 4][(4 * c4 + 1) % 16]),
-                            f * __uint_as_float(u[c4 / 4][(4 * c4 + 2) % 16]), f * __uint_as_float(u[c4 / 4][(4 * c4 + 3) % 16]));
+            for (int c8 = 0; c8 < 2; ++c8) {
+              uint32_t pk[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                __nv_bfloat162 v2 = __floats2bfloat162_rn(ov[8 * c8 + 2 * e], ov[8 * c8 + 2 * e + 1]);
+                pk[e] = *reinterpret_cast<uint32_t*>(&v2);
+              }
+              *reinterpret_cast<uint4*>(dst + 16 * q + 8 * c8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+          } else {
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4)
+              *reinterpret_cast<float4*>(dst + 16 * q + 4 * c4) =
+                  make_float4(ov[4 * c4], ov[4 * c4 + 1], ov[4 * c4 + 2], ov[4 * c4 + 3]);
+          }
         }
       }
       return true;
     };
     bool ok = true;
-    for (int j = 0; j < n && ok; ++j) {
-      const int bl = min(T, a.L - j * T);
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(Q_S_FULL + (j % C::SBUF)), (j / C::SBUF) & 1));
+    int pend_rb = -1, pend_i = 0, pend_u = 0, pend_bl = 0;  // a finished row block awaiting its epilogue
+    UnitIter<T> it;
+    for (it.start(a.L, nb); ok && it.valid(); it.next()) {
+      const int k = it.k;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(Q_S_FULL + (k % C::SBUF)), (k / C::SBUF) & 1));
+      if (ok && k >= C::PBUF)
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(Q_P_FREE + (k % C::PBUF)), ((k - C::PBUF) / C::PBUF) & 1));
       if (!ok) break;
       tc_fence_after();
-      const float ginv = exp2f(-static_cast<float>(bl) * log2g) * sd;
-      const uint32_t tS = tmem + C::COL_S + (j % C::SBUF) * T + lane_off;
-      if (j >= C::PBUF)
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(Q_P_FREE + (j % C::PBUF)), ((j - C::PBUF) / C::PBUF) & 1));
-      if (!ok) break;
+      // P = S'' gamma^((u-w-1) T) / sqrt(d_k); causal mask on the diagonal block.
+      const float pf = exp2f(static_cast<float>((it.u - it.w - 1) * T) * log2g) * sd;
+      const bool diag = (it.u == it.w);
+      const uint32_t tS = tmem + C::COL_S + (k % C::SBUF) * T + lane_off;
 #pragma unroll
       for (int half = 0; half < T / 64; ++half) {
-        uint32_t u[4][16];
+        uint32_t u16[4][16];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) tmem_ld16(tS + half * 64 + 16 * q, u[q]);
+        for (int q = 0; q < 4; ++q) tmem_ld16(tS + half * 64 + 16 * q, u16[q]);
         tmem_wait_ld();
         if (half == T / 64 - 1) {
           tc_fence_before();
-          mbar_arrive(bar(Q_S_FREE + (j % C::SBUF)));
+          mbar_arrive(bar(Q_S_FREE + (k % C::SBUF)));
         }
         if (my_row >= 0) {
 #pragma unroll
@@ -954,19 +1148,25 @@ __global__ void __launch_bounds__(Cfg2<DK, T>::THREADS, 1)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int c0 = half * 64 + 8 * c8 + 2 * e;
-              const float p0 = (c0 <= my_row) ? __uint_as_float(u[c8 / 2][(8 * c8 + 2 * e) % 16]) * ginv : 0.f;
-              const float p1 = (c0 + 1 <= my_row) ? __uint_as_float(u[c8 / 2][(8 * c8 + 2 * e + 1) % 16]) * ginv : 0.f;
+              const float p0 = (!diag || c0 <= my_row) ? __uint_as_float(u16[c8 / 2][(8 * c8 + 2 * e) % 16]) * pf : 0.f;
+              const float p1 = (!diag || c0 + 1 <= my_row) ? __uint_as_float(u16[c8 / 2][(8 * c8 + 2 * e + 1) % 16]) * pf : 0.f;
               pk[e] = pack_f16x2(p0, p1);
             }
-            st_shared_v4(sP(j) + half * T * 128 + sw128(my_row, c8), pk[0], pk[1], pk[2], pk[3]);
+            st_shared_v4(sP(k) + half * T * 128 + sw128(my_row, c8), pk[0], pk[1], pk[2], pk[3]);
           }
         }
       }
       fence_proxy_async_smem();
-      mbar_arrive(bar(Q_P_FULL + (j % C::PBUF)));
-      if (j >= 1) ok = epilogue(j - 1);
+      mbar_arrive(bar(Q_P_FULL + (k % C::PBUF)));
+      if (pend_rb >= 0) {
+        ok = epilogue(pend_rb, pend_i, pend_u, pend_bl);
+        pend_rb = -1;
+      }
+      if (it.rb_done()) {
+        pend_rb = it.rb; pend_i = it.i; pend_u = it.u; pend_bl = it.bl;
+      }
     }
-    if (ok && n >= 1) epilogue(n - 1);
+    if (ok && pend_rb >= 0) epilogue(pend_rb, pend_i, pend_u, pend_bl);
   }
 
   tc_fence_before();
@@ -1020,53 +1220,74 @@ bool force_serial_kernel() {
   return serial;
 }
 
-template <int DK, int T, typename Tout>
-cudaError_t launch_pipe(const RetentionCall& c, const HeadParams& hp, cudaStream_t s, const CUtensorMap& mq,
-                        const CUtensorMap& mk, const CUtensorMap& mv, const TcArgs& a) {
-  using Cf = Cfg2<DK, T>;
-  auto kern = tc_chunkwise_pipe_kernel<DK, T, Tout>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM);
-  if (e != cudaSuccess) return e;
-  const Dims& d = c.dims;
-  dim3 grid(static_cast<unsigned>(d.d_v / kDVS), static_cast<unsigned>(d.heads), static_cast<unsigned>(d.batch));
-  kern<<<grid, Cf::THREADS, Cf::SMEM, s>>>(mq, mk, mv, a, hp);
-  return cudaGetLastError();
-}
+// Rows per unit of the pipelined kernel: 64 for d_k = 256 (shared memory), else min(B, 128).
+int pipe_tile_rows(int64_t d_k, int64_t chunk) { return d_k == 256 ? 64 : static_cast<int>(chunk < 128 ? chunk : 128); }
 
-template <int DK, int T, typename Tout>
-cudaError_t launch_cfg(const RetentionCall& c, const HeadParams& hp, cudaStream_t s) {
-  using Cf = Cfg<DK, T>;
-  CUtensorMap mq, mk, mv;
-  const Dims& d = c.dims;
-  if (!make_map(&mq, c.q, d.batch, d.seqlen, d.heads, d.d_k, T) ||
-      !make_map(&mk, c.k, d.batch, d.seqlen, d.heads, d.d_k, T) ||
-      !make_map(&mv, c.v, d.batch, d.seqlen, d.heads, d.d_v, T))
-    return cudaErrorInvalidValue;
+TcArgs make_args(const RetentionCall& c, int n_chunks, int nb) {
   TcArgs a;
   a.o = c.o;
   a.state_in = c.state_in;
   a.state_out = c.state_out;
-  a.L = static_cast<int>(d.seqlen);
-  a.heads = static_cast<int>(d.heads);
-  a.dv = static_cast<int>(d.d_v);
-  a.n_chunks = static_cast<int>((d.seqlen + T - 1) / T);
+  a.L = static_cast<int>(c.dims.seqlen);
+  a.heads = static_cast<int>(c.dims.heads);
+  a.dv = static_cast<int>(c.dims.d_v);
+  a.n_chunks = n_chunks;
   a.pos0 = c.pos0;
   a.flags = c.flags;
-  if constexpr (Cfg2<DK, T>::FITS) {
-    if (!force_serial_kernel()) return launch_pipe<DK, T, Tout>(c, hp, s, mq, mk, mv, a);
-  }
+  a.nb = nb;
+  return a;
+}
+
+bool make_maps(const RetentionCall& c, int T, CUtensorMap* mq, CUtensorMap* mk, CUtensorMap* mv) {
+  const Dims& d = c.dims;
+  return make_map(mq, c.q, d.batch, d.seqlen, d.heads, d.d_k, T) &&
+         make_map(mk, c.k, d.batch, d.seqlen, d.heads, d.d_k, T) &&
+         make_map(mv, c.v, d.batch, d.seqlen, d.heads, d.d_v, T);
+}
+
+dim3 tc_grid(const Dims& d) {
+  return dim3(static_cast<unsigned>(d.d_v / kDVS), static_cast<unsigned>(d.heads), static_cast<unsigned>(d.batch));
+}
+
+// Pipelined kernel: units of T rows, nb = B / T per chunk.
+template <int DK, int T, typename Tout>
+cudaError_t launch_pipe(const RetentionCall& c, const HeadParams& hp, cudaStream_t s) {
+  using Cf = Cfg3<DK, T>;
+  static_assert(Cf::FITS, "pipelined kernel does not fit this tile");
+  CUtensorMap mq, mk, mv;
+  if (!make_maps(c, T, &mq, &mk, &mv)) return cudaErrorInvalidValue;
+  const int nb = static_cast<int>(c.chunk / T);
+  const TcArgs a = make_args(c, static_cast<int>((c.dims.seqlen + c.chunk - 1) / c.chunk), nb);
+  auto kern = tc_chunkwise_pipe_kernel<DK, T, Tout>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM);
+  if (e != cudaSuccess) return e;
+  kern<<<tc_grid(c.dims), Cf::THREADS, Cf::SMEM, s>>>(mq, mk, mv, a, hp);
+  return cudaGetLastError();
+}
+
+// Serial kernel: one chunk of B = T rows per step (chunk-relative scaled operands).
+template <int DK, int T, typename Tout>
+cudaError_t launch_serial(const RetentionCall& c, const HeadParams& hp, cudaStream_t s) {
+  using Cf = Cfg<DK, T>;
+  CUtensorMap mq, mk, mv;
+  if (!make_maps(c, T, &mq, &mk, &mv)) return cudaErrorInvalidValue;
+  const TcArgs a = make_args(c, static_cast<int>((c.dims.seqlen + T - 1) / T), 1);
   auto kern = tc_chunkwise_kernel<DK, T, Tout>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM);
   if (e != cudaSuccess) return e;
-  dim3 grid(static_cast<unsigned>(d.d_v / kDVS), static_cast<unsigned>(d.heads), static_cast<unsigned>(d.batch));
-  kern<<<grid, kThreads, Cf::SMEM, s>>>(mq, mk, mv, a, hp);
+  kern<<<tc_grid(c.dims), kThreads, Cf::SMEM, s>>>(mq, mk, mv, a, hp);
   return cudaGetLastError();
 }
 
 template <int DK, typename Tout>
 cudaError_t launch_dk(const RetentionCall& c, const HeadParams& hp, cudaStream_t s) {
-  if (c.chunk == 64) return launch_cfg<DK, 64, Tout>(c, hp, s);
-  return launch_cfg<DK, 128, Tout>(c, hp, s);
+  if (force_serial_kernel()) {
+    if (c.chunk == 64) return launch_serial<DK, 64, Tout>(c, hp, s);
+    return launch_serial<DK, 128, Tout>(c, hp, s);
+  }
+  if (pipe_tile_rows(DK, c.chunk) == 64) return launch_pipe<DK, 64, Tout>(c, hp, s);
+  if constexpr (DK != 256) return launch_pipe<DK, 128, Tout>(c, hp, s);
+  return cudaErrorInvalidValue;
 }
 
 template <typename Tout>
@@ -1090,7 +1311,8 @@ bool tc_chunkwise_supported(const RetentionCall& c) {
   if (c.flags & RETNET_F_NORM_R) return false;
   if (d.d_k != 64 && d.d_k != 128 && d.d_k != 256) return false;
   if (d.d_v % kDVS != 0) return false;
-  if (c.chunk != 64 && c.chunk != 128) return false;
+  if (c.chunk != 64 && c.chunk != 128 && c.chunk != 256 && c.chunk != 512) return false;
+  if (force_serial_kernel() && c.chunk > 128) return false;
   if (d.seqlen < 1 || d.seqlen > (1LL << 30) || d.heads > 65535 || d.batch > 65535) return false;
   if (!aligned16(c.q) || !aligned16(c.k) || !aligned16(c.v) || !aligned16(c.o)) return false;
   if ((c.state_in && !aligned16(c.state_in)) || (c.state_out && !aligned16(c.state_out))) return false;
@@ -1106,10 +1328,12 @@ bool tc_chunkwise_supported(const RetentionCall& c) {
 
 bool tc_driver_ready() { return encode_fn() != nullptr; }
 
-// Host-side part of the scaled-operand condition: every head keeps gamma^B >= 2^-12.
+// Host-side part of the scaled-operand condition: every head keeps gamma^T >= 2^-12, where T
+// is the scaling span (the unit rows of the pipelined kernel, the whole chunk for the serial one).
 bool tc_chunkwise_heads_ok(const RetentionCall& c, const HeadParams& hp) {
+  const double span = force_serial_kernel() ? static_cast<double>(c.chunk) : pipe_tile_rows(c.dims.d_k, c.chunk);
   for (int64_t h = 0; h < c.dims.heads; ++h)
-    if (static_cast<double>(hp.log2g[h]) * static_cast<double>(c.chunk) < -12.0) return false;
+    if (static_cast<double>(hp.log2g[h]) * span < -12.0) return false;
   return true;
 }
 

@@ -150,6 +150,9 @@ def test_chunkwise_kernel_choice(lib):
     assert rn.retnet_chunkwise_kernel((1, 64, 8, 96), 128, rn.BF16, f, 64, g8) == 0      # d_k 96
     assert rn.retnet_chunkwise_kernel((1, 64, 8, 128), 96, rn.BF16, f, 64, g8) == 0      # d_v 96
     assert rn.retnet_chunkwise_kernel((1, 64, 8, 128), 128, rn.BF16, f, 32, g8) == 0     # chunk 32
+    assert rn.retnet_chunkwise_kernel((4, 4096, 8, 256), 256, rn.BF16, f, 256, g8) == 1  # chunk 256
+    assert rn.retnet_chunkwise_kernel((2, 8192, 8, 256), 512, rn.BF16, f, 512, g8) == 1  # chunk 512
+    assert rn.retnet_chunkwise_kernel((1, 64, 8, 128), 128, rn.BF16, f, 384, g8) == 0    # chunk 384
     # gamma^B < 2^-12 for some head: the scaled tensor-core form does not apply
     assert rn.retnet_chunkwise_kernel((1, 64, 2, 128), 128, rn.BF16, f, 128, np.array([0.9, 0.99], np.float32)) == 0
     assert rn.retnet_chunkwise_kernel((1, 64, 2, 128), 128, rn.BF16, f, 0, g8) == -4
