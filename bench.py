@@ -225,6 +225,69 @@ def bench_decode(rn, device, stream, steps, warmup, peaks):
                          "peak_source": peaks["source"]}}
 
 
+def bench_long(rn, device, stream, steps, peaks):
+    """Long-sequence chunkwise forward (chunks 128 and 512): TFLOP/s against the bf16 peak."""
+    import torch
+
+    import synth_inputs as si
+    c = LONG
+    b, L, h, dk, dv = c["batch"], c["seqlen"], c["heads"], c["d_k"], c["d_v"]
+    q, k, v = si.qkv(b, L, h, dk, dv, 3, "bf16")
+    q, k, v = q.to(device), k.to(device), v.to(device)
+    o = torch.empty(b, L, h, dv, dtype=torch.bfloat16, device=device)
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+    out = {"workload": c["workload"]}
+    for B in (128, 512):
+        path = rn.retnet_chunkwise_kernel((b, L, h, dk), dv, rn.BF16, FLAGS, B, g)
+
+        def step(i):
+            rn.retnet_retention_chunkwise(q, k, v, o, g, th, 0, FLAGS, B, stream=stream)
+
+        for i in range(2):
+            step(i)
+        torch.cuda.synchronize()
+        secs = time_steps(step, steps, stream) / steps
+        flops = b * L * h * flops_per_token_head(dk, dv, B)
+        byt = b * L * h * bytes_per_token_head(dk, dv)
+        out[f"chunk{B}"] = {"us_per_step": secs * 1e6, "tokens_per_s": b * L / secs, "tflops": flops / secs / 1e12,
+                            "frac_bf16_peak": flops / secs / 1e12 / peaks["bf16"], "gbs": byt / secs / 1e9,
+                            "frac_hbm": byt / secs / 1e9 / peaks["hbm"],
+                            "kernel": "tcgen05" if path == 1 else "fp32 CUDA cores", "gpu_launches": steps}
+    return out
+
+
+def bench_msr(rn, device, stream, steps, peaks):
+    """MSR forward: chunkwise retention (chunk 256, bf16 out) then GroupNorm + swish gate."""
+    import torch
+
+    import synth_inputs as si
+    c = MSR
+    b, L, h, dk, dv, B = c["batch"], c["seqlen"], c["heads"], c["d_k"], c["d_v"], c["chunk"]
+    q, k, v = si.qkv(b, L, h, dk, dv, 5, "bf16")
+    q, k, v = q.to(device), k.to(device), v.to(device)
+    gt = si.gate(b, L, h, dv, 5, "bf16").to(device)
+    y = torch.empty(b, L, h, dv, dtype=torch.bfloat16, device=device)
+    out = torch.empty(b, L, h * dv, dtype=torch.bfloat16, device=device)
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+    path = rn.retnet_chunkwise_kernel((b, L, h, dk), dv, rn.BF16, FLAGS, B, g)
+
+    def step(i):
+        rn.retnet_retention_chunkwise(q, k, v, y, g, th, 0, FLAGS, B, stream=stream)
+        rn.retnet_msr_epilogue(y.view(b, L, h * dv), gt, out, h, 1e-5, stream)
+
+    for i in range(2):
+        step(i)
+    torch.cuda.synchronize()
+    secs = time_steps(step, steps, stream) / steps
+    flops = b * L * h * flops_per_token_head(dk, dv, B)
+    byt = b * L * h * (bytes_per_token_head(dk, dv) + 2 * dv * 2 + 2 * dv)  # + y re-read, g, out
+    return {"workload": c["workload"], "us_per_step": secs * 1e6, "tokens_per_s": b * L / secs,
+            "tflops": flops / secs / 1e12, "frac_bf16_peak": flops / secs / 1e12 / peaks["bf16"],
+            "gbs": byt / secs / 1e9, "frac_hbm": byt / secs / 1e9 / peaks["hbm"],
+            "kernel": "tcgen05 + epilogue" if path == 1 else "fp32 CUDA cores + epilogue",
+            "gpu_launches": 2 * steps}
+
+
 def oracle_sample(cfg, budget_s):
     """Size a bounded sample of the workload for the fp64 oracle: whole batch rows (all heads)."""
     import oracle
@@ -358,6 +421,10 @@ def main_ours(args):
                        "d2h_bytes_per_step": ho.numel() * ho.element_size(), "steps": e2e_steps}
     if world == 1 and "decode" in args.sections:
         line["decode"] = bench_decode(rn, device, stream, args.decode_steps, 3, peaks)
+    if world == 1 and "long" in args.sections:
+        line["long"] = bench_long(rn, device, stream, 10, peaks)
+    if world == 1 and "msr" in args.sections:
+        line["msr"] = bench_msr(rn, device, stream, 10, peaks)
     clocks.stop()
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, args.cpu_seconds)
@@ -398,8 +465,8 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--sections", default="e2e,decode",
-                    help="comma list of extra legs to run beside the timed step: e2e, decode")
+    ap.add_argument("--sections", default="e2e,decode,long,msr",
+                    help="comma list of extra legs to run beside the timed step: e2e, decode, long, msr")
     ap.add_argument("--decode-steps", type=int, default=200)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

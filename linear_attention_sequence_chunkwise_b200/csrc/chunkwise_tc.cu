@@ -419,15 +419,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (dk >= 0) put_r16(dk, rv);
+        uint32_t w64[4][16];
 #pragma unroll
-        for (int c16 = 0; c16 < kDVS / 16; ++c16) {
-          uint32_t u[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) u[e] = __float_as_uint(g0 * rv[16 * c16 + e]);
-          tmem_st16(tmem + C::COL_R + blk * kDVS + 16 * c16 + lane_off, u);
-        }
+        for (int e = 0; e < kDVS; ++e) w64[e / 16][e % 16] = __float_as_uint(g0 * rv[e]);
+        tmem_st_wait(tmem + C::COL_R + blk * kDVS + lane_off, w64);
       }
-      tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar(B_R_READY));
@@ -447,9 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int half = 0; half < T / 64; ++half) {
           uint32_t u[4][16];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) tmem_ld16(tmem + C::COL_S + half * 64 + 16 * q + lane_off, u[q]);
-          tmem_wait_ld();
+          tmem_ld_wait(tmem + C::COL_S + half * 64 + lane_off, u);
           if (my_row >= 0) {
 #pragma unroll
             for (int c8 = 0; c8 < 8; ++c8) {
@@ -482,21 +476,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int blk = 0; blk < C::RBLK; ++blk) {
           const int dk = state_row(blk);
           uint32_t u[4][16];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) tmem_ld16(tmem + C::COL_R + blk * kDVS + 16 * q + lane_off, u[q]);
-          tmem_wait_ld();
+          tmem_ld_wait(tmem + C::COL_R + blk * kDVS + lane_off, u);
           float rv[kDVS];
 #pragma unroll
           for (int c = 0; c < kDVS; ++c) rv[c] = __uint_as_float(u[c / 16][c % 16]);
           if (!last) {
             if (dk >= 0) put_r16(dk, rv);
+            uint32_t w64[4][16];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint32_t w16[16];
-#pragma unroll
-              for (int e = 0; e < 16; ++e) w16[e] = __float_as_uint(gn * rv[16 * q + e]);
-              tmem_st16(tmem + C::COL_R + blk * kDVS + 16 * q + lane_off, w16);
-            }
+            for (int e = 0; e < kDVS; ++e) w64[e / 16][e % 16] = __float_as_uint(gn * rv[e]);
+            tmem_st_wait(tmem + C::COL_R + blk * kDVS + lane_off, w64);
           } else if (dk >= 0 && sbase_g_out) {
 #pragma unroll
             for (int c4 = 0; c4 < kDVS / 4; ++c4)
@@ -504,7 +493,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                   make_float4(rv[4 * c4], rv[4 * c4 + 1], rv[4 * c4 + 2], rv[4 * c4 + 3]);
           }
         }
-        tmem_wait_st();
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(bar(B_R_READY));
@@ -516,9 +504,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       {
         uint32_t u[4][16];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) tmem_ld16(tmem + C::COL_O + 16 * q + lane_off, u[q]);
-        tmem_wait_ld();
+        tmem_ld_wait(tmem + C::COL_O + lane_off, u);
         tc_fence_before();
         mbar_arrive(bar(B_O_FREE));
         if (my_row >= 0 && my_row < bl) {
@@ -576,42 +562,54 @@ __global__ void __launch_bounds__(kThreads, 1)
 //   1 warp TMA, 1 warp MMA issuer (one unit ahead: S and dR of unit k+1 before X/PV of unit k).
 // ============================================================================================
 
-template <int DK, int T>
+template <int DK, int T, int DVS>
 struct Cfg3 {
-  static constexpr int RBLK = DK > 128 ? 2 : 1;
+  static constexpr int NDV = DVS / 64;              // 64-column boxes of the d_v slice
+  static constexpr int RBLK = DK > 128 ? 2 : 1;     // 128-row blocks of the state increment
   static constexpr int MR = DK >= 128 ? 128 : 64;
-  static constexpr int WARPS_S = 4 * RBLK;
+  static constexpr int WARPS_S = 4 * RBLK * NDV;    // one thread per (d_k row, 64 columns)
   static constexpr int WARP_S0 = 4;
   static constexpr int WARP_CONV0 = WARP_S0 + WARPS_S;
-  static constexpr int WARP_TMA = WARP_CONV0 + 4;
+  static constexpr int CONV_WARPS = 4;
+  static constexpr int NCONV = 32 * CONV_WARPS;
+  static constexpr int WARP_TMA = WARP_CONV0 + CONV_WARPS;
   static constexpr int WARP_MMA = WARP_TMA + 1;
   static constexpr int THREADS = 32 * (WARP_MMA + 1);
   static constexpr int QBYTES = T * DK * 2;
-  static constexpr int VBYTES = T * kDVS * 2;
+  static constexpr int VBYTES = T * DVS * 2;
   static constexpr int STAGE = 2 * QBYTES + VBYTES;
   static constexpr int PBYTES = T * T * 2;
-  static constexpr int RBYTES = DK * kDVS * 2;
-  // TMEM: O[2], X[2] (64 columns each), S[SBUF] (T columns), dR[DRBUF] (RBLK x 64 columns).
-  static constexpr int SBUF = (4 * kDVS + 2 * T + RBLK * kDVS <= 512) ? 2 : 1;
-  static constexpr int DRBUF = (4 * kDVS + SBUF * T + 2 * RBLK * kDVS <= 512) ? 2 : 1;
+  static constexpr int RBYTES = DK * DVS * 2;
+  // TMEM: O[2] (DVS columns each), X[XBUF] (cross accumulators; none when the slice is 128
+  // wide, which then runs one sub-block per chunk only), S[SBUF] (T columns), dR[DRBUF]
+  // (RBLK x DVS columns).
+  static constexpr int XBUF = DVS == 64 ? 2 : 0;
+  static constexpr int SBUF = ((2 + XBUF) * DVS + 2 * T + RBLK * DVS <= 512) ? 2 : 1;
+  static constexpr int DRBUF = ((2 + XBUF) * DVS + SBUF * T + 2 * RBLK * DVS <= 512) ? 2 : 1;
   static constexpr int COL_O = 0;
-  static constexpr int COL_X = 2 * kDVS;
-  static constexpr int COL_S = 4 * kDVS;
-  static constexpr int COL_DR = 4 * kDVS + SBUF * T;
-  static constexpr int USED = COL_DR + DRBUF * RBLK * kDVS;
+  static constexpr int COL_X = 2 * DVS;
+  static constexpr int COL_S = (2 + XBUF) * DVS;
+  static constexpr int COL_DR = COL_S + SBUF * T;
+  static constexpr int USED = COL_DR + DRBUF * RBLK * DVS;
   static constexpr int TMEM_COLS = USED <= 128 ? 128 : (USED <= 256 ? 256 : 512);
-  // shared memory: stages, P[PBUF], R16[RBUF], rotation tables (Q and K, double-buffered), barriers
+  // shared memory: stages, P[PBUF], R16[RBUF], rotation tables (Q and K, double-buffered),
+  // barriers.  A second fp16 state buffer is kept only while three stages still fit.
   static constexpr int NBARS = 3 * 4 + 2 * 10 + 2;
   static constexpr int TABBYTES = 2 * 2 * (DK / 2) * 8;
   static constexpr int BUDGET = 227 * 1024 - 1024;
   static constexpr int TAIL = TABBYTES + NBARS * 8 + 16;
   static constexpr int PBUF = (2 * STAGE + 2 * PBYTES + RBYTES + TAIL <= BUDGET) ? 2 : 1;
-  static constexpr int RBUF = (2 * STAGE + PBUF * PBYTES + 2 * RBYTES + TAIL <= BUDGET) ? 2 : 1;
+  static constexpr int NS_R2 = (BUDGET - (PBUF * PBYTES + 2 * RBYTES + TAIL)) / STAGE;
+  static constexpr int NS_R1 = (BUDGET - (PBUF * PBYTES + RBYTES + TAIL)) / STAGE;
+  static constexpr int RBUF = (NS_R2 >= 3 || NS_R1 < 3) && NS_R2 >= 2 ? 2 : 1;
   static constexpr int FIXED = PBUF * PBYTES + RBUF * RBYTES + TAIL;
   static constexpr int NS_FIT = (BUDGET - FIXED) / STAGE;
   static constexpr int NS = NS_FIT > 4 ? 4 : NS_FIT;
   static constexpr int SMEM = NS * STAGE + FIXED + 1024;
-  static constexpr bool FITS = NS >= 2 && USED <= 512;
+  static constexpr bool FITS = NS >= 2 && USED <= 512 && (DVS == 64 || DVS == 128);
+  // Columns per TMEM load batch: 18 warps leave 96 registers a thread (five warps share one
+  // sub-partition's register file), too few to hold 64 loaded columns next to the state.
+  static constexpr int LDW = THREADS > 512 ? 32 : 64;
 };
 
 // Barrier slots of the pipelined kernel ([2] = indexed by buffer).
@@ -688,13 +686,21 @@ struct UnitIter {
 
 // Converter role of the pipelined kernel: like Converter, with the sub-block-local row scales
 // and separate rotation bases for the unit's query rows (block u) and key rows (block w).
-template <int DK, int T>
+// NC threads; thread lt owns 16-byte column slot cs = lt % CS and rows r0 + RS k.  The row
+// scale is carried inside the rotation factor: F_q(r) = gamma^(r+1) e^{i (p_r) theta_j} and
+// F_k(c) = gamma^(T-1-c) e^{i (p_c) theta_j}, each advanced by one complex product per row step.
+template <int DK, int T, int NC, int NDV>
 struct UnitConverter {
-  static constexpr int CS = DK / 8;    // 16-byte column slots across the DK/64 boxes
-  static constexpr int RS = 128 / CS;  // row step of one thread
-  static constexpr int NR = T / RS;    // rows per thread
-  float2 W[4], Z[4];                   // e^{i r0 theta_j}, e^{i RS theta_j} for the thread's pairs
-  float2 cur, stepT, stepB;            // table producer (lt < DK/2): chunk base, e^{iT theta}, e^{iB theta}
+  static constexpr int CS = DK / 8;   // 16-byte column slots across the DK/64 boxes
+  static constexpr int RS = NC / CS;  // row step of one thread
+  static constexpr int NR = T / RS;   // rows per thread
+  static constexpr int G = NR < 4 ? NR : 4;  // rows per load batch
+  static constexpr int VR = NC / 8;   // V rows per pass (8 slots of one 64-column box)
+  static constexpr int VP = T / VR;   // V passes
+  static constexpr int VG = VP < 4 ? VP : 4;
+  static_assert(NR >= 1 && NR % G == 0 && VP >= 1 && VP % VG == 0, "converter tiling");
+  float2 W[4], Z[4];                  // e^{i r0 theta_j}, e^{i RS theta_j} for the thread's pairs
+  float2 cur, stepT, stepB;           // table producer (lt < DK/2): chunk base, e^{iT theta}, e^{iB theta}
   int cs, r0, lt, cur_chunk;
 
   __device__ void init(int lt_, int nb, const HeadParams& hp) {
@@ -747,67 +753,68 @@ struct UnitConverter {
     const uint32_t box = (cs / 8) * T * 128;
     const uint32_t chunk = cs % 8;
     const float xstep = decay_pow(log2g, RS), zstep = exp2f(-static_cast<float>(RS) * log2g);
-    float xi = decay_pow(log2g, r0 + 1);
-    float zeta = decay_pow(log2g, T - 1 - r0);
-    float2 Fq[4], Fk[4];
+    const float xi0 = decay_pow(log2g, r0 + 1), zeta0 = decay_pow(log2g, T - 1 - r0);
+    float2 Fq[4], Fk[4], Zq[4], Zk[4];
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj) {
-      Fq[jj] = xpos ? cmul(bq[4 * cs + jj], W[jj]) : make_float2(1.f, 0.f);
-      Fk[jj] = xpos ? cmul(bk[4 * cs + jj], W[jj]) : make_float2(1.f, 0.f);
+      const float2 fq = xpos ? cmul(bq[4 * cs + jj], W[jj]) : make_float2(1.f, 0.f);
+      const float2 fk = xpos ? cmul(bk[4 * cs + jj], W[jj]) : make_float2(1.f, 0.f);
+      Fq[jj] = make_float2(xi0 * fq.x, xi0 * fq.y);
+      Fk[jj] = make_float2(zeta0 * fk.x, zeta0 * fk.y);
+      Zq[jj] = make_float2(xstep * Z[jj].x, xstep * Z[jj].y);
+      Zk[jj] = make_float2(zstep * Z[jj].x, zstep * Z[jj].y);
     }
-    static_assert(NR % 4 == 0, "rows per thread must be a multiple of 4");
 #pragma unroll 1
-    for (int kg = 0; kg < NR; kg += 4) {
-      uint32_t q4[4][4], k4[4][4];
+    for (int kg = 0; kg < NR; kg += G) {
+      uint32_t q4[G][4], k4[G][4];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
+      for (int k = 0; k < G; ++k) {
         const uint32_t off = box + sw128(r0 + RS * (kg + k), chunk);
         ld_shared_v4(sq + off, q4[k][0], q4[k][1], q4[k][2], q4[k][3]);
         ld_shared_v4(sk + off, k4[k][0], k4[k][1], k4[k][2], k4[k][3]);
       }
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
+      for (int k = 0; k < G; ++k) {
         uint32_t qo[4], ko[4];
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
           const float q0 = __uint_as_float(q4[k][jj] << 16), q1 = __uint_as_float(q4[k][jj] & 0xffff0000u);
           const float k0 = __uint_as_float(k4[k][jj] << 16), k1 = __uint_as_float(k4[k][jj] & 0xffff0000u);
-          const float cq = Fq[jj].x, sq_ = Fq[jj].y, ck = Fk[jj].x, sk_ = Fk[jj].y;
-          qo[jj] = pack_f16x2(xi * (q0 * cq - q1 * sq_), xi * (q0 * sq_ + q1 * cq));
-          ko[jj] = pack_f16x2(zeta * (k0 * ck - k1 * sk_), zeta * (k0 * sk_ + k1 * ck));
-          Fq[jj] = cmul(Fq[jj], Z[jj]);
-          Fk[jj] = cmul(Fk[jj], Z[jj]);
+          qo[jj] = pack_f16x2(q0 * Fq[jj].x - q1 * Fq[jj].y, q0 * Fq[jj].y + q1 * Fq[jj].x);
+          ko[jj] = pack_f16x2(k0 * Fk[jj].x - k1 * Fk[jj].y, k0 * Fk[jj].y + k1 * Fk[jj].x);
+          Fq[jj] = cmul(Fq[jj], Zq[jj]);
+          Fk[jj] = cmul(Fk[jj], Zk[jj]);
         }
         const uint32_t off = box + sw128(r0 + RS * (kg + k), chunk);
         st_shared_v4(sq + off, qo[0], qo[1], qo[2], qo[3]);
         st_shared_v4(sk + off, ko[0], ko[1], ko[2], ko[3]);
-        xi *= xstep;
-        zeta *= zstep;
       }
     }
+    // V: each 64-column box, slot lt % 8, rows lt / 8 + VR k.
 #pragma unroll 1
-    for (int kg = 0; kg < T / 16; kg += 4) {
-      uint32_t v4[4][4];
+    for (int kg = 0; kg < NDV * VP; kg += VG) {
+      const uint32_t vb = sv + (kg / VP) * T * 128;
+      uint32_t v4[VG][4];
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        ld_shared_v4(sv + sw128(lt / 8 + 16 * (kg + k), lt % 8), v4[k][0], v4[k][1], v4[k][2], v4[k][3]);
+      for (int k = 0; k < VG; ++k)
+        ld_shared_v4(vb + sw128(lt / 8 + VR * (kg % VP + k), lt % 8), v4[k][0], v4[k][1], v4[k][2], v4[k][3]);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
+      for (int k = 0; k < VG; ++k) {
         uint32_t vo[4];
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj)
           vo[jj] = pack_f16x2(__uint_as_float(v4[k][jj] << 16), __uint_as_float(v4[k][jj] & 0xffff0000u));
-        st_shared_v4(sv + sw128(lt / 8 + 16 * (kg + k), lt % 8), vo[0], vo[1], vo[2], vo[3]);
+        st_shared_v4(vb + sw128(lt / 8 + VR * (kg % VP + k), lt % 8), vo[0], vo[1], vo[2], vo[3]);
       }
     }
   }
 };
 
-template <int DK, int T, typename Tout>
-__global__ void __launch_bounds__(Cfg3<DK, T>::THREADS, 1)
+template <int DK, int T, int DVS, typename Tout>
+__global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
     tc_chunkwise_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v, TcArgs a, HeadParams hp) {
-  using C = Cfg3<DK, T>;
+  using C = Cfg3<DK, T, DVS>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_addr(smem_raw);
   const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
@@ -835,7 +842,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T>::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < 4; ++s) {
       mbar_init(bar(Q_TMA_FULL + s), 1);
-      mbar_init(bar(Q_CONV_FULL + s), 128);
+      mbar_init(bar(Q_CONV_FULL + s), C::NCONV);
       mbar_init(bar(Q_STAGE_EMPTY + s), 1);
     }
     for (int k = 0; k < 2; ++k) {
@@ -849,7 +856,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T>::THREADS, 1)
       mbar_init(bar(Q_R16_FREE + k), 1);
       mbar_init(bar(Q_O_FULL + k), 1);
       mbar_init(bar(Q_O_FREE + k), 128);
-      mbar_init(bar(Q_TAB + k), 128);
+      mbar_init(bar(Q_TAB + k), C::NCONV);
     }
     mbar_init(bar(Q_DRAIN), 1);
     fence_mbar_init();
@@ -883,7 +890,9 @@ __global__ void __launch_bounds__(Cfg3<DK, T>::THREADS, 1)
           tma_load_4d(sQ(s) + bx * T * 128, &tm_q, bar(Q_TMA_FULL + s), bx * 64, h, tq, b);
           tma_load_4d(sK(s) + bx * T * 128, &tm_k, bar(Q_TMA_FULL + s), bx * 64, h, tk, b);
         }
-        tma_load_4d(sV(s), &tm_v, bar(Q_TMA_FULL + s), dvb * kDVS, h, tk, b);
+#pragma unroll
+        for (int bx = 0; bx < C::NDV; ++bx)
+          tma_load_4d(sV(s) + bx * T * 128, &tm_v, bar(Q_TMA_FULL + s), dvb * DVS + 64 * bx, h, tk, b);
         issued[s]++;
       }
       // Every load this thread issued must have landed before the CTA may exit.
@@ -894,8 +903,8 @@ __global__ void __launch_bounds__(Cfg3<DK, T>::THREADS, 1)
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t ID_S = idesc_f16_f32(T, T, 0, 0);
-      constexpr uint32_t ID_X = idesc_f16_f32(T, kDVS, 0, 1);
-      constexpr uint32_t ID_R = idesc_f16_f32(C::MR, kDVS, 1, 1);
+      constexpr uint32_t ID_X = idesc_f16_f32(T, DVS, 0, 1);
+      constexpr uint32_t ID_R = idesc_f16_f32(C::MR, DVS, 1, 1);
       // Descriptors are built once per operand tile and advanced by constants (the start
       // address field never carries: every operand lies below 256 KB of shared memory).
       auto kstep = [](int kk) -> uint64_t { return static_cast<uint64_t>(((kk / 4) * T * 128 + (kk % 4) * 32) >> 4); };
@@ -914,13 +923,13 @@ __global__ void __launch_bounds__(Cfg3<DK, T>::THREADS, 1)
         for (int kk = 0; kk < DK / 16; ++kk) mma_f16_ss(tS, dq + kstep(kk), dk + kstep(kk), ID_S, kk > 0);
         mma_commit(bar(Q_S_FULL + (f.k % C::SBUF)));
         if (f.last_row()) {
-          const uint32_t tD = tmem + C::COL_DR + (f.dr % C::DRBUF) * C::RBLK * kDVS;
+          const uint32_t tD = tmem + C::COL_DR + (f.dr % C::DRBUF) * C::RBLK * DVS;
           const uint64_t dkm = sdesc_sw128(sK(s), T * 128, 1024), dv = sdesc_sw128(sV(s), T * 128, 1024);
 #pragma unroll
           for (int blk = 0; blk < C::RBLK; ++blk)
 #pragma unroll
             for (int ks = 0; ks < T / 16; ++ks)
-              mma_f16_ss(tD + blk * kDVS, dkm + static_cast<uint64_t>((blk * 2 * T * 128 + ks * 2048) >> 4),
+              mma_f16_ss(tD + blk * DVS, dkm + static_cast<uint64_t>((blk * 2 * T * 128 + ks * 2048) >> 4),
                          dv + static_cast<uint64_t>((ks * 2048) >> 4), ID_R, ks > 0);
           mma_commit(bar(Q_DR_FULL + (f.dr % C::DRBUF)));
         }
@@ -929,12 +938,12 @@ __global__ void __launch_bounds__(Cfg3<DK, T>::THREADS, 1)
       // Cross term of the row block (first unit only) and P V into O.
       auto back = [&](const UnitIter<T>& q) -> bool {
         const int s = q.k % C::NS;
-        const uint32_t tO = tmem + C::COL_O + (q.rb & 1) * kDVS;
+        const uint32_t tO = tmem + C::COL_O + (q.rb & 1) * DVS;
         if (q.w == 0) {
           if (!mbar_wait(bar(Q_R16_FULL + (q.i % C::RBUF)), (q.i / C::RBUF) & 1)) return false;
           if (q.rb >= 2 && !mbar_wait(bar(Q_O_FREE + (q.rb & 1)), ((q.rb - 2) >> 1) & 1)) return false;
           tc_fence_after();
-          const uint32_t tX = (nb > 1) ? tmem + C::COL_X + (q.rb & 1) * kDVS : tO;
+          const uint32_t tX = (C::XBUF > 0 && nb > 1) ? tmem + C::COL_X + (q.rb & 1) * DVS : tO;
           const uint64_t dq = sdesc_sw128(sQ(s), 16, 1024), dr = sdesc_sw128(sR(q.i), DK * 128, 1024);
 #pragma unroll
           for (int kk = 0; kk < DK / 16; ++kk)
@@ -971,7 +980,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T>::THREADS, 1)
     }
   } else if (warp >= C::WARP_CONV0) {
     // ------------------------------------------------------------------ converters
-    UnitConverter<DK, T> cv;
+    UnitConverter<DK, T, C::NCONV, C::NDV> cv;
     cv.init(threadIdx.x - 32 * C::WARP_CONV0, nb, hp);
     const bool xpos = (a.flags & RETNET_F_XPOS) != 0;
     bool ok = true;
@@ -981,7 +990,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T>::THREADS, 1)
       float2* tq = tab + (it.k & 1) * DK;
       float2* tk = tq + DK / 2;
       if (xpos) cv.put_bases(tq, tk, it.i, it.u, it.w, it.t0(), a.pos0, hp);
-      // Table buffer (k & 1) is complete once all 128 converters arrived; a thread that
+      // Table buffer (k & 1) is complete once all converters arrived; a thread that
       // rewrites it two units later has passed this wait, so every read of it is done.
       mbar_arrive(bar(Q_TAB + (it.k & 1)));
       ok = mbar_wait(bar(Q_TAB + (it.k & 1)), (it.k >> 1) & 1);
@@ -993,25 +1002,30 @@ __global__ void __launch_bounds__(Cfg3<DK, T>::THREADS, 1)
     }
   } else if (warp >= C::WARP_S0) {
     // ------------------------------------------------------------------ state group
+    // Thread = (d_k row, 64-column box ch of the slice); warp % 4 selects its TMEM lane quarter.
+    constexpr int RC = 64;
     const int ws = warp - C::WARP_S0;
-    const int blk = ws / 4;
+    const int blk = (ws / 4) % C::RBLK;
+    const int ch = ws / (4 * C::RBLK);
     const uint32_t lane_off = static_cast<uint32_t>(32 * (warp % 4)) << 16;
     const int dk = (DK == 64) ? (lane < 16 ? 16 * (warp % 4) + lane : -1) : blk * 128 + 32 * (warp % 4) + lane;
     const int64_t bh = static_cast<int64_t>(b) * a.heads + h;
     const size_t srow = static_cast<size_t>(a.dv);
-    float R[kDVS];
+    const int col0 = dvb * DVS + ch * RC;
+    float R[RC];
 #pragma unroll
-    for (int c = 0; c < kDVS; ++c) R[c] = 0.f;
+    for (int c = 0; c < RC; ++c) R[c] = 0.f;
     if (dk >= 0 && a.state_in) {
-      const float* src = a.state_in + static_cast<size_t>(bh) * DK * a.dv + dvb * kDVS + dk * srow;
+      const float* src = a.state_in + static_cast<size_t>(bh) * DK * a.dv + col0 + dk * srow;
 #pragma unroll
-      for (int c4 = 0; c4 < kDVS / 4; ++c4) {
+      for (int c4 = 0; c4 < RC / 4; ++c4) {
         const float4 x = *reinterpret_cast<const float4*>(src + 4 * c4);
         R[4 * c4] = x.x; R[4 * c4 + 1] = x.y; R[4 * c4 + 2] = x.z; R[4 * c4 + 3] = x.w;
       }
     }
     auto put_r16 = [&](uint32_t base) {
       if (dk < 0) return;
+      base += ch * DK * 128;
 #pragma unroll
       for (int c8 = 0; c8 < 8; ++c8)
         st_shared_v4(base + sw128(dk, c8), pack_f16x2(sd * R[8 * c8 + 0], sd * R[8 * c8 + 1]),
@@ -1029,21 +1043,25 @@ __global__ void __launch_bounds__(Cfg3<DK, T>::THREADS, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(Q_DR_FULL + (it.dr % C::DRBUF)), (it.dr / C::DRBUF) & 1));
       if (!ok) break;
       tc_fence_after();
-      uint32_t u[4][16];
-      const uint32_t tD = tmem + C::COL_DR + (it.dr % C::DRBUF) * C::RBLK * kDVS + blk * kDVS + lane_off;
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) tmem_ld16(tD + 16 * q4, u[q4]);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar(Q_DR_FREE + (it.dr % C::DRBUF)));
       // Horner form of R_i = gamma^b' R_{i-1} + sum_w gamma^(b'-(w+1)T) dR_w:
       //   w = 0: R = gamma^(b'-(nbw-1)T) R + hh dR_0;  w > 0: R = gamma^T R + hh dR_w,
       //   hh = gamma^(b' - nbw T) (1 for a full chunk).
       const float g = (it.w == 0) ? exp2f(static_cast<float>(it.bl - (it.nbw - 1) * T) * log2g)
                                   : decay_pow(log2g, T);
       const float hh = exp2f(static_cast<float>(it.bl - it.nbw * T) * log2g);
+      const uint32_t tD = tmem + C::COL_DR + (it.dr % C::DRBUF) * C::RBLK * DVS + blk * DVS + ch * RC + lane_off;
+      constexpr int SW = C::LDW / 2;  // columns per load next to the 64 state registers
 #pragma unroll
-      for (int c = 0; c < kDVS; ++c) R[c] = fmaf(g, R[c], hh * __uint_as_float(u[c / 16][c % 16]));
+      for (int grp = 0; grp < RC / SW; ++grp) {
+        uint32_t u[SW / 16][16];
+        tmem_ld_wait(tD + SW * grp, u);
+        if (grp == RC / SW - 1) {
+          tc_fence_before();
+          mbar_arrive(bar(Q_DR_FREE + (it.dr % C::DRBUF)));
+        }
+#pragma unroll
+        for (int c = 0; c < SW; ++c) R[SW * grp + c] = fmaf(g, R[SW * grp + c], hh * __uint_as_float(u[c / 16][c % 16]));
+      }
       if (it.w + 1 < it.nbw) continue;  // chunk not finished
       const int nxt = it.i + 1;
       if (nxt * nb * T < a.L) {
@@ -1056,9 +1074,9 @@ __global__ void __launch_bounds__(Cfg3<DK, T>::THREADS, 1)
         fence_proxy_async_smem();
         mbar_arrive(bar(Q_R16_FULL + (nxt % C::RBUF)));
       } else if (dk >= 0 && a.state_out) {
-        float* dst = a.state_out + static_cast<size_t>(bh) * DK * a.dv + dvb * kDVS + dk * srow;
+        float* dst = a.state_out + static_cast<size_t>(bh) * DK * a.dv + col0 + dk * srow;
 #pragma unroll
-        for (int c4 = 0; c4 < kDVS / 4; ++c4)
+        for (int c4 = 0; c4 < RC / 4; ++c4)
           *reinterpret_cast<float4*>(dst + 4 * c4) = make_float4(R[4 * c4], R[4 * c4 + 1], R[4 * c4 + 2], R[4 * c4 + 3]);
       }
     }
@@ -1076,42 +1094,68 @@ __global__ void __launch_bounds__(Cfg3<DK, T>::THREADS, 1)
       const int t = i * nb * T + u * T + (my_row < 0 ? 0 : my_row);
       const float f = row_factor_f32(gam, sd, a.pos0 + t, a.flags) / sd;
       const float gx = (nb > 1) ? exp2f(static_cast<float>(u * T) * log2g) : 0.f;
-      Tout* dst = static_cast<Tout*>(a.o) + ((static_cast<int64_t>(b) * a.L + t) * a.heads + h) * a.dv + dvb * kDVS;
-      // 16 columns at a time: O (and X) from TMEM, o = (O + gamma^(uT) X) * s / c_p, 16-byte stores.
-#pragma unroll 1
-      for (int q = 0; q < 4; ++q) {
-        uint32_t uo[16], ux[16];
-        tmem_ld16(tmem + C::COL_O + (rb & 1) * kDVS + 16 * q + lane_off, uo);
-        if (nb > 1) tmem_ld16(tmem + C::COL_X + (rb & 1) * kDVS + 16 * q + lane_off, ux);
-        tmem_wait_ld();
-        if (q == 3) {
-          tc_fence_before();
-          mbar_arrive(bar(Q_O_FREE + (rb & 1)));
-        }
-        if (live) {
-          float ov[16];
+      Tout* dst = static_cast<Tout*>(a.o) + ((static_cast<int64_t>(b) * a.L + t) * a.heads + h) * a.dv + dvb * DVS;
+      // O (and X) from TMEM, o = (O + gamma^(uT) X) * s / c_p, 16-byte stores of 16 columns.
+      auto store16 = [&](int q, const float (&ov)[16]) {
+        if constexpr (sizeof(Tout) == 2) {
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            float x = __uint_as_float(uo[c]);
-            if (nb > 1) x = fmaf(gx, __uint_as_float(ux[c]), x);
-            ov[c] = f * x;
-          }
-          if constexpr (sizeof(Tout) == 2) {
+          for (int c8 = 0; c8 < 2; ++c8) {
+            uint32_t pk[4];
 #pragma unroll
-            for (int c8 = 0; c8 < 2; ++c8) {
-              uint32_t pk[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                __nv_bfloat162 v2 = __floats2bfloat162_rn(ov[8 * c8 + 2 * e], ov[8 * c8 + 2 * e + 1]);
-                pk[e] = *reinterpret_cast<uint32_t*>(&v2);
-              }
-              *reinterpret_cast<uint4*>(dst + 16 * q + 8 * c8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            for (int e = 0; e < 4; ++e) {
+              __nv_bfloat162 v2 = __floats2bfloat162_rn(ov[8 * c8 + 2 * e], ov[8 * c8 + 2 * e + 1]);
+              pk[e] = *reinterpret_cast<uint32_t*>(&v2);
             }
-          } else {
+            *reinterpret_cast<uint4*>(dst + 16 * q + 8 * c8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+        } else {
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4)
-              *reinterpret_cast<float4*>(dst + 16 * q + 4 * c4) =
-                  make_float4(ov[4 * c4], ov[4 * c4 + 1], ov[4 * c4 + 2], ov[4 * c4 + 3]);
+          for (int c4 = 0; c4 < 4; ++c4)
+            *reinterpret_cast<float4*>(dst + 16 * q + 4 * c4) =
+                make_float4(ov[4 * c4], ov[4 * c4 + 1], ov[4 * c4 + 2], ov[4 * c4 + 3]);
+        }
+      };
+      const uint32_t tO = tmem + C::COL_O + (rb & 1) * DVS + lane_off;
+      const uint32_t tX = tmem + C::COL_X + (rb & 1) * DVS + lane_off;
+      if (C::XBUF == 0 || nb == 1) {
+        // No cross accumulator: O alone, LDW columns per load.
+#pragma unroll
+        for (int grp = 0; grp < DVS / C::LDW; ++grp) {
+          uint32_t uo[C::LDW / 16][16];
+          tmem_ld_wait(tO + grp * C::LDW, uo);
+          if (grp == DVS / C::LDW - 1) {
+            tc_fence_before();
+            mbar_arrive(bar(Q_O_FREE + (rb & 1)));
+          }
+          if (live) {
+#pragma unroll
+            for (int e = 0; e < C::LDW / 16; ++e) {
+              float ov[16];
+#pragma unroll
+              for (int c = 0; c < 16; ++c) ov[c] = f * __uint_as_float(uo[e][c]);
+              store16(grp * (C::LDW / 16) + e, ov);
+            }
+          }
+        }
+      } else {
+        // O and X, LDW / 2 columns of each per load.
+        constexpr int HW = C::LDW / 2;
+#pragma unroll 1
+        for (int grp = 0; grp < DVS / HW; ++grp) {
+          uint32_t uo[HW / 16][16], ux[HW / 16][16];
+          tmem_ld_wait(tO + grp * HW, uo, tX + grp * HW, ux);
+          if (grp == DVS / HW - 1) {
+            tc_fence_before();
+            mbar_arrive(bar(Q_O_FREE + (rb & 1)));
+          }
+          if (live) {
+#pragma unroll
+            for (int e = 0; e < HW / 16; ++e) {
+              float ov[16];
+#pragma unroll
+              for (int c = 0; c < 16; ++c) ov[c] = f * fmaf(gx, __uint_as_float(ux[e][c]), __uint_as_float(uo[e][c]));
+              store16(grp * (HW / 16) + e, ov);
+            }
           }
         }
       }
@@ -1132,27 +1176,26 @@ __global__ void __launch_bounds__(Cfg3<DK, T>::THREADS, 1)
       const bool diag = (it.u == it.w);
       const uint32_t tS = tmem + C::COL_S + (k % C::SBUF) * T + lane_off;
 #pragma unroll
-      for (int half = 0; half < T / 64; ++half) {
-        uint32_t u16[4][16];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) tmem_ld16(tS + half * 64 + 16 * q, u16[q]);
-        tmem_wait_ld();
-        if (half == T / 64 - 1) {
+      for (int grp = 0; grp < T / C::LDW; ++grp) {
+        uint32_t u16[C::LDW / 16][16];
+        tmem_ld_wait(tS + grp * C::LDW, u16);
+        if (grp == T / C::LDW - 1) {
           tc_fence_before();
           mbar_arrive(bar(Q_S_FREE + (k % C::SBUF)));
         }
         if (my_row >= 0) {
 #pragma unroll
-          for (int c8 = 0; c8 < 8; ++c8) {
+          for (int c8 = 0; c8 < C::LDW / 8; ++c8) {
+            const int col = grp * C::LDW + 8 * c8;
             uint32_t pk[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const int c0 = half * 64 + 8 * c8 + 2 * e;
+              const int c0 = col + 2 * e;
               const float p0 = (!diag || c0 <= my_row) ? __uint_as_float(u16[c8 / 2][(8 * c8 + 2 * e) % 16]) * pf : 0.f;
               const float p1 = (!diag || c0 + 1 <= my_row) ? __uint_as_float(u16[c8 / 2][(8 * c8 + 2 * e + 1) % 16]) * pf : 0.f;
               pk[e] = pack_f16x2(p0, p1);
             }
-            st_shared_v4(sP(k) + half * T * 128 + sw128(my_row, c8), pk[0], pk[1], pk[2], pk[3]);
+            st_shared_v4(sP(k) + (col / 64) * T * 128 + sw128(my_row, (col % 64) / 8), pk[0], pk[1], pk[2], pk[3]);
           }
         }
       }
@@ -1223,6 +1266,17 @@ bool force_serial_kernel() {
 // Rows per unit of the pipelined kernel: 64 for d_k = 256 (shared memory), else min(B, 128).
 int pipe_tile_rows(int64_t d_k, int64_t chunk) { return d_k == 256 ? 64 : static_cast<int>(chunk < 128 ? chunk : 128); }
 
+// 128-column d_v slices (S and the Q/K conversion shared by twice the columns) need one
+// sub-block per chunk (no cross accumulator in tensor memory) and d_k <= 128.  They halve the
+// CTA count, so they are taken only when the wide grid still fills the GPU.
+bool pipe_wide_slice(const RetentionCall& c, int T) {
+  if (!(c.dims.d_k <= 128 && T == 64 && c.chunk == 64 && c.dims.d_v % 128 == 0)) return false;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return false;
+  return c.dims.batch * c.dims.heads * (c.dims.d_v / 128) >= sms;
+}
+
 TcArgs make_args(const RetentionCall& c, int n_chunks, int nb) {
   TcArgs a;
   a.o = c.o;
@@ -1245,23 +1299,24 @@ bool make_maps(const RetentionCall& c, int T, CUtensorMap* mq, CUtensorMap* mk, 
          make_map(mv, c.v, d.batch, d.seqlen, d.heads, d.d_v, T);
 }
 
-dim3 tc_grid(const Dims& d) {
-  return dim3(static_cast<unsigned>(d.d_v / kDVS), static_cast<unsigned>(d.heads), static_cast<unsigned>(d.batch));
+dim3 tc_grid(const Dims& d, int dvs) {
+  return dim3(static_cast<unsigned>(d.d_v / dvs), static_cast<unsigned>(d.heads), static_cast<unsigned>(d.batch));
 }
 
-// Pipelined kernel: units of T rows, nb = B / T per chunk.
-template <int DK, int T, typename Tout>
+// Pipelined kernel: units of T rows, nb = B / T per chunk, d_v slices of DVS columns.
+template <int DK, int T, int DVS, typename Tout>
 cudaError_t launch_pipe(const RetentionCall& c, const HeadParams& hp, cudaStream_t s) {
-  using Cf = Cfg3<DK, T>;
+  using Cf = Cfg3<DK, T, DVS>;
   static_assert(Cf::FITS, "pipelined kernel does not fit this tile");
   CUtensorMap mq, mk, mv;
   if (!make_maps(c, T, &mq, &mk, &mv)) return cudaErrorInvalidValue;
   const int nb = static_cast<int>(c.chunk / T);
   const TcArgs a = make_args(c, static_cast<int>((c.dims.seqlen + c.chunk - 1) / c.chunk), nb);
-  auto kern = tc_chunkwise_pipe_kernel<DK, T, Tout>;
+  if (Cf::XBUF == 0 && nb != 1) return cudaErrorInvalidValue;
+  auto kern = tc_chunkwise_pipe_kernel<DK, T, DVS, Tout>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<tc_grid(c.dims), Cf::THREADS, Cf::SMEM, s>>>(mq, mk, mv, a, hp);
+  kern<<<tc_grid(c.dims, DVS), Cf::THREADS, Cf::SMEM, s>>>(mq, mk, mv, a, hp);
   return cudaGetLastError();
 }
 
@@ -1275,7 +1330,7 @@ cudaError_t launch_serial(const RetentionCall& c, const HeadParams& hp, cudaStre
   auto kern = tc_chunkwise_kernel<DK, T, Tout>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<tc_grid(c.dims), kThreads, Cf::SMEM, s>>>(mq, mk, mv, a, hp);
+  kern<<<tc_grid(c.dims, kDVS), kThreads, Cf::SMEM, s>>>(mq, mk, mv, a, hp);
   return cudaGetLastError();
 }
 
@@ -1285,8 +1340,12 @@ cudaError_t launch_dk(const RetentionCall& c, const HeadParams& hp, cudaStream_t
     if (c.chunk == 64) return launch_serial<DK, 64, Tout>(c, hp, s);
     return launch_serial<DK, 128, Tout>(c, hp, s);
   }
-  if (pipe_tile_rows(DK, c.chunk) == 64) return launch_pipe<DK, 64, Tout>(c, hp, s);
-  if constexpr (DK != 256) return launch_pipe<DK, 128, Tout>(c, hp, s);
+  const int T = pipe_tile_rows(DK, c.chunk);
+  if constexpr (DK != 256) {
+    if (pipe_wide_slice(c, T)) return launch_pipe<DK, 64, 128, Tout>(c, hp, s);
+  }
+  if (T == 64) return launch_pipe<DK, 64, 64, Tout>(c, hp, s);
+  if constexpr (DK != 256) return launch_pipe<DK, 128, 64, Tout>(c, hp, s);
   return cudaErrorInvalidValue;
 }
 

@@ -140,27 +140,123 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t addr, uint32_t lbo, uin
 
 // ---- tcgen05: TMEM <-> registers --------------------------------------------------------------
 
-// 32 lanes x 32 bits, 16 consecutive columns: thread i of the warp reads lane (warp base + i).
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-      "%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
-        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-}
+// TMEM loads, 32 lanes x 32 bits: thread i of the warp reads lane (warp base + i), consecutive
+// columns into consecutive registers.  tcgen05.ld completes asynchronously, and an inline-asm
+// output is taken by the compiler as written when its statement ends; so every load here is
+// issued together with its tcgen05.wait::ld in ONE asm statement, which leaves the compiler no
+// point at which it could read, move or spill a destination register before the data lands.
 
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+// 16 columns.
+__device__ __forceinline__ void tmem_ld_wait(uint32_t taddr, uint32_t (&r)[1][16]) {
   asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-      "%15, %16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
-      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15}, [%16]; tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0][0]), "=r"(r[0][1]), "=r"(r[0][2]), "=r"(r[0][3]), "=r"(r[0][4]), "=r"(r[0][5]), "=r"(r[0][6]),
+        "=r"(r[0][7]), "=r"(r[0][8]), "=r"(r[0][9]), "=r"(r[0][10]), "=r"(r[0][11]), "=r"(r[0][12]),
+        "=r"(r[0][13]), "=r"(r[0][14]), "=r"(r[0][15])
+      : "r"(taddr)
       : "memory");
 }
 
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// 16 columns from each of two addresses, one wait.
+__device__ __forceinline__ void tmem_ld_wait(uint32_t ta, uint32_t (&ra)[1][16], uint32_t tb, uint32_t (&rb)[1][16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15}, [%32]; tcgen05.ld.sync.aligned.32x32b.x16.b32 {%16, %17, %18, %19, "
+      "%20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%33]; "
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(ra[0][0]), "=r"(ra[0][1]), "=r"(ra[0][2]), "=r"(ra[0][3]), "=r"(ra[0][4]), "=r"(ra[0][5]),
+        "=r"(ra[0][6]), "=r"(ra[0][7]), "=r"(ra[0][8]), "=r"(ra[0][9]), "=r"(ra[0][10]), "=r"(ra[0][11]),
+        "=r"(ra[0][12]), "=r"(ra[0][13]), "=r"(ra[0][14]), "=r"(ra[0][15]), "=r"(rb[0][0]), "=r"(rb[0][1]),
+        "=r"(rb[0][2]), "=r"(rb[0][3]), "=r"(rb[0][4]), "=r"(rb[0][5]), "=r"(rb[0][6]), "=r"(rb[0][7]),
+        "=r"(rb[0][8]), "=r"(rb[0][9]), "=r"(rb[0][10]), "=r"(rb[0][11]), "=r"(rb[0][12]), "=r"(rb[0][13]),
+        "=r"(rb[0][14]), "=r"(rb[0][15])
+      : "r"(ta), "r"(tb)
+      : "memory");
+}
+
+// 32 columns.
+__device__ __forceinline__ void tmem_ld_wait(uint32_t taddr, uint32_t (&r)[2][16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31}, [%32]; tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0][0]), "=r"(r[0][1]), "=r"(r[0][2]), "=r"(r[0][3]), "=r"(r[0][4]), "=r"(r[0][5]), "=r"(r[0][6]),
+        "=r"(r[0][7]), "=r"(r[0][8]), "=r"(r[0][9]), "=r"(r[0][10]), "=r"(r[0][11]), "=r"(r[0][12]),
+        "=r"(r[0][13]), "=r"(r[0][14]), "=r"(r[0][15]), "=r"(r[1][0]), "=r"(r[1][1]), "=r"(r[1][2]),
+        "=r"(r[1][3]), "=r"(r[1][4]), "=r"(r[1][5]), "=r"(r[1][6]), "=r"(r[1][7]), "=r"(r[1][8]), "=r"(r[1][9]),
+        "=r"(r[1][10]), "=r"(r[1][11]), "=r"(r[1][12]), "=r"(r[1][13]), "=r"(r[1][14]), "=r"(r[1][15])
+      : "r"(taddr)
+      : "memory");
+}
+
+// 64 columns.
+__device__ __forceinline__ void tmem_ld_wait(uint32_t taddr, uint32_t (&r)[4][16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+      "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64]; "
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0][0]), "=r"(r[0][1]), "=r"(r[0][2]), "=r"(r[0][3]), "=r"(r[0][4]), "=r"(r[0][5]), "=r"(r[0][6]),
+        "=r"(r[0][7]), "=r"(r[0][8]), "=r"(r[0][9]), "=r"(r[0][10]), "=r"(r[0][11]), "=r"(r[0][12]),
+        "=r"(r[0][13]), "=r"(r[0][14]), "=r"(r[0][15]), "=r"(r[1][0]), "=r"(r[1][1]), "=r"(r[1][2]),
+        "=r"(r[1][3]), "=r"(r[1][4]), "=r"(r[1][5]), "=r"(r[1][6]), "=r"(r[1][7]), "=r"(r[1][8]), "=r"(r[1][9]),
+        "=r"(r[1][10]), "=r"(r[1][11]), "=r"(r[1][12]), "=r"(r[1][13]), "=r"(r[1][14]), "=r"(r[1][15]),
+        "=r"(r[2][0]), "=r"(r[2][1]), "=r"(r[2][2]), "=r"(r[2][3]), "=r"(r[2][4]), "=r"(r[2][5]), "=r"(r[2][6]),
+        "=r"(r[2][7]), "=r"(r[2][8]), "=r"(r[2][9]), "=r"(r[2][10]), "=r"(r[2][11]), "=r"(r[2][12]),
+        "=r"(r[2][13]), "=r"(r[2][14]), "=r"(r[2][15]), "=r"(r[3][0]), "=r"(r[3][1]), "=r"(r[3][2]),
+        "=r"(r[3][3]), "=r"(r[3][4]), "=r"(r[3][5]), "=r"(r[3][6]), "=r"(r[3][7]), "=r"(r[3][8]), "=r"(r[3][9]),
+        "=r"(r[3][10]), "=r"(r[3][11]), "=r"(r[3][12]), "=r"(r[3][13]), "=r"(r[3][14]), "=r"(r[3][15])
+      : "r"(taddr)
+      : "memory");
+}
+
+// 32 columns from each of two addresses, one wait.
+__device__ __forceinline__ void tmem_ld_wait(uint32_t ta, uint32_t (&ra)[2][16], uint32_t tb, uint32_t (&rb)[2][16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31}, [%64]; tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32, %33, %34, %35, %36, %37, "
+      "%38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, "
+      "%56, %57, %58, %59, %60, %61, %62, %63}, [%65]; tcgen05.wait::ld.sync.aligned;"
+      : "=r"(ra[0][0]), "=r"(ra[0][1]), "=r"(ra[0][2]), "=r"(ra[0][3]), "=r"(ra[0][4]), "=r"(ra[0][5]),
+        "=r"(ra[0][6]), "=r"(ra[0][7]), "=r"(ra[0][8]), "=r"(ra[0][9]), "=r"(ra[0][10]), "=r"(ra[0][11]),
+        "=r"(ra[0][12]), "=r"(ra[0][13]), "=r"(ra[0][14]), "=r"(ra[0][15]), "=r"(ra[1][0]), "=r"(ra[1][1]),
+        "=r"(ra[1][2]), "=r"(ra[1][3]), "=r"(ra[1][4]), "=r"(ra[1][5]), "=r"(ra[1][6]), "=r"(ra[1][7]),
+        "=r"(ra[1][8]), "=r"(ra[1][9]), "=r"(ra[1][10]), "=r"(ra[1][11]), "=r"(ra[1][12]), "=r"(ra[1][13]),
+        "=r"(ra[1][14]), "=r"(ra[1][15]), "=r"(rb[0][0]), "=r"(rb[0][1]), "=r"(rb[0][2]), "=r"(rb[0][3]),
+        "=r"(rb[0][4]), "=r"(rb[0][5]), "=r"(rb[0][6]), "=r"(rb[0][7]), "=r"(rb[0][8]), "=r"(rb[0][9]),
+        "=r"(rb[0][10]), "=r"(rb[0][11]), "=r"(rb[0][12]), "=r"(rb[0][13]), "=r"(rb[0][14]), "=r"(rb[0][15]),
+        "=r"(rb[1][0]), "=r"(rb[1][1]), "=r"(rb[1][2]), "=r"(rb[1][3]), "=r"(rb[1][4]), "=r"(rb[1][5]),
+        "=r"(rb[1][6]), "=r"(rb[1][7]), "=r"(rb[1][8]), "=r"(rb[1][9]), "=r"(rb[1][10]), "=r"(rb[1][11]),
+        "=r"(rb[1][12]), "=r"(rb[1][13]), "=r"(rb[1][14]), "=r"(rb[1][15])
+      : "r"(ta), "r"(tb)
+      : "memory");
+}
+
+// TMEM store of 64 columns, with its tcgen05.wait::st in the same statement (the source
+// registers stay untouched until the store has read them).
+__device__ __forceinline__ void tmem_st_wait(uint32_t taddr, const uint32_t (&r)[4][16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
+      "%29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, "
+      "%47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, "
+      "%64}; tcgen05.wait::st.sync.aligned;"
+      ::"r"(taddr),
+        "r"(r[0][0]), "r"(r[0][1]), "r"(r[0][2]), "r"(r[0][3]), "r"(r[0][4]), "r"(r[0][5]), "r"(r[0][6]),
+        "r"(r[0][7]), "r"(r[0][8]), "r"(r[0][9]), "r"(r[0][10]), "r"(r[0][11]), "r"(r[0][12]), "r"(r[0][13]),
+        "r"(r[0][14]), "r"(r[0][15]), "r"(r[1][0]), "r"(r[1][1]), "r"(r[1][2]), "r"(r[1][3]), "r"(r[1][4]),
+        "r"(r[1][5]), "r"(r[1][6]), "r"(r[1][7]), "r"(r[1][8]), "r"(r[1][9]), "r"(r[1][10]), "r"(r[1][11]),
+        "r"(r[1][12]), "r"(r[1][13]), "r"(r[1][14]), "r"(r[1][15]), "r"(r[2][0]), "r"(r[2][1]), "r"(r[2][2]),
+        "r"(r[2][3]), "r"(r[2][4]), "r"(r[2][5]), "r"(r[2][6]), "r"(r[2][7]), "r"(r[2][8]), "r"(r[2][9]),
+        "r"(r[2][10]), "r"(r[2][11]), "r"(r[2][12]), "r"(r[2][13]), "r"(r[2][14]), "r"(r[2][15]), "r"(r[3][0]),
+        "r"(r[3][1]), "r"(r[3][2]), "r"(r[3][3]), "r"(r[3][4]), "r"(r[3][5]), "r"(r[3][6]), "r"(r[3][7]),
+        "r"(r[3][8]), "r"(r[3][9]), "r"(r[3][10]), "r"(r[3][11]), "r"(r[3][12]), "r"(r[3][13]), "r"(r[3][14]),
+        "r"(r[3][15])
+      : "memory");
+}
 
 // ---- small helpers -------------------------------------------------------------------------
 

@@ -58,6 +58,20 @@ def test_tc_matches_oracle(dk, dv, B, L):
     assert err(so, Sref) <= TOL_BF16
 
 
+@pytest.mark.parametrize("b,h,dk,dv,L", [(10, 16, 128, 128, 200), (5, 16, 64, 256, 130)])
+def test_tc_wide_slices(b, h, dk, dv, L):
+    """Enough (batch, head) pairs for the 128-column d_v slices (chunk 64): same bar."""
+    B = 64
+    q, k, v = si.qkv(b, L, h, dk, dv, 80 + dk, "bf16")
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+    ref, Sref, _ = oracle.recurrent(q, k, v, g, th, 0, FLAGS)
+    o, so = run_tc(q, k, v, g, th, B, want_state=True)
+    e = err(o, ref)
+    print(f"wide slices b={b} h={h} dk={dk} dv={dv}: max|err|/rms = {e:.3e}")
+    assert e <= TOL_BF16
+    assert err(so, Sref) <= TOL_BF16
+
+
 @pytest.mark.parametrize("flags", [0, rn.F_XPOS, rn.F_SCALE_SQRT_D, rn.F_NORM_D, FLAGS])
 def test_tc_flag_combinations(flags):
     b, L, h, dk, dv, B = 1, 200, 4, 128, 64, 64
