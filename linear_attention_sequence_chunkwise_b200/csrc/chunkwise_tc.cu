@@ -908,14 +908,21 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
       // Descriptors are built once per operand tile and advanced by constants (the start
       // address field never carries: every operand lies below 256 KB of shared memory).
       auto kstep = [](int kk) -> uint64_t { return static_cast<uint64_t>(((kk / 4) * T * 128 + (kk % 4) * 32) >> 4); };
-      // S'' of the unit and, for the last row block, the state increment Kz_w^T V_w.
-      auto front = [&](const UnitIter<T>& f) -> bool {
-        const int s = f.k % C::NS;
-        if (!mbar_wait(bar(Q_CONV_FULL + s), (f.k / C::NS) & 1)) return false;
-        if (f.k >= C::SBUF && !mbar_wait(bar(Q_S_FREE + (f.k % C::SBUF)), ((f.k - C::SBUF) / C::SBUF) & 1)) return false;
+      // The three MMA groups of a unit: F = S'' and, on the last row block, the state increment
+      // Kz_w^T V_w; X = the cross term of a row block (its first unit); P = P V into O.  Each
+      // has a non-blocking readiness test.  The issuer takes whichever group is ready -- X and P
+      // of the oldest unit first, F at most LA units ahead -- so a late conversion of a later
+      // unit never holds back the output (and the stage release) of an earlier one.
+      auto f_ready = [&](const UnitIter<T>& f) -> bool {
+        if (!mbar_test(bar(Q_CONV_FULL + f.k % C::NS), (f.k / C::NS) & 1)) return false;
+        if (f.k >= C::SBUF && !mbar_test(bar(Q_S_FREE + (f.k % C::SBUF)), ((f.k - C::SBUF) / C::SBUF) & 1)) return false;
         if (f.last_row() && f.dr >= C::DRBUF &&
-            !mbar_wait(bar(Q_DR_FREE + (f.dr % C::DRBUF)), ((f.dr - C::DRBUF) / C::DRBUF) & 1))
+            !mbar_test(bar(Q_DR_FREE + (f.dr % C::DRBUF)), ((f.dr - C::DRBUF) / C::DRBUF) & 1))
           return false;
+        return true;
+      };
+      auto f_issue = [&](const UnitIter<T>& f) {
+        const int s = f.k % C::NS;
         tc_fence_after();
         const uint32_t tS = tmem + C::COL_S + (f.k % C::SBUF) * T;
         const uint64_t dq = sdesc_sw128(sQ(s), 16, 1024), dk = sdesc_sw128(sK(s), 16, 1024);
@@ -933,25 +940,29 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
                          dv + static_cast<uint64_t>((ks * 2048) >> 4), ID_R, ks > 0);
           mma_commit(bar(Q_DR_FULL + (f.dr % C::DRBUF)));
         }
-        return true;
       };
-      // Cross term of the row block (first unit only) and P V into O.
-      auto back = [&](const UnitIter<T>& q) -> bool {
+      auto x_ready = [&](const UnitIter<T>& q) -> bool {
+        if (!mbar_test(bar(Q_R16_FULL + (q.i % C::RBUF)), (q.i / C::RBUF) & 1)) return false;
+        return q.rb < 2 || mbar_test(bar(Q_O_FREE + (q.rb & 1)), ((q.rb - 2) >> 1) & 1);
+      };
+      auto x_issue = [&](const UnitIter<T>& q) {
         const int s = q.k % C::NS;
-        const uint32_t tO = tmem + C::COL_O + (q.rb & 1) * DVS;
-        if (q.w == 0) {
-          if (!mbar_wait(bar(Q_R16_FULL + (q.i % C::RBUF)), (q.i / C::RBUF) & 1)) return false;
-          if (q.rb >= 2 && !mbar_wait(bar(Q_O_FREE + (q.rb & 1)), ((q.rb - 2) >> 1) & 1)) return false;
-          tc_fence_after();
-          const uint32_t tX = (C::XBUF > 0 && nb > 1) ? tmem + C::COL_X + (q.rb & 1) * DVS : tO;
-          const uint64_t dq = sdesc_sw128(sQ(s), 16, 1024), dr = sdesc_sw128(sR(q.i), DK * 128, 1024);
-#pragma unroll
-          for (int kk = 0; kk < DK / 16; ++kk)
-            mma_f16_ss(tX, dq + kstep(kk), dr + static_cast<uint64_t>((kk * 2048) >> 4), ID_X, kk > 0);
-          if (q.last_row()) mma_commit(bar(Q_R16_FREE + (q.i % C::RBUF)));
-        }
-        if (!mbar_wait(bar(Q_P_FULL + (q.k % C::PBUF)), (q.k / C::PBUF) & 1)) return false;
         tc_fence_after();
+        const uint32_t tO = tmem + C::COL_O + (q.rb & 1) * DVS;
+        const uint32_t tX = (C::XBUF > 0 && nb > 1) ? tmem + C::COL_X + (q.rb & 1) * DVS : tO;
+        const uint64_t dq = sdesc_sw128(sQ(s), 16, 1024), dr = sdesc_sw128(sR(q.i), DK * 128, 1024);
+#pragma unroll
+        for (int kk = 0; kk < DK / 16; ++kk)
+          mma_f16_ss(tX, dq + kstep(kk), dr + static_cast<uint64_t>((kk * 2048) >> 4), ID_X, kk > 0);
+        if (q.last_row()) mma_commit(bar(Q_R16_FREE + (q.i % C::RBUF)));
+      };
+      auto p_ready = [&](const UnitIter<T>& q) -> bool {
+        return mbar_test(bar(Q_P_FULL + (q.k % C::PBUF)), (q.k / C::PBUF) & 1);
+      };
+      auto p_issue = [&](const UnitIter<T>& q) {
+        const int s = q.k % C::NS;
+        tc_fence_after();
+        const uint32_t tO = tmem + C::COL_O + (q.rb & 1) * DVS;
         const uint64_t dp = sdesc_sw128(sP(q.k), 16, 1024), dv = sdesc_sw128(sV(s), T * 128, 1024);
         const uint32_t acc0 = (q.w > 0 || nb == 1) ? 1u : 0u;
 #pragma unroll
@@ -960,20 +971,39 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
         mma_commit(bar(Q_P_FREE + (q.k % C::PBUF)));
         if (q.rb_done()) mma_commit(bar(Q_O_FULL + (q.rb & 1)));
         mma_commit(bar(Q_STAGE_EMPTY + s));
-        return true;
       };
+      constexpr int LA = 2;  // F of unit f only while f <= q + LA (q = oldest unit with P pending)
       UnitIter<T> f, q;
       f.start(a.L, nb);
       q.start(a.L, nb);
-      bool ok = front(f);
-      f.next();
-      while (ok && q.valid()) {
-        if (f.valid()) {
-          ok = front(f);
-          f.next();
+      bool x_done = false;
+      long long idle_since = clock64();
+      while (q.valid()) {
+        bool progress = false;
+        if (q.k < f.k) {  // F of unit q has been issued
+          if (q.w == 0 && !x_done && x_ready(q)) {
+            x_issue(q);
+            x_done = true;
+            progress = true;
+          }
+          if ((q.w != 0 || x_done) && p_ready(q)) {
+            p_issue(q);
+            q.next();
+            x_done = false;
+            progress = true;
+          }
         }
-        if (ok) ok = back(q);
-        q.next();
+        if (!progress && f.valid() && f.k <= q.k + LA && f_ready(f)) {
+          f_issue(f);
+          f.next();
+          progress = true;
+        }
+        if (progress) {
+          idle_since = clock64();
+        } else if (clock64() - idle_since > 4000000000LL) {
+          atomicAdd(&g_wait_timeouts, 1u);  // same bound and report as a blocking wait
+          break;
+        }
       }
       mma_commit(bar(Q_DRAIN));
       mbar_wait(bar(Q_DRAIN), 0);
