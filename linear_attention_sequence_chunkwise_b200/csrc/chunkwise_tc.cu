@@ -27,6 +27,9 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <algorithm>
+#include <cmath>
+
 #include "launch.h"
 #include "sm100_ptx.cuh"
 
@@ -52,6 +55,11 @@ struct TcArgs {
   int64_t pos0;
   uint32_t flags;
   int nb;  // sub-blocks of T rows per chunk (pipelined kernel)
+  // Sequence segments (pipelined kernel): CTA segment s writes the outputs of chunks
+  // [seg_lo[s], seg_hi[s]) and first replays the state over chunks [0, seg_lo[s]).
+  int n_seg;
+  int seg_lo[4];
+  int seg_hi[4];
 };
 
 template <int DK, int T>
@@ -567,7 +575,11 @@ struct Cfg3 {
   static constexpr int NDV = DVS / 64;              // 64-column boxes of the d_v slice
   static constexpr int RBLK = DK > 128 ? 2 : 1;     // 128-row blocks of the state increment
   static constexpr int MR = DK >= 128 ? 128 : 64;
-  static constexpr int WARPS_S = 4 * RBLK * NDV;    // one thread per (d_k row, 64 columns)
+  // RTM: the fp32 state lives in tensor memory (the increment's columns) and each state
+  // increment accumulates into it; otherwise the state group holds it in registers, one
+  // thread per (d_k row, 64 columns).  RTM needs one sub-block per chunk (the 128-wide slice).
+  static constexpr bool RTM = DVS == 128;
+  static constexpr int WARPS_S = RTM ? 4 * RBLK : 4 * RBLK * NDV;
   static constexpr int WARP_S0 = 4;
   static constexpr int WARP_CONV0 = WARP_S0 + WARPS_S;
   static constexpr int CONV_WARPS = 4;
@@ -647,38 +659,48 @@ __device__ __forceinline__ float row_factor_f32(float gamma, float sqrt_dk_inv, 
   return f;
 }
 
-// Walks the units of the whole sequence in the order every role processes them:
-// for chunk i, for row block u < nbw_i, for column block w <= u  (nbw_i = ceil(b'_i / T)).
-template <int T>
+// Walks the units of the CTA's part of the sequence in the order every role processes them:
+// for chunk i < c_hi, for row block u < nbw_i, for column block w <= u  (nbw_i = ceil(b'_i / T)).
+// Chunks below c_lo are state replay only: just their last row block (u = nbw_i - 1), whose
+// units carry the state increments.
+template <int T, bool SEG>
 struct UnitIter {
   int L, nb;         // sequence length, sub-blocks per full chunk
+  int lo, hi;        // first chunk with outputs, end of the CTA's chunks (SEG only)
   int i, u, w;       // current unit
   int nbw, bl;       // sub-blocks and length of chunk i
-  int k;             // unit sequence number
-  int rb;            // row-block sequence number (for O/X buffers)
+  int k;             // unit sequence number (stages, TMA, conversion)
+  int kf_;           // sequence number among output units (SEG only; equals k otherwise)
+  int rb;            // row-block sequence number among output units (O/X buffers)
   int dr;            // sequence number of state-increment units (u == nbw - 1)
-  __device__ void start(int L_, int nb_) {
+  __device__ void start(int L_, int nb_, int c_lo_, int c_hi_) {
     L = L_;
     nb = nb_;
-    i = 0; u = 0; w = 0; k = 0; rb = 0; dr = 0;
-    set_chunk();
+    lo = c_lo_;
+    hi = c_hi_;
+    i = 0; k = 0; kf_ = 0; rb = 0; dr = 0;
+    if (valid()) set_chunk();
   }
   __device__ void set_chunk() {
     bl = min(nb * T, L - i * nb * T);
     nbw = (bl + T - 1) / T;
+    u = pre() ? nbw - 1 : 0;
+    w = 0;
   }
-  __device__ bool valid() const { return i * nb * T < L; }
+  __device__ bool valid() const { return (!SEG || i < hi) && i * nb * T < L; }
+  __device__ bool pre() const { return SEG && i < lo; }     // state replay only
+  __device__ int kf() const { return SEG ? kf_ : k; }
   __device__ bool last_row() const { return u == nbw - 1; }  // this unit carries a state increment
   __device__ bool rb_done() const { return w == u; }         // last unit of its row block
   __device__ int t0() const { return i * nb * T; }          // chunk start (token)
   __device__ void next() {
     if (last_row()) ++dr;
+    if (SEG && !pre()) ++kf_;
     ++k;
     if (w < u) { ++w; return; }
-    ++rb;
+    if (!pre()) ++rb;
     w = 0;
     if (u + 1 < nbw) { ++u; return; }
-    u = 0;
     ++i;
     if (valid()) set_chunk();
   }
@@ -748,6 +770,8 @@ struct UnitConverter {
   }
 
   // In place: q -> gamma^(r+1) rot(q), k -> gamma^(T-1-r) rot(k) as fp16 (r local); v -> fp16.
+  // WITH_Q = false (state replay) leaves the Q tile alone.
+  template <bool WITH_Q>
   __device__ void convert(uint32_t sq, uint32_t sk, uint32_t sv, const float2* bq, const float2* bk, bool xpos,
                           float log2g) const {
     const uint32_t box = (cs / 8) * T * 128;
@@ -770,7 +794,7 @@ struct UnitConverter {
 #pragma unroll
       for (int k = 0; k < G; ++k) {
         const uint32_t off = box + sw128(r0 + RS * (kg + k), chunk);
-        ld_shared_v4(sq + off, q4[k][0], q4[k][1], q4[k][2], q4[k][3]);
+        if (WITH_Q) ld_shared_v4(sq + off, q4[k][0], q4[k][1], q4[k][2], q4[k][3]);
         ld_shared_v4(sk + off, k4[k][0], k4[k][1], k4[k][2], k4[k][3]);
       }
 #pragma unroll
@@ -778,15 +802,17 @@ struct UnitConverter {
         uint32_t qo[4], ko[4];
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
-          const float q0 = __uint_as_float(q4[k][jj] << 16), q1 = __uint_as_float(q4[k][jj] & 0xffff0000u);
+          if (WITH_Q) {
+            const float q0 = __uint_as_float(q4[k][jj] << 16), q1 = __uint_as_float(q4[k][jj] & 0xffff0000u);
+            qo[jj] = pack_f16x2(q0 * Fq[jj].x - q1 * Fq[jj].y, q0 * Fq[jj].y + q1 * Fq[jj].x);
+            Fq[jj] = cmul(Fq[jj], Zq[jj]);
+          }
           const float k0 = __uint_as_float(k4[k][jj] << 16), k1 = __uint_as_float(k4[k][jj] & 0xffff0000u);
-          qo[jj] = pack_f16x2(q0 * Fq[jj].x - q1 * Fq[jj].y, q0 * Fq[jj].y + q1 * Fq[jj].x);
           ko[jj] = pack_f16x2(k0 * Fk[jj].x - k1 * Fk[jj].y, k0 * Fk[jj].y + k1 * Fk[jj].x);
-          Fq[jj] = cmul(Fq[jj], Zq[jj]);
           Fk[jj] = cmul(Fk[jj], Zk[jj]);
         }
         const uint32_t off = box + sw128(r0 + RS * (kg + k), chunk);
-        st_shared_v4(sq + off, qo[0], qo[1], qo[2], qo[3]);
+        if (WITH_Q) st_shared_v4(sq + off, qo[0], qo[1], qo[2], qo[3]);
         st_shared_v4(sk + off, ko[0], ko[1], ko[2], ko[3]);
       }
     }
@@ -810,7 +836,7 @@ struct UnitConverter {
   }
 };
 
-template <int DK, int T, int DVS, typename Tout>
+template <int DK, int T, int DVS, bool SEG, typename Tout>
 __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
     tc_chunkwise_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v, TcArgs a, HeadParams hp) {
@@ -821,7 +847,22 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
   uint8_t* gbase = smem_raw + (sbase - raw_addr);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int dvb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int n_dvb = a.dv / DVS;
+  const int dvb = SEG ? blockIdx.x % n_dvb : blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  // Output chunks [c_lo, c_hi); [0, c_lo) replays the state.  Without segments the bounds are
+  // compile-time constants and every replay branch folds away.
+  int c_lo = 0, c_hi = 0x7fffffff;
+  if constexpr (SEG) {
+    const int seg = blockIdx.x / n_dvb;
+    c_lo = a.seg_lo[0];
+    c_hi = a.seg_hi[0];
+#pragma unroll
+    for (int i = 1; i < 4; ++i)  // (a constant-index select keeps the kernel parameters in place)
+      if (seg == i) {
+        c_lo = a.seg_lo[i];
+        c_hi = a.seg_hi[i];
+      }
+  }
   const float log2g = hp.log2g[h];
   const int nb = a.nb;
   const float sd = rsqrtf(static_cast<float>(DK));  // carried by P and the fp16 state copy
@@ -879,15 +920,16 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int issued[4] = {0, 0, 0, 0};
-      UnitIter<T> it;
-      for (it.start(a.L, nb); it.valid(); it.next()) {
+      UnitIter<T, SEG> it;
+      for (it.start(a.L, nb, c_lo, c_hi); it.valid(); it.next()) {
         const int s = it.k % C::NS;
         if (it.k >= C::NS && !mbar_wait(bar(Q_STAGE_EMPTY + s), ((it.k / C::NS) - 1) & 1)) break;
-        mbar_arrive_expect_tx(bar(Q_TMA_FULL + s), C::STAGE);
+        const bool with_q = !it.pre();  // state replay needs K and V only
+        mbar_arrive_expect_tx(bar(Q_TMA_FULL + s), with_q ? C::STAGE : C::STAGE - C::QBYTES);
         const int tq = it.t0() + it.u * T, tk = it.t0() + it.w * T;
 #pragma unroll
         for (int bx = 0; bx < DK / 64; ++bx) {
-          tma_load_4d(sQ(s) + bx * T * 128, &tm_q, bar(Q_TMA_FULL + s), bx * 64, h, tq, b);
+          if (with_q) tma_load_4d(sQ(s) + bx * T * 128, &tm_q, bar(Q_TMA_FULL + s), bx * 64, h, tq, b);
           tma_load_4d(sK(s) + bx * T * 128, &tm_k, bar(Q_TMA_FULL + s), bx * 64, h, tk, b);
         }
 #pragma unroll
@@ -913,22 +955,31 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
       // has a non-blocking readiness test.  The issuer takes whichever group is ready -- X and P
       // of the oldest unit first, F at most LA units ahead -- so a late conversion of a later
       // unit never holds back the output (and the stage release) of an earlier one.
-      auto f_ready = [&](const UnitIter<T>& f) -> bool {
+      auto f_ready = [&](const UnitIter<T, SEG>& f) -> bool {
         if (!mbar_test(bar(Q_CONV_FULL + f.k % C::NS), (f.k / C::NS) & 1)) return false;
-        if (f.k >= C::SBUF && !mbar_test(bar(Q_S_FREE + (f.k % C::SBUF)), ((f.k - C::SBUF) / C::SBUF) & 1)) return false;
-        if (f.last_row() && f.dr >= C::DRBUF &&
-            !mbar_test(bar(Q_DR_FREE + (f.dr % C::DRBUF)), ((f.dr - C::DRBUF) / C::DRBUF) & 1))
+        if (!f.pre() && f.kf() >= C::SBUF &&
+            !mbar_test(bar(Q_S_FREE + (f.kf() % C::SBUF)), ((f.kf() - C::SBUF) / C::SBUF) & 1))
           return false;
+        if constexpr (C::RTM) {
+          // the state group has scaled the resident state for this chunk (slot dr & 1)
+          if (!mbar_test(bar(Q_DR_FREE + (f.dr & 1)), (f.dr >> 1) & 1)) return false;
+        } else {
+          if (f.last_row() && f.dr >= C::DRBUF &&
+              !mbar_test(bar(Q_DR_FREE + (f.dr % C::DRBUF)), ((f.dr - C::DRBUF) / C::DRBUF) & 1))
+            return false;
+        }
         return true;
       };
-      auto f_issue = [&](const UnitIter<T>& f) {
+      auto f_issue = [&](const UnitIter<T, SEG>& f) {
         const int s = f.k % C::NS;
         tc_fence_after();
-        const uint32_t tS = tmem + C::COL_S + (f.k % C::SBUF) * T;
-        const uint64_t dq = sdesc_sw128(sQ(s), 16, 1024), dk = sdesc_sw128(sK(s), 16, 1024);
+        if (!f.pre()) {
+          const uint32_t tS = tmem + C::COL_S + (f.kf() % C::SBUF) * T;
+          const uint64_t dq = sdesc_sw128(sQ(s), 16, 1024), dk = sdesc_sw128(sK(s), 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < DK / 16; ++kk) mma_f16_ss(tS, dq + kstep(kk), dk + kstep(kk), ID_S, kk > 0);
-        mma_commit(bar(Q_S_FULL + (f.k % C::SBUF)));
+          for (int kk = 0; kk < DK / 16; ++kk) mma_f16_ss(tS, dq + kstep(kk), dk + kstep(kk), ID_S, kk > 0);
+          mma_commit(bar(Q_S_FULL + (f.kf() % C::SBUF)));
+        }
         if (f.last_row()) {
           const uint32_t tD = tmem + C::COL_DR + (f.dr % C::DRBUF) * C::RBLK * DVS;
           const uint64_t dkm = sdesc_sw128(sK(s), T * 128, 1024), dv = sdesc_sw128(sV(s), T * 128, 1024);
@@ -937,45 +988,49 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
 #pragma unroll
             for (int ks = 0; ks < T / 16; ++ks)
               mma_f16_ss(tD + blk * DVS, dkm + static_cast<uint64_t>((blk * 2 * T * 128 + ks * 2048) >> 4),
-                         dv + static_cast<uint64_t>((ks * 2048) >> 4), ID_R, ks > 0);
+                         dv + static_cast<uint64_t>((ks * 2048) >> 4), ID_R, (C::RTM || ks > 0) ? 1u : 0u);
           mma_commit(bar(Q_DR_FULL + (f.dr % C::DRBUF)));
         }
+        if (f.pre()) mma_commit(bar(Q_STAGE_EMPTY + s));  // a replay unit has no P V
       };
-      auto x_ready = [&](const UnitIter<T>& q) -> bool {
-        if (!mbar_test(bar(Q_R16_FULL + (q.i % C::RBUF)), (q.i / C::RBUF) & 1)) return false;
+      auto x_ready = [&](const UnitIter<T, SEG>& q) -> bool {
+        const int ri = q.i - c_lo;  // fp16 state copies are written for output chunks only
+        if (!mbar_test(bar(Q_R16_FULL + (ri % C::RBUF)), (ri / C::RBUF) & 1)) return false;
         return q.rb < 2 || mbar_test(bar(Q_O_FREE + (q.rb & 1)), ((q.rb - 2) >> 1) & 1);
       };
-      auto x_issue = [&](const UnitIter<T>& q) {
+      auto x_issue = [&](const UnitIter<T, SEG>& q) {
         const int s = q.k % C::NS;
         tc_fence_after();
         const uint32_t tO = tmem + C::COL_O + (q.rb & 1) * DVS;
         const uint32_t tX = (C::XBUF > 0 && nb > 1) ? tmem + C::COL_X + (q.rb & 1) * DVS : tO;
-        const uint64_t dq = sdesc_sw128(sQ(s), 16, 1024), dr = sdesc_sw128(sR(q.i), DK * 128, 1024);
+        const int ri = q.i - c_lo;
+        const uint64_t dq = sdesc_sw128(sQ(s), 16, 1024), dr = sdesc_sw128(sR(ri), DK * 128, 1024);
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk)
           mma_f16_ss(tX, dq + kstep(kk), dr + static_cast<uint64_t>((kk * 2048) >> 4), ID_X, kk > 0);
-        if (q.last_row()) mma_commit(bar(Q_R16_FREE + (q.i % C::RBUF)));
+        if (q.last_row()) mma_commit(bar(Q_R16_FREE + (ri % C::RBUF)));
       };
-      auto p_ready = [&](const UnitIter<T>& q) -> bool {
-        return mbar_test(bar(Q_P_FULL + (q.k % C::PBUF)), (q.k / C::PBUF) & 1);
+      auto p_ready = [&](const UnitIter<T, SEG>& q) -> bool {
+        return mbar_test(bar(Q_P_FULL + (q.kf() % C::PBUF)), (q.kf() / C::PBUF) & 1);
       };
-      auto p_issue = [&](const UnitIter<T>& q) {
+      auto p_issue = [&](const UnitIter<T, SEG>& q) {
         const int s = q.k % C::NS;
         tc_fence_after();
         const uint32_t tO = tmem + C::COL_O + (q.rb & 1) * DVS;
-        const uint64_t dp = sdesc_sw128(sP(q.k), 16, 1024), dv = sdesc_sw128(sV(s), T * 128, 1024);
+        const uint64_t dp = sdesc_sw128(sP(q.kf()), 16, 1024), dv = sdesc_sw128(sV(s), T * 128, 1024);
         const uint32_t acc0 = (q.w > 0 || nb == 1) ? 1u : 0u;
 #pragma unroll
         for (int kk = 0; kk < T / 16; ++kk)
           mma_f16_ss(tO, dp + kstep(kk), dv + static_cast<uint64_t>((kk * 2048) >> 4), ID_X, kk > 0 ? 1u : acc0);
-        mma_commit(bar(Q_P_FREE + (q.k % C::PBUF)));
+        mma_commit(bar(Q_P_FREE + (q.kf() % C::PBUF)));
         if (q.rb_done()) mma_commit(bar(Q_O_FULL + (q.rb & 1)));
         mma_commit(bar(Q_STAGE_EMPTY + s));
       };
       constexpr int LA = 2;  // F of unit f only while f <= q + LA (q = oldest unit with P pending)
-      UnitIter<T> f, q;
-      f.start(a.L, nb);
-      q.start(a.L, nb);
+      UnitIter<T, SEG> f, q;
+      f.start(a.L, nb, c_lo, c_hi);
+      q.start(a.L, nb, c_lo, c_hi);
+      while (q.valid() && q.pre()) q.next();  // q walks output units only
       bool x_done = false;
       long long idle_since = clock64();
       while (q.valid()) {
@@ -1014,8 +1069,8 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
     cv.init(threadIdx.x - 32 * C::WARP_CONV0, nb, hp);
     const bool xpos = (a.flags & RETNET_F_XPOS) != 0;
     bool ok = true;
-    UnitIter<T> it;
-    for (it.start(a.L, nb); ok && it.valid(); it.next()) {
+    UnitIter<T, SEG> it;
+    for (it.start(a.L, nb, c_lo, c_hi); ok && it.valid(); it.next()) {
       const int s = it.k % C::NS;
       float2* tq = tab + (it.k & 1) * DK;
       float2* tk = tq + DK / 2;
@@ -1026,88 +1081,197 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
       ok = mbar_wait(bar(Q_TAB + (it.k & 1)), (it.k >> 1) & 1);
       if (ok) ok = mbar_wait(bar(Q_TMA_FULL + s), (it.k / C::NS) & 1);
       if (!ok) break;
-      cv.convert(sQ(s), sK(s), sV(s), tq, tk, xpos, log2g);
+      if (it.pre())
+        cv.template convert<false>(sQ(s), sK(s), sV(s), tq, tk, xpos, log2g);
+      else
+        cv.template convert<true>(sQ(s), sK(s), sV(s), tq, tk, xpos, log2g);
       fence_proxy_async_smem();
       mbar_arrive(bar(Q_CONV_FULL + s));
     }
   } else if (warp >= C::WARP_S0) {
     // ------------------------------------------------------------------ state group
-    // Thread = (d_k row, 64-column box ch of the slice); warp % 4 selects its TMEM lane quarter.
-    constexpr int RC = 64;
-    const int ws = warp - C::WARP_S0;
-    const int blk = (ws / 4) % C::RBLK;
-    const int ch = ws / (4 * C::RBLK);
-    const uint32_t lane_off = static_cast<uint32_t>(32 * (warp % 4)) << 16;
-    const int dk = (DK == 64) ? (lane < 16 ? 16 * (warp % 4) + lane : -1) : blk * 128 + 32 * (warp % 4) + lane;
-    const int64_t bh = static_cast<int64_t>(b) * a.heads + h;
-    const size_t srow = static_cast<size_t>(a.dv);
-    const int col0 = dvb * DVS + ch * RC;
-    float R[RC];
-#pragma unroll
-    for (int c = 0; c < RC; ++c) R[c] = 0.f;
-    if (dk >= 0 && a.state_in) {
-      const float* src = a.state_in + static_cast<size_t>(bh) * DK * a.dv + col0 + dk * srow;
-#pragma unroll
-      for (int c4 = 0; c4 < RC / 4; ++c4) {
-        const float4 x = *reinterpret_cast<const float4*>(src + 4 * c4);
-        R[4 * c4] = x.x; R[4 * c4 + 1] = x.y; R[4 * c4 + 2] = x.z; R[4 * c4 + 3] = x.w;
-      }
-    }
-    auto put_r16 = [&](uint32_t base) {
-      if (dk < 0) return;
-      base += ch * DK * 128;
-#pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8)
-        st_shared_v4(base + sw128(dk, c8), pack_f16x2(sd * R[8 * c8 + 0], sd * R[8 * c8 + 1]),
-                     pack_f16x2(sd * R[8 * c8 + 2], sd * R[8 * c8 + 3]),
-                     pack_f16x2(sd * R[8 * c8 + 4], sd * R[8 * c8 + 5]),
-                     pack_f16x2(sd * R[8 * c8 + 6], sd * R[8 * c8 + 7]));
-    };
-    put_r16(sR(0));
-    fence_proxy_async_smem();
-    mbar_arrive(bar(Q_R16_FULL + 0));
-    bool ok = true;
-    UnitIter<T> it;
-    for (it.start(a.L, nb); ok && it.valid(); it.next()) {
-      if (!it.last_row()) continue;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(Q_DR_FULL + (it.dr % C::DRBUF)), (it.dr / C::DRBUF) & 1));
-      if (!ok) break;
-      tc_fence_after();
-      // Horner form of R_i = gamma^b' R_{i-1} + sum_w gamma^(b'-(w+1)T) dR_w:
-      //   w = 0: R = gamma^(b'-(nbw-1)T) R + hh dR_0;  w > 0: R = gamma^T R + hh dR_w,
-      //   hh = gamma^(b' - nbw T) (1 for a full chunk).
-      const float g = (it.w == 0) ? exp2f(static_cast<float>(it.bl - (it.nbw - 1) * T) * log2g)
-                                  : decay_pow(log2g, T);
-      const float hh = exp2f(static_cast<float>(it.bl - it.nbw * T) * log2g);
-      const uint32_t tD = tmem + C::COL_DR + (it.dr % C::DRBUF) * C::RBLK * DVS + blk * DVS + ch * RC + lane_off;
-      constexpr int SW = C::LDW / 2;  // columns per load next to the 64 state registers
-#pragma unroll
-      for (int grp = 0; grp < RC / SW; ++grp) {
-        uint32_t u[SW / 16][16];
-        tmem_ld_wait(tD + SW * grp, u);
-        if (grp == RC / SW - 1) {
-          tc_fence_before();
-          mbar_arrive(bar(Q_DR_FREE + (it.dr % C::DRBUF)));
+    if constexpr (C::RTM) {
+      // The fp32 state stays in tensor memory; thread = one d_k row (its TMEM lane), all
+      // DVS columns.  Before chunk i's increment accumulates into it, the state group reads
+      // R_{i-1}, writes its fp16 copy (output chunks only) and stores gamma^T R_{i-1} back.
+      // With Kz = gamma^(T-1-c) rot(k) the increment of a chunk of b' rows is
+      // gamma^(b'-T) (Kz^T V); the factor is 1 except on the last chunk, where state_out takes it.
+      const int ws = warp - C::WARP_S0;
+      const int blk = ws / 4;
+      const uint32_t lane_off = static_cast<uint32_t>(32 * (warp % 4)) << 16;
+      const int dk = (DK == 64) ? (lane < 16 ? 16 * (warp % 4) + lane : -1) : blk * 128 + 32 * (warp % 4) + lane;
+      const int64_t bh = static_cast<int64_t>(b) * a.heads + h;
+      const size_t srow = static_cast<size_t>(a.dv);
+      const uint32_t tR = tmem + C::COL_DR + blk * DVS + lane_off;
+      const float gT = decay_pow(log2g, T);
+      constexpr int GW = 32;  // columns per batch
+      bool ok = true;
+      int last_dr = -1, last_bl = T;
+      UnitIter<T, SEG> it;
+      for (it.start(a.L, nb, c_lo, c_hi); ok && it.valid(); it.next()) {
+        const int d = it.dr;
+        if (d > 0) {  // the previous increment has landed: the master holds R_{i-1}
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(Q_DR_FULL + 0), (d - 1) & 1));
+          if (!ok) break;
+          tc_fence_after();
         }
+        const bool out = !it.pre();
+        const int ri = it.i - c_lo;
+        if (out && ri >= C::RBUF) {
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(Q_R16_FREE + (ri % C::RBUF)), ((ri - C::RBUF) / C::RBUF) & 1));
+          if (!ok) break;
+        }
+        const uint32_t r16 = sR(ri);
+#pragma unroll 1
+        for (int grp = 0; grp < DVS / GW; ++grp) {
+          uint32_t u[GW / 16][16];
+          if (d > 0) {
+            tmem_ld_wait(tR + GW * grp, u);
+          } else {  // chunk 0: the master starts from state_in (or zeros)
 #pragma unroll
-        for (int c = 0; c < SW; ++c) R[SW * grp + c] = fmaf(g, R[SW * grp + c], hh * __uint_as_float(u[c / 16][c % 16]));
+            for (int c = 0; c < GW; ++c) u[c / 16][c % 16] = 0u;
+            if (dk >= 0 && a.state_in) {
+              const float* src = a.state_in + static_cast<size_t>(bh) * DK * a.dv + dvb * DVS + GW * grp + dk * srow;
+#pragma unroll
+              for (int c4 = 0; c4 < GW / 4; ++c4) {
+                const float4 x = *reinterpret_cast<const float4*>(src + 4 * c4);
+                u[(4 * c4) / 16][(4 * c4) % 16] = __float_as_uint(x.x);
+                u[(4 * c4 + 1) / 16][(4 * c4 + 1) % 16] = __float_as_uint(x.y);
+                u[(4 * c4 + 2) / 16][(4 * c4 + 2) % 16] = __float_as_uint(x.z);
+                u[(4 * c4 + 3) / 16][(4 * c4 + 3) % 16] = __float_as_uint(x.w);
+              }
+            }
+          }
+          if (out && dk >= 0) {
+            // fp16 copy (times 1/sqrt(d_k)) into box (column / 64), 16-byte slots of 8 columns
+#pragma unroll
+            for (int c8 = 0; c8 < GW / 8; ++c8) {
+              const int col = GW * grp + 8 * c8;
+              const uint32_t* x = &u[(8 * c8) / 16][(8 * c8) % 16];
+              st_shared_v4(r16 + (col / 64) * DK * 128 + sw128(dk, (col % 64) / 8),
+                           pack_f16x2(sd * __uint_as_float(x[0]), sd * __uint_as_float(x[1])),
+                           pack_f16x2(sd * __uint_as_float(x[2]), sd * __uint_as_float(x[3])),
+                           pack_f16x2(sd * __uint_as_float(x[4]), sd * __uint_as_float(x[5])),
+                           pack_f16x2(sd * __uint_as_float(x[6]), sd * __uint_as_float(x[7])));
+            }
+          }
+#pragma unroll
+          for (int c = 0; c < GW; ++c) u[c / 16][c % 16] = __float_as_uint(gT * __uint_as_float(u[c / 16][c % 16]));
+          tmem_st_wait(tR + GW * grp, u);
+        }
+        if (out) fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(bar(Q_DR_FREE + (d & 1)));  // the master is ready for this chunk's increment
+        if (out) mbar_arrive(bar(Q_R16_FULL + (ri % C::RBUF)));
+        last_dr = d;
+        last_bl = it.bl;
       }
-      if (it.w + 1 < it.nbw) continue;  // chunk not finished
-      const int nxt = it.i + 1;
-      if (nxt * nb * T < a.L) {
-        // R16 buffer of chunk nxt was last read by the cross terms of chunk nxt - RBUF.
-        const int prev = nxt - C::RBUF;
-        if (prev >= 0)
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(Q_R16_FREE + (prev % C::RBUF)), (prev / C::RBUF) & 1));
-        if (!ok) break;
-        put_r16(sR(nxt));
-        fence_proxy_async_smem();
-        mbar_arrive(bar(Q_R16_FULL + (nxt % C::RBUF)));
-      } else if (dk >= 0 && a.state_out) {
-        float* dst = a.state_out + static_cast<size_t>(bh) * DK * a.dv + col0 + dk * srow;
+      // End of the sequence: R_last = gamma^(b'-T) * master once the last increment landed.
+      if (ok && last_dr >= 0 && (!SEG || c_hi * nb * T >= a.L)) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(Q_DR_FULL + 0), last_dr & 1));
+        tc_fence_after();
+        if (ok && a.state_out) {
+          const float hh = exp2f(static_cast<float>(last_bl - T) * log2g);
+#pragma unroll 1
+          for (int grp = 0; grp < DVS / GW; ++grp) {
+            uint32_t u[GW / 16][16];
+            tmem_ld_wait(tR + GW * grp, u);
+            if (dk >= 0) {
+              float* dst = a.state_out + static_cast<size_t>(bh) * DK * a.dv + dvb * DVS + GW * grp + dk * srow;
 #pragma unroll
-        for (int c4 = 0; c4 < RC / 4; ++c4)
-          *reinterpret_cast<float4*>(dst + 4 * c4) = make_float4(R[4 * c4], R[4 * c4 + 1], R[4 * c4 + 2], R[4 * c4 + 3]);
+              for (int c4 = 0; c4 < GW / 4; ++c4)
+                *reinterpret_cast<float4*>(dst + 4 * c4) =
+                    make_float4(hh * __uint_as_float(u[(4 * c4) / 16][(4 * c4) % 16]),
+                                hh * __uint_as_float(u[(4 * c4 + 1) / 16][(4 * c4 + 1) % 16]),
+                                hh * __uint_as_float(u[(4 * c4 + 2) / 16][(4 * c4 + 2) % 16]),
+                                hh * __uint_as_float(u[(4 * c4 + 3) / 16][(4 * c4 + 3) % 16]));
+            }
+          }
+        }
+      }
+    } else {
+      // Thread = (d_k row, 64-column box ch of the slice); warp % 4 selects its TMEM lane quarter.
+      constexpr int RC = 64;
+      const int ws = warp - C::WARP_S0;
+      const int blk = (ws / 4) % C::RBLK;
+      const int ch = ws / (4 * C::RBLK);
+      const uint32_t lane_off = static_cast<uint32_t>(32 * (warp % 4)) << 16;
+      const int dk = (DK == 64) ? (lane < 16 ? 16 * (warp % 4) + lane : -1) : blk * 128 + 32 * (warp % 4) + lane;
+      const int64_t bh = static_cast<int64_t>(b) * a.heads + h;
+      const size_t srow = static_cast<size_t>(a.dv);
+      const int col0 = dvb * DVS + ch * RC;
+      float R[RC];
+  #pragma unroll
+      for (int c = 0; c < RC; ++c) R[c] = 0.f;
+      if (dk >= 0 && a.state_in) {
+        const float* src = a.state_in + static_cast<size_t>(bh) * DK * a.dv + col0 + dk * srow;
+  #pragma unroll
+        for (int c4 = 0; c4 < RC / 4; ++c4) {
+          const float4 x = *reinterpret_cast<const float4*>(src + 4 * c4);
+          R[4 * c4] = x.x; R[4 * c4 + 1] = x.y; R[4 * c4 + 2] = x.z; R[4 * c4 + 3] = x.w;
+        }
+      }
+      auto put_r16 = [&](uint32_t base) {
+        if (dk < 0) return;
+        base += ch * DK * 128;
+  #pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8)
+          st_shared_v4(base + sw128(dk, c8), pack_f16x2(sd * R[8 * c8 + 0], sd * R[8 * c8 + 1]),
+                       pack_f16x2(sd * R[8 * c8 + 2], sd * R[8 * c8 + 3]),
+                       pack_f16x2(sd * R[8 * c8 + 4], sd * R[8 * c8 + 5]),
+                       pack_f16x2(sd * R[8 * c8 + 6], sd * R[8 * c8 + 7]));
+      };
+      if (c_lo == 0) {  // otherwise written once the replay reaches the first output chunk
+        put_r16(sR(0));
+        fence_proxy_async_smem();
+        mbar_arrive(bar(Q_R16_FULL + 0));
+      }
+      bool ok = true;
+      UnitIter<T, SEG> it;
+      for (it.start(a.L, nb, c_lo, c_hi); ok && it.valid(); it.next()) {
+        if (!it.last_row()) continue;
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(Q_DR_FULL + (it.dr % C::DRBUF)), (it.dr / C::DRBUF) & 1));
+        if (!ok) break;
+        tc_fence_after();
+        // Horner form of R_i = gamma^b' R_{i-1} + sum_w gamma^(b'-(w+1)T) dR_w:
+        //   w = 0: R = gamma^(b'-(nbw-1)T) R + hh dR_0;  w > 0: R = gamma^T R + hh dR_w,
+        //   hh = gamma^(b' - nbw T) (1 for a full chunk).
+        const float g = (it.w == 0) ? exp2f(static_cast<float>(it.bl - (it.nbw - 1) * T) * log2g)
+                                    : decay_pow(log2g, T);
+        const float hh = exp2f(static_cast<float>(it.bl - it.nbw * T) * log2g);
+        const uint32_t tD = tmem + C::COL_DR + (it.dr % C::DRBUF) * C::RBLK * DVS + blk * DVS + ch * RC + lane_off;
+        constexpr int SW = C::LDW / 2;  // columns per load next to the 64 state registers
+  #pragma unroll
+        for (int grp = 0; grp < RC / SW; ++grp) {
+          uint32_t u[SW / 16][16];
+          tmem_ld_wait(tD + SW * grp, u);
+          if (grp == RC / SW - 1) {
+            tc_fence_before();
+            mbar_arrive(bar(Q_DR_FREE + (it.dr % C::DRBUF)));
+          }
+  #pragma unroll
+          for (int c = 0; c < SW; ++c) R[SW * grp + c] = fmaf(g, R[SW * grp + c], hh * __uint_as_float(u[c / 16][c % 16]));
+        }
+        if (it.w + 1 < it.nbw) continue;  // chunk not finished
+        const int nxt = it.i + 1;
+        const bool seq_end = nxt * nb * T >= a.L;
+        if (!seq_end && nxt < c_hi) {
+          if (nxt < c_lo) continue;  // still replaying
+          // fp16 copy ri of output chunk nxt; its buffer was last read by the cross terms of
+          // output chunk ri - RBUF.
+          const int ri = nxt - c_lo, prev = ri - C::RBUF;
+          if (prev >= 0)
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(Q_R16_FREE + (prev % C::RBUF)), (prev / C::RBUF) & 1));
+          if (!ok) break;
+          put_r16(sR(ri));
+          fence_proxy_async_smem();
+          mbar_arrive(bar(Q_R16_FULL + (ri % C::RBUF)));
+        } else if (seq_end && dk >= 0 && a.state_out) {
+          float* dst = a.state_out + static_cast<size_t>(bh) * DK * a.dv + col0 + dk * srow;
+  #pragma unroll
+          for (int c4 = 0; c4 < RC / 4; ++c4)
+            *reinterpret_cast<float4*>(dst + 4 * c4) = make_float4(R[4 * c4], R[4 * c4 + 1], R[4 * c4 + 2], R[4 * c4 + 3]);
+        }
       }
     }
   } else {
@@ -1193,9 +1357,10 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
     };
     bool ok = true;
     int pend_rb = -1, pend_i = 0, pend_u = 0, pend_bl = 0;  // a finished row block awaiting its epilogue
-    UnitIter<T> it;
-    for (it.start(a.L, nb); ok && it.valid(); it.next()) {
-      const int k = it.k;
+    UnitIter<T, SEG> it;
+    for (it.start(a.L, nb, c_lo, c_hi); ok && it.valid(); it.next()) {
+      if (it.pre()) continue;  // replay units have no scores
+      const int k = it.kf();
       ok = __all_sync(0xffffffffu, mbar_wait(bar(Q_S_FULL + (k % C::SBUF)), (k / C::SBUF) & 1));
       if (ok && k >= C::PBUF)
         ok = __all_sync(0xffffffffu, mbar_wait(bar(Q_P_FREE + (k % C::PBUF)), ((k - C::PBUF) / C::PBUF) & 1));
@@ -1296,15 +1461,46 @@ bool force_serial_kernel() {
 // Rows per unit of the pipelined kernel: 64 for d_k = 256 (shared memory), else min(B, 128).
 int pipe_tile_rows(int64_t d_k, int64_t chunk) { return d_k == 256 ? 64 : static_cast<int>(chunk < 128 ? chunk : 128); }
 
-// 128-column d_v slices (S and the Q/K conversion shared by twice the columns) need one
-// sub-block per chunk (no cross accumulator in tensor memory) and d_k <= 128.  They halve the
-// CTA count, so they are taken only when the wide grid still fills the GPU.
+// 128-column d_v slices share S and the Q/K conversion across twice the output columns
+// (about 1.6x the work per SM); they need one sub-block per chunk (no cross accumulator in
+// tensor memory) and d_k <= 128.  The halved CTA count is made up by sequence segments.
 bool pipe_wide_slice(const RetentionCall& c, int T) {
-  if (!(c.dims.d_k <= 128 && T == 64 && c.chunk == 64 && c.dims.d_v % 128 == 0)) return false;
+  return c.dims.d_k <= 128 && T == 64 && c.chunk == 64 && c.dims.d_v % 128 == 0;
+}
+
+int sm_count() {
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return false;
-  return c.dims.batch * c.dims.heads * (c.dims.d_v / 128) >= sms;
+    return 0;
+  return sms;
+}
+
+// Sequence segments.  With fewer (batch, head, d_v slice) CTAs than SMs, the chunks are split
+// into n_seg consecutive segments, one CTA each; the CTA of segment s first replays the state
+// over chunks [0, lo_s) (K and V only: TMA, conversion, state increment), then produces the
+// outputs of [lo_s, hi_s).  A replayed chunk costs about kReplayCost of an output chunk, and
+// the boundaries equalise rho * lo_s + (hi_s - lo_s) across segments.
+constexpr double kReplayCost = 0.45;
+void plan_segments(TcArgs& a, int64_t ctas, int sms) {
+  const int n = a.n_chunks;
+  int n_seg = (ctas > 0 && sms > 0) ? static_cast<int>(sms / ctas) : 1;
+  n_seg = std::min(n_seg, 4);
+  n_seg = std::min(n_seg, n / 4);  // at least four chunks a segment
+  if (n_seg < 2) return;
+  const double rho = kReplayCost, keep = 1.0 - rho;
+  const double cost = n * rho / (1.0 - std::pow(keep, n_seg));
+  double x = 0.0;
+  int prev = 0;
+  for (int s = 0; s < n_seg; ++s) {
+    x = keep * x + cost;
+    int hi = (s == n_seg - 1) ? n : static_cast<int>(std::lround(x));
+    hi = std::max(hi, prev + 1);
+    hi = std::min(hi, n - (n_seg - 1 - s));
+    a.seg_lo[s] = prev;
+    a.seg_hi[s] = hi;
+    prev = hi;
+  }
+  a.n_seg = n_seg;
 }
 
 TcArgs make_args(const RetentionCall& c, int n_chunks, int nb) {
@@ -1319,6 +1515,9 @@ TcArgs make_args(const RetentionCall& c, int n_chunks, int nb) {
   a.pos0 = c.pos0;
   a.flags = c.flags;
   a.nb = nb;
+  a.n_seg = 1;
+  for (int s = 0; s < 4; ++s) a.seg_lo[s] = a.seg_hi[s] = 0;
+  a.seg_hi[0] = n_chunks;
   return a;
 }
 
@@ -1343,10 +1542,15 @@ cudaError_t launch_pipe(const RetentionCall& c, const HeadParams& hp, cudaStream
   const int nb = static_cast<int>(c.chunk / T);
   const TcArgs a = make_args(c, static_cast<int>((c.dims.seqlen + c.chunk - 1) / c.chunk), nb);
   if (Cf::XBUF == 0 && nb != 1) return cudaErrorInvalidValue;
-  auto kern = tc_chunkwise_pipe_kernel<DK, T, DVS, Tout>;
+  TcArgs as = a;
+  dim3 grid = tc_grid(c.dims, DVS);
+  plan_segments(as, static_cast<int64_t>(grid.x) * grid.y * grid.z, sm_count());
+  grid.x *= as.n_seg;
+  auto kern = as.n_seg > 1 ? tc_chunkwise_pipe_kernel<DK, T, DVS, true, Tout>
+                           : tc_chunkwise_pipe_kernel<DK, T, DVS, false, Tout>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<tc_grid(c.dims, DVS), Cf::THREADS, Cf::SMEM, s>>>(mq, mk, mv, a, hp);
+  kern<<<grid, Cf::THREADS, Cf::SMEM, s>>>(mq, mk, mv, as, hp);
   return cudaGetLastError();
 }
 

@@ -248,6 +248,21 @@ __device__ __forceinline__ void tmem_ld_wait(uint32_t ta, uint32_t (&ra)[2][16],
       : "memory");
 }
 
+// TMEM store of 32 columns with its wait.
+__device__ __forceinline__ void tmem_st_wait(uint32_t taddr, const uint32_t (&r)[2][16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
+      "%29, %30, %31, %32}; tcgen05.wait::st.sync.aligned;"
+      ::"r"(taddr),
+        "r"(r[0][0]), "r"(r[0][1]), "r"(r[0][2]), "r"(r[0][3]), "r"(r[0][4]), "r"(r[0][5]), "r"(r[0][6]),
+        "r"(r[0][7]), "r"(r[0][8]), "r"(r[0][9]), "r"(r[0][10]), "r"(r[0][11]), "r"(r[0][12]), "r"(r[0][13]),
+        "r"(r[0][14]), "r"(r[0][15]), "r"(r[1][0]), "r"(r[1][1]), "r"(r[1][2]), "r"(r[1][3]), "r"(r[1][4]),
+        "r"(r[1][5]), "r"(r[1][6]), "r"(r[1][7]), "r"(r[1][8]), "r"(r[1][9]), "r"(r[1][10]), "r"(r[1][11]),
+        "r"(r[1][12]), "r"(r[1][13]), "r"(r[1][14]), "r"(r[1][15])
+      : "memory");
+}
+
 // TMEM store of 64 columns, with its tcgen05.wait::st in the same statement (the source
 // registers stay untouched until the store has read them).
 __device__ __forceinline__ void tmem_st_wait(uint32_t taddr, const uint32_t (&r)[4][16]) {

@@ -72,6 +72,25 @@ def test_tc_wide_slices(b, h, dk, dv, L):
     assert err(so, Sref) <= TOL_BF16
 
 
+@pytest.mark.parametrize("dk,dv,B,L,with_state", [(128, 128, 64, 64 * 9 + 5, False), (128, 64, 64, 64 * 17, True),
+                                                  (256, 64, 128, 128 * 8 + 30, True), (64, 128, 256, 256 * 8, False),
+                                                  (128, 128, 64, 64 * 33 + 1, True)])
+def test_tc_sequence_segments(dk, dv, B, L, with_state):
+    """Few (batch, head) pairs and many chunks: the sequence is split over CTAs that replay
+    the state over the earlier chunks.  Outputs and the final state against the oracle."""
+    b, h = 1, 2
+    q, k, v = si.qkv(b, L, h, dk, dv, 90 + dk + B, "bf16")
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+    S0 = si.decode_state(b, h, dk, dv, 91, std=0.3) if with_state else None
+    pos0 = 321 if with_state else 0
+    ref, Sref, _ = oracle.recurrent(q, k, v, g, th, pos0, FLAGS, S0)
+    o, so = run_tc(q, k, v, g, th, B, pos0=pos0, state_in=S0, want_state=True)
+    e = err(o, ref)
+    print(f"segments dk={dk} dv={dv} B={B} L={L}: max|err|/rms = {e:.3e}")
+    assert e <= TOL_BF16
+    assert err(so, Sref) <= TOL_BF16
+
+
 @pytest.mark.parametrize("flags", [0, rn.F_XPOS, rn.F_SCALE_SQRT_D, rn.F_NORM_D, FLAGS])
 def test_tc_flag_combinations(flags):
     b, L, h, dk, dv, B = 1, 200, 4, 128, 64, 64
