@@ -125,9 +125,11 @@ RETNET_API retnet_status_t retnet_retention_parallel(const void* q, const void* 
  *   z_in/z_out: device fp32 [batch][heads][d_k], the key-sum state (gamma z + k) that the
  *              R~ row sum needs across calls; read/written only with RETNET_F_NORM_R; NULL
  *              means zeros / not written.
- * Kernels: bf16 q, k, v with d_k in {64, 128, 256}, d_v a multiple of 64 (<= 512) and
- * chunk in {64, 128, 256, 512} run on the tcgen05 tensor-core kernel; every other case runs
- * on the fp32 CUDA-core kernel.
+ * Kernels: bf16 q, k, v without RETNET_F_NORM_R, with d_k in {64, 128, 256}, d_v a multiple
+ * of 64, chunk in {64, 128, 256, 512}, 16-byte aligned tensors and gamma^T >= 2^-12 for every
+ * head (T = 64, or 128 when d_k <= 128 and chunk >= 128: the sub-block the kernel scales its
+ * fp16 operands within) run on the tcgen05 tensor-core kernel; every other case runs on the
+ * fp32 CUDA-core kernel.  retnet_chunkwise_kernel reports which one a call takes.
  */
 RETNET_API retnet_status_t retnet_retention_chunkwise(const void* q, const void* k, const void* v, void* o,
                                            retnet_dims_t dims, retnet_dtype_t in_dtype,
