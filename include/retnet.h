@@ -58,6 +58,7 @@
 #ifndef RETNET_H
 #define RETNET_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 /* Exported symbols of libretnet.so (the library is built with hidden default visibility). */
@@ -137,6 +138,41 @@ RETNET_API retnet_status_t retnet_retention_chunkwise(const void* q, const void*
                                            const float* theta, int64_t pos0, uint32_t flags,
                                            int64_t chunk, const float* state_in, float* state_out,
                                            const float* z_in, float* z_out, void* stream);
+
+/*
+ * retnet_retention_chunkwise with a caller-owned device workspace.  The result is the same
+ * function of the same arguments (§2.4 read as a scan over chunks: R_i = gamma^B R_{i-1} +
+ * K_[i]^T (V_[i] (.) zeta) is associative, so the chunks may be cut into consecutive segments
+ * whose own states are combined by R = gamma^len R + W).  When the tensor-core kernel runs
+ * with fewer (batch, head, d_v slice) units than SMs, it cuts the sequence into up to four
+ * segments: a first launch computes the states of the earlier segments (cut again into
+ * sub-segments, up to six states) in parallel, a second produces every segment's outputs
+ * starting from state_in carried over the earlier sub-segments.  Without a workspace the same split runs as one launch in which each later segment
+ * first replays the earlier chunks' state.
+ *   workspace: device memory, 16-byte aligned, workspace_bytes long, not overlapping any other
+ *              argument; its contents on entry are irrelevant and are overwritten (the
+ *              sub-segment states, fp32).  NULL (or smaller than one state,
+ *              batch * heads * d_k * d_v * 4 bytes) means no workspace.  retnet_chunkwise_workspace_size gives the size that allows the
+ *              full split.  The workspace is in use until the call's work on `stream`
+ *              completes; two calls sharing one workspace must be ordered on the device.
+ * Other arguments, errors and kernels as retnet_retention_chunkwise; a misaligned workspace
+ * is RETNET_ERR_BAD_PARAM.
+ */
+RETNET_API retnet_status_t retnet_retention_chunkwise_ws(const void* q, const void* k, const void* v, void* o,
+                                              retnet_dims_t dims, retnet_dtype_t in_dtype,
+                                              retnet_dtype_t out_dtype, const float* gamma,
+                                              const float* theta, int64_t pos0, uint32_t flags,
+                                              int64_t chunk, const float* state_in, float* state_out,
+                                              const float* z_in, float* z_out, void* workspace,
+                                              size_t workspace_bytes, void* stream);
+
+/*
+ * Workspace size (bytes) that lets retnet_retention_chunkwise_ws use its full segment split
+ * for these dimensions: 6 * batch * heads * d_k * d_v * sizeof(float) (room for the states of
+ * six pre-pass sub-segments).  Host-only; no device
+ * access.  RETNET_ERR_NULL_PTR without `bytes`, RETNET_ERR_BAD_SHAPE for negative sizes.
+ */
+RETNET_API retnet_status_t retnet_chunkwise_workspace_size(retnet_dims_t dims, size_t* bytes);
 
 /*
  * One recurrent decode step (§2.2) for a whole batch: for the token at absolute position

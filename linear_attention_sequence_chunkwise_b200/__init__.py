@@ -30,9 +30,9 @@ BF16 = 1
 
 STATUS = {0: "RETNET_OK", 1: "RETNET_ERR_NULL_PTR", 2: "RETNET_ERR_BAD_SHAPE", 3: "RETNET_ERR_BAD_DTYPE",
           4: "RETNET_ERR_BAD_PARAM", 5: "RETNET_ERR_UNSUPPORTED", 6: "RETNET_ERR_CUDA"}
-EXPORTS = ("retnet_retention_parallel", "retnet_retention_chunkwise", "retnet_retention_step",
-           "retnet_msr_epilogue", "retnet_chunkwise_kernel", "retnet_debug_wait_timeouts", "retnet_status_string",
-           "retnet_version")
+EXPORTS = ("retnet_retention_parallel", "retnet_retention_chunkwise", "retnet_retention_chunkwise_ws",
+           "retnet_chunkwise_workspace_size", "retnet_retention_step", "retnet_msr_epilogue",
+           "retnet_chunkwise_kernel", "retnet_debug_wait_timeouts", "retnet_status_string", "retnet_version")
 
 
 class RetnetError(RuntimeError):
@@ -67,11 +67,15 @@ def load(path: str = None):
     lib.retnet_retention_parallel.argtypes = [_vp, _vp, _vp, _vp, Dims, _i32, _i32, _fp, _fp, _i64, _u32, _vp]
     lib.retnet_retention_chunkwise.argtypes = [_vp, _vp, _vp, _vp, Dims, _i32, _i32, _fp, _fp, _i64, _u32, _i64,
                                                _vp, _vp, _vp, _vp, _vp]
+    lib.retnet_retention_chunkwise_ws.argtypes = [_vp, _vp, _vp, _vp, Dims, _i32, _i32, _fp, _fp, _i64, _u32,
+                                                  _i64, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+    lib.retnet_chunkwise_workspace_size.argtypes = [Dims, ctypes.POINTER(ctypes.c_size_t)]
+    lib.retnet_chunkwise_workspace_size.restype = _i32
     lib.retnet_retention_step.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _fp,
                                           _fp, _i64, _u32, _vp]
     lib.retnet_msr_epilogue.argtypes = [_vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_float, _i32, _i32, _vp]
-    for name in ("retnet_retention_parallel", "retnet_retention_chunkwise", "retnet_retention_step",
-                 "retnet_msr_epilogue"):
+    for name in ("retnet_retention_parallel", "retnet_retention_chunkwise", "retnet_retention_chunkwise_ws",
+                 "retnet_retention_step", "retnet_msr_epilogue"):
         getattr(lib, name).restype = _i32
     lib.retnet_chunkwise_kernel.argtypes = [Dims, _i32, _u32, _i64, _fp]
     lib.retnet_chunkwise_kernel.restype = _i32
@@ -163,6 +167,40 @@ def retnet_retention_parallel(q, k, v, o, gamma, theta=None, pos0=0, flags=F_ALL
     _check(load().retnet_retention_parallel(_ptr(q), _ptr(k), _ptr(v), _ptr(o), Dims(b, L, h, dk, dv),
                                             _dtype_code(q), _dtype_code(o), _fptr(g), _fptr(th), int(pos0),
                                             int(flags), _stream(stream)))
+
+
+def _chunkwise_args(q, k, v, o, gamma, theta, state_in, state_out, z_in, z_out):
+    _require_cuda(q, k, v, o, state_in, state_out, z_in, z_out)
+    b, L, h, dk = q.shape
+    dv = v.shape[-1]
+    if tuple(k.shape) != (b, L, h, dk) or tuple(v.shape) != (b, L, h, dv) or tuple(o.shape) != (b, L, h, dv):
+        raise ValueError("shape mismatch between q, k, v, o")
+    for s in (state_in, state_out):
+        if s is not None and not isinstance(s, int) and tuple(s.shape) != (b, h, dk, dv):
+            raise ValueError("state must be (batch, heads, d_k, d_v) float32")
+    for z in (z_in, z_out):
+        if z is not None and not isinstance(z, int) and tuple(z.shape) != (b, h, dk):
+            raise ValueError("z must be (batch, heads, d_k) float32")
+    return Dims(b, L, h, dk, dv), _host_f32(gamma, h), _host_f32(theta, dk // 2)
+
+
+def retnet_chunkwise_workspace_size(dims) -> int:
+    """Bytes of workspace for retnet_retention_chunkwise_ws; dims = (batch, seqlen, heads, d_k, d_v)."""
+    out = ctypes.c_size_t(0)
+    _check(load().retnet_chunkwise_workspace_size(Dims(*[int(x) for x in dims]), ctypes.byref(out)))
+    return out.value
+
+
+def retnet_retention_chunkwise_ws(q, k, v, o, gamma, theta=None, pos0=0, flags=F_ALL, chunk=64, state_in=None,
+                                  state_out=None, z_in=None, z_out=None, workspace=None, stream=None):
+    """Chunkwise form with a caller-owned device workspace (a uint8 CUDA tensor, or None)."""
+    d, g, th = _chunkwise_args(q, k, v, o, gamma, theta, state_in, state_out, z_in, z_out)
+    _require_cuda(workspace)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().retnet_retention_chunkwise_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(o), d, _dtype_code(q),
+                                                _dtype_code(o), _fptr(g), _fptr(th), int(pos0), int(flags),
+                                                int(chunk), _ptr(state_in), _ptr(state_out), _ptr(z_in),
+                                                _ptr(z_out), _ptr(workspace), ws_bytes, _stream(stream)))
 
 
 def retnet_retention_chunkwise(q, k, v, o, gamma, theta=None, pos0=0, flags=F_ALL, chunk=64, state_in=None,

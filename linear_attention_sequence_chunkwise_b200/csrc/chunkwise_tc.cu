@@ -44,6 +44,8 @@ constexpr int kWarpTma = 8;
 constexpr int kWarpMma = 9;
 constexpr int kDVS = 64;  // d_v slice per CTA
 
+constexpr int kMaxSub = 6;  // pre-pass states of the two-pass form (workspace capacity)
+
 struct TcArgs {
   void* o;
   const float* state_in;
@@ -60,6 +62,22 @@ struct TcArgs {
   int n_seg;
   int seg_lo[4];
   int seg_hi[4];
+  // Two-pass form: the pre-pass computes the state of each sub-segment j, chunks
+  // [sub_lo[j], sub_hi[j]) from a zero start, into ws (fp32 [j][batch][head][d_k][d_v]);
+  // output segment s starts from state_in carried over the first sub_before[s] of them.
+  int n_sub;
+  int sub_lo[kMaxSub];
+  int sub_hi[kMaxSub];
+  int sub_before[4];
+  float* ws;
+};
+
+// Sequence-segment modes of the pipelined kernel.
+enum : int {
+  SEG_NONE = 0,     // one CTA walks the whole sequence of its slice
+  SEG_REPLAY = 1,   // segment s replays the state over chunks [0, lo_s), then outputs [lo_s, hi_s)
+  SEG_FROM_WS = 2,  // segment s starts from state_in and the states of segments < s (workspace)
+  SEG_STATE = 3     // pre-pass: segment s accumulates its own state (from zero) into the workspace
 };
 
 template <int DK, int T>
@@ -663,22 +681,25 @@ __device__ __forceinline__ float row_factor_f32(float gamma, float sqrt_dk_inv, 
 // for chunk i < c_hi, for row block u < nbw_i, for column block w <= u  (nbw_i = ceil(b'_i / T)).
 // Chunks below c_lo are state replay only: just their last row block (u = nbw_i - 1), whose
 // units carry the state increments.
-template <int T, bool SEG>
+template <int T, int SM>
 struct UnitIter {
+  static constexpr bool SEG = SM != SEG_NONE;
+  static constexpr bool PRE = SM == SEG_REPLAY || SM == SEG_STATE;  // some chunks update the state only
   int L, nb;         // sequence length, sub-blocks per full chunk
-  int lo, hi;        // first chunk with outputs, end of the CTA's chunks (SEG only)
+  int lo, hi;        // first output chunk (chunks below only update the state), end (SEG only)
   int i, u, w;       // current unit
   int nbw, bl;       // sub-blocks and length of chunk i
   int k;             // unit sequence number (stages, TMA, conversion)
-  int kf_;           // sequence number among output units (SEG only; equals k otherwise)
+  int kf_;           // sequence number among output units (PRE only; equals k otherwise)
   int rb;            // row-block sequence number among output units (O/X buffers)
   int dr;            // sequence number of state-increment units (u == nbw - 1)
-  __device__ void start(int L_, int nb_, int c_lo_, int c_hi_) {
+  __device__ void start(int L_, int nb_, int first, int c_lo_, int c_hi_) {
     L = L_;
     nb = nb_;
     lo = c_lo_;
     hi = c_hi_;
-    i = 0; k = 0; kf_ = 0; rb = 0; dr = 0;
+    i = SEG ? first : 0;
+    k = 0; kf_ = 0; rb = 0; dr = 0;
     if (valid()) set_chunk();
   }
   __device__ void set_chunk() {
@@ -688,14 +709,14 @@ struct UnitIter {
     w = 0;
   }
   __device__ bool valid() const { return (!SEG || i < hi) && i * nb * T < L; }
-  __device__ bool pre() const { return SEG && i < lo; }     // state replay only
-  __device__ int kf() const { return SEG ? kf_ : k; }
+  __device__ bool pre() const { return PRE && i < lo; }     // state update only
+  __device__ int kf() const { return PRE ? kf_ : k; }
   __device__ bool last_row() const { return u == nbw - 1; }  // this unit carries a state increment
   __device__ bool rb_done() const { return w == u; }         // last unit of its row block
   __device__ int t0() const { return i * nb * T; }          // chunk start (token)
   __device__ void next() {
     if (last_row()) ++dr;
-    if (SEG && !pre()) ++kf_;
+    if (PRE && !pre()) ++kf_;
     ++k;
     if (w < u) { ++w; return; }
     if (!pre()) ++rb;
@@ -771,13 +792,14 @@ struct UnitConverter {
 
   // In place: q -> gamma^(r+1) rot(q), k -> gamma^(T-1-r) rot(k) as fp16 (r local); v -> fp16.
   // WITH_Q = false (state replay) leaves the Q tile alone.
+  // zmul multiplies the K row scales (the state pre-pass decays K to its segment's end).
   template <bool WITH_Q>
   __device__ void convert(uint32_t sq, uint32_t sk, uint32_t sv, const float2* bq, const float2* bk, bool xpos,
-                          float log2g) const {
+                          float log2g, float zmul = 1.f) const {
     const uint32_t box = (cs / 8) * T * 128;
     const uint32_t chunk = cs % 8;
     const float xstep = decay_pow(log2g, RS), zstep = exp2f(-static_cast<float>(RS) * log2g);
-    const float xi0 = decay_pow(log2g, r0 + 1), zeta0 = decay_pow(log2g, T - 1 - r0);
+    const float xi0 = decay_pow(log2g, r0 + 1), zeta0 = decay_pow(log2g, T - 1 - r0) * zmul;
     float2 Fq[4], Fk[4], Zq[4], Zk[4];
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj) {
@@ -836,11 +858,12 @@ struct UnitConverter {
   }
 };
 
-template <int DK, int T, int DVS, bool SEG, typename Tout>
+template <int DK, int T, int DVS, int SM, typename Tout>
 __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
     tc_chunkwise_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v, TcArgs a, HeadParams hp) {
   using C = Cfg3<DK, T, DVS>;
+  constexpr bool SEG = SM != SEG_NONE;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_addr(smem_raw);
   const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
@@ -849,22 +872,72 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int n_dvb = a.dv / DVS;
   const int dvb = SEG ? blockIdx.x % n_dvb : blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  // Output chunks [c_lo, c_hi); [0, c_lo) replays the state.  Without segments the bounds are
-  // compile-time constants and every replay branch folds away.
-  int c_lo = 0, c_hi = 0x7fffffff;
-  if constexpr (SEG) {
-    const int seg = blockIdx.x / n_dvb;
-    c_lo = a.seg_lo[0];
-    c_hi = a.seg_hi[0];
+  const float log2g = hp.log2g[h];
+  const int nb = a.nb;
+  // The CTA visits chunks [c_first, c_hi); those below c_lo only update the state (the replay
+  // of earlier segments, or the whole segment in the state pre-pass); outputs start at c_lo.
+  // Without segments the bounds are compile-time constants and every such branch folds away.
+  int seg = 0, s_lo = 0, s_hi = 0x7fffffff;
+  if constexpr (SM == SEG_STATE) {  // seg = the pre-pass sub-segment
+    seg = blockIdx.x / n_dvb;
+    s_lo = a.sub_lo[0];
+    s_hi = a.sub_hi[0];
+#pragma unroll
+    for (int i = 1; i < kMaxSub; ++i)
+      if (seg == i) {
+        s_lo = a.sub_lo[i];
+        s_hi = a.sub_hi[i];
+      }
+  } else if constexpr (SEG) {
+    seg = blockIdx.x / n_dvb;
+    s_lo = a.seg_lo[0];
+    s_hi = a.seg_hi[0];
 #pragma unroll
     for (int i = 1; i < 4; ++i)  // (a constant-index select keeps the kernel parameters in place)
       if (seg == i) {
-        c_lo = a.seg_lo[i];
-        c_hi = a.seg_hi[i];
+        s_lo = a.seg_lo[i];
+        s_hi = a.seg_hi[i];
       }
   }
-  const float log2g = hp.log2g[h];
-  const int nb = a.nb;
+  const int c_first = (SM == SEG_REPLAY) ? 0 : s_lo;
+  const int c_lo = (SM == SEG_STATE) ? s_hi : s_lo;
+  const int c_hi = s_hi;
+  // Start state of a two-pass output segment: state_in carried over the earlier segments,
+  // R = gamma^len_j R + W_j (row dk, columns [col, col + n) of the slice).
+  auto start_state = [&](int dk, int col, int n, float* R) {
+    const int64_t bh = static_cast<int64_t>(b) * a.heads + h;
+    for (int c = 0; c < n; ++c) R[c] = 0.f;
+    if (a.state_in) {
+      const float* src = a.state_in + static_cast<size_t>(bh) * DK * a.dv + col + static_cast<size_t>(dk) * a.dv;
+      for (int c4 = 0; c4 < n / 4; ++c4) {
+        const float4 x = *reinterpret_cast<const float4*>(src + 4 * c4);
+        R[4 * c4] = x.x; R[4 * c4 + 1] = x.y; R[4 * c4 + 2] = x.z; R[4 * c4 + 3] = x.w;
+      }
+    }
+    if constexpr (SM == SEG_FROM_WS) {
+      int n_before = a.sub_before[0];
+#pragma unroll
+      for (int t = 1; t < 4; ++t)  // constant-index selects, as above
+        if (t == seg) n_before = a.sub_before[t];
+      for (int j = 0; j < n_before; ++j) {
+        int chunks_j = 0;
+#pragma unroll
+        for (int t = 0; t < kMaxSub; ++t)
+          if (t == j) chunks_j = a.sub_hi[t] - a.sub_lo[t];
+        const int len_j = chunks_j * nb * T;
+        const float gl = exp2f(static_cast<float>(len_j) * log2g);
+        const size_t plane = static_cast<size_t>(gridDim.z) * a.heads * DK * a.dv;
+        const float* w = a.ws + j * plane + static_cast<size_t>(bh) * DK * a.dv + col + static_cast<size_t>(dk) * a.dv;
+        for (int c4 = 0; c4 < n / 4; ++c4) {
+          const float4 x = *reinterpret_cast<const float4*>(w + 4 * c4);
+          R[4 * c4] = fmaf(gl, R[4 * c4], x.x);
+          R[4 * c4 + 1] = fmaf(gl, R[4 * c4 + 1], x.y);
+          R[4 * c4 + 2] = fmaf(gl, R[4 * c4 + 2], x.z);
+          R[4 * c4 + 3] = fmaf(gl, R[4 * c4 + 3], x.w);
+        }
+      }
+    }
+  };
   const float sd = rsqrtf(static_cast<float>(DK));  // carried by P and the fp16 state copy
 
   const uint32_t sP0 = sbase + C::NS * C::STAGE;
@@ -920,8 +993,8 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int issued[4] = {0, 0, 0, 0};
-      UnitIter<T, SEG> it;
-      for (it.start(a.L, nb, c_lo, c_hi); it.valid(); it.next()) {
+      UnitIter<T, SM> it;
+      for (it.start(a.L, nb, c_first, c_lo, c_hi); it.valid(); it.next()) {
         const int s = it.k % C::NS;
         if (it.k >= C::NS && !mbar_wait(bar(Q_STAGE_EMPTY + s), ((it.k / C::NS) - 1) & 1)) break;
         const bool with_q = !it.pre();  // state replay needs K and V only
@@ -955,7 +1028,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
       // has a non-blocking readiness test.  The issuer takes whichever group is ready -- X and P
       // of the oldest unit first, F at most LA units ahead -- so a late conversion of a later
       // unit never holds back the output (and the stage release) of an earlier one.
-      auto f_ready = [&](const UnitIter<T, SEG>& f) -> bool {
+      auto f_ready = [&](const UnitIter<T, SM>& f) -> bool {
         if (!mbar_test(bar(Q_CONV_FULL + f.k % C::NS), (f.k / C::NS) & 1)) return false;
         if (!f.pre() && f.kf() >= C::SBUF &&
             !mbar_test(bar(Q_S_FREE + (f.kf() % C::SBUF)), ((f.kf() - C::SBUF) / C::SBUF) & 1))
@@ -970,7 +1043,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
         }
         return true;
       };
-      auto f_issue = [&](const UnitIter<T, SEG>& f) {
+      auto f_issue = [&](const UnitIter<T, SM>& f) {
         const int s = f.k % C::NS;
         tc_fence_after();
         if (!f.pre()) {
@@ -993,12 +1066,12 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
         }
         if (f.pre()) mma_commit(bar(Q_STAGE_EMPTY + s));  // a replay unit has no P V
       };
-      auto x_ready = [&](const UnitIter<T, SEG>& q) -> bool {
+      auto x_ready = [&](const UnitIter<T, SM>& q) -> bool {
         const int ri = q.i - c_lo;  // fp16 state copies are written for output chunks only
         if (!mbar_test(bar(Q_R16_FULL + (ri % C::RBUF)), (ri / C::RBUF) & 1)) return false;
         return q.rb < 2 || mbar_test(bar(Q_O_FREE + (q.rb & 1)), ((q.rb - 2) >> 1) & 1);
       };
-      auto x_issue = [&](const UnitIter<T, SEG>& q) {
+      auto x_issue = [&](const UnitIter<T, SM>& q) {
         const int s = q.k % C::NS;
         tc_fence_after();
         const uint32_t tO = tmem + C::COL_O + (q.rb & 1) * DVS;
@@ -1010,10 +1083,10 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
           mma_f16_ss(tX, dq + kstep(kk), dr + static_cast<uint64_t>((kk * 2048) >> 4), ID_X, kk > 0);
         if (q.last_row()) mma_commit(bar(Q_R16_FREE + (ri % C::RBUF)));
       };
-      auto p_ready = [&](const UnitIter<T, SEG>& q) -> bool {
+      auto p_ready = [&](const UnitIter<T, SM>& q) -> bool {
         return mbar_test(bar(Q_P_FULL + (q.kf() % C::PBUF)), (q.kf() / C::PBUF) & 1);
       };
-      auto p_issue = [&](const UnitIter<T, SEG>& q) {
+      auto p_issue = [&](const UnitIter<T, SM>& q) {
         const int s = q.k % C::NS;
         tc_fence_after();
         const uint32_t tO = tmem + C::COL_O + (q.rb & 1) * DVS;
@@ -1026,11 +1099,32 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
         if (q.rb_done()) mma_commit(bar(Q_O_FULL + (q.rb & 1)));
         mma_commit(bar(Q_STAGE_EMPTY + s));
       };
+      if constexpr (SM == SEG_STATE) {
+        // State pre-pass: every increment Kz'^T V accumulates into one tensor-memory tile
+        // (Kz' carries the decay to the segment's end), committed once at the end.
+        UnitIter<T, SM> f;
+        bool first = true;
+        for (f.start(a.L, nb, c_first, c_lo, c_hi); f.valid(); f.next()) {
+          const int s = f.k % C::NS;
+          if (!mbar_wait(bar(Q_CONV_FULL + s), (f.k / C::NS) & 1)) break;
+          tc_fence_after();
+          const uint64_t dkm = sdesc_sw128(sK(s), T * 128, 1024), dv = sdesc_sw128(sV(s), T * 128, 1024);
+#pragma unroll
+          for (int blk = 0; blk < C::RBLK; ++blk)
+#pragma unroll
+            for (int ks = 0; ks < T / 16; ++ks)
+              mma_f16_ss(tmem + C::COL_DR + blk * DVS, dkm + static_cast<uint64_t>((blk * 2 * T * 128 + ks * 2048) >> 4),
+                         dv + static_cast<uint64_t>((ks * 2048) >> 4), ID_R, (first && ks == 0) ? 0u : 1u);
+          first = false;
+          mma_commit(bar(Q_STAGE_EMPTY + s));
+        }
+        mma_commit(bar(Q_DR_FULL + 0));
+      }
       constexpr int LA = 2;  // F of unit f only while f <= q + LA (q = oldest unit with P pending)
-      UnitIter<T, SEG> f, q;
-      f.start(a.L, nb, c_lo, c_hi);
-      q.start(a.L, nb, c_lo, c_hi);
-      while (q.valid() && q.pre()) q.next();  // q walks output units only
+      UnitIter<T, SM> f, q;
+      f.start(a.L, nb, c_first, c_lo, c_hi);
+      q.start(a.L, nb, c_first, c_lo, c_hi);
+      while (q.valid() && q.pre()) q.next();  // q walks output units only (none in the pre-pass)
       bool x_done = false;
       long long idle_since = clock64();
       while (q.valid()) {
@@ -1069,8 +1163,8 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
     cv.init(threadIdx.x - 32 * C::WARP_CONV0, nb, hp);
     const bool xpos = (a.flags & RETNET_F_XPOS) != 0;
     bool ok = true;
-    UnitIter<T, SEG> it;
-    for (it.start(a.L, nb, c_lo, c_hi); ok && it.valid(); it.next()) {
+    UnitIter<T, SM> it;
+    for (it.start(a.L, nb, c_first, c_lo, c_hi); ok && it.valid(); it.next()) {
       const int s = it.k % C::NS;
       float2* tq = tab + (it.k & 1) * DK;
       float2* tk = tq + DK / 2;
@@ -1081,16 +1175,48 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
       ok = mbar_wait(bar(Q_TAB + (it.k & 1)), (it.k >> 1) & 1);
       if (ok) ok = mbar_wait(bar(Q_TMA_FULL + s), (it.k / C::NS) & 1);
       if (!ok) break;
-      if (it.pre())
+      if constexpr (SM == SEG_STATE) {
+        // K of column block w decays to the segment's end E: gamma^(E - 1 - t) in all
+        const int e_tok = min(c_hi * nb * T, a.L), blk_end = it.t0() + (it.w + 1) * T;
+        cv.template convert<false>(sQ(s), sK(s), sV(s), tq, tk, xpos, log2g,
+                                   exp2f(static_cast<float>(e_tok - blk_end) * log2g));
+      } else if (SM == SEG_REPLAY && it.pre()) {
         cv.template convert<false>(sQ(s), sK(s), sV(s), tq, tk, xpos, log2g);
-      else
+      } else {
         cv.template convert<true>(sQ(s), sK(s), sV(s), tq, tk, xpos, log2g);
+      }
       fence_proxy_async_smem();
       mbar_arrive(bar(Q_CONV_FULL + s));
     }
   } else if (warp >= C::WARP_S0) {
     // ------------------------------------------------------------------ state group
-    if constexpr (C::RTM) {
+    if constexpr (SM == SEG_STATE) {
+      // State pre-pass: once the last increment has landed, the accumulated segment state
+      // (thread = one d_k row, all DVS columns) goes to the workspace.
+      const int blk = (warp - C::WARP_S0) / 4;
+      const uint32_t lane_off = static_cast<uint32_t>(32 * (warp % 4)) << 16;
+      const int dk = (DK == 64) ? (lane < 16 ? 16 * (warp % 4) + lane : -1) : blk * 128 + 32 * (warp % 4) + lane;
+      if (__all_sync(0xffffffffu, mbar_wait(bar(Q_DR_FULL + 0), 0))) {
+        tc_fence_after();
+        const size_t plane = static_cast<size_t>(gridDim.z) * a.heads * DK * a.dv;
+        float* dst = a.ws + seg * plane + (static_cast<size_t>(b) * a.heads + h) * DK * a.dv + dvb * DVS +
+                     static_cast<size_t>(dk < 0 ? 0 : dk) * a.dv;
+#pragma unroll 1
+        for (int grp = 0; grp < DVS / 32; ++grp) {
+          uint32_t u[2][16];
+          tmem_ld_wait(tmem + C::COL_DR + blk * DVS + 32 * grp + lane_off, u);
+          if (dk >= 0) {
+#pragma unroll
+            for (int c4 = 0; c4 < 8; ++c4)
+              *reinterpret_cast<float4*>(dst + 32 * grp + 4 * c4) =
+                  make_float4(__uint_as_float(u[(4 * c4) / 16][(4 * c4) % 16]),
+                              __uint_as_float(u[(4 * c4 + 1) / 16][(4 * c4 + 1) % 16]),
+                              __uint_as_float(u[(4 * c4 + 2) / 16][(4 * c4 + 2) % 16]),
+                              __uint_as_float(u[(4 * c4 + 3) / 16][(4 * c4 + 3) % 16]));
+          }
+        }
+      }
+    } else if constexpr (C::RTM) {
       // The fp32 state stays in tensor memory; thread = one d_k row (its TMEM lane), all
       // DVS columns.  Before chunk i's increment accumulates into it, the state group reads
       // R_{i-1}, writes its fp16 copy (output chunks only) and stores gamma^T R_{i-1} back.
@@ -1107,8 +1233,8 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
       constexpr int GW = 32;  // columns per batch
       bool ok = true;
       int last_dr = -1, last_bl = T;
-      UnitIter<T, SEG> it;
-      for (it.start(a.L, nb, c_lo, c_hi); ok && it.valid(); it.next()) {
+      UnitIter<T, SM> it;
+      for (it.start(a.L, nb, c_first, c_lo, c_hi); ok && it.valid(); it.next()) {
         const int d = it.dr;
         if (d > 0) {  // the previous increment has landed: the master holds R_{i-1}
           ok = __all_sync(0xffffffffu, mbar_wait(bar(Q_DR_FULL + 0), (d - 1) & 1));
@@ -1127,20 +1253,16 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
           uint32_t u[GW / 16][16];
           if (d > 0) {
             tmem_ld_wait(tR + GW * grp, u);
-          } else {  // chunk 0: the master starts from state_in (or zeros)
+          } else {  // first chunk: the master starts from state_in (carried over earlier segments)
+            float r0v[GW];
+            if (dk >= 0) {
+              start_state(dk, dvb * DVS + GW * grp, GW, r0v);
+            } else {
 #pragma unroll
-            for (int c = 0; c < GW; ++c) u[c / 16][c % 16] = 0u;
-            if (dk >= 0 && a.state_in) {
-              const float* src = a.state_in + static_cast<size_t>(bh) * DK * a.dv + dvb * DVS + GW * grp + dk * srow;
-#pragma unroll
-              for (int c4 = 0; c4 < GW / 4; ++c4) {
-                const float4 x = *reinterpret_cast<const float4*>(src + 4 * c4);
-                u[(4 * c4) / 16][(4 * c4) % 16] = __float_as_uint(x.x);
-                u[(4 * c4 + 1) / 16][(4 * c4 + 1) % 16] = __float_as_uint(x.y);
-                u[(4 * c4 + 2) / 16][(4 * c4 + 2) % 16] = __float_as_uint(x.z);
-                u[(4 * c4 + 3) / 16][(4 * c4 + 3) % 16] = __float_as_uint(x.w);
-              }
+              for (int c = 0; c < GW; ++c) r0v[c] = 0.f;
             }
+#pragma unroll
+            for (int c = 0; c < GW; ++c) u[c / 16][c % 16] = __float_as_uint(r0v[c]);
           }
           if (out && dk >= 0) {
             // fp16 copy (times 1/sqrt(d_k)) into box (column / 64), 16-byte slots of 8 columns
@@ -1203,14 +1325,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
       float R[RC];
   #pragma unroll
       for (int c = 0; c < RC; ++c) R[c] = 0.f;
-      if (dk >= 0 && a.state_in) {
-        const float* src = a.state_in + static_cast<size_t>(bh) * DK * a.dv + col0 + dk * srow;
-  #pragma unroll
-        for (int c4 = 0; c4 < RC / 4; ++c4) {
-          const float4 x = *reinterpret_cast<const float4*>(src + 4 * c4);
-          R[4 * c4] = x.x; R[4 * c4 + 1] = x.y; R[4 * c4 + 2] = x.z; R[4 * c4 + 3] = x.w;
-        }
-      }
+      if (dk >= 0) start_state(dk, col0, RC, R);
       auto put_r16 = [&](uint32_t base) {
         if (dk < 0) return;
         base += ch * DK * 128;
@@ -1221,14 +1336,14 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
                        pack_f16x2(sd * R[8 * c8 + 4], sd * R[8 * c8 + 5]),
                        pack_f16x2(sd * R[8 * c8 + 6], sd * R[8 * c8 + 7]));
       };
-      if (c_lo == 0) {  // otherwise written once the replay reaches the first output chunk
+      if (c_first == c_lo) {  // otherwise written once the replay reaches the first output chunk
         put_r16(sR(0));
         fence_proxy_async_smem();
         mbar_arrive(bar(Q_R16_FULL + 0));
       }
       bool ok = true;
-      UnitIter<T, SEG> it;
-      for (it.start(a.L, nb, c_lo, c_hi); ok && it.valid(); it.next()) {
+      UnitIter<T, SM> it;
+      for (it.start(a.L, nb, c_first, c_lo, c_hi); ok && it.valid(); it.next()) {
         if (!it.last_row()) continue;
         ok = __all_sync(0xffffffffu, mbar_wait(bar(Q_DR_FULL + (it.dr % C::DRBUF)), (it.dr / C::DRBUF) & 1));
         if (!ok) break;
@@ -1357,8 +1472,8 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
     };
     bool ok = true;
     int pend_rb = -1, pend_i = 0, pend_u = 0, pend_bl = 0;  // a finished row block awaiting its epilogue
-    UnitIter<T, SEG> it;
-    for (it.start(a.L, nb, c_lo, c_hi); ok && it.valid(); it.next()) {
+    UnitIter<T, SM> it;
+    for (it.start(a.L, nb, c_first, c_lo, c_hi); ok && it.valid(); it.next()) {
       if (it.pre()) continue;  // replay units have no scores
       const int k = it.kf();
       ok = __all_sync(0xffffffffu, mbar_wait(bar(Q_S_FULL + (k % C::SBUF)), (k / C::SBUF) & 1));
@@ -1480,14 +1595,24 @@ int sm_count() {
 // over chunks [0, lo_s) (K and V only: TMA, conversion, state increment), then produces the
 // outputs of [lo_s, hi_s).  A replayed chunk costs about kReplayCost of an output chunk, and
 // the boundaries equalise rho * lo_s + (hi_s - lo_s) across segments.
+// With a workspace (two passes) nothing is replayed: a pre-pass launch computes each
+// segment's own state in parallel and the segments split the chunks evenly (rho = 0).
 constexpr double kReplayCost = 0.45;
-void plan_segments(TcArgs& a, int64_t ctas, int sms) {
+void plan_segments(TcArgs& a, int64_t ctas, int sms, double rho, int max_seg) {
   const int n = a.n_chunks;
   int n_seg = (ctas > 0 && sms > 0) ? static_cast<int>(sms / ctas) : 1;
-  n_seg = std::min(n_seg, 4);
+  n_seg = std::min(n_seg, max_seg);
   n_seg = std::min(n_seg, n / 4);  // at least four chunks a segment
   if (n_seg < 2) return;
-  const double rho = kReplayCost, keep = 1.0 - rho;
+  if (rho <= 0.0) {
+    for (int s = 0; s < n_seg; ++s) {
+      a.seg_lo[s] = static_cast<int>(static_cast<int64_t>(n) * s / n_seg);
+      a.seg_hi[s] = static_cast<int>(static_cast<int64_t>(n) * (s + 1) / n_seg);
+    }
+    a.n_seg = n_seg;
+    return;
+  }
+  const double keep = 1.0 - rho;
   const double cost = n * rho / (1.0 - std::pow(keep, n_seg));
   double x = 0.0;
   int prev = 0;
@@ -1505,6 +1630,7 @@ void plan_segments(TcArgs& a, int64_t ctas, int sms) {
 
 TcArgs make_args(const RetentionCall& c, int n_chunks, int nb) {
   TcArgs a;
+  a.ws = nullptr;
   a.o = c.o;
   a.state_in = c.state_in;
   a.state_out = c.state_out;
@@ -1516,7 +1642,9 @@ TcArgs make_args(const RetentionCall& c, int n_chunks, int nb) {
   a.flags = c.flags;
   a.nb = nb;
   a.n_seg = 1;
-  for (int s = 0; s < 4; ++s) a.seg_lo[s] = a.seg_hi[s] = 0;
+  a.n_sub = 0;
+  for (int s = 0; s < 4; ++s) a.seg_lo[s] = a.seg_hi[s] = a.sub_before[s] = 0;
+  for (int j = 0; j < kMaxSub; ++j) a.sub_lo[j] = a.sub_hi[j] = 0;
   a.seg_hi[0] = n_chunks;
   return a;
 }
@@ -1543,15 +1671,47 @@ cudaError_t launch_pipe(const RetentionCall& c, const HeadParams& hp, cudaStream
   const TcArgs a = make_args(c, static_cast<int>((c.dims.seqlen + c.chunk - 1) / c.chunk), nb);
   if (Cf::XBUF == 0 && nb != 1) return cudaErrorInvalidValue;
   TcArgs as = a;
-  dim3 grid = tc_grid(c.dims, DVS);
-  plan_segments(as, static_cast<int64_t>(grid.x) * grid.y * grid.z, sm_count());
-  grid.x *= as.n_seg;
-  auto kern = as.n_seg > 1 ? tc_chunkwise_pipe_kernel<DK, T, DVS, true, Tout>
-                           : tc_chunkwise_pipe_kernel<DK, T, DVS, false, Tout>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM);
+  const dim3 grid = tc_grid(c.dims, DVS);
+  const int64_t ctas = static_cast<int64_t>(grid.x) * grid.y * grid.z;
+  // The two-pass form keeps one state per pre-pass sub-segment in the caller's workspace.
+  const size_t state_bytes = sizeof(float) * static_cast<size_t>(c.dims.batch * c.dims.heads * c.dims.d_k * c.dims.d_v);
+  const int max_states = c.ws ? static_cast<int>(std::min<size_t>(c.ws_bytes / state_bytes, kMaxSub)) : 0;
+  const int sms = sm_count();
+  if (max_states >= 1) {
+    plan_segments(as, ctas, sms, 0.0, std::min(4, max_states + 1));
+  } else {
+    plan_segments(as, ctas, sms, kReplayCost, 4);
+  }
+  auto run = [&](auto kern, unsigned nx) -> cudaError_t {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM);
+    if (e != cudaSuccess) return e;
+    kern<<<dim3(grid.x * nx, grid.y, grid.z), Cf::THREADS, Cf::SMEM, s>>>(mq, mk, mv, as, hp);
+    return cudaGetLastError();
+  };
+  if (as.n_seg < 2) return run(tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_NONE, Tout>, 1);
+  if (max_states < 1) return run(tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_REPLAY, Tout>, as.n_seg);
+  // Pre-pass: each of the first n_seg - 1 segments split into n_split sub-segments, as many
+  // as the SMs, the workspace and two chunks a sub-segment allow.
+  const int n_pre = as.n_seg - 1;
+  int n_split = static_cast<int>(sms / (ctas * n_pre));
+  n_split = std::min(n_split, max_states / n_pre);
+  n_split = std::min(n_split, (as.seg_hi[0] - as.seg_lo[0]) / 2);
+  n_split = std::max(n_split, 1);
+  int j = 0;
+  for (int sg = 0; sg < as.n_seg; ++sg) {
+    as.sub_before[sg] = j;
+    if (sg == n_pre) break;
+    const int lo = as.seg_lo[sg], len = as.seg_hi[sg] - lo;
+    for (int p = 0; p < n_split; ++p, ++j) {
+      as.sub_lo[j] = lo + len * p / n_split;
+      as.sub_hi[j] = lo + len * (p + 1) / n_split;
+    }
+  }
+  as.n_sub = j;
+  as.ws = static_cast<float*>(c.ws);
+  const cudaError_t e = run(tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_STATE, Tout>, as.n_sub);
   if (e != cudaSuccess) return e;
-  kern<<<grid, Cf::THREADS, Cf::SMEM, s>>>(mq, mk, mv, as, hp);
-  return cudaGetLastError();
+  return run(tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_FROM_WS, Tout>, as.n_seg);
 }
 
 // Serial kernel: one chunk of B = T rows per step (chunk-relative scaled operands).

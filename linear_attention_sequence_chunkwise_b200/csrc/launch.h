@@ -23,6 +23,10 @@ struct RetentionCall {
   float* state_out;
   const float* z_in;
   float* z_out;
+  // Caller-owned device workspace for the two-pass sequence segments of the tensor-core
+  // kernel (segment states); nullptr = single-launch segments that replay the state.
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
 };
 
 // fp32 CUDA-core kernel: the parallel form (chunk >= seqlen, no state) and the chunkwise

@@ -98,20 +98,24 @@ retnet_status_t retnet_retention_parallel(const void* q, const void* k, const vo
   return from_cuda(launch_simt_retention(c, hp, static_cast<cudaStream_t>(stream)));
 }
 
-retnet_status_t retnet_retention_chunkwise(const void* q, const void* k, const void* v, void* o, retnet_dims_t dims,
-                                           retnet_dtype_t in_dtype, retnet_dtype_t out_dtype, const float* gamma,
-                                           const float* theta, int64_t pos0, uint32_t flags, int64_t chunk,
-                                           const float* state_in, float* state_out, const float* z_in,
-                                           float* z_out, void* stream) {
+namespace {
+retnet_status_t chunkwise_impl(const void* q, const void* k, const void* v, void* o, retnet_dims_t dims,
+                               retnet_dtype_t in_dtype, retnet_dtype_t out_dtype, const float* gamma,
+                               const float* theta, int64_t pos0, uint32_t flags, int64_t chunk,
+                               const float* state_in, float* state_out, const float* z_in, float* z_out,
+                               void* workspace, size_t workspace_bytes, void* stream) {
   retnet_status_t st = check_common(dims, in_dtype, out_dtype, pos0, flags, true);
   if (st != RETNET_OK) return st;
   if (chunk <= 0) return RETNET_ERR_BAD_PARAM;
   if (dims.seqlen > 0 && (!q || !k || !v || !o)) return RETNET_ERR_NULL_PTR;
+  if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 15u) != 0) return RETNET_ERR_BAD_PARAM;
   HeadParams hp;
   if ((st = fill_params(&hp, gamma, theta, dims.heads, dims.d_k, flags)) != RETNET_OK) return st;
   if ((st = check_device()) != RETNET_OK) return st;
   RetentionCall c{q, k, v, o, Dims{dims.batch, dims.seqlen, dims.heads, dims.d_k, dims.d_v}, in_dtype, out_dtype,
                   pos0, flags, chunk, true, state_in, state_out, z_in, z_out};
+  c.ws = workspace;
+  c.ws_bytes = workspace ? workspace_bytes : 0;
   if (dims.seqlen == 0) {
     // No tokens: the state passes through unchanged.
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -134,6 +138,35 @@ retnet_status_t retnet_retention_chunkwise(const void* q, const void* k, const v
     return from_cuda(launch_tc_chunkwise(c, hp, static_cast<cudaStream_t>(stream)));
   }
   return from_cuda(launch_simt_retention(c, hp, static_cast<cudaStream_t>(stream)));
+}
+}  // namespace
+
+retnet_status_t retnet_retention_chunkwise(const void* q, const void* k, const void* v, void* o, retnet_dims_t dims,
+                                           retnet_dtype_t in_dtype, retnet_dtype_t out_dtype, const float* gamma,
+                                           const float* theta, int64_t pos0, uint32_t flags, int64_t chunk,
+                                           const float* state_in, float* state_out, const float* z_in,
+                                           float* z_out, void* stream) {
+  return chunkwise_impl(q, k, v, o, dims, in_dtype, out_dtype, gamma, theta, pos0, flags, chunk, state_in, state_out,
+                        z_in, z_out, nullptr, 0, stream);
+}
+
+retnet_status_t retnet_retention_chunkwise_ws(const void* q, const void* k, const void* v, void* o,
+                                              retnet_dims_t dims, retnet_dtype_t in_dtype, retnet_dtype_t out_dtype,
+                                              const float* gamma, const float* theta, int64_t pos0, uint32_t flags,
+                                              int64_t chunk, const float* state_in, float* state_out,
+                                              const float* z_in, float* z_out, void* workspace,
+                                              size_t workspace_bytes, void* stream) {
+  return chunkwise_impl(q, k, v, o, dims, in_dtype, out_dtype, gamma, theta, pos0, flags, chunk, state_in, state_out,
+                        z_in, z_out, workspace, workspace_bytes, stream);
+}
+
+retnet_status_t retnet_chunkwise_workspace_size(retnet_dims_t dims, size_t* bytes) {
+  if (!bytes) return RETNET_ERR_NULL_PTR;
+  if (dims.batch < 0 || dims.seqlen < 0 || dims.heads < 0 || dims.d_k < 0 || dims.d_v < 0) return RETNET_ERR_BAD_SHAPE;
+  // Up to six pre-pass states, fp32 [6][batch][heads][d_k][d_v].
+  *bytes = 6 * sizeof(float) * static_cast<size_t>(dims.batch) * static_cast<size_t>(dims.heads) *
+           static_cast<size_t>(dims.d_k) * static_cast<size_t>(dims.d_v);
+  return RETNET_OK;
 }
 
 int retnet_chunkwise_kernel(retnet_dims_t dims, retnet_dtype_t in_dtype, uint32_t flags, int64_t chunk,

@@ -116,6 +116,27 @@ def test_chunkwise_and_step_validation(lib):
                                      None) == 4
 
 
+def test_chunkwise_workspace_entry_points(lib):
+    """Workspace size is the documented bound; the workspace variant validates like the plain call
+    and rejects a misaligned workspace before touching a device."""
+    assert rn.retnet_chunkwise_workspace_size((2, 100, 3, 128, 64)) == 6 * 2 * 3 * 128 * 64 * 4
+    assert rn.retnet_chunkwise_workspace_size((0, 0, 0, 0, 0)) == 0
+    out = ctypes.c_size_t(0)
+    assert lib.retnet_chunkwise_workspace_size(rn.Dims(1, 8, -2, 4, 4), ctypes.byref(out)) == 2
+    assert lib.retnet_chunkwise_workspace_size(rn.Dims(1, 8, 2, 4, 4), None) == 1
+    g = _gamma(2)
+    gp = g.ctypes.data_as(rn._fp)
+    d = rn.Dims(1, 8, 2, 4, 4)
+    # chunk <= 0, NULL o: as the plain call
+    assert lib.retnet_retention_chunkwise_ws(FAKE, FAKE, FAKE, FAKE, d, 0, 0, gp, None, 0, 0, 0, None, None, None,
+                                             None, FAKE, 4096, None) == 4
+    assert lib.retnet_retention_chunkwise_ws(FAKE, FAKE, FAKE, None, d, 0, 0, gp, None, 0, 0, 16, None, None, None,
+                                             None, FAKE, 4096, None) == 1
+    # misaligned workspace
+    assert lib.retnet_retention_chunkwise_ws(FAKE, FAKE, FAKE, FAKE, d, 0, 0, gp, None, 0, 0, 16, None, None, None,
+                                             None, FAKE + 8, 4096, None) == 4
+
+
 def test_epilogue_validation(lib):
     f = lib.retnet_msr_epilogue
     assert f(FAKE, FAKE, FAKE, 4, 2, 12, 1e-5, 0, 0, None) == 2          # d_v not a multiple of 8

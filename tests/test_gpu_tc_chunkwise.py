@@ -91,6 +91,56 @@ def test_tc_sequence_segments(dk, dv, B, L, with_state):
     assert err(so, Sref) <= TOL_BF16
 
 
+@pytest.mark.parametrize("dk,dv,B,L,with_state", [(128, 128, 64, 64 * 9 + 5, True), (128, 64, 64, 64 * 17, False),
+                                                  (256, 64, 128, 128 * 8 + 30, True), (64, 128, 256, 256 * 8, True),
+                                                  (128, 128, 64, 64 * 33 + 1, False)])
+def test_tc_two_pass_segments(dk, dv, B, L, with_state):
+    """The workspace form: segment states from a pre-pass launch, every segment's outputs from
+    state_in carried over the earlier ones.  Against the oracle, and the workspace sizes that
+    allow 2, 3 or 4 segments give the same bar."""
+    b, h = 1, 2
+    q, k, v = si.qkv(b, L, h, dk, dv, 95 + dk + B, "bf16")
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+    S0 = si.decode_state(b, h, dk, dv, 96, std=0.3) if with_state else None
+    pos0 = 555 if with_state else 0
+    ref, Sref, _ = oracle.recurrent(q, k, v, g, th, pos0, FLAGS, S0)
+    full = rn.retnet_chunkwise_workspace_size((b, L, h, dk, dv))
+    for nbytes in (full // 3, 2 * full // 3, full):
+        ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+        o = torch.empty(b, L, h, dv, device="cuda")
+        so = torch.empty(b, h, dk, dv, device="cuda")
+        rn.retnet_retention_chunkwise_ws(dev(q), dev(k), dev(v), o, g, th, pos0, FLAGS, B,
+                                         None if S0 is None else dev(S0), so, workspace=ws)
+        torch.cuda.synchronize()
+        e = err(o, ref)
+        print(f"two-pass dk={dk} dv={dv} B={B} L={L} ws={nbytes}: max|err|/rms = {e:.3e}")
+        assert e <= TOL_BF16
+        assert err(so, Sref) <= TOL_BF16
+
+
+def test_tc_two_pass_full_workload():
+    """b8/L2048/h8/d128/chunk 64 through the workspace form: within the bf16 bar of the plain
+    call's output (the two round the segment-boundary state differently) and of the oracle on
+    sampled (batch, head) pairs."""
+    b, L, h, dk, dv, B = 8, 2048, 8, 128, 128, 64
+    q, k, v = si.qkv(b, L, h, dk, dv, 97, "bf16")
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+    qd, kd, vd = dev(q), dev(k), dev(v)
+    o1 = torch.empty(b, L, h, dv, device="cuda")
+    o2 = torch.empty_like(o1)
+    rn.retnet_retention_chunkwise(qd, kd, vd, o1, g, th, 0, FLAGS, B)
+    ws = torch.empty(rn.retnet_chunkwise_workspace_size((b, L, h, dk, dv)), dtype=torch.uint8, device="cuda")
+    rn.retnet_retention_chunkwise_ws(qd, kd, vd, o2, g, th, 0, FLAGS, B, workspace=ws)
+    torch.cuda.synchronize()
+    rms = o1.float().pow(2).mean().sqrt().item()
+    assert (o1 - o2).abs().max().item() / rms <= TOL_BF16
+    for bb, hh in ((0, 0), (7, 7)):
+        sl = lambda x: x[bb:bb + 1, :, hh:hh + 1]
+        ref = oracle.recurrent(sl(q).contiguous(), sl(k).contiguous(), sl(v).contiguous(), g[hh:hh + 1], th, 0,
+                               FLAGS)[0]
+        assert err(sl(o2.cpu()).contiguous(), ref) <= TOL_BF16
+
+
 @pytest.mark.parametrize("flags", [0, rn.F_XPOS, rn.F_SCALE_SQRT_D, rn.F_NORM_D, FLAGS])
 def test_tc_flag_combinations(flags):
     b, L, h, dk, dv, B = 1, 200, 4, 128, 64, 64
