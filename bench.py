@@ -174,9 +174,10 @@ def make_main_inputs(cfg, device, rank):
     return sets
 
 
-def run_chunkwise(rn, s, cfg, gamma, theta, stream):
+def run_chunkwise(rn, s, cfg, gamma, theta, stream, ws):
+    """One step: the chunkwise call with its workspace (allocated once by the caller)."""
     q, k, v, o = s
-    rn.retnet_retention_chunkwise(q, k, v, o, gamma, theta, 0, FLAGS, cfg["chunk"], stream=stream)
+    rn.retnet_retention_chunkwise_ws(q, k, v, o, gamma, theta, 0, FLAGS, cfg["chunk"], workspace=ws, stream=stream)
 
 
 def time_steps(fn, steps, stream):
@@ -345,12 +346,14 @@ def main_ours(args):
     path = rn.retnet_chunkwise_kernel((b, L, h, dk), dv, rn.BF16, FLAGS, B, gamma)
     dtype_label = "f16" if path == 1 else "f32"  # arithmetic type of the kernel that runs
     sets = make_main_inputs(cfg, device, rank)
+    ws = torch.empty(rn.retnet_chunkwise_workspace_size((b, L, h, dk, dv)), dtype=torch.uint8, device=device)
+    launches = rn.retnet_chunkwise_launches((b, L, h, dk), dv, rn.BF16, FLAGS, B, gamma, ws.numel())
     stream = torch.cuda.current_stream()
     clocks = ClockSampler(torch.cuda.current_device())
     clocks.start()
 
     def step(i):
-        run_chunkwise(rn, sets[i % N_SETS], cfg, gamma, theta, stream)
+        run_chunkwise(rn, sets[i % N_SETS], cfg, gamma, theta, stream, ws)
 
     for i in range(args.warmup):
         step(i)
@@ -387,9 +390,13 @@ def main_ours(args):
         "tflops": tflops, "frac_bf16_peak": tflops * 1e12 / (peaks["bf16"] * 1e12),
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm"], "unit": "GB/s",
                      "frac": achieved_gbs / peaks["hbm"], "traffic": ncu_traffic("chunkwise_tc") if path == 1 else None,
-                     "peak_source": peaks["source"], "algorithmic_bytes_per_launch": alg_bytes,
-                     "launch_us": per_launch * 1e6},
-        "gpu_launches": args.steps,
+                     "peak_source": peaks["source"], "algorithmic_bytes_per_step": alg_bytes,
+                     "step_us": per_launch * 1e6,
+                     "scope": "one step = the chunkwise call: " + (
+                         "segment-state pre-pass + output pass (two launches)" if launches == 2 else "one launch")},
+        "gpu_launches": args.steps * launches,
+        "launches_per_step": launches,
+        "workspace_bytes": ws.numel(),
         "clocks": clk,
     }
     # e2e: host buffers in pinned memory, copies inside the timed region, through the same C call
@@ -406,7 +413,7 @@ def main_ours(args):
         dq.copy_(hq[0], non_blocking=True)
         dk_.copy_(hq[1], non_blocking=True)
         dv_.copy_(hq[2], non_blocking=True)
-        run_chunkwise(rn, (dq, dk_, dv_, do), cfg, gamma, theta, stream)
+        run_chunkwise(rn, (dq, dk_, dv_, do), cfg, gamma, theta, stream, ws)
         ho.copy_(do, non_blocking=True)
 
     if e2e_steps:

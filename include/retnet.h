@@ -211,6 +211,17 @@ RETNET_API int retnet_chunkwise_kernel(retnet_dims_t dims, retnet_dtype_t in_dty
                                        const float* gamma);
 
 /*
+ * Kernel launches retnet_retention_chunkwise_ws makes for these arguments on the current
+ * device (workspace_bytes = 0: retnet_retention_chunkwise): 0 without tokens, 1 for one
+ * launch, 2 when the two-pass sequence segments run (pre-pass + outputs); negative = the
+ * negated status the call would return.  Reads the device's SM count; no device memory
+ * is touched.  gamma: host float[heads].  Assumes 16-byte aligned buffers, as
+ * retnet_chunkwise_kernel does.
+ */
+RETNET_API int retnet_chunkwise_launches(retnet_dims_t dims, retnet_dtype_t in_dtype, uint32_t flags, int64_t chunk,
+                                         const float* gamma, size_t workspace_bytes);
+
+/*
  * Number of bounded waits that gave up inside the tensor-core kernel since the last clear
  * (a kernel that hits one abandons its output, releases what it holds and returns rather
  * than hang).  Synchronises with the device.  With clear != 0 the count is reset to 0.

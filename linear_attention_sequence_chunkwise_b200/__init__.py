@@ -32,7 +32,8 @@ STATUS = {0: "RETNET_OK", 1: "RETNET_ERR_NULL_PTR", 2: "RETNET_ERR_BAD_SHAPE", 3
           4: "RETNET_ERR_BAD_PARAM", 5: "RETNET_ERR_UNSUPPORTED", 6: "RETNET_ERR_CUDA"}
 EXPORTS = ("retnet_retention_parallel", "retnet_retention_chunkwise", "retnet_retention_chunkwise_ws",
            "retnet_chunkwise_workspace_size", "retnet_retention_step", "retnet_msr_epilogue",
-           "retnet_chunkwise_kernel", "retnet_debug_wait_timeouts", "retnet_status_string", "retnet_version")
+           "retnet_chunkwise_kernel", "retnet_chunkwise_launches", "retnet_debug_wait_timeouts",
+           "retnet_status_string", "retnet_version")
 
 
 class RetnetError(RuntimeError):
@@ -79,6 +80,8 @@ def load(path: str = None):
         getattr(lib, name).restype = _i32
     lib.retnet_chunkwise_kernel.argtypes = [Dims, _i32, _u32, _i64, _fp]
     lib.retnet_chunkwise_kernel.restype = _i32
+    lib.retnet_chunkwise_launches.argtypes = [Dims, _i32, _u32, _i64, _fp, ctypes.c_size_t]
+    lib.retnet_chunkwise_launches.restype = _i32
     lib.retnet_debug_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint), _i32]
     lib.retnet_debug_wait_timeouts.restype = _i32
     lib.retnet_status_string.argtypes = [_i32]
@@ -260,6 +263,15 @@ def retnet_chunkwise_kernel(shape_qk, d_v, in_dtype, flags, chunk, gamma):
     b, L, h, dk = shape_qk
     g = _host_f32(gamma, h)
     return load().retnet_chunkwise_kernel(Dims(b, L, h, dk, d_v), int(in_dtype), int(flags), int(chunk), _fptr(g))
+
+
+def retnet_chunkwise_launches(shape_qk, d_v, in_dtype, flags, chunk, gamma, workspace_bytes=0):
+    """Kernel launches of a chunkwise call on the current device (2 = two-pass segments),
+    negative (-status) if it would be rejected.  shape_qk = (batch, L, heads, d_k)."""
+    b, L, h, dk = shape_qk
+    g = _host_f32(gamma, h)
+    return load().retnet_chunkwise_launches(Dims(b, L, h, dk, d_v), int(in_dtype), int(flags), int(chunk), _fptr(g),
+                                            int(workspace_bytes))
 
 
 def retnet_debug_wait_timeouts(clear=True):

@@ -1576,6 +1576,21 @@ bool force_serial_kernel() {
 // Rows per unit of the pipelined kernel: 64 for d_k = 256 (shared memory), else min(B, 128).
 int pipe_tile_rows(int64_t d_k, int64_t chunk) { return d_k == 256 ? 64 : static_cast<int>(chunk < 128 ? chunk : 128); }
 
+// Segment plan of a call (see plan_segments); returns how many pre-pass states the caller's
+// workspace holds (0: no workspace, single-launch replay form).
+int sm_count();
+void plan_segments(TcArgs& a, int64_t ctas, int sms, double rho, int max_seg);
+constexpr double kReplayCost = 0.45;  // a replayed chunk, relative to an output chunk (measured)
+int plan_call(const RetentionCall& c, int64_t ctas, int sms, TcArgs& as) {
+  const size_t state_bytes = sizeof(float) * static_cast<size_t>(c.dims.batch * c.dims.heads * c.dims.d_k * c.dims.d_v);
+  const int max_states = (c.ws && state_bytes > 0) ? static_cast<int>(std::min<size_t>(c.ws_bytes / state_bytes, kMaxSub)) : 0;
+  if (max_states >= 1)
+    plan_segments(as, ctas, sms, 0.0, std::min(4, max_states + 1));
+  else
+    plan_segments(as, ctas, sms, kReplayCost, 4);
+  return max_states;
+}
+
 // 128-column d_v slices share S and the Q/K conversion across twice the output columns
 // (about 1.6x the work per SM); they need one sub-block per chunk (no cross accumulator in
 // tensor memory) and d_k <= 128.  The halved CTA count is made up by sequence segments.
@@ -1597,7 +1612,6 @@ int sm_count() {
 // the boundaries equalise rho * lo_s + (hi_s - lo_s) across segments.
 // With a workspace (two passes) nothing is replayed: a pre-pass launch computes each
 // segment's own state in parallel and the segments split the chunks evenly (rho = 0).
-constexpr double kReplayCost = 0.45;
 void plan_segments(TcArgs& a, int64_t ctas, int sms, double rho, int max_seg) {
   const int n = a.n_chunks;
   int n_seg = (ctas > 0 && sms > 0) ? static_cast<int>(sms / ctas) : 1;
@@ -1673,15 +1687,8 @@ cudaError_t launch_pipe(const RetentionCall& c, const HeadParams& hp, cudaStream
   TcArgs as = a;
   const dim3 grid = tc_grid(c.dims, DVS);
   const int64_t ctas = static_cast<int64_t>(grid.x) * grid.y * grid.z;
-  // The two-pass form keeps one state per pre-pass sub-segment in the caller's workspace.
-  const size_t state_bytes = sizeof(float) * static_cast<size_t>(c.dims.batch * c.dims.heads * c.dims.d_k * c.dims.d_v);
-  const int max_states = c.ws ? static_cast<int>(std::min<size_t>(c.ws_bytes / state_bytes, kMaxSub)) : 0;
   const int sms = sm_count();
-  if (max_states >= 1) {
-    plan_segments(as, ctas, sms, 0.0, std::min(4, max_states + 1));
-  } else {
-    plan_segments(as, ctas, sms, kReplayCost, 4);
-  }
+  const int max_states = plan_call(c, ctas, sms, as);
   auto run = [&](auto kern, unsigned nx) -> cudaError_t {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM);
     if (e != cudaSuccess) return e;
@@ -1795,6 +1802,17 @@ cudaError_t tc_wait_timeouts(unsigned int* count, bool clear) {
   if (e != cudaSuccess || !clear || *count == 0) return e;
   const unsigned int zero = 0;
   return cudaMemcpyToSymbol(sm100::g_wait_timeouts, &zero, sizeof(unsigned int));
+}
+
+int tc_chunkwise_launches(const RetentionCall& c) {
+  if (force_serial_kernel()) return 1;
+  const int T = pipe_tile_rows(c.dims.d_k, c.chunk);
+  const int dvs = pipe_wide_slice(c, T) ? 128 : 64;
+  const int nb = static_cast<int>(c.chunk / T);
+  TcArgs as = make_args(c, static_cast<int>((c.dims.seqlen + c.chunk - 1) / c.chunk), nb);
+  const int64_t ctas = (c.dims.d_v / dvs) * c.dims.heads * c.dims.batch;
+  const int max_states = plan_call(c, ctas, sm_count(), as);
+  return (as.n_seg > 1 && max_states >= 1) ? 2 : 1;
 }
 
 cudaError_t launch_tc_chunkwise(const RetentionCall& c, const HeadParams& hp, cudaStream_t s) {

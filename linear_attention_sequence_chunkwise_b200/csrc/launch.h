@@ -40,6 +40,8 @@ bool tc_chunkwise_heads_ok(const RetentionCall& c, const HeadParams& hp);
 // The driver entry point that encodes TMA tensor maps could be resolved.
 bool tc_driver_ready();
 cudaError_t launch_tc_chunkwise(const RetentionCall& c, const HeadParams& hp, cudaStream_t s);
+// Kernel launches launch_tc_chunkwise makes for this call on the current device (1 or 2).
+int tc_chunkwise_launches(const RetentionCall& c);
 // Reads (and optionally clears) the count of bounded waits that gave up in the tensor-core kernel.
 cudaError_t tc_wait_timeouts(unsigned int* count, bool clear);
 

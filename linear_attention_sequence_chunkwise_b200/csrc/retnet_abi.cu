@@ -169,6 +169,21 @@ retnet_status_t retnet_chunkwise_workspace_size(retnet_dims_t dims, size_t* byte
   return RETNET_OK;
 }
 
+int retnet_chunkwise_launches(retnet_dims_t dims, retnet_dtype_t in_dtype, uint32_t flags, int64_t chunk,
+                              const float* gamma, size_t workspace_bytes) {
+  const int path = retnet_chunkwise_kernel(dims, in_dtype, flags, chunk, gamma);
+  if (path < 0) return path;
+  if (dims.seqlen == 0) return 0;
+  if (path == 0) return 1;
+  const retnet_status_t st = check_device();
+  if (st != RETNET_OK) return -static_cast<int>(st);
+  RetentionCall c{nullptr, nullptr, nullptr, nullptr, Dims{dims.batch, dims.seqlen, dims.heads, dims.d_k, dims.d_v},
+                  in_dtype, RETNET_BF16, 0, flags, chunk, true, nullptr, nullptr, nullptr, nullptr};
+  c.ws = workspace_bytes ? reinterpret_cast<void*>(static_cast<uintptr_t>(256)) : nullptr;  // only its size matters
+  c.ws_bytes = workspace_bytes;
+  return tc_chunkwise_launches(c);
+}
+
 int retnet_chunkwise_kernel(retnet_dims_t dims, retnet_dtype_t in_dtype, uint32_t flags, int64_t chunk,
                             const float* gamma) {
   retnet_status_t st = check_common(dims, in_dtype, RETNET_F32, 0, flags, true);

@@ -118,6 +118,18 @@ def test_tc_two_pass_segments(dk, dv, B, L, with_state):
         assert err(so, Sref) <= TOL_BF16
 
 
+def test_tc_launch_count():
+    """The launch-count query follows the plan: two launches only for the workspace form with
+    segments (few (batch, head) pairs), one otherwise."""
+    g = si.gamma_schedule(8)
+    ws = rn.retnet_chunkwise_workspace_size((8, 2048, 8, 128, 128))
+    assert rn.retnet_chunkwise_launches((8, 2048, 8, 128), 128, rn.BF16, FLAGS, 64, g, ws) == 2
+    assert rn.retnet_chunkwise_launches((8, 2048, 8, 128), 128, rn.BF16, FLAGS, 64, g, 0) == 1
+    assert rn.retnet_chunkwise_launches((32, 2048, 8, 128), 128, rn.BF16, FLAGS, 64, g, 10 ** 9) == 1
+    assert rn.retnet_chunkwise_launches((8, 0, 8, 128), 128, rn.BF16, FLAGS, 64, g, ws) == 0
+    assert rn.retnet_chunkwise_launches((8, 2048, 8, 128), 128, rn.F32, FLAGS, 64, g, ws) == 1
+
+
 def test_tc_two_pass_full_workload():
     """b8/L2048/h8/d128/chunk 64 through the workspace form: within the bf16 bar of the plain
     call's output (the two round the segment-boundary state differently) and of the oracle on
