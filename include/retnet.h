@@ -167,6 +167,33 @@ RETNET_API retnet_status_t retnet_retention_chunkwise_ws(const void* q, const vo
                                               size_t workspace_bytes, void* stream);
 
 /*
+ * Allocation-free variant of retnet_retention_chunkwise_ws.  The pages have no counterpart:
+ * it is the same computation with the segment states kept in a static device array of
+ * RETNET_STATIC_SCRATCH_BYTES inside the library (one per device), for callers that cannot
+ * allocate device memory -- hosts that link only this C library and have no device
+ * allocator, or code that must not allocate on its hot path (cudaMalloc / cudaFree
+ * synchronise the device).  The library allocates nothing for it.
+ *   Limits: a call whose single segment state, batch * heads * d_k * d_v * 4 bytes, exceeds
+ *   RETNET_STATIC_SCRATCH_BYTES returns RETNET_ERR_UNSUPPORTED (use the _ws form with a
+ *   workspace of retnet_chunkwise_workspace_size bytes instead); smaller calls use as many
+ *   segment states as fit.
+ *   Zeroing: nothing in the scratch has to start at zero; every call overwrites what it reads.
+ *   Concurrency: the scratch is shared by every call on a device, so calls whose work
+ *   overlaps on the GPU (two streams, two host threads) race on it and give wrong results;
+ *   order them on the device.
+ *   Set-up: the first call on each device looks up the scratch's address (a CUDA symbol
+ *   query, made with that device current); make that first call outside any stream capture.
+ * Other arguments, results and errors as retnet_retention_chunkwise.
+ */
+#define RETNET_STATIC_SCRATCH_BYTES (16u << 20)
+RETNET_API retnet_status_t retnet_retention_chunkwise_static(const void* q, const void* k, const void* v, void* o,
+                                                  retnet_dims_t dims, retnet_dtype_t in_dtype,
+                                                  retnet_dtype_t out_dtype, const float* gamma,
+                                                  const float* theta, int64_t pos0, uint32_t flags,
+                                                  int64_t chunk, const float* state_in, float* state_out,
+                                                  const float* z_in, float* z_out, void* stream);
+
+/*
  * Workspace size (bytes) that lets retnet_retention_chunkwise_ws use its full segment split
  * for these dimensions: 6 * batch * heads * d_k * d_v * sizeof(float) (room for the states of
  * six pre-pass sub-segments).  Host-only; no device

@@ -30,7 +30,9 @@ BF16 = 1
 
 STATUS = {0: "RETNET_OK", 1: "RETNET_ERR_NULL_PTR", 2: "RETNET_ERR_BAD_SHAPE", 3: "RETNET_ERR_BAD_DTYPE",
           4: "RETNET_ERR_BAD_PARAM", 5: "RETNET_ERR_UNSUPPORTED", 6: "RETNET_ERR_CUDA"}
+STATIC_SCRATCH_BYTES = 16 << 20  # RETNET_STATIC_SCRATCH_BYTES
 EXPORTS = ("retnet_retention_parallel", "retnet_retention_chunkwise", "retnet_retention_chunkwise_ws",
+           "retnet_retention_chunkwise_static",
            "retnet_chunkwise_workspace_size", "retnet_retention_step", "retnet_msr_epilogue",
            "retnet_chunkwise_kernel", "retnet_chunkwise_launches", "retnet_debug_wait_timeouts",
            "retnet_status_string", "retnet_version")
@@ -70,13 +72,15 @@ def load(path: str = None):
                                                _vp, _vp, _vp, _vp, _vp]
     lib.retnet_retention_chunkwise_ws.argtypes = [_vp, _vp, _vp, _vp, Dims, _i32, _i32, _fp, _fp, _i64, _u32,
                                                   _i64, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+    lib.retnet_retention_chunkwise_static.argtypes = [_vp, _vp, _vp, _vp, Dims, _i32, _i32, _fp, _fp, _i64, _u32,
+                                                      _i64, _vp, _vp, _vp, _vp, _vp]
     lib.retnet_chunkwise_workspace_size.argtypes = [Dims, ctypes.POINTER(ctypes.c_size_t)]
     lib.retnet_chunkwise_workspace_size.restype = _i32
     lib.retnet_retention_step.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _fp,
                                           _fp, _i64, _u32, _vp]
     lib.retnet_msr_epilogue.argtypes = [_vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_float, _i32, _i32, _vp]
     for name in ("retnet_retention_parallel", "retnet_retention_chunkwise", "retnet_retention_chunkwise_ws",
-                 "retnet_retention_step", "retnet_msr_epilogue"):
+                 "retnet_retention_chunkwise_static", "retnet_retention_step", "retnet_msr_epilogue"):
         getattr(lib, name).restype = _i32
     lib.retnet_chunkwise_kernel.argtypes = [Dims, _i32, _u32, _i64, _fp]
     lib.retnet_chunkwise_kernel.restype = _i32
@@ -204,6 +208,17 @@ def retnet_retention_chunkwise_ws(q, k, v, o, gamma, theta=None, pos0=0, flags=F
                                                 _dtype_code(o), _fptr(g), _fptr(th), int(pos0), int(flags),
                                                 int(chunk), _ptr(state_in), _ptr(state_out), _ptr(z_in),
                                                 _ptr(z_out), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def retnet_retention_chunkwise_static(q, k, v, o, gamma, theta=None, pos0=0, flags=F_ALL, chunk=64, state_in=None,
+                                      state_out=None, z_in=None, z_out=None, stream=None):
+    """Chunkwise form with the library's static device scratch (no workspace argument, no
+    allocation); calls that overlap on the GPU race on the scratch -- see the C header."""
+    d, g, th = _chunkwise_args(q, k, v, o, gamma, theta, state_in, state_out, z_in, z_out)
+    _check(load().retnet_retention_chunkwise_static(_ptr(q), _ptr(k), _ptr(v), _ptr(o), d, _dtype_code(q),
+                                                    _dtype_code(o), _fptr(g), _fptr(th), int(pos0), int(flags),
+                                                    int(chunk), _ptr(state_in), _ptr(state_out), _ptr(z_in),
+                                                    _ptr(z_out), _stream(stream)))
 
 
 def retnet_retention_chunkwise(q, k, v, o, gamma, theta=None, pos0=0, flags=F_ALL, chunk=64, state_in=None,

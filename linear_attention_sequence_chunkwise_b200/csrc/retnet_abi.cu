@@ -5,6 +5,8 @@
 // caller's stream.  Nothing is allocated; no state survives the call.
 #include <math.h>
 
+#include <atomic>
+
 #include "launch.h"
 
 using namespace retnet;
@@ -158,6 +160,58 @@ retnet_status_t retnet_retention_chunkwise_ws(const void* q, const void* k, cons
                                               size_t workspace_bytes, void* stream) {
   return chunkwise_impl(q, k, v, o, dims, in_dtype, out_dtype, gamma, theta, pos0, flags, chunk, state_in, state_out,
                         z_in, z_out, workspace, workspace_bytes, stream);
+}
+
+// ---- allocation-free variant ---------------------------------------------------------------
+// Segment states of the two-pass form in a file-scope device array instead of a caller's
+// workspace: for callers that cannot allocate device memory -- hosts that link only this C
+// library and have no device allocator of their own, and code that must not allocate on its
+// hot path because cudaMalloc / cudaFree synchronise the device.  The array exists once per
+// device (per context); nothing in it needs to start at zero (each call overwrites the states
+// it reads).  Calls that overlap on the GPU share it and race.
+static __device__ __align__(256) unsigned char g_chunkwise_scratch[RETNET_STATIC_SCRATCH_BYTES];
+
+namespace {
+// Device address of the scratch on the current device, looked up (cudaGetSymbolAddress, with
+// that device current) on the first call per device and cached.
+constexpr int kMaxDevices = 64;
+std::atomic<void*> g_scratch_addr[kMaxDevices];
+
+retnet_status_t static_scratch(void** ptr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return RETNET_ERR_CUDA;
+  if (dev >= 0 && dev < kMaxDevices) {
+    void* p = g_scratch_addr[dev].load(std::memory_order_acquire);
+    if (p) {
+      *ptr = p;
+      return RETNET_OK;
+    }
+  }
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_chunkwise_scratch) != cudaSuccess || !p) return RETNET_ERR_CUDA;
+  if (dev >= 0 && dev < kMaxDevices) g_scratch_addr[dev].store(p, std::memory_order_release);
+  *ptr = p;
+  return RETNET_OK;
+}
+}  // namespace
+
+retnet_status_t retnet_retention_chunkwise_static(const void* q, const void* k, const void* v, void* o,
+                                                  retnet_dims_t dims, retnet_dtype_t in_dtype,
+                                                  retnet_dtype_t out_dtype, const float* gamma, const float* theta,
+                                                  int64_t pos0, uint32_t flags, int64_t chunk,
+                                                  const float* state_in, float* state_out, const float* z_in,
+                                                  float* z_out, void* stream) {
+  if (dims.batch >= 0 && dims.heads >= 0 && dims.d_k >= 0 && dims.d_v >= 0) {
+    // One segment state must fit the static scratch; larger calls are rejected, not degraded.
+    const double state_bytes = 4.0 * static_cast<double>(dims.batch) * static_cast<double>(dims.heads) *
+                               static_cast<double>(dims.d_k) * static_cast<double>(dims.d_v);
+    if (state_bytes > static_cast<double>(RETNET_STATIC_SCRATCH_BYTES)) return RETNET_ERR_UNSUPPORTED;
+  }
+  void* scratch = nullptr;
+  const retnet_status_t st = static_scratch(&scratch);
+  if (st != RETNET_OK) return st;
+  return chunkwise_impl(q, k, v, o, dims, in_dtype, out_dtype, gamma, theta, pos0, flags, chunk, state_in,
+                        state_out, z_in, z_out, scratch, RETNET_STATIC_SCRATCH_BYTES, stream);
 }
 
 retnet_status_t retnet_chunkwise_workspace_size(retnet_dims_t dims, size_t* bytes) {

@@ -137,6 +137,18 @@ def test_chunkwise_workspace_entry_points(lib):
                                              None, FAKE + 8, 4096, None) == 4
 
 
+def test_static_scratch_entry_point_limits(lib):
+    """The allocation-free chunkwise call rejects, before touching a device, a call whose one
+    segment state exceeds the static scratch; the header and the binding agree on its size."""
+    m = re.search(r"#define RETNET_STATIC_SCRATCH_BYTES \((\d+)u << (\d+)\)", open(HEADER).read())
+    assert m and int(m.group(1)) << int(m.group(2)) == rn.STATIC_SCRATCH_BYTES
+    g = _gamma(16)
+    gp = g.ctypes.data_as(rn._fp)
+    big = rn.Dims(64, 8, 16, 256, 512)  # one state = 512 MiB
+    assert lib.retnet_retention_chunkwise_static(FAKE, FAKE, FAKE, FAKE, big, 1, 1, gp, None, 0, 0, 64, None, None,
+                                                 None, None, None) == 5
+
+
 def test_epilogue_validation(lib):
     f = lib.retnet_msr_epilogue
     assert f(FAKE, FAKE, FAKE, 4, 2, 12, 1e-5, 0, 0, None) == 2          # d_v not a multiple of 8
