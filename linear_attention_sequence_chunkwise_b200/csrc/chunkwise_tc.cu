@@ -594,10 +594,13 @@ struct Cfg3 {
   static constexpr int RBLK = DK > 128 ? 2 : 1;     // 128-row blocks of the state increment
   static constexpr int MR = DK >= 128 ? 128 : 64;
   // RTM: the fp32 state lives in tensor memory (the increment's columns) and each state
-  // increment accumulates into it; otherwise the state group holds it in registers, one
-  // thread per (d_k row, 64 columns).  RTM needs one sub-block per chunk (the 128-wide slice).
-  static constexpr bool RTM = DVS == 128;
-  static constexpr int WARPS_S = RTM ? 4 * RBLK : 4 * RBLK * NDV;
+  // increment accumulates into it (four state warps, a thread per TMEM lane, all its 128-row
+  // blocks); otherwise the state group holds it in registers, one thread per (d_k row, 64
+  // columns).  Taken for the 128-wide slice and for d_k = 256 (where eight register warps
+  // would push the CTA to 18 warps and 96 registers).
+  static constexpr bool RTM = DVS == 128 || DK == 256;
+  static constexpr int WARPS_S = RTM ? 4 : 4 * RBLK * NDV;
+  static constexpr int BPT = RTM ? RBLK : 1;  // 128-row state blocks per state thread
   static constexpr int WARP_S0 = 4;
   static constexpr int WARP_CONV0 = WARP_S0 + WARPS_S;
   static constexpr int CONV_WARPS = 4;
@@ -636,7 +639,7 @@ struct Cfg3 {
   static constexpr int NS_FIT = (BUDGET - FIXED) / STAGE;
   static constexpr int NS = NS_FIT > 4 ? 4 : NS_FIT;
   static constexpr int SMEM = NS * STAGE + FIXED + 1024;
-  static constexpr bool FITS = NS >= 2 && USED <= 512 && (DVS == 64 || DVS == 128);
+  static constexpr bool FITS = NS >= 2 && USED <= 512 && (DVS == 64 || DVS == 128) && (!RTM || DRBUF == 1);
   // Columns per TMEM load batch: 18 warps leave 96 registers a thread (five warps share one
   // sub-partition's register file), too few to hold 64 loaded columns next to the state.
   static constexpr int LDW = THREADS > 512 ? 32 : 64;
@@ -1193,120 +1196,136 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
     if constexpr (SM == SEG_STATE) {
       // State pre-pass: once the last increment has landed, the accumulated segment state
       // (thread = one d_k row, all DVS columns) goes to the workspace.
-      const int blk = (warp - C::WARP_S0) / 4;
       const uint32_t lane_off = static_cast<uint32_t>(32 * (warp % 4)) << 16;
-      const int dk = (DK == 64) ? (lane < 16 ? 16 * (warp % 4) + lane : -1) : blk * 128 + 32 * (warp % 4) + lane;
       if (__all_sync(0xffffffffu, mbar_wait(bar(Q_DR_FULL + 0), 0))) {
         tc_fence_after();
         const size_t plane = static_cast<size_t>(gridDim.z) * a.heads * DK * a.dv;
-        float* dst = a.ws + seg * plane + (static_cast<size_t>(b) * a.heads + h) * DK * a.dv + dvb * DVS +
-                     static_cast<size_t>(dk < 0 ? 0 : dk) * a.dv;
 #pragma unroll 1
-        for (int grp = 0; grp < DVS / 32; ++grp) {
-          uint32_t u[2][16];
-          tmem_ld_wait(tmem + C::COL_DR + blk * DVS + 32 * grp + lane_off, u);
-          if (dk >= 0) {
+        for (int bk = 0; bk < C::BPT; ++bk) {
+          const int blk = C::BPT > 1 ? bk : (warp - C::WARP_S0) / 4 % C::RBLK;
+          const int dk = (DK == 64) ? (lane < 16 ? 16 * (warp % 4) + lane : -1) : blk * 128 + 32 * (warp % 4) + lane;
+          float* dst = a.ws + seg * plane + (static_cast<size_t>(b) * a.heads + h) * DK * a.dv + dvb * DVS +
+                       static_cast<size_t>(dk < 0 ? 0 : dk) * a.dv;
+#pragma unroll 1
+          for (int grp = 0; grp < DVS / 32; ++grp) {
+            uint32_t u[2][16];
+            tmem_ld_wait(tmem + C::COL_DR + blk * DVS + 32 * grp + lane_off, u);
+            if (dk >= 0) {
 #pragma unroll
-            for (int c4 = 0; c4 < 8; ++c4)
-              *reinterpret_cast<float4*>(dst + 32 * grp + 4 * c4) =
-                  make_float4(__uint_as_float(u[(4 * c4) / 16][(4 * c4) % 16]),
-                              __uint_as_float(u[(4 * c4 + 1) / 16][(4 * c4 + 1) % 16]),
-                              __uint_as_float(u[(4 * c4 + 2) / 16][(4 * c4 + 2) % 16]),
-                              __uint_as_float(u[(4 * c4 + 3) / 16][(4 * c4 + 3) % 16]));
+              for (int c4 = 0; c4 < 8; ++c4)
+                *reinterpret_cast<float4*>(dst + 32 * grp + 4 * c4) =
+                    make_float4(__uint_as_float(u[(4 * c4) / 16][(4 * c4) % 16]),
+                                __uint_as_float(u[(4 * c4 + 1) / 16][(4 * c4 + 1) % 16]),
+                                __uint_as_float(u[(4 * c4 + 2) / 16][(4 * c4 + 2) % 16]),
+                                __uint_as_float(u[(4 * c4 + 3) / 16][(4 * c4 + 3) % 16]));
+            }
           }
         }
       }
     } else if constexpr (C::RTM) {
-      // The fp32 state stays in tensor memory; thread = one d_k row (its TMEM lane), all
-      // DVS columns.  Before chunk i's increment accumulates into it, the state group reads
-      // R_{i-1}, writes its fp16 copy (output chunks only) and stores gamma^T R_{i-1} back.
-      // With Kz = gamma^(T-1-c) rot(k) the increment of a chunk of b' rows is
-      // gamma^(b'-T) (Kz^T V); the factor is 1 except on the last chunk, where state_out takes it.
-      const int ws = warp - C::WARP_S0;
-      const int blk = ws / 4;
+      // The fp32 state stays in tensor memory as a master M; thread = one TMEM lane, i.e. one
+      // d_k row in each of its BPT 128-row blocks, all DVS columns.  Before every increment
+      // Kz_w^T V_w (the column blocks w of a chunk's last row block) accumulates into M, the
+      // state group scales M by gamma^T; at w = 0 M holds R_{i-1}, whose fp16 copy (output
+      // chunks only) is written first.  This is the Horner form of
+      //   R_i = gamma^b' R_{i-1} + sum_w gamma^(b'-(w+1)T) Kz_w^T V_w = hh * M,
+      // hh = gamma^(b' - nbw T): 1 except on the last chunk, where state_out takes it.
       const uint32_t lane_off = static_cast<uint32_t>(32 * (warp % 4)) << 16;
-      const int dk = (DK == 64) ? (lane < 16 ? 16 * (warp % 4) + lane : -1) : blk * 128 + 32 * (warp % 4) + lane;
       const int64_t bh = static_cast<int64_t>(b) * a.heads + h;
       const size_t srow = static_cast<size_t>(a.dv);
-      const uint32_t tR = tmem + C::COL_DR + blk * DVS + lane_off;
       const float gT = decay_pow(log2g, T);
       constexpr int GW = 32;  // columns per batch
+      auto row_of = [&](int blk) -> int {
+        return (DK == 64) ? (lane < 16 ? 16 * (warp % 4) + lane : -1) : blk * 128 + 32 * (warp % 4) + lane;
+      };
       bool ok = true;
-      int last_dr = -1, last_bl = T;
+      int last_dr = -1, last_bl = T, last_nbw = 1;
       UnitIter<T, SM> it;
       for (it.start(a.L, nb, c_first, c_lo, c_hi); ok && it.valid(); it.next()) {
+        if (!it.last_row()) continue;
         const int d = it.dr;
-        if (d > 0) {  // the previous increment has landed: the master holds R_{i-1}
+        if (d > 0) {  // the previous increment has landed
           ok = __all_sync(0xffffffffu, mbar_wait(bar(Q_DR_FULL + 0), (d - 1) & 1));
           if (!ok) break;
           tc_fence_after();
         }
-        const bool out = !it.pre();
+        const bool copy = !it.pre() && it.w == 0;  // M = R_{i-1}: write its fp16 copy
         const int ri = it.i - c_lo;
-        if (out && ri >= C::RBUF) {
+        if (copy && ri >= C::RBUF) {
           ok = __all_sync(0xffffffffu, mbar_wait(bar(Q_R16_FREE + (ri % C::RBUF)), ((ri - C::RBUF) / C::RBUF) & 1));
           if (!ok) break;
         }
         const uint32_t r16 = sR(ri);
 #pragma unroll 1
-        for (int grp = 0; grp < DVS / GW; ++grp) {
-          uint32_t u[GW / 16][16];
-          if (d > 0) {
-            tmem_ld_wait(tR + GW * grp, u);
-          } else {  // first chunk: the master starts from state_in (carried over earlier segments)
-            float r0v[GW];
-            if (dk >= 0) {
-              start_state(dk, dvb * DVS + GW * grp, GW, r0v);
-            } else {
+        for (int bk = 0; bk < C::BPT; ++bk) {
+          const int dk = row_of(bk);
+          const uint32_t tR = tmem + C::COL_DR + bk * DVS + lane_off;
+#pragma unroll 1
+          for (int grp = 0; grp < DVS / GW; ++grp) {
+            uint32_t u[GW / 16][16];
+            if (d > 0) {
+              tmem_ld_wait(tR + GW * grp, u);
+            } else {  // first increment: M starts from state_in (carried over earlier segments)
+              float r0v[GW];
+              if (dk >= 0) {
+                start_state(dk, dvb * DVS + GW * grp, GW, r0v);
+              } else {
 #pragma unroll
-              for (int c = 0; c < GW; ++c) r0v[c] = 0.f;
+                for (int c = 0; c < GW; ++c) r0v[c] = 0.f;
+              }
+#pragma unroll
+              for (int c = 0; c < GW; ++c) u[c / 16][c % 16] = __float_as_uint(r0v[c]);
+            }
+            if (copy && dk >= 0) {
+              // fp16 copy (times 1/sqrt(d_k)) into box (column / 64), 16-byte slots of 8 columns
+#pragma unroll
+              for (int c8 = 0; c8 < GW / 8; ++c8) {
+                const int col = GW * grp + 8 * c8;
+                const uint32_t* x = &u[(8 * c8) / 16][(8 * c8) % 16];
+                st_shared_v4(r16 + (col / 64) * DK * 128 + sw128(dk, (col % 64) / 8),
+                             pack_f16x2(sd * __uint_as_float(x[0]), sd * __uint_as_float(x[1])),
+                             pack_f16x2(sd * __uint_as_float(x[2]), sd * __uint_as_float(x[3])),
+                             pack_f16x2(sd * __uint_as_float(x[4]), sd * __uint_as_float(x[5])),
+                             pack_f16x2(sd * __uint_as_float(x[6]), sd * __uint_as_float(x[7])));
+              }
             }
 #pragma unroll
-            for (int c = 0; c < GW; ++c) u[c / 16][c % 16] = __float_as_uint(r0v[c]);
+            for (int c = 0; c < GW; ++c) u[c / 16][c % 16] = __float_as_uint(gT * __uint_as_float(u[c / 16][c % 16]));
+            tmem_st_wait(tR + GW * grp, u);
           }
-          if (out && dk >= 0) {
-            // fp16 copy (times 1/sqrt(d_k)) into box (column / 64), 16-byte slots of 8 columns
-#pragma unroll
-            for (int c8 = 0; c8 < GW / 8; ++c8) {
-              const int col = GW * grp + 8 * c8;
-              const uint32_t* x = &u[(8 * c8) / 16][(8 * c8) % 16];
-              st_shared_v4(r16 + (col / 64) * DK * 128 + sw128(dk, (col % 64) / 8),
-                           pack_f16x2(sd * __uint_as_float(x[0]), sd * __uint_as_float(x[1])),
-                           pack_f16x2(sd * __uint_as_float(x[2]), sd * __uint_as_float(x[3])),
-                           pack_f16x2(sd * __uint_as_float(x[4]), sd * __uint_as_float(x[5])),
-                           pack_f16x2(sd * __uint_as_float(x[6]), sd * __uint_as_float(x[7])));
-            }
-          }
-#pragma unroll
-          for (int c = 0; c < GW; ++c) u[c / 16][c % 16] = __float_as_uint(gT * __uint_as_float(u[c / 16][c % 16]));
-          tmem_st_wait(tR + GW * grp, u);
         }
-        if (out) fence_proxy_async_smem();
+        if (copy) fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(bar(Q_DR_FREE + (d & 1)));  // the master is ready for this chunk's increment
-        if (out) mbar_arrive(bar(Q_R16_FULL + (ri % C::RBUF)));
+        mbar_arrive(bar(Q_DR_FREE + (d & 1)));  // M is ready for this increment
+        if (copy) mbar_arrive(bar(Q_R16_FULL + (ri % C::RBUF)));
         last_dr = d;
         last_bl = it.bl;
+        last_nbw = it.nbw;
       }
-      // End of the sequence: R_last = gamma^(b'-T) * master once the last increment landed.
+      // End of the sequence: R_last = hh * M once the last increment landed.
       if (ok && last_dr >= 0 && (!SEG || c_hi * nb * T >= a.L)) {
         ok = __all_sync(0xffffffffu, mbar_wait(bar(Q_DR_FULL + 0), last_dr & 1));
         tc_fence_after();
         if (ok && a.state_out) {
-          const float hh = exp2f(static_cast<float>(last_bl - T) * log2g);
+          const float hh = exp2f(static_cast<float>(last_bl - last_nbw * T) * log2g);
 #pragma unroll 1
-          for (int grp = 0; grp < DVS / GW; ++grp) {
-            uint32_t u[GW / 16][16];
-            tmem_ld_wait(tR + GW * grp, u);
-            if (dk >= 0) {
-              float* dst = a.state_out + static_cast<size_t>(bh) * DK * a.dv + dvb * DVS + GW * grp + dk * srow;
+          for (int bk = 0; bk < C::BPT; ++bk) {
+            const int dk = row_of(bk);
+            const uint32_t tR = tmem + C::COL_DR + bk * DVS + lane_off;
+#pragma unroll 1
+            for (int grp = 0; grp < DVS / GW; ++grp) {
+              uint32_t u[GW / 16][16];
+              tmem_ld_wait(tR + GW * grp, u);
+              if (dk >= 0) {
+                float* dst = a.state_out + static_cast<size_t>(bh) * DK * a.dv + dvb * DVS + GW * grp + dk * srow;
 #pragma unroll
-              for (int c4 = 0; c4 < GW / 4; ++c4)
-                *reinterpret_cast<float4*>(dst + 4 * c4) =
-                    make_float4(hh * __uint_as_float(u[(4 * c4) / 16][(4 * c4) % 16]),
-                                hh * __uint_as_float(u[(4 * c4 + 1) / 16][(4 * c4 + 1) % 16]),
-                                hh * __uint_as_float(u[(4 * c4 + 2) / 16][(4 * c4 + 2) % 16]),
-                                hh * __uint_as_float(u[(4 * c4 + 3) / 16][(4 * c4 + 3) % 16]));
+                for (int c4 = 0; c4 < GW / 4; ++c4)
+                  *reinterpret_cast<float4*>(dst + 4 * c4) =
+                      make_float4(hh * __uint_as_float(u[(4 * c4) / 16][(4 * c4) % 16]),
+                                  hh * __uint_as_float(u[(4 * c4 + 1) / 16][(4 * c4 + 1) % 16]),
+                                  hh * __uint_as_float(u[(4 * c4 + 2) / 16][(4 * c4 + 2) % 16]),
+                                  hh * __uint_as_float(u[(4 * c4 + 3) / 16][(4 * c4 + 3) % 16]));
+              }
             }
           }
         }
