@@ -588,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 //   1 warp TMA, 1 warp MMA issuer (one unit ahead: S and dR of unit k+1 before X/PV of unit k).
 // ============================================================================================
 
-template <int DK, int T, int DVS>
+template <int DK, int T, int DVS, bool PRE = false>
 struct Cfg3 {
   static constexpr int NDV = DVS / 64;              // 64-column boxes of the d_v slice
   static constexpr int RBLK = DK > 128 ? 2 : 1;     // 128-row blocks of the state increment
@@ -603,7 +603,7 @@ struct Cfg3 {
   static constexpr int BPT = RTM ? RBLK : 1;  // 128-row state blocks per state thread
   static constexpr int WARP_S0 = 4;
   static constexpr int WARP_CONV0 = WARP_S0 + WARPS_S;
-  static constexpr int CONV_WARPS = 4;
+  static constexpr int CONV_WARPS = PRE ? 0 : 4;  // PRE: tiles arrive converted (pre-pass)
   static constexpr int NCONV = 32 * CONV_WARPS;
   static constexpr int WARP_TMA = WARP_CONV0 + CONV_WARPS;
   static constexpr int WARP_MMA = WARP_TMA + 1;
@@ -861,11 +861,13 @@ struct UnitConverter {
   }
 };
 
-template <int DK, int T, int DVS, int SM, typename Tout>
-__global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
+template <int DK, int T, int DVS, int SM, bool PRE, typename Tout>
+__global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE>::THREADS, 1)
     tc_chunkwise_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v, TcArgs a, HeadParams hp) {
-  using C = Cfg3<DK, T, DVS>;
+  using C = Cfg3<DK, T, DVS, PRE>;
+  // Stage ready for the MMAs: converted in place, or (PRE) landed already converted.
+  constexpr int Q_READY = PRE ? Q_TMA_FULL : Q_CONV_FULL;
   constexpr bool SEG = SM != SEG_NONE;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_addr(smem_raw);
@@ -959,7 +961,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < 4; ++s) {
       mbar_init(bar(Q_TMA_FULL + s), 1);
-      mbar_init(bar(Q_CONV_FULL + s), C::NCONV);
+      if (!PRE) mbar_init(bar(Q_CONV_FULL + s), C::NCONV);
       mbar_init(bar(Q_STAGE_EMPTY + s), 1);
     }
     for (int k = 0; k < 2; ++k) {
@@ -973,7 +975,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
       mbar_init(bar(Q_R16_FREE + k), 1);
       mbar_init(bar(Q_O_FULL + k), 1);
       mbar_init(bar(Q_O_FREE + k), 128);
-      mbar_init(bar(Q_TAB + k), C::NCONV);
+      if (!PRE) mbar_init(bar(Q_TAB + k), C::NCONV);
     }
     mbar_init(bar(Q_DRAIN), 1);
     fence_mbar_init();
@@ -1032,7 +1034,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
       // of the oldest unit first, F at most LA units ahead -- so a late conversion of a later
       // unit never holds back the output (and the stage release) of an earlier one.
       auto f_ready = [&](const UnitIter<T, SM>& f) -> bool {
-        if (!mbar_test(bar(Q_CONV_FULL + f.k % C::NS), (f.k / C::NS) & 1)) return false;
+        if (!mbar_test(bar(Q_READY + f.k % C::NS), (f.k / C::NS) & 1)) return false;
         if (!f.pre() && f.kf() >= C::SBUF &&
             !mbar_test(bar(Q_S_FREE + (f.kf() % C::SBUF)), ((f.kf() - C::SBUF) / C::SBUF) & 1))
           return false;
@@ -1109,7 +1111,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
         bool first = true;
         for (f.start(a.L, nb, c_first, c_lo, c_hi); f.valid(); f.next()) {
           const int s = f.k % C::NS;
-          if (!mbar_wait(bar(Q_CONV_FULL + s), (f.k / C::NS) & 1)) break;
+          if (!mbar_wait(bar(Q_READY + s), (f.k / C::NS) & 1)) break;
           tc_fence_after();
           const uint64_t dkm = sdesc_sw128(sK(s), T * 128, 1024), dv = sdesc_sw128(sV(s), T * 128, 1024);
 #pragma unroll
@@ -1162,6 +1164,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
     }
   } else if (warp >= C::WARP_CONV0) {
     // ------------------------------------------------------------------ converters
+    if constexpr (!PRE) {
     UnitConverter<DK, T, C::NCONV, C::NDV> cv;
     cv.init(threadIdx.x - 32 * C::WARP_CONV0, nb, hp);
     const bool xpos = (a.flags & RETNET_F_XPOS) != 0;
@@ -1190,6 +1193,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
       }
       fence_proxy_async_smem();
       mbar_arrive(bar(Q_CONV_FULL + s));
+    }
     }
   } else if (warp >= C::WARP_S0) {
     // ------------------------------------------------------------------ state group
@@ -1549,6 +1553,69 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS>::THREADS, 1)
   }
 }
 
+// ============================================================================================
+// Conversion pre-pass (chunks of several sub-blocks).  The pipelined kernel converts Q_u, K_w
+// and V_w for every unit (u, w), i.e. (nb + 1) / 2 times per token; this kernel writes fp16
+// copies that already carry its operand scaling, once per token, and the pipelined kernel then
+// loads MMA-ready tiles (no converter role).  With r = t mod T the row inside its T-row
+// sub-block (chunks start at multiples of B, and T divides B):
+//   q~ = gamma^(r+1) rot(q),   k~ = gamma^(T-1-r) rot(k),   v~ = v   (fp16),
+// the rotation by the absolute position p = pos0 + t.  Thread = (token, 8-element slot of
+// d_k) across every head (the rotation factors are computed once), then (8-element slots of v).
+// ============================================================================================
+template <int DK, int T>
+__global__ void __launch_bounds__(256) tc_convert_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
+                                                         const uint4* __restrict__ v, uint4* __restrict__ qo,
+                                                         uint4* __restrict__ ko, uint4* __restrict__ vo,
+                                                         int64_t tokens, int L, int heads, int dv, int64_t pos0,
+                                                         uint32_t flags, HeadParams hp) {
+  constexpr int S = DK / 8;  // 16-byte slots of a head row of q or k
+  const int64_t n_qk = tokens * S;
+  const int64_t n_v = tokens * heads * (dv / 8);
+  const bool xpos = (flags & RETNET_F_XPOS) != 0;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_qk + n_v;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    if (i < n_qk) {
+      const int64_t n = i / S;
+      const int sl = static_cast<int>(i % S);
+      const int t = static_cast<int>(n % L), r = t % T;
+      float2 f[4];
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        float sn = 0.f, c = 1.f;
+        if (xpos) xpos_sincos(pos0 + t, hp.theta[4 * sl + jj], &sn, &c);
+        f[jj] = make_float2(c, sn);
+      }
+      for (int h = 0; h < heads; ++h) {
+        const int64_t off = (n * heads + h) * S + sl;
+        const uint4 xq = q[off], xk = k[off];
+        const float l2g = hp.log2g[h];
+        const float xi = decay_pow(l2g, r + 1), zeta = decay_pow(l2g, T - 1 - r);
+        const uint32_t wq[4] = {xq.x, xq.y, xq.z, xq.w}, wk[4] = {xk.x, xk.y, xk.z, xk.w};
+        uint32_t oq[4], ok[4];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const float q0 = __uint_as_float(wq[jj] << 16), q1 = __uint_as_float(wq[jj] & 0xffff0000u);
+          const float k0 = __uint_as_float(wk[jj] << 16), k1 = __uint_as_float(wk[jj] & 0xffff0000u);
+          oq[jj] = pack_f16x2(xi * (q0 * f[jj].x - q1 * f[jj].y), xi * (q0 * f[jj].y + q1 * f[jj].x));
+          ok[jj] = pack_f16x2(zeta * (k0 * f[jj].x - k1 * f[jj].y), zeta * (k0 * f[jj].y + k1 * f[jj].x));
+        }
+        qo[off] = make_uint4(oq[0], oq[1], oq[2], oq[3]);
+        ko[off] = make_uint4(ok[0], ok[1], ok[2], ok[3]);
+      }
+    } else {
+      const int64_t j = i - n_qk;
+      const uint4 x = v[j];
+      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj)
+        o[jj] = pack_f16x2(__uint_as_float(w[jj] << 16), __uint_as_float(w[jj] & 0xffff0000u));
+      vo[j] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+}
+
 // ---- host side -------------------------------------------------------------------------------
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -1608,6 +1675,30 @@ int plan_call(const RetentionCall& c, int64_t ctas, int sms, TcArgs& as) {
   else
     plan_segments(as, ctas, sms, kReplayCost, 4);
   return max_states;
+}
+
+// fp16 copies of the conversion pre-pass in the caller's workspace (256-byte aligned parts).
+struct PreCopies {
+  void* q;
+  void* k;
+  void* v;
+};
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+size_t pre_copy_bytes(const Dims& d) {
+  const size_t tok = static_cast<size_t>(d.batch) * static_cast<size_t>(d.seqlen) * static_cast<size_t>(d.heads);
+  return 2 * align256(tok * d.d_k * 2) + align256(tok * d.d_v * 2);
+}
+PreCopies pre_copies(const RetentionCall& c) {
+  const size_t tok = static_cast<size_t>(c.dims.batch) * static_cast<size_t>(c.dims.seqlen) *
+                     static_cast<size_t>(c.dims.heads);
+  char* base = static_cast<char*>(c.ws);
+  const size_t qk = align256(tok * c.dims.d_k * 2);
+  return PreCopies{base, base + qk, base + 2 * qk};
+}
+// The pre-pass pays one extra read and write of q, k, v; it saves the (nb + 1) / 2-fold
+// reconversion of chunks of nb >= 2 sub-blocks.  Not combined with sequence segments.
+bool pre_convert_applies(const RetentionCall& c, int nb, int n_seg) {
+  return nb >= 2 && n_seg < 2 && c.ws && c.ws_bytes >= pre_copy_bytes(c.dims);
 }
 
 // 128-column d_v slices share S and the Q/K conversion across twice the output columns
@@ -1697,6 +1788,7 @@ dim3 tc_grid(const Dims& d, int dvs) {
 template <int DK, int T, int DVS, typename Tout>
 cudaError_t launch_pipe(const RetentionCall& c, const HeadParams& hp, cudaStream_t s) {
   using Cf = Cfg3<DK, T, DVS>;
+  using CfP = Cfg3<DK, T, DVS, true>;
   static_assert(Cf::FITS, "pipelined kernel does not fit this tile");
   CUtensorMap mq, mk, mv;
   if (!make_maps(c, T, &mq, &mk, &mv)) return cudaErrorInvalidValue;
@@ -1714,8 +1806,38 @@ cudaError_t launch_pipe(const RetentionCall& c, const HeadParams& hp, cudaStream
     kern<<<dim3(grid.x * nx, grid.y, grid.z), Cf::THREADS, Cf::SMEM, s>>>(mq, mk, mv, as, hp);
     return cudaGetLastError();
   };
-  if (as.n_seg < 2) return run(tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_NONE, Tout>, 1);
-  if (max_states < 1) return run(tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_REPLAY, Tout>, as.n_seg);
+  if (as.n_seg < 2) {
+    if constexpr (Cf::XBUF > 0) {
+      // Chunks of several sub-blocks, no segments, and a workspace that holds the fp16
+      // copies: convert once in a pre-pass, then run the kernel without converters.
+      if (pre_convert_applies(c, nb, as.n_seg)) {
+        const PreCopies pc = pre_copies(c);
+        const int64_t tokens = c.dims.batch * c.dims.seqlen;
+        const int64_t items = tokens * (DK / 8) + tokens * c.dims.heads * (c.dims.d_v / 8);
+        const int blocks = static_cast<int>(std::min<int64_t>((items + 255) / 256, static_cast<int64_t>(sms) * 8));
+        tc_convert_kernel<DK, T><<<blocks, 256, 0, s>>>(
+            static_cast<const uint4*>(c.q), static_cast<const uint4*>(c.k), static_cast<const uint4*>(c.v),
+            static_cast<uint4*>(pc.q), static_cast<uint4*>(pc.k), static_cast<uint4*>(pc.v), tokens,
+            static_cast<int>(c.dims.seqlen), static_cast<int>(c.dims.heads), static_cast<int>(c.dims.d_v), c.pos0,
+            c.flags, hp);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        RetentionCall cc = c;
+        cc.q = pc.q;
+        cc.k = pc.k;
+        cc.v = pc.v;
+        CUtensorMap pq, pk, pv;
+        if (!make_maps(cc, T, &pq, &pk, &pv)) return cudaErrorInvalidValue;
+        auto kern = tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_NONE, true, Tout>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, CfP::SMEM);
+        if (e != cudaSuccess) return e;
+        kern<<<grid, CfP::THREADS, CfP::SMEM, s>>>(pq, pk, pv, as, hp);
+        return cudaGetLastError();
+      }
+    }
+    return run(tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_NONE, false, Tout>, 1);
+  }
+  if (max_states < 1) return run(tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_REPLAY, false, Tout>, as.n_seg);
   // Pre-pass: each of the first n_seg - 1 segments split into n_split sub-segments, as many
   // as the SMs, the workspace and two chunks a sub-segment allow.
   const int n_pre = as.n_seg - 1;
@@ -1735,9 +1857,9 @@ cudaError_t launch_pipe(const RetentionCall& c, const HeadParams& hp, cudaStream
   }
   as.n_sub = j;
   as.ws = static_cast<float*>(c.ws);
-  const cudaError_t e = run(tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_STATE, Tout>, as.n_sub);
+  const cudaError_t e = run(tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_STATE, false, Tout>, as.n_sub);
   if (e != cudaSuccess) return e;
-  return run(tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_FROM_WS, Tout>, as.n_seg);
+  return run(tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_FROM_WS, false, Tout>, as.n_seg);
 }
 
 // Serial kernel: one chunk of B = T rows per step (chunk-relative scaled operands).
@@ -1831,6 +1953,7 @@ int tc_chunkwise_launches(const RetentionCall& c) {
   TcArgs as = make_args(c, static_cast<int>((c.dims.seqlen + c.chunk - 1) / c.chunk), nb);
   const int64_t ctas = (c.dims.d_v / dvs) * c.dims.heads * c.dims.batch;
   const int max_states = plan_call(c, ctas, sm_count(), as);
+  if (dvs == 64 && pre_convert_applies(c, nb, as.n_seg)) return 2;  // conversion pre-pass + kernel
   return (as.n_seg > 1 && max_states >= 1) ? 2 : 1;
 }
 

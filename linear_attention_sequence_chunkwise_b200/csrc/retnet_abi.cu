@@ -217,9 +217,14 @@ retnet_status_t retnet_retention_chunkwise_static(const void* q, const void* k, 
 retnet_status_t retnet_chunkwise_workspace_size(retnet_dims_t dims, size_t* bytes) {
   if (!bytes) return RETNET_ERR_NULL_PTR;
   if (dims.batch < 0 || dims.seqlen < 0 || dims.heads < 0 || dims.d_k < 0 || dims.d_v < 0) return RETNET_ERR_BAD_SHAPE;
-  // Up to six pre-pass states, fp32 [6][batch][heads][d_k][d_v].
-  *bytes = 6 * sizeof(float) * static_cast<size_t>(dims.batch) * static_cast<size_t>(dims.heads) *
-           static_cast<size_t>(dims.d_k) * static_cast<size_t>(dims.d_v);
+  // The larger of its two uses (never both in one call): up to six segment states, fp32
+  // [6][batch][heads][d_k][d_v]; or the fp16 copies of q, k, v of the conversion pre-pass.
+  const size_t states = 6 * sizeof(float) * static_cast<size_t>(dims.batch) * static_cast<size_t>(dims.heads) *
+                        static_cast<size_t>(dims.d_k) * static_cast<size_t>(dims.d_v);
+  const size_t tok = static_cast<size_t>(dims.batch) * static_cast<size_t>(dims.seqlen) * static_cast<size_t>(dims.heads);
+  auto a256 = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  const size_t copies = 2 * a256(tok * static_cast<size_t>(dims.d_k) * 2) + a256(tok * static_cast<size_t>(dims.d_v) * 2);
+  *bytes = states > copies ? states : copies;
   return RETNET_OK;
 }
 

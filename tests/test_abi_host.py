@@ -119,7 +119,12 @@ def test_chunkwise_and_step_validation(lib):
 def test_chunkwise_workspace_entry_points(lib):
     """Workspace size is the documented bound; the workspace variant validates like the plain call
     and rejects a misaligned workspace before touching a device."""
-    assert rn.retnet_chunkwise_workspace_size((2, 100, 3, 128, 64)) == 6 * 2 * 3 * 128 * 64 * 4
+    a256 = lambda x: (x + 255) // 256 * 256
+    for dims in ((2, 100, 3, 128, 64), (1, 4096, 2, 64, 128)):
+        b, L, h, dk, dv = dims
+        states = 6 * b * h * dk * dv * 4
+        copies = 2 * a256(b * L * h * dk * 2) + a256(b * L * h * dv * 2)
+        assert rn.retnet_chunkwise_workspace_size(dims) == max(states, copies)
     assert rn.retnet_chunkwise_workspace_size((0, 0, 0, 0, 0)) == 0
     out = ctypes.c_size_t(0)
     assert lib.retnet_chunkwise_workspace_size(rn.Dims(1, 8, -2, 4, 4), ctypes.byref(out)) == 2
