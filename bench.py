@@ -237,12 +237,14 @@ def bench_long(rn, device, stream, steps, peaks):
     q, k, v = q.to(device), k.to(device), v.to(device)
     o = torch.empty(b, L, h, dv, dtype=torch.bfloat16, device=device)
     g, th = si.gamma_schedule(h), si.theta_schedule(dk)
-    out = {"workload": c["workload"]}
+    ws = torch.empty(rn.retnet_chunkwise_workspace_size((b, L, h, dk, dv)), dtype=torch.uint8, device=device)
+    out = {"workload": c["workload"], "workspace_bytes": ws.numel()}
     for B in (128, 512):
         path = rn.retnet_chunkwise_kernel((b, L, h, dk), dv, rn.BF16, FLAGS, B, g)
+        launches = rn.retnet_chunkwise_launches((b, L, h, dk), dv, rn.BF16, FLAGS, B, g, ws.numel())
 
         def step(i):
-            rn.retnet_retention_chunkwise(q, k, v, o, g, th, 0, FLAGS, B, stream=stream)
+            rn.retnet_retention_chunkwise_ws(q, k, v, o, g, th, 0, FLAGS, B, workspace=ws, stream=stream)
 
         for i in range(2):
             step(i)
@@ -253,7 +255,8 @@ def bench_long(rn, device, stream, steps, peaks):
         out[f"chunk{B}"] = {"us_per_step": secs * 1e6, "tokens_per_s": b * L / secs, "tflops": flops / secs / 1e12,
                             "frac_bf16_peak": flops / secs / 1e12 / peaks["bf16"], "gbs": byt / secs / 1e9,
                             "frac_hbm": byt / secs / 1e9 / peaks["hbm"],
-                            "kernel": "tcgen05" if path == 1 else "fp32 CUDA cores", "gpu_launches": steps}
+                            "kernel": "tcgen05" if path == 1 else "fp32 CUDA cores",
+                            "launches_per_step": launches, "gpu_launches": launches * steps}
     return out
 
 
@@ -271,9 +274,11 @@ def bench_msr(rn, device, stream, steps, peaks):
     out = torch.empty(b, L, h * dv, dtype=torch.bfloat16, device=device)
     g, th = si.gamma_schedule(h), si.theta_schedule(dk)
     path = rn.retnet_chunkwise_kernel((b, L, h, dk), dv, rn.BF16, FLAGS, B, g)
+    ws = torch.empty(rn.retnet_chunkwise_workspace_size((b, L, h, dk, dv)), dtype=torch.uint8, device=device)
+    launches = rn.retnet_chunkwise_launches((b, L, h, dk), dv, rn.BF16, FLAGS, B, g, ws.numel()) + 1
 
     def step(i):
-        rn.retnet_retention_chunkwise(q, k, v, y, g, th, 0, FLAGS, B, stream=stream)
+        rn.retnet_retention_chunkwise_ws(q, k, v, y, g, th, 0, FLAGS, B, workspace=ws, stream=stream)
         rn.retnet_msr_epilogue(y.view(b, L, h * dv), gt, out, h, 1e-5, stream)
 
     for i in range(2):
@@ -286,7 +291,7 @@ def bench_msr(rn, device, stream, steps, peaks):
             "tflops": flops / secs / 1e12, "frac_bf16_peak": flops / secs / 1e12 / peaks["bf16"],
             "gbs": byt / secs / 1e9, "frac_hbm": byt / secs / 1e9 / peaks["hbm"],
             "kernel": "tcgen05 + epilogue" if path == 1 else "fp32 CUDA cores + epilogue",
-            "gpu_launches": 2 * steps}
+            "workspace_bytes": ws.numel(), "launches_per_step": launches, "gpu_launches": launches * steps}
 
 
 def oracle_sample(cfg, budget_s):
