@@ -56,7 +56,8 @@ struct TcArgs {
   int n_chunks;
   int64_t pos0;
   uint32_t flags;
-  int nb;  // sub-blocks of T rows per chunk (pipelined kernel)
+  int nb;     // sub-blocks of T rows per chunk (pipelined kernel)
+  int batch;
   // Sequence segments (pipelined kernel): CTA segment s writes the outputs of chunks
   // [seg_lo[s], seg_hi[s]) and first replays the state over chunks [0, seg_lo[s]).
   int n_seg;
@@ -876,7 +877,11 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE>::THREADS, 1)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int n_dvb = a.dv / DVS;
-  const int dvb = SEG ? blockIdx.x % n_dvb : blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  // Grid: (slice [x segment], head, batch); the output pass of the two-pass form puts the
+  // segment in z instead (segment-major), so that its segment-0 CTAs, which do not need the
+  // pre-pass, are dispatched first.
+  const int dvb = (SEG && SM != SEG_FROM_WS) ? blockIdx.x % n_dvb : blockIdx.x, h = blockIdx.y;
+  const int b = (SM == SEG_FROM_WS) ? blockIdx.z % a.batch : blockIdx.z;
   const float log2g = hp.log2g[h];
   const int nb = a.nb;
   // The CTA visits chunks [c_first, c_hi); those below c_lo only update the state (the replay
@@ -884,6 +889,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE>::THREADS, 1)
   // Without segments the bounds are compile-time constants and every such branch folds away.
   int seg = 0, s_lo = 0, s_hi = 0x7fffffff;
   if constexpr (SM == SEG_STATE) {  // seg = the pre-pass sub-segment
+    griddep_launch_dependents();    // the output pass may start on the SMs this grid leaves idle
     seg = blockIdx.x / n_dvb;
     s_lo = a.sub_lo[0];
     s_hi = a.sub_hi[0];
@@ -894,7 +900,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE>::THREADS, 1)
         s_hi = a.sub_hi[i];
       }
   } else if constexpr (SEG) {
-    seg = blockIdx.x / n_dvb;
+    seg = (SM == SEG_FROM_WS) ? blockIdx.z / a.batch : blockIdx.x / n_dvb;
     s_lo = a.seg_lo[0];
     s_hi = a.seg_hi[0];
 #pragma unroll
@@ -924,6 +930,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE>::THREADS, 1)
 #pragma unroll
       for (int t = 1; t < 4; ++t)  // constant-index selects, as above
         if (t == seg) n_before = a.sub_before[t];
+      if (n_before > 0) griddep_wait();  // the pre-pass states are complete and visible
       for (int j = 0; j < n_before; ++j) {
         int chunks_j = 0;
 #pragma unroll
@@ -931,7 +938,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE>::THREADS, 1)
           if (t == j) chunks_j = a.sub_hi[t] - a.sub_lo[t];
         const int len_j = chunks_j * nb * T;
         const float gl = exp2f(static_cast<float>(len_j) * log2g);
-        const size_t plane = static_cast<size_t>(gridDim.z) * a.heads * DK * a.dv;
+        const size_t plane = static_cast<size_t>(a.batch) * a.heads * DK * a.dv;
         const float* w = a.ws + j * plane + static_cast<size_t>(bh) * DK * a.dv + col + static_cast<size_t>(dk) * a.dv;
         for (int c4 = 0; c4 < n / 4; ++c4) {
           const float4 x = *reinterpret_cast<const float4*>(w + 4 * c4);
@@ -1203,7 +1210,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE>::THREADS, 1)
       const uint32_t lane_off = static_cast<uint32_t>(32 * (warp % 4)) << 16;
       if (__all_sync(0xffffffffu, mbar_wait(bar(Q_DR_FULL + 0), 0))) {
         tc_fence_after();
-        const size_t plane = static_cast<size_t>(gridDim.z) * a.heads * DK * a.dv;
+        const size_t plane = static_cast<size_t>(a.batch) * a.heads * DK * a.dv;
 #pragma unroll 1
         for (int bk = 0; bk < C::BPT; ++bk) {
           const int blk = C::BPT > 1 ? bk : (warp - C::WARP_S0) / 4 % C::RBLK;
@@ -1760,6 +1767,7 @@ TcArgs make_args(const RetentionCall& c, int n_chunks, int nb) {
   a.state_out = c.state_out;
   a.L = static_cast<int>(c.dims.seqlen);
   a.heads = static_cast<int>(c.dims.heads);
+  a.batch = static_cast<int>(c.dims.batch);
   a.dv = static_cast<int>(c.dims.d_v);
   a.n_chunks = n_chunks;
   a.pos0 = c.pos0;
@@ -1857,9 +1865,25 @@ cudaError_t launch_pipe(const RetentionCall& c, const HeadParams& hp, cudaStream
   }
   as.n_sub = j;
   as.ws = static_cast<float*>(c.ws);
-  const cudaError_t e = run(tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_STATE, false, Tout>, as.n_sub);
+  cudaError_t e = run(tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_STATE, false, Tout>, as.n_sub);
   if (e != cudaSuccess) return e;
-  return run(tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_FROM_WS, false, Tout>, as.n_seg);
+  // Output pass, launched as a programmatic dependent of the pre-pass (segment-major grid):
+  // its segment-0 CTAs run on the SMs the pre-pass leaves idle; later segments wait on the
+  // device (griddepcontrol.wait) before they read the pre-pass states.
+  auto kern = tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_FROM_WS, false, Tout>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid.x, grid.y, grid.z * as.n_seg);
+  cfg.blockDim = dim3(Cf::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = Cf::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, as, hp);
 }
 
 // Serial kernel: one chunk of B = T rows per step (chunk-relative scaled operands).

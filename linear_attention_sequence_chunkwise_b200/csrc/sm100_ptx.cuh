@@ -47,6 +47,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Count of bounded waits that gave up in kernels of the including file (a kernel that hits
 // one stops its work, releases what it holds and returns; the host reads and clears it).
+// Programmatic dependent launch: let the grid launched after this one (with the
+// programmatic-serialization attribute) start; and, in that grid, wait until the grid before
+// it has completed and its memory writes are visible.
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Non-blocking probe of an mbarrier phase.
 __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   uint32_t ok;
