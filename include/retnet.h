@@ -167,6 +167,30 @@ RETNET_API retnet_status_t retnet_retention_chunkwise_ws(const void* q, const vo
                                               size_t workspace_bytes, void* stream);
 
 /*
+ * Sequence sharding (§2.4 read as an associative scan over chunks; sequence-parallel use
+ * across GPUs).  The state a sequence leaves behind from a zero start,
+ *   W = sum_t gamma^(L-1-t) rot_{pos0+t}(k_t)^T v_t      -> state_out [batch][heads][d_k][d_v] fp32,
+ * without outputs (q is not needed).  A shard of a longer sequence starting at position pos0
+ * contributes W; the state after it is gamma^L R_before + W (retnet_state_advance).  Runs the
+ * tensor-core state pass: the shapes and dtypes of the tensor-core chunkwise kernel (bf16,
+ * no RETNET_F_NORM_R), else RETNET_ERR_UNSUPPORTED.  k, v as for retnet_retention_chunkwise.
+ */
+RETNET_API retnet_status_t retnet_chunkwise_segment_state(const void* k, const void* v, retnet_dims_t dims,
+                                               retnet_dtype_t in_dtype, const float* gamma,
+                                               const float* theta, int64_t pos0, uint32_t flags,
+                                               int64_t chunk, float* state_out, void* stream);
+
+/*
+ * state <- gamma_h^len * state + w, in place, for fp32 [batch][heads][d_k][d_v] states (the
+ * combination step of a sequence split into shards: R after a shard of len tokens whose own
+ * state is w).  gamma: host float[heads]; gamma^len is taken in fp64.  state and w 16-byte
+ * aligned, d_k * d_v a multiple of 4; they may not overlap unless equal.
+ */
+RETNET_API retnet_status_t retnet_state_advance(float* state, const float* w, int64_t batch, int64_t heads,
+                                     int64_t d_k, int64_t d_v, const float* gamma, int64_t len,
+                                     void* stream);
+
+/*
  * Allocation-free variant of retnet_retention_chunkwise_ws.  The pages have no counterpart:
  * it is the same computation with the segment states kept in a static device array of
  * RETNET_STATIC_SCRATCH_BYTES inside the library (one per device), for callers that cannot

@@ -32,7 +32,7 @@ STATUS = {0: "RETNET_OK", 1: "RETNET_ERR_NULL_PTR", 2: "RETNET_ERR_BAD_SHAPE", 3
           4: "RETNET_ERR_BAD_PARAM", 5: "RETNET_ERR_UNSUPPORTED", 6: "RETNET_ERR_CUDA"}
 STATIC_SCRATCH_BYTES = 16 << 20  # RETNET_STATIC_SCRATCH_BYTES
 EXPORTS = ("retnet_retention_parallel", "retnet_retention_chunkwise", "retnet_retention_chunkwise_ws",
-           "retnet_retention_chunkwise_static",
+           "retnet_retention_chunkwise_static", "retnet_chunkwise_segment_state", "retnet_state_advance",
            "retnet_chunkwise_workspace_size", "retnet_retention_step", "retnet_msr_epilogue",
            "retnet_chunkwise_kernel", "retnet_chunkwise_launches", "retnet_debug_wait_timeouts",
            "retnet_status_string", "retnet_version")
@@ -74,6 +74,10 @@ def load(path: str = None):
                                                   _i64, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
     lib.retnet_retention_chunkwise_static.argtypes = [_vp, _vp, _vp, _vp, Dims, _i32, _i32, _fp, _fp, _i64, _u32,
                                                       _i64, _vp, _vp, _vp, _vp, _vp]
+    lib.retnet_chunkwise_segment_state.argtypes = [_vp, _vp, Dims, _i32, _fp, _fp, _i64, _u32, _i64, _vp, _vp]
+    lib.retnet_chunkwise_segment_state.restype = _i32
+    lib.retnet_state_advance.argtypes = [_vp, _vp, _i64, _i64, _i64, _i64, _fp, _i64, _vp]
+    lib.retnet_state_advance.restype = _i32
     lib.retnet_chunkwise_workspace_size.argtypes = [Dims, ctypes.POINTER(ctypes.c_size_t)]
     lib.retnet_chunkwise_workspace_size.restype = _i32
     lib.retnet_retention_step.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _fp,
@@ -219,6 +223,31 @@ def retnet_retention_chunkwise_static(q, k, v, o, gamma, theta=None, pos0=0, fla
                                                     _dtype_code(o), _fptr(g), _fptr(th), int(pos0), int(flags),
                                                     int(chunk), _ptr(state_in), _ptr(state_out), _ptr(z_in),
                                                     _ptr(z_out), _stream(stream)))
+
+
+def retnet_chunkwise_segment_state(k, v, state_out, gamma, theta=None, pos0=0, flags=F_ALL, chunk=64, stream=None):
+    """State a sequence's chunks leave behind from a zero start (no outputs): k (b,L,h,d_k),
+    v (b,L,h,d_v) bf16; state_out (b,h,d_k,d_v) float32."""
+    _require_cuda(k, v, state_out)
+    b, L, h, dk = k.shape
+    dv = v.shape[-1]
+    if tuple(v.shape) != (b, L, h, dv) or tuple(state_out.shape) != (b, h, dk, dv):
+        raise ValueError("shape mismatch between k, v, state_out")
+    g = _host_f32(gamma, h)
+    th = _host_f32(theta, dk // 2)
+    _check(load().retnet_chunkwise_segment_state(_ptr(k), _ptr(v), Dims(b, L, h, dk, dv), _dtype_code(k), _fptr(g),
+                                                 _fptr(th), int(pos0), int(flags), int(chunk), _ptr(state_out),
+                                                 _stream(stream)))
+
+
+def retnet_state_advance(state, w, gamma, length, stream=None):
+    """state <- gamma^length * state + w in place (both (b,h,d_k,d_v) float32 CUDA tensors)."""
+    _require_cuda(state, w)
+    b, h, dk, dv = state.shape
+    if tuple(w.shape) != (b, h, dk, dv):
+        raise ValueError("state and w must have the same shape")
+    g = _host_f32(gamma, h)
+    _check(load().retnet_state_advance(_ptr(state), _ptr(w), b, h, dk, dv, _fptr(g), int(length), _stream(stream)))
 
 
 def retnet_retention_chunkwise(q, k, v, o, gamma, theta=None, pos0=0, flags=F_ALL, chunk=64, state_in=None,

@@ -1969,6 +1969,68 @@ cudaError_t tc_wait_timeouts(unsigned int* count, bool clear) {
   return cudaMemcpyToSymbol(sm100::g_wait_timeouts, &zero, sizeof(unsigned int));
 }
 
+namespace {
+template <int DK, int T, typename Tout>
+cudaError_t launch_segment_state_t(const RetentionCall& c, const HeadParams& hp, cudaStream_t s) {
+  using Cf = Cfg3<DK, T, 64>;
+  CUtensorMap mq, mk, mv;
+  // The state pass never loads Q: its map is built over K (a valid tensor of the same shape).
+  RetentionCall cc = c;
+  cc.q = c.k;
+  if (!make_maps(cc, T, &mq, &mk, &mv)) return cudaErrorInvalidValue;
+  const int nb = static_cast<int>(c.chunk / T);
+  const int n_chunks = static_cast<int>((c.dims.seqlen + c.chunk - 1) / c.chunk);
+  TcArgs a = make_args(c, n_chunks, nb);
+  a.n_seg = 1;
+  a.n_sub = 1;
+  a.sub_lo[0] = 0;
+  a.sub_hi[0] = n_chunks;
+  a.ws = c.state_out;  // sub-segment 0 of the workspace layout is [batch][heads][d_k][d_v]
+  auto kern = tc_chunkwise_pipe_kernel<DK, T, 64, SEG_STATE, false, Tout>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM);
+  if (e != cudaSuccess) return e;
+  kern<<<tc_grid(c.dims, 64), Cf::THREADS, Cf::SMEM, s>>>(mq, mk, mv, a, hp);
+  return cudaGetLastError();
+}
+
+template <int DK>
+cudaError_t launch_segment_state_dk(const RetentionCall& c, const HeadParams& hp, cudaStream_t s) {
+  if (pipe_tile_rows(DK, c.chunk) == 64) return launch_segment_state_t<DK, 64, __nv_bfloat16>(c, hp, s);
+  if constexpr (DK != 256) return launch_segment_state_t<DK, 128, __nv_bfloat16>(c, hp, s);
+  return cudaErrorInvalidValue;
+}
+
+// state <- gamma_h^len * state + w over [batch][heads][d_k][d_v] (fp32, float4 per thread).
+__global__ void state_advance_kernel(float4* __restrict__ state, const float4* __restrict__ w, int64_t n4,
+                                     int64_t per_head4, int heads, HeadParams hp) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float f = hp.gamma[static_cast<int>((i / per_head4) % heads)];
+    const float4 x = state[i], y = w[i];
+    state[i] = make_float4(fmaf(f, x.x, y.x), fmaf(f, x.y, y.y), fmaf(f, x.z, y.z), fmaf(f, x.w, y.w));
+  }
+}
+}  // namespace
+
+cudaError_t launch_tc_segment_state(const RetentionCall& c, const HeadParams& hp, cudaStream_t s) {
+  switch (c.dims.d_k) {
+    case 64: return launch_segment_state_dk<64>(c, hp, s);
+    case 128: return launch_segment_state_dk<128>(c, hp, s);
+    default: return launch_segment_state_dk<256>(c, hp, s);
+  }
+}
+
+// hp.gamma carries gamma_h^len per head here (computed on the host in fp64).
+cudaError_t launch_state_advance(float* state, const float* w, const Dims& d, const HeadParams& hp, cudaStream_t s) {
+  const int64_t n4 = d.batch * d.heads * d.d_k * d.d_v / 4;
+  if (n4 == 0) return cudaSuccess;
+  const int64_t per_head4 = d.d_k * d.d_v / 4;
+  const int blocks = static_cast<int>(std::min<int64_t>((n4 + 255) / 256, 148 * 8));
+  state_advance_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<float4*>(state), reinterpret_cast<const float4*>(w),
+                                              n4, per_head4, static_cast<int>(d.heads), hp);
+  return cudaGetLastError();
+}
+
 int tc_chunkwise_launches(const RetentionCall& c) {
   if (force_serial_kernel()) return 1;
   const int T = pipe_tile_rows(c.dims.d_k, c.chunk);

@@ -42,6 +42,11 @@ bool tc_driver_ready();
 cudaError_t launch_tc_chunkwise(const RetentionCall& c, const HeadParams& hp, cudaStream_t s);
 // Kernel launches launch_tc_chunkwise makes for this call on the current device (1 or 2).
 int tc_chunkwise_launches(const RetentionCall& c);
+// The state a sequence's chunks leave behind from a zero start, into c.state_out (tensor-core
+// shapes only; q is not read).
+cudaError_t launch_tc_segment_state(const RetentionCall& c, const HeadParams& hp, cudaStream_t s);
+// state <- g_h * state + w, g_h = hp.gamma[h] (fp32 [batch][heads][d_k][d_v], d_k*d_v % 4 == 0).
+cudaError_t launch_state_advance(float* state, const float* w, const Dims& d, const HeadParams& hp, cudaStream_t s);
 // Reads (and optionally clears) the count of bounded waits that gave up in the tensor-core kernel.
 cudaError_t tc_wait_timeouts(unsigned int* count, bool clear);
 

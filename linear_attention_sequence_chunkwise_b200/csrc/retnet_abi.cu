@@ -228,6 +228,49 @@ retnet_status_t retnet_chunkwise_workspace_size(retnet_dims_t dims, size_t* byte
   return RETNET_OK;
 }
 
+retnet_status_t retnet_chunkwise_segment_state(const void* k, const void* v, retnet_dims_t dims,
+                                               retnet_dtype_t in_dtype, const float* gamma, const float* theta,
+                                               int64_t pos0, uint32_t flags, int64_t chunk, float* state_out,
+                                               void* stream) {
+  retnet_status_t st = check_common(dims, in_dtype, RETNET_F32, pos0, flags, true);
+  if (st != RETNET_OK) return st;
+  if (chunk <= 0) return RETNET_ERR_BAD_PARAM;
+  if (!state_out) return RETNET_ERR_NULL_PTR;
+  if (dims.seqlen > 0 && (!k || !v)) return RETNET_ERR_NULL_PTR;
+  HeadParams hp;
+  if ((st = fill_params(&hp, gamma, theta, dims.heads, dims.d_k, flags)) != RETNET_OK) return st;
+  if ((st = check_device()) != RETNET_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dims.seqlen == 0) {
+    const size_t sbytes = sizeof(float) * static_cast<size_t>(dims.batch * dims.heads * dims.d_k * dims.d_v);
+    return cudaMemsetAsync(state_out, 0, sbytes, s) == cudaSuccess ? RETNET_OK : RETNET_ERR_CUDA;
+  }
+  // q is not read; k stands in for it so that the shape checks see three valid tensors.
+  RetentionCall c{k, k, v, state_out, Dims{dims.batch, dims.seqlen, dims.heads, dims.d_k, dims.d_v}, in_dtype,
+                  RETNET_F32, pos0, flags, chunk, true, nullptr, state_out, nullptr, nullptr};
+  if (!tc_chunkwise_supported(c) || !tc_chunkwise_heads_ok(c, hp)) return RETNET_ERR_UNSUPPORTED;
+  if (!tc_driver_ready()) return RETNET_ERR_CUDA;
+  return from_cuda(launch_tc_segment_state(c, hp, s));
+}
+
+retnet_status_t retnet_state_advance(float* state, const float* w, int64_t batch, int64_t heads, int64_t d_k,
+                                     int64_t d_v, const float* gamma, int64_t len, void* stream) {
+  if (!state || !w || !gamma) return RETNET_ERR_NULL_PTR;
+  if (batch < 0 || heads <= 0 || d_k <= 0 || d_v <= 0 || heads > RETNET_MAX_HEADS) return RETNET_ERR_BAD_SHAPE;
+  if ((d_k * d_v) % 4 != 0) return RETNET_ERR_BAD_SHAPE;
+  if (len < 0) return RETNET_ERR_BAD_PARAM;
+  if ((reinterpret_cast<uintptr_t>(state) & 15u) || (reinterpret_cast<uintptr_t>(w) & 15u)) return RETNET_ERR_BAD_PARAM;
+  HeadParams hp;
+  for (int64_t h = 0; h < heads; ++h) {
+    const double g = gamma[h];
+    if (!(g > 0.0 && g < 1.0)) return RETNET_ERR_BAD_PARAM;
+    hp.gamma[h] = static_cast<float>(exp(static_cast<double>(len) * log(g)));  // gamma^len in fp64
+  }
+  retnet_status_t st = check_device();
+  if (st != RETNET_OK) return st;
+  return from_cuda(launch_state_advance(state, w, Dims{batch, 0, heads, d_k, d_v}, hp, static_cast<cudaStream_t>(stream)));
+}
+
 int retnet_chunkwise_launches(retnet_dims_t dims, retnet_dtype_t in_dtype, uint32_t flags, int64_t chunk,
                               const float* gamma, size_t workspace_bytes) {
   const int path = retnet_chunkwise_kernel(dims, in_dtype, flags, chunk, gamma);

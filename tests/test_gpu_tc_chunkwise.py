@@ -143,6 +143,38 @@ def test_tc_preconverted(dk, dv, B, L, with_state):
     assert err(so, Sref) <= TOL_BF16
 
 
+@pytest.mark.parametrize("case", ["dv1024", "pos0_large", "one_token_ws", "gamma_near_one"])
+def test_tc_edge_cases(case):
+    """Widest value dimension (16 slices), an xPos position near 2^26 (where an fp32 angle is
+    off by radians: the kernel reduces p * theta in fp64; the oracle's D~ prefix is a plain
+    O(pos0) sum, which bounds how far this can go),
+    a single-token call through the workspace form, and heads up to gamma = 1 - 2^-24 (the
+    largest fp32 below 1)."""
+    b, L, h, dk, dv, B, pos0 = 1, 300, 2, 128, 64, 64, 0
+    if case == "dv1024":
+        dv = 1024
+    elif case == "pos0_large":
+        pos0 = (1 << 26) + 12345
+    elif case == "one_token_ws":
+        L = 1
+    elif case == "gamma_near_one":
+        h, L = 20, 150
+    q, k, v = si.qkv(b, L, h, dk, dv, 120, "bf16")
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+    assert rn.retnet_chunkwise_kernel((b, L, h, dk), dv, rn.BF16, FLAGS, B, g) == 1
+    S0 = si.decode_state(b, h, dk, dv, 121, std=0.2)
+    ref, Sref, _ = oracle.recurrent(q, k, v, g, th, pos0, FLAGS, S0)
+    o = torch.empty(b, L, h, dv, device="cuda")
+    so = torch.empty(b, h, dk, dv, device="cuda")
+    ws = torch.empty(rn.retnet_chunkwise_workspace_size((b, L, h, dk, dv)), dtype=torch.uint8, device="cuda")
+    rn.retnet_retention_chunkwise_ws(dev(q), dev(k), dev(v), o, g, th, pos0, FLAGS, B, dev(S0), so, workspace=ws)
+    torch.cuda.synchronize()
+    e = err(o, ref)
+    print(f"edge {case}: max|err|/rms = {e:.3e}")
+    assert e <= TOL_BF16
+    assert err(so, Sref) <= TOL_BF16
+
+
 def test_tc_launch_count():
     """The launch-count query follows the plan: two launches only for the workspace form with
     segments (few (batch, head) pairs), one otherwise."""
