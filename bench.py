@@ -261,7 +261,9 @@ def bench_long(rn, device, stream, steps, peaks):
 
 
 def bench_msr(rn, device, stream, steps, peaks):
-    """MSR forward: chunkwise retention (chunk 256, bf16 out) then GroupNorm + swish gate."""
+    """MSR forward (chunk 256, bf16 out): the fused kernel (retention, GroupNorm and swish gate
+    in one tensor-core kernel per cluster of d_v slices), and beside it the two-kernel form
+    (chunkwise retention to HBM, then the GroupNorm + gate kernel)."""
     import torch
 
     import synth_inputs as si
@@ -275,23 +277,35 @@ def bench_msr(rn, device, stream, steps, peaks):
     g, th = si.gamma_schedule(h), si.theta_schedule(dk)
     path = rn.retnet_chunkwise_kernel((b, L, h, dk), dv, rn.BF16, FLAGS, B, g)
     ws = torch.empty(rn.retnet_chunkwise_workspace_size((b, L, h, dk, dv)), dtype=torch.uint8, device=device)
-    launches = rn.retnet_chunkwise_launches((b, L, h, dk), dv, rn.BF16, FLAGS, B, g, ws.numel()) + 1
+    two_launches = rn.retnet_chunkwise_launches((b, L, h, dk), dv, rn.BF16, FLAGS, B, g, ws.numel()) + 1
+    fused_launches = rn.retnet_msr_chunkwise_launches((b, L, h, dk), dv, rn.BF16, FLAGS, B, g, ws.numel())
 
-    def step(i):
+    def two_kernel(i):
         rn.retnet_retention_chunkwise_ws(q, k, v, y, g, th, 0, FLAGS, B, workspace=ws, stream=stream)
         rn.retnet_msr_epilogue(y.view(b, L, h * dv), gt, out, h, 1e-5, stream)
 
-    for i in range(2):
-        step(i)
-    torch.cuda.synchronize()
-    secs = time_steps(step, steps, stream) / steps
+    def fused(i):
+        rn.retnet_msr_chunkwise(q, k, v, gt.view(b, L, h, dv), out.view(b, L, h, dv), g, th, 0, FLAGS, B, 1e-5,
+                                workspace=ws, stream=stream)
+
     flops = b * L * h * flops_per_token_head(dk, dv, B)
-    byt = b * L * h * (bytes_per_token_head(dk, dv) + 2 * dv * 2 + 2 * dv)  # + y re-read, g, out
-    return {"workload": c["workload"], "us_per_step": secs * 1e6, "tokens_per_s": b * L / secs,
-            "tflops": flops / secs / 1e12, "frac_bf16_peak": flops / secs / 1e12 / peaks["bf16"],
-            "gbs": byt / secs / 1e9, "frac_hbm": byt / secs / 1e9 / peaks["hbm"],
-            "kernel": "tcgen05 + epilogue" if path == 1 else "fp32 CUDA cores + epilogue",
-            "workspace_bytes": ws.numel(), "launches_per_step": launches, "gpu_launches": launches * steps}
+    res = {"workload": c["workload"], "workspace_bytes": ws.numel()}
+    legs = [("two_kernel", two_kernel, two_launches, 4 * dv, "tcgen05 + epilogue" if path == 1 else
+             "fp32 CUDA cores + epilogue")]
+    if fused_launches > 0:
+        legs.insert(0, ("fused", fused, fused_launches, 2 * dv, "tcgen05, fused GroupNorm + gate"))
+    for name, fn, launches, extra, kernel in legs:
+        for i in range(2):
+            fn(i)
+        torch.cuda.synchronize()
+        secs = time_steps(fn, steps, stream) / steps
+        # algorithmic bytes: q, k, v, out (+ the gate; the two-kernel form also re-reads y and writes out)
+        byt = b * L * h * (bytes_per_token_head(dk, dv) + extra)
+        res[name] = {"us_per_step": secs * 1e6, "tokens_per_s": b * L / secs, "tflops": flops / secs / 1e12,
+                     "frac_bf16_peak": flops / secs / 1e12 / peaks["bf16"], "gbs": byt / secs / 1e9,
+                     "frac_hbm": byt / secs / 1e9 / peaks["hbm"], "kernel": kernel, "launches_per_step": launches,
+                     "gpu_launches": launches * steps}
+    return res
 
 
 def oracle_sample(cfg, budget_s):

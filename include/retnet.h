@@ -252,6 +252,31 @@ RETNET_API retnet_status_t retnet_msr_epilogue(const void* y, const void* g, voi
                                     retnet_dtype_t out_dtype, void* stream);
 
 /*
+ * Chunkwise retention with the MSR epilogue (§三.2) fused into the tensor-core kernel:
+ *   out = swish(g) (.) GroupNorm_h(o),  o the output retnet_retention_chunkwise_ws would write,
+ * with the GroupNorm of retnet_msr_epilogue (per (token, head) row of d_v values, biased
+ * variance, eps >= 0 inside the root, unit affine).  The retention output itself is never
+ * written to memory: the d_v / 64 CTAs of a (batch, head) form one thread-block cluster and
+ * pool each row's statistics in distributed shared memory.
+ *   q, k, v, state_in, state_out, gamma, theta, pos0, flags, chunk, workspace: as for
+ *   retnet_retention_chunkwise_ws (the workspace only feeds the conversion pre-pass of chunks
+ *   of several sub-blocks; sequences are never split into segments here).
+ *   g:   gate [batch][seqlen][heads][d_v] in_dtype, 16-byte aligned;
+ *   out: [batch][seqlen][heads][d_v] out_dtype, must not overlap q, k, v or g.
+ * Handled: what the tensor-core kernel handles (retnet_chunkwise_kernel == 1: bf16 inputs,
+ * d_k in {64, 128, 256}, no RETNET_F_NORM_R, ...) with d_v in {64, 128, 192, 256}.
+ * Anything else returns RETNET_ERR_UNSUPPORTED without touching the device; run
+ * retnet_retention_chunkwise_ws then retnet_msr_epilogue for those.  seqlen == 0 copies
+ * state_in to state_out (or clears it) as the other chunkwise entry points do.
+ */
+RETNET_API retnet_status_t retnet_msr_chunkwise(const void* q, const void* k, const void* v, const void* g,
+                                     void* out, retnet_dims_t dims, retnet_dtype_t in_dtype,
+                                     retnet_dtype_t out_dtype, const float* gamma, const float* theta,
+                                     int64_t pos0, uint32_t flags, int64_t chunk, float eps,
+                                     const float* state_in, float* state_out, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+
+/*
  * Which kernel retnet_retention_chunkwise runs for these arguments (host-only decision, no
  * device access): 1 = the tcgen05 tensor-core kernel, 0 = the fp32 CUDA-core kernel,
  * negative = the arguments would be rejected (the negated status).  Device pointers that
@@ -271,6 +296,16 @@ RETNET_API int retnet_chunkwise_kernel(retnet_dims_t dims, retnet_dtype_t in_dty
  */
 RETNET_API int retnet_chunkwise_launches(retnet_dims_t dims, retnet_dtype_t in_dtype, uint32_t flags, int64_t chunk,
                                          const float* gamma, size_t workspace_bytes);
+
+/*
+ * Kernel launches retnet_msr_chunkwise makes for these arguments on the current device: 0
+ * without tokens, 1 (the fused kernel), 2 (conversion pre-pass + fused kernel, for chunks of
+ * several sub-blocks when workspace_bytes covers the fp16 copies); negative = the negated
+ * status the call would return (-RETNET_ERR_UNSUPPORTED for shapes it does not handle).
+ * Same assumptions as retnet_chunkwise_launches.
+ */
+RETNET_API int retnet_msr_chunkwise_launches(retnet_dims_t dims, retnet_dtype_t in_dtype, uint32_t flags,
+                                             int64_t chunk, const float* gamma, size_t workspace_bytes);
 
 /*
  * Number of bounded waits that gave up inside the tensor-core kernel since the last clear

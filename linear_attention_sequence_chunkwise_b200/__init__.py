@@ -10,6 +10,7 @@ The functions carry the C names:
   retnet_retention_chunkwise  -- §2.4 Chunkwise Recurrent Mode
   retnet_retention_step       -- §2.2 Recurrent Mode, one decode token for a batch
   retnet_msr_epilogue         -- §三.2 GroupNorm per head, then the swish gate
+  retnet_msr_chunkwise        -- §2.4 and §三.2 in one kernel (the retention output stays on chip)
 with the §三.3 normalisations chosen by flags.  Tensors are dense BLHD (see the header).
 """
 import ctypes
@@ -34,6 +35,7 @@ STATIC_SCRATCH_BYTES = 16 << 20  # RETNET_STATIC_SCRATCH_BYTES
 EXPORTS = ("retnet_retention_parallel", "retnet_retention_chunkwise", "retnet_retention_chunkwise_ws",
            "retnet_retention_chunkwise_static", "retnet_chunkwise_segment_state", "retnet_state_advance",
            "retnet_chunkwise_workspace_size", "retnet_retention_step", "retnet_msr_epilogue",
+           "retnet_msr_chunkwise", "retnet_msr_chunkwise_launches",
            "retnet_chunkwise_kernel", "retnet_chunkwise_launches", "retnet_debug_wait_timeouts",
            "retnet_status_string", "retnet_version")
 
@@ -83,8 +85,13 @@ def load(path: str = None):
     lib.retnet_retention_step.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _fp,
                                           _fp, _i64, _u32, _vp]
     lib.retnet_msr_epilogue.argtypes = [_vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_float, _i32, _i32, _vp]
+    lib.retnet_msr_chunkwise.argtypes = [_vp, _vp, _vp, _vp, _vp, Dims, _i32, _i32, _fp, _fp, _i64, _u32, _i64,
+                                         ctypes.c_float, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+    lib.retnet_msr_chunkwise_launches.argtypes = [Dims, _i32, _u32, _i64, _fp, ctypes.c_size_t]
+    lib.retnet_msr_chunkwise_launches.restype = _i32
     for name in ("retnet_retention_parallel", "retnet_retention_chunkwise", "retnet_retention_chunkwise_ws",
-                 "retnet_retention_chunkwise_static", "retnet_retention_step", "retnet_msr_epilogue"):
+                 "retnet_retention_chunkwise_static", "retnet_retention_step", "retnet_msr_epilogue",
+                 "retnet_msr_chunkwise"):
         getattr(lib, name).restype = _i32
     lib.retnet_chunkwise_kernel.argtypes = [Dims, _i32, _u32, _i64, _fp]
     lib.retnet_chunkwise_kernel.restype = _i32
@@ -293,12 +300,37 @@ def retnet_msr_epilogue(y, g, out, heads, eps=1e-5, stream=None):
     _require_cuda(y, g, out)
     if tuple(g.shape) != tuple(y.shape) or tuple(out.shape) != tuple(y.shape):
         raise ValueError("y, g and out must have one shape")
+    if g.dtype != y.dtype:
+        raise ValueError("y and g must have one dtype (the C call reads both as in_dtype)")
     total = y.numel()
     last = y.shape[-1]
     dv = last if (y.dim() >= 2 and y.shape[-2] == heads) else last // heads
     tokens = total // (heads * dv)
     _check(load().retnet_msr_epilogue(_ptr(y), _ptr(g), _ptr(out), tokens, heads, dv, float(eps), _dtype_code(y),
                                       _dtype_code(out), _stream(stream)))
+
+
+def retnet_msr_chunkwise(q, k, v, g, out, gamma, theta=None, pos0=0, flags=F_XPOS | F_SCALE_SQRT_D | F_NORM_D,
+                         chunk=64, eps=1e-5, state_in=None, state_out=None, workspace=None, stream=None):
+    """swish(g) (.) GroupNorm_h(chunkwise retention) into ``out`` in one fused kernel: q,k (b,L,h,d_k),
+    v,g,out (b,L,h,d_v); raises with RETNET_ERR_UNSUPPORTED for shapes the fused kernel does not take."""
+    d, gm, th = _chunkwise_args(q, k, v, out, gamma, theta, state_in, state_out, None, None)
+    _require_cuda(g, workspace)
+    if tuple(g.shape) != tuple(v.shape) or g.dtype != q.dtype:
+        raise ValueError("g must have the shape of v and the dtype of q")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().retnet_msr_chunkwise(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(out), d, _dtype_code(q),
+                                       _dtype_code(out), _fptr(gm), _fptr(th), int(pos0), int(flags), int(chunk),
+                                       float(eps), _ptr(state_in), _ptr(state_out), _ptr(workspace), ws_bytes,
+                                       _stream(stream)))
+
+
+def retnet_msr_chunkwise_launches(shape_qk, d_v, in_dtype, flags, chunk, gamma, workspace_bytes=0):
+    """Kernel launches retnet_msr_chunkwise makes (negative: the negated status it would return)."""
+    b, L, h, dk = shape_qk
+    gm = _host_f32(gamma, h)
+    return load().retnet_msr_chunkwise_launches(Dims(b, L, h, dk, d_v), int(in_dtype), int(flags), int(chunk),
+                                                _fptr(gm), int(workspace_bytes))
 
 
 def retnet_chunkwise_kernel(shape_qk, d_v, in_dtype, flags, chunk, gamma):

@@ -45,6 +45,7 @@ constexpr int kWarpMma = 9;
 constexpr int kDVS = 64;  // d_v slice per CTA
 
 constexpr int kMaxSub = 6;  // pre-pass states of the two-pass form (workspace capacity)
+constexpr int kMaxCluster = 4;  // d_v slices a fused GroupNorm epilogue combines (d_v <= 256)
 
 struct TcArgs {
   void* o;
@@ -58,6 +59,9 @@ struct TcArgs {
   uint32_t flags;
   int nb;     // sub-blocks of T rows per chunk (pipelined kernel)
   int batch;
+  // Fused MSR epilogue: out = GroupNorm_h(o) * swish(gate), written to o's place.
+  const void* gate;
+  float eps;
   // Sequence segments (pipelined kernel): CTA segment s writes the outputs of chunks
   // [seg_lo[s], seg_hi[s]) and first replays the state over chunks [0, seg_lo[s]).
   int n_seg;
@@ -589,7 +593,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 //   1 warp TMA, 1 warp MMA issuer (one unit ahead: S and dR of unit k+1 before X/PV of unit k).
 // ============================================================================================
 
-template <int DK, int T, int DVS, bool PRE = false>
+template <int DK, int T, int DVS, bool PRE = false, bool FUSE = false>
 struct Cfg3 {
   static constexpr int NDV = DVS / 64;              // 64-column boxes of the d_v slice
   static constexpr int RBLK = DK > 128 ? 2 : 1;     // 128-row blocks of the state increment
@@ -628,10 +632,13 @@ struct Cfg3 {
   static constexpr int TMEM_COLS = USED <= 128 ? 128 : (USED <= 256 ? 256 : 512);
   // shared memory: stages, P[PBUF], R16[RBUF], rotation tables (Q and K, double-buffered),
   // barriers.  A second fp16 state buffer is kept only while three stages still fit.
-  static constexpr int NBARS = 3 * 4 + 2 * 10 + 2;
+  static constexpr int NBARS = 3 * 4 + 2 * 10 + 1 + 2 + 2;
+  // FUSE (GroupNorm + gate in the epilogue): per-row (mean, M2) of every CTA of the cluster
+  // (the d_v slices of a head, at most kMaxCluster), double-buffered by row block.
+  static constexpr int XBYTES = FUSE ? 2 * kMaxCluster * T * 8 : 0;
   static constexpr int TABBYTES = 2 * 2 * (DK / 2) * 8;
   static constexpr int BUDGET = 227 * 1024 - 1024;
-  static constexpr int TAIL = TABBYTES + NBARS * 8 + 16;
+  static constexpr int TAIL = TABBYTES + NBARS * 8 + 16 + XBYTES;
   static constexpr int PBUF = (2 * STAGE + 2 * PBYTES + RBYTES + TAIL <= BUDGET) ? 2 : 1;
   static constexpr int NS_R2 = (BUDGET - (PBUF * PBYTES + 2 * RBYTES + TAIL)) / STAGE;
   static constexpr int NS_R1 = (BUDGET - (PBUF * PBYTES + RBYTES + TAIL)) / STAGE;
@@ -662,7 +669,8 @@ enum : int {
   Q_O_FULL = 28,       // [2] O (and X) of a row block complete (commit)
   Q_O_FREE = 30,       // [2] O/X read by the epilogue
   Q_DRAIN = 32,
-  Q_TAB = 33           // [2] rotation tables written (converters)
+  Q_TAB = 33,          // [2] rotation tables written (converters)
+  Q_XFULL = 35         // [2] FUSE: the row statistics of every CTA of the cluster have landed here
 };
 
 __device__ __forceinline__ float2 cpow_mul(float2 base, float2 step, int n) {
@@ -862,11 +870,12 @@ struct UnitConverter {
   }
 };
 
-template <int DK, int T, int DVS, int SM, bool PRE, typename Tout>
-__global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE>::THREADS, 1)
+template <int DK, int T, int DVS, int SM, bool PRE, bool FUSE, typename Tout>
+__global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE>::THREADS, 1)
     tc_chunkwise_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v, TcArgs a, HeadParams hp) {
-  using C = Cfg3<DK, T, DVS, PRE>;
+  using C = Cfg3<DK, T, DVS, PRE, FUSE>;
+  static_assert(!FUSE || (SM == SEG_NONE && DVS == 64), "the fused epilogue runs unsplit, 64-column slices");
   // Stage ready for the MMAs: converted in place, or (PRE) landed already converted.
   constexpr int Q_READY = PRE ? Q_TMA_FULL : Q_CONV_FULL;
   constexpr bool SEG = SM != SEG_NONE;
@@ -959,6 +968,12 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE>::THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + tail_off + C::TABBYTES);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::NBARS);
   auto bar = [&](int i) { return smem_addr(bars + i); };
+  // FUSE: row statistics from the cluster, [slot][cta rank][row] of (mean, M2) over 64 columns.
+  const uint32_t xbuf0 = smem_addr(tmem_holder) + 16;
+  auto xaddr = [&](int slot, int rank, int row) {
+    return xbuf0 + static_cast<uint32_t>(((slot * kMaxCluster + rank) * T + row) * 8);
+  };
+  const int n_cl = a.dv / DVS;  // cluster size under FUSE: every d_v slice of the head
   auto sQ = [&](int s) { return sbase + s * C::STAGE; };
   auto sK = [&](int s) { return sbase + s * C::STAGE + C::QBYTES; };
   auto sV = [&](int s) { return sbase + s * C::STAGE + 2 * C::QBYTES; };
@@ -983,6 +998,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE>::THREADS, 1)
       mbar_init(bar(Q_O_FULL + k), 1);
       mbar_init(bar(Q_O_FREE + k), 128);
       if (!PRE) mbar_init(bar(Q_TAB + k), C::NCONV);
+      if (FUSE) mbar_init(bar(Q_XFULL + k), 1);  // armed once a use, the rest is transaction bytes
     }
     mbar_init(bar(Q_DRAIN), 1);
     fence_mbar_init();
@@ -999,6 +1015,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE>::THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if constexpr (FUSE) cluster_sync();  // every CTA's barriers exist before any remote arrival
   const uint32_t tmem = *tmem_holder;
 
   if (warp == C::WARP_TMA) {
@@ -1426,11 +1443,35 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE>::THREADS, 1)
     const float gam = hp.gamma[h];
     // Epilogue of row block (chunk i, block u), O/X buffer rb & 1.
     auto epilogue = [&](int rb, int i, int u, int bl) -> bool {
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(Q_O_FULL + (rb & 1)), (rb >> 1) & 1))) return false;
-      tc_fence_after();
       const int rows = min(T, bl - u * T);
       const bool live = my_row >= 0 && my_row < rows;
       const int t = i * nb * T + u * T + (my_row < 0 ? 0 : my_row);
+      // FUSE output rows and columns of this lane.  With T = 64 the rows sit in lanes 0-15 of
+      // each warp; lane l + 16 then writes the upper half of the columns of lane l's row.
+      constexpr bool SPLIT = FUSE && T == 64;
+      constexpr int EC = SPLIT ? DVS / 2 : DVS;
+      const int erow = SPLIT ? 16 * warp + (lane & 15) : my_row;
+      const bool elive = erow >= 0 && erow < rows;
+      const int64_t eoff = ((static_cast<int64_t>(b) * a.L + (i * nb * T + u * T + (erow < 0 ? 0 : erow))) * a.heads + h) *
+                               a.dv + dvb * DVS + (SPLIT ? (lane >> 4) * EC : 0);
+      const uint4* egp = nullptr;
+      if constexpr (FUSE) {
+        // the gate slice of this lane, into L1 now; the same row of the next row block (the
+        // next T tokens: row blocks run in sequence order here) into L2
+        egp = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.gate) + eoff);
+        const char* cur = reinterpret_cast<const char*>(egp);
+        if (elive) {
+          asm volatile("prefetch.global.L1 [%0];" ::"l"(cur));
+          asm volatile("prefetch.global.L1 [%0];" ::"l"(cur + EC * 2 - 1));
+        }
+        if (erow >= 0 && (i * nb * T + u * T + erow) + T < a.L) {
+          const char* nx = cur + static_cast<int64_t>(T) * a.heads * a.dv * 2;
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(nx));
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(nx + EC * 2 - 1));
+        }
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(Q_O_FULL + (rb & 1)), (rb >> 1) & 1))) return false;
+      tc_fence_after();
       const float f = row_factor_f32(gam, sd, a.pos0 + t, a.flags) / sd;
       const float gx = (nb > 1) ? exp2f(static_cast<float>(u * T) * log2g) : 0.f;
       Tout* dst = static_cast<Tout*>(a.o) + ((static_cast<int64_t>(b) * a.L + t) * a.heads + h) * a.dv + dvb * DVS;
@@ -1456,6 +1497,115 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE>::THREADS, 1)
       };
       const uint32_t tO = tmem + C::COL_O + (rb & 1) * DVS + lane_off;
       const uint32_t tX = tmem + C::COL_X + (rb & 1) * DVS + lane_off;
+      if constexpr (FUSE) {
+        // MSR epilogue in the kernel ("阅读笔记：RetNet" §三.2): the head's d_v columns are spread
+        // over the n_cl CTAs of this cluster.  Each CTA takes (mean, M2) of its 64 columns of a
+        // row and stores them into every CTA's shared memory (st.async, counted in transaction
+        // bytes on that CTA's barrier); the pooled statistics (Chan's combination of equal-count
+        // groups) normalise the row, which is then multiplied by swish(gate).  Biased variance,
+        // eps inside the root.  Slot rb & 1 is written again for row block rb + 2 only after
+        // its writer has seen every CTA's statistics of row block rb + 1, which each CTA sends
+        // after it has finished reading the slot for row block rb: two slots need no release
+        // barrier.
+        float y[DVS];
+#pragma unroll
+        for (int grp = 0; grp < DVS / 32; ++grp) {
+          uint32_t uo[2][16], ux[2][16];
+          if (C::XBUF > 0 && nb > 1) {
+            tmem_ld_wait(tO + 32 * grp, uo, tX + 32 * grp, ux);
+          } else {
+            tmem_ld_wait(tO + 32 * grp, uo);
+          }
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float ov = __uint_as_float(uo[c / 16][c % 16]);
+            y[32 * grp + c] = (C::XBUF > 0 && nb > 1) ? f * fmaf(gx, __uint_as_float(ux[c / 16][c % 16]), ov) : f * ov;
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar(Q_O_FREE + (rb & 1)));
+        float mean_i = 0.f, m2 = 0.f;
+#pragma unroll
+        for (int c = 0; c < DVS; ++c) mean_i += y[c];
+        mean_i *= 1.f / DVS;
+#pragma unroll
+        for (int c = 0; c < DVS; ++c) m2 = fmaf(y[c] - mean_i, y[c] - mean_i, m2);
+        const int slot = rb & 1;
+        const uint32_t me = cluster_ctarank();
+        if (warp == 0 && lane == 0) mbar_arrive_expect_tx(bar(Q_XFULL + slot), static_cast<uint32_t>(n_cl * T * 8));
+        if (my_row >= 0) {
+          for (int pr = 0; pr < n_cl; ++pr)
+            st_async_v2(map_shared_rank(xaddr(slot, me, my_row), pr), mean_i, m2,
+                        map_shared_rank(bar(Q_XFULL + slot), pr));
+        }
+        if (!__all_sync(0xffffffffu, mbar_wait_cluster(bar(Q_XFULL + slot), (rb >> 1) & 1))) return false;
+        // this lane's EC columns of the row
+        float yv[EC];
+#pragma unroll
+        for (int c = 0; c < EC; ++c) {
+          if constexpr (SPLIT) {
+            const float up = __shfl_up_sync(0xffffffffu, y[EC + c], 16);
+            yv[c] = lane >= 16 ? up : y[c];
+          } else {
+            yv[c] = y[c];
+          }
+        }
+        if (elive) {
+          // gate loads in flight together where registers allow (half rows), else 16 columns at a time
+          uint4 gv[SPLIT ? EC / 8 : 2];
+          if constexpr (SPLIT) {
+#pragma unroll
+            for (int j = 0; j < EC / 8; ++j) gv[j] = __ldg(egp + j);
+          }
+          float mean = 0.f, m2t = 0.f;
+          for (int pr = 0; pr < n_cl; ++pr) {
+            float2 st;
+            asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(st.x), "=f"(st.y) : "r"(xaddr(slot, pr, erow)));
+            mean += st.x;
+            m2t += st.y;
+          }
+          mean /= static_cast<float>(n_cl);
+          for (int pr = 0; pr < n_cl; ++pr) {
+            float mx;
+            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(mx) : "r"(xaddr(slot, pr, erow)));
+            m2t = fmaf(static_cast<float>(DVS) * (mx - mean), mx - mean, m2t);
+          }
+          const float inv = rsqrtf(m2t / static_cast<float>(DVS * n_cl) + a.eps);
+          Tout* edst = static_cast<Tout*>(a.o) + eoff;
+#pragma unroll
+          for (int q = 0; q < EC / 16; ++q) {
+            const uint4 g0 = SPLIT ? gv[(2 * q) % (SPLIT ? EC / 8 : 2)] : __ldg(egp + 2 * q);
+            const uint4 g1 = SPLIT ? gv[(2 * q + 1) % (SPLIT ? EC / 8 : 2)] : __ldg(egp + 2 * q + 1);
+            const uint32_t gw[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+            float ov[16];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              // swish(g) = g / (1 + e^-g); the fast divide is exact enough here (2 ulp)
+              const float ga = __uint_as_float(gw[e] << 16), gb = __uint_as_float(gw[e] & 0xffff0000u);
+              ov[2 * e] = (yv[16 * q + 2 * e] - mean) * inv * __fdividef(ga, 1.f + __expf(-ga));
+              ov[2 * e + 1] = (yv[16 * q + 2 * e + 1] - mean) * inv * __fdividef(gb, 1.f + __expf(-gb));
+            }
+            if constexpr (sizeof(Tout) == 2) {
+#pragma unroll
+              for (int c8 = 0; c8 < 2; ++c8) {
+                uint32_t pk[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  __nv_bfloat162 v2 = __floats2bfloat162_rn(ov[8 * c8 + 2 * e], ov[8 * c8 + 2 * e + 1]);
+                  pk[e] = *reinterpret_cast<uint32_t*>(&v2);
+                }
+                *reinterpret_cast<uint4*>(edst + 16 * q + 8 * c8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              }
+            } else {
+#pragma unroll
+              for (int c4 = 0; c4 < 4; ++c4)
+                *reinterpret_cast<float4*>(edst + 16 * q + 4 * c4) =
+                    make_float4(ov[4 * c4], ov[4 * c4 + 1], ov[4 * c4 + 2], ov[4 * c4 + 3]);
+            }
+          }
+        }
+        return true;
+      }
       if (C::XBUF == 0 || nb == 1) {
         // No cross accumulator: O alone, LDW columns per load.
 #pragma unroll
@@ -1558,6 +1708,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE>::THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
+  if constexpr (FUSE) cluster_sync();  // no CTA leaves while a peer may still write into it
 }
 
 // ============================================================================================
@@ -1712,7 +1863,7 @@ bool pre_convert_applies(const RetentionCall& c, int nb, int n_seg) {
 // (about 1.6x the work per SM); they need one sub-block per chunk (no cross accumulator in
 // tensor memory) and d_k <= 128.  The halved CTA count is made up by sequence segments.
 bool pipe_wide_slice(const RetentionCall& c, int T) {
-  return c.dims.d_k <= 128 && T == 64 && c.chunk == 64 && c.dims.d_v % 128 == 0;
+  return !c.gate && c.dims.d_k <= 128 && T == 64 && c.chunk == 64 && c.dims.d_v % 128 == 0;
 }
 
 int sm_count() {
@@ -1768,6 +1919,8 @@ TcArgs make_args(const RetentionCall& c, int n_chunks, int nb) {
   a.L = static_cast<int>(c.dims.seqlen);
   a.heads = static_cast<int>(c.dims.heads);
   a.batch = static_cast<int>(c.dims.batch);
+  a.gate = c.gate;
+  a.eps = c.eps;
   a.dv = static_cast<int>(c.dims.d_v);
   a.n_chunks = n_chunks;
   a.pos0 = c.pos0;
@@ -1792,6 +1945,63 @@ dim3 tc_grid(const Dims& d, int dvs) {
   return dim3(static_cast<unsigned>(d.d_v / dvs), static_cast<unsigned>(d.heads), static_cast<unsigned>(d.batch));
 }
 
+// Fused MSR epilogue: the d_v slices of a head form one thread-block cluster (n_cl <=
+// kMaxCluster CTAs) that pools the GroupNorm statistics in distributed shared memory.  With
+// chunks of several sub-blocks and room in the workspace the conversion pre-pass runs first.
+template <int DK, int T, typename Tout>
+cudaError_t launch_fused(const RetentionCall& c, const HeadParams& hp, cudaStream_t s, const CUtensorMap& mq,
+                         const CUtensorMap& mk, const CUtensorMap& mv, const TcArgs& a, int nb) {
+  const int n_cl = static_cast<int>(c.dims.d_v / 64);
+  if (n_cl < 1 || n_cl > kMaxCluster) return cudaErrorInvalidValue;
+  const dim3 grid = tc_grid(c.dims, 64);
+  auto launch = [&](auto kern, int threads, int smem, const CUtensorMap& q, const CUtensorMap& k,
+                    const CUtensorMap& v) -> cudaError_t {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(threads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = n_cl;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, q, k, v, a, hp);
+  };
+  if constexpr (Cfg3<DK, T, 64>::XBUF > 0) {
+    if (pre_convert_applies(c, nb, 1)) {
+      const PreCopies pc = pre_copies(c);
+      const int64_t tokens = c.dims.batch * c.dims.seqlen;
+      const int64_t items = tokens * (DK / 8) + tokens * c.dims.heads * (c.dims.d_v / 8);
+      const int blocks = static_cast<int>(std::min<int64_t>((items + 255) / 256, static_cast<int64_t>(sm_count()) * 8));
+      tc_convert_kernel<DK, T><<<blocks, 256, 0, s>>>(
+          static_cast<const uint4*>(c.q), static_cast<const uint4*>(c.k), static_cast<const uint4*>(c.v),
+          static_cast<uint4*>(pc.q), static_cast<uint4*>(pc.k), static_cast<uint4*>(pc.v), tokens,
+          static_cast<int>(c.dims.seqlen), static_cast<int>(c.dims.heads), static_cast<int>(c.dims.d_v), c.pos0,
+          c.flags, hp);
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+      RetentionCall cc = c;
+      cc.q = pc.q;
+      cc.k = pc.k;
+      cc.v = pc.v;
+      CUtensorMap pq, pk, pv;
+      if (!make_maps(cc, T, &pq, &pk, &pv)) return cudaErrorInvalidValue;
+      using CP = Cfg3<DK, T, 64, true, true>;
+      static_assert(CP::FITS, "fused kernel does not fit this tile");
+      return launch(tc_chunkwise_pipe_kernel<DK, T, 64, SEG_NONE, true, true, Tout>, CP::THREADS, CP::SMEM, pq, pk,
+                    pv);
+    }
+  }
+  using CF = Cfg3<DK, T, 64, false, true>;
+  static_assert(CF::FITS, "fused kernel does not fit this tile");
+  return launch(tc_chunkwise_pipe_kernel<DK, T, 64, SEG_NONE, false, true, Tout>, CF::THREADS, CF::SMEM, mq, mk, mv);
+}
+
 // Pipelined kernel: units of T rows, nb = B / T per chunk, d_v slices of DVS columns.
 template <int DK, int T, int DVS, typename Tout>
 cudaError_t launch_pipe(const RetentionCall& c, const HeadParams& hp, cudaStream_t s) {
@@ -1803,6 +2013,10 @@ cudaError_t launch_pipe(const RetentionCall& c, const HeadParams& hp, cudaStream
   const int nb = static_cast<int>(c.chunk / T);
   const TcArgs a = make_args(c, static_cast<int>((c.dims.seqlen + c.chunk - 1) / c.chunk), nb);
   if (Cf::XBUF == 0 && nb != 1) return cudaErrorInvalidValue;
+  if (c.gate) {  // fused MSR epilogue: no segments, one cluster per (batch, head)
+    if constexpr (DVS == 64) return launch_fused<DK, T, Tout>(c, hp, s, mq, mk, mv, a, nb);
+    return cudaErrorInvalidValue;
+  }
   TcArgs as = a;
   const dim3 grid = tc_grid(c.dims, DVS);
   const int64_t ctas = static_cast<int64_t>(grid.x) * grid.y * grid.z;
@@ -1836,16 +2050,16 @@ cudaError_t launch_pipe(const RetentionCall& c, const HeadParams& hp, cudaStream
         cc.v = pc.v;
         CUtensorMap pq, pk, pv;
         if (!make_maps(cc, T, &pq, &pk, &pv)) return cudaErrorInvalidValue;
-        auto kern = tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_NONE, true, Tout>;
+        auto kern = tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_NONE, true, false, Tout>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, CfP::SMEM);
         if (e != cudaSuccess) return e;
         kern<<<grid, CfP::THREADS, CfP::SMEM, s>>>(pq, pk, pv, as, hp);
         return cudaGetLastError();
       }
     }
-    return run(tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_NONE, false, Tout>, 1);
+    return run(tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_NONE, false, false, Tout>, 1);
   }
-  if (max_states < 1) return run(tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_REPLAY, false, Tout>, as.n_seg);
+  if (max_states < 1) return run(tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_REPLAY, false, false, Tout>, as.n_seg);
   // Pre-pass: each of the first n_seg - 1 segments split into n_split sub-segments, as many
   // as the SMs, the workspace and two chunks a sub-segment allow.
   const int n_pre = as.n_seg - 1;
@@ -1865,12 +2079,12 @@ cudaError_t launch_pipe(const RetentionCall& c, const HeadParams& hp, cudaStream
   }
   as.n_sub = j;
   as.ws = static_cast<float*>(c.ws);
-  cudaError_t e = run(tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_STATE, false, Tout>, as.n_sub);
+  cudaError_t e = run(tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_STATE, false, false, Tout>, as.n_sub);
   if (e != cudaSuccess) return e;
   // Output pass, launched as a programmatic dependent of the pre-pass (segment-major grid):
   // its segment-0 CTAs run on the SMs the pre-pass leaves idle; later segments wait on the
   // device (griddepcontrol.wait) before they read the pre-pass states.
-  auto kern = tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_FROM_WS, false, Tout>;
+  auto kern = tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_FROM_WS, false, false, Tout>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -1951,6 +2165,11 @@ bool tc_chunkwise_supported(const RetentionCall& c) {
   return true;
 }
 
+bool tc_fused_supported(const RetentionCall& c) {
+  return tc_chunkwise_supported(c) && !force_serial_kernel() && c.dims.d_v % 64 == 0 &&
+         c.dims.d_v / 64 <= kMaxCluster && aligned16(c.gate);
+}
+
 bool tc_driver_ready() { return encode_fn() != nullptr; }
 
 // Host-side part of the scaled-operand condition: every head keeps gamma^T >= 2^-12, where T
@@ -1986,7 +2205,7 @@ cudaError_t launch_segment_state_t(const RetentionCall& c, const HeadParams& hp,
   a.sub_lo[0] = 0;
   a.sub_hi[0] = n_chunks;
   a.ws = c.state_out;  // sub-segment 0 of the workspace layout is [batch][heads][d_k][d_v]
-  auto kern = tc_chunkwise_pipe_kernel<DK, T, 64, SEG_STATE, false, Tout>;
+  auto kern = tc_chunkwise_pipe_kernel<DK, T, 64, SEG_STATE, false, false, Tout>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM);
   if (e != cudaSuccess) return e;
   kern<<<tc_grid(c.dims, 64), Cf::THREADS, Cf::SMEM, s>>>(mq, mk, mv, a, hp);
@@ -2038,6 +2257,7 @@ int tc_chunkwise_launches(const RetentionCall& c) {
   const int nb = static_cast<int>(c.chunk / T);
   TcArgs as = make_args(c, static_cast<int>((c.dims.seqlen + c.chunk - 1) / c.chunk), nb);
   const int64_t ctas = (c.dims.d_v / dvs) * c.dims.heads * c.dims.batch;
+  if (c.gate) return pre_convert_applies(c, nb, 1) ? 2 : 1;  // fused epilogue: never segmented
   const int max_states = plan_call(c, ctas, sm_count(), as);
   if (dvs == 64 && pre_convert_applies(c, nb, as.n_seg)) return 2;  // conversion pre-pass + kernel
   return (as.n_seg > 1 && max_states >= 1) ? 2 : 1;

@@ -27,6 +27,10 @@ struct RetentionCall {
   // kernel (segment states); nullptr = single-launch segments that replay the state.
   void* ws = nullptr;
   size_t ws_bytes = 0;
+  // Fused MSR epilogue (tensor-core kernel): o <- GroupNorm_h(o) * swish(gate), gate laid out
+  // as o; nullptr = plain retention output.
+  const void* gate = nullptr;
+  float eps = 0.f;
 };
 
 // fp32 CUDA-core kernel: the parallel form (chunk >= seqlen, no state) and the chunkwise
@@ -37,6 +41,9 @@ cudaError_t launch_simt_retention(const RetentionCall& c, const HeadParams& hp, 
 // and buffers are ones it handles, `heads_ok` whether every head keeps gamma^chunk >= 2^-12.
 bool tc_chunkwise_supported(const RetentionCall& c);
 bool tc_chunkwise_heads_ok(const RetentionCall& c, const HeadParams& hp);
+// The tensor-core kernel with the MSR epilogue fused (c.gate set) handles this call: a
+// tensor-core shape with d_v a multiple of 64 and at most 256, gate 16-byte aligned.
+bool tc_fused_supported(const RetentionCall& c);
 // The driver entry point that encodes TMA tensor maps could be resolved.
 bool tc_driver_ready();
 cudaError_t launch_tc_chunkwise(const RetentionCall& c, const HeadParams& hp, cudaStream_t s);

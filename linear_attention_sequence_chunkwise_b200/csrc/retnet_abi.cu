@@ -105,7 +105,14 @@ retnet_status_t chunkwise_impl(const void* q, const void* k, const void* v, void
                                retnet_dtype_t in_dtype, retnet_dtype_t out_dtype, const float* gamma,
                                const float* theta, int64_t pos0, uint32_t flags, int64_t chunk,
                                const float* state_in, float* state_out, const float* z_in, float* z_out,
-                               void* workspace, size_t workspace_bytes, void* stream) {
+                               void* workspace, size_t workspace_bytes, void* stream, const void* gate = nullptr,
+                               float eps = 0.f);
+retnet_status_t chunkwise_impl(const void* q, const void* k, const void* v, void* o, retnet_dims_t dims,
+                               retnet_dtype_t in_dtype, retnet_dtype_t out_dtype, const float* gamma,
+                               const float* theta, int64_t pos0, uint32_t flags, int64_t chunk,
+                               const float* state_in, float* state_out, const float* z_in, float* z_out,
+                               void* workspace, size_t workspace_bytes, void* stream, const void* gate,
+                               float eps) {
   retnet_status_t st = check_common(dims, in_dtype, out_dtype, pos0, flags, true);
   if (st != RETNET_OK) return st;
   if (chunk <= 0) return RETNET_ERR_BAD_PARAM;
@@ -118,6 +125,12 @@ retnet_status_t chunkwise_impl(const void* q, const void* k, const void* v, void
                   pos0, flags, chunk, true, state_in, state_out, z_in, z_out};
   c.ws = workspace;
   c.ws_bytes = workspace ? workspace_bytes : 0;
+  if (gate) {
+    // Fused MSR epilogue: the tensor-core kernel only, decided on the host before any launch.
+    c.gate = gate;
+    c.eps = eps;
+    if (dims.seqlen > 0 && !(tc_fused_supported(c) && tc_chunkwise_heads_ok(c, hp))) return RETNET_ERR_UNSUPPORTED;
+  }
   if (dims.seqlen == 0) {
     // No tokens: the state passes through unchanged.
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -160,6 +173,19 @@ retnet_status_t retnet_retention_chunkwise_ws(const void* q, const void* k, cons
                                               size_t workspace_bytes, void* stream) {
   return chunkwise_impl(q, k, v, o, dims, in_dtype, out_dtype, gamma, theta, pos0, flags, chunk, state_in, state_out,
                         z_in, z_out, workspace, workspace_bytes, stream);
+}
+
+retnet_status_t retnet_msr_chunkwise(const void* q, const void* k, const void* v, const void* g, void* out,
+                                     retnet_dims_t dims, retnet_dtype_t in_dtype, retnet_dtype_t out_dtype,
+                                     const float* gamma, const float* theta, int64_t pos0, uint32_t flags,
+                                     int64_t chunk, float eps, const float* state_in, float* state_out,
+                                     void* workspace, size_t workspace_bytes, void* stream) {
+  if (!(eps >= 0.f) || !isfinite(eps)) return RETNET_ERR_BAD_PARAM;
+  if (dims.seqlen > 0 && !g) return RETNET_ERR_NULL_PTR;
+  if (flags & RETNET_F_NORM_R) return RETNET_ERR_UNSUPPORTED;
+  // (without tokens nothing reads g: the call only passes the state through)
+  return chunkwise_impl(q, k, v, out, dims, in_dtype, out_dtype, gamma, theta, pos0, flags, chunk, state_in,
+                        state_out, nullptr, nullptr, workspace, workspace_bytes, stream, g, eps);
 }
 
 // ---- allocation-free variant ---------------------------------------------------------------
@@ -283,6 +309,26 @@ int retnet_chunkwise_launches(retnet_dims_t dims, retnet_dtype_t in_dtype, uint3
                   in_dtype, RETNET_BF16, 0, flags, chunk, true, nullptr, nullptr, nullptr, nullptr};
   c.ws = workspace_bytes ? reinterpret_cast<void*>(static_cast<uintptr_t>(256)) : nullptr;  // only its size matters
   c.ws_bytes = workspace_bytes;
+  return tc_chunkwise_launches(c);
+}
+
+int retnet_msr_chunkwise_launches(retnet_dims_t dims, retnet_dtype_t in_dtype, uint32_t flags, int64_t chunk,
+                                  const float* gamma, size_t workspace_bytes) {
+  if (flags & RETNET_F_NORM_R) return -static_cast<int>(RETNET_ERR_UNSUPPORTED);
+  const int path = retnet_chunkwise_kernel(dims, in_dtype, flags, chunk, gamma);
+  if (path < 0) return path;
+  if (dims.seqlen == 0) return 0;
+  if (path == 0) return -static_cast<int>(RETNET_ERR_UNSUPPORTED);
+  const retnet_status_t st = check_device();
+  if (st != RETNET_OK) return -static_cast<int>(st);
+  alignas(16) static const uint32_t kAligned[4] = {0, 0, 0, 0};
+  RetentionCall c{kAligned, kAligned, kAligned, const_cast<uint32_t*>(kAligned),
+                  Dims{dims.batch, dims.seqlen, dims.heads, dims.d_k, dims.d_v}, in_dtype, RETNET_BF16, 0, flags,
+                  chunk, true, nullptr, nullptr, nullptr, nullptr};
+  c.ws = workspace_bytes ? reinterpret_cast<void*>(static_cast<uintptr_t>(256)) : nullptr;  // only its size matters
+  c.ws_bytes = workspace_bytes;
+  c.gate = kAligned;
+  if (!tc_fused_supported(c)) return -static_cast<int>(RETNET_ERR_UNSUPPORTED);
   return tc_chunkwise_launches(c);
 }
 

@@ -68,6 +68,65 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
 
 static __device__ unsigned int g_wait_timeouts = 0;
 
+// ---- thread-block clusters: distributed shared memory, remote mbarrier arrivals --------------
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// All threads of all CTAs of the cluster (the CTAs of a cluster are co-scheduled, so every one
+// of them reaches it: used once after set-up and once before exit, never inside a loop).
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Address of the same shared-memory location in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t map_shared_rank(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void st_cluster_v2(uint32_t addr, float a, float b) {
+  asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(a), "f"(b) : "memory");
+}
+// Asynchronous 8-byte store into another CTA's shared memory that completes 8 bytes of
+// transaction count on that CTA's mbarrier (both addresses from map_shared_rank): the data is
+// visible to whoever observes the phase it completes, with no fence on the sending side.
+__device__ __forceinline__ void st_async_v2(uint32_t remote_addr, float a, float b, uint32_t remote_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(remote_addr),
+               "f"(a), "f"(b), "r"(remote_bar)
+               : "memory");
+}
+// Arrive on an mbarrier of another CTA of the cluster; release at cluster scope orders this
+// thread's earlier writes (to that CTA's shared memory) before the arrival.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t remote_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
+}
+// Bounded wait on a local mbarrier whose arrivals come from the cluster (acquire at cluster scope).
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, long long budget = 4000000000LL) {
+  auto probe = [&]() -> bool {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+  };
+  if (probe()) return true;
+  const long long t0 = clock64();
+  while (!probe()) {
+    if (clock64() - t0 > budget) {
+      atomicAdd(&g_wait_timeouts, 1u);
+      return false;
+    }
+  }
+  return true;
+}
+
+
 // Waits for the phase with the given parity to complete, for at most `budget` SM clock
 // cycles.  Returns false (and counts a timeout) if it gave up.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long long budget = 4000000000LL) {

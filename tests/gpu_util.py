@@ -43,3 +43,36 @@ def bf16_round(x):
 # inputs, 1e-2 with bf16 inputs and fp32 accumulation.
 TOL_F32 = 1e-4
 TOL_BF16 = 1e-2
+
+
+def err_msr(gpu, ref, y_ref, g, heads, eps=1e-5, bf16_out=False):
+    """Error of an MSR output against the oracle's ``ref`` = swish(g) (.) GroupNorm(y_ref), in
+    units of the bar that the retention output y itself meets.
+
+    If y carries errors |dy| <= tol * rms(y) (the chunkwise bar), then within one (token, head)
+    row of mean m and deviation sd, the normalised value y^ = (y - m) / sd moves by at most
+    tol * rms(y) * (2 + |y^|) / sd (one term for dy, one for dm, |y^| for d sd; m and sd are
+    1-Lipschitz in the row's max norm), and the output by |swish(g)| times that.  Returned: the
+    smallest tol that explains the observed differences, max over elements of
+    |out - ref| * sd_row / (rms(y) * (2 + |y^|) * |swish(g)|), net of a bf16 output's own
+    rounding when bf16_out.  (m, sd, y^ and swish(g) here only size the bound.)
+    """
+    y = np.asarray(y_ref, dtype=np.float64)
+    dv = y.shape[-1]
+    rows = y.reshape(-1, heads, dv)
+    gg = np.asarray(g.double().numpy() if hasattr(g, "double") else g, dtype=np.float64).reshape(rows.shape)
+    r = np.asarray(ref, dtype=np.float64).reshape(rows.shape)
+    m = rows.mean(axis=-1, keepdims=True)
+    sd = np.sqrt(((rows - m) ** 2).mean(axis=-1, keepdims=True) + eps)
+    yh = (rows - m) / sd
+    sw = np.abs(gg / (1.0 + np.exp(-gg)))
+    out = gpu.detach().double().cpu().numpy().reshape(rows.shape)
+    diff = np.abs(out - r)
+    if bf16_out:
+        diff = np.maximum(diff - 2.0 ** -8 * np.abs(r), 0.0)
+    rms_y = float(np.sqrt((y ** 2).mean()))
+    scale = rms_y * (2.0 + np.abs(yh)) * sw / sd
+    ok = scale > 0
+    if not ok.all() and diff[~ok].max() > 0:
+        return float("inf")
+    return float((diff[ok] / scale[ok]).max())

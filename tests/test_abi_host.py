@@ -165,6 +165,22 @@ def test_epilogue_validation(lib):
     assert f(FAKE, FAKE, FAKE, 0, 2, 16, 1e-5, 0, 0, None) == 0          # no tokens: no work
 
 
+def test_fused_msr_validation(lib):
+    """The fused MSR entry point checks eps, the gate pointer and the norm-R flag on the host."""
+    g = _gamma(2)
+    gp = g.ctypes.data_as(rn._fp)
+    d = rn.Dims(1, 64, 2, 128, 128)
+    f = lib.retnet_msr_chunkwise
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, d, 1, 0, gp, None, 0, 0, 64, -1.0, None, None, None, 0, None) == 4
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, d, 1, 0, gp, None, 0, 0, 64, float("inf"), None, None, None, 0,
+             None) == 4
+    assert f(FAKE, FAKE, FAKE, None, FAKE, d, 1, 0, gp, None, 0, 0, 64, 1e-5, None, None, None, 0, None) == 1
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, d, 1, 0, gp, None, 0, rn.F_NORM_R, 64, 1e-5, None, None, None, 0,
+             None) == 5
+    assert lib.retnet_msr_chunkwise_launches(d, 1, rn.F_NORM_R, 64, gp, 0) == -5
+    assert lib.retnet_msr_chunkwise_launches(rn.Dims(1, 64, 2, 128, 128), 1, 0, 0, gp, 0) == -4  # chunk 0
+
+
 def test_binding_raises_without_library(tmp_path):
     import importlib
     mod = importlib.import_module("linear_attention_sequence_chunkwise_b200")

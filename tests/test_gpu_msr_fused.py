@@ -1,0 +1,123 @@
+"""Parity of the fused MSR kernel (chunkwise retention + GroupNorm + swish gate in one
+tensor-core kernel, the d_v slices of a head in one thread-block cluster) against the fp64
+oracle: oracle.msr_epilogue of the oracle's retention output.
+
+Bar: the retention output's own bar (max|dy|/rms(y) <= 1e-2 with bf16 inputs) carried through
+the row normalisation and the gate (gpu_util.err_msr: the GroupNorm divides each row's error by
+the row's deviation and the gate multiplies it by |swish(g)|), net of a bf16 output's own
+rounding.  The state hand-off is held to the chunkwise bar directly.
+"""
+import numpy as np
+import pytest
+import torch
+
+import linear_attention_sequence_chunkwise_b200 as rn
+import oracle
+import synth_inputs as si
+from gpu_util import TOL_BF16, dev, err, err_msr, require_gpu
+
+pytestmark = pytest.mark.gpu
+FLAGS = rn.F_XPOS | rn.F_SCALE_SQRT_D | rn.F_NORM_D
+EPS = 1e-5
+
+
+@pytest.fixture(autouse=True)
+def _gpu(cuda_lib):
+    require_gpu()
+    rn.retnet_debug_wait_timeouts(clear=True)
+    yield
+    assert rn.retnet_debug_wait_timeouts(clear=True) == 0
+
+
+def gate(b, L, h, dv, seed):
+    return si.randn((b, L, h, dv), seed, "bf16")
+
+
+def fused(q, k, v, gt, g, th, B, pos0=0, state_in=None, want_state=False, out_dtype=torch.float32,
+          workspace=True):
+    b, L, h, dk = q.shape
+    dv = v.shape[-1]
+    ws = None
+    if workspace:
+        ws = torch.empty(rn.retnet_chunkwise_workspace_size((b, L, h, dk, dv)), dtype=torch.uint8, device="cuda")
+    n = rn.retnet_msr_chunkwise_launches((b, L, h, dk), dv, rn.BF16, FLAGS, B, g,
+                                         0 if ws is None else ws.numel())
+    assert n in (1, 2), n
+    out = torch.empty(b, L, h, dv, device="cuda", dtype=out_dtype)
+    so = torch.empty(b, h, dk, dv, device="cuda") if want_state else None
+    rn.retnet_msr_chunkwise(dev(q), dev(k), dev(v), dev(gt), out, g, th, pos0, FLAGS, B, EPS,
+                            None if state_in is None else dev(state_in), so, ws)
+    torch.cuda.synchronize()
+    return out, so, n
+
+
+def reference(q, k, v, gt, g, th, B, pos0=0, state_in=None):
+    y, S, _ = oracle.chunkwise(q, k, v, g, B, th, pos0, FLAGS, state_in=state_in)
+    h = q.shape[2]
+    return oracle.msr_epilogue(y, gt, h, eps=EPS), y, S
+
+
+@pytest.mark.parametrize("dk,dv,B,L", [(64, 64, 64, 130), (128, 128, 64, 300), (128, 192, 128, 300),
+                                       (256, 256, 64, 200), (256, 256, 256, 520), (64, 256, 512, 513),
+                                       (128, 128, 256, 257), (256, 128, 128, 129), (128, 64, 64, 1)])
+@pytest.mark.parametrize("workspace", [True, False])
+def test_fused_msr_matches_oracle(dk, dv, B, L, workspace):
+    b, h = 2, 3
+    q, k, v = si.qkv(b, L, h, dk, dv, 300 + dk + B, "bf16")
+    gt = gate(b, L, h, dv, 7000 + dv)
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+    ref, y, Sref = reference(q, k, v, gt, g, th, B)
+    out, so, n = fused(q, k, v, gt, g, th, B, want_state=True, workspace=workspace)
+    e = err_msr(out, ref, y, gt, h, EPS)
+    print(f"dk={dk} dv={dv} B={B} L={L} ws={workspace} launches={n}: msr err {e:.3e}, "
+          f"max|err|/rms {err(out, ref):.3e}")
+    assert e <= TOL_BF16
+    assert err(so, Sref) <= TOL_BF16
+
+
+def test_fused_msr_bf16_out_state_in_pos0():
+    """bf16 output, a carried-in state and a large start position, against the same bar."""
+    b, L, h, dk, dv, B = 2, 333, 4, 256, 256, 256
+    q, k, v = si.qkv(b, L, h, dk, dv, 321, "bf16")
+    gt = gate(b, L, h, dv, 322)
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+    S0 = si.decode_state(b, h, dk, dv, 323, std=0.05)
+    pos0 = (1 << 20) + 77
+    ref, y, Sref = reference(q, k, v, gt, g, th, B, pos0=pos0, state_in=S0)
+    out, so, _ = fused(q, k, v, gt, g, th, B, pos0=pos0, state_in=S0, want_state=True, out_dtype=torch.bfloat16)
+    assert err_msr(out, ref, y, gt, h, EPS, bf16_out=True) <= TOL_BF16
+    assert err(so, Sref) <= TOL_BF16
+
+
+def test_fused_no_worse_than_two_kernel_path():
+    """The fused kernel and chunkwise + retnet_msr_epilogue (fp32 between them) against the
+    oracle: fusing the epilogue loses no accuracy."""
+    b, L, h, dk, dv, B = 2, 700, 4, 128, 256, 128
+    q, k, v = si.qkv(b, L, h, dk, dv, 401, "bf16")
+    gt = gate(b, L, h, dv, 402)
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+    ref, y_ref, _ = reference(q, k, v, gt, g, th, B)
+    out, _, _ = fused(q, k, v, gt, g, th, B)
+    y = torch.empty(b, L, h, dv, device="cuda")
+    rn.retnet_retention_chunkwise(dev(q), dev(k), dev(v), y, g, th, 0, FLAGS, B)
+    two = torch.empty_like(y)
+    rn.retnet_msr_epilogue(y, dev(gt).float(), two, h, EPS)  # y and g share one dtype
+    torch.cuda.synchronize()
+    e_fused, e_two = err_msr(out, ref, y_ref, gt, h, EPS), err_msr(two, ref, y_ref, gt, h, EPS)
+    print(f"fused {e_fused:.3e}, two kernels {e_two:.3e}")
+    assert e_fused <= TOL_BF16 and e_two <= TOL_BF16
+    assert e_fused <= 1.5 * e_two + 1e-3
+
+
+def test_fused_unsupported_shapes_are_rejected():
+    b, L, h, dk = 1, 64, 2, 128
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+    # d_v = 320 needs five CTAs a cluster; the norm-R flag has no tensor-core path
+    for dv, flags in ((320, FLAGS), (128, FLAGS | rn.F_NORM_R)):
+        assert rn.retnet_msr_chunkwise_launches((b, L, h, dk), dv, rn.BF16, flags, 64, g) == -5
+        q, k, v = si.qkv(b, L, h, dk, dv, 5, "bf16")
+        gt = gate(b, L, h, dv, 6)
+        out = torch.full((b, L, h, dv), 7.0, device="cuda")
+        with pytest.raises(RuntimeError, match="UNSUPPORTED"):
+            rn.retnet_msr_chunkwise(dev(q), dev(k), dev(v), dev(gt), out, g, th, 0, flags, 64, EPS)
+        assert bool((out == 7.0).all())  # nothing was launched
