@@ -610,7 +610,11 @@ struct Cfg3 {
   static constexpr int WARP_CONV0 = WARP_S0 + WARPS_S;
   static constexpr int CONV_WARPS = PRE ? 0 : 4;  // PRE: tiles arrive converted (pre-pass)
   static constexpr int NCONV = 32 * CONV_WARPS;
-  static constexpr int WARP_TMA = WARP_CONV0 + CONV_WARPS;
+  // PRE with FUSE: four epilogue warps take O (and X) out of TMEM and run the GroupNorm, so
+  // that the P warps only make P (the plain epilogue is too short to pay for the warps)
+  static constexpr int EPI_WARPS = (PRE && FUSE) ? 4 : 0;
+  static constexpr int WARP_EPI0 = WARP_CONV0 + CONV_WARPS;
+  static constexpr int WARP_TMA = WARP_EPI0 + EPI_WARPS;
   static constexpr int WARP_MMA = WARP_TMA + 1;
   static constexpr int THREADS = 32 * (WARP_MMA + 1);
   static constexpr int QBYTES = T * DK * 2;
@@ -1186,7 +1190,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE>::THREADS, 1)
       mma_commit(bar(Q_DRAIN));
       mbar_wait(bar(Q_DRAIN), 0);
     }
-  } else if (warp >= C::WARP_CONV0) {
+  } else if (warp >= C::WARP_CONV0 && warp < C::WARP_CONV0 + C::CONV_WARPS) {
     // ------------------------------------------------------------------ converters
     if constexpr (!PRE) {
     UnitConverter<DK, T, C::NCONV, C::NDV> cv;
@@ -1219,7 +1223,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE>::THREADS, 1)
       mbar_arrive(bar(Q_CONV_FULL + s));
     }
     }
-  } else if (warp >= C::WARP_S0) {
+  } else if (warp >= C::WARP_S0 && warp < C::WARP_S0 + C::WARPS_S) {
     // ------------------------------------------------------------------ state group
     if constexpr (SM == SEG_STATE) {
       // State pre-pass: once the last increment has landed, the accumulated segment state
@@ -1438,8 +1442,12 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE>::THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------------ P / epilogue group
-    const uint32_t lane_off = static_cast<uint32_t>(32 * warp) << 16;
-    const int my_row = (T == 128) ? 32 * warp + lane : (lane < 16 ? 16 * warp + lane : -1);
+    // (warps 0-3; with EPI_WARPS the epilogue runs on its own four warps, same TMEM lanes)
+    static_assert(C::WARP_EPI0 % 4 == 0, "epilogue warps must cover the four TMEM lane quarters in order");
+    const bool is_epi = C::EPI_WARPS > 0 && warp >= C::WARP_EPI0;
+    const int gwarp = is_epi ? warp - C::WARP_EPI0 : warp;
+    const uint32_t lane_off = static_cast<uint32_t>(32 * gwarp) << 16;
+    const int my_row = (T == 128) ? 32 * gwarp + lane : (lane < 16 ? 16 * gwarp + lane : -1);
     const float gam = hp.gamma[h];
     // Epilogue of row block (chunk i, block u), O/X buffer rb & 1.
     auto epilogue = [&](int rb, int i, int u, int bl) -> bool {
@@ -1450,7 +1458,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE>::THREADS, 1)
       // each warp; lane l + 16 then writes the upper half of the columns of lane l's row.
       constexpr bool SPLIT = FUSE && T == 64;
       constexpr int EC = SPLIT ? DVS / 2 : DVS;
-      const int erow = SPLIT ? 16 * warp + (lane & 15) : my_row;
+      const int erow = SPLIT ? 16 * gwarp + (lane & 15) : my_row;
       const bool elive = erow >= 0 && erow < rows;
       const int64_t eoff = ((static_cast<int64_t>(b) * a.L + (i * nb * T + u * T + (erow < 0 ? 0 : erow))) * a.heads + h) *
                                a.dv + dvb * DVS + (SPLIT ? (lane >> 4) * EC : 0);
@@ -1532,7 +1540,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE>::THREADS, 1)
         for (int c = 0; c < DVS; ++c) m2 = fmaf(y[c] - mean_i, y[c] - mean_i, m2);
         const int slot = rb & 1;
         const uint32_t me = cluster_ctarank();
-        if (warp == 0 && lane == 0) mbar_arrive_expect_tx(bar(Q_XFULL + slot), static_cast<uint32_t>(n_cl * T * 8));
+        if (gwarp == 0 && lane == 0) mbar_arrive_expect_tx(bar(Q_XFULL + slot), static_cast<uint32_t>(n_cl * T * 8));
         if (my_row >= 0) {
           for (int pr = 0; pr < n_cl; ++pr)
             st_async_v2(map_shared_rank(xaddr(slot, me, my_row), pr), mean_i, m2,
@@ -1655,6 +1663,10 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE>::THREADS, 1)
     UnitIter<T, SM> it;
     for (it.start(a.L, nb, c_first, c_lo, c_hi); ok && it.valid(); it.next()) {
       if (it.pre()) continue;  // replay units have no scores
+      if (is_epi) {
+        if (it.rb_done()) ok = epilogue(it.rb, it.i, it.u, it.bl);
+        continue;
+      }
       const int k = it.kf();
       ok = __all_sync(0xffffffffu, mbar_wait(bar(Q_S_FULL + (k % C::SBUF)), (k / C::SBUF) & 1));
       if (ok && k >= C::PBUF)
@@ -1691,6 +1703,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE>::THREADS, 1)
       }
       fence_proxy_async_smem();
       mbar_arrive(bar(Q_P_FULL + (k % C::PBUF)));
+      if (C::EPI_WARPS > 0) continue;
       if (pend_rb >= 0) {
         ok = epilogue(pend_rb, pend_i, pend_u, pend_bl);
         pend_rb = -1;

@@ -5,8 +5,13 @@ oracle: oracle.msr_epilogue of the oracle's retention output.
 Bar: the retention output's own bar (max|dy|/rms(y) <= 1e-2 with bf16 inputs) carried through
 the row normalisation and the gate (gpu_util.err_msr: the GroupNorm divides each row's error by
 the row's deviation and the gate multiplies it by |swish(g)|), net of a bf16 output's own
-rounding.  The state hand-off is held to the chunkwise bar directly.
+rounding.  The plain max|err|/rms(out) is printed too and held to 2e-2: it is at most 7.9e-3
+on these cases except (d_k 256, d_v 128, chunk 128, L 129) at 1.5e-2, where rows of few
+tokens (small deviation) meet large gates; the two-kernel form gives the same figure, and an
+fp64 emulation of the kernel's operand roundings puts most of it on the fp16 rounding of the
+scaled, rotated q and k.  The state hand-off is held to the chunkwise bar directly.
 """
+TOL_OUT = 2e-2
 import numpy as np
 import pytest
 import torch
@@ -69,9 +74,10 @@ def test_fused_msr_matches_oracle(dk, dv, B, L, workspace):
     ref, y, Sref = reference(q, k, v, gt, g, th, B)
     out, so, n = fused(q, k, v, gt, g, th, B, want_state=True, workspace=workspace)
     e = err_msr(out, ref, y, gt, h, EPS)
-    print(f"dk={dk} dv={dv} B={B} L={L} ws={workspace} launches={n}: msr err {e:.3e}, "
-          f"max|err|/rms {err(out, ref):.3e}")
+    e_out = err(out, ref)
+    print(f"dk={dk} dv={dv} B={B} L={L} ws={workspace} launches={n}: msr err {e:.3e}, max|err|/rms {e_out:.3e}")
     assert e <= TOL_BF16
+    assert e_out <= TOL_OUT
     assert err(so, Sref) <= TOL_BF16
 
 
