@@ -150,11 +150,18 @@ RETNET_API retnet_status_t retnet_retention_chunkwise(const void* q, const void*
  * starting from state_in carried over the earlier sub-segments.  Without a workspace the same split runs as one launch in which each later segment
  * first replays the earlier chunks' state.
  *   workspace: device memory, 16-byte aligned, workspace_bytes long, not overlapping any other
- *              argument; its contents on entry are irrelevant and are overwritten (the
- *              sub-segment states, fp32).  NULL (or smaller than one state,
- *              batch * heads * d_k * d_v * 4 bytes) means no workspace.  retnet_chunkwise_workspace_size gives the size that allows the
- *              full split.  The workspace is in use until the call's work on `stream`
- *              completes; two calls sharing one workspace must be ordered on the device.
+ *              argument; its contents on entry are irrelevant and are overwritten.  It holds,
+ *              with RETNET_F_NORM_R, first the R~ row factors (fp32 [batch][seqlen][heads])
+ *              and the key-sum pass's segment values (fp32 [batch * heads][64][d_k]), each
+ *              rounded up to 256 bytes: §三.3's R~ then runs on the tensor-core kernel, a key-
+ *              sum pass over q and k before it, z_in/z_out carried by that pass; without the
+ *              room R~ runs on the CUDA-core kernel; then either the sub-segment states
+ *              (fp32, one is batch * heads * d_k * d_v * 4 bytes; fewer than one means no
+ *              split of this kind) or, for chunks of several 64-row sub-blocks without a
+ *              split, fp16 copies of q, k, v that a conversion pre-pass writes once.
+ *              retnet_chunkwise_workspace_size gives the size that allows all of it.  The
+ *              workspace is in use until the call's work on `stream` completes; two calls
+ *              sharing one workspace must be ordered on the device.
  * Other arguments, errors and kernels as retnet_retention_chunkwise; a misaligned workspace
  * is RETNET_ERR_BAD_PARAM.
  */
@@ -218,10 +225,15 @@ RETNET_API retnet_status_t retnet_retention_chunkwise_static(const void* q, cons
                                                   const float* z_in, float* z_out, void* stream);
 
 /*
- * Workspace size (bytes) that lets retnet_retention_chunkwise_ws use its full segment split
- * for these dimensions: 6 * batch * heads * d_k * d_v * sizeof(float) (room for the states of
- * six pre-pass sub-segments).  Host-only; no device
- * access.  RETNET_ERR_NULL_PTR without `bytes`, RETNET_ERR_BAD_SHAPE for negative sizes.
+ * Workspace size (bytes) that lets retnet_retention_chunkwise_ws use all its forms for these
+ * dimensions, with a256(x) = x rounded up to a multiple of 256:
+ *   a256(4 * batch * seqlen * heads)                        (R~ row factors)
+ *   + a256(4 * batch * heads * d_k * 64)                     (R~ key-sum segment values)
+ *   + max(6 * batch * heads * d_k * d_v * 4,                 (six sub-segment states)
+ *         2 * a256(2 * batch * seqlen * heads * d_k) + a256(2 * batch * seqlen * heads * d_v))
+ *                                                            (fp16 copies of q, k, v).
+ * Host-only; no device access.  RETNET_ERR_NULL_PTR without `bytes`, RETNET_ERR_BAD_SHAPE for
+ * negative sizes.
  */
 RETNET_API retnet_status_t retnet_chunkwise_workspace_size(retnet_dims_t dims, size_t* bytes);
 

@@ -62,6 +62,8 @@ struct TcArgs {
   // Fused MSR epilogue: out = GroupNorm_h(o) * swish(gate), written to o's place.
   const void* gate;
   float eps;
+  // R~ normalisation: per-row factor [batch][L][heads] folded into the output scale (or nullptr)
+  const float* rden;
   // Sequence segments (pipelined kernel): CTA segment s writes the outputs of chunks
   // [seg_lo[s], seg_hi[s]) and first replays the state over chunks [0, seg_lo[s]).
   int n_seg;
@@ -1480,7 +1482,8 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE>::THREADS, 1)
       }
       if (!__all_sync(0xffffffffu, mbar_wait(bar(Q_O_FULL + (rb & 1)), (rb >> 1) & 1))) return false;
       tc_fence_after();
-      const float f = row_factor_f32(gam, sd, a.pos0 + t, a.flags) / sd;
+      float f = row_factor_f32(gam, sd, a.pos0 + t, a.flags) / sd;
+      if (a.rden && my_row >= 0 && my_row < rows) f *= __ldg(a.rden + (static_cast<int64_t>(b) * a.L + t) * a.heads + h);
       const float gx = (nb > 1) ? exp2f(static_cast<float>(u * T) * log2g) : 0.f;
       Tout* dst = static_cast<Tout*>(a.o) + ((static_cast<int64_t>(b) * a.L + t) * a.heads + h) * a.dv + dvb * DVS;
       // O (and X) from TMEM, o = (O + gamma^(uT) X) * s / c_p, 16-byte stores of 16 columns.
@@ -1934,6 +1937,7 @@ TcArgs make_args(const RetentionCall& c, int n_chunks, int nb) {
   a.batch = static_cast<int>(c.dims.batch);
   a.gate = c.gate;
   a.eps = c.eps;
+  a.rden = c.rden;
   a.dv = static_cast<int>(c.dims.d_v);
   a.n_chunks = n_chunks;
   a.pos0 = c.pos0;
@@ -2160,7 +2164,8 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 bool tc_chunkwise_supported(const RetentionCall& c) {
   const Dims& d = c.dims;
   if (c.in_dtype != RETNET_BF16) return false;
-  if (c.flags & RETNET_F_NORM_R) return false;
+  // R~ needs the row factors of the key-sum pass, in the caller's workspace
+  if ((c.flags & RETNET_F_NORM_R) && (!c.rden || force_serial_kernel())) return false;
   if (d.d_k != 64 && d.d_k != 128 && d.d_k != 256) return false;
   if (d.d_v % kDVS != 0) return false;
   if (c.chunk != 64 && c.chunk != 128 && c.chunk != 256 && c.chunk != 512) return false;
@@ -2265,6 +2270,12 @@ cudaError_t launch_state_advance(float* state, const float* w, const Dims& d, co
 
 int tc_chunkwise_launches(const RetentionCall& c) {
   if (force_serial_kernel()) return 1;
+  if (c.rden) {  // key-sum pass, then the kernels of the same call without R~
+    RetentionCall cc = c;
+    cc.rden = nullptr;
+    cc.flags &= ~static_cast<uint32_t>(RETNET_F_NORM_R);
+    return key_sum_launches(c.dims) + tc_chunkwise_launches(cc);
+  }
   const int T = pipe_tile_rows(c.dims.d_k, c.chunk);
   const int dvs = pipe_wide_slice(c, T) ? 128 : 64;
   const int nb = static_cast<int>(c.chunk / T);
@@ -2277,6 +2288,10 @@ int tc_chunkwise_launches(const RetentionCall& c) {
 }
 
 cudaError_t launch_tc_chunkwise(const RetentionCall& c, const HeadParams& hp, cudaStream_t s) {
+  if (c.rden) {
+    cudaError_t e = launch_key_sum(c, hp, s);
+    if (e != cudaSuccess) return e;
+  }
   if (c.out_dtype == RETNET_F32) return launch_out<float>(c, hp, s);
   return launch_out<__nv_bfloat16>(c, hp, s);
 }

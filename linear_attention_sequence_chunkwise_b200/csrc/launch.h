@@ -31,7 +31,21 @@ struct RetentionCall {
   // as o; nullptr = plain retention output.
   const void* gate = nullptr;
   float eps = 0.f;
+  // R~ normalisation on the tensor-core kernel: per-row factor 1 / max(|sum of scores|, 1),
+  // fp32 [batch][seqlen][heads], written by launch_key_sum (caller's workspace); nullptr = none.
+  // rden_seg: the key-sum pass's segment end values, fp32 [batch * heads][<= 64][d_k].
+  float* rden = nullptr;
+  float* rden_seg = nullptr;
 };
+
+// Sequence segments of the key-sum pass, at most; and the workspace bytes of the R~ factors
+// plus those segment values (each part rounded up to 256 bytes).
+constexpr int kMaxKeySumSegments = 64;
+inline size_t rden_region_bytes(const Dims& d) {
+  auto a256 = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  return a256(sizeof(float) * static_cast<size_t>(d.batch * d.seqlen * d.heads)) +
+         a256(sizeof(float) * static_cast<size_t>(d.batch * d.heads * d.d_k) * kMaxKeySumSegments);
+}
 
 // fp32 CUDA-core kernel: the parallel form (chunk >= seqlen, no state) and the chunkwise
 // form for any shape.
@@ -54,6 +68,11 @@ int tc_chunkwise_launches(const RetentionCall& c);
 cudaError_t launch_tc_segment_state(const RetentionCall& c, const HeadParams& hp, cudaStream_t s);
 // state <- g_h * state + w, g_h = hp.gamma[h] (fp32 [batch][heads][d_k][d_v], d_k*d_v % 4 == 0).
 cudaError_t launch_state_advance(float* state, const float* w, const Dims& d, const HeadParams& hp, cudaStream_t s);
+// The R~ row factors of a chunkwise call into c.rden (and z_out from z_in): bf16 q, k, d_k in
+// [64, 256], one pass over the keys.
+cudaError_t launch_key_sum(const RetentionCall& c, const HeadParams& hp, cudaStream_t s);
+// Kernel launches of launch_key_sum (1, or 2 when the sequence is cut into segments).
+int key_sum_launches(const Dims& d);
 // Reads (and optionally clears) the count of bounded waits that gave up in the tensor-core kernel.
 cudaError_t tc_wait_timeouts(unsigned int* count, bool clear);
 

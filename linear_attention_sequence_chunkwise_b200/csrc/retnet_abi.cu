@@ -101,6 +101,19 @@ retnet_status_t retnet_retention_parallel(const void* q, const void* k, const vo
 }
 
 namespace {
+// R~ on the tensor-core kernel: its row factors and the key-sum pass's segment values take
+// the front of the workspace, the rest serves the segment states or the conversion copies as
+// without R~.
+void carve_rden(RetentionCall& c) {
+  const size_t rb = rden_region_bytes(c.dims);
+  if (!(c.flags & RETNET_F_NORM_R) || !c.ws || c.ws_bytes < rb || c.dims.seqlen == 0) return;
+  c.rden = static_cast<float*>(c.ws);
+  const size_t rows = (sizeof(float) * static_cast<size_t>(c.dims.batch * c.dims.seqlen * c.dims.heads) + 255) &
+                      ~static_cast<size_t>(255);
+  c.rden_seg = reinterpret_cast<float*>(static_cast<char*>(c.ws) + rows);
+  c.ws = c.ws_bytes > rb ? static_cast<char*>(c.ws) + rb : nullptr;
+  c.ws_bytes -= rb;
+}
 retnet_status_t chunkwise_impl(const void* q, const void* k, const void* v, void* o, retnet_dims_t dims,
                                retnet_dtype_t in_dtype, retnet_dtype_t out_dtype, const float* gamma,
                                const float* theta, int64_t pos0, uint32_t flags, int64_t chunk,
@@ -125,6 +138,7 @@ retnet_status_t chunkwise_impl(const void* q, const void* k, const void* v, void
                   pos0, flags, chunk, true, state_in, state_out, z_in, z_out};
   c.ws = workspace;
   c.ws_bytes = workspace ? workspace_bytes : 0;
+  carve_rden(c);
   if (gate) {
     // Fused MSR epilogue: the tensor-core kernel only, decided on the host before any launch.
     c.gate = gate;
@@ -250,7 +264,10 @@ retnet_status_t retnet_chunkwise_workspace_size(retnet_dims_t dims, size_t* byte
   const size_t tok = static_cast<size_t>(dims.batch) * static_cast<size_t>(dims.seqlen) * static_cast<size_t>(dims.heads);
   auto a256 = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
   const size_t copies = 2 * a256(tok * static_cast<size_t>(dims.d_k) * 2) + a256(tok * static_cast<size_t>(dims.d_v) * 2);
-  *bytes = states > copies ? states : copies;
+  // plus, in front, the R~ row factors (fp32 [batch][seqlen][heads]) and the key-sum pass's
+  // segment values (fp32 [batch * heads][64][d_k])
+  const Dims d{dims.batch, dims.seqlen, dims.heads, dims.d_k, dims.d_v};
+  *bytes = rden_region_bytes(d) + (states > copies ? states : copies);
   return RETNET_OK;
 }
 
@@ -299,16 +316,22 @@ retnet_status_t retnet_state_advance(float* state, const float* w, int64_t batch
 
 int retnet_chunkwise_launches(retnet_dims_t dims, retnet_dtype_t in_dtype, uint32_t flags, int64_t chunk,
                               const float* gamma, size_t workspace_bytes) {
-  const int path = retnet_chunkwise_kernel(dims, in_dtype, flags, chunk, gamma);
+  // the kernel choice without R~ (R~ itself needs the workspace, below)
+  const int path = retnet_chunkwise_kernel(dims, in_dtype, flags & ~static_cast<uint32_t>(RETNET_F_NORM_R), chunk,
+                                           gamma);
   if (path < 0) return path;
   if (dims.seqlen == 0) return 0;
   if (path == 0) return 1;
   const retnet_status_t st = check_device();
   if (st != RETNET_OK) return -static_cast<int>(st);
-  RetentionCall c{nullptr, nullptr, nullptr, nullptr, Dims{dims.batch, dims.seqlen, dims.heads, dims.d_k, dims.d_v},
-                  in_dtype, RETNET_BF16, 0, flags, chunk, true, nullptr, nullptr, nullptr, nullptr};
+  alignas(16) static const uint32_t kAligned[4] = {0, 0, 0, 0};
+  RetentionCall c{kAligned, kAligned, kAligned, const_cast<uint32_t*>(kAligned),
+                  Dims{dims.batch, dims.seqlen, dims.heads, dims.d_k, dims.d_v}, in_dtype, RETNET_BF16, 0, flags,
+                  chunk, true, nullptr, nullptr, nullptr, nullptr};
   c.ws = workspace_bytes ? reinterpret_cast<void*>(static_cast<uintptr_t>(256)) : nullptr;  // only its size matters
   c.ws_bytes = workspace_bytes;
+  carve_rden(c);
+  if (!tc_chunkwise_supported(c)) return 1;  // R~ without room for its factors: the CUDA-core kernel
   return tc_chunkwise_launches(c);
 }
 

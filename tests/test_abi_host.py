@@ -124,7 +124,8 @@ def test_chunkwise_workspace_entry_points(lib):
         b, L, h, dk, dv = dims
         states = 6 * b * h * dk * dv * 4
         copies = 2 * a256(b * L * h * dk * 2) + a256(b * L * h * dv * 2)
-        assert rn.retnet_chunkwise_workspace_size(dims) == max(states, copies)
+        rden = a256(b * L * h * 4) + a256(b * h * dk * 64 * 4)  # R~ row factors and key-sum segments, in front
+        assert rn.retnet_chunkwise_workspace_size(dims) == rden + max(states, copies)
     assert rn.retnet_chunkwise_workspace_size((0, 0, 0, 0, 0)) == 0
     out = ctypes.c_size_t(0)
     assert lib.retnet_chunkwise_workspace_size(rn.Dims(1, 8, -2, 4, 4), ctypes.byref(out)) == 2

@@ -11,7 +11,7 @@ import torch
 import linear_attention_sequence_chunkwise_b200 as rn
 import oracle
 import synth_inputs as si
-from gpu_util import TOL_BF16, dev, err, err_bf16_out, require_gpu
+from gpu_util import TOL_BF16, TOL_F32, dev, err, err_bf16_out, require_gpu
 
 pytestmark = pytest.mark.gpu
 FLAGS = rn.F_XPOS | rn.F_SCALE_SQRT_D | rn.F_NORM_D
@@ -293,3 +293,68 @@ def test_serial_kernel_variant_in_subprocess():
                         "-k", "tc_matches_oracle or tc_state_in or tc_flag", os.path.join(here, "test_gpu_tc_chunkwise.py")],
                        env=env, capture_output=True, text=True, timeout=900)
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
+
+
+@pytest.mark.parametrize("dk,dv,B,L,pos0,bias,with_state", [
+    (128, 128, 64, 300, 0, 0.5, False),   # 128-column slices, one launch after the key sum
+    (64, 64, 128, 517, 7, 0.0, True),     # carried-in state and key sum
+    (256, 128, 256, 600, 1000, 0.5, True),  # pre-converted, 4 sub-blocks a chunk
+    (128, 256, 512, 1100, 0, 0.3, False),
+    (128, 128, 64, 64 * 33 + 1, 0, 0.5, True),  # few pairs: two-pass segments after the key sum
+    (256, 64, 64, 1, 3, 0.5, True)])
+def test_tc_norm_r_matches_oracle(dk, dv, B, L, pos0, bias, with_state):
+    """R~ on the tensor-core kernel (workspace form): a key-sum pass writes each row's factor
+    1/max(|sum of scores|, 1) and z_out, the kernel folds it into its row scale.  Outputs,
+    state and z against the oracle; q and k carry a mean (bias) so that most rows' sums exceed
+    1 and the normalisation is active.
+
+    Bar: R~ divides each row by its own D_n = max(|sum of scores|, 1) >= 1, which leaves rows of
+    very different sizes (early rows keep D ~ 1, later ones are divided by tens), so max|err| /
+    rms over the normalised output weighs an early row's ordinary error by the shrunken rms of
+    the rest.  The bf16 bar is applied to the output scaled back by the oracle's D_n
+    (out * D_n against the oracle's output without R~, which is ref * D_n exactly); a wrong
+    row factor on the GPU shows there as its relative error.  The plain figure is printed."""
+    b, h = 2, 3
+    q, k, v = si.qkv(b, L, h, dk, dv, 900 + dk + B, "bf16")
+    q = (q.float() + bias).to(q.dtype)
+    k = (k.float() + bias).to(k.dtype)
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+    S0 = si.decode_state(b, h, dk, dv, 901, std=0.05) if with_state else None
+    z0 = si.randn((b, h, dk), 902, "f32", std=3.0) if with_state else None
+    ref, Sref, zref = oracle.chunkwise(q, k, v, g, B, th, pos0, oracle.F_ALL, state_in=S0, z_in=z0)
+    plain, _, _ = oracle.chunkwise(q, k, v, g, B, th, pos0, FLAGS, state_in=S0, z_in=z0)
+    ref, plain = np.asarray(ref), np.asarray(plain)
+    # D_n = ||plain_n|| / ||ref_n|| per (token, head) row (ref = plain / D_n)
+    D = np.sqrt((plain ** 2).sum(-1, keepdims=True) / np.maximum((ref ** 2).sum(-1, keepdims=True), 1e-300))
+    assert np.all(D >= 1 - 1e-9)
+    if bias:
+        active = np.mean(D[..., 0] > 1 + 1e-9)
+        assert active > 0.3, active
+    nbytes = rn.retnet_chunkwise_workspace_size((b, L, h, dk, dv))
+    n = rn.retnet_chunkwise_launches((b, L, h, dk), dv, rn.BF16, oracle.F_ALL, B, g, nbytes)
+    assert n >= 2, n  # the key-sum pass, then the tensor-core kernel(s)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    o = torch.empty(b, L, h, dv, device="cuda")
+    so = torch.empty(b, h, dk, dv, device="cuda")
+    zo = torch.empty(b, h, dk, device="cuda")
+    rn.retnet_retention_chunkwise_ws(dev(q), dev(k), dev(v), o, g, th, pos0, oracle.F_ALL, B,
+                                     None if S0 is None else dev(S0), so, None if z0 is None else dev(z0), zo,
+                                     workspace=ws)
+    torch.cuda.synchronize()
+    e = err(o.cpu().double().numpy() * D, plain)
+    print(f"R~ dk={dk} dv={dv} B={B} L={L} launches={n}: rescaled max|err|/rms = {e:.3e}, "
+          f"plain {err(o, ref):.3e}")
+    assert e <= TOL_BF16
+    assert err(so, Sref) <= TOL_BF16
+    assert err(zo, zref) <= TOL_F32
+
+
+def test_tc_norm_r_needs_room_for_its_factors():
+    """R~ with a workspace too small for the row factors takes the CUDA-core kernel (one
+    launch); with room, the key-sum pass comes first."""
+    g = si.gamma_schedule(4)
+    a256 = lambda x: (x + 255) // 256 * 256
+    need = a256(2 * 300 * 4 * 4) + a256(2 * 4 * 128 * 64 * 4)  # row factors + key-sum segment values
+    assert rn.retnet_chunkwise_launches((2, 300, 4, 128), 64, rn.BF16, oracle.F_ALL, 64, g, need - 256) == 1
+    # two key-sum passes (the sequence in segments), then the kernel (no room for a split)
+    assert rn.retnet_chunkwise_launches((2, 300, 4, 128), 64, rn.BF16, oracle.F_ALL, 64, g, need) == 3
