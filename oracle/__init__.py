@@ -51,8 +51,10 @@ def _load():
         lib.oracle_msr_epilogue.argtypes = [dp, dp, dp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                             ctypes.c_double, ctypes.c_int]
         lib.oracle_num_threads.argtypes = [ctypes.c_int]
+        lib.oracle_backward.argtypes = [dp, dp, dp, dp, dp, dp, dp, _Dims, dp, dp, ctypes.c_int64, ctypes.c_uint,
+                                        dp, dp, ctypes.c_int]
         for f in (lib.oracle_parallel, lib.oracle_recurrent, lib.oracle_chunkwise,
-                  lib.oracle_msr_epilogue, lib.oracle_num_threads):
+                  lib.oracle_msr_epilogue, lib.oracle_num_threads, lib.oracle_backward):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -160,3 +162,22 @@ def msr_epilogue(y, g, heads, eps=1e-5, nthreads=0):
                                      int(nthreads))
     assert rc == 0
     return out
+
+
+def backward(q, k, v, dout, gamma, theta=None, pos0=0, flags=F_ALL & ~F_NORM_R, state_in=None, nthreads=0):
+    """Gradient of the retention output O (with an optional state_in before the first token)
+    with respect to q, k, v and state_in, given dO (product rule on the definition; no R~).
+
+    Returns (dq, dk, dv, dstate) in fp64; dstate is None without state_in.
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(dout)
+    b, L, h, dk = q.shape
+    dv = v.shape[-1]
+    gq, gk, gv = np.zeros(q.shape), np.zeros(k.shape), np.zeros(v.shape)
+    si = None if state_in is None else _f64(state_in)
+    ds = None if state_in is None else np.zeros((b, h, dk, dv))
+    g, th = _f64(gamma), _theta_arr(theta, dk)
+    rc = _load().oracle_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(gq), _ptr(gk), _ptr(gv), _dims(q, v),
+                                 _ptr(g), _ptr(th), int(pos0), int(flags), _ptr(si), _ptr(ds), int(nthreads))
+    assert rc == 0, "the oracle's gradient does not cover R~"
+    return gq, gk, gv, ds

@@ -331,3 +331,102 @@ int oracle_msr_epilogue(const double *y, const double *g, double *out, int64_t t
     }
     return 0;
 }
+
+/*
+ * Gradient of the retention forward, for training ([RN] §2.4 notes that training uses the
+ * chunkwise form; its outputs are those of the parallel form, so the gradient is that of the
+ * definition).  With q~_n, k~_n the rotated rows (xPos), f_n the row factor of §三.3 (no R~)
+ * and an optional state S0 before the first token (the chunkwise / recurrent state_in):
+ *     O_n = f_n [ sum_{m<=n} gamma^(n-m) (q~_n . k~_m) v_m  +  gamma^(n+1) q~_n S0 ].
+ * Given dO (the gradient of a loss with respect to O), by the product rule:
+ *     dq~_n = f_n [ sum_{m<=n} gamma^(n-m) (dO_n . v_m) k~_m  +  gamma^(n+1) S0 dO_n ]
+ *     dk~_m = sum_{n>=m} f_n gamma^(n-m) (dO_n . v_m) q~_n
+ *     dv_m  = sum_{n>=m} f_n gamma^(n-m) (q~_n . k~_m) dO_n
+ *     dS0   = sum_n f_n gamma^(n+1) q~_n^T dO_n
+ * and dq_n = R(p theta)^T dq~_n, dk_m = R(p theta)^T dk~_m (the rotation is orthogonal).
+ * R~ (a division by a function of q and k) is not covered: flags with it return -1.
+ * state_in and dstate (both [batch][heads][d_k][d_v]) may be NULL.
+ */
+static void xpos_rotate_back(const double *y, double *x, int64_t d, const double *theta, int64_t p, int on) {
+    if (!on) {
+        memcpy(x, y, sizeof(double) * (size_t)d);
+        return;
+    }
+    for (int64_t j = 0; j < d / 2; ++j) {
+        double a = (double)p * theta[j];
+        double c = cos(a), s = sin(a);
+        double y0 = y[2 * j], y1 = y[2 * j + 1];
+        x[2 * j] = y0 * c + y1 * s;
+        x[2 * j + 1] = -y0 * s + y1 * c;
+    }
+}
+
+int oracle_backward(const double *q, const double *k, const double *v, const double *dout, double *dq, double *dk,
+                    double *dv, oracle_dims_t d, const double *gamma, const double *theta, int64_t pos0,
+                    unsigned flags, const double *state_in, double *dstate, int nthreads) {
+    if (flags & ORACLE_F_NORM_R) return -1;
+    set_threads(nthreads);
+    const int xpos = (flags & ORACLE_F_XPOS) != 0;
+    const int64_t pairs = d.batch * d.heads, L = d.seqlen, dk_ = d.d_k, dv_ = d.d_v;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < pairs; ++bh) {
+        int64_t b = bh / d.heads, hh = bh % d.heads;
+        double g = gamma[hh];
+        double *qr = (double *)malloc(sizeof(double) * (size_t)(L * dk_));
+        double *kr = (double *)malloc(sizeof(double) * (size_t)(L * dk_));
+        double *f = (double *)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+        double *tq = (double *)malloc(sizeof(double) * (size_t)dk_);
+        double *tk = (double *)malloc(sizeof(double) * (size_t)dk_);
+        const double *S0 = state_in ? state_in + bh * dk_ * dv_ : NULL;
+        for (int64_t t = 0; t < L; ++t) {
+            xpos_rotate(row_qk(q, &d, b, t, hh), qr + t * dk_, dk_, theta, pos0 + t, xpos);
+            xpos_rotate(row_qk(k, &d, b, t, hh), kr + t * dk_, dk_, theta, pos0 + t, xpos);
+            f[t] = row_factor(g, dk_, pos0 + t, flags);
+        }
+        for (int64_t n = 0; n < L; ++n) { /* dq */
+            const double *don = row_v(dout, &d, b, n, hh);
+            memset(tq, 0, sizeof(double) * (size_t)dk_);
+            for (int64_t m = 0; m <= n; ++m) {
+                double w = pow(g, (double)(n - m)) * dot(don, row_v(v, &d, b, m, hh), dv_);
+                for (int64_t i = 0; i < dk_; ++i) tq[i] += w * kr[m * dk_ + i];
+            }
+            if (S0) {
+                double gn = pow(g, (double)(n + 1));
+                for (int64_t i = 0; i < dk_; ++i) tq[i] += gn * dot(S0 + i * dv_, don, dv_);
+            }
+            for (int64_t i = 0; i < dk_; ++i) tq[i] *= f[n];
+            xpos_rotate_back(tq, (double *)row_qk(dq, &d, b, n, hh), dk_, theta, pos0 + n, xpos);
+        }
+        for (int64_t m = 0; m < L; ++m) { /* dk, dv */
+            const double *vm = row_v(v, &d, b, m, hh);
+            double *dvm = (double *)row_v(dv, &d, b, m, hh);
+            memset(tk, 0, sizeof(double) * (size_t)dk_);
+            memset(dvm, 0, sizeof(double) * (size_t)dv_);
+            for (int64_t n = m; n < L; ++n) {
+                const double *don = row_v(dout, &d, b, n, hh);
+                double a = f[n] * pow(g, (double)(n - m));
+                double wk = a * dot(don, vm, dv_);
+                double wv = a * dot(qr + n * dk_, kr + m * dk_, dk_);
+                for (int64_t i = 0; i < dk_; ++i) tk[i] += wk * qr[n * dk_ + i];
+                for (int64_t j = 0; j < dv_; ++j) dvm[j] += wv * don[j];
+            }
+            xpos_rotate_back(tk, (double *)row_qk(dk, &d, b, m, hh), dk_, theta, pos0 + m, xpos);
+        }
+        if (dstate) { /* dS0 */
+            double *dS = dstate + bh * dk_ * dv_;
+            memset(dS, 0, sizeof(double) * (size_t)(dk_ * dv_));
+            for (int64_t n = 0; n < L; ++n) {
+                const double *don = row_v(dout, &d, b, n, hh);
+                double a = f[n] * pow(g, (double)(n + 1));
+                for (int64_t i = 0; i < dk_; ++i)
+                    for (int64_t j = 0; j < dv_; ++j) dS[i * dv_ + j] += a * qr[n * dk_ + i] * don[j];
+            }
+        }
+        free(qr);
+        free(kr);
+        free(f);
+        free(tq);
+        free(tk);
+    }
+    return 0;
+}

@@ -35,6 +35,13 @@ MUTANTS = [
      "double sw = 1.0 / (1.0 + exp(-gr[j]));", None),
     ("chunk_cross_term_dropped", "acc[j] += xi * cr;", "acc[j] += 0.0 * xi * cr;", None),
     ("state_in_ignored", "if (state_in) memcpy(S, state_in + bh * ssz", "if (0) memcpy(S, state_in + bh * ssz", None),
+    ("bwd_state_term_dropped", "tq[i] += gn * dot(S0 + i * dv_, don, dv_);",
+     "tq[i] += 0.0 * gn * dot(S0 + i * dv_, don, dv_);", None),
+    ("bwd_rotation_not_transposed", "x[2 * j] = y0 * c + y1 * s;", "x[2 * j] = y0 * c - y1 * s;", None),
+    ("bwd_dk_dv_without_row_factor", "double a = f[n] * pow(g, (double)(n - m));",
+     "double a = pow(g, (double)(n - m));", None),
+    ("bwd_dstate_decay_off_by_one", "double a = f[n] * pow(g, (double)(n + 1));",
+     "double a = f[n] * pow(g, (double)n);", None),
 ]
 
 

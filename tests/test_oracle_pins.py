@@ -295,3 +295,53 @@ def test_gamma_schedule_golden():
     want = np.array([float.fromhex(r[1]) for r in rows])
     got = si.gamma_schedule(16).astype(np.float64)
     assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("flags,pos0", [(oracle.F_XPOS | oracle.F_SCALE_SQRT_D | oracle.F_NORM_D, 5), (0, 0),
+                                        (oracle.F_XPOS, 123)])
+def test_backward_is_the_derivative_of_the_recurrent_form(flags, pos0):
+    """oracle.backward against central finite differences of oracle.recurrent (the page's §2.2
+    form, with a state before the first token) for L = sum(dO * O): every element of q, k, v
+    and the state.  Exact up to the difference quotient's own error (h = 1e-5, fp64)."""
+    rng = np.random.default_rng(31)
+    b, L, h, dk, dv = 1, 6, 2, 4, 3
+    q, k = rng.standard_normal((b, L, h, dk)), rng.standard_normal((b, L, h, dk))
+    v, do = rng.standard_normal((b, L, h, dv)), rng.standard_normal((b, L, h, dv))
+    S0 = rng.standard_normal((b, h, dk, dv))
+    g = np.array([0.9, 0.7])
+    th = np.array([0.3, 1.1])
+    gq, gk, gv, gs = oracle.backward(q, k, v, do, g, th, pos0, flags, state_in=S0)
+
+    def loss(q_, k_, v_, s_):
+        o, _, _ = oracle.recurrent(q_, k_, v_, g, th, pos0, flags, state_in=s_)
+        return float((o * do).sum())
+
+    eps = 1e-5
+    for name, x, grad in (("q", q, gq), ("k", k, gk), ("v", v, gv), ("state", S0, gs)):
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args = {"q": (q, k, v, S0), "k": (q, k, v, S0), "v": (q, k, v, S0), "state": (q, k, v, S0)}[name]
+            a_p, a_m = list(args), list(args)
+            pos = ["q", "k", "v", "state"].index(name)
+            a_p[pos], a_m[pos] = xp, xm
+            fd[idx] = (loss(*a_p) - loss(*a_m)) / (2 * eps)
+        scale = max(np.abs(fd).max(), 1e-12)
+        assert np.abs(grad - fd).max() / scale < 1e-7, (name, np.abs(grad - fd).max() / scale)
+
+
+def test_backward_without_state_and_linearity():
+    """Without a state the state gradient is absent; dv is linear in dO and does not depend on v
+    (O is linear in v), checked on two dO."""
+    rng = np.random.default_rng(32)
+    q, k = rng.standard_normal((2, 9, 1, 4)), rng.standard_normal((2, 9, 1, 4))
+    v = rng.standard_normal((2, 9, 1, 2))
+    d1, d2 = rng.standard_normal((2, 9, 1, 2)), rng.standard_normal((2, 9, 1, 2))
+    g = np.array([0.8])
+    _, _, a, s = oracle.backward(q, k, v, d1, g, None, 0, oracle.F_SCALE_SQRT_D)
+    _, _, b_, _ = oracle.backward(q, k, 3 * v + 1, d2, g, None, 0, oracle.F_SCALE_SQRT_D)
+    _, _, c, _ = oracle.backward(q, k, v, 2 * d1 - d2, g, None, 0, oracle.F_SCALE_SQRT_D)
+    assert s is None
+    np.testing.assert_allclose(c, 2 * a - b_, rtol=1e-12, atol=1e-12)
