@@ -308,6 +308,36 @@ def bench_msr(rn, device, stream, steps, peaks):
     return res
 
 
+def bench_backward(rn, device, stream, steps, peaks):
+    """Gradient of the forward (dq, dk, dv) on the headline workload, bf16 inputs, fp32 out:
+    the fp32 CUDA-core first path (O(L^2) per (batch, head)), against the bf16 tensor peak with
+    2x the forward's algorithmic FLOPs (the usual backward/forward ratio)."""
+    import torch
+
+    import synth_inputs as si
+    c = MAIN
+    b, L, h, dk, dv, B = c["batch"], c["seqlen"], c["heads"], c["d_k"], c["d_v"], c["chunk"]
+    q, k, v = si.qkv(b, L, h, dk, dv, 11, "bf16")
+    q, k, v = q.to(device), k.to(device), v.to(device)
+    do = si.randn((b, L, h, dv), 12, "bf16").to(device)
+    dq, dk_ = torch.empty(b, L, h, dk, device=device), torch.empty(b, L, h, dk, device=device)
+    dv_ = torch.empty(b, L, h, dv, device=device)
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+    ws = torch.empty(rn.retnet_backward_workspace_size((b, L, h, dk, dv)), dtype=torch.uint8, device=device)
+
+    def step(i):
+        rn.retnet_retention_backward(q, k, v, do, dq, dk_, dv_, g, th, 0, FLAGS, workspace=ws, stream=stream)
+
+    step(0)
+    torch.cuda.synchronize()
+    secs = time_steps(step, steps, stream) / steps
+    flops = 2 * b * L * h * flops_per_token_head(dk, dv, B)
+    tf = flops / secs / 1e12
+    return {"workload": "backward_" + c["workload"], "us_per_step": secs * 1e6, "tokens_per_s": b * L / secs,
+            "tflops": tf, "frac_bf16_peak": tf / peaks["bf16"], "kernel": "fp32 CUDA cores (first path)",
+            "launches_per_step": 3, "gpu_launches": 3 * steps}
+
+
 def oracle_sample(cfg, budget_s):
     """Size a bounded sample of the workload for the fp64 oracle: whole batch rows (all heads)."""
     import oracle
@@ -451,6 +481,8 @@ def main_ours(args):
         line["long"] = bench_long(rn, device, stream, 10, peaks)
     if world == 1 and "msr" in args.sections:
         line["msr"] = bench_msr(rn, device, stream, 10, peaks)
+    if world == 1 and "backward" in args.sections:
+        line["backward"] = bench_backward(rn, device, stream, 3, peaks)
     clocks.stop()
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, args.cpu_seconds)
@@ -491,8 +523,8 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--sections", default="e2e,decode,long,msr",
-                    help="comma list of extra legs to run beside the timed step: e2e, decode, long, msr")
+    ap.add_argument("--sections", default="e2e,decode,long,msr,backward",
+                    help="comma list of extra legs to run beside the timed step: e2e, decode, long, msr, backward")
     ap.add_argument("--decode-steps", type=int, default=200)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

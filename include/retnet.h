@@ -289,6 +289,32 @@ RETNET_API retnet_status_t retnet_msr_chunkwise(const void* q, const void* k, co
                                      size_t workspace_bytes, void* stream);
 
 /*
+ * Gradient of the retention forward, for training (§2.4: training runs the chunkwise form,
+ * whose outputs are those of the parallel form §2.3, so this is the derivative of that
+ * definition).  With q~, k~ the xPos-rotated rows, f_n the row factor of §三.3 and S0 =
+ * state_in (the state before the first token, as for retnet_retention_chunkwise):
+ *   O_n = f_n [ sum_{m<=n} gamma^(n-m) (q~_n . k~_m) v_m + gamma^(n+1) q~_n S0 ],
+ * and for a loss with gradient dout = dL/dO:
+ *   dq, dk: [batch][seqlen][heads][d_k] fp32;  dv: [batch][seqlen][heads][d_v] fp32;
+ *   dstate: [batch][heads][d_k][d_v] fp32, dL/dS0 (may be NULL: not computed).
+ *   q, k, v, dout in in_dtype (dout laid out as v); state_in fp32 or NULL (zeros).
+ *   workspace: device memory of retnet_backward_workspace_size bytes (16-byte aligned):
+ *   the rotated q and k in fp32.
+ * Runs on fp32 CUDA cores, O(seqlen^2) per (batch, head): a first path, not a tuned one.
+ * d_k, d_v <= 256 and seqlen <= 524280, else RETNET_ERR_UNSUPPORTED; RETNET_F_NORM_R (R~, a
+ * division by a function of q and k) is RETNET_ERR_UNSUPPORTED.  Outputs do not alias inputs.
+ */
+RETNET_API retnet_status_t retnet_retention_backward(const void* q, const void* k, const void* v,
+                                          const void* dout, float* dq, float* dk, float* dv,
+                                          retnet_dims_t dims, retnet_dtype_t in_dtype,
+                                          const float* gamma, const float* theta, int64_t pos0,
+                                          uint32_t flags, const float* state_in, float* dstate,
+                                          void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes of retnet_retention_backward: 2 * 4 * batch * seqlen * heads * d_k. */
+RETNET_API retnet_status_t retnet_backward_workspace_size(retnet_dims_t dims, size_t* bytes);
+
+/*
  * Which kernel retnet_retention_chunkwise runs for these arguments (host-only decision, no
  * device access): 1 = the tcgen05 tensor-core kernel, 0 = the fp32 CUDA-core kernel,
  * negative = the arguments would be rejected (the negated status).  Device pointers that

@@ -11,6 +11,7 @@ The functions carry the C names:
   retnet_retention_step       -- §2.2 Recurrent Mode, one decode token for a batch
   retnet_msr_epilogue         -- §三.2 GroupNorm per head, then the swish gate
   retnet_msr_chunkwise        -- §2.4 and §三.2 in one kernel (the retention output stays on chip)
+  retnet_retention_backward   -- gradient of the forward (dq, dk, dv, d state) for training
 with the §三.3 normalisations chosen by flags.  Tensors are dense BLHD (see the header).
 """
 import ctypes
@@ -35,7 +36,8 @@ STATIC_SCRATCH_BYTES = 16 << 20  # RETNET_STATIC_SCRATCH_BYTES
 EXPORTS = ("retnet_retention_parallel", "retnet_retention_chunkwise", "retnet_retention_chunkwise_ws",
            "retnet_retention_chunkwise_static", "retnet_chunkwise_segment_state", "retnet_state_advance",
            "retnet_chunkwise_workspace_size", "retnet_retention_step", "retnet_msr_epilogue",
-           "retnet_msr_chunkwise", "retnet_msr_chunkwise_launches",
+           "retnet_msr_chunkwise", "retnet_msr_chunkwise_launches", "retnet_retention_backward",
+           "retnet_backward_workspace_size",
            "retnet_chunkwise_kernel", "retnet_chunkwise_launches", "retnet_debug_wait_timeouts",
            "retnet_status_string", "retnet_version")
 
@@ -88,6 +90,11 @@ def load(path: str = None):
     lib.retnet_msr_chunkwise.argtypes = [_vp, _vp, _vp, _vp, _vp, Dims, _i32, _i32, _fp, _fp, _i64, _u32, _i64,
                                          ctypes.c_float, _vp, _vp, _vp, ctypes.c_size_t, _vp]
     lib.retnet_msr_chunkwise_launches.argtypes = [Dims, _i32, _u32, _i64, _fp, ctypes.c_size_t]
+    lib.retnet_retention_backward.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, Dims, _i32, _fp, _fp, _i64, _u32,
+                                              _vp, _vp, _vp, ctypes.c_size_t, _vp]
+    lib.retnet_retention_backward.restype = _i32
+    lib.retnet_backward_workspace_size.argtypes = [Dims, ctypes.POINTER(ctypes.c_size_t)]
+    lib.retnet_backward_workspace_size.restype = _i32
     lib.retnet_msr_chunkwise_launches.restype = _i32
     for name in ("retnet_retention_parallel", "retnet_retention_chunkwise", "retnet_retention_chunkwise_ws",
                  "retnet_retention_chunkwise_static", "retnet_retention_step", "retnet_msr_epilogue",
@@ -331,6 +338,39 @@ def retnet_msr_chunkwise_launches(shape_qk, d_v, in_dtype, flags, chunk, gamma, 
     gm = _host_f32(gamma, h)
     return load().retnet_msr_chunkwise_launches(Dims(b, L, h, dk, d_v), int(in_dtype), int(flags), int(chunk),
                                                 _fptr(gm), int(workspace_bytes))
+
+
+def retnet_backward_workspace_size(dims) -> int:
+    """Bytes of workspace for retnet_retention_backward; dims = (batch, seqlen, heads, d_k, d_v)."""
+    out = ctypes.c_size_t(0)
+    _check(load().retnet_backward_workspace_size(Dims(*[int(x) for x in dims]), ctypes.byref(out)))
+    return out.value
+
+
+def retnet_retention_backward(q, k, v, dout, dq, dk, dv, gamma, theta=None, pos0=0,
+                              flags=F_XPOS | F_SCALE_SQRT_D | F_NORM_D, state_in=None, dstate=None, workspace=None,
+                              stream=None):
+    """Gradient of the forward into fp32 dq, dk (shape of q), dv (shape of v) and dstate
+    (batch, heads, d_k, d_v) if given; dout has v's shape and q's dtype."""
+    _require_cuda(q, k, v, dout, dq, dk, dv, state_in, dstate, workspace)
+    b, L, h, d_k = q.shape
+    d_v = v.shape[-1]
+    for t, shp in ((k, q.shape), (dq, q.shape), (dk, q.shape), (v, (b, L, h, d_v)), (dout, (b, L, h, d_v)),
+                   (dv, (b, L, h, d_v))):
+        if tuple(t.shape) != tuple(shp):
+            raise ValueError("shape mismatch between q, k, v, dout and the gradients")
+    if dout.dtype != q.dtype:
+        raise ValueError("dout must have the dtype of q")
+    dims = (b, L, h, d_k, d_v)
+    if workspace is None:
+        import torch
+        workspace = torch.empty(retnet_backward_workspace_size(dims), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    gm, th = _host_f32(gamma, h), _host_f32(theta, d_k // 2)
+    _check(load().retnet_retention_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                                            Dims(*dims), _dtype_code(q), _fptr(gm), _fptr(th), int(pos0), int(flags),
+                                            _ptr(state_in), _ptr(dstate), _ptr(workspace), ws_bytes,
+                                            _stream(stream)))
 
 
 def retnet_chunkwise_kernel(shape_qk, d_v, in_dtype, flags, chunk, gamma):

@@ -90,6 +90,28 @@ struct StepCall {
 };
 cudaError_t launch_step(const StepCall& c, const HeadParams& hp, cudaStream_t s);
 
+// Gradient of the retention forward (dq, dk, dv, d state) on fp32 CUDA cores.
+struct BackwardCall {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* dout;
+  float* dq;
+  float* dk;
+  float* dv;
+  Dims dims;
+  retnet_dtype_t in_dtype;
+  int64_t pos0;
+  uint32_t flags;
+  const float* state_in;  // S0 before the first token (or nullptr)
+  float* dstate;          // gradient of S0 (or nullptr)
+  void* ws;               // backward_workspace_bytes(dims): rotated q and k, fp32
+};
+size_t backward_workspace_bytes(const Dims& d);
+bool backward_supported(const Dims& d);
+int backward_launches(const BackwardCall& c);
+cudaError_t launch_backward(const BackwardCall& c, const HeadParams& hp, cudaStream_t s);
+
 cudaError_t launch_msr_epilogue(const void* y, const void* g, void* out, int64_t tokens, int64_t heads,
                                 int64_t d_v, float eps, retnet_dtype_t in_dtype, retnet_dtype_t out_dtype,
                                 cudaStream_t s);

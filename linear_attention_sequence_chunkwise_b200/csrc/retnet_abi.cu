@@ -395,6 +395,40 @@ retnet_status_t retnet_retention_step(const void* q, const void* k, const void* 
   return from_cuda(launch_step(c, hp, static_cast<cudaStream_t>(stream)));
 }
 
+retnet_status_t retnet_backward_workspace_size(retnet_dims_t dims, size_t* bytes) {
+  if (!bytes) return RETNET_ERR_NULL_PTR;
+  if (dims.batch < 0 || dims.seqlen < 0 || dims.heads < 0 || dims.d_k < 0 || dims.d_v < 0) return RETNET_ERR_BAD_SHAPE;
+  *bytes = backward_workspace_bytes(Dims{dims.batch, dims.seqlen, dims.heads, dims.d_k, dims.d_v});
+  return RETNET_OK;
+}
+
+retnet_status_t retnet_retention_backward(const void* q, const void* k, const void* v, const void* dout, float* dq,
+                                          float* dk, float* dv, retnet_dims_t dims, retnet_dtype_t in_dtype,
+                                          const float* gamma, const float* theta, int64_t pos0, uint32_t flags,
+                                          const float* state_in, float* dstate, void* workspace,
+                                          size_t workspace_bytes, void* stream) {
+  retnet_status_t st = check_common(dims, in_dtype, RETNET_F32, pos0, flags, true);
+  if (st != RETNET_OK) return st;
+  if (flags & RETNET_F_NORM_R) return RETNET_ERR_UNSUPPORTED;
+  const Dims d{dims.batch, dims.seqlen, dims.heads, dims.d_k, dims.d_v};
+  if (!backward_supported(d) || (dims.seqlen + 7) / 8 > 65535 || dims.batch * dims.heads > 0x7fffffffLL)
+    return RETNET_ERR_UNSUPPORTED;
+  if (dims.seqlen == 0) {
+    if (dstate) {
+      const size_t sb = sizeof(float) * static_cast<size_t>(dims.batch * dims.heads * dims.d_k * dims.d_v);
+      if (cudaMemsetAsync(dstate, 0, sb, static_cast<cudaStream_t>(stream)) != cudaSuccess) return RETNET_ERR_CUDA;
+    }
+    return RETNET_OK;
+  }
+  if (!q || !k || !v || !dout || !dq || !dk || !dv || !workspace) return RETNET_ERR_NULL_PTR;
+  if (workspace_bytes < backward_workspace_bytes(d) || !aligned16(workspace)) return RETNET_ERR_BAD_PARAM;
+  HeadParams hp;
+  if ((st = fill_params(&hp, gamma, theta, dims.heads, dims.d_k, flags)) != RETNET_OK) return st;
+  if ((st = check_device()) != RETNET_OK) return st;
+  BackwardCall c{q, k, v, dout, dq, dk, dv, d, in_dtype, pos0, flags, state_in, dstate, workspace};
+  return from_cuda(launch_backward(c, hp, static_cast<cudaStream_t>(stream)));
+}
+
 retnet_status_t retnet_msr_epilogue(const void* y, const void* g, void* out, int64_t tokens, int64_t heads,
                                     int64_t d_v, float eps, retnet_dtype_t in_dtype, retnet_dtype_t out_dtype,
                                     void* stream) {

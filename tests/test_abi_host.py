@@ -182,6 +182,25 @@ def test_fused_msr_validation(lib):
     assert lib.retnet_msr_chunkwise_launches(rn.Dims(1, 64, 2, 128, 128), 1, 0, 0, gp, 0) == -4  # chunk 0
 
 
+def test_backward_validation(lib):
+    """The gradient entry point: workspace size formula, R~ unsupported, NULL and workspace
+    checks before any device access."""
+    assert rn.retnet_backward_workspace_size((2, 10, 3, 64, 32)) == 2 * 4 * 2 * 10 * 3 * 64
+    g = _gamma(2)
+    gp = g.ctypes.data_as(rn._fp)
+    d = rn.Dims(1, 8, 2, 64, 64)
+    f = lib.retnet_retention_backward
+    args = lambda q=FAKE, ws=FAKE, wsb=1 << 20, flags=0: (q, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, d, 0, gp, None, 0,
+                                                          flags, None, None, ws, wsb, None)
+    assert f(*args(flags=rn.F_NORM_R)) == 5
+    assert f(*args(q=None)) == 1
+    assert f(*args(ws=None)) == 1
+    assert f(*args(wsb=16)) == 4
+    assert f(*args(ws=FAKE + 8)) == 4
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, rn.Dims(1, 8, 2, 512, 64), 0, gp, None, 0, 0, None, None,
+             FAKE, 1 << 30, None) == 5  # d_k beyond the gradient kernels' 256
+
+
 def test_binding_raises_without_library(tmp_path):
     import importlib
     mod = importlib.import_module("linear_attention_sequence_chunkwise_b200")

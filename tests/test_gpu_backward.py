@@ -1,0 +1,65 @@
+"""Parity of the retention gradient (retnet_retention_backward, fp32 CUDA cores) against the
+fp64 oracle's gradient (pinned by finite differences in test_oracle_pins.py).
+
+Bar: max|err|/rms(oracle) <= 1e-4 for every output (the arithmetic is fp32; bf16 inputs are
+exact in both).
+"""
+import numpy as np
+import pytest
+import torch
+
+import linear_attention_sequence_chunkwise_b200 as rn
+import oracle
+import synth_inputs as si
+from gpu_util import TOL_F32, dev, err, require_gpu
+
+pytestmark = pytest.mark.gpu
+FLAGS = rn.F_XPOS | rn.F_SCALE_SQRT_D | rn.F_NORM_D
+
+
+@pytest.fixture(autouse=True)
+def _gpu(cuda_lib):
+    require_gpu()
+
+
+@pytest.mark.parametrize("b,L,h,dk,dv,dtype,flags,pos0,with_state", [
+    (2, 100, 3, 64, 32, "f32", FLAGS, 5, True),
+    (1, 200, 2, 128, 128, "bf16", FLAGS, 0, False),
+    (1, 70, 2, 256, 256, "bf16", FLAGS, 1000, True),
+    (2, 37, 2, 6, 5, "f32", FLAGS, 3, True),   # ragged widths: lanes past d_k, d_v idle
+    (1, 1, 1, 64, 64, "f32", FLAGS, 0, True),  # one token
+    (1, 90, 4, 32, 64, "bf16", 0, 0, True),    # no rotation, no row factors
+])
+def test_backward_matches_oracle(b, L, h, dk, dv, dtype, flags, pos0, with_state):
+    q, k, v = si.qkv(b, L, h, dk, dv, 500 + dk + L, dtype)
+    do = si.randn((b, L, h, dv), 501 + L, dtype)
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+    S0 = si.decode_state(b, h, dk, dv, 502, std=0.3) if with_state else None
+    rq, rk, rv, rs = oracle.backward(q, k, v, do, g, th, pos0, flags, state_in=S0)
+    dq = torch.empty(b, L, h, dk, device="cuda")
+    dk_ = torch.empty_like(dq)
+    dv_ = torch.empty(b, L, h, dv, device="cuda")
+    ds = torch.empty(b, h, dk, dv, device="cuda")
+    rn.retnet_retention_backward(dev(q), dev(k), dev(v), dev(do), dq, dk_, dv_, g, th, pos0, flags,
+                                 state_in=None if S0 is None else dev(S0), dstate=ds)
+    torch.cuda.synchronize()
+    if S0 is None:  # dS0 does not depend on S0: the oracle gives it with a zero state
+        _, _, _, rs = oracle.backward(q, k, v, do, g, th, pos0, flags, state_in=np.zeros((b, h, dk, dv)))
+    errs = [err(dq, rq), err(dk_, rk), err(dv_, rv), err(ds, rs)]
+    print(f"backward b={b} L={L} h={h} dk={dk} dv={dv} {dtype}: dq/dk/dv/dS0 errors " +
+          " ".join(f"{e:.2e}" for e in errs))
+    assert max(errs) <= TOL_F32
+
+
+def test_backward_rejects_norm_r_and_checks_workspace():
+    b, L, h, dk, dv = 1, 16, 1, 64, 64
+    q, k, v = si.qkv(b, L, h, dk, dv, 9, "f32")
+    g = si.gamma_schedule(h)
+    out = [torch.empty(b, L, h, d, device="cuda") for d in (dk, dk, dv)]
+    with pytest.raises(RuntimeError, match="UNSUPPORTED"):
+        rn.retnet_retention_backward(dev(q), dev(k), dev(v), dev(v), *out, g, si.theta_schedule(dk),
+                                     flags=rn.F_ALL)
+    small = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(RuntimeError, match="BAD_PARAM"):
+        rn.retnet_retention_backward(dev(q), dev(k), dev(v), dev(v), *out, g, si.theta_schedule(dk),
+                                     workspace=small)
