@@ -309,9 +309,9 @@ def bench_msr(rn, device, stream, steps, peaks):
 
 
 def bench_backward(rn, device, stream, steps, peaks):
-    """Gradient of the forward (dq, dk, dv) on the headline workload, bf16 inputs, fp32 out:
-    the fp32 CUDA-core first path (O(L^2) per (batch, head)), against the bf16 tensor peak with
-    2x the forward's algorithmic FLOPs (the usual backward/forward ratio)."""
+    """Gradient of the forward (dq, dk, dv) on the headline workload, bf16 inputs, fp32 out, on
+    the path the library takes (tensor cores: six runs of the chunkwise kernel), against the
+    bf16 tensor peak with 2x the forward's algorithmic FLOPs (the usual backward/forward ratio)."""
     import torch
 
     import synth_inputs as si
@@ -324,6 +324,8 @@ def bench_backward(rn, device, stream, steps, peaks):
     dv_ = torch.empty(b, L, h, dv, device=device)
     g, th = si.gamma_schedule(h), si.theta_schedule(dk)
     ws = torch.empty(rn.retnet_backward_workspace_size((b, L, h, dk, dv)), dtype=torch.uint8, device=device)
+    path = rn.retnet_backward_kernel((b, L, h, dk), dv, rn.BF16, FLAGS, g, ws.numel())
+    launches = rn.retnet_backward_launches((b, L, h, dk), dv, rn.BF16, FLAGS, g, ws.numel())
 
     def step(i):
         rn.retnet_retention_backward(q, k, v, do, dq, dk_, dv_, g, th, 0, FLAGS, workspace=ws, stream=stream)
@@ -334,8 +336,9 @@ def bench_backward(rn, device, stream, steps, peaks):
     flops = 2 * b * L * h * flops_per_token_head(dk, dv, B)
     tf = flops / secs / 1e12
     return {"workload": "backward_" + c["workload"], "us_per_step": secs * 1e6, "tokens_per_s": b * L / secs,
-            "tflops": tf, "frac_bf16_peak": tf / peaks["bf16"], "kernel": "fp32 CUDA cores (first path)",
-            "launches_per_step": 3, "gpu_launches": 3 * steps}
+            "tflops": tf, "frac_bf16_peak": tf / peaks["bf16"],
+            "kernel": "tcgen05 (six chunkwise runs)" if path == 1 else "fp32 CUDA cores",
+            "workspace_bytes": ws.numel(), "launches_per_step": launches, "gpu_launches": launches * steps}
 
 
 def oracle_sample(cfg, budget_s):

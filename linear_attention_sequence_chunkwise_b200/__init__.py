@@ -37,7 +37,7 @@ EXPORTS = ("retnet_retention_parallel", "retnet_retention_chunkwise", "retnet_re
            "retnet_retention_chunkwise_static", "retnet_chunkwise_segment_state", "retnet_state_advance",
            "retnet_chunkwise_workspace_size", "retnet_retention_step", "retnet_msr_epilogue",
            "retnet_msr_chunkwise", "retnet_msr_chunkwise_launches", "retnet_retention_backward",
-           "retnet_backward_workspace_size",
+           "retnet_backward_workspace_size", "retnet_backward_kernel", "retnet_backward_launches",
            "retnet_chunkwise_kernel", "retnet_chunkwise_launches", "retnet_debug_wait_timeouts",
            "retnet_status_string", "retnet_version")
 
@@ -95,6 +95,10 @@ def load(path: str = None):
     lib.retnet_retention_backward.restype = _i32
     lib.retnet_backward_workspace_size.argtypes = [Dims, ctypes.POINTER(ctypes.c_size_t)]
     lib.retnet_backward_workspace_size.restype = _i32
+    lib.retnet_backward_kernel.argtypes = [Dims, _i32, _u32, _fp, ctypes.c_size_t]
+    lib.retnet_backward_kernel.restype = _i32
+    lib.retnet_backward_launches.argtypes = [Dims, _i32, _u32, _fp, ctypes.c_size_t, _i32, _i32]
+    lib.retnet_backward_launches.restype = _i32
     lib.retnet_msr_chunkwise_launches.restype = _i32
     for name in ("retnet_retention_parallel", "retnet_retention_chunkwise", "retnet_retention_chunkwise_ws",
                  "retnet_retention_chunkwise_static", "retnet_retention_step", "retnet_msr_epilogue",
@@ -345,6 +349,22 @@ def retnet_backward_workspace_size(dims) -> int:
     out = ctypes.c_size_t(0)
     _check(load().retnet_backward_workspace_size(Dims(*[int(x) for x in dims]), ctypes.byref(out)))
     return out.value
+
+
+def retnet_backward_kernel(shape_qk, d_v, in_dtype, flags, gamma, workspace_bytes):
+    """1 if a gradient call of this shape runs on the tensor cores, 0 for the CUDA-core path."""
+    b, L, h, dk = shape_qk
+    return load().retnet_backward_kernel(Dims(b, L, h, dk, d_v), int(in_dtype), int(flags),
+                                         _fptr(_host_f32(gamma, h)), int(workspace_bytes))
+
+
+def retnet_backward_launches(shape_qk, d_v, in_dtype, flags, gamma, workspace_bytes, with_state=False,
+                             with_dstate=False):
+    """Kernel launches of a gradient call (negative: the negated status it would return)."""
+    b, L, h, dk = shape_qk
+    return load().retnet_backward_launches(Dims(b, L, h, dk, d_v), int(in_dtype), int(flags),
+                                           _fptr(_host_f32(gamma, h)), int(workspace_bytes), int(bool(with_state)),
+                                           int(bool(with_dstate)))
 
 
 def retnet_retention_backward(q, k, v, dout, dq, dk, dv, gamma, theta=None, pos0=0,

@@ -8,8 +8,9 @@
 //   dv_m  = sum_{n>=m} f_n g^(n-m) (q~_n . k~_m) dO_n
 //   dS0   = sum_n f_n g^(n+1) q~_n^T dO_n,       dq = R^T dq~, dk = R^T dk~.
 //
-// fp32 CUDA cores: a first, exact-in-structure path (O(L^2) per (batch, head), like the
-// parallel form), not a tuned one.  A prep kernel writes q~, k~ (fp32) to the workspace; the
+// fp32 CUDA cores: the path for fp32 inputs and other shapes (O(L^2) per (batch, head), like
+// the parallel form); bf16 inputs with d_k, d_v in {64, 128, 256} take the tensor-core path of
+// backward_tc.cu when the workspace holds its operands.  A prep kernel writes q~, k~ (fp32) to the workspace; the
 // dq kernel gives each warp one row n and sweeps the keys m <= n in tiles of 32 staged in
 // shared memory (lane = key for the dot products, lane = column for the accumulation); the
 // dk/dv kernel does the same for a key row m over the queries n >= m; the state kernel
@@ -272,9 +273,8 @@ size_t backward_workspace_bytes(const Dims& d) {
 
 bool backward_supported(const Dims& d) { return d.d_k <= kBwdMaxD && d.d_v <= kBwdMaxD && d.d_k % 2 == 0; }
 
-int backward_launches(const BackwardCall& c) { return c.dstate ? 4 : 3; }
-
 cudaError_t launch_backward(const BackwardCall& c, const HeadParams& hp, cudaStream_t s) {
+  if (backward_tc_applies(c, hp)) return launch_backward_tc(c, hp, s);
   if (c.in_dtype == RETNET_BF16) return launch_backward_t<__nv_bfloat16>(c, hp, s);
   return launch_backward_t<float>(c, hp, s);
 }

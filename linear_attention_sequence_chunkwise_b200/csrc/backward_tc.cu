@@ -1,0 +1,319 @@
+// backward_tc.cu -- the gradient of backward.cu on the tensor cores, as runs of the
+// tcgen05 chunkwise forward kernel.  Each gradient sum has the shape of a retention output:
+// a decayed, causal (or, read backwards, anti-causal) sum of value rows weighted by query .
+// key products ("阅读笔记：RetNet" §2.3, §2.4; notation of backward.cu):
+//   dq~_n / f_n = sum_{m<=n} g^(n-m) (dO_n . v_m) k~_m + g^(n+1) dO_n S0^T
+//        -> retention with query dO, key v, value k~, start state S0^T (forward order);
+//   dk~_m = sum_{n>=m} g^(n-m) (v_m . dO_n) (f_n q~_n)
+//        -> retention over the reversed sequence (t' = L-1-t): query v, key dO, value f q~;
+//   dv_m  = sum_{n>=m} g^(n-m) (q~_n . k~_m) (f_n dO_n)
+//        -> reversed: query k, key q, value f dO, with the kernel's own xPos rotation at the
+//           reversed positions and theta negated (the score of query t'_m and key t'_n turns
+//           by (t'_n - t'_m)(-theta) = (n - m) theta, which is q~_n . k~_m);
+//   dS0   = sum_n g^(n+1) (f_n q~_n)^T dO_n  (a plain reduction over the sequence).
+// A prep kernel writes the operands (rotations, row factors, reversal) in bf16: exact copies
+// for q, k, v, dO; k~, f q~ and f dO, which are not bf16 numbers, as two parts hi + lo (hi the
+// rounded value, lo the rounded remainder, together good to about 2^-17), and each run whose
+// value operand is one of them runs once per part (the runs are linear in the value).  A post
+// kernel adds the parts' outputs, scales dq by f, turns dq and dk back (R^T) and undoes the
+// reversal of dk and dv.
+#include <algorithm>
+
+#include "launch.h"
+
+namespace retnet {
+namespace {
+
+__device__ __forceinline__ __nv_bfloat16 to_bf16(float x) { return __float2bfloat16_rn(x); }
+
+// Row factor s / c_p of §三.3 in fp32 (relative error ~1e-7, far below the hi + lo split's
+// 2^-17): s = 1/sqrt(d_k), c_p^2 = (1 - gamma^(p+1)) / (1 - gamma) by expm1 / log1p.
+__device__ __forceinline__ float row_f(float gamma, int d_k, int64_t p, uint32_t flags) {
+  float f = (flags & RETNET_F_SCALE_SQRT_D) ? rsqrtf(static_cast<float>(d_k)) : 1.f;
+  if (flags & RETNET_F_NORM_D) {
+    const float om = 1.f - gamma;
+    f *= rsqrtf(-expm1f(static_cast<float>(p + 1) * log1pf(-om)) / om);
+  }
+  return f;
+}
+
+// Thread = (row (b, t, h), rotary pair j of d_k): k~ forward; q, k copied reversed; f q~ reversed.
+__device__ __forceinline__ void split_store(__nv_bfloat16* hi, __nv_bfloat16* lo, int64_t i, float x) {
+  const __nv_bfloat16 a = to_bf16(x);
+  hi[i] = a;
+  lo[i] = to_bf16(x - __bfloat162float(a));
+}
+
+__global__ void bwd_tc_prep_qk(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                               __nv_bfloat16* __restrict__ kt, __nv_bfloat16* __restrict__ ktl,
+                               __nv_bfloat16* __restrict__ qR, __nv_bfloat16* __restrict__ kR,
+                               __nv_bfloat16* __restrict__ fqR, __nv_bfloat16* __restrict__ fqRl, int64_t rows, int L,
+                               int heads, int d_k, int64_t pos0, uint32_t flags, HeadParams hp) {
+  const int np = d_k / 2;
+  const bool xpos = (flags & RETNET_F_XPOS) != 0;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < rows * np;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = i / np;
+    const int j = static_cast<int>(i % np);
+    const int h = static_cast<int>(row % heads);
+    const int64_t bt = row / heads;
+    const int t = static_cast<int>(bt % L);
+    const int64_t rrow = (bt - t + (L - 1 - t)) * heads + h;  // the same (b, h) at t' = L-1-t
+    float c = 1.f, s = 0.f;
+    if (xpos) xpos_sincos(pos0 + t, hp.theta[j], &s, &c);
+    const float f = row_f(hp.gamma[h], d_k, pos0 + t, flags);
+    const int64_t o = row * d_k + 2 * j, ro = rrow * d_k + 2 * j;
+    const __nv_bfloat16 q0 = q[o], q1 = q[o + 1], k0 = k[o], k1 = k[o + 1];
+    const float fq0 = __bfloat162float(q0), fq1 = __bfloat162float(q1);
+    const float fk0 = __bfloat162float(k0), fk1 = __bfloat162float(k1);
+    split_store(kt, ktl, o, fk0 * c - fk1 * s);
+    split_store(kt, ktl, o + 1, fk0 * s + fk1 * c);
+    qR[ro] = q0;
+    qR[ro + 1] = q1;
+    kR[ro] = k0;
+    kR[ro + 1] = k1;
+    split_store(fqR, fqRl, ro, f * (fq0 * c - fq1 * s));
+    split_store(fqR, fqRl, ro + 1, f * (fq0 * s + fq1 * c));
+  }
+}
+
+// Thread = (row, column of d_v): v and dO copied reversed; f dO reversed.
+__global__ void bwd_tc_prep_v(const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ dout,
+                              __nv_bfloat16* __restrict__ vR, __nv_bfloat16* __restrict__ doR,
+                              __nv_bfloat16* __restrict__ fdoR, __nv_bfloat16* __restrict__ fdoRl, int64_t rows, int L,
+                              int heads, int d_k, int d_v,
+                              int64_t pos0, uint32_t flags, HeadParams hp) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < rows * d_v;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = i / d_v;
+    const int j = static_cast<int>(i % d_v);
+    const int h = static_cast<int>(row % heads);
+    const int64_t bt = row / heads;
+    const int t = static_cast<int>(bt % L);
+    const int64_t ro = ((bt - t + (L - 1 - t)) * heads + h) * d_v + j;
+    const float f = row_f(hp.gamma[h], d_k, pos0 + t, flags);
+    const __nv_bfloat16 dd = dout[row * d_v + j];
+    vR[ro] = v[row * d_v + j];
+    doR[ro] = dd;
+    split_store(fdoR, fdoRl, ro, f * __bfloat162float(dd));
+  }
+}
+
+// S0^T per (batch, head): [d_k][d_v] -> [d_v][d_k].
+__global__ void bwd_tc_transpose(const float* __restrict__ s, float* __restrict__ st, int64_t n, int d_k, int d_v) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t m = i / (static_cast<int64_t>(d_k) * d_v);
+    const int r = static_cast<int>(i % (static_cast<int64_t>(d_k) * d_v));
+    const int a = r / d_v, bb = r % d_v;
+    st[(m * d_v + bb) * d_k + a] = s[i];
+  }
+}
+
+// Thread = (row, rotary pair j): dq <- R^T (f dq) in place; dk <- R^T dk~R at the reversed row.
+__global__ void bwd_tc_post_qk(float* __restrict__ dq, const float* __restrict__ dql, const float* __restrict__ dkR,
+                               const float* __restrict__ dkRl, float* __restrict__ dk, int64_t rows, int L, int heads,
+                               int d_k, int64_t pos0, uint32_t flags, HeadParams hp) {
+  const int np = d_k / 2;
+  const bool xpos = (flags & RETNET_F_XPOS) != 0;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < rows * np;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = i / np;
+    const int j = static_cast<int>(i % np);
+    const int h = static_cast<int>(row % heads);
+    const int64_t bt = row / heads;
+    const int t = static_cast<int>(bt % L);
+    const int64_t rrow = (bt - t + (L - 1 - t)) * heads + h;
+    float c = 1.f, s = 0.f;
+    if (xpos) xpos_sincos(pos0 + t, hp.theta[j], &s, &c);
+    const float f = row_f(hp.gamma[h], d_k, pos0 + t, flags);
+    const int64_t o = row * d_k + 2 * j, ro = rrow * d_k + 2 * j;
+    const float y0 = f * (dq[o] + dql[o]), y1 = f * (dq[o + 1] + dql[o + 1]);
+    dq[o] = fmaf(y0, c, y1 * s);
+    dq[o + 1] = fmaf(y1, c, -y0 * s);
+    const float z0 = dkR[ro] + dkRl[ro], z1 = dkR[ro + 1] + dkRl[ro + 1];
+    dk[o] = fmaf(z0, c, z1 * s);
+    dk[o + 1] = fmaf(z1, c, -z0 * s);
+  }
+}
+
+__global__ void bwd_tc_post_v(const float* __restrict__ dvR, const float* __restrict__ dvRl, float* __restrict__ dv,
+                              int64_t rows, int L, int heads, int d_v) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < rows * d_v;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = i / d_v;
+    const int j = static_cast<int>(i % d_v);
+    const int h = static_cast<int>(row % heads);
+    const int64_t bt = row / heads;
+    const int t = static_cast<int>(bt % L);
+    const int64_t r = ((bt - t + (L - 1 - t)) * heads + h) * d_v + j;
+    dv[i] = dvR[r] + dvRl[r];
+  }
+}
+
+// dS0[i][j] = sum_t' g^(L-t') fqR[t'][i] doR[t'][j]  (t' = L-1-n, so g^(n+1)): CTA = (b * h,
+// 32-row block of d_k), thread = (row i, columns j).
+__global__ void __launch_bounds__(256) bwd_tc_dstate(const __nv_bfloat16* __restrict__ fqR,
+                                                     const __nv_bfloat16* __restrict__ fqRl,
+                                                     const __nv_bfloat16* __restrict__ doR, float* __restrict__ dstate,
+                                                     int L, int heads, int d_k, int d_v, HeadParams hp) {
+  const int bh = blockIdx.x, b = bh / heads, h = bh % heads;
+  const float lg = hp.log2g[h];
+  for (int e = threadIdx.x; e < 32 * d_v; e += blockDim.x) {
+    const int i = blockIdx.y * 32 + e / d_v, j = e % d_v;
+    if (i >= d_k) continue;
+    float s = 0.f;
+    for (int tp = 0; tp < L; ++tp) {
+      const int64_t r = (static_cast<int64_t>(b) * L + tp) * heads + h;
+      s = fmaf(exp2f(static_cast<float>(L - tp) * lg) *
+                   (__bfloat162float(fqR[r * d_k + i]) + __bfloat162float(fqRl[r * d_k + i])),
+               __bfloat162float(doR[r * d_v + j]), s);
+    }
+    dstate[(static_cast<int64_t>(bh) * d_k + i) * d_v + j] = s;
+  }
+}
+
+constexpr int kBwdChunk = 64;
+
+size_t a256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct TcLayout {
+  size_t kt, ktl, qR, kR, fqR, fqRl, vR, doR, fdoR, fdoRl, dkR, dkRl, dqL, dvR, dvRl, s0t, fwd, total;
+};
+TcLayout tc_layout(const Dims& d) {
+  const size_t tok = static_cast<size_t>(d.batch * d.seqlen * d.heads);
+  const size_t bk = a256(tok * d.d_k * 2), bv = a256(tok * d.d_v * 2);
+  TcLayout l{};
+  size_t off = 0;
+  l.kt = off; off += bk;
+  l.ktl = off; off += bk;
+  l.qR = off; off += bk;
+  l.kR = off; off += bk;
+  l.fqR = off; off += bk;
+  l.fqRl = off; off += bk;
+  l.vR = off; off += bv;
+  l.doR = off; off += bv;
+  l.fdoR = off; off += bv;
+  l.fdoRl = off; off += bv;
+  l.dkR = off; off += a256(tok * d.d_k * 4);
+  l.dkRl = off; off += a256(tok * d.d_k * 4);
+  l.dqL = off; off += a256(tok * d.d_k * 4);
+  l.dvR = off; off += a256(tok * d.d_v * 4);
+  l.dvRl = off; off += a256(tok * d.d_v * 4);
+  l.s0t = off; off += a256(static_cast<size_t>(d.batch * d.heads * d.d_k * d.d_v) * 4);
+  l.fwd = off;
+  // the forward runs' own workspace (two-pass segment states), shared by the three in turn
+  const size_t states = 6 * 4 * static_cast<size_t>(d.batch * d.heads * d.d_k * d.d_v);
+  off += a256(states);
+  l.total = off;
+  return l;
+}
+
+// The six forward runs (three sums, value hi and lo parts), described without launching.
+constexpr int kRuns = 6;
+void tc_calls(const BackwardCall& c, char* ws, const TcLayout& l, RetentionCall out[kRuns]) {
+  const Dims& d = c.dims;
+  const Dims d1{d.batch, d.seqlen, d.heads, d.d_v, d.d_k};  // key dim d_v, value dim d_k
+  const Dims d3{d.batch, d.seqlen, d.heads, d.d_k, d.d_v};
+  auto base = [&](const void* q, const void* k, const void* v, void* o, const Dims& dd, uint32_t flags,
+                  const float* s_in) {
+    RetentionCall r{q, k, v, o, dd, RETNET_BF16, RETNET_F32, 0, flags, kBwdChunk, true, s_in, nullptr, nullptr,
+                    nullptr};
+    r.ws = ws + l.fwd;
+    r.ws_bytes = l.total - l.fwd;
+    return r;
+  };
+  out[0] = base(c.dout, c.v, ws + l.kt, c.dq, d1, 0u, c.state_in ? reinterpret_cast<const float*>(ws + l.s0t) : nullptr);
+  out[1] = base(c.dout, c.v, ws + l.ktl, ws + l.dqL, d1, 0u, nullptr);
+  out[2] = base(ws + l.vR, ws + l.doR, ws + l.fqR, ws + l.dkR, d1, 0u, nullptr);
+  out[3] = base(ws + l.vR, ws + l.doR, ws + l.fqRl, ws + l.dkRl, d1, 0u, nullptr);
+  out[4] = base(ws + l.kR, ws + l.qR, ws + l.fdoR, ws + l.dvR, d3, c.flags & RETNET_F_XPOS, nullptr);
+  out[5] = base(ws + l.kR, ws + l.qR, ws + l.fdoRl, ws + l.dvRl, d3, c.flags & RETNET_F_XPOS, nullptr);
+}
+
+// Head parameters of each run: the kernels rotate by whatever theta they are given (a call
+// without xPos carries zeros), so the dq and dk runs get zeros and the dv runs -theta.
+HeadParams run_params(const HeadParams& hp, int run) {
+  HeadParams r = hp;
+  for (int j = 0; j < kMaxPairs; ++j) r.theta[j] = run >= 4 ? -hp.theta[j] : 0.f;
+  return r;
+}
+
+}  // namespace
+
+size_t backward_tc_workspace_bytes(const Dims& d) { return tc_layout(d).total; }
+
+bool backward_tc_applies(const BackwardCall& c, const HeadParams& hp) {
+  const Dims& d = c.dims;
+  if (c.in_dtype != RETNET_BF16 || !tc_driver_ready()) return false;
+  auto dim_ok = [](int64_t x) { return x == 64 || x == 128 || x == 256; };
+  if (!dim_ok(d.d_k) || !dim_ok(d.d_v) || d.seqlen < 1) return false;
+  if (!c.ws || c.ws_bytes < backward_tc_workspace_bytes(d)) return false;
+  RetentionCall calls[kRuns];
+  tc_calls(c, static_cast<char*>(c.ws), tc_layout(d), calls);
+  for (int i = 0; i < kRuns; ++i)
+    if (!tc_chunkwise_supported(calls[i]) || !tc_chunkwise_heads_ok(calls[i], run_params(hp, i))) return false;
+  return true;
+}
+
+cudaError_t launch_backward_tc(const BackwardCall& c, const HeadParams& hp, cudaStream_t s) {
+  const Dims& d = c.dims;
+  const TcLayout l = tc_layout(d);
+  char* ws = static_cast<char*>(c.ws);
+  const int64_t rows = d.batch * d.seqlen * d.heads;
+  const int L = static_cast<int>(d.seqlen), H = static_cast<int>(d.heads), dk = static_cast<int>(d.d_k),
+            dv = static_cast<int>(d.d_v);
+  auto blocks = [](int64_t items) { return static_cast<int>(std::min<int64_t>((items + 255) / 256, 148 * 16)); };
+  auto* kt = reinterpret_cast<__nv_bfloat16*>(ws + l.kt);
+  auto* ktl = reinterpret_cast<__nv_bfloat16*>(ws + l.ktl);
+  auto* fqRl = reinterpret_cast<__nv_bfloat16*>(ws + l.fqRl);
+  auto* fdoRl = reinterpret_cast<__nv_bfloat16*>(ws + l.fdoRl);
+  auto* qR = reinterpret_cast<__nv_bfloat16*>(ws + l.qR);
+  auto* kR = reinterpret_cast<__nv_bfloat16*>(ws + l.kR);
+  auto* fqR = reinterpret_cast<__nv_bfloat16*>(ws + l.fqR);
+  auto* vR = reinterpret_cast<__nv_bfloat16*>(ws + l.vR);
+  auto* doR = reinterpret_cast<__nv_bfloat16*>(ws + l.doR);
+  auto* fdoR = reinterpret_cast<__nv_bfloat16*>(ws + l.fdoR);
+  bwd_tc_prep_qk<<<blocks(rows * (dk / 2)), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(c.q),
+                                                          static_cast<const __nv_bfloat16*>(c.k), kt, ktl, qR, kR, fqR,
+                                                          fqRl, rows, L, H, dk, c.pos0, c.flags, hp);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  bwd_tc_prep_v<<<blocks(rows * dv), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(c.v),
+                                                   static_cast<const __nv_bfloat16*>(c.dout), vR, doR, fdoR, fdoRl, rows,
+                                                   L, H, dk, dv, c.pos0, c.flags, hp);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (c.state_in) {
+    const int64_t n = d.batch * d.heads * d.d_k * d.d_v;
+    bwd_tc_transpose<<<blocks(n), 256, 0, s>>>(c.state_in, reinterpret_cast<float*>(ws + l.s0t), n, dk, dv);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  RetentionCall calls[kRuns];
+  tc_calls(c, ws, l, calls);
+  for (int i = 0; i < kRuns; ++i)
+    if ((e = launch_tc_chunkwise(calls[i], run_params(hp, i), s)) != cudaSuccess) return e;
+  bwd_tc_post_qk<<<blocks(rows * (dk / 2)), 256, 0, s>>>(c.dq, reinterpret_cast<const float*>(ws + l.dqL),
+                                                          reinterpret_cast<const float*>(ws + l.dkR),
+                                                          reinterpret_cast<const float*>(ws + l.dkRl), c.dk, rows, L, H,
+                                                          dk, c.pos0, c.flags, hp);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  bwd_tc_post_v<<<blocks(rows * dv), 256, 0, s>>>(reinterpret_cast<const float*>(ws + l.dvR),
+                                                   reinterpret_cast<const float*>(ws + l.dvRl), c.dv, rows, L, H, dv);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (c.dstate) {
+    const dim3 gs(static_cast<unsigned>(d.batch * d.heads), static_cast<unsigned>((dk + 31) / 32));
+    bwd_tc_dstate<<<gs, 256, 0, s>>>(fqR, fqRl, doR, c.dstate, L, H, dk, dv, hp);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+int backward_tc_launches(const BackwardCall& c) {
+  RetentionCall calls[kRuns];
+  tc_calls(c, static_cast<char*>(c.ws), tc_layout(c.dims), calls);
+  int n = 2 + 2 + (c.state_in ? 1 : 0) + (c.dstate ? 1 : 0);
+  for (int i = 0; i < kRuns; ++i) n += tc_chunkwise_launches(calls[i]);
+  return n;
+}
+
+}  // namespace retnet

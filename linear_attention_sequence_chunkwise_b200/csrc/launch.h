@@ -105,11 +105,19 @@ struct BackwardCall {
   uint32_t flags;
   const float* state_in;  // S0 before the first token (or nullptr)
   float* dstate;          // gradient of S0 (or nullptr)
-  void* ws;               // backward_workspace_bytes(dims): rotated q and k, fp32
+  void* ws;               // workspace (see backward_workspace_bytes)
+  size_t ws_bytes;
 };
+// Bytes the CUDA-core path needs (rotated q and k in fp32); the tensor-core path needs
+// backward_tc_workspace_bytes (more; it is taken when the workspace has it).
 size_t backward_workspace_bytes(const Dims& d);
+size_t backward_tc_workspace_bytes(const Dims& d);
 bool backward_supported(const Dims& d);
-int backward_launches(const BackwardCall& c);
+// The tensor-core path (three runs of the chunkwise kernel) handles this call: bf16 inputs,
+// d_k and d_v in {64, 128, 256}, room in the workspace, every run supported by the kernel.
+bool backward_tc_applies(const BackwardCall& c, const HeadParams& hp);
+int backward_tc_launches(const BackwardCall& c);
+cudaError_t launch_backward_tc(const BackwardCall& c, const HeadParams& hp, cudaStream_t s);
 cudaError_t launch_backward(const BackwardCall& c, const HeadParams& hp, cudaStream_t s);
 
 cudaError_t launch_msr_epilogue(const void* y, const void* g, void* out, int64_t tokens, int64_t heads,

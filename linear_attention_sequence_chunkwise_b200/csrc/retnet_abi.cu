@@ -5,6 +5,7 @@
 // caller's stream.  Nothing is allocated; no state survives the call.
 #include <math.h>
 
+#include <algorithm>
 #include <atomic>
 
 #include "launch.h"
@@ -398,8 +399,44 @@ retnet_status_t retnet_retention_step(const void* q, const void* k, const void* 
 retnet_status_t retnet_backward_workspace_size(retnet_dims_t dims, size_t* bytes) {
   if (!bytes) return RETNET_ERR_NULL_PTR;
   if (dims.batch < 0 || dims.seqlen < 0 || dims.heads < 0 || dims.d_k < 0 || dims.d_v < 0) return RETNET_ERR_BAD_SHAPE;
-  *bytes = backward_workspace_bytes(Dims{dims.batch, dims.seqlen, dims.heads, dims.d_k, dims.d_v});
+  const Dims d{dims.batch, dims.seqlen, dims.heads, dims.d_k, dims.d_v};
+  *bytes = std::max(backward_workspace_bytes(d), backward_tc_workspace_bytes(d));
   return RETNET_OK;
+}
+
+int retnet_backward_kernel(retnet_dims_t dims, retnet_dtype_t in_dtype, uint32_t flags, const float* gamma,
+                           size_t workspace_bytes) {
+  retnet_status_t st = check_common(dims, in_dtype, RETNET_F32, 0, flags, true);
+  if (st != RETNET_OK) return -static_cast<int>(st);
+  if (flags & RETNET_F_NORM_R) return -static_cast<int>(RETNET_ERR_UNSUPPORTED);
+  HeadParams hp;
+  st = fill_params(&hp, gamma, nullptr, dims.heads, dims.d_k, flags & ~static_cast<uint32_t>(RETNET_F_XPOS));
+  if (st != RETNET_OK) return -static_cast<int>(st);
+  alignas(16) static const uint32_t kAligned[4] = {0, 0, 0, 0};
+  float* fake = const_cast<float*>(reinterpret_cast<const float*>(kAligned));
+  BackwardCall c{kAligned, kAligned, kAligned, kAligned, fake, fake, fake,
+                 Dims{dims.batch, dims.seqlen, dims.heads, dims.d_k, dims.d_v}, in_dtype, 0, flags, nullptr, nullptr,
+                 reinterpret_cast<void*>(static_cast<uintptr_t>(256)), workspace_bytes};
+  return backward_tc_applies(c, hp) ? 1 : 0;
+}
+
+int retnet_backward_launches(retnet_dims_t dims, retnet_dtype_t in_dtype, uint32_t flags, const float* gamma,
+                             size_t workspace_bytes, int with_state, int with_dstate) {
+  const int path = retnet_backward_kernel(dims, in_dtype, flags, gamma, workspace_bytes);
+  if (path < 0) return path;
+  if (dims.seqlen == 0) return with_dstate ? 1 : 0;  // a memset (no kernel of ours)
+  if (path == 0) return with_dstate ? 4 : 3;
+  const retnet_status_t st = check_device();
+  if (st != RETNET_OK) return -static_cast<int>(st);
+  HeadParams hp;
+  fill_params(&hp, gamma, nullptr, dims.heads, dims.d_k, flags & ~static_cast<uint32_t>(RETNET_F_XPOS));
+  alignas(16) static const uint32_t kAligned[4] = {0, 0, 0, 0};
+  float* fake = const_cast<float*>(reinterpret_cast<const float*>(kAligned));
+  BackwardCall c{kAligned, kAligned, kAligned, kAligned, fake, fake, fake,
+                 Dims{dims.batch, dims.seqlen, dims.heads, dims.d_k, dims.d_v}, in_dtype, 0, flags,
+                 with_state ? fake : nullptr, with_dstate ? fake : nullptr,
+                 reinterpret_cast<void*>(static_cast<uintptr_t>(256)), workspace_bytes};
+  return backward_tc_launches(c);
 }
 
 retnet_status_t retnet_retention_backward(const void* q, const void* k, const void* v, const void* dout, float* dq,
@@ -425,7 +462,7 @@ retnet_status_t retnet_retention_backward(const void* q, const void* k, const vo
   HeadParams hp;
   if ((st = fill_params(&hp, gamma, theta, dims.heads, dims.d_k, flags)) != RETNET_OK) return st;
   if ((st = check_device()) != RETNET_OK) return st;
-  BackwardCall c{q, k, v, dout, dq, dk, dv, d, in_dtype, pos0, flags, state_in, dstate, workspace};
+  BackwardCall c{q, k, v, dout, dq, dk, dv, d, in_dtype, pos0, flags, state_in, dstate, workspace, workspace_bytes};
   return from_cuda(launch_backward(c, hp, static_cast<cudaStream_t>(stream)));
 }
 
