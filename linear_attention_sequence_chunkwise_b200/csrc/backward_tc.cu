@@ -37,65 +37,76 @@ __device__ __forceinline__ float row_f(float gamma, int d_k, int64_t p, uint32_t
   return f;
 }
 
-// Thread = (row (b, t, h), rotary pair j of d_k): k~ forward; q, k copied reversed; f q~ reversed.
 __device__ __forceinline__ void split_store(__nv_bfloat16* hi, __nv_bfloat16* lo, int64_t i, float x) {
   const __nv_bfloat16 a = to_bf16(x);
   hi[i] = a;
   lo[i] = to_bf16(x - __bfloat162float(a));
 }
 
-__global__ void bwd_tc_prep_qk(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-                               __nv_bfloat16* __restrict__ kt, __nv_bfloat16* __restrict__ ktl,
-                               __nv_bfloat16* __restrict__ qR, __nv_bfloat16* __restrict__ kR,
-                               __nv_bfloat16* __restrict__ fqR, __nv_bfloat16* __restrict__ fqRl, int64_t rows, int L,
-                               int heads, int d_k, int64_t pos0, uint32_t flags, HeadParams hp) {
-  const int np = d_k / 2;
+// The elementwise kernels run one CTA per token (b, t): the rotation of pair j is the same for
+// every head, and each head's row factor is computed once, into shared memory.
+__device__ __forceinline__ void row_factors(float* sf, int heads, int d_k, int64_t p, uint32_t flags,
+                                            const HeadParams& hp) {
+  for (int h = threadIdx.x; h < heads; h += blockDim.x) sf[h] = row_f(hp.gamma[h], d_k, p, flags);
+  __syncthreads();
+}
+
+// Token (b, t): k~ forward; q, k copied reversed; f q~ reversed (split).
+__global__ void __launch_bounds__(128) bwd_tc_prep_qk(const __nv_bfloat16* __restrict__ q,
+                                                      const __nv_bfloat16* __restrict__ k,
+                                                      __nv_bfloat16* __restrict__ kt, __nv_bfloat16* __restrict__ ktl,
+                                                      __nv_bfloat16* __restrict__ qR, __nv_bfloat16* __restrict__ kR,
+                                                      __nv_bfloat16* __restrict__ fqR,
+                                                      __nv_bfloat16* __restrict__ fqRl, int L, int heads, int d_k,
+                                                      int64_t pos0, uint32_t flags, HeadParams hp) {
+  __shared__ float sf[RETNET_MAX_HEADS];
+  const int64_t bt = blockIdx.x;
+  const int t = static_cast<int>(bt % L);
+  const int64_t rbt = bt - t + (L - 1 - t);  // the same b at t' = L-1-t
+  row_factors(sf, heads, d_k, pos0 + t, flags, hp);
   const bool xpos = (flags & RETNET_F_XPOS) != 0;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < rows * np;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t row = i / np;
-    const int j = static_cast<int>(i % np);
-    const int h = static_cast<int>(row % heads);
-    const int64_t bt = row / heads;
-    const int t = static_cast<int>(bt % L);
-    const int64_t rrow = (bt - t + (L - 1 - t)) * heads + h;  // the same (b, h) at t' = L-1-t
+  for (int j = threadIdx.x; j < d_k / 2; j += blockDim.x) {
     float c = 1.f, s = 0.f;
     if (xpos) xpos_sincos(pos0 + t, hp.theta[j], &s, &c);
-    const float f = row_f(hp.gamma[h], d_k, pos0 + t, flags);
-    const int64_t o = row * d_k + 2 * j, ro = rrow * d_k + 2 * j;
-    const __nv_bfloat16 q0 = q[o], q1 = q[o + 1], k0 = k[o], k1 = k[o + 1];
-    const float fq0 = __bfloat162float(q0), fq1 = __bfloat162float(q1);
-    const float fk0 = __bfloat162float(k0), fk1 = __bfloat162float(k1);
-    split_store(kt, ktl, o, fk0 * c - fk1 * s);
-    split_store(kt, ktl, o + 1, fk0 * s + fk1 * c);
-    qR[ro] = q0;
-    qR[ro + 1] = q1;
-    kR[ro] = k0;
-    kR[ro + 1] = k1;
-    split_store(fqR, fqRl, ro, f * (fq0 * c - fq1 * s));
-    split_store(fqR, fqRl, ro + 1, f * (fq0 * s + fq1 * c));
+    for (int h = 0; h < heads; ++h) {
+      const int64_t o = (bt * heads + h) * d_k + 2 * j, ro = (rbt * heads + h) * d_k + 2 * j;
+      const __nv_bfloat162 q2 = *reinterpret_cast<const __nv_bfloat162*>(q + o);
+      const __nv_bfloat162 k2 = *reinterpret_cast<const __nv_bfloat162*>(k + o);
+      const float2 qf = __bfloat1622float2(q2), kf = __bfloat1622float2(k2);
+      *reinterpret_cast<__nv_bfloat162*>(qR + ro) = q2;
+      *reinterpret_cast<__nv_bfloat162*>(kR + ro) = k2;
+      split_store(kt, ktl, o, kf.x * c - kf.y * s);
+      split_store(kt, ktl, o + 1, kf.x * s + kf.y * c);
+      const float f = sf[h];
+      split_store(fqR, fqRl, ro, f * (qf.x * c - qf.y * s));
+      split_store(fqR, fqRl, ro + 1, f * (qf.x * s + qf.y * c));
+    }
   }
 }
 
-// Thread = (row, column of d_v): v and dO copied reversed; f dO reversed.
-__global__ void bwd_tc_prep_v(const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ dout,
-                              __nv_bfloat16* __restrict__ vR, __nv_bfloat16* __restrict__ doR,
-                              __nv_bfloat16* __restrict__ fdoR, __nv_bfloat16* __restrict__ fdoRl, int64_t rows, int L,
-                              int heads, int d_k, int d_v,
-                              int64_t pos0, uint32_t flags, HeadParams hp) {
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < rows * d_v;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t row = i / d_v;
-    const int j = static_cast<int>(i % d_v);
-    const int h = static_cast<int>(row % heads);
-    const int64_t bt = row / heads;
-    const int t = static_cast<int>(bt % L);
-    const int64_t ro = ((bt - t + (L - 1 - t)) * heads + h) * d_v + j;
-    const float f = row_f(hp.gamma[h], d_k, pos0 + t, flags);
-    const __nv_bfloat16 dd = dout[row * d_v + j];
-    vR[ro] = v[row * d_v + j];
-    doR[ro] = dd;
-    split_store(fdoR, fdoRl, ro, f * __bfloat162float(dd));
+// Token (b, t): v and dO copied reversed; f dO reversed (split).  Thread = column pair.
+__global__ void __launch_bounds__(128) bwd_tc_prep_v(const __nv_bfloat16* __restrict__ v,
+                                                     const __nv_bfloat16* __restrict__ dout,
+                                                     __nv_bfloat16* __restrict__ vR, __nv_bfloat16* __restrict__ doR,
+                                                     __nv_bfloat16* __restrict__ fdoR,
+                                                     __nv_bfloat16* __restrict__ fdoRl, int L, int heads, int d_k,
+                                                     int d_v, int64_t pos0, uint32_t flags, HeadParams hp) {
+  __shared__ float sf[RETNET_MAX_HEADS];
+  const int64_t bt = blockIdx.x;
+  const int t = static_cast<int>(bt % L);
+  const int64_t rbt = bt - t + (L - 1 - t);
+  row_factors(sf, heads, d_k, pos0 + t, flags, hp);
+  const int half = d_v / 2;
+  for (int e = threadIdx.x; e < heads * half; e += blockDim.x) {
+    const int h = e / half, j = 2 * (e % half);
+    const int64_t o = (bt * heads + h) * d_v + j, ro = (rbt * heads + h) * d_v + j;
+    const __nv_bfloat162 v2 = *reinterpret_cast<const __nv_bfloat162*>(v + o);
+    const __nv_bfloat162 d2 = *reinterpret_cast<const __nv_bfloat162*>(dout + o);
+    *reinterpret_cast<__nv_bfloat162*>(vR + ro) = v2;
+    *reinterpret_cast<__nv_bfloat162*>(doR + ro) = d2;
+    const float2 df = __bfloat1622float2(d2);
+    split_store(fdoR, fdoRl, ro, sf[h] * df.x);
+    split_store(fdoR, fdoRl, ro + 1, sf[h] * df.y);
   }
 }
 
@@ -110,44 +121,44 @@ __global__ void bwd_tc_transpose(const float* __restrict__ s, float* __restrict_
   }
 }
 
-// Thread = (row, rotary pair j): dq <- R^T (f dq) in place; dk <- R^T dk~R at the reversed row.
-__global__ void bwd_tc_post_qk(float* __restrict__ dq, const float* __restrict__ dql, const float* __restrict__ dkR,
-                               const float* __restrict__ dkRl, float* __restrict__ dk, int64_t rows, int L, int heads,
-                               int d_k, int64_t pos0, uint32_t flags, HeadParams hp) {
-  const int np = d_k / 2;
+// Token (b, t): dq <- R^T (f (dq + dq_lo)) in place; dk <- R^T (dk~R + dk~R_lo) at the reversed row.
+__global__ void __launch_bounds__(128) bwd_tc_post_qk(float* __restrict__ dq, const float* __restrict__ dql,
+                                                      const float* __restrict__ dkR, const float* __restrict__ dkRl,
+                                                      float* __restrict__ dk, int L, int heads, int d_k, int64_t pos0,
+                                                      uint32_t flags, HeadParams hp) {
+  __shared__ float sf[RETNET_MAX_HEADS];
+  const int64_t bt = blockIdx.x;
+  const int t = static_cast<int>(bt % L);
+  const int64_t rbt = bt - t + (L - 1 - t);
+  row_factors(sf, heads, d_k, pos0 + t, flags, hp);
   const bool xpos = (flags & RETNET_F_XPOS) != 0;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < rows * np;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t row = i / np;
-    const int j = static_cast<int>(i % np);
-    const int h = static_cast<int>(row % heads);
-    const int64_t bt = row / heads;
-    const int t = static_cast<int>(bt % L);
-    const int64_t rrow = (bt - t + (L - 1 - t)) * heads + h;
+  for (int j = threadIdx.x; j < d_k / 2; j += blockDim.x) {
     float c = 1.f, s = 0.f;
     if (xpos) xpos_sincos(pos0 + t, hp.theta[j], &s, &c);
-    const float f = row_f(hp.gamma[h], d_k, pos0 + t, flags);
-    const int64_t o = row * d_k + 2 * j, ro = rrow * d_k + 2 * j;
-    const float y0 = f * (dq[o] + dql[o]), y1 = f * (dq[o + 1] + dql[o + 1]);
-    dq[o] = fmaf(y0, c, y1 * s);
-    dq[o + 1] = fmaf(y1, c, -y0 * s);
-    const float z0 = dkR[ro] + dkRl[ro], z1 = dkR[ro + 1] + dkRl[ro + 1];
-    dk[o] = fmaf(z0, c, z1 * s);
-    dk[o + 1] = fmaf(z1, c, -z0 * s);
+    for (int h = 0; h < heads; ++h) {
+      const int64_t o = (bt * heads + h) * d_k + 2 * j, ro = (rbt * heads + h) * d_k + 2 * j;
+      const float2 a = *reinterpret_cast<const float2*>(dq + o), al = *reinterpret_cast<const float2*>(dql + o);
+      const float y0 = sf[h] * (a.x + al.x), y1 = sf[h] * (a.y + al.y);
+      *reinterpret_cast<float2*>(dq + o) = make_float2(fmaf(y0, c, y1 * s), fmaf(y1, c, -y0 * s));
+      const float2 z = *reinterpret_cast<const float2*>(dkR + ro), zl = *reinterpret_cast<const float2*>(dkRl + ro);
+      const float z0 = z.x + zl.x, z1 = z.y + zl.y;
+      *reinterpret_cast<float2*>(dk + o) = make_float2(fmaf(z0, c, z1 * s), fmaf(z1, c, -z0 * s));
+    }
   }
 }
 
-__global__ void bwd_tc_post_v(const float* __restrict__ dvR, const float* __restrict__ dvRl, float* __restrict__ dv,
-                              int64_t rows, int L, int heads, int d_v) {
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < rows * d_v;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t row = i / d_v;
-    const int j = static_cast<int>(i % d_v);
-    const int h = static_cast<int>(row % heads);
-    const int64_t bt = row / heads;
-    const int t = static_cast<int>(bt % L);
-    const int64_t r = ((bt - t + (L - 1 - t)) * heads + h) * d_v + j;
-    dv[i] = dvR[r] + dvRl[r];
+// Token (b, t): dv <- dvR + dvR_lo at the reversed row (float2 a thread).
+__global__ void __launch_bounds__(128) bwd_tc_post_v(const float* __restrict__ dvR, const float* __restrict__ dvRl,
+                                                     float* __restrict__ dv, int L, int heads, int d_v) {
+  const int64_t bt = blockIdx.x;
+  const int t = static_cast<int>(bt % L);
+  const int64_t rbt = bt - t + (L - 1 - t);
+  const int half = d_v / 2;
+  for (int e = threadIdx.x; e < heads * half; e += blockDim.x) {
+    const int h = e / half, j = 2 * (e % half);
+    const int64_t o = (bt * heads + h) * d_v + j, ro = (rbt * heads + h) * d_v + j;
+    const float2 a = *reinterpret_cast<const float2*>(dvR + ro), b = *reinterpret_cast<const float2*>(dvRl + ro);
+    *reinterpret_cast<float2*>(dv + o) = make_float2(a.x + b.x, a.y + b.y);
   }
 }
 
@@ -249,6 +260,8 @@ bool backward_tc_applies(const BackwardCall& c, const HeadParams& hp) {
   auto dim_ok = [](int64_t x) { return x == 64 || x == 128 || x == 256; };
   if (!dim_ok(d.d_k) || !dim_ok(d.d_v) || d.seqlen < 1) return false;
   if (!c.ws || c.ws_bytes < backward_tc_workspace_bytes(d)) return false;
+  auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  if (!al16(c.q) || !al16(c.k) || !al16(c.dk) || !al16(c.dv) || !al16(c.ws)) return false;  // vector accesses
   RetentionCall calls[kRuns];
   tc_calls(c, static_cast<char*>(c.ws), tc_layout(d), calls);
   for (int i = 0; i < kRuns; ++i)
@@ -260,7 +273,6 @@ cudaError_t launch_backward_tc(const BackwardCall& c, const HeadParams& hp, cuda
   const Dims& d = c.dims;
   const TcLayout l = tc_layout(d);
   char* ws = static_cast<char*>(c.ws);
-  const int64_t rows = d.batch * d.seqlen * d.heads;
   const int L = static_cast<int>(d.seqlen), H = static_cast<int>(d.heads), dk = static_cast<int>(d.d_k),
             dv = static_cast<int>(d.d_v);
   auto blocks = [](int64_t items) { return static_cast<int>(std::min<int64_t>((items + 255) / 256, 148 * 16)); };
@@ -274,14 +286,14 @@ cudaError_t launch_backward_tc(const BackwardCall& c, const HeadParams& hp, cuda
   auto* vR = reinterpret_cast<__nv_bfloat16*>(ws + l.vR);
   auto* doR = reinterpret_cast<__nv_bfloat16*>(ws + l.doR);
   auto* fdoR = reinterpret_cast<__nv_bfloat16*>(ws + l.fdoR);
-  bwd_tc_prep_qk<<<blocks(rows * (dk / 2)), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(c.q),
-                                                          static_cast<const __nv_bfloat16*>(c.k), kt, ktl, qR, kR, fqR,
-                                                          fqRl, rows, L, H, dk, c.pos0, c.flags, hp);
+  const unsigned tokens = static_cast<unsigned>(d.batch * d.seqlen);
+  bwd_tc_prep_qk<<<tokens, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(c.q), static_cast<const __nv_bfloat16*>(c.k),
+                                         kt, ktl, qR, kR, fqR, fqRl, L, H, dk, c.pos0, c.flags, hp);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  bwd_tc_prep_v<<<blocks(rows * dv), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(c.v),
-                                                   static_cast<const __nv_bfloat16*>(c.dout), vR, doR, fdoR, fdoRl, rows,
-                                                   L, H, dk, dv, c.pos0, c.flags, hp);
+  bwd_tc_prep_v<<<tokens, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(c.v),
+                                        static_cast<const __nv_bfloat16*>(c.dout), vR, doR, fdoR, fdoRl, L, H, dk, dv,
+                                        c.pos0, c.flags, hp);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (c.state_in) {
     const int64_t n = d.batch * d.heads * d.d_k * d.d_v;
@@ -292,13 +304,12 @@ cudaError_t launch_backward_tc(const BackwardCall& c, const HeadParams& hp, cuda
   tc_calls(c, ws, l, calls);
   for (int i = 0; i < kRuns; ++i)
     if ((e = launch_tc_chunkwise(calls[i], run_params(hp, i), s)) != cudaSuccess) return e;
-  bwd_tc_post_qk<<<blocks(rows * (dk / 2)), 256, 0, s>>>(c.dq, reinterpret_cast<const float*>(ws + l.dqL),
-                                                          reinterpret_cast<const float*>(ws + l.dkR),
-                                                          reinterpret_cast<const float*>(ws + l.dkRl), c.dk, rows, L, H,
-                                                          dk, c.pos0, c.flags, hp);
+  bwd_tc_post_qk<<<tokens, 128, 0, s>>>(c.dq, reinterpret_cast<const float*>(ws + l.dqL),
+                                         reinterpret_cast<const float*>(ws + l.dkR),
+                                         reinterpret_cast<const float*>(ws + l.dkRl), c.dk, L, H, dk, c.pos0, c.flags, hp);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  bwd_tc_post_v<<<blocks(rows * dv), 256, 0, s>>>(reinterpret_cast<const float*>(ws + l.dvR),
-                                                   reinterpret_cast<const float*>(ws + l.dvRl), c.dv, rows, L, H, dv);
+  bwd_tc_post_v<<<tokens, 128, 0, s>>>(reinterpret_cast<const float*>(ws + l.dvR),
+                                        reinterpret_cast<const float*>(ws + l.dvRl), c.dv, L, H, dv);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (c.dstate) {
     const dim3 gs(static_cast<unsigned>(d.batch * d.heads), static_cast<unsigned>((dk + 31) / 32));
