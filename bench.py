@@ -310,7 +310,7 @@ def bench_msr(rn, device, stream, steps, peaks):
 
 def bench_backward(rn, device, stream, steps, peaks):
     """Gradient of the forward (dq, dk, dv) on the headline workload, bf16 inputs, fp32 out, on
-    the path the library takes (tensor cores: six runs of the chunkwise kernel), against the
+    the path the library takes (tensor cores: three runs of the chunkwise kernel), against the
     bf16 tensor peak with 2x the forward's algorithmic FLOPs (the usual backward/forward ratio)."""
     import torch
 
@@ -337,7 +337,7 @@ def bench_backward(rn, device, stream, steps, peaks):
     tf = flops / secs / 1e12
     return {"workload": "backward_" + c["workload"], "us_per_step": secs * 1e6, "tokens_per_s": b * L / secs,
             "tflops": tf, "frac_bf16_peak": tf / peaks["bf16"],
-            "kernel": "tcgen05 (six chunkwise runs)" if path == 1 else "fp32 CUDA cores",
+            "kernel": "tcgen05 (three chunkwise runs, hi|lo values)" if path == 1 else "fp32 CUDA cores",
             "workspace_bytes": ws.numel(), "launches_per_step": launches, "gpu_launches": launches * steps}
 
 

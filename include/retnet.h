@@ -303,10 +303,10 @@ RETNET_API retnet_status_t retnet_msr_chunkwise(const void* q, const void* k, co
  * Paths: bf16 inputs with d_k and d_v in {64, 128, 256} and a workspace of
  * retnet_backward_workspace_size bytes run on the tensor cores: each gradient sum has the shape
  * of a retention output (dq: query dO, key v, value k~; dk: read backwards, query v, key dO,
- * value f q~; dv: backwards, query k, key q, value f dO), so runs of the chunkwise kernel compute
- * them: k~, f q~ and f dO, which are not bf16 numbers, go in as two bf16 parts (hi + lo), one
- * run each (six runs; max|err|/rms <= 1e-2).  Every other call runs on fp32 CUDA cores,
- * O(seqlen^2) per (batch, head).
+ * value f q~; dv: backwards, query k, key q, value f dO), so three runs of the chunkwise kernel
+ * compute them: k~, f q~ and f dO, which are not bf16 numbers, go in as two bf16 parts (hi +
+ * lo) side by side in a value of twice the width (max|err|/rms <= 1e-2).  Every other call runs
+ * on fp32 CUDA cores, O(seqlen^2) per (batch, head).
  * d_k, d_v <= 256 and seqlen <= 524280, else RETNET_ERR_UNSUPPORTED; RETNET_F_NORM_R (R~, a
  * division by a function of q and k) is RETNET_ERR_UNSUPPORTED.  Outputs do not alias inputs.
  */
@@ -319,14 +319,14 @@ RETNET_API retnet_status_t retnet_retention_backward(const void* q, const void* 
 
 /*
  * Workspace bytes that let retnet_retention_backward take the tensor-core path where it
- * applies (bf16 operands of the six chunkwise runs, their fp32 outputs, S0^T and the runs'
+ * applies (bf16 operands of the three chunkwise runs, their fp32 outputs, S0^T and the runs'
  * segment states); at least 2 * 4 * batch * seqlen * heads * d_k, what the CUDA-core path needs.
  */
 RETNET_API retnet_status_t retnet_backward_workspace_size(retnet_dims_t dims, size_t* bytes);
 
 /*
  * Which path retnet_retention_backward takes for these arguments with a workspace of
- * workspace_bytes (host-only; assumes 16-byte aligned buffers): 1 = tensor cores (six runs of
+ * workspace_bytes (host-only; assumes 16-byte aligned buffers): 1 = tensor cores (three runs of
  * the chunkwise forward kernel), 0 = fp32 CUDA cores, negative = the negated status.
  */
 RETNET_API int retnet_backward_kernel(retnet_dims_t dims, retnet_dtype_t in_dtype, uint32_t flags,

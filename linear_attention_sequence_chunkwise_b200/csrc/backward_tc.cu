@@ -13,10 +13,10 @@
 //   dS0   = sum_n g^(n+1) (f_n q~_n)^T dO_n  (a plain reduction over the sequence).
 // A prep kernel writes the operands (rotations, row factors, reversal) in bf16: exact copies
 // for q, k, v, dO; k~, f q~ and f dO, which are not bf16 numbers, as two parts hi + lo (hi the
-// rounded value, lo the rounded remainder, together good to about 2^-17), and each run whose
-// value operand is one of them runs once per part (the runs are linear in the value).  A post
-// kernel adds the parts' outputs, scales dq by f, turns dq and dk back (R^T) and undoes the
-// reversal of dk and dv.
+// rounded value, lo the rounded remainder, together good to about 2^-17) side by side in a
+// value row of twice the width (the runs are linear in the value, so one run gives both
+// parts' outputs, sharing its scores).  A post kernel adds the two halves of each output row,
+// scales dq by f, turns dq and dk back (R^T) and undoes the reversal of dk and dv.
 #include <algorithm>
 
 #include "launch.h"
@@ -37,10 +37,12 @@ __device__ __forceinline__ float row_f(float gamma, int d_k, int64_t p, uint32_t
   return f;
 }
 
-__device__ __forceinline__ void split_store(__nv_bfloat16* hi, __nv_bfloat16* lo, int64_t i, float x) {
+
+// x as bf16 hi (at i) + lo (at i + w): lo is the rounded remainder.
+__device__ __forceinline__ void split_store(__nv_bfloat16* p, int64_t i, int w, float x) {
   const __nv_bfloat16 a = to_bf16(x);
-  hi[i] = a;
-  lo[i] = to_bf16(x - __bfloat162float(a));
+  p[i] = a;
+  p[i + w] = to_bf16(x - __bfloat162float(a));
 }
 
 // The elementwise kernels run one CTA per token (b, t): the rotation of pair j is the same for
@@ -51,14 +53,14 @@ __device__ __forceinline__ void row_factors(float* sf, int heads, int d_k, int64
   __syncthreads();
 }
 
-// Token (b, t): k~ forward; q, k copied reversed; f q~ reversed (split).
+// Token (b, t): k~ (forward order) and f q~ (reversed) as hi | lo rows of width 2 d_k; q, k
+// copied reversed.
 __global__ void __launch_bounds__(128) bwd_tc_prep_qk(const __nv_bfloat16* __restrict__ q,
                                                       const __nv_bfloat16* __restrict__ k,
-                                                      __nv_bfloat16* __restrict__ kt, __nv_bfloat16* __restrict__ ktl,
-                                                      __nv_bfloat16* __restrict__ qR, __nv_bfloat16* __restrict__ kR,
-                                                      __nv_bfloat16* __restrict__ fqR,
-                                                      __nv_bfloat16* __restrict__ fqRl, int L, int heads, int d_k,
-                                                      int64_t pos0, uint32_t flags, HeadParams hp) {
+                                                      __nv_bfloat16* __restrict__ ktw, __nv_bfloat16* __restrict__ qR,
+                                                      __nv_bfloat16* __restrict__ kR, __nv_bfloat16* __restrict__ fqRw,
+                                                      int L, int heads, int d_k, int64_t pos0, uint32_t flags,
+                                                      HeadParams hp) {
   __shared__ float sf[RETNET_MAX_HEADS];
   const int64_t bt = blockIdx.x;
   const int t = static_cast<int>(bt % L);
@@ -69,27 +71,28 @@ __global__ void __launch_bounds__(128) bwd_tc_prep_qk(const __nv_bfloat16* __res
     float c = 1.f, s = 0.f;
     if (xpos) xpos_sincos(pos0 + t, hp.theta[j], &s, &c);
     for (int h = 0; h < heads; ++h) {
-      const int64_t o = (bt * heads + h) * d_k + 2 * j, ro = (rbt * heads + h) * d_k + 2 * j;
+      const int64_t row = bt * heads + h, rrow = rbt * heads + h;
+      const int64_t o = row * d_k + 2 * j, ro = rrow * d_k + 2 * j;
+      const int64_t ow = row * 2 * d_k + 2 * j, row_w = rrow * 2 * d_k + 2 * j;
       const __nv_bfloat162 q2 = *reinterpret_cast<const __nv_bfloat162*>(q + o);
       const __nv_bfloat162 k2 = *reinterpret_cast<const __nv_bfloat162*>(k + o);
       const float2 qf = __bfloat1622float2(q2), kf = __bfloat1622float2(k2);
       *reinterpret_cast<__nv_bfloat162*>(qR + ro) = q2;
       *reinterpret_cast<__nv_bfloat162*>(kR + ro) = k2;
-      split_store(kt, ktl, o, kf.x * c - kf.y * s);
-      split_store(kt, ktl, o + 1, kf.x * s + kf.y * c);
+      split_store(ktw, ow, d_k, kf.x * c - kf.y * s);
+      split_store(ktw, ow + 1, d_k, kf.x * s + kf.y * c);
       const float f = sf[h];
-      split_store(fqR, fqRl, ro, f * (qf.x * c - qf.y * s));
-      split_store(fqR, fqRl, ro + 1, f * (qf.x * s + qf.y * c));
+      split_store(fqRw, row_w, d_k, f * (qf.x * c - qf.y * s));
+      split_store(fqRw, row_w + 1, d_k, f * (qf.x * s + qf.y * c));
     }
   }
 }
 
-// Token (b, t): v and dO copied reversed; f dO reversed (split).  Thread = column pair.
+// Token (b, t): v and dO copied reversed; f dO reversed as hi | lo rows of width 2 d_v.
 __global__ void __launch_bounds__(128) bwd_tc_prep_v(const __nv_bfloat16* __restrict__ v,
                                                      const __nv_bfloat16* __restrict__ dout,
                                                      __nv_bfloat16* __restrict__ vR, __nv_bfloat16* __restrict__ doR,
-                                                     __nv_bfloat16* __restrict__ fdoR,
-                                                     __nv_bfloat16* __restrict__ fdoRl, int L, int heads, int d_k,
+                                                     __nv_bfloat16* __restrict__ fdoRw, int L, int heads, int d_k,
                                                      int d_v, int64_t pos0, uint32_t flags, HeadParams hp) {
   __shared__ float sf[RETNET_MAX_HEADS];
   const int64_t bt = blockIdx.x;
@@ -100,32 +103,36 @@ __global__ void __launch_bounds__(128) bwd_tc_prep_v(const __nv_bfloat16* __rest
   for (int e = threadIdx.x; e < heads * half; e += blockDim.x) {
     const int h = e / half, j = 2 * (e % half);
     const int64_t o = (bt * heads + h) * d_v + j, ro = (rbt * heads + h) * d_v + j;
+    const int64_t row_w = (rbt * heads + h) * 2 * d_v + j;
     const __nv_bfloat162 v2 = *reinterpret_cast<const __nv_bfloat162*>(v + o);
     const __nv_bfloat162 d2 = *reinterpret_cast<const __nv_bfloat162*>(dout + o);
     *reinterpret_cast<__nv_bfloat162*>(vR + ro) = v2;
     *reinterpret_cast<__nv_bfloat162*>(doR + ro) = d2;
     const float2 df = __bfloat1622float2(d2);
-    split_store(fdoR, fdoRl, ro, sf[h] * df.x);
-    split_store(fdoR, fdoRl, ro + 1, sf[h] * df.y);
+    split_store(fdoRw, row_w, d_v, sf[h] * df.x);
+    split_store(fdoRw, row_w + 1, d_v, sf[h] * df.y);
   }
 }
 
-// S0^T per (batch, head): [d_k][d_v] -> [d_v][d_k].
+// S0^T per (batch, head), as the start state of the wide dq run: [d_k][d_v] -> [d_v][2 d_k],
+// the lo half zero (the state term enters once).
 __global__ void bwd_tc_transpose(const float* __restrict__ s, float* __restrict__ st, int64_t n, int d_k, int d_v) {
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t m = i / (static_cast<int64_t>(d_k) * d_v);
     const int r = static_cast<int>(i % (static_cast<int64_t>(d_k) * d_v));
     const int a = r / d_v, bb = r % d_v;
-    st[(m * d_v + bb) * d_k + a] = s[i];
+    float* row = st + (m * d_v + bb) * 2 * d_k;
+    row[a] = s[i];
+    row[d_k + a] = 0.f;
   }
 }
 
-// Token (b, t): dq <- R^T (f (dq + dq_lo)) in place; dk <- R^T (dk~R + dk~R_lo) at the reversed row.
-__global__ void __launch_bounds__(128) bwd_tc_post_qk(float* __restrict__ dq, const float* __restrict__ dql,
-                                                      const float* __restrict__ dkR, const float* __restrict__ dkRl,
-                                                      float* __restrict__ dk, int L, int heads, int d_k, int64_t pos0,
-                                                      uint32_t flags, HeadParams hp) {
+// Token (b, t): dq = R^T (f (hi + lo halves of the dq run's row)); dk = R^T (halves of the dk
+// run's reversed row).
+__global__ void __launch_bounds__(128) bwd_tc_post_qk(const float* __restrict__ oq, const float* __restrict__ okR,
+                                                      float* __restrict__ dq, float* __restrict__ dk, int L, int heads,
+                                                      int d_k, int64_t pos0, uint32_t flags, HeadParams hp) {
   __shared__ float sf[RETNET_MAX_HEADS];
   const int64_t bt = blockIdx.x;
   const int t = static_cast<int>(bt % L);
@@ -136,36 +143,38 @@ __global__ void __launch_bounds__(128) bwd_tc_post_qk(float* __restrict__ dq, co
     float c = 1.f, s = 0.f;
     if (xpos) xpos_sincos(pos0 + t, hp.theta[j], &s, &c);
     for (int h = 0; h < heads; ++h) {
-      const int64_t o = (bt * heads + h) * d_k + 2 * j, ro = (rbt * heads + h) * d_k + 2 * j;
-      const float2 a = *reinterpret_cast<const float2*>(dq + o), al = *reinterpret_cast<const float2*>(dql + o);
-      const float y0 = sf[h] * (a.x + al.x), y1 = sf[h] * (a.y + al.y);
+      const int64_t row = bt * heads + h, rrow = rbt * heads + h;
+      const int64_t o = row * d_k + 2 * j;
+      const float* a = oq + row * 2 * d_k + 2 * j;
+      const float2 ah = *reinterpret_cast<const float2*>(a), al = *reinterpret_cast<const float2*>(a + d_k);
+      const float y0 = sf[h] * (ah.x + al.x), y1 = sf[h] * (ah.y + al.y);
       *reinterpret_cast<float2*>(dq + o) = make_float2(fmaf(y0, c, y1 * s), fmaf(y1, c, -y0 * s));
-      const float2 z = *reinterpret_cast<const float2*>(dkR + ro), zl = *reinterpret_cast<const float2*>(dkRl + ro);
-      const float z0 = z.x + zl.x, z1 = z.y + zl.y;
+      const float* z = okR + rrow * 2 * d_k + 2 * j;
+      const float2 zh = *reinterpret_cast<const float2*>(z), zl = *reinterpret_cast<const float2*>(z + d_k);
+      const float z0 = zh.x + zl.x, z1 = zh.y + zl.y;
       *reinterpret_cast<float2*>(dk + o) = make_float2(fmaf(z0, c, z1 * s), fmaf(z1, c, -z0 * s));
     }
   }
 }
 
-// Token (b, t): dv <- dvR + dvR_lo at the reversed row (float2 a thread).
-__global__ void __launch_bounds__(128) bwd_tc_post_v(const float* __restrict__ dvR, const float* __restrict__ dvRl,
-                                                     float* __restrict__ dv, int L, int heads, int d_v) {
+// Token (b, t): dv = hi + lo halves of the dv run's reversed row (float2 a thread).
+__global__ void __launch_bounds__(128) bwd_tc_post_v(const float* __restrict__ ovR, float* __restrict__ dv, int L,
+                                                     int heads, int d_v) {
   const int64_t bt = blockIdx.x;
   const int t = static_cast<int>(bt % L);
   const int64_t rbt = bt - t + (L - 1 - t);
   const int half = d_v / 2;
   for (int e = threadIdx.x; e < heads * half; e += blockDim.x) {
     const int h = e / half, j = 2 * (e % half);
-    const int64_t o = (bt * heads + h) * d_v + j, ro = (rbt * heads + h) * d_v + j;
-    const float2 a = *reinterpret_cast<const float2*>(dvR + ro), b = *reinterpret_cast<const float2*>(dvRl + ro);
-    *reinterpret_cast<float2*>(dv + o) = make_float2(a.x + b.x, a.y + b.y);
+    const float* a = ovR + (rbt * heads + h) * 2 * d_v + j;
+    const float2 ah = *reinterpret_cast<const float2*>(a), al = *reinterpret_cast<const float2*>(a + d_v);
+    *reinterpret_cast<float2*>(dv + (bt * heads + h) * d_v + j) = make_float2(ah.x + al.x, ah.y + al.y);
   }
 }
 
-// dS0[i][j] = sum_t' g^(L-t') fqR[t'][i] doR[t'][j]  (t' = L-1-n, so g^(n+1)): CTA = (b * h,
-// 32-row block of d_k), thread = (row i, columns j).
-__global__ void __launch_bounds__(256) bwd_tc_dstate(const __nv_bfloat16* __restrict__ fqR,
-                                                     const __nv_bfloat16* __restrict__ fqRl,
+// dS0[i][j] = sum_t' g^(L-t') (f q~)R[t'][i] doR[t'][j]  (t' = L-1-n, so g^(n+1)), f q~ from its
+// two parts: CTA = (b * h, 32-row block of d_k), thread = (row i, columns j).
+__global__ void __launch_bounds__(256) bwd_tc_dstate(const __nv_bfloat16* __restrict__ fqRw,
                                                      const __nv_bfloat16* __restrict__ doR, float* __restrict__ dstate,
                                                      int L, int heads, int d_k, int d_v, HeadParams hp) {
   const int bh = blockIdx.x, b = bh / heads, h = bh % heads;
@@ -176,9 +185,8 @@ __global__ void __launch_bounds__(256) bwd_tc_dstate(const __nv_bfloat16* __rest
     float s = 0.f;
     for (int tp = 0; tp < L; ++tp) {
       const int64_t r = (static_cast<int64_t>(b) * L + tp) * heads + h;
-      s = fmaf(exp2f(static_cast<float>(L - tp) * lg) *
-                   (__bfloat162float(fqR[r * d_k + i]) + __bfloat162float(fqRl[r * d_k + i])),
-               __bfloat162float(doR[r * d_v + j]), s);
+      const float fq = __bfloat162float(fqRw[r * 2 * d_k + i]) + __bfloat162float(fqRw[r * 2 * d_k + d_k + i]);
+      s = fmaf(exp2f(static_cast<float>(L - tp) * lg) * fq, __bfloat162float(doR[r * d_v + j]), s);
     }
     dstate[(static_cast<int64_t>(bh) * d_k + i) * d_v + j] = s;
   }
@@ -189,43 +197,37 @@ constexpr int kBwdChunk = 64;
 size_t a256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct TcLayout {
-  size_t kt, ktl, qR, kR, fqR, fqRl, vR, doR, fdoR, fdoRl, dkR, dkRl, dqL, dvR, dvRl, s0t, fwd, total;
+  size_t ktw, qR, kR, fqRw, vR, doR, fdoRw, oq, okR, ovR, s0t, fwd, total;
 };
 TcLayout tc_layout(const Dims& d) {
   const size_t tok = static_cast<size_t>(d.batch * d.seqlen * d.heads);
-  const size_t bk = a256(tok * d.d_k * 2), bv = a256(tok * d.d_v * 2);
+  const size_t dk = static_cast<size_t>(d.d_k), dv = static_cast<size_t>(d.d_v);
   TcLayout l{};
   size_t off = 0;
-  l.kt = off; off += bk;
-  l.ktl = off; off += bk;
-  l.qR = off; off += bk;
-  l.kR = off; off += bk;
-  l.fqR = off; off += bk;
-  l.fqRl = off; off += bk;
-  l.vR = off; off += bv;
-  l.doR = off; off += bv;
-  l.fdoR = off; off += bv;
-  l.fdoRl = off; off += bv;
-  l.dkR = off; off += a256(tok * d.d_k * 4);
-  l.dkRl = off; off += a256(tok * d.d_k * 4);
-  l.dqL = off; off += a256(tok * d.d_k * 4);
-  l.dvR = off; off += a256(tok * d.d_v * 4);
-  l.dvRl = off; off += a256(tok * d.d_v * 4);
-  l.s0t = off; off += a256(static_cast<size_t>(d.batch * d.heads * d.d_k * d.d_v) * 4);
+  l.ktw = off; off += a256(tok * 2 * dk * 2);
+  l.qR = off; off += a256(tok * dk * 2);
+  l.kR = off; off += a256(tok * dk * 2);
+  l.fqRw = off; off += a256(tok * 2 * dk * 2);
+  l.vR = off; off += a256(tok * dv * 2);
+  l.doR = off; off += a256(tok * dv * 2);
+  l.fdoRw = off; off += a256(tok * 2 * dv * 2);
+  l.oq = off; off += a256(tok * 2 * dk * 4);
+  l.okR = off; off += a256(tok * 2 * dk * 4);
+  l.ovR = off; off += a256(tok * 2 * dv * 4);
+  l.s0t = off; off += a256(static_cast<size_t>(d.batch * d.heads) * dv * 2 * dk * 4);
   l.fwd = off;
   // the forward runs' own workspace (two-pass segment states), shared by the three in turn
-  const size_t states = 6 * 4 * static_cast<size_t>(d.batch * d.heads * d.d_k * d.d_v);
-  off += a256(states);
+  off += a256(6 * 4 * static_cast<size_t>(d.batch * d.heads) * 2 * dk * dv);
   l.total = off;
   return l;
 }
 
-// The six forward runs (three sums, value hi and lo parts), described without launching.
-constexpr int kRuns = 6;
+// The three forward runs (values of twice the width: hi | lo), described without launching.
+constexpr int kRuns = 3;
 void tc_calls(const BackwardCall& c, char* ws, const TcLayout& l, RetentionCall out[kRuns]) {
   const Dims& d = c.dims;
-  const Dims d1{d.batch, d.seqlen, d.heads, d.d_v, d.d_k};  // key dim d_v, value dim d_k
-  const Dims d3{d.batch, d.seqlen, d.heads, d.d_k, d.d_v};
+  const Dims d1{d.batch, d.seqlen, d.heads, d.d_v, 2 * d.d_k};  // key dim d_v, value dim 2 d_k
+  const Dims d3{d.batch, d.seqlen, d.heads, d.d_k, 2 * d.d_v};
   auto base = [&](const void* q, const void* k, const void* v, void* o, const Dims& dd, uint32_t flags,
                   const float* s_in) {
     RetentionCall r{q, k, v, o, dd, RETNET_BF16, RETNET_F32, 0, flags, kBwdChunk, true, s_in, nullptr, nullptr,
@@ -234,19 +236,17 @@ void tc_calls(const BackwardCall& c, char* ws, const TcLayout& l, RetentionCall 
     r.ws_bytes = l.total - l.fwd;
     return r;
   };
-  out[0] = base(c.dout, c.v, ws + l.kt, c.dq, d1, 0u, c.state_in ? reinterpret_cast<const float*>(ws + l.s0t) : nullptr);
-  out[1] = base(c.dout, c.v, ws + l.ktl, ws + l.dqL, d1, 0u, nullptr);
-  out[2] = base(ws + l.vR, ws + l.doR, ws + l.fqR, ws + l.dkR, d1, 0u, nullptr);
-  out[3] = base(ws + l.vR, ws + l.doR, ws + l.fqRl, ws + l.dkRl, d1, 0u, nullptr);
-  out[4] = base(ws + l.kR, ws + l.qR, ws + l.fdoR, ws + l.dvR, d3, c.flags & RETNET_F_XPOS, nullptr);
-  out[5] = base(ws + l.kR, ws + l.qR, ws + l.fdoRl, ws + l.dvRl, d3, c.flags & RETNET_F_XPOS, nullptr);
+  out[0] = base(c.dout, c.v, ws + l.ktw, ws + l.oq, d1, 0u,
+                c.state_in ? reinterpret_cast<const float*>(ws + l.s0t) : nullptr);
+  out[1] = base(ws + l.vR, ws + l.doR, ws + l.fqRw, ws + l.okR, d1, 0u, nullptr);
+  out[2] = base(ws + l.kR, ws + l.qR, ws + l.fdoRw, ws + l.ovR, d3, c.flags & RETNET_F_XPOS, nullptr);
 }
 
 // Head parameters of each run: the kernels rotate by whatever theta they are given (a call
-// without xPos carries zeros), so the dq and dk runs get zeros and the dv runs -theta.
+// without xPos carries zeros), so the dq and dk runs get zeros and the dv run -theta.
 HeadParams run_params(const HeadParams& hp, int run) {
   HeadParams r = hp;
-  for (int j = 0; j < kMaxPairs; ++j) r.theta[j] = run >= 4 ? -hp.theta[j] : 0.f;
+  for (int j = 0; j < kMaxPairs; ++j) r.theta[j] = run == 2 ? -hp.theta[j] : 0.f;
   return r;
 }
 
@@ -261,7 +261,7 @@ bool backward_tc_applies(const BackwardCall& c, const HeadParams& hp) {
   if (!dim_ok(d.d_k) || !dim_ok(d.d_v) || d.seqlen < 1) return false;
   if (!c.ws || c.ws_bytes < backward_tc_workspace_bytes(d)) return false;
   auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
-  if (!al16(c.q) || !al16(c.k) || !al16(c.dk) || !al16(c.dv) || !al16(c.ws)) return false;  // vector accesses
+  if (!al16(c.q) || !al16(c.k) || !al16(c.dq) || !al16(c.dk) || !al16(c.dv) || !al16(c.ws)) return false;
   RetentionCall calls[kRuns];
   tc_calls(c, static_cast<char*>(c.ws), tc_layout(d), calls);
   for (int i = 0; i < kRuns; ++i)
@@ -275,45 +275,34 @@ cudaError_t launch_backward_tc(const BackwardCall& c, const HeadParams& hp, cuda
   char* ws = static_cast<char*>(c.ws);
   const int L = static_cast<int>(d.seqlen), H = static_cast<int>(d.heads), dk = static_cast<int>(d.d_k),
             dv = static_cast<int>(d.d_v);
-  auto blocks = [](int64_t items) { return static_cast<int>(std::min<int64_t>((items + 255) / 256, 148 * 16)); };
-  auto* kt = reinterpret_cast<__nv_bfloat16*>(ws + l.kt);
-  auto* ktl = reinterpret_cast<__nv_bfloat16*>(ws + l.ktl);
-  auto* fqRl = reinterpret_cast<__nv_bfloat16*>(ws + l.fqRl);
-  auto* fdoRl = reinterpret_cast<__nv_bfloat16*>(ws + l.fdoRl);
-  auto* qR = reinterpret_cast<__nv_bfloat16*>(ws + l.qR);
-  auto* kR = reinterpret_cast<__nv_bfloat16*>(ws + l.kR);
-  auto* fqR = reinterpret_cast<__nv_bfloat16*>(ws + l.fqR);
-  auto* vR = reinterpret_cast<__nv_bfloat16*>(ws + l.vR);
-  auto* doR = reinterpret_cast<__nv_bfloat16*>(ws + l.doR);
-  auto* fdoR = reinterpret_cast<__nv_bfloat16*>(ws + l.fdoR);
+  auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16*>(ws + off); };
+  auto fp = [&](size_t off) { return reinterpret_cast<float*>(ws + off); };
   const unsigned tokens = static_cast<unsigned>(d.batch * d.seqlen);
   bwd_tc_prep_qk<<<tokens, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(c.q), static_cast<const __nv_bfloat16*>(c.k),
-                                         kt, ktl, qR, kR, fqR, fqRl, L, H, dk, c.pos0, c.flags, hp);
+                                         bf(l.ktw), bf(l.qR), bf(l.kR), bf(l.fqRw), L, H, dk, c.pos0, c.flags, hp);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   bwd_tc_prep_v<<<tokens, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(c.v),
-                                        static_cast<const __nv_bfloat16*>(c.dout), vR, doR, fdoR, fdoRl, L, H, dk, dv,
-                                        c.pos0, c.flags, hp);
+                                        static_cast<const __nv_bfloat16*>(c.dout), bf(l.vR), bf(l.doR), bf(l.fdoRw), L,
+                                        H, dk, dv, c.pos0, c.flags, hp);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (c.state_in) {
     const int64_t n = d.batch * d.heads * d.d_k * d.d_v;
-    bwd_tc_transpose<<<blocks(n), 256, 0, s>>>(c.state_in, reinterpret_cast<float*>(ws + l.s0t), n, dk, dv);
+    const int blocks = static_cast<int>(std::min<int64_t>((n + 255) / 256, 148 * 16));
+    bwd_tc_transpose<<<blocks, 256, 0, s>>>(c.state_in, fp(l.s0t), n, dk, dv);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   RetentionCall calls[kRuns];
   tc_calls(c, ws, l, calls);
   for (int i = 0; i < kRuns; ++i)
     if ((e = launch_tc_chunkwise(calls[i], run_params(hp, i), s)) != cudaSuccess) return e;
-  bwd_tc_post_qk<<<tokens, 128, 0, s>>>(c.dq, reinterpret_cast<const float*>(ws + l.dqL),
-                                         reinterpret_cast<const float*>(ws + l.dkR),
-                                         reinterpret_cast<const float*>(ws + l.dkRl), c.dk, L, H, dk, c.pos0, c.flags, hp);
+  bwd_tc_post_qk<<<tokens, 128, 0, s>>>(fp(l.oq), fp(l.okR), c.dq, c.dk, L, H, dk, c.pos0, c.flags, hp);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  bwd_tc_post_v<<<tokens, 128, 0, s>>>(reinterpret_cast<const float*>(ws + l.dvR),
-                                        reinterpret_cast<const float*>(ws + l.dvRl), c.dv, L, H, dv);
+  bwd_tc_post_v<<<tokens, 128, 0, s>>>(fp(l.ovR), c.dv, L, H, dv);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (c.dstate) {
     const dim3 gs(static_cast<unsigned>(d.batch * d.heads), static_cast<unsigned>((dk + 31) / 32));
-    bwd_tc_dstate<<<gs, 256, 0, s>>>(fqR, fqRl, doR, c.dstate, L, H, dk, dv, hp);
+    bwd_tc_dstate<<<gs, 256, 0, s>>>(bf(l.fqRw), bf(l.doR), c.dstate, L, H, dk, dv, hp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return cudaSuccess;
