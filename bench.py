@@ -51,7 +51,7 @@ def bytes_per_token_head(dk, dv, elt=2):
 
 def ncu_traffic(name):
     """DRAM bytes per launch from the committed ncu record, if the kernel's sources still hash
-    to the profiled version (else None: the counters no longer describe this build)."""
+    to the profiled version (else None: the counters no longer describe the compiled kernels)."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
