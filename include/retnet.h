@@ -353,11 +353,12 @@ RETNET_API int retnet_chunkwise_kernel(retnet_dims_t dims, retnet_dtype_t in_dty
 
 /*
  * Kernel launches retnet_retention_chunkwise_ws makes for these arguments on the current
- * device (workspace_bytes = 0: retnet_retention_chunkwise): 0 without tokens, 1 for one
- * launch, 2 when the two-pass sequence segments run (pre-pass + outputs); negative = the
- * negated status the call would return.  Reads the device's SM count; no device memory
- * is touched.  gamma: host float[heads].  Assumes 16-byte aligned buffers, as
- * retnet_chunkwise_kernel does.
+ * device (workspace_bytes = 0: retnet_retention_chunkwise): 0 without tokens; else 1, or 2
+ * when a pre-pass runs first (the two-pass sequence segments' state pass, or the conversion
+ * pre-pass), plus, with RETNET_F_NORM_R on the tensor-core path, the key-sum pass (1 launch,
+ * or 2 when it cuts the sequence into segments); negative = the negated status the call would
+ * return.  Reads the device's SM count; no device memory is touched.  gamma: host
+ * float[heads].  Assumes 16-byte aligned buffers, as retnet_chunkwise_kernel does.
  */
 RETNET_API int retnet_chunkwise_launches(retnet_dims_t dims, retnet_dtype_t in_dtype, uint32_t flags, int64_t chunk,
                                          const float* gamma, size_t workspace_bytes);
