@@ -90,7 +90,8 @@ enum {
     RETNET_F_XPOS = 1u,         /* xPos rotation of q and k (§2.3 Theta) */
     RETNET_F_SCALE_SQRT_D = 2u, /* QK^T / sqrt(d_k) (§三.3) */
     RETNET_F_NORM_D = 4u,       /* D~ row normalisation (§三.3) */
-    RETNET_F_NORM_R = 8u        /* R~ normalisation by max(|row sum|, 1) (§三.3) */
+    RETNET_F_NORM_R = 8u,       /* R~ normalisation by max(|row sum|, 1) (§三.3) */
+    RETNET_F_PRECISE = 16u      /* tensor-core kernel with split fp16 operands (see Precision) */
 };
 
 typedef struct {

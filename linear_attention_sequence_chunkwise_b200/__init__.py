@@ -26,6 +26,7 @@ F_XPOS = 1
 F_SCALE_SQRT_D = 2
 F_NORM_D = 4
 F_NORM_R = 8
+F_PRECISE = 16  # split fp16 operands (hi + lo) on the tensor-core kernel
 F_ALL = F_XPOS | F_SCALE_SQRT_D | F_NORM_D | F_NORM_R
 F32 = 0
 BF16 = 1

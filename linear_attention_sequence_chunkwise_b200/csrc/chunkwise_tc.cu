@@ -595,7 +595,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 //   1 warp TMA, 1 warp MMA issuer (one unit ahead: S and dR of unit k+1 before X/PV of unit k).
 // ============================================================================================
 
-template <int DK, int T, int DVS, bool PRE = false, bool FUSE = false>
+template <int DK, int T, int DVS, bool PRE = false, bool FUSE = false, bool HL = false>
 struct Cfg3 {
   static constexpr int NDV = DVS / 64;              // 64-column boxes of the d_v slice
   static constexpr int RBLK = DK > 128 ? 2 : 1;     // 128-row blocks of the state increment
@@ -621,9 +621,15 @@ struct Cfg3 {
   static constexpr int THREADS = 32 * (WARP_MMA + 1);
   static constexpr int QBYTES = T * DK * 2;
   static constexpr int VBYTES = T * DVS * 2;
-  static constexpr int STAGE = 2 * QBYTES + VBYTES;
+  // HL (split operands): every rounded fp16 operand -- the scaled, rotated q and k, the masked
+  // scores P and the state copy -- is held as hi + lo, hi = fp16(x), lo = fp16(x - hi), so a
+  // product of two of them keeps ~22 significant bits; the stage holds [Q hi][K hi][V][Q lo][K lo].
+  static constexpr int QT = HL ? 2 : 1;
+  static constexpr int STAGE = 2 * QBYTES * QT + VBYTES;
   static constexpr int PBYTES = T * T * 2;
   static constexpr int RBYTES = DK * DVS * 2;
+  static constexpr int PB = PBYTES * QT;  // one P buffer (hi, then lo)
+  static constexpr int RB = RBYTES * QT;  // one fp16 state buffer (hi, then lo)
   // TMEM: O[2] (DVS columns each), X[XBUF] (cross accumulators; none when the slice is 128
   // wide, which then runs one sub-block per chunk only), S[SBUF] (T columns), dR[DRBUF]
   // (RBLK x DVS columns).
@@ -645,15 +651,17 @@ struct Cfg3 {
   static constexpr int TABBYTES = 2 * 2 * (DK / 2) * 8;
   static constexpr int BUDGET = 227 * 1024 - 1024;
   static constexpr int TAIL = TABBYTES + NBARS * 8 + 16 + XBYTES;
-  static constexpr int PBUF = (2 * STAGE + 2 * PBYTES + RBYTES + TAIL <= BUDGET) ? 2 : 1;
-  static constexpr int NS_R2 = (BUDGET - (PBUF * PBYTES + 2 * RBYTES + TAIL)) / STAGE;
-  static constexpr int NS_R1 = (BUDGET - (PBUF * PBYTES + RBYTES + TAIL)) / STAGE;
+  static constexpr int PBUF = (2 * STAGE + 2 * PB + RB + TAIL <= BUDGET) ? 2 : 1;
+  static constexpr int NS_R2 = (BUDGET - (PBUF * PB + 2 * RB + TAIL)) / STAGE;
+  static constexpr int NS_R1 = (BUDGET - (PBUF * PB + RB + TAIL)) / STAGE;
   static constexpr int RBUF = (NS_R2 >= 3 || NS_R1 < 3) && NS_R2 >= 2 ? 2 : 1;
-  static constexpr int FIXED = PBUF * PBYTES + RBUF * RBYTES + TAIL;
+  static constexpr int FIXED = PBUF * PB + RBUF * RB + TAIL;
   static constexpr int NS_FIT = (BUDGET - FIXED) / STAGE;
   static constexpr int NS = NS_FIT > 4 ? 4 : NS_FIT;
   static constexpr int SMEM = NS * STAGE + FIXED + 1024;
-  static constexpr bool FITS = NS >= 2 && USED <= 512 && (DVS == 64 || DVS == 128) && (!RTM || DRBUF == 1);
+  // split operands at d_k = 256 leave room for one stage only (the units then run in turn)
+  static constexpr bool FITS = NS >= (HL ? 1 : 2) && USED <= 512 && (DVS == 64 || DVS == 128) && (!RTM || DRBUF == 1) &&
+                               (!HL || (T == 64 && DVS == 64));
   // Columns per TMEM load batch: 18 warps leave 96 registers a thread (five warps share one
   // sub-partition's register file), too few to hold 64 loaded columns next to the state.
   static constexpr int LDW = THREADS > 512 ? 32 : 64;
@@ -811,9 +819,10 @@ struct UnitConverter {
   // In place: q -> gamma^(r+1) rot(q), k -> gamma^(T-1-r) rot(k) as fp16 (r local); v -> fp16.
   // WITH_Q = false (state replay) leaves the Q tile alone.
   // zmul multiplies the K row scales (the state pre-pass decays K to its segment's end).
-  template <bool WITH_Q>
+  // HL: the tiles take the fp16 hi parts, sql / skl (same layout) the lo parts.
+  template <bool WITH_Q, bool HL = false>
   __device__ void convert(uint32_t sq, uint32_t sk, uint32_t sv, const float2* bq, const float2* bk, bool xpos,
-                          float log2g, float zmul = 1.f) const {
+                          float log2g, float zmul = 1.f, uint32_t sql = 0, uint32_t skl = 0) const {
     const uint32_t box = (cs / 8) * T * 128;
     const uint32_t chunk = cs % 8;
     const float xstep = decay_pow(log2g, RS), zstep = exp2f(-static_cast<float>(RS) * log2g);
@@ -839,21 +848,35 @@ struct UnitConverter {
       }
 #pragma unroll
       for (int k = 0; k < G; ++k) {
-        uint32_t qo[4], ko[4];
+        uint32_t qo[4], ko[4], ql[4], kl[4];
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
           if (WITH_Q) {
             const float q0 = __uint_as_float(q4[k][jj] << 16), q1 = __uint_as_float(q4[k][jj] & 0xffff0000u);
-            qo[jj] = pack_f16x2(q0 * Fq[jj].x - q1 * Fq[jj].y, q0 * Fq[jj].y + q1 * Fq[jj].x);
+            const float x0 = q0 * Fq[jj].x - q1 * Fq[jj].y, x1 = q0 * Fq[jj].y + q1 * Fq[jj].x;
+            if (HL) {
+              split_f16x2(x0, x1, qo[jj], ql[jj]);
+            } else {
+              qo[jj] = pack_f16x2(x0, x1);
+            }
             Fq[jj] = cmul(Fq[jj], Zq[jj]);
           }
           const float k0 = __uint_as_float(k4[k][jj] << 16), k1 = __uint_as_float(k4[k][jj] & 0xffff0000u);
-          ko[jj] = pack_f16x2(k0 * Fk[jj].x - k1 * Fk[jj].y, k0 * Fk[jj].y + k1 * Fk[jj].x);
+          const float y0 = k0 * Fk[jj].x - k1 * Fk[jj].y, y1 = k0 * Fk[jj].y + k1 * Fk[jj].x;
+          if (HL) {
+            split_f16x2(y0, y1, ko[jj], kl[jj]);
+          } else {
+            ko[jj] = pack_f16x2(y0, y1);
+          }
           Fk[jj] = cmul(Fk[jj], Zk[jj]);
         }
         const uint32_t off = box + sw128(r0 + RS * (kg + k), chunk);
         if (WITH_Q) st_shared_v4(sq + off, qo[0], qo[1], qo[2], qo[3]);
         st_shared_v4(sk + off, ko[0], ko[1], ko[2], ko[3]);
+        if (HL) {
+          if (WITH_Q) st_shared_v4(sql + off, ql[0], ql[1], ql[2], ql[3]);
+          st_shared_v4(skl + off, kl[0], kl[1], kl[2], kl[3]);
+        }
       }
     }
     // V: each 64-column box, slot lt % 8, rows lt / 8 + VR k.
@@ -876,12 +899,15 @@ struct UnitConverter {
   }
 };
 
-template <int DK, int T, int DVS, int SM, bool PRE, bool FUSE, typename Tout>
-__global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE>::THREADS, 1)
+template <int DK, int T, int DVS, int SM, bool PRE, bool FUSE, typename Tout, bool HL = false>
+__global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL>::THREADS, 1)
     tc_chunkwise_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                             const __grid_constant__ CUtensorMap tm_v, TcArgs a, HeadParams hp) {
-  using C = Cfg3<DK, T, DVS, PRE, FUSE>;
+                             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_ql,
+                             const __grid_constant__ CUtensorMap tm_kl, TcArgs a, HeadParams hp) {
+  // tm_ql, tm_kl: the lo parts of pre-converted split operands (HL with PRE); unused otherwise.
+  using C = Cfg3<DK, T, DVS, PRE, FUSE, HL>;
   static_assert(!FUSE || (SM == SEG_NONE && DVS == 64), "the fused epilogue runs unsplit, 64-column slices");
+  static_assert(!HL || SM == SEG_NONE, "split operands run without sequence segments");
   // Stage ready for the MMAs: converted in place, or (PRE) landed already converted.
   constexpr int Q_READY = PRE ? Q_TMA_FULL : Q_CONV_FULL;
   constexpr bool SEG = SM != SEG_NONE;
@@ -968,8 +994,8 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE>::THREADS, 1)
   const float sd = rsqrtf(static_cast<float>(DK));  // carried by P and the fp16 state copy
 
   const uint32_t sP0 = sbase + C::NS * C::STAGE;
-  const uint32_t sR0 = sP0 + C::PBUF * C::PBYTES;
-  const int tail_off = C::NS * C::STAGE + C::PBUF * C::PBYTES + C::RBUF * C::RBYTES;
+  const uint32_t sR0 = sP0 + C::PBUF * C::PB;
+  const int tail_off = C::NS * C::STAGE + C::PBUF * C::PB + C::RBUF * C::RB;
   float2* tab = reinterpret_cast<float2*>(gbase + tail_off);
   uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + tail_off + C::TABBYTES);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::NBARS);
@@ -983,8 +1009,12 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE>::THREADS, 1)
   auto sQ = [&](int s) { return sbase + s * C::STAGE; };
   auto sK = [&](int s) { return sbase + s * C::STAGE + C::QBYTES; };
   auto sV = [&](int s) { return sbase + s * C::STAGE + 2 * C::QBYTES; };
-  auto sP = [&](int k) { return sP0 + (k % C::PBUF) * C::PBYTES; };
-  auto sR = [&](int i) { return sR0 + (i % C::RBUF) * C::RBYTES; };
+  // HL: lo parts of Q and K after V in the stage; P and the state copy keep their lo part
+  // right after the hi part of the same buffer
+  auto sQl = [&](int s) { return sbase + s * C::STAGE + 2 * C::QBYTES + C::VBYTES; };
+  auto sKl = [&](int s) { return sbase + s * C::STAGE + 3 * C::QBYTES + C::VBYTES; };
+  auto sP = [&](int k) { return sP0 + (k % C::PBUF) * C::PB; };
+  auto sR = [&](int i) { return sR0 + (i % C::RBUF) * C::RB; };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < 4; ++s) {
@@ -1017,6 +1047,10 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE>::THREADS, 1)
     prefetch_tensormap(&tm_q);
     prefetch_tensormap(&tm_k);
     prefetch_tensormap(&tm_v);
+    if (HL && PRE) {
+      prefetch_tensormap(&tm_ql);
+      prefetch_tensormap(&tm_kl);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -1033,12 +1067,18 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE>::THREADS, 1)
         const int s = it.k % C::NS;
         if (it.k >= C::NS && !mbar_wait(bar(Q_STAGE_EMPTY + s), ((it.k / C::NS) - 1) & 1)) break;
         const bool with_q = !it.pre();  // state replay needs K and V only
-        mbar_arrive_expect_tx(bar(Q_TMA_FULL + s), with_q ? C::STAGE : C::STAGE - C::QBYTES);
+        // bytes that land: Q (unless replay) and K, with their lo parts when pre-converted split
+        constexpr int QK_PARTS = (HL && PRE) ? 2 : 1;
+        mbar_arrive_expect_tx(bar(Q_TMA_FULL + s), (with_q ? 2 : 1) * C::QBYTES * QK_PARTS + C::VBYTES);
         const int tq = it.t0() + it.u * T, tk = it.t0() + it.w * T;
 #pragma unroll
         for (int bx = 0; bx < DK / 64; ++bx) {
           if (with_q) tma_load_4d(sQ(s) + bx * T * 128, &tm_q, bar(Q_TMA_FULL + s), bx * 64, h, tq, b);
           tma_load_4d(sK(s) + bx * T * 128, &tm_k, bar(Q_TMA_FULL + s), bx * 64, h, tk, b);
+          if constexpr (HL && PRE) {
+            if (with_q) tma_load_4d(sQl(s) + bx * T * 128, &tm_ql, bar(Q_TMA_FULL + s), bx * 64, h, tq, b);
+            tma_load_4d(sKl(s) + bx * T * 128, &tm_kl, bar(Q_TMA_FULL + s), bx * 64, h, tk, b);
+          }
         }
 #pragma unroll
         for (int bx = 0; bx < C::NDV; ++bx)
@@ -1086,6 +1126,13 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE>::THREADS, 1)
           const uint64_t dq = sdesc_sw128(sQ(s), 16, 1024), dk = sdesc_sw128(sK(s), 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < DK / 16; ++kk) mma_f16_ss(tS, dq + kstep(kk), dk + kstep(kk), ID_S, kk > 0);
+          if constexpr (HL) {  // S += Qlo Khi^T + Qhi Klo^T (the lo x lo term is below 2^-22)
+            const uint64_t dql = sdesc_sw128(sQl(s), 16, 1024), dkl = sdesc_sw128(sKl(s), 16, 1024);
+#pragma unroll
+            for (int kk = 0; kk < DK / 16; ++kk) mma_f16_ss(tS, dql + kstep(kk), dk + kstep(kk), ID_S, 1u);
+#pragma unroll
+            for (int kk = 0; kk < DK / 16; ++kk) mma_f16_ss(tS, dq + kstep(kk), dkl + kstep(kk), ID_S, 1u);
+          }
           mma_commit(bar(Q_S_FULL + (f.kf() % C::SBUF)));
         }
         if (f.last_row()) {
@@ -1097,6 +1144,15 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE>::THREADS, 1)
             for (int ks = 0; ks < T / 16; ++ks)
               mma_f16_ss(tD + blk * DVS, dkm + static_cast<uint64_t>((blk * 2 * T * 128 + ks * 2048) >> 4),
                          dv + static_cast<uint64_t>((ks * 2048) >> 4), ID_R, (C::RTM || ks > 0) ? 1u : 0u);
+          if constexpr (HL) {  // + Klo^T V (V is exact in fp16)
+            const uint64_t dklm = sdesc_sw128(sKl(s), T * 128, 1024);
+#pragma unroll
+            for (int blk = 0; blk < C::RBLK; ++blk)
+#pragma unroll
+              for (int ks = 0; ks < T / 16; ++ks)
+                mma_f16_ss(tD + blk * DVS, dklm + static_cast<uint64_t>((blk * 2 * T * 128 + ks * 2048) >> 4),
+                           dv + static_cast<uint64_t>((ks * 2048) >> 4), ID_R, 1u);
+          }
           mma_commit(bar(Q_DR_FULL + (f.dr % C::DRBUF)));
         }
         if (f.pre()) mma_commit(bar(Q_STAGE_EMPTY + s));  // a replay unit has no P V
@@ -1116,6 +1172,15 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE>::THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk)
           mma_f16_ss(tX, dq + kstep(kk), dr + static_cast<uint64_t>((kk * 2048) >> 4), ID_X, kk > 0);
+        if constexpr (HL) {  // + Qlo Rhi + Qhi Rlo
+          const uint64_t dql = sdesc_sw128(sQl(s), 16, 1024), drl = sdesc_sw128(sR(ri) + C::RBYTES, DK * 128, 1024);
+#pragma unroll
+          for (int kk = 0; kk < DK / 16; ++kk)
+            mma_f16_ss(tX, dql + kstep(kk), dr + static_cast<uint64_t>((kk * 2048) >> 4), ID_X, 1u);
+#pragma unroll
+          for (int kk = 0; kk < DK / 16; ++kk)
+            mma_f16_ss(tX, dq + kstep(kk), drl + static_cast<uint64_t>((kk * 2048) >> 4), ID_X, 1u);
+        }
         if (q.last_row()) mma_commit(bar(Q_R16_FREE + (ri % C::RBUF)));
       };
       auto p_ready = [&](const UnitIter<T, SM>& q) -> bool {
@@ -1130,6 +1195,12 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE>::THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < T / 16; ++kk)
           mma_f16_ss(tO, dp + kstep(kk), dv + static_cast<uint64_t>((kk * 2048) >> 4), ID_X, kk > 0 ? 1u : acc0);
+        if constexpr (HL) {  // + Plo V
+          const uint64_t dpl = sdesc_sw128(sP(q.kf()) + C::PBYTES, 16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < T / 16; ++kk)
+            mma_f16_ss(tO, dpl + kstep(kk), dv + static_cast<uint64_t>((kk * 2048) >> 4), ID_X, 1u);
+        }
         mma_commit(bar(Q_P_FREE + (q.kf() % C::PBUF)));
         if (q.rb_done()) mma_commit(bar(Q_O_FULL + (q.rb & 1)));
         mma_commit(bar(Q_STAGE_EMPTY + s));
@@ -1219,7 +1290,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE>::THREADS, 1)
       } else if (SM == SEG_REPLAY && it.pre()) {
         cv.template convert<false>(sQ(s), sK(s), sV(s), tq, tk, xpos, log2g);
       } else {
-        cv.template convert<true>(sQ(s), sK(s), sV(s), tq, tk, xpos, log2g);
+        cv.template convert<true, HL>(sQ(s), sK(s), sV(s), tq, tk, xpos, log2g, 1.f, sQl(s), sKl(s));
       }
       fence_proxy_async_smem();
       mbar_arrive(bar(Q_CONV_FULL + s));
@@ -1316,11 +1387,20 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE>::THREADS, 1)
               for (int c8 = 0; c8 < GW / 8; ++c8) {
                 const int col = GW * grp + 8 * c8;
                 const uint32_t* x = &u[(8 * c8) / 16][(8 * c8) % 16];
-                st_shared_v4(r16 + (col / 64) * DK * 128 + sw128(dk, (col % 64) / 8),
-                             pack_f16x2(sd * __uint_as_float(x[0]), sd * __uint_as_float(x[1])),
-                             pack_f16x2(sd * __uint_as_float(x[2]), sd * __uint_as_float(x[3])),
-                             pack_f16x2(sd * __uint_as_float(x[4]), sd * __uint_as_float(x[5])),
-                             pack_f16x2(sd * __uint_as_float(x[6]), sd * __uint_as_float(x[7])));
+                const uint32_t off = (col / 64) * DK * 128 + sw128(dk, (col % 64) / 8);
+                if constexpr (HL) {
+                  uint32_t hi[4], lo[4];
+#pragma unroll
+                  for (int e = 0; e < 4; ++e)
+                    split_f16x2(sd * __uint_as_float(x[2 * e]), sd * __uint_as_float(x[2 * e + 1]), hi[e], lo[e]);
+                  st_shared_v4(r16 + off, hi[0], hi[1], hi[2], hi[3]);
+                  st_shared_v4(r16 + C::RBYTES + off, lo[0], lo[1], lo[2], lo[3]);
+                } else {
+                  st_shared_v4(r16 + off, pack_f16x2(sd * __uint_as_float(x[0]), sd * __uint_as_float(x[1])),
+                               pack_f16x2(sd * __uint_as_float(x[2]), sd * __uint_as_float(x[3])),
+                               pack_f16x2(sd * __uint_as_float(x[4]), sd * __uint_as_float(x[5])),
+                               pack_f16x2(sd * __uint_as_float(x[6]), sd * __uint_as_float(x[7])));
+                }
               }
             }
 #pragma unroll
@@ -1383,11 +1463,20 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE>::THREADS, 1)
         if (dk < 0) return;
         base += ch * DK * 128;
   #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8)
-          st_shared_v4(base + sw128(dk, c8), pack_f16x2(sd * R[8 * c8 + 0], sd * R[8 * c8 + 1]),
-                       pack_f16x2(sd * R[8 * c8 + 2], sd * R[8 * c8 + 3]),
-                       pack_f16x2(sd * R[8 * c8 + 4], sd * R[8 * c8 + 5]),
-                       pack_f16x2(sd * R[8 * c8 + 6], sd * R[8 * c8 + 7]));
+        for (int c8 = 0; c8 < 8; ++c8) {
+          if constexpr (HL) {
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) split_f16x2(sd * R[8 * c8 + 2 * e], sd * R[8 * c8 + 2 * e + 1], hi[e], lo[e]);
+            st_shared_v4(base + sw128(dk, c8), hi[0], hi[1], hi[2], hi[3]);
+            st_shared_v4(base + C::RBYTES + sw128(dk, c8), lo[0], lo[1], lo[2], lo[3]);
+          } else {
+            st_shared_v4(base + sw128(dk, c8), pack_f16x2(sd * R[8 * c8 + 0], sd * R[8 * c8 + 1]),
+                         pack_f16x2(sd * R[8 * c8 + 2], sd * R[8 * c8 + 3]),
+                         pack_f16x2(sd * R[8 * c8 + 4], sd * R[8 * c8 + 5]),
+                         pack_f16x2(sd * R[8 * c8 + 6], sd * R[8 * c8 + 7]));
+          }
+        }
       };
       if (c_first == c_lo) {  // otherwise written once the replay reaches the first output chunk
         put_r16(sR(0));
@@ -1692,15 +1781,21 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE>::THREADS, 1)
 #pragma unroll
           for (int c8 = 0; c8 < C::LDW / 8; ++c8) {
             const int col = grp * C::LDW + 8 * c8;
-            uint32_t pk[4];
+            uint32_t pk[4], pl[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int c0 = col + 2 * e;
               const float p0 = (!diag || c0 <= my_row) ? __uint_as_float(u16[c8 / 2][(8 * c8 + 2 * e) % 16]) * pf : 0.f;
               const float p1 = (!diag || c0 + 1 <= my_row) ? __uint_as_float(u16[c8 / 2][(8 * c8 + 2 * e + 1) % 16]) * pf : 0.f;
-              pk[e] = pack_f16x2(p0, p1);
+              if (HL) {
+                split_f16x2(p0, p1, pk[e], pl[e]);
+              } else {
+                pk[e] = pack_f16x2(p0, p1);
+              }
             }
-            st_shared_v4(sP(k) + (col / 64) * T * 128 + sw128(my_row, (col % 64) / 8), pk[0], pk[1], pk[2], pk[3]);
+            const uint32_t poff = (col / 64) * T * 128 + sw128(my_row, (col % 64) / 8);
+            st_shared_v4(sP(k) + poff, pk[0], pk[1], pk[2], pk[3]);
+            if (HL) st_shared_v4(sP(k) + C::PBYTES + poff, pl[0], pl[1], pl[2], pl[3]);
           }
         }
       }
@@ -1737,10 +1832,12 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE>::THREADS, 1)
 // the rotation by the absolute position p = pos0 + t.  Thread = (token, 8-element slot of
 // d_k) across every head (the rotation factors are computed once), then (8-element slots of v).
 // ============================================================================================
-template <int DK, int T>
+// HL: q~ and k~ as split operands, hi parts into qo / ko, lo parts into qlo / klo.
+template <int DK, int T, bool HL = false>
 __global__ void __launch_bounds__(256) tc_convert_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
                                                          const uint4* __restrict__ v, uint4* __restrict__ qo,
                                                          uint4* __restrict__ ko, uint4* __restrict__ vo,
+                                                         uint4* __restrict__ qlo, uint4* __restrict__ klo,
                                                          int64_t tokens, int L, int heads, int dv, int64_t pos0,
                                                          uint32_t flags, HeadParams hp) {
   constexpr int S = DK / 8;  // 16-byte slots of a head row of q or k
@@ -1766,16 +1863,27 @@ __global__ void __launch_bounds__(256) tc_convert_kernel(const uint4* __restrict
         const float l2g = hp.log2g[h];
         const float xi = decay_pow(l2g, r + 1), zeta = decay_pow(l2g, T - 1 - r);
         const uint32_t wq[4] = {xq.x, xq.y, xq.z, xq.w}, wk[4] = {xk.x, xk.y, xk.z, xk.w};
-        uint32_t oq[4], ok[4];
+        uint32_t oq[4], ok[4], lq[4], lk[4];
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
           const float q0 = __uint_as_float(wq[jj] << 16), q1 = __uint_as_float(wq[jj] & 0xffff0000u);
           const float k0 = __uint_as_float(wk[jj] << 16), k1 = __uint_as_float(wk[jj] & 0xffff0000u);
-          oq[jj] = pack_f16x2(xi * (q0 * f[jj].x - q1 * f[jj].y), xi * (q0 * f[jj].y + q1 * f[jj].x));
-          ok[jj] = pack_f16x2(zeta * (k0 * f[jj].x - k1 * f[jj].y), zeta * (k0 * f[jj].y + k1 * f[jj].x));
+          const float x0 = xi * (q0 * f[jj].x - q1 * f[jj].y), x1 = xi * (q0 * f[jj].y + q1 * f[jj].x);
+          const float y0 = zeta * (k0 * f[jj].x - k1 * f[jj].y), y1 = zeta * (k0 * f[jj].y + k1 * f[jj].x);
+          if (HL) {
+            split_f16x2(x0, x1, oq[jj], lq[jj]);
+            split_f16x2(y0, y1, ok[jj], lk[jj]);
+          } else {
+            oq[jj] = pack_f16x2(x0, x1);
+            ok[jj] = pack_f16x2(y0, y1);
+          }
         }
         qo[off] = make_uint4(oq[0], oq[1], oq[2], oq[3]);
         ko[off] = make_uint4(ok[0], ok[1], ok[2], ok[3]);
+        if (HL) {
+          qlo[off] = make_uint4(lq[0], lq[1], lq[2], lq[3]);
+          klo[off] = make_uint4(lk[0], lk[1], lk[2], lk[3]);
+        }
       }
     } else {
       const int64_t j = i - n_qk;
@@ -1833,8 +1941,10 @@ bool force_serial_kernel() {
   return serial;
 }
 
-// Rows per unit of the pipelined kernel: 64 for d_k = 256 (shared memory), else min(B, 128).
+// Rows per unit of the pipelined kernel: 64 for d_k = 256 (shared memory), else min(B, 128);
+// split operands (precise calls) always take 64-row units.
 int pipe_tile_rows(int64_t d_k, int64_t chunk) { return d_k == 256 ? 64 : static_cast<int>(chunk < 128 ? chunk : 128); }
+int pipe_tile_rows(const RetentionCall& c) { return c.precise ? 64 : pipe_tile_rows(c.dims.d_k, c.chunk); }
 
 // Segment plan of a call (see plan_segments); returns how many pre-pass states the caller's
 // workspace holds (0: no workspace, single-launch replay form).
@@ -1851,28 +1961,31 @@ int plan_call(const RetentionCall& c, int64_t ctas, int sms, TcArgs& as) {
   return max_states;
 }
 
-// fp16 copies of the conversion pre-pass in the caller's workspace (256-byte aligned parts).
+// fp16 copies of the conversion pre-pass in the caller's workspace (256-byte aligned parts):
+// q~, k~, v, and for split operands the lo parts of q~ and k~ after them.
 struct PreCopies {
   void* q;
   void* k;
   void* v;
+  void* ql;
+  void* kl;
 };
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
-size_t pre_copy_bytes(const Dims& d) {
+size_t pre_copy_bytes(const Dims& d, bool hl) {
   const size_t tok = static_cast<size_t>(d.batch) * static_cast<size_t>(d.seqlen) * static_cast<size_t>(d.heads);
-  return 2 * align256(tok * d.d_k * 2) + align256(tok * d.d_v * 2);
+  return (hl ? 4 : 2) * align256(tok * d.d_k * 2) + align256(tok * d.d_v * 2);
 }
 PreCopies pre_copies(const RetentionCall& c) {
   const size_t tok = static_cast<size_t>(c.dims.batch) * static_cast<size_t>(c.dims.seqlen) *
                      static_cast<size_t>(c.dims.heads);
   char* base = static_cast<char*>(c.ws);
-  const size_t qk = align256(tok * c.dims.d_k * 2);
-  return PreCopies{base, base + qk, base + 2 * qk};
+  const size_t qk = align256(tok * c.dims.d_k * 2), vb = align256(tok * c.dims.d_v * 2);
+  return PreCopies{base, base + qk, base + 2 * qk, base + 2 * qk + vb, base + 3 * qk + vb};
 }
 // The pre-pass pays one extra read and write of q, k, v; it saves the (nb + 1) / 2-fold
 // reconversion of chunks of nb >= 2 sub-blocks.  Not combined with sequence segments.
 bool pre_convert_applies(const RetentionCall& c, int nb, int n_seg) {
-  return nb >= 2 && n_seg < 2 && c.ws && c.ws_bytes >= pre_copy_bytes(c.dims);
+  return nb >= 2 && n_seg < 2 && c.ws && c.ws_bytes >= pre_copy_bytes(c.dims, c.precise);
 }
 
 // 128-column d_v slices share S and the Q/K conversion across twice the output columns
@@ -1962,61 +2075,114 @@ dim3 tc_grid(const Dims& d, int dvs) {
   return dim3(static_cast<unsigned>(d.d_v / dvs), static_cast<unsigned>(d.heads), static_cast<unsigned>(d.batch));
 }
 
-// Fused MSR epilogue: the d_v slices of a head form one thread-block cluster (n_cl <=
-// kMaxCluster CTAs) that pools the GroupNorm statistics in distributed shared memory.  With
-// chunks of several sub-blocks and room in the workspace the conversion pre-pass runs first.
-template <int DK, int T, typename Tout>
-cudaError_t launch_fused(const RetentionCall& c, const HeadParams& hp, cudaStream_t s, const CUtensorMap& mq,
-                         const CUtensorMap& mk, const CUtensorMap& mv, const TcArgs& a, int nb) {
-  const int n_cl = static_cast<int>(c.dims.d_v / 64);
-  if (n_cl < 1 || n_cl > kMaxCluster) return cudaErrorInvalidValue;
-  const dim3 grid = tc_grid(c.dims, 64);
-  auto launch = [&](auto kern, int threads, int smem, const CUtensorMap& q, const CUtensorMap& k,
-                    const CUtensorMap& v) -> cudaError_t {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = dim3(threads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+// Conversion pre-pass into the workspace copies (pc), then tensor maps over them.
+template <int DK, int T, bool HL>
+cudaError_t run_convert(const RetentionCall& c, const HeadParams& hp, cudaStream_t s, const PreCopies& pc,
+                        CUtensorMap* m) {
+  const int64_t tokens = c.dims.batch * c.dims.seqlen;
+  const int64_t items = tokens * (DK / 8) + tokens * c.dims.heads * (c.dims.d_v / 8);
+  const int blocks = static_cast<int>(std::min<int64_t>((items + 255) / 256, static_cast<int64_t>(sm_count()) * 8));
+  tc_convert_kernel<DK, T, HL><<<blocks, 256, 0, s>>>(
+      static_cast<const uint4*>(c.q), static_cast<const uint4*>(c.k), static_cast<const uint4*>(c.v),
+      static_cast<uint4*>(pc.q), static_cast<uint4*>(pc.k), static_cast<uint4*>(pc.v), static_cast<uint4*>(pc.ql),
+      static_cast<uint4*>(pc.kl), tokens, static_cast<int>(c.dims.seqlen), static_cast<int>(c.dims.heads),
+      static_cast<int>(c.dims.d_v), c.pos0, c.flags, hp);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  RetentionCall cc = c;
+  cc.q = pc.q;
+  cc.k = pc.k;
+  cc.v = pc.v;
+  if (!make_maps(cc, T, &m[0], &m[1], &m[2])) return cudaErrorInvalidValue;
+  m[3] = m[0];
+  m[4] = m[1];
+  if (HL) {
+    const Dims& d = c.dims;
+    if (!make_map(&m[3], pc.ql, d.batch, d.seqlen, d.heads, d.d_k, T) ||
+        !make_map(&m[4], pc.kl, d.batch, d.seqlen, d.heads, d.d_k, T))
+      return cudaErrorInvalidValue;
+  }
+  return cudaSuccess;
+}
+
+// One launch of the pipelined kernel over the (d_v slice, head, batch) grid.  cluster > 0: the
+// d_v slices of a head form one thread-block cluster of that many CTAs (the fused GroupNorm
+// epilogue uses cluster-scope instructions, so it is launched as a cluster even with one CTA);
+// cluster = 0: no cluster.
+template <typename K>
+cudaError_t launch_kernel(K kern, dim3 grid, int threads, int smem, cudaStream_t s, const CUtensorMap* m,
+                          const TcArgs& a, const HeadParams& hp, int cluster) {
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(threads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  if (cluster > 0) {
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = n_cl;
+    attr[0].val.clusterDim.x = cluster;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, q, k, v, a, hp);
-  };
+  }
+  return cudaLaunchKernelEx(&cfg, kern, m[0], m[1], m[2], m[3], m[4], a, hp);
+}
+
+// Fused MSR epilogue (c.gate) and split operands (HL): one CTA per (batch, head, 64-column d_v
+// slice), no sequence segments.  With the gate, the d_v slices of a head form one thread-block
+// cluster (n_cl <= kMaxCluster CTAs) that pools the GroupNorm statistics in distributed shared
+// memory.  With chunks of several sub-blocks and room in the workspace the conversion pre-pass
+// runs first.
+template <int DK, int T, typename Tout, bool HL>
+cudaError_t launch_unsplit(const RetentionCall& c, const HeadParams& hp, cudaStream_t s, const CUtensorMap* maps,
+                           const TcArgs& a, int nb) {
+  const bool fuse = c.gate != nullptr;
+  const int n_cl = fuse ? static_cast<int>(c.dims.d_v / 64) : 1;
+  if (n_cl < 1 || n_cl > kMaxCluster) return cudaErrorInvalidValue;
+  const dim3 grid = tc_grid(c.dims, 64);
   if constexpr (Cfg3<DK, T, 64>::XBUF > 0) {
     if (pre_convert_applies(c, nb, 1)) {
-      const PreCopies pc = pre_copies(c);
-      const int64_t tokens = c.dims.batch * c.dims.seqlen;
-      const int64_t items = tokens * (DK / 8) + tokens * c.dims.heads * (c.dims.d_v / 8);
-      const int blocks = static_cast<int>(std::min<int64_t>((items + 255) / 256, static_cast<int64_t>(sm_count()) * 8));
-      tc_convert_kernel<DK, T><<<blocks, 256, 0, s>>>(
-          static_cast<const uint4*>(c.q), static_cast<const uint4*>(c.k), static_cast<const uint4*>(c.v),
-          static_cast<uint4*>(pc.q), static_cast<uint4*>(pc.k), static_cast<uint4*>(pc.v), tokens,
-          static_cast<int>(c.dims.seqlen), static_cast<int>(c.dims.heads), static_cast<int>(c.dims.d_v), c.pos0,
-          c.flags, hp);
-      cudaError_t e = cudaGetLastError();
+      CUtensorMap pm[5];
+      cudaError_t e = run_convert<DK, T, HL>(c, hp, s, pre_copies(c), pm);
       if (e != cudaSuccess) return e;
-      RetentionCall cc = c;
-      cc.q = pc.q;
-      cc.k = pc.k;
-      cc.v = pc.v;
-      CUtensorMap pq, pk, pv;
-      if (!make_maps(cc, T, &pq, &pk, &pv)) return cudaErrorInvalidValue;
-      using CP = Cfg3<DK, T, 64, true, true>;
-      static_assert(CP::FITS, "fused kernel does not fit this tile");
-      return launch(tc_chunkwise_pipe_kernel<DK, T, 64, SEG_NONE, true, true, Tout>, CP::THREADS, CP::SMEM, pq, pk,
-                    pv);
+      if (fuse) {
+        using CP = Cfg3<DK, T, 64, true, true, HL>;
+        static_assert(CP::FITS, "fused kernel does not fit this tile");
+        return launch_kernel(tc_chunkwise_pipe_kernel<DK, T, 64, SEG_NONE, true, true, Tout, HL>, grid, CP::THREADS,
+                             CP::SMEM, s, pm, a, hp, n_cl);
+      }
+      using CP = Cfg3<DK, T, 64, true, false, HL>;
+      static_assert(CP::FITS, "pipelined kernel does not fit this tile");
+      return launch_kernel(tc_chunkwise_pipe_kernel<DK, T, 64, SEG_NONE, true, false, Tout, HL>, grid, CP::THREADS,
+                           CP::SMEM, s, pm, a, hp, 0);
     }
   }
-  using CF = Cfg3<DK, T, 64, false, true>;
-  static_assert(CF::FITS, "fused kernel does not fit this tile");
-  return launch(tc_chunkwise_pipe_kernel<DK, T, 64, SEG_NONE, false, true, Tout>, CF::THREADS, CF::SMEM, mq, mk, mv);
+  if (fuse) {
+    using CF = Cfg3<DK, T, 64, false, true, HL>;
+    static_assert(CF::FITS, "fused kernel does not fit this tile");
+    return launch_kernel(tc_chunkwise_pipe_kernel<DK, T, 64, SEG_NONE, false, true, Tout, HL>, grid, CF::THREADS,
+                         CF::SMEM, s, maps, a, hp, n_cl);
+  }
+  using CF = Cfg3<DK, T, 64, false, false, HL>;
+  static_assert(CF::FITS, "pipelined kernel does not fit this tile");
+  return launch_kernel(tc_chunkwise_pipe_kernel<DK, T, 64, SEG_NONE, false, false, Tout, HL>, grid, CF::THREADS,
+                       CF::SMEM, s, maps, a, hp, 0);
+}
+
+// Split operands (precise calls: RETNET_F_PRECISE, R~ and the fused MSR epilogue): 64-row units,
+// 64-column d_v slices, no sequence segments.
+template <int DK, typename Tout>
+cudaError_t launch_pipe_hl(const RetentionCall& c, const HeadParams& hp, cudaStream_t s) {
+  CUtensorMap m[5];
+  if (!make_maps(c, 64, &m[0], &m[1], &m[2])) return cudaErrorInvalidValue;
+  m[3] = m[0];
+  m[4] = m[1];
+  const int nb = static_cast<int>(c.chunk / 64);
+  const TcArgs a = make_args(c, static_cast<int>((c.dims.seqlen + c.chunk - 1) / c.chunk), nb);
+  return launch_unsplit<DK, 64, Tout, true>(c, hp, s, m, a, nb);
 }
 
 // Pipelined kernel: units of T rows, nb = B / T per chunk, d_v slices of DVS columns.
@@ -2027,11 +2193,12 @@ cudaError_t launch_pipe(const RetentionCall& c, const HeadParams& hp, cudaStream
   static_assert(Cf::FITS, "pipelined kernel does not fit this tile");
   CUtensorMap mq, mk, mv;
   if (!make_maps(c, T, &mq, &mk, &mv)) return cudaErrorInvalidValue;
+  const CUtensorMap m5[5] = {mq, mk, mv, mq, mk};
   const int nb = static_cast<int>(c.chunk / T);
   const TcArgs a = make_args(c, static_cast<int>((c.dims.seqlen + c.chunk - 1) / c.chunk), nb);
   if (Cf::XBUF == 0 && nb != 1) return cudaErrorInvalidValue;
   if (c.gate) {  // fused MSR epilogue: no segments, one cluster per (batch, head)
-    if constexpr (DVS == 64) return launch_fused<DK, T, Tout>(c, hp, s, mq, mk, mv, a, nb);
+    if constexpr (DVS == 64) return launch_unsplit<DK, T, Tout, false>(c, hp, s, m5, a, nb);
     return cudaErrorInvalidValue;
   }
   TcArgs as = a;
@@ -2042,7 +2209,7 @@ cudaError_t launch_pipe(const RetentionCall& c, const HeadParams& hp, cudaStream
   auto run = [&](auto kern, unsigned nx) -> cudaError_t {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM);
     if (e != cudaSuccess) return e;
-    kern<<<dim3(grid.x * nx, grid.y, grid.z), Cf::THREADS, Cf::SMEM, s>>>(mq, mk, mv, as, hp);
+    kern<<<dim3(grid.x * nx, grid.y, grid.z), Cf::THREADS, Cf::SMEM, s>>>(mq, mk, mv, mq, mk, as, hp);
     return cudaGetLastError();
   };
   if (as.n_seg < 2) {
@@ -2050,28 +2217,11 @@ cudaError_t launch_pipe(const RetentionCall& c, const HeadParams& hp, cudaStream
       // Chunks of several sub-blocks, no segments, and a workspace that holds the fp16
       // copies: convert once in a pre-pass, then run the kernel without converters.
       if (pre_convert_applies(c, nb, as.n_seg)) {
-        const PreCopies pc = pre_copies(c);
-        const int64_t tokens = c.dims.batch * c.dims.seqlen;
-        const int64_t items = tokens * (DK / 8) + tokens * c.dims.heads * (c.dims.d_v / 8);
-        const int blocks = static_cast<int>(std::min<int64_t>((items + 255) / 256, static_cast<int64_t>(sms) * 8));
-        tc_convert_kernel<DK, T><<<blocks, 256, 0, s>>>(
-            static_cast<const uint4*>(c.q), static_cast<const uint4*>(c.k), static_cast<const uint4*>(c.v),
-            static_cast<uint4*>(pc.q), static_cast<uint4*>(pc.k), static_cast<uint4*>(pc.v), tokens,
-            static_cast<int>(c.dims.seqlen), static_cast<int>(c.dims.heads), static_cast<int>(c.dims.d_v), c.pos0,
-            c.flags, hp);
-        cudaError_t e = cudaGetLastError();
+        CUtensorMap pm[5];
+        cudaError_t e = run_convert<DK, T, false>(c, hp, s, pre_copies(c), pm);
         if (e != cudaSuccess) return e;
-        RetentionCall cc = c;
-        cc.q = pc.q;
-        cc.k = pc.k;
-        cc.v = pc.v;
-        CUtensorMap pq, pk, pv;
-        if (!make_maps(cc, T, &pq, &pk, &pv)) return cudaErrorInvalidValue;
-        auto kern = tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_NONE, true, false, Tout>;
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, CfP::SMEM);
-        if (e != cudaSuccess) return e;
-        kern<<<grid, CfP::THREADS, CfP::SMEM, s>>>(pq, pk, pv, as, hp);
-        return cudaGetLastError();
+        return launch_kernel(tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_NONE, true, false, Tout>, grid, CfP::THREADS,
+                             CfP::SMEM, s, pm, as, hp, 0);
       }
     }
     return run(tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_NONE, false, false, Tout>, 1);
@@ -2114,7 +2264,7 @@ cudaError_t launch_pipe(const RetentionCall& c, const HeadParams& hp, cudaStream
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, as, hp);
+  return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mq, mk, as, hp);
 }
 
 // Serial kernel: one chunk of B = T rows per step (chunk-relative scaled operands).
@@ -2137,6 +2287,7 @@ cudaError_t launch_dk(const RetentionCall& c, const HeadParams& hp, cudaStream_t
     if (c.chunk == 64) return launch_serial<DK, 64, Tout>(c, hp, s);
     return launch_serial<DK, 128, Tout>(c, hp, s);
   }
+  if (c.precise) return launch_pipe_hl<DK, Tout>(c, hp, s);
   const int T = pipe_tile_rows(DK, c.chunk);
   if constexpr (DK != 256) {
     if (pipe_wide_slice(c, T)) return launch_pipe<DK, 64, 128, Tout>(c, hp, s);
@@ -2169,7 +2320,7 @@ bool tc_chunkwise_supported(const RetentionCall& c) {
   if (d.d_k != 64 && d.d_k != 128 && d.d_k != 256) return false;
   if (d.d_v % kDVS != 0) return false;
   if (c.chunk != 64 && c.chunk != 128 && c.chunk != 256 && c.chunk != 512) return false;
-  if (force_serial_kernel() && c.chunk > 128) return false;
+  if (force_serial_kernel() && (c.chunk > 128 || c.precise)) return false;
   if (d.seqlen < 1 || d.seqlen > (1LL << 30) || d.heads > 65535 || d.batch > 65535) return false;
   if (!aligned16(c.q) || !aligned16(c.k) || !aligned16(c.v) || !aligned16(c.o)) return false;
   if ((c.state_in && !aligned16(c.state_in)) || (c.state_out && !aligned16(c.state_out))) return false;
@@ -2193,7 +2344,7 @@ bool tc_driver_ready() { return encode_fn() != nullptr; }
 // Host-side part of the scaled-operand condition: every head keeps gamma^T >= 2^-12, where T
 // is the scaling span (the unit rows of the pipelined kernel, the whole chunk for the serial one).
 bool tc_chunkwise_heads_ok(const RetentionCall& c, const HeadParams& hp) {
-  const double span = force_serial_kernel() ? static_cast<double>(c.chunk) : pipe_tile_rows(c.dims.d_k, c.chunk);
+  const double span = force_serial_kernel() ? static_cast<double>(c.chunk) : pipe_tile_rows(c);
   for (int64_t h = 0; h < c.dims.heads; ++h)
     if (static_cast<double>(hp.log2g[h]) * span < -12.0) return false;
   return true;
@@ -2226,7 +2377,7 @@ cudaError_t launch_segment_state_t(const RetentionCall& c, const HeadParams& hp,
   auto kern = tc_chunkwise_pipe_kernel<DK, T, 64, SEG_STATE, false, false, Tout>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<tc_grid(c.dims, 64), Cf::THREADS, Cf::SMEM, s>>>(mq, mk, mv, a, hp);
+  kern<<<tc_grid(c.dims, 64), Cf::THREADS, Cf::SMEM, s>>>(mq, mk, mv, mq, mk, a, hp);
   return cudaGetLastError();
 }
 
@@ -2276,12 +2427,13 @@ int tc_chunkwise_launches(const RetentionCall& c) {
     cc.flags &= ~static_cast<uint32_t>(RETNET_F_NORM_R);
     return key_sum_launches(c.dims) + tc_chunkwise_launches(cc);
   }
-  const int T = pipe_tile_rows(c.dims.d_k, c.chunk);
-  const int dvs = pipe_wide_slice(c, T) ? 128 : 64;
+  const int T = pipe_tile_rows(c);
+  const int dvs = (!c.precise && pipe_wide_slice(c, T)) ? 128 : 64;
   const int nb = static_cast<int>(c.chunk / T);
   TcArgs as = make_args(c, static_cast<int>((c.dims.seqlen + c.chunk - 1) / c.chunk), nb);
   const int64_t ctas = (c.dims.d_v / dvs) * c.dims.heads * c.dims.batch;
-  if (c.gate) return pre_convert_applies(c, nb, 1) ? 2 : 1;  // fused epilogue: never segmented
+  // fused epilogue and split operands: never segmented
+  if (c.gate || c.precise) return pre_convert_applies(c, nb, 1) ? 2 : 1;
   const int max_states = plan_call(c, ctas, sm_count(), as);
   if (dvs == 64 && pre_convert_applies(c, nb, as.n_seg)) return 2;  // conversion pre-pass + kernel
   return (as.n_seg > 1 && max_states >= 1) ? 2 : 1;

@@ -36,6 +36,9 @@ struct RetentionCall {
   // rden_seg: the key-sum pass's segment end values, fp32 [batch * heads][<= 64][d_k].
   float* rden = nullptr;
   float* rden_seg = nullptr;
+  // Split fp16 operands (hi + lo) on the tensor-core kernel: RETNET_F_PRECISE, R~ and the fused
+  // MSR epilogue, whose normalisations magnify the operand rounding of a single fp16 copy.
+  bool precise = false;
 };
 
 // Sequence segments of the key-sum pass, at most; and the workspace bytes of the R~ factors

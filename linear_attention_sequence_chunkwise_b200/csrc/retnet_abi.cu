@@ -14,7 +14,8 @@ using namespace retnet;
 
 namespace {
 
-constexpr uint32_t kAllFlags = RETNET_F_XPOS | RETNET_F_SCALE_SQRT_D | RETNET_F_NORM_D | RETNET_F_NORM_R;
+constexpr uint32_t kAllFlags =
+    RETNET_F_XPOS | RETNET_F_SCALE_SQRT_D | RETNET_F_NORM_D | RETNET_F_NORM_R | RETNET_F_PRECISE;
 
 bool valid_dtype(retnet_dtype_t t) { return t == RETNET_F32 || t == RETNET_BF16; }
 
@@ -140,6 +141,7 @@ retnet_status_t chunkwise_impl(const void* q, const void* k, const void* v, void
   c.ws = workspace;
   c.ws_bytes = workspace ? workspace_bytes : 0;
   carve_rden(c);
+  c.precise = (flags & RETNET_F_PRECISE) || c.rden || gate;
   if (gate) {
     // Fused MSR epilogue: the tensor-core kernel only, decided on the host before any launch.
     c.gate = gate;
@@ -197,8 +199,9 @@ retnet_status_t retnet_msr_chunkwise(const void* q, const void* k, const void* v
                                      void* workspace, size_t workspace_bytes, void* stream) {
   if (!(eps >= 0.f) || !isfinite(eps)) return RETNET_ERR_BAD_PARAM;
   if (dims.seqlen > 0 && !g) return RETNET_ERR_NULL_PTR;
-  if (flags & RETNET_F_NORM_R) return RETNET_ERR_UNSUPPORTED;
   // (without tokens nothing reads g: the call only passes the state through)
+  // R~ needs its row factors in the workspace (a too small one is caught before the launch)
+  if ((flags & RETNET_F_NORM_R) && dims.seqlen > 0 && !workspace) return RETNET_ERR_UNSUPPORTED;
   return chunkwise_impl(q, k, v, out, dims, in_dtype, out_dtype, gamma, theta, pos0, flags, chunk, state_in,
                         state_out, nullptr, nullptr, workspace, workspace_bytes, stream, g, eps);
 }
@@ -259,12 +262,13 @@ retnet_status_t retnet_chunkwise_workspace_size(retnet_dims_t dims, size_t* byte
   if (!bytes) return RETNET_ERR_NULL_PTR;
   if (dims.batch < 0 || dims.seqlen < 0 || dims.heads < 0 || dims.d_k < 0 || dims.d_v < 0) return RETNET_ERR_BAD_SHAPE;
   // The larger of its two uses (never both in one call): up to six segment states, fp32
-  // [6][batch][heads][d_k][d_v]; or the fp16 copies of q, k, v of the conversion pre-pass.
+  // [6][batch][heads][d_k][d_v]; or the fp16 copies of q, k, v of the conversion pre-pass, with
+  // the lo parts of q and k for split operands.
   const size_t states = 6 * sizeof(float) * static_cast<size_t>(dims.batch) * static_cast<size_t>(dims.heads) *
                         static_cast<size_t>(dims.d_k) * static_cast<size_t>(dims.d_v);
   const size_t tok = static_cast<size_t>(dims.batch) * static_cast<size_t>(dims.seqlen) * static_cast<size_t>(dims.heads);
   auto a256 = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
-  const size_t copies = 2 * a256(tok * static_cast<size_t>(dims.d_k) * 2) + a256(tok * static_cast<size_t>(dims.d_v) * 2);
+  const size_t copies = 4 * a256(tok * static_cast<size_t>(dims.d_k) * 2) + a256(tok * static_cast<size_t>(dims.d_v) * 2);
   // plus, in front, the R~ row factors (fp32 [batch][seqlen][heads]) and the key-sum pass's
   // segment values (fp32 [batch * heads][64][d_k])
   const Dims d{dims.batch, dims.seqlen, dims.heads, dims.d_k, dims.d_v};
@@ -332,17 +336,20 @@ int retnet_chunkwise_launches(retnet_dims_t dims, retnet_dtype_t in_dtype, uint3
   c.ws = workspace_bytes ? reinterpret_cast<void*>(static_cast<uintptr_t>(256)) : nullptr;  // only its size matters
   c.ws_bytes = workspace_bytes;
   carve_rden(c);
+  c.precise = (flags & RETNET_F_PRECISE) || c.rden;
   if (!tc_chunkwise_supported(c)) return 1;  // R~ without room for its factors: the CUDA-core kernel
   return tc_chunkwise_launches(c);
 }
 
 int retnet_msr_chunkwise_launches(retnet_dims_t dims, retnet_dtype_t in_dtype, uint32_t flags, int64_t chunk,
                                   const float* gamma, size_t workspace_bytes) {
-  if (flags & RETNET_F_NORM_R) return -static_cast<int>(RETNET_ERR_UNSUPPORTED);
-  const int path = retnet_chunkwise_kernel(dims, in_dtype, flags, chunk, gamma);
+  const int path = retnet_chunkwise_kernel(dims, in_dtype, flags & ~static_cast<uint32_t>(RETNET_F_NORM_R), chunk,
+                                           gamma);
   if (path < 0) return path;
   if (dims.seqlen == 0) return 0;
   if (path == 0) return -static_cast<int>(RETNET_ERR_UNSUPPORTED);
+  const Dims dd{dims.batch, dims.seqlen, dims.heads, dims.d_k, dims.d_v};
+  if ((flags & RETNET_F_NORM_R) && workspace_bytes < rden_region_bytes(dd)) return -static_cast<int>(RETNET_ERR_UNSUPPORTED);
   const retnet_status_t st = check_device();
   if (st != RETNET_OK) return -static_cast<int>(st);
   alignas(16) static const uint32_t kAligned[4] = {0, 0, 0, 0};
@@ -351,7 +358,9 @@ int retnet_msr_chunkwise_launches(retnet_dims_t dims, retnet_dtype_t in_dtype, u
                   chunk, true, nullptr, nullptr, nullptr, nullptr};
   c.ws = workspace_bytes ? reinterpret_cast<void*>(static_cast<uintptr_t>(256)) : nullptr;  // only its size matters
   c.ws_bytes = workspace_bytes;
+  carve_rden(c);
   c.gate = kAligned;
+  c.precise = true;
   if (!tc_fused_supported(c)) return -static_cast<int>(RETNET_ERR_UNSUPPORTED);
   return tc_chunkwise_launches(c);
 }
@@ -369,6 +378,7 @@ int retnet_chunkwise_kernel(retnet_dims_t dims, retnet_dtype_t in_dtype, uint32_
   RetentionCall c{kAligned, kAligned, kAligned, const_cast<uint32_t*>(kAligned),
                   Dims{dims.batch, dims.seqlen, dims.heads, dims.d_k, dims.d_v}, in_dtype, RETNET_F32, 0, flags,
                   chunk, true, nullptr, nullptr, nullptr, nullptr};
+  c.precise = (flags & (RETNET_F_PRECISE | RETNET_F_NORM_R)) != 0;
   return (tc_chunkwise_supported(c) && tc_chunkwise_heads_ok(c, hp)) ? 1 : 0;
 }
 

@@ -84,7 +84,7 @@ def test_parallel_validation(lib):
     assert _par(lib, ok, _gamma(2, 1.0)) == 4                            # gamma = 1
     assert _par(lib, ok, _gamma(2, 0.0)) == 4                            # gamma = 0
     assert _par(lib, ok, np.array([0.9, np.nan], np.float32)) == 4       # gamma NaN
-    assert _par(lib, ok, _gamma(2), flags=16) == 4                       # unknown flag bit
+    assert _par(lib, ok, _gamma(2), flags=32) == 4                       # unknown flag bit
     assert _par(lib, (1, 8, 2, 5, 4), _gamma(2), np.ones(2), flags=rn.F_XPOS) == 4  # odd d_k with xPos
     assert _par(lib, ok, _gamma(2), None, flags=rn.F_XPOS) == 1          # xPos without theta
     assert _par(lib, ok, _gamma(2), np.array([1.0, np.inf]), flags=rn.F_XPOS) == 4  # theta inf
@@ -123,7 +123,7 @@ def test_chunkwise_workspace_entry_points(lib):
     for dims in ((2, 100, 3, 128, 64), (1, 4096, 2, 64, 128)):
         b, L, h, dk, dv = dims
         states = 6 * b * h * dk * dv * 4
-        copies = 2 * a256(b * L * h * dk * 2) + a256(b * L * h * dv * 2)
+        copies = 4 * a256(b * L * h * dk * 2) + a256(b * L * h * dv * 2)  # q~, k~ hi and lo; v
         rden = a256(b * L * h * 4) + a256(b * h * dk * 64 * 4)  # R~ row factors and key-sum segments, in front
         assert rn.retnet_chunkwise_workspace_size(dims) == rden + max(states, copies)
     assert rn.retnet_chunkwise_workspace_size((0, 0, 0, 0, 0)) == 0
@@ -167,7 +167,8 @@ def test_epilogue_validation(lib):
 
 
 def test_fused_msr_validation(lib):
-    """The fused MSR entry point checks eps, the gate pointer and the norm-R flag on the host."""
+    """The fused MSR entry point checks eps, the gate pointer and, for R~, that there is a
+    workspace for the row factors, on the host."""
     g = _gamma(2)
     gp = g.ctypes.data_as(rn._fp)
     d = rn.Dims(1, 64, 2, 128, 128)

@@ -2,16 +2,13 @@
 tensor-core kernel, the d_v slices of a head in one thread-block cluster) against the fp64
 oracle: oracle.msr_epilogue of the oracle's retention output.
 
-Bar: the retention output's own bar (max|dy|/rms(y) <= 1e-2 with bf16 inputs) carried through
-the row normalisation and the gate (gpu_util.err_msr: the GroupNorm divides each row's error by
-the row's deviation and the gate multiplies it by |swish(g)|), net of a bf16 output's own
-rounding.  The plain max|err|/rms(out) is printed too and held to 2e-2: it is at most 7.9e-3
-on these cases except (d_k 256, d_v 128, chunk 128, L 129) at 1.5e-2, where rows of few
-tokens (small deviation) meet large gates; the two-kernel form gives the same figure, and an
-fp64 emulation of the kernel's operand roundings puts most of it on the fp16 rounding of the
-scaled, rotated q and k.  The state hand-off is held to the chunkwise bar directly.
+Bar: the plain max|err|/rms(out) <= 1e-2 of bf16 inputs on the post-epilogue output (net of a
+bf16 output's own rounding).  The GroupNorm divides each row by its own deviation, so a row of
+few tokens whose scores nearly cancel magnifies the operand rounding of the retention output;
+the fused kernel therefore always runs with split fp16 operands (hi + lo, about 22 significant
+bits), which keeps the post-epilogue error near the fp32 level.  gpu_util.err_msr (the
+retention bar carried through the normalisation) is printed beside it.
 """
-TOL_OUT = 2e-2
 import numpy as np
 import pytest
 import torch
@@ -19,7 +16,7 @@ import torch
 import linear_attention_sequence_chunkwise_b200 as rn
 import oracle
 import synth_inputs as si
-from gpu_util import TOL_BF16, dev, err, err_msr, require_gpu
+from gpu_util import TOL_BF16, dev, err, err_bf16_out, err_msr, require_gpu
 
 pytestmark = pytest.mark.gpu
 FLAGS = rn.F_XPOS | rn.F_SCALE_SQRT_D | rn.F_NORM_D
@@ -76,8 +73,7 @@ def test_fused_msr_matches_oracle(dk, dv, B, L, workspace):
     e = err_msr(out, ref, y, gt, h, EPS)
     e_out = err(out, ref)
     print(f"dk={dk} dv={dv} B={B} L={L} ws={workspace} launches={n}: msr err {e:.3e}, max|err|/rms {e_out:.3e}")
-    assert e <= TOL_BF16
-    assert e_out <= TOL_OUT
+    assert e_out <= TOL_BF16
     assert err(so, Sref) <= TOL_BF16
 
 
@@ -91,13 +87,15 @@ def test_fused_msr_bf16_out_state_in_pos0():
     pos0 = (1 << 20) + 77
     ref, y, Sref = reference(q, k, v, gt, g, th, B, pos0=pos0, state_in=S0)
     out, so, _ = fused(q, k, v, gt, g, th, B, pos0=pos0, state_in=S0, want_state=True, out_dtype=torch.bfloat16)
-    assert err_msr(out, ref, y, gt, h, EPS, bf16_out=True) <= TOL_BF16
+    e = err_bf16_out(out, ref)
+    print(f"bf16 out, state in, pos0 {pos0}: max|err|/rms net of bf16 rounding {e:.3e}")
+    assert e <= TOL_BF16
     assert err(so, Sref) <= TOL_BF16
 
 
 def test_fused_no_worse_than_two_kernel_path():
-    """The fused kernel and chunkwise + retnet_msr_epilogue (fp32 between them) against the
-    oracle: fusing the epilogue loses no accuracy."""
+    """The fused kernel and chunkwise (split operands) + retnet_msr_epilogue (fp32 between them)
+    against the oracle: fusing the epilogue loses no accuracy."""
     b, L, h, dk, dv, B = 2, 700, 4, 128, 256, 128
     q, k, v = si.qkv(b, L, h, dk, dv, 401, "bf16")
     gt = gate(b, L, h, dv, 402)
@@ -105,20 +103,45 @@ def test_fused_no_worse_than_two_kernel_path():
     ref, y_ref, _ = reference(q, k, v, gt, g, th, B)
     out, _, _ = fused(q, k, v, gt, g, th, B)
     y = torch.empty(b, L, h, dv, device="cuda")
-    rn.retnet_retention_chunkwise(dev(q), dev(k), dev(v), y, g, th, 0, FLAGS, B)
+    rn.retnet_retention_chunkwise(dev(q), dev(k), dev(v), y, g, th, 0, FLAGS | rn.F_PRECISE, B)
     two = torch.empty_like(y)
     rn.retnet_msr_epilogue(y, dev(gt).float(), two, h, EPS)  # y and g share one dtype
     torch.cuda.synchronize()
-    e_fused, e_two = err_msr(out, ref, y_ref, gt, h, EPS), err_msr(two, ref, y_ref, gt, h, EPS)
+    e_fused, e_two = err(out, ref), err(two, ref)
     print(f"fused {e_fused:.3e}, two kernels {e_two:.3e}")
     assert e_fused <= TOL_BF16 and e_two <= TOL_BF16
-    assert e_fused <= 1.5 * e_two + 1e-3
+    assert e_fused <= 1.5 * e_two + 1e-4
+
+
+@pytest.mark.parametrize("dk,dv,B,L", [(128, 128, 64, 300), (256, 256, 256, 520)])
+def test_fused_msr_with_norm_r(dk, dv, B, L):
+    """R~ (§三.3) before the GroupNorm: the key-sum pass writes the row factors into the
+    workspace, the fused kernel folds them into its row scale (the GroupNorm then sees each row
+    divided by max(|row sum|, 1), which changes the result only through eps)."""
+    b, h = 2, 3
+    q, k, v = si.qkv(b, L, h, dk, dv, 500 + dk + B, "bf16")
+    q = (q.float() + 0.5).to(q.dtype)  # most row sums exceed 1: the normalisation is active
+    k = (k.float() + 0.5).to(k.dtype)
+    gt = gate(b, L, h, dv, 501)
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+    flags = FLAGS | rn.F_NORM_R
+    y, _, _ = oracle.chunkwise(q, k, v, g, B, th, 0, flags)
+    ref = oracle.msr_epilogue(y, gt, h, eps=EPS)
+    ws = torch.empty(rn.retnet_chunkwise_workspace_size((b, L, h, dk, dv)), dtype=torch.uint8, device="cuda")
+    n = rn.retnet_msr_chunkwise_launches((b, L, h, dk), dv, rn.BF16, flags, B, g, ws.numel())
+    assert n >= 2, n  # the key-sum pass, then the fused kernel (after the conversion pre-pass)
+    out = torch.empty(b, L, h, dv, device="cuda")
+    rn.retnet_msr_chunkwise(dev(q), dev(k), dev(v), dev(gt), out, g, th, 0, flags, B, EPS, workspace=ws)
+    torch.cuda.synchronize()
+    e = err(out, ref)
+    print(f"fused MSR with R~ dk={dk} dv={dv} B={B} L={L} launches={n}: max|err|/rms {e:.3e}")
+    assert e <= TOL_BF16
 
 
 def test_fused_unsupported_shapes_are_rejected():
     b, L, h, dk = 1, 64, 2, 128
     g, th = si.gamma_schedule(h), si.theta_schedule(dk)
-    # d_v = 320 needs five CTAs a cluster; the norm-R flag has no tensor-core path
+    # d_v = 320 needs five CTAs a cluster; R~ needs a workspace for its row factors
     for dv, flags in ((320, FLAGS), (128, FLAGS | rn.F_NORM_R)):
         assert rn.retnet_msr_chunkwise_launches((b, L, h, dk), dv, rn.BF16, flags, 64, g) == -5
         q, k, v = si.qkv(b, L, h, dk, dv, 5, "bf16")

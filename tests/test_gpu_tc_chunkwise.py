@@ -308,12 +308,13 @@ def test_tc_norm_r_matches_oracle(dk, dv, B, L, pos0, bias, with_state):
     state and z against the oracle; q and k carry a mean (bias) so that most rows' sums exceed
     1 and the normalisation is active.
 
-    Bar: R~ divides each row by its own D_n = max(|sum of scores|, 1) >= 1, which leaves rows of
-    very different sizes (early rows keep D ~ 1, later ones are divided by tens), so max|err| /
-    rms over the normalised output weighs an early row's ordinary error by the shrunken rms of
-    the rest.  The bf16 bar is applied to the output scaled back by the oracle's D_n
-    (out * D_n against the oracle's output without R~, which is ref * D_n exactly); a wrong
-    row factor on the GPU shows there as its relative error.  The plain figure is printed."""
+    Bar: the plain max|err|/rms <= 1e-2 on the R~-normalised output.  R~ divides each row by
+    its own D_n = max(|sum of scores|, 1), which leaves rows of very different sizes (early rows
+    keep D ~ 1, later ones are divided by tens), so the rms over the normalised output is small
+    against the early rows' values; R~ calls therefore run with split fp16 operands (hi + lo).
+    The output scaled back by the oracle's D_n (against the oracle's output without R~, which
+    is ref * D_n exactly) is printed and held to the same bar: a wrong row factor on the GPU
+    shows there as its relative error."""
     b, h = 2, 3
     q, k, v = si.qkv(b, L, h, dk, dv, 900 + dk + B, "bf16")
     q = (q.float() + bias).to(q.dtype)
@@ -342,8 +343,10 @@ def test_tc_norm_r_matches_oracle(dk, dv, B, L, pos0, bias, with_state):
                                      workspace=ws)
     torch.cuda.synchronize()
     e = err(o.cpu().double().numpy() * D, plain)
-    print(f"R~ dk={dk} dv={dv} B={B} L={L} launches={n}: rescaled max|err|/rms = {e:.3e}, "
-          f"plain {err(o, ref):.3e}")
+    e_plain = err(o, ref)
+    print(f"R~ dk={dk} dv={dv} B={B} L={L} launches={n}: plain max|err|/rms = {e_plain:.3e}, "
+          f"rescaled {e:.3e}")
+    assert e_plain <= TOL_BF16
     assert e <= TOL_BF16
     assert err(so, Sref) <= TOL_BF16
     assert err(zo, zref) <= TOL_F32
