@@ -11,9 +11,12 @@ Alongside the step (1 GPU only), the same line carries: the decode step on the w
 "batch 64, h 16, d_k 256, d_v 512, fp32 state" (state GB/s), and, where enabled, the
 long-sequence and MSR workloads.  --impl reference times the fp64 CPU oracle instead.
 
-Multi-GPU (torchrun, one process per GPU): every rank runs its own batch (weak scaling);
-the path has no exchange step, so the only collectives are the barrier and the max of the
-timed durations.
+Multi-GPU (one process per GPU): every rank runs its own batch (weak scaling); the path has no
+exchange step, so the only collectives of the timed step are the barrier and the max of the
+timed durations.  `--gpus N` without a torchrun environment relaunches this script under
+torch.distributed.run with N processes; a run whose world size differs from --gpus fails.  The
+sequence-sharded leg (`seqshard`) runs one long sequence cut into one shard per rank, whose
+states cross ranks in one all-gather (the path's only real exchange).
 """
 import argparse
 import json
@@ -199,26 +202,27 @@ def bench_decode(rn, device, stream, steps, warmup, peaks):
     c = DECODE
     b, h, dk, dv = c["batch"], c["heads"], c["d_k"], c["d_v"]
     S = si.decode_state(b, h, dk, dv, 4).to(device)
-    toks = []
-    for t in range(16):
+    toks = []  # new q, k, v for every step, as the workload states (the same draws as the parity test)
+    for t in range(steps + warmup):
         q, k, v = si.decode_token(b, h, dk, dv, 4, t)
         toks.append((q.to(device), k.to(device), v.to(device)))
     o = torch.empty(b, h, dv, device=device)
     g, th = si.gamma_schedule(h), si.theta_schedule(dk)
 
     def step(i):
-        q, k, v = toks[i % len(toks)]
+        q, k, v = toks[i]
         rn.retnet_retention_step(q, k, v, o, S, g, th, i, FLAGS, None, stream)
 
     for i in range(warmup):
         step(i)
     torch.cuda.synchronize()
-    secs = time_steps(step, steps, stream)
+    secs = time_steps(lambda i: step(warmup + i), steps, stream)
     per = secs / steps
     state_bytes = 2 * b * h * dk * dv * 4
     io_bytes = b * h * (2 * dk + dv) * 2 + b * h * dv * 4
     gbs = (state_bytes + io_bytes) / per / 1e9
-    return {"workload": c["workload"], "steps": steps, "us_per_step": per * 1e6,
+    return {"workload": c["workload"], "steps": steps, "positions": f"{warmup}..{warmup + steps - 1}",
+            "us_per_step": per * 1e6,
             "bytes_per_step": state_bytes + io_bytes, "gbs": gbs, "frac_of_measured_hbm": gbs / peaks["hbm"],
             "frac_of_8tbs": gbs / 8000.0, "gpu_launches": steps,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s",
@@ -263,7 +267,8 @@ def bench_long(rn, device, stream, steps, peaks):
 def bench_msr(rn, device, stream, steps, peaks):
     """MSR forward (chunk 256, bf16 out): the fused kernel (retention, GroupNorm and swish gate
     in one tensor-core kernel per cluster of d_v slices), and beside it the two-kernel form
-    (chunkwise retention to HBM, then the GroupNorm + gate kernel)."""
+    (chunkwise retention to HBM, then the GroupNorm + gate kernel).  Both with split fp16
+    operands, which the post-epilogue accuracy needs."""
     import torch
 
     import synth_inputs as si
@@ -275,13 +280,14 @@ def bench_msr(rn, device, stream, steps, peaks):
     y = torch.empty(b, L, h, dv, dtype=torch.bfloat16, device=device)
     out = torch.empty(b, L, h * dv, dtype=torch.bfloat16, device=device)
     g, th = si.gamma_schedule(h), si.theta_schedule(dk)
-    path = rn.retnet_chunkwise_kernel((b, L, h, dk), dv, rn.BF16, FLAGS, B, g)
+    path = rn.retnet_chunkwise_kernel((b, L, h, dk), dv, rn.BF16, FLAGS | rn.F_PRECISE, B, g)
     ws = torch.empty(rn.retnet_chunkwise_workspace_size((b, L, h, dk, dv)), dtype=torch.uint8, device=device)
-    two_launches = rn.retnet_chunkwise_launches((b, L, h, dk), dv, rn.BF16, FLAGS, B, g, ws.numel()) + 1
+    two_launches = rn.retnet_chunkwise_launches((b, L, h, dk), dv, rn.BF16, FLAGS | rn.F_PRECISE, B, g,
+                                                ws.numel()) + 1
     fused_launches = rn.retnet_msr_chunkwise_launches((b, L, h, dk), dv, rn.BF16, FLAGS, B, g, ws.numel())
 
     def two_kernel(i):
-        rn.retnet_retention_chunkwise_ws(q, k, v, y, g, th, 0, FLAGS, B, workspace=ws, stream=stream)
+        rn.retnet_retention_chunkwise_ws(q, k, v, y, g, th, 0, FLAGS | rn.F_PRECISE, B, workspace=ws, stream=stream)
         rn.retnet_msr_epilogue(y.view(b, L, h * dv), gt, out, h, 1e-5, stream)
 
     def fused(i):
@@ -290,10 +296,10 @@ def bench_msr(rn, device, stream, steps, peaks):
 
     flops = b * L * h * flops_per_token_head(dk, dv, B)
     res = {"workload": c["workload"], "workspace_bytes": ws.numel()}
-    legs = [("two_kernel", two_kernel, two_launches, 4 * dv, "tcgen05 + epilogue" if path == 1 else
+    legs = [("two_kernel", two_kernel, two_launches, 4 * dv, "tcgen05 split operands + epilogue" if path == 1 else
              "fp32 CUDA cores + epilogue")]
     if fused_launches > 0:
-        legs.insert(0, ("fused", fused, fused_launches, 2 * dv, "tcgen05, fused GroupNorm + gate"))
+        legs.insert(0, ("fused", fused, fused_launches, 2 * dv, "tcgen05 split operands, fused GroupNorm + gate"))
     for name, fn, launches, extra, kernel in legs:
         for i in range(2):
             fn(i)
@@ -339,6 +345,70 @@ def bench_backward(rn, device, stream, steps, peaks):
             "tflops": tf, "frac_bf16_peak": tf / peaks["bf16"],
             "kernel": "tcgen05 (three chunkwise runs, hi|lo values)" if path == 1 else "fp32 CUDA cores",
             "workspace_bytes": ws.numel(), "launches_per_step": launches, "gpu_launches": launches * steps}
+
+
+def bench_flag_variants(rn, device, stream, steps, peaks, ws):
+    """The headline workload with R~ (key-sum pass + split operands) and with split operands
+    alone (RETNET_F_PRECISE), beside the timed step's single-copy operands."""
+    import torch
+
+    import synth_inputs as si
+    c = MAIN
+    b, L, h, dk, dv, B = c["batch"], c["seqlen"], c["heads"], c["d_k"], c["d_v"], c["chunk"]
+    q, k, v = si.qkv(b, L, h, dk, dv, 2, "bf16")
+    q, k, v = q.to(device), k.to(device), v.to(device)
+    o = torch.empty(b, L, h, dv, dtype=torch.bfloat16, device=device)
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+    out = {"workload": c["workload"]}
+    byt = b * L * h * bytes_per_token_head(dk, dv)
+    for name, fl in (("norm_r", FLAGS | rn.F_NORM_R), ("precise", FLAGS | rn.F_PRECISE)):
+        launches = rn.retnet_chunkwise_launches((b, L, h, dk), dv, rn.BF16, fl, B, g, ws.numel())
+
+        def step(i):
+            rn.retnet_retention_chunkwise_ws(q, k, v, o, g, th, 0, fl, B, workspace=ws, stream=stream)
+
+        for i in range(3):
+            step(i)
+        torch.cuda.synchronize()
+        secs = time_steps(step, steps, stream) / steps
+        out[name] = {"us_per_step": secs * 1e6, "tokens_per_s": b * L / secs, "gbs": byt / secs / 1e9,
+                     "frac_hbm": byt / secs / 1e9 / peaks["hbm"], "launches_per_step": launches,
+                     "gpu_launches": launches * steps}
+    return out
+
+
+def bench_seqshard(rn, device, stream, steps, world, rank):
+    """One long sequence (b2 / L8192 / h16 / d_k 256 / d_v 512, chunk 128) cut into one shard
+    per rank: each rank computes its shard's state, the states are all-gathered (NCCL), each
+    rank folds the earlier ones into its start state and runs its shard (strong scaling: the
+    sequence is fixed).  Timed on the device, max over ranks."""
+    import torch
+
+    import synth_inputs as si
+    from linear_attention_sequence_chunkwise_b200 import seqshard
+    c = LONG
+    b, L, h, dk, dv, B = c["batch"], c["seqlen"], c["heads"], c["d_k"], c["d_v"], 128
+    Ls = L // world
+    q, k, v = si.qkv(b, Ls, h, dk, dv, 3 + 100 * rank, "bf16")
+    q, k, v = q.to(device), k.to(device), v.to(device)
+    o = torch.empty(b, Ls, h, dv, dtype=torch.bfloat16, device=device)
+    so = torch.empty(b, h, dk, dv, dtype=torch.float32, device=device)
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+
+    def step(i):
+        seqshard.retention_chunkwise_sharded(q, k, v, o, g, th, 0, FLAGS, B, state_out=so)
+
+    for i in range(3):
+        step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    secs = max_over_ranks(time_steps(step, steps, stream), world, device) / steps
+    return {"workload": f"seqshard_{c['workload']}_B{B}", "shards": world, "tokens_per_shard": Ls,
+            "us_per_step": secs * 1e6, "tokens_per_s": b * L / secs, "scaling": "strong",
+            "exchange": "one all-gather of b*h*d_k*d_v fp32 per rank (NCCL)",
+            # segment-state pass, one state advance per earlier shard, the shard's chunkwise call
+            "gpu_launches_per_rank_step": 1 + rank + rn.retnet_chunkwise_launches((b, Ls, h, dk), dv, rn.BF16, FLAGS,
+                                                                                 B, g, 0)}
 
 
 def oracle_sample(cfg, budget_s):
@@ -486,6 +556,19 @@ def main_ours(args):
         line["msr"] = bench_msr(rn, device, stream, 10, peaks)
     if world == 1 and "backward" in args.sections:
         line["backward"] = bench_backward(rn, device, stream, 3, peaks)
+    if world == 1 and "variants" in args.sections:
+        line["variants"] = bench_flag_variants(rn, device, stream, 20, peaks, ws)
+    if "seqshard" in args.sections:
+        import datetime
+
+        import torch.distributed as dist
+        own_group = not dist.is_initialized()
+        if own_group:  # one rank: a one-member NCCL group carries the (trivial) all-gather
+            dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0, world_size=1,
+                                    timeout=datetime.timedelta(seconds=120), device_id=device)
+        line["seqshard"] = bench_seqshard(rn, device, stream, 5, world, rank)
+        if own_group:
+            dist.destroy_process_group()
     clocks.stop()
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, args.cpu_seconds)
@@ -520,15 +603,55 @@ def main_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def _free_port():
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def relaunch(n):
+    """Run this script under torch.distributed.run with n processes (one per GPU); returns its
+    exit status.  Rank 0's JSON line reaches stdout through the launcher."""
+    import subprocess
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={_free_port()}", os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
+def main_stub(args):
+    """Launch plumbing only (no GPU, no kernels, nothing timed): every rank joins a gloo group,
+    the ranks are counted with an all-reduce, and rank 0 prints the count.  Used by the CPU
+    tests of the multi-process launch."""
+    world, rank, _ = dist_env()
+    seen = 1
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+        t = torch.ones(1)
+        dist.all_reduce(t)
+        seen = int(t.item())
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps({"stub": True, "n_gpus": world, "ranks_seen": seen, "value": None}), flush=True)
+
+
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--sections", default="e2e,decode,long,msr,backward",
-                    help="comma list of extra legs to run beside the timed step: e2e, decode, long, msr, backward")
-    ap.add_argument("--decode-steps", type=int, default=200)
+    ap.add_argument("--sections", default="e2e,decode,long,msr,backward,variants,seqshard",
+                    help="comma list of extra legs to run beside the timed step: e2e, decode, long, msr, backward, "
+                         "variants, seqshard")
+    ap.add_argument("--decode-steps", type=int, default=1024)
+    ap.add_argument("--stub", action="store_true",
+                    help="check the multi-process launch only (CPU, gloo): print the rank count, run no kernels")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     a = ap.parse_args(argv)
@@ -539,7 +662,15 @@ def parse_args(argv=None):
 
 if __name__ == "__main__":
     args = parse_args()
-    if args.impl == "reference":
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(relaunch(args.gpus))
+    if int(os.environ.get("WORLD_SIZE", "1")) != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but the launcher started {os.environ.get('WORLD_SIZE', '1')} ranks",
+              file=sys.stderr)
+        sys.exit(2)
+    if args.stub:
+        main_stub(args)
+    elif args.impl == "reference":
         main_reference(args)
     else:
         main_ours(args)

@@ -213,8 +213,14 @@ RETNET_API retnet_status_t retnet_state_advance(float* state, const float* w, in
  *   Concurrency: the scratch is shared by every call on a device, so calls whose work
  *   overlaps on the GPU (two streams, two host threads) race on it and give wrong results;
  *   order them on the device.
- *   Set-up: the first call on each device looks up the scratch's address (a CUDA symbol
- *   query, made with that device current); make that first call outside any stream capture.
+ *   R~: with RETNET_F_NORM_R the row factors and the key-sum values (the front region that
+ *   retnet_chunkwise_workspace_size describes) take the front of the scratch when they fit,
+ *   and R~ then runs on the tensor-core kernel; when they do not fit, the call runs on the
+ *   fp32 CUDA-core kernel (retnet_chunkwise_launches with RETNET_STATIC_SCRATCH_BYTES tells).
+ *   Set-up: every call looks up the scratch's address in the current device's context (a
+ *   host-side CUDA symbol query, nothing cached, so a device reset leaves no stale address);
+ *   the first call on a device may load the library's module there, so make it outside any
+ *   stream capture.
  * Other arguments, results and errors as retnet_retention_chunkwise.
  */
 #define RETNET_STATIC_SCRATCH_BYTES (16u << 20)

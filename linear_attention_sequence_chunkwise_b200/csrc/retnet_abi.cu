@@ -2,11 +2,12 @@
 //
 // Each entry point checks its arguments on the host, fills the per-head parameter block
 // (gamma, log2 gamma, theta) from the caller's host arrays, and enqueues the kernels on the
-// caller's stream.  Nothing is allocated; no state survives the call.
+// caller's stream.  Nothing is allocated.  Device state that outlives a call: the count of
+// bounded waits that gave up (read by retnet_debug_wait_timeouts) and the static scratch of
+// retnet_retention_chunkwise_static (one array per device, below).
 #include <math.h>
 
 #include <algorithm>
-#include <atomic>
 
 #include "launch.h"
 
@@ -216,24 +217,13 @@ retnet_status_t retnet_msr_chunkwise(const void* q, const void* k, const void* v
 static __device__ __align__(256) unsigned char g_chunkwise_scratch[RETNET_STATIC_SCRATCH_BYTES];
 
 namespace {
-// Device address of the scratch on the current device, looked up (cudaGetSymbolAddress, with
-// that device current) on the first call per device and cached.
-constexpr int kMaxDevices = 64;
-std::atomic<void*> g_scratch_addr[kMaxDevices];
-
+// Device address of the scratch in the current device's context.  Host code cannot use the
+// array's name as a device address, so every call asks the runtime (cudaGetSymbolAddress, a
+// host-side query, with the calling thread's device current); nothing is cached, so a device
+// reset or a recreated context never leaves a stale address behind.
 retnet_status_t static_scratch(void** ptr) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return RETNET_ERR_CUDA;
-  if (dev >= 0 && dev < kMaxDevices) {
-    void* p = g_scratch_addr[dev].load(std::memory_order_acquire);
-    if (p) {
-      *ptr = p;
-      return RETNET_OK;
-    }
-  }
   void* p = nullptr;
   if (cudaGetSymbolAddress(&p, g_chunkwise_scratch) != cudaSuccess || !p) return RETNET_ERR_CUDA;
-  if (dev >= 0 && dev < kMaxDevices) g_scratch_addr[dev].store(p, std::memory_order_release);
   *ptr = p;
   return RETNET_OK;
 }

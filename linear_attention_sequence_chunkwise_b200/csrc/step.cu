@@ -171,10 +171,10 @@ cudaError_t launch_typed(const StepCall& c, const HeadParams& hp, cudaStream_t s
   a.heads = c.heads;
   a.pos = c.pos;
   a.flags = c.flags;
+  // at most 4 * (2 * 512 + 8 * 128 + 2) = 8200 bytes (d_k <= RETNET_MAX_DK): within the default
+  // 48 KB of dynamic shared memory, so no per-launch attribute call is needed
   const size_t smem = sizeof(float) * (size_t)(2 * c.d_k + kWarps * kColsPerPass + 2);
-  cudaError_t e = cudaFuncSetAttribute(step_kernel<Tin, Tout>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
+  static_assert(sizeof(float) * (2 * RETNET_MAX_DK + kWarps * kColsPerPass + 2) <= 48 * 1024, "step smem");
   const int64_t blocks = c.batch * c.heads;
   step_kernel<Tin, Tout><<<static_cast<unsigned>(blocks), kThreads, smem, s>>>(a, hp);
   return cudaGetLastError();

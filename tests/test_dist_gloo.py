@@ -1,9 +1,10 @@
 """Multi-process host logic of bench.py on CPU (gloo, world size 2, 127.0.0.1).
 
-The retention path shards by batch with no exchange step, so the only collectives the
-benchmark uses are a barrier and the MAX of the per-rank timings; the reference arm runs
-on rank 0 only.  These run here without a GPU.
+The retention path shards by batch with no exchange step, so the only collectives the timed
+step uses are a barrier and the MAX of the per-rank timings; the reference arm runs on rank 0
+only; `--gpus N` starts N ranks.  These run here without a GPU.
 """
+import json
 import os
 import socket
 import subprocess
@@ -58,6 +59,33 @@ def test_max_over_ranks_and_rank_local_inputs():
 
 def test_reference_arm_runs_on_rank0_only():
     env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
-    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
-                        "--warmup", "0"], env=env, capture_output=True, text=True, timeout=300)
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--impl", "reference",
+                        "--steps", "1", "--warmup", "0"], env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def _clean_env():
+    env = dict(os.environ)
+    for key in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT", "LOCAL_WORLD_SIZE"):
+        env.pop(key, None)
+    return env
+
+
+def test_gpus_flag_starts_that_many_ranks():
+    """`bench.py --gpus 2` outside torchrun relaunches itself with two processes; the stub leg
+    (launch plumbing only, gloo on CPU) counts the ranks that joined and rank 0 reports them."""
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--stub", "--steps", "1",
+                        "--warmup", "3"], env=_clean_env(), capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    rec = json.loads(lines[0])
+    assert rec["n_gpus"] == 2 and rec["ranks_seen"] == 2 and rec["value"] is None
+
+
+def test_rank_count_mismatch_fails_loudly():
+    """A launcher that starts fewer ranks than --gpus asks for is an error, not a 1-GPU number."""
+    env = dict(_clean_env(), RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--stub"], env=env,
+                       capture_output=True, text=True, timeout=120)
+    assert r.returncode == 2 and "--gpus 2" in r.stderr

@@ -21,6 +21,9 @@ FLAGS = rn.F_XPOS | rn.F_SCALE_SQRT_D | rn.F_NORM_D
 @pytest.fixture(autouse=True)
 def _gpu(cuda_lib):
     require_gpu()
+    rn.retnet_debug_wait_timeouts(clear=True)
+    yield
+    assert rn.retnet_debug_wait_timeouts(clear=True) == 0  # no bounded wait in the runs gave up
 
 
 @pytest.mark.parametrize("b,L,h,dk,dv,dtype,flags,pos0,with_state", [
