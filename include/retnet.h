@@ -53,7 +53,12 @@
  * exactly, the rotated q, k, the masked scores and the chunk state are rounded to fp16 once
  * each.  fp16 has three more mantissa bits than bf16 and a smaller range, so finite results
  * need |q|, |k|, |v| < 32768, |q.k| / sqrt(d_k) < 65504 and state entries below
- * 65504 * sqrt(d_k).
+ * 65504 * sqrt(d_k); the kernels count every rounding outside that range
+ * (retnet_fp16_range_errors), so a call that left it is detected rather than silent.
+ * RETNET_F_PRECISE (and R~, and the fused MSR call) carries each rounded operand as two fp16
+ * numbers, hi = fp16(x) and lo = fp16(x - hi), and sums the hi*hi, lo*hi and hi*lo products:
+ * about 22 significant bits per operand, at about twice the tensor-core work; the results
+ * then agree with an fp64 evaluation to about 1e-5 of their rms.
  */
 #ifndef RETNET_H
 #define RETNET_H
@@ -387,6 +392,17 @@ RETNET_API int retnet_msr_chunkwise_launches(retnet_dims_t dims, retnet_dtype_t 
  * Returns RETNET_OK or RETNET_ERR_CUDA; *count receives the value before any clear.
  */
 RETNET_API retnet_status_t retnet_debug_wait_timeouts(unsigned int* count, int clear);
+
+/*
+ * Count of device threads that, since the last clear, rounded a tensor-core operand outside
+ * the fp16 range (a magnitude of 65520 or more becomes inf; a NaN counts too): the scaled,
+ * rotated q and k, v, the masked scores or the fp16 state copy (see Precision).  A call whose
+ * bf16 inputs leave that range produces non-finite outputs on the tensor-core kernel and
+ * raises this count; the fp32 CUDA-core kernel (fp32 inputs) has no such limit.  Synchronises
+ * with the device; with clear != 0 the count is reset to 0.  Returns RETNET_OK or
+ * RETNET_ERR_CUDA; *count receives the value before any clear.
+ */
+RETNET_API retnet_status_t retnet_fp16_range_errors(unsigned int* count, int clear);
 
 /* Static, NUL-terminated description of a status code (never NULL). */
 RETNET_API const char* retnet_status_string(retnet_status_t status);

@@ -40,6 +40,7 @@ EXPORTS = ("retnet_retention_parallel", "retnet_retention_chunkwise", "retnet_re
            "retnet_msr_chunkwise", "retnet_msr_chunkwise_launches", "retnet_retention_backward",
            "retnet_backward_workspace_size", "retnet_backward_kernel", "retnet_backward_launches",
            "retnet_chunkwise_kernel", "retnet_chunkwise_launches", "retnet_debug_wait_timeouts",
+           "retnet_fp16_range_errors",
            "retnet_status_string", "retnet_version")
 
 
@@ -111,6 +112,8 @@ def load(path: str = None):
     lib.retnet_chunkwise_launches.restype = _i32
     lib.retnet_debug_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint), _i32]
     lib.retnet_debug_wait_timeouts.restype = _i32
+    lib.retnet_fp16_range_errors.argtypes = [ctypes.POINTER(ctypes.c_uint), _i32]
+    lib.retnet_fp16_range_errors.restype = _i32
     lib.retnet_status_string.argtypes = [_i32]
     lib.retnet_status_string.restype = ctypes.c_char_p
     lib.retnet_version.argtypes = []
@@ -415,6 +418,14 @@ def retnet_debug_wait_timeouts(clear=True):
     """Bounded waits that gave up in the tensor-core kernel since the last clear (synchronises)."""
     c = ctypes.c_uint(0)
     _check(load().retnet_debug_wait_timeouts(ctypes.byref(c), 1 if clear else 0))
+    return c.value
+
+
+def retnet_fp16_range_errors(clear=True):
+    """Device threads that rounded a tensor-core operand outside the fp16 range since the last
+    clear (synchronises); nonzero means some output of those calls is not finite."""
+    c = ctypes.c_uint(0)
+    _check(load().retnet_fp16_range_errors(ctypes.byref(c), 1 if clear else 0))
     return c.value
 
 

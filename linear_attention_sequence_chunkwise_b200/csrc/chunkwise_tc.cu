@@ -190,7 +190,7 @@ struct Converter {
 
   // In place: q -> xi (.) rot(q), k -> zeta (.) rot(k) as fp16; v -> fp16.
   __device__ void convert(uint32_t sq, uint32_t sk, uint32_t sv, const float2* base, bool xpos, float log2g,
-                          int bl) const {
+                          int bl, float& mx) const {
     const uint32_t box = (cs / 8) * T * 128;  // this slot's 64-wide box
     const uint32_t chunk = cs % 8;
     const float xstep = decay_pow(log2g, RS), zstep = exp2f(-static_cast<float>(RS) * log2g);
@@ -219,8 +219,11 @@ struct Converter {
           const float c = F[jj].x, sn = F[jj].y;
           const float q0 = __uint_as_float(q4[k][jj] << 16), q1 = __uint_as_float(q4[k][jj] & 0xffff0000u);
           const float k0 = __uint_as_float(k4[k][jj] << 16), k1 = __uint_as_float(k4[k][jj] & 0xffff0000u);
-          qo[jj] = pack_f16x2(xi * (q0 * c - q1 * sn), xi * (q0 * sn + q1 * c));
-          ko[jj] = pack_f16x2(zeta * (k0 * c - k1 * sn), zeta * (k0 * sn + k1 * c));
+          const float x0 = xi * (q0 * c - q1 * sn), x1 = xi * (q0 * sn + q1 * c);
+          const float y0 = zeta * (k0 * c - k1 * sn), y1 = zeta * (k0 * sn + k1 * c);
+          mx = absmax(absmax(absmax(absmax(mx, x0), x1), y0), y1);
+          qo[jj] = pack_f16x2(x0, x1);
+          ko[jj] = pack_f16x2(y0, y1);
           F[jj] = cmul(F[jj], Z[jj]);
         }
         const uint32_t off = box + sw128(r0 + RS * (kg + k), chunk);
@@ -241,8 +244,11 @@ struct Converter {
       for (int k = 0; k < 4; ++k) {
         uint32_t vo[4];
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj)
-          vo[jj] = pack_f16x2(__uint_as_float(v4[k][jj] << 16), __uint_as_float(v4[k][jj] & 0xffff0000u));
+        for (int jj = 0; jj < 4; ++jj) {
+          const float v0 = __uint_as_float(v4[k][jj] << 16), v1 = __uint_as_float(v4[k][jj] & 0xffff0000u);
+          mx = absmax(absmax(mx, v0), v1);
+          vo[jj] = pack_f16x2(v0, v1);
+        }
         st_shared_v4(sv + sw128(lt / 8 + 16 * (kg + k), lt % 8), vo[0], vo[1], vo[2], vo[3]);
       }
     }
@@ -394,6 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     cv.init(threadIdx.x - 32 * kWarpConv0, hp);
     const bool xpos = (a.flags & RETNET_F_XPOS) != 0;
     bool ok = true;
+    float mx = 0.f;  // largest magnitude rounded to fp16
     for (int i = 0; i < n && ok; ++i) {
       const int s = i % C::NS;
       const int bl = min(T, a.L - i * T);
@@ -405,10 +412,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = mbar_wait(bar(B_TAB0 + (i & 1)), (i >> 1) & 1);
       if (ok) ok = mbar_wait(bar(B_TMA_FULL + s), (i / C::NS) & 1);
       if (!ok) break;
-      cv.convert(sQ(s), sK(s), sV(s), base, xpos, log2g, bl);
+      cv.convert(sQ(s), sK(s), sV(s), base, xpos, log2g, bl, mx);
       fence_proxy_async_smem();
       mbar_arrive(bar(B_CONV_FULL + s));
     }
+    report_fp16_range(mx);
   } else {
     // ------------------------------------------------------------------ TMEM warpgroup
     const uint32_t lane_off = static_cast<uint32_t>(32 * warp) << 16;
@@ -425,7 +433,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // Write R (64 fp32 of one state row) as fp16 into the cross-term operand (MN-major,
     // rows = d_k, 128 B = 64 d_v per row, 128-byte swizzle).
+    float mx = 0.f;  // largest magnitude rounded to fp16 (P and the state copy)
     auto put_r16 = [&](int dk, const float* rv) {
+#pragma unroll
+      for (int c = 0; c < 64; ++c) mx = absmax(mx, sd * rv[c]);
 #pragma unroll
       for (int c8 = 0; c8 < 8; ++c8)
         st_shared_v4(sR + sw128(dk, c8), pack_f16x2(sd * rv[8 * c8 + 0], sd * rv[8 * c8 + 1]),
@@ -486,6 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int c0 = half * 64 + 8 * c8 + 2 * e;
                 const float p0 = (c0 <= my_row) ? __uint_as_float(u[c8 / 2][(8 * c8 + 2 * e) % 16]) * ginv : 0.f;
                 const float p1 = (c0 + 1 <= my_row) ? __uint_as_float(u[c8 / 2][(8 * c8 + 2 * e + 1) % 16]) * ginv : 0.f;
+                mx = absmax(absmax(mx, p0), p1);
                 pk[e] = pack_f16x2(p0, p1);
               }
               st_shared_v4(sP + half * T * 128 + sw128(my_row, c8), pk[0], pk[1], pk[2], pk[3]);
@@ -566,6 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    report_fp16_range(mx);
   }
 
   tc_fence_before();
@@ -820,9 +833,10 @@ struct UnitConverter {
   // WITH_Q = false (state replay) leaves the Q tile alone.
   // zmul multiplies the K row scales (the state pre-pass decays K to its segment's end).
   // HL: the tiles take the fp16 hi parts, sql / skl (same layout) the lo parts.
+  // mx: the largest magnitude rounded to fp16 so far (range check, reported at the end).
   template <bool WITH_Q, bool HL = false>
   __device__ void convert(uint32_t sq, uint32_t sk, uint32_t sv, const float2* bq, const float2* bk, bool xpos,
-                          float log2g, float zmul = 1.f, uint32_t sql = 0, uint32_t skl = 0) const {
+                          float log2g, float& mx, float zmul = 1.f, uint32_t sql = 0, uint32_t skl = 0) const {
     const uint32_t box = (cs / 8) * T * 128;
     const uint32_t chunk = cs % 8;
     const float xstep = decay_pow(log2g, RS), zstep = exp2f(-static_cast<float>(RS) * log2g);
@@ -854,6 +868,7 @@ struct UnitConverter {
           if (WITH_Q) {
             const float q0 = __uint_as_float(q4[k][jj] << 16), q1 = __uint_as_float(q4[k][jj] & 0xffff0000u);
             const float x0 = q0 * Fq[jj].x - q1 * Fq[jj].y, x1 = q0 * Fq[jj].y + q1 * Fq[jj].x;
+            mx = absmax(absmax(mx, x0), x1);
             if (HL) {
               split_f16x2(x0, x1, qo[jj], ql[jj]);
             } else {
@@ -863,6 +878,7 @@ struct UnitConverter {
           }
           const float k0 = __uint_as_float(k4[k][jj] << 16), k1 = __uint_as_float(k4[k][jj] & 0xffff0000u);
           const float y0 = k0 * Fk[jj].x - k1 * Fk[jj].y, y1 = k0 * Fk[jj].y + k1 * Fk[jj].x;
+          mx = absmax(absmax(mx, y0), y1);
           if (HL) {
             split_f16x2(y0, y1, ko[jj], kl[jj]);
           } else {
@@ -891,8 +907,11 @@ struct UnitConverter {
       for (int k = 0; k < VG; ++k) {
         uint32_t vo[4];
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj)
-          vo[jj] = pack_f16x2(__uint_as_float(v4[k][jj] << 16), __uint_as_float(v4[k][jj] & 0xffff0000u));
+        for (int jj = 0; jj < 4; ++jj) {
+          const float v0 = __uint_as_float(v4[k][jj] << 16), v1 = __uint_as_float(v4[k][jj] & 0xffff0000u);
+          mx = absmax(absmax(mx, v0), v1);
+          vo[jj] = pack_f16x2(v0, v1);
+        }
         st_shared_v4(vb + sw128(lt / 8 + VR * (kg % VP + k), lt % 8), vo[0], vo[1], vo[2], vo[3]);
       }
     }
@@ -1270,6 +1289,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL>::THREADS, 1)
     cv.init(threadIdx.x - 32 * C::WARP_CONV0, nb, hp);
     const bool xpos = (a.flags & RETNET_F_XPOS) != 0;
     bool ok = true;
+    float mx = 0.f;  // largest magnitude rounded to fp16
     UnitIter<T, SM> it;
     for (it.start(a.L, nb, c_first, c_lo, c_hi); ok && it.valid(); it.next()) {
       const int s = it.k % C::NS;
@@ -1285,16 +1305,17 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL>::THREADS, 1)
       if constexpr (SM == SEG_STATE) {
         // K of column block w decays to the segment's end E: gamma^(E - 1 - t) in all
         const int e_tok = min(c_hi * nb * T, a.L), blk_end = it.t0() + (it.w + 1) * T;
-        cv.template convert<false>(sQ(s), sK(s), sV(s), tq, tk, xpos, log2g,
+        cv.template convert<false>(sQ(s), sK(s), sV(s), tq, tk, xpos, log2g, mx,
                                    exp2f(static_cast<float>(e_tok - blk_end) * log2g));
       } else if (SM == SEG_REPLAY && it.pre()) {
-        cv.template convert<false>(sQ(s), sK(s), sV(s), tq, tk, xpos, log2g);
+        cv.template convert<false>(sQ(s), sK(s), sV(s), tq, tk, xpos, log2g, mx);
       } else {
-        cv.template convert<true, HL>(sQ(s), sK(s), sV(s), tq, tk, xpos, log2g, 1.f, sQl(s), sKl(s));
+        cv.template convert<true, HL>(sQ(s), sK(s), sV(s), tq, tk, xpos, log2g, mx, 1.f, sQl(s), sKl(s));
       }
       fence_proxy_async_smem();
       mbar_arrive(bar(Q_CONV_FULL + s));
     }
+    report_fp16_range(mx);
     }
   } else if (warp >= C::WARP_S0 && warp < C::WARP_S0 + C::WARPS_S) {
     // ------------------------------------------------------------------ state group
@@ -1344,6 +1365,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL>::THREADS, 1)
         return (DK == 64) ? (lane < 16 ? 16 * (warp % 4) + lane : -1) : blk * 128 + 32 * (warp % 4) + lane;
       };
       bool ok = true;
+      float smx = 0.f;  // largest state-copy magnitude rounded to fp16
       int last_dr = -1, last_bl = T, last_nbw = 1;
       UnitIter<T, SM> it;
       for (it.start(a.L, nb, c_first, c_lo, c_hi); ok && it.valid(); it.next()) {
@@ -1388,6 +1410,8 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL>::THREADS, 1)
                 const int col = GW * grp + 8 * c8;
                 const uint32_t* x = &u[(8 * c8) / 16][(8 * c8) % 16];
                 const uint32_t off = (col / 64) * DK * 128 + sw128(dk, (col % 64) / 8);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) smx = absmax(smx, sd * __uint_as_float(x[e]));
                 if constexpr (HL) {
                   uint32_t hi[4], lo[4];
 #pragma unroll
@@ -1416,6 +1440,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL>::THREADS, 1)
         last_bl = it.bl;
         last_nbw = it.nbw;
       }
+      report_fp16_range(smx);
       // End of the sequence: R_last = hh * M once the last increment landed.
       if (ok && last_dr >= 0 && (!SEG || c_hi * nb * T >= a.L)) {
         ok = __all_sync(0xffffffffu, mbar_wait(bar(Q_DR_FULL + 0), last_dr & 1));
@@ -1459,9 +1484,12 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL>::THREADS, 1)
   #pragma unroll
       for (int c = 0; c < RC; ++c) R[c] = 0.f;
       if (dk >= 0) start_state(dk, col0, RC, R);
+      float smx = 0.f;  // largest state-copy magnitude rounded to fp16
       auto put_r16 = [&](uint32_t base) {
         if (dk < 0) return;
         base += ch * DK * 128;
+  #pragma unroll
+        for (int c = 0; c < 64; ++c) smx = absmax(smx, sd * R[c]);
   #pragma unroll
         for (int c8 = 0; c8 < 8; ++c8) {
           if constexpr (HL) {
@@ -1530,6 +1558,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL>::THREADS, 1)
             *reinterpret_cast<float4*>(dst + 4 * c4) = make_float4(R[4 * c4], R[4 * c4 + 1], R[4 * c4 + 2], R[4 * c4 + 3]);
         }
       }
+      report_fp16_range(smx);
     }
   } else {
     // ------------------------------------------------------------------ P / epilogue group
@@ -1751,6 +1780,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL>::THREADS, 1)
       return true;
     };
     bool ok = true;
+    float pmx = 0.f;  // largest |P| rounded to fp16
     int pend_rb = -1, pend_i = 0, pend_u = 0, pend_bl = 0;  // a finished row block awaiting its epilogue
     UnitIter<T, SM> it;
     for (it.start(a.L, nb, c_first, c_lo, c_hi); ok && it.valid(); it.next()) {
@@ -1787,6 +1817,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL>::THREADS, 1)
               const int c0 = col + 2 * e;
               const float p0 = (!diag || c0 <= my_row) ? __uint_as_float(u16[c8 / 2][(8 * c8 + 2 * e) % 16]) * pf : 0.f;
               const float p1 = (!diag || c0 + 1 <= my_row) ? __uint_as_float(u16[c8 / 2][(8 * c8 + 2 * e + 1) % 16]) * pf : 0.f;
+              pmx = absmax(absmax(pmx, p0), p1);
               if (HL) {
                 split_f16x2(p0, p1, pk[e], pl[e]);
               } else {
@@ -1811,6 +1842,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL>::THREADS, 1)
       }
     }
     if (ok && pend_rb >= 0) epilogue(pend_rb, pend_i, pend_u, pend_bl);
+    report_fp16_range(pmx);
   }
 
   tc_fence_before();
@@ -1844,6 +1876,7 @@ __global__ void __launch_bounds__(256) tc_convert_kernel(const uint4* __restrict
   const int64_t n_qk = tokens * S;
   const int64_t n_v = tokens * heads * (dv / 8);
   const bool xpos = (flags & RETNET_F_XPOS) != 0;
+  float mx = 0.f;  // largest magnitude rounded to fp16
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_qk + n_v;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     if (i < n_qk) {
@@ -1870,6 +1903,7 @@ __global__ void __launch_bounds__(256) tc_convert_kernel(const uint4* __restrict
           const float k0 = __uint_as_float(wk[jj] << 16), k1 = __uint_as_float(wk[jj] & 0xffff0000u);
           const float x0 = xi * (q0 * f[jj].x - q1 * f[jj].y), x1 = xi * (q0 * f[jj].y + q1 * f[jj].x);
           const float y0 = zeta * (k0 * f[jj].x - k1 * f[jj].y), y1 = zeta * (k0 * f[jj].y + k1 * f[jj].x);
+          mx = absmax(absmax(absmax(absmax(mx, x0), x1), y0), y1);
           if (HL) {
             split_f16x2(x0, x1, oq[jj], lq[jj]);
             split_f16x2(y0, y1, ok[jj], lk[jj]);
@@ -1891,11 +1925,15 @@ __global__ void __launch_bounds__(256) tc_convert_kernel(const uint4* __restrict
       const uint32_t w[4] = {x.x, x.y, x.z, x.w};
       uint32_t o[4];
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj)
-        o[jj] = pack_f16x2(__uint_as_float(w[jj] << 16), __uint_as_float(w[jj] & 0xffff0000u));
+      for (int jj = 0; jj < 4; ++jj) {
+        const float v0 = __uint_as_float(w[jj] << 16), v1 = __uint_as_float(w[jj] & 0xffff0000u);
+        mx = absmax(absmax(mx, v0), v1);
+        o[jj] = pack_f16x2(v0, v1);
+      }
       vo[j] = make_uint4(o[0], o[1], o[2], o[3]);
     }
   }
+  report_fp16_range(mx);
 }
 
 // ---- host side -------------------------------------------------------------------------------
@@ -2348,6 +2386,13 @@ bool tc_chunkwise_heads_ok(const RetentionCall& c, const HeadParams& hp) {
   for (int64_t h = 0; h < c.dims.heads; ++h)
     if (static_cast<double>(hp.log2g[h]) * span < -12.0) return false;
   return true;
+}
+
+cudaError_t tc_fp16_overflows(unsigned int* count, bool clear) {
+  cudaError_t e = cudaMemcpyFromSymbol(count, sm100::g_fp16_overflows, sizeof(unsigned int));
+  if (e != cudaSuccess || !clear || *count == 0) return e;
+  const unsigned int zero = 0;
+  return cudaMemcpyToSymbol(sm100::g_fp16_overflows, &zero, sizeof(unsigned int));
 }
 
 cudaError_t tc_wait_timeouts(unsigned int* count, bool clear) {

@@ -378,6 +378,12 @@ retnet_status_t retnet_debug_wait_timeouts(unsigned int* count, int clear) {
   return from_cuda(tc_wait_timeouts(count, clear != 0));
 }
 
+retnet_status_t retnet_fp16_range_errors(unsigned int* count, int clear) {
+  if (!count) return RETNET_ERR_NULL_PTR;
+  if (cudaDeviceSynchronize() != cudaSuccess) return RETNET_ERR_CUDA;
+  return from_cuda(tc_fp16_overflows(count, clear != 0));
+}
+
 retnet_status_t retnet_retention_step(const void* q, const void* k, const void* v, void* o, int64_t batch,
                                       int64_t heads, int64_t d_k, int64_t d_v, retnet_dtype_t in_dtype,
                                       retnet_dtype_t out_dtype, float* state, float* z, const float* gamma,

@@ -67,6 +67,20 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
 }
 
 static __device__ unsigned int g_wait_timeouts = 0;
+// Threads that rounded a value outside the fp16 range (magnitude >= 65520 becomes inf, or NaN)
+// when forming a tensor-core operand: bf16 inputs span a far wider range than fp16 operands.
+static __device__ unsigned int g_fp16_overflows = 0;
+
+// One report per thread: mx is the largest magnitude the thread rounded to fp16 (NaN-safe).
+__device__ __forceinline__ void report_fp16_range(float mx) {
+  if (!(mx < 65520.f)) atomicAdd(&g_fp16_overflows, 1u);
+}
+// Largest magnitude so far, NaN sticky (max.NaN propagates a NaN where fmaxf would drop it).
+__device__ __forceinline__ float absmax(float m, float x) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(m), "f"(fabsf(x)));
+  return r;
+}
 
 // ---- thread-block clusters: distributed shared memory, remote mbarrier arrivals --------------
 

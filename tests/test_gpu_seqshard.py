@@ -24,7 +24,9 @@ FLAGS = rn.F_XPOS | rn.F_SCALE_SQRT_D | rn.F_NORM_D
 def _gpu(cuda_lib):
     require_gpu()
     rn.retnet_debug_wait_timeouts(clear=True)
+    rn.retnet_fp16_range_errors(clear=True)
     yield
+    assert rn.retnet_fp16_range_errors(clear=True) == 0  # no tensor-core operand left the fp16 range
     assert rn.retnet_debug_wait_timeouts(clear=True) == 0
 
 

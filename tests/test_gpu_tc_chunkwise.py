@@ -21,7 +21,9 @@ FLAGS = rn.F_XPOS | rn.F_SCALE_SQRT_D | rn.F_NORM_D
 def _gpu(cuda_lib):
     require_gpu()
     rn.retnet_debug_wait_timeouts(clear=True)
+    rn.retnet_fp16_range_errors(clear=True)
     yield
+    assert rn.retnet_fp16_range_errors(clear=True) == 0  # no tensor-core operand left the fp16 range
     assert rn.retnet_debug_wait_timeouts(clear=True) == 0
 
 
@@ -361,3 +363,31 @@ def test_tc_norm_r_needs_room_for_its_factors():
     assert rn.retnet_chunkwise_launches((2, 300, 4, 128), 64, rn.BF16, oracle.F_ALL, 64, g, need - 256) == 1
     # two key-sum passes (the sequence in segments), then the kernel (no room for a split)
     assert rn.retnet_chunkwise_launches((2, 300, 4, 128), 64, rn.BF16, oracle.F_ALL, 64, g, need) == 3
+
+
+def test_fp16_range_is_reported():
+    """bf16 inputs beyond the fp16 operand range (a value of v above 65504, a q element whose
+    rotated, scaled copy exceeds it): the tensor-core kernel rounds them to inf, and the range
+    counter says so -- no silent non-finite output.  In-range calls leave it at zero, with
+    single and split operands and with the conversion pre-pass."""
+    b, L, h, dk, dv = 1, 256, 2, 64, 64
+    q, k, v = si.qkv(b, L, h, dk, dv, 1500, "bf16")
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+    ws = torch.empty(rn.retnet_chunkwise_workspace_size((b, L, h, dk, dv)), dtype=torch.uint8, device="cuda")
+    v_big = v.clone()
+    v_big[0, 70, 1, 5] = 70000.0
+    q_big = q.clone()
+    q_big[0, 130, 0, 10] = 1.0e5
+    for flags in (FLAGS, FLAGS | rn.F_PRECISE):
+        for B, wsp in ((64, None), (128, ws)):  # in-kernel converters; conversion pre-pass
+            o = torch.empty(b, L, h, dv, device="cuda")
+            rn.retnet_fp16_range_errors(clear=True)
+            rn.retnet_retention_chunkwise_ws(dev(q), dev(k), dev(v), o, g, th, 0, flags, B, workspace=wsp)
+            assert rn.retnet_fp16_range_errors(clear=True) == 0
+            assert bool(torch.isfinite(o).all())
+            for qq, vv in ((q, v_big), (q_big, v)):
+                rn.retnet_retention_chunkwise_ws(dev(qq), dev(k), dev(vv), o, g, th, 0, flags, B, workspace=wsp)
+                n = rn.retnet_fp16_range_errors(clear=True)
+                print(f"flags={flags} B={B} ws={wsp is not None}: {n} range reports, "
+                      f"finite={bool(torch.isfinite(o).all())}")
+                assert n > 0
