@@ -664,10 +664,17 @@ struct Cfg3 {
   static constexpr int TABBYTES = 2 * 2 * (DK / 2) * 8;
   static constexpr int BUDGET = 227 * 1024 - 1024;
   static constexpr int TAIL = TABBYTES + NBARS * 8 + 16 + XBYTES;
-  static constexpr int PBUF = (2 * STAGE + 2 * PB + RB + TAIL <= BUDGET) ? 2 : 1;
-  static constexpr int NS_R2 = (BUDGET - (PBUF * PB + 2 * RB + TAIL)) / STAGE;
-  static constexpr int NS_R1 = (BUDGET - (PBUF * PB + RB + TAIL)) / STAGE;
-  static constexpr int RBUF = (NS_R2 >= 3 || NS_R1 < 3) && NS_R2 >= 2 ? 2 : 1;
+  // Buffer counts.  A second fp16 state buffer takes the cross term of chunk i off the state
+  // group's path to chunk i + 1 (with one buffer the copy of R_i waits for that MMA), so it is
+  // preferred as long as three stages remain, over a second P buffer.
+  static constexpr int ns_for(int pbuf, int rbuf) { return (BUDGET - (pbuf * PB + rbuf * RB + TAIL)) / STAGE; }
+  static constexpr int PBUF0 = (2 * STAGE + 2 * PB + RB + TAIL <= BUDGET) ? 2 : 1;
+  static constexpr int NS_R2 = ns_for(PBUF0, 2);
+  static constexpr int NS_R1 = ns_for(PBUF0, 1);
+  static constexpr int RBUF0 = (NS_R2 >= 3 || NS_R1 < 3) && NS_R2 >= 2 ? 2 : 1;
+  static constexpr bool TRADE = RBUF0 == 1 && PBUF0 == 2 && ns_for(1, 2) >= 3;
+  static constexpr int PBUF = TRADE ? 1 : PBUF0;
+  static constexpr int RBUF = TRADE ? 2 : RBUF0;
   static constexpr int FIXED = PBUF * PB + RBUF * RB + TAIL;
   static constexpr int NS_FIT = (BUDGET - FIXED) / STAGE;
   static constexpr int NS = NS_FIT > 4 ? 4 : NS_FIT;
