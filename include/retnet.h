@@ -394,6 +394,18 @@ RETNET_API int retnet_msr_chunkwise_launches(retnet_dims_t dims, retnet_dtype_t 
 RETNET_API retnet_status_t retnet_debug_wait_timeouts(unsigned int* count, int clear);
 
 /*
+ * Testing aid for the bounded waits above: sets, for the tensor-core kernels of the current
+ * device, how many SM clock cycles a wait for another role's progress may last before it gives
+ * up (cycles > 0, at least 100), or restores the default of 4e9 cycles (about 2 s; cycles <= 0).
+ * With a small budget waits give up: the kernel then stops its work, waits with the full budget
+ * for the TMA copies and MMAs it already issued, frees its tensor memory and returns; the
+ * outputs of such a call are undefined and retnet_debug_wait_timeouts counts the give-ups.
+ * Not for production calls.  Synchronises with the device.  RETNET_OK, RETNET_ERR_BAD_PARAM
+ * (0 < cycles < 100) or RETNET_ERR_CUDA.
+ */
+RETNET_API retnet_status_t retnet_debug_set_wait_budget(long long cycles);
+
+/*
  * Count of device threads that, since the last clear, rounded a tensor-core operand outside
  * the fp16 range (a magnitude of 65520 or more becomes inf; a NaN counts too): the scaled,
  * rotated q and k, v, the masked scores or the fp16 state copy (see Precision).  A call whose

@@ -40,7 +40,7 @@ EXPORTS = ("retnet_retention_parallel", "retnet_retention_chunkwise", "retnet_re
            "retnet_msr_chunkwise", "retnet_msr_chunkwise_launches", "retnet_retention_backward",
            "retnet_backward_workspace_size", "retnet_backward_kernel", "retnet_backward_launches",
            "retnet_chunkwise_kernel", "retnet_chunkwise_launches", "retnet_debug_wait_timeouts",
-           "retnet_fp16_range_errors",
+           "retnet_fp16_range_errors", "retnet_debug_set_wait_budget",
            "retnet_status_string", "retnet_version")
 
 
@@ -114,6 +114,8 @@ def load(path: str = None):
     lib.retnet_debug_wait_timeouts.restype = _i32
     lib.retnet_fp16_range_errors.argtypes = [ctypes.POINTER(ctypes.c_uint), _i32]
     lib.retnet_fp16_range_errors.restype = _i32
+    lib.retnet_debug_set_wait_budget.argtypes = [ctypes.c_longlong]
+    lib.retnet_debug_set_wait_budget.restype = _i32
     lib.retnet_status_string.argtypes = [_i32]
     lib.retnet_status_string.restype = ctypes.c_char_p
     lib.retnet_version.argtypes = []
@@ -419,6 +421,11 @@ def retnet_debug_wait_timeouts(clear=True):
     c = ctypes.c_uint(0)
     _check(load().retnet_debug_wait_timeouts(ctypes.byref(c), 1 if clear else 0))
     return c.value
+
+
+def retnet_debug_set_wait_budget(cycles=0):
+    """Testing aid: pipeline-wait budget of the tensor-core kernels in SM cycles (0 = default)."""
+    _check(load().retnet_debug_set_wait_budget(int(cycles)))
 
 
 def retnet_fp16_range_errors(clear=True):

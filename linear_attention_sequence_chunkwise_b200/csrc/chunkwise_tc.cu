@@ -334,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // Every load this thread issued must have landed before the CTA may exit.
       for (int s = 0; s < C::NS; ++s)
-        if (issued[s] > 0) mbar_wait(bar(B_TMA_FULL + s), (issued[s] - 1) & 1);
+        if (issued[s] > 0) mbar_wait(bar(B_TMA_FULL + s), (issued[s] - 1) & 1, kDrainBudget);
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------------ MMA issuer
@@ -392,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // Drain: every MMA issued above completes before TMEM is released.
       mma_commit(bar(B_DRAIN));
-      mbar_wait(bar(B_DRAIN), 0);
+      mbar_wait(bar(B_DRAIN), 0, kDrainBudget);
     }
   } else if (warp >= kWarpConv0) {
     // ------------------------------------------------------------------ converters
@@ -1113,7 +1113,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL>::THREADS, 1)
       }
       // Every load this thread issued must have landed before the CTA may exit.
       for (int s = 0; s < C::NS; ++s)
-        if (issued[s] > 0) mbar_wait(bar(Q_TMA_FULL + s), (issued[s] - 1) & 1);
+        if (issued[s] > 0) mbar_wait(bar(Q_TMA_FULL + s), (issued[s] - 1) & 1, kDrainBudget);
     }
   } else if (warp == C::WARP_MMA) {
     // ------------------------------------------------------------------ MMA issuer
@@ -1281,13 +1281,13 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL>::THREADS, 1)
         }
         if (progress) {
           idle_since = clock64();
-        } else if (clock64() - idle_since > 4000000000LL) {
+        } else if (clock64() - idle_since > *const_cast<volatile long long*>(&g_wait_budget)) {
           atomicAdd(&g_wait_timeouts, 1u);  // same bound and report as a blocking wait
           break;
         }
       }
       mma_commit(bar(Q_DRAIN));
-      mbar_wait(bar(Q_DRAIN), 0);
+      mbar_wait(bar(Q_DRAIN), 0, kDrainBudget);
     }
   } else if (warp >= C::WARP_CONV0 && warp < C::WARP_CONV0 + C::CONV_WARPS) {
     // ------------------------------------------------------------------ converters
@@ -2393,6 +2393,11 @@ bool tc_chunkwise_heads_ok(const RetentionCall& c, const HeadParams& hp) {
   for (int64_t h = 0; h < c.dims.heads; ++h)
     if (static_cast<double>(hp.log2g[h]) * span < -12.0) return false;
   return true;
+}
+
+cudaError_t tc_set_wait_budget(long long cycles) {
+  const long long v = cycles > 0 ? cycles : sm100::kDrainBudget;
+  return cudaMemcpyToSymbol(sm100::g_wait_budget, &v, sizeof(long long));
 }
 
 cudaError_t tc_fp16_overflows(unsigned int* count, bool clear) {

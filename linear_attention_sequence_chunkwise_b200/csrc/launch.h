@@ -78,6 +78,8 @@ cudaError_t launch_key_sum(const RetentionCall& c, const HeadParams& hp, cudaStr
 int key_sum_launches(const Dims& d);
 // Reads (and optionally clears) the count of bounded waits that gave up in the tensor-core kernel.
 cudaError_t tc_wait_timeouts(unsigned int* count, bool clear);
+// Sets the pipeline-wait budget of the tensor-core kernels (SM cycles; <= 0 restores the default).
+cudaError_t tc_set_wait_budget(long long cycles);
 // Reads (and optionally clears) the count of threads that rounded a tensor-core operand outside
 // the fp16 range.
 cudaError_t tc_fp16_overflows(unsigned int* count, bool clear);

@@ -378,6 +378,12 @@ retnet_status_t retnet_debug_wait_timeouts(unsigned int* count, int clear) {
   return from_cuda(tc_wait_timeouts(count, clear != 0));
 }
 
+retnet_status_t retnet_debug_set_wait_budget(long long cycles) {
+  if (cycles > 0 && cycles < 100) return RETNET_ERR_BAD_PARAM;
+  if (cudaDeviceSynchronize() != cudaSuccess) return RETNET_ERR_CUDA;
+  return from_cuda(tc_set_wait_budget(cycles));
+}
+
 retnet_status_t retnet_fp16_range_errors(unsigned int* count, int clear) {
   if (!count) return RETNET_ERR_NULL_PTR;
   if (cudaDeviceSynchronize() != cudaSuccess) return RETNET_ERR_CUDA;

@@ -67,6 +67,12 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
 }
 
 static __device__ unsigned int g_wait_timeouts = 0;
+// Budget, in SM clock cycles, of a wait for another role's progress (about 2 s by default).  A
+// host-side testing aid may lower it so that waits give up; waits for work this thread already
+// issued (TMA loads, MMAs) always take kDrainBudget, so a kernel that gave up never leaves with
+// copies or products in flight.
+constexpr long long kDrainBudget = 4000000000LL;
+static __device__ long long g_wait_budget = kDrainBudget;
 // Threads that rounded a value outside the fp16 range (magnitude >= 65520 becomes inf, or NaN)
 // when forming a tensor-core operand: bf16 inputs span a far wider range than fp16 operands.
 static __device__ unsigned int g_fp16_overflows = 0;
@@ -117,7 +123,7 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t remote_bar) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
 }
 // Bounded wait on a local mbarrier whose arrivals come from the cluster (acquire at cluster scope).
-__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, long long budget = 4000000000LL) {
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, long long budget = -1) {
   auto probe = [&]() -> bool {
     uint32_t ok;
     asm volatile(
@@ -130,6 +136,7 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
     return ok != 0;
   };
   if (probe()) return true;
+  if (budget < 0) budget = *const_cast<volatile long long*>(&g_wait_budget);
   const long long t0 = clock64();
   while (!probe()) {
     if (clock64() - t0 > budget) {
@@ -142,9 +149,11 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
 
 
 // Waits for the phase with the given parity to complete, for at most `budget` SM clock
-// cycles.  Returns false (and counts a timeout) if it gave up.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long long budget = 4000000000LL) {
+// cycles (default: the pipeline budget g_wait_budget).  Returns false (and counts a timeout)
+// if it gave up.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long long budget = -1) {
   if (mbar_try_wait(bar, parity)) return true;
+  if (budget < 0) budget = *const_cast<volatile long long*>(&g_wait_budget);
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
     if (clock64() - t0 > budget) {

@@ -391,3 +391,33 @@ def test_fp16_range_is_reported():
                 print(f"flags={flags} B={B} ws={wsp is not None}: {n} range reports, "
                       f"finite={bool(torch.isfinite(o).all())}")
                 assert n > 0
+
+
+def test_bounded_waits_give_up_and_recover():
+    """The give-up path of the kernel's bounded waits.  With the wait budget lowered to 500 SM
+    cycles (a testing aid) the roles' waits for one another give up: the call must return (no
+    hang), count its give-ups, drain the TMA copies and MMAs already issued and free its tensor
+    memory.  After the default budget is restored the same call is bit-identical to one made
+    before, and counts nothing.  (A plain launch, no thread-block clusters.)"""
+    b, L, h, dk, dv, B = 1, 640, 2, 64, 64, 64
+    q, k, v = (dev(x) for x in si.qkv(b, L, h, dk, dv, 1600, "bf16"))
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+    assert rn.retnet_chunkwise_kernel((b, L, h, dk), dv, rn.BF16, FLAGS, B, g) == 1
+    o_ref, o_bad, o_again = (torch.empty(b, L, h, dv, device="cuda") for _ in range(3))
+    rn.retnet_retention_chunkwise(q, k, v, o_ref, g, th, 0, FLAGS, B)
+    torch.cuda.synchronize()
+    assert rn.retnet_debug_wait_timeouts(clear=True) == 0
+    rn.retnet_debug_set_wait_budget(500)
+    try:
+        rn.retnet_retention_chunkwise(q, k, v, o_bad, g, th, 0, FLAGS, B)
+        torch.cuda.synchronize()
+        gave_up = rn.retnet_debug_wait_timeouts(clear=True)
+    finally:
+        rn.retnet_debug_set_wait_budget(0)
+    rn.retnet_fp16_range_errors(clear=True)  # (the abandoned call's buffers are undefined)
+    print(f"waits that gave up with a 500-cycle budget: {gave_up}")
+    assert gave_up > 0
+    rn.retnet_retention_chunkwise(q, k, v, o_again, g, th, 0, FLAGS, B)
+    torch.cuda.synchronize()
+    assert torch.equal(o_again, o_ref)
+    assert rn.retnet_debug_wait_timeouts(clear=True) == 0
