@@ -114,7 +114,11 @@ typedef struct {
  * position pos0 >= 0 (pos0 moves the rotation and the D~ row counts; no earlier tokens
  * contribute).  q, k, v: in_dtype; o: out_dtype.  gamma: host float[heads] in (0,1);
  * theta: host float[d_k/2] (may be NULL without RETNET_F_XPOS).  seqlen may be 0 (no work).
- * Cost is O(seqlen^2) per (batch, head).
+ * Kernels: bf16 inputs without RETNET_F_NORM_R, on the shapes the tensor-core chunkwise kernel
+ * takes (see retnet_retention_chunkwise), run on the tensor cores: a sequence of up to 512
+ * tokens as one masked tile of 64, 128, 256 or 512 rows (the O(seqlen^2) product itself), a
+ * longer one in 512-token chunks (the same sum re-associated, §2.4).  Other calls run the fp32
+ * CUDA-core kernel, O(seqlen^2) per (batch, head).
  */
 RETNET_API retnet_status_t retnet_retention_parallel(const void* q, const void* k, const void* v, void* o,
                                           retnet_dims_t dims, retnet_dtype_t in_dtype,

@@ -100,6 +100,20 @@ retnet_status_t retnet_retention_parallel(const void* q, const void* k, const vo
   if ((st = check_device()) != RETNET_OK) return st;
   RetentionCall c{q, k, v, o, Dims{dims.batch, dims.seqlen, dims.heads, dims.d_k, dims.d_v}, in_dtype, out_dtype,
                   pos0, flags, dims.seqlen, false, nullptr, nullptr, nullptr, nullptr};
+  // bf16 inputs without R~ (whose row sums need a workspace) run on the tensor-core kernel: a
+  // sequence of up to 512 tokens is one chunk of the smallest size that holds it, i.e. the
+  // masked B x B product of §2.3 itself (no state: every token's history is in the tile); a
+  // longer one is cut into 512-token chunks, §2.4's re-association of the same sum.
+  if (in_dtype == RETNET_BF16 && !(flags & RETNET_F_NORM_R)) {
+    RetentionCall t = c;
+    t.chunk = dims.seqlen <= 64 ? 64 : dims.seqlen <= 128 ? 128 : dims.seqlen <= 256 ? 256 : 512;
+    t.has_state = true;  // (no state_in / state_out: a zero start, nothing written)
+    t.precise = (flags & RETNET_F_PRECISE) != 0;
+    if (tc_chunkwise_supported(t) && tc_chunkwise_heads_ok(t, hp)) {
+      if (!tc_driver_ready()) return RETNET_ERR_CUDA;
+      return from_cuda(launch_tc_chunkwise(t, hp, static_cast<cudaStream_t>(stream)));
+    }
+  }
   return from_cuda(launch_simt_retention(c, hp, static_cast<cudaStream_t>(stream)));
 }
 

@@ -203,3 +203,26 @@ def test_degenerate_sizes():
     n = np.arange(1, L + 1)
     geo = -np.expm1(n * np.log1p(-(1 - 0.96875))) / (1 - 0.96875)
     np.testing.assert_allclose(o.cpu().double().numpy()[0, :, 0, 0], geo, rtol=2e-6)
+
+
+@pytest.mark.parametrize("b,L,h,dk,dv,flags,pos0", [
+    (2, 64, 2, 64, 64, oracle.F_XPOS | oracle.F_SCALE_SQRT_D | oracle.F_NORM_D, 0),
+    (1, 200, 3, 128, 128, oracle.F_XPOS | oracle.F_SCALE_SQRT_D | oracle.F_NORM_D, 9),
+    (2, 512, 2, 128, 64, oracle.F_SCALE_SQRT_D, 0),
+    (1, 1, 2, 256, 64, oracle.F_XPOS | oracle.F_NORM_D, 3),
+    (1, 700, 2, 64, 128, oracle.F_XPOS | oracle.F_SCALE_SQRT_D | oracle.F_NORM_D, 0)])
+def test_parallel_bf16_on_tensor_cores(b, L, h, dk, dv, flags, pos0):
+    """bf16 parallel form (§2.3) on the tensor-core kernel: one masked tile of the whole
+    sequence up to 512 tokens, 512-token chunks beyond; single fp16 operands at the bf16 bar,
+    split operands (RETNET_F_PRECISE) at the fp32 bar."""
+    q, k, v = si.qkv(b, L, h, dk, dv, 1700 + L, "bf16")
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+    ref = oracle.parallel(q, k, v, g, th, pos0, flags)
+    for fl, tol in ((flags, TOL_BF16), (flags | rn.F_PRECISE, TOL_F32)):
+        o = torch.empty(b, L, h, dv, device="cuda")
+        rn.retnet_retention_parallel(dev(q), dev(k), dev(v), o, g, th, pos0, fl)
+        torch.cuda.synchronize()
+        e = err(o, ref)
+        print(f"parallel bf16 L={L} dk={dk} flags={fl}: {e:.3e}")
+        assert e <= tol
+    assert rn.retnet_debug_wait_timeouts(clear=True) == 0
