@@ -246,8 +246,12 @@ RETNET_API retnet_status_t retnet_retention_chunkwise_static(const void* q, cons
  *   a256(4 * batch * seqlen * heads)                        (R~ row factors)
  *   + a256(4 * batch * heads * d_k * 64)                     (R~ key-sum segment values)
  *   + max(6 * batch * heads * d_k * d_v * 4,                 (six sub-segment states)
- *         2 * a256(2 * batch * seqlen * heads * d_k) + a256(2 * batch * seqlen * heads * d_v))
- *                                                            (fp16 copies of q, k, v).
+ *         4 * a256(2 * batch * seqlen * heads * d_k) + a256(2 * batch * seqlen * heads * d_v),
+ *                                                            (fp16 copies of q, k (hi and lo), v)
+ *         2 * a256(2 * batch * seqlen * heads * d_k) + a256(2 * batch * seqlen * heads * d_v)
+ *         + P)                                               (fp16 copies, then the P tiles)
+ *   with P = a256(batch * heads * ceil(seqlen / 512) * 36 * 64 * 64 * 2) for d_k = 256, else 0
+ *   (the masked score tiles that the P pass computes once per head, for chunks of 128 to 512).
  * Host-only; no device access.  RETNET_ERR_NULL_PTR without `bytes`, RETNET_ERR_BAD_SHAPE for
  * negative sizes.
  */

@@ -608,7 +608,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 //   1 warp TMA, 1 warp MMA issuer (one unit ahead: S and dR of unit k+1 before X/PV of unit k).
 // ============================================================================================
 
-template <int DK, int T, int DVS, bool PRE = false, bool FUSE = false, bool HL = false>
+template <int DK, int T, int DVS, bool PRE = false, bool FUSE = false, bool HL = false, bool PS = false>
 struct Cfg3 {
   static constexpr int NDV = DVS / 64;              // 64-column boxes of the d_v slice
   static constexpr int RBLK = DK > 128 ? 2 : 1;     // 128-row blocks of the state increment
@@ -638,10 +638,12 @@ struct Cfg3 {
   // scores P and the state copy -- is held as hi + lo, hi = fp16(x), lo = fp16(x - hi), so a
   // product of two of them keeps ~22 significant bits; the stage holds [Q hi][K hi][V][Q lo][K lo].
   static constexpr int QT = HL ? 2 : 1;
-  static constexpr int STAGE = 2 * QBYTES * QT + VBYTES;
   static constexpr int PBYTES = T * T * 2;
+  // PS (P tiles computed by the P pass): the stage also holds the unit's P tile, [Q][K][V][P],
+  // and there is no P buffer of the P warps.
+  static constexpr int STAGE = 2 * QBYTES * QT + VBYTES + (PS ? PBYTES : 0);
   static constexpr int RBYTES = DK * DVS * 2;
-  static constexpr int PB = PBYTES * QT;  // one P buffer (hi, then lo)
+  static constexpr int PB = PS ? 0 : PBYTES * QT;  // one P buffer (hi, then lo)
   static constexpr int RB = RBYTES * QT;  // one fp16 state buffer (hi, then lo)
   // TMEM: O[2] (DVS columns each), X[XBUF] (cross accumulators; none when the slice is 128
   // wide, which then runs one sub-block per chunk only), S[SBUF] (T columns), dR[DRBUF]
@@ -681,7 +683,7 @@ struct Cfg3 {
   static constexpr int SMEM = NS * STAGE + FIXED + 1024;
   // split operands at d_k = 256 leave room for one stage only (the units then run in turn)
   static constexpr bool FITS = NS >= (HL ? 1 : 2) && USED <= 512 && (DVS == 64 || DVS == 128) && (!RTM || DRBUF == 1) &&
-                               (!HL || (T == 64 && DVS == 64));
+                               (!HL || (T == 64 && DVS == 64)) && (!PS || (PRE && !HL && !FUSE));
   // Columns per TMEM load batch: 18 warps leave 96 registers a thread (five warps share one
   // sub-partition's register file), too few to hold 64 loaded columns next to the state.
   static constexpr int LDW = THREADS > 512 ? 32 : 64;
@@ -925,13 +927,15 @@ struct UnitConverter {
   }
 };
 
-template <int DK, int T, int DVS, int SM, bool PRE, bool FUSE, typename Tout, bool HL = false>
-__global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL>::THREADS, 1)
+template <int DK, int T, int DVS, int SM, bool PRE, bool FUSE, typename Tout, bool HL = false, bool PS = false>
+__global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL, PS>::THREADS, 1)
     tc_chunkwise_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_ql,
                              const __grid_constant__ CUtensorMap tm_kl, TcArgs a, HeadParams hp) {
-  // tm_ql, tm_kl: the lo parts of pre-converted split operands (HL with PRE); unused otherwise.
-  using C = Cfg3<DK, T, DVS, PRE, FUSE, HL>;
+  // tm_ql, tm_kl: the lo parts of pre-converted split operands (HL with PRE); with PS, tm_ql is
+  // the map of the P tiles ([tile][T][T] fp16, box T x T) and tm_kl is unused; unused otherwise.
+  using C = Cfg3<DK, T, DVS, PRE, FUSE, HL, PS>;
+  static_assert(!PS || (PRE && !HL && !FUSE && SM == SEG_NONE), "P tiles from the P pass: pre-converted, unsplit");
   static_assert(!FUSE || (SM == SEG_NONE && DVS == 64), "the fused epilogue runs unsplit, 64-column slices");
   static_assert(!HL || SM == SEG_NONE, "split operands run without sequence segments");
   // Stage ready for the MMAs: converted in place, or (PRE) landed already converted.
@@ -1039,6 +1043,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL>::THREADS, 1)
   // right after the hi part of the same buffer
   auto sQl = [&](int s) { return sbase + s * C::STAGE + 2 * C::QBYTES + C::VBYTES; };
   auto sKl = [&](int s) { return sbase + s * C::STAGE + 3 * C::QBYTES + C::VBYTES; };
+  auto sPs = [&](int s) { return sbase + s * C::STAGE + 2 * C::QBYTES + C::VBYTES; };  // PS: the unit's P tile
   auto sP = [&](int k) { return sP0 + (k % C::PBUF) * C::PB; };
   auto sR = [&](int i) { return sR0 + (i % C::RBUF) * C::RB; };
 
@@ -1077,6 +1082,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL>::THREADS, 1)
       prefetch_tensormap(&tm_ql);
       prefetch_tensormap(&tm_kl);
     }
+    if (PS) prefetch_tensormap(&tm_ql);
   }
   tc_fence_before();
   __syncthreads();
@@ -1092,15 +1098,19 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL>::THREADS, 1)
       for (it.start(a.L, nb, c_first, c_lo, c_hi); it.valid(); it.next()) {
         const int s = it.k % C::NS;
         if (it.k >= C::NS && !mbar_wait(bar(Q_STAGE_EMPTY + s), ((it.k / C::NS) - 1) & 1)) break;
-        const bool with_q = !it.pre();  // state replay needs K and V only
-        // bytes that land: Q (unless replay) and K, with their lo parts when pre-converted split
+        // Q unless state replay; with P tiles from the P pass (PS), Q only for the cross term (the
+        // first unit of a row block) and K only for the state increment (the last row block)
+        const bool with_q = !it.pre() && (!PS || it.w == 0);
+        const bool with_k = !PS || it.last_row();
+        // bytes that land: Q and K as needed, with their lo parts when pre-converted split
         constexpr int QK_PARTS = (HL && PRE) ? 2 : 1;
-        mbar_arrive_expect_tx(bar(Q_TMA_FULL + s), (with_q ? 2 : 1) * C::QBYTES * QK_PARTS + C::VBYTES);
+        mbar_arrive_expect_tx(bar(Q_TMA_FULL + s), ((with_q ? 1 : 0) + (with_k ? 1 : 0)) * C::QBYTES * QK_PARTS +
+                                                       C::VBYTES + (PS ? C::PBYTES : 0));
         const int tq = it.t0() + it.u * T, tk = it.t0() + it.w * T;
 #pragma unroll
         for (int bx = 0; bx < DK / 64; ++bx) {
           if (with_q) tma_load_4d(sQ(s) + bx * T * 128, &tm_q, bar(Q_TMA_FULL + s), bx * 64, h, tq, b);
-          tma_load_4d(sK(s) + bx * T * 128, &tm_k, bar(Q_TMA_FULL + s), bx * 64, h, tk, b);
+          if (with_k) tma_load_4d(sK(s) + bx * T * 128, &tm_k, bar(Q_TMA_FULL + s), bx * 64, h, tk, b);
           if constexpr (HL && PRE) {
             if (with_q) tma_load_4d(sQl(s) + bx * T * 128, &tm_ql, bar(Q_TMA_FULL + s), bx * 64, h, tq, b);
             tma_load_4d(sKl(s) + bx * T * 128, &tm_kl, bar(Q_TMA_FULL + s), bx * 64, h, tk, b);
@@ -1109,6 +1119,10 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL>::THREADS, 1)
 #pragma unroll
         for (int bx = 0; bx < C::NDV; ++bx)
           tma_load_4d(sV(s) + bx * T * 128, &tm_v, bar(Q_TMA_FULL + s), dvb * DVS + 64 * bx, h, tk, b);
+        if constexpr (PS) {  // the P tile of unit (u, w) of chunk i: ((b h) n_chunks + i) U + u (u + 1) / 2 + w
+          const int tile = ((b * a.heads + h) * a.n_chunks + it.i) * (nb * (nb + 1) / 2) + it.u * (it.u + 1) / 2 + it.w;
+          tma_load_4d(sPs(s), &tm_ql, bar(Q_TMA_FULL + s), 0, 0, tile, 0);
+        }
         issued[s]++;
       }
       // Every load this thread issued must have landed before the CTA may exit.
@@ -1131,7 +1145,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL>::THREADS, 1)
       // unit never holds back the output (and the stage release) of an earlier one.
       auto f_ready = [&](const UnitIter<T, SM>& f) -> bool {
         if (!mbar_test(bar(Q_READY + f.k % C::NS), (f.k / C::NS) & 1)) return false;
-        if (!f.pre() && f.kf() >= C::SBUF &&
+        if (!PS && !f.pre() && f.kf() >= C::SBUF &&
             !mbar_test(bar(Q_S_FREE + (f.kf() % C::SBUF)), ((f.kf() - C::SBUF) / C::SBUF) & 1))
           return false;
         if constexpr (C::RTM) {
@@ -1147,7 +1161,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL>::THREADS, 1)
       auto f_issue = [&](const UnitIter<T, SM>& f) {
         const int s = f.k % C::NS;
         tc_fence_after();
-        if (!f.pre()) {
+        if (!PS && !f.pre()) {
           const uint32_t tS = tmem + C::COL_S + (f.kf() % C::SBUF) * T;
           const uint64_t dq = sdesc_sw128(sQ(s), 16, 1024), dk = sdesc_sw128(sK(s), 16, 1024);
 #pragma unroll
@@ -1210,13 +1224,14 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL>::THREADS, 1)
         if (q.last_row()) mma_commit(bar(Q_R16_FREE + (ri % C::RBUF)));
       };
       auto p_ready = [&](const UnitIter<T, SM>& q) -> bool {
+        if constexpr (PS) return true;  // the P tile came with the unit's stage (F issued after it landed)
         return mbar_test(bar(Q_P_FULL + (q.kf() % C::PBUF)), (q.kf() / C::PBUF) & 1);
       };
       auto p_issue = [&](const UnitIter<T, SM>& q) {
         const int s = q.k % C::NS;
         tc_fence_after();
         const uint32_t tO = tmem + C::COL_O + (q.rb & 1) * DVS;
-        const uint64_t dp = sdesc_sw128(sP(q.kf()), 16, 1024), dv = sdesc_sw128(sV(s), T * 128, 1024);
+        const uint64_t dp = sdesc_sw128(PS ? sPs(s) : sP(q.kf()), 16, 1024), dv = sdesc_sw128(sV(s), T * 128, 1024);
         const uint32_t acc0 = (q.w > 0 || nb == 1) ? 1u : 0u;
 #pragma unroll
         for (int kk = 0; kk < T / 16; ++kk)
@@ -1227,7 +1242,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL>::THREADS, 1)
           for (int kk = 0; kk < T / 16; ++kk)
             mma_f16_ss(tO, dpl + kstep(kk), dv + static_cast<uint64_t>((kk * 2048) >> 4), ID_X, 1u);
         }
-        mma_commit(bar(Q_P_FREE + (q.kf() % C::PBUF)));
+        if (!PS) mma_commit(bar(Q_P_FREE + (q.kf() % C::PBUF)));
         if (q.rb_done()) mma_commit(bar(Q_O_FULL + (q.rb & 1)));
         mma_commit(bar(Q_STAGE_EMPTY + s));
       };
@@ -1792,7 +1807,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL>::THREADS, 1)
     UnitIter<T, SM> it;
     for (it.start(a.L, nb, c_first, c_lo, c_hi); ok && it.valid(); it.next()) {
       if (it.pre()) continue;  // replay units have no scores
-      if (is_epi) {
+      if (is_epi || PS) {  // (with P tiles from the P pass these warps only run the epilogue)
         if (it.rb_done()) ok = epilogue(it.rb, it.i, it.u, it.bl);
         continue;
       }
@@ -1943,6 +1958,117 @@ __global__ void __launch_bounds__(256) tc_convert_kernel(const uint4* __restrict
   report_fp16_range(mx);
 }
 
+// ============================================================================================
+// P pass (chunks of several 64-row sub-blocks, d_k = 256).  Each d_v slice of a head needs the
+// same masked scores P_{u,w} = (Qx_u Kz_w^T) gamma^((u-w-1)T) / sqrt(d_k) (causal mask on the
+// diagonal block u = w) for every unit (u, w) of every chunk; the pipelined kernel computing
+// them itself repeats that work for each of the d_v / 64 slices.  This kernel computes each P
+// tile once, from the conversion pre-pass's copies, into the workspace: fp16, row-major
+// [tile][T][T], tile = ((b heads + h) n_chunks + i) U + u (u + 1) / 2 + w, U = nb (nb + 1) / 2.
+// The pipelined kernel (PS) then loads P by TMA beside V.  One CTA a tile: warp 4 loads Q_u
+// and K_w (TMA, 128-byte swizzle), issues the DK / 16 MMAs into tensor memory; warps 0-3 scale,
+// mask and store the rows.  The causal mask, the row scale and the rounding to fp16 are those
+// of the P warps of the pipelined kernel, so the results are bit-identical.
+// ============================================================================================
+template <int DK, int T>
+__global__ void __launch_bounds__(160, 1) tc_p_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                                      const __grid_constant__ CUtensorMap tm_k, uint4* __restrict__ P,
+                                                      int L, int heads, int n_chunks, int nb, HeadParams hp) {
+  static_assert(T == 64, "P pass: 64-row sub-blocks");
+  constexpr int QB = T * DK * 2;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_addr(smem_raw);
+  const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (sbase - raw_addr);
+  const uint32_t sQ = sbase, sK = sbase + QB;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + 2 * QB);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2);
+  const int U = nb * (nb + 1) / 2;
+  const int unit = blockIdx.x, i = blockIdx.y, bh = blockIdx.z;
+  int u = 0;
+  while ((u + 1) * (u + 2) / 2 <= unit) ++u;
+  const int w = unit - u * (u + 1) / 2;
+  const int t0 = i * nb * T;
+  if (t0 + u * T >= L) return;  // a row block past the end of a short last chunk: never read
+  const int h = bh % heads, b = bh / heads;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_addr(bars), 1);
+    mbar_init(smem_addr(bars + 1), 1);
+    fence_mbar_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(smem_addr(tmem_holder), 64);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const float log2g = hp.log2g[h];
+  if (warp == 4) {
+    if (lane == 0) {
+      prefetch_tensormap(&tm_q);
+      prefetch_tensormap(&tm_k);
+      mbar_arrive_expect_tx(smem_addr(bars), 2 * QB);
+#pragma unroll
+      for (int bx = 0; bx < DK / 64; ++bx) {
+        tma_load_4d(sQ + bx * T * 128, &tm_q, smem_addr(bars), bx * 64, h, t0 + u * T, b);
+        tma_load_4d(sK + bx * T * 128, &tm_k, smem_addr(bars), bx * 64, h, t0 + w * T, b);
+      }
+      // the loads are waited for with the full budget: they were issued and always land
+      if (mbar_wait(smem_addr(bars), 0, kDrainBudget)) {
+        tc_fence_after();
+        constexpr uint32_t ID_S = idesc_f16_f32(T, T, 0, 0);
+        const uint64_t dq = sdesc_sw128(sQ, 16, 1024), dk = sdesc_sw128(sK, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < DK / 16; ++kk) {
+          const uint64_t ks = static_cast<uint64_t>(((kk / 4) * T * 128 + (kk % 4) * 32) >> 4);
+          mma_f16_ss(tmem, dq + ks, dk + ks, ID_S, kk > 0);
+        }
+      }
+      mma_commit(smem_addr(bars + 1));  // (after no MMA it arrives at once)
+      mbar_wait(smem_addr(bars + 1), 0, kDrainBudget);
+    }
+  } else {
+    // rows of the M = 64 accumulator: lanes 0-15 of each warp's 32-lane quarter
+    const uint32_t lane_off = static_cast<uint32_t>(32 * warp) << 16;
+    const int my_row = lane < 16 ? 16 * warp + lane : -1;
+    float pmx = 0.f;
+    if (__all_sync(0xffffffffu, mbar_wait(smem_addr(bars + 1), 0))) {
+      tc_fence_after();
+      const float pf = exp2f(static_cast<float>((u - w - 1) * T) * log2g) * rsqrtf(static_cast<float>(DK));
+      const bool diag = (u == w);
+      uint32_t r[4][16];
+      tmem_ld_wait(tmem + lane_off, r);
+      if (my_row >= 0) {
+        const int64_t tile = (static_cast<int64_t>(bh) * n_chunks + i) * U + unit;
+        uint4* dst = P + (tile * T + my_row) * (T * 2 / 16);
+#pragma unroll
+        for (int c8 = 0; c8 < T / 8; ++c8) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c0 = 8 * c8 + 2 * e;
+            const float p0 = (!diag || c0 <= my_row) ? __uint_as_float(r[c0 / 16][c0 % 16]) * pf : 0.f;
+            const float p1 = (!diag || c0 + 1 <= my_row) ? __uint_as_float(r[(c0 + 1) / 16][(c0 + 1) % 16]) * pf : 0.f;
+            pmx = absmax(absmax(pmx, p0), p1);
+            pk[e] = pack_f16x2(p0, p1);
+          }
+          dst[c8] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+      }
+    }
+    report_fp16_range(pmx);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 64);
+  }
+}
+
 // ---- host side -------------------------------------------------------------------------------
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -1970,6 +2096,20 @@ bool make_map(CUtensorMap* m, const void* base, int64_t b, int64_t L, int64_t h,
   cuuint64_t strides[3] = {static_cast<cuuint64_t>(d * 2), static_cast<cuuint64_t>(h * d * 2),
                            static_cast<cuuint64_t>(L * h * d * 2)};
   cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(T), 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Map over P tiles [tile][T][T] fp16 (2-byte elements), box of one T x T tile, 128-byte swizzle.
+bool make_map_p(CUtensorMap* m, const void* base, int64_t tiles, int T) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(tiles), 1};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(T * 2), static_cast<cuuint64_t>(T * T * 2),
+                           static_cast<cuuint64_t>(tiles * T * T * 2)};
+  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(T), 1, 1};
   cuuint32_t es[4] = {1, 1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -2031,6 +2171,22 @@ PreCopies pre_copies(const RetentionCall& c) {
 // reconversion of chunks of nb >= 2 sub-blocks.  Not combined with sequence segments.
 bool pre_convert_applies(const RetentionCall& c, int nb, int n_seg) {
   return nb >= 2 && n_seg < 2 && c.ws && c.ws_bytes >= pre_copy_bytes(c.dims, c.precise);
+}
+
+// P pass (d_k = 256, 64-row sub-blocks, chunks of several of them, single operands, no fused
+// epilogue, no segments): the P tiles of every unit of every chunk, after the fp16 copies.
+int64_t p_tiles(const Dims& d, int64_t chunk, int T) {
+  const int64_t nb = chunk / T, n_chunks = (d.seqlen + chunk - 1) / chunk;
+  return d.batch * d.heads * n_chunks * (nb * (nb + 1) / 2);
+}
+size_t p_tile_bytes(const Dims& d, int64_t chunk, int T) {
+  return align256(static_cast<size_t>(p_tiles(d, chunk, T)) * T * T * 2);
+}
+bool p_pass_applies(const RetentionCall& c, int T, int nb, int n_seg) {
+  if (c.dims.d_k != 256 || T != 64 || nb < 2 || c.precise || c.gate || n_seg >= 2 || !c.ws) return false;
+  const int64_t n_chunks = (c.dims.seqlen + c.chunk - 1) / c.chunk;
+  if (n_chunks > 65535 || c.dims.batch * c.dims.heads > 65535 || p_tiles(c.dims, c.chunk, T) >= (1LL << 31)) return false;
+  return c.ws_bytes >= pre_copy_bytes(c.dims, false) + p_tile_bytes(c.dims, c.chunk, T);
 }
 
 // 128-column d_v slices share S and the Q/K conversion across twice the output columns
@@ -2265,6 +2421,28 @@ cudaError_t launch_pipe(const RetentionCall& c, const HeadParams& hp, cudaStream
         CUtensorMap pm[5];
         cudaError_t e = run_convert<DK, T, false>(c, hp, s, pre_copies(c), pm);
         if (e != cudaSuccess) return e;
+        if constexpr (DK == 256 && T == 64 && DVS == 64) {
+          if (p_pass_applies(c, T, nb, as.n_seg)) {
+            // P tiles once per head (P pass), then the pipelined kernel loads them beside V
+            void* ptiles = static_cast<char*>(c.ws) + pre_copy_bytes(c.dims, false);
+            const int64_t n_chunks = (c.dims.seqlen + c.chunk - 1) / c.chunk;
+            const int U = nb * (nb + 1) / 2;
+            constexpr int PSMEM = 2 * T * DK * 2 + 1024 + 64;
+            e = cudaFuncSetAttribute(tc_p_kernel<DK, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, PSMEM);
+            if (e != cudaSuccess) return e;
+            tc_p_kernel<DK, T><<<dim3(U, static_cast<unsigned>(n_chunks), static_cast<unsigned>(c.dims.batch * c.dims.heads)),
+                                 160, PSMEM, s>>>(pm[0], pm[1], static_cast<uint4*>(ptiles),
+                                                  static_cast<int>(c.dims.seqlen), static_cast<int>(c.dims.heads),
+                                                  static_cast<int>(n_chunks), nb, hp);
+            e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+            if (!make_map_p(&pm[3], ptiles, p_tiles(c.dims, c.chunk, T), T)) return cudaErrorInvalidValue;
+            using CPS = Cfg3<DK, T, DVS, true, false, false, true>;
+            static_assert(CPS::FITS, "pipelined kernel with P tiles does not fit this tile");
+            return launch_kernel(tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_NONE, true, false, Tout, false, true>, grid,
+                                 CPS::THREADS, CPS::SMEM, s, pm, as, hp, 0);
+          }
+        }
         return launch_kernel(tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_NONE, true, false, Tout>, grid, CfP::THREADS,
                              CfP::SMEM, s, pm, as, hp, 0);
       }
@@ -2492,7 +2670,8 @@ int tc_chunkwise_launches(const RetentionCall& c) {
   // fused epilogue and split operands: never segmented
   if (c.gate || c.precise) return pre_convert_applies(c, nb, 1) ? 2 : 1;
   const int max_states = plan_call(c, ctas, sm_count(), as);
-  if (dvs == 64 && pre_convert_applies(c, nb, as.n_seg)) return 2;  // conversion pre-pass + kernel
+  if (dvs == 64 && pre_convert_applies(c, nb, as.n_seg))  // conversion pre-pass (+ P pass) + kernel
+    return p_pass_applies(c, T, nb, as.n_seg) ? 3 : 2;
   return (as.n_seg > 1 && max_states >= 1) ? 2 : 1;
 }
 

@@ -273,10 +273,17 @@ retnet_status_t retnet_chunkwise_workspace_size(retnet_dims_t dims, size_t* byte
   const size_t tok = static_cast<size_t>(dims.batch) * static_cast<size_t>(dims.seqlen) * static_cast<size_t>(dims.heads);
   auto a256 = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
   const size_t copies = 4 * a256(tok * static_cast<size_t>(dims.d_k) * 2) + a256(tok * static_cast<size_t>(dims.d_v) * 2);
+  // with d_k = 256 the P pass's tiles after the single-operand copies, at most (chunks of 512)
+  // ceil(seqlen / 512) * 36 tiles of 64 x 64 fp16 per (batch, head)
+  const size_t ptiles = dims.d_k == 256 ? a256(static_cast<size_t>(dims.batch) * static_cast<size_t>(dims.heads) *
+                                                static_cast<size_t>((dims.seqlen + 511) / 512) * 36 * 64 * 64 * 2)
+                                        : 0;
+  const size_t single = 2 * a256(tok * static_cast<size_t>(dims.d_k) * 2) + a256(tok * static_cast<size_t>(dims.d_v) * 2);
+  const size_t copies_all = copies > single + ptiles ? copies : single + ptiles;
   // plus, in front, the R~ row factors (fp32 [batch][seqlen][heads]) and the key-sum pass's
   // segment values (fp32 [batch * heads][64][d_k])
   const Dims d{dims.batch, dims.seqlen, dims.heads, dims.d_k, dims.d_v};
-  *bytes = rden_region_bytes(d) + (states > copies ? states : copies);
+  *bytes = rden_region_bytes(d) + (states > copies_all ? states : copies_all);
   return RETNET_OK;
 }
 

@@ -120,12 +120,15 @@ def test_chunkwise_workspace_entry_points(lib):
     """Workspace size is the documented bound; the workspace variant validates like the plain call
     and rejects a misaligned workspace before touching a device."""
     a256 = lambda x: (x + 255) // 256 * 256
-    for dims in ((2, 100, 3, 128, 64), (1, 4096, 2, 64, 128)):
+    for dims in ((2, 100, 3, 128, 64), (1, 4096, 2, 64, 128), (2, 1000, 3, 256, 128), (2, 8192, 16, 256, 512)):
         b, L, h, dk, dv = dims
         states = 6 * b * h * dk * dv * 4
         copies = 4 * a256(b * L * h * dk * 2) + a256(b * L * h * dv * 2)  # q~, k~ hi and lo; v
+        # d_k 256: the P pass's tiles (at most 36 tiles of 64 x 64 fp16 per 512 tokens) after single copies
+        ptiles = a256(b * h * ((L + 511) // 512) * 36 * 64 * 64 * 2) if dk == 256 else 0
+        single = 2 * a256(b * L * h * dk * 2) + a256(b * L * h * dv * 2)
         rden = a256(b * L * h * 4) + a256(b * h * dk * 64 * 4)  # R~ row factors and key-sum segments, in front
-        assert rn.retnet_chunkwise_workspace_size(dims) == rden + max(states, copies)
+        assert rn.retnet_chunkwise_workspace_size(dims) == rden + max(states, copies, single + ptiles)
     assert rn.retnet_chunkwise_workspace_size((0, 0, 0, 0, 0)) == 0
     out = ctypes.c_size_t(0)
     assert lib.retnet_chunkwise_workspace_size(rn.Dims(1, 8, -2, 4, 4), ctypes.byref(out)) == 2

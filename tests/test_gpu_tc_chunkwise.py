@@ -421,3 +421,39 @@ def test_bounded_waits_give_up_and_recover():
     torch.cuda.synchronize()
     assert torch.equal(o_again, o_ref)
     assert rn.retnet_debug_wait_timeouts(clear=True) == 0
+
+
+@pytest.mark.parametrize("dv,B,L,pos0,with_state", [(64, 128, 300, 0, False), (192, 256, 1100, 7, True),
+                                                    (128, 512, 513, 0, True), (64, 512, 129, 3, False),
+                                                    (512, 128, 400, 0, True)])
+def test_tc_p_pass_matches_oracle(dv, B, L, pos0, with_state):
+    """d_k 256 with chunks of several 64-row sub-blocks: the P pass computes every masked score
+    tile once per head into the workspace and the pipelined kernel loads them beside V (three
+    launches: conversion pre-pass, P pass, kernel).  Against the oracle, and bit-identical to the
+    same call with a workspace one byte too small for the P tiles (the kernel then forms P itself
+    from the same operands, in the same order)."""
+    b, h, dk = 2, 3, 256
+    q, k, v = si.qkv(b, L, h, dk, dv, 1800 + B + L, "bf16")
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+    S0 = si.decode_state(b, h, dk, dv, 1801, std=0.05) if with_state else None
+    ref, Sref, _ = oracle.chunkwise(q, k, v, g, B, th, pos0, FLAGS, state_in=S0)
+    full = rn.retnet_chunkwise_workspace_size((b, L, h, dk, dv))
+    a256 = lambda x: (x + 255) // 256 * 256
+    copies = 2 * a256(b * L * h * dk * 2) + a256(b * L * h * dv * 2)
+    tiles = b * h * ((L + B - 1) // B) * ((B // 64) * (B // 64 + 1) // 2)
+    small = copies + a256(tiles * 64 * 64 * 2) - 1  # room for the copies, not for the P tiles
+    assert rn.retnet_chunkwise_launches((b, L, h, dk), dv, rn.BF16, FLAGS, B, g, full) == 3
+    assert rn.retnet_chunkwise_launches((b, L, h, dk), dv, rn.BF16, FLAGS, B, g, small) == 2
+    outs = []
+    for nbytes in (full, small):
+        ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+        o = torch.empty(b, L, h, dv, device="cuda")
+        so = torch.empty(b, h, dk, dv, device="cuda")
+        rn.retnet_retention_chunkwise_ws(dev(q), dev(k), dev(v), o, g, th, pos0, FLAGS, B,
+                                         None if S0 is None else dev(S0), so, workspace=ws)
+        torch.cuda.synchronize()
+        outs.append((o, so))
+    e, es = err(outs[0][0], ref), err(outs[0][1], Sref)
+    print(f"P pass dv={dv} B={B} L={L}: out {e:.3e}, state {es:.3e}")
+    assert e <= TOL_BF16 and es <= TOL_BF16
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
