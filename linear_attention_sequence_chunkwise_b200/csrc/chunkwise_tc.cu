@@ -639,9 +639,12 @@ struct Cfg3 {
   // product of two of them keeps ~22 significant bits; the stage holds [Q hi][K hi][V][Q lo][K lo].
   static constexpr int QT = HL ? 2 : 1;
   static constexpr int PBYTES = T * T * 2;
-  // PS (P tiles computed by the P pass): the stage also holds the unit's P tile, [Q][K][V][P],
-  // and there is no P buffer of the P warps.
-  static constexpr int STAGE = 2 * QBYTES * QT + VBYTES + (PS ? PBYTES : 0);
+  // PS (P tiles computed by the P pass): a stage holds the unit's V and P tiles, [V][P]; Q (for
+  // the cross term, once a row block) and K (for the state increment, last row block) get areas
+  // of their own, two slots each; there is no P buffer of the P warps.
+  static constexpr int QSLOTS = 2, KSLOTS = 2;
+  static constexpr int AREAS = PS ? (QSLOTS + KSLOTS) * QBYTES : 0;
+  static constexpr int STAGE = PS ? VBYTES + PBYTES : 2 * QBYTES * QT + VBYTES;
   static constexpr int RBYTES = DK * DVS * 2;
   static constexpr int PB = PS ? 0 : PBYTES * QT;  // one P buffer (hi, then lo)
   static constexpr int RB = RBYTES * QT;  // one fp16 state buffer (hi, then lo)
@@ -659,7 +662,7 @@ struct Cfg3 {
   static constexpr int TMEM_COLS = USED <= 128 ? 128 : (USED <= 256 ? 256 : 512);
   // shared memory: stages, P[PBUF], R16[RBUF], rotation tables (Q and K, double-buffered),
   // barriers.  A second fp16 state buffer is kept only while three stages still fit.
-  static constexpr int NBARS = 3 * 4 + 2 * 10 + 1 + 2 + 2;
+  static constexpr int NBARS = 3 * 6 + 2 * 10 + 1 + 2 + 2 + 4 * 2;
   // FUSE (GroupNorm + gate in the epilogue): per-row (mean, M2) of every CTA of the cluster
   // (the d_v slices of a head, at most kMaxCluster), double-buffered by row block.
   static constexpr int XBYTES = FUSE ? 2 * kMaxCluster * T * 8 : 0;
@@ -669,7 +672,7 @@ struct Cfg3 {
   // Buffer counts.  A second fp16 state buffer takes the cross term of chunk i off the state
   // group's path to chunk i + 1 (with one buffer the copy of R_i waits for that MMA), so it is
   // preferred as long as three stages remain, over a second P buffer.
-  static constexpr int ns_for(int pbuf, int rbuf) { return (BUDGET - (pbuf * PB + rbuf * RB + TAIL)) / STAGE; }
+  static constexpr int ns_for(int pbuf, int rbuf) { return (BUDGET - (pbuf * PB + rbuf * RB + AREAS + TAIL)) / STAGE; }
   static constexpr int PBUF0 = (2 * STAGE + 2 * PB + RB + TAIL <= BUDGET) ? 2 : 1;
   static constexpr int NS_R2 = ns_for(PBUF0, 2);
   static constexpr int NS_R1 = ns_for(PBUF0, 1);
@@ -677,9 +680,10 @@ struct Cfg3 {
   static constexpr bool TRADE = RBUF0 == 1 && PBUF0 == 2 && ns_for(1, 2) >= 3;
   static constexpr int PBUF = TRADE ? 1 : PBUF0;
   static constexpr int RBUF = TRADE ? 2 : RBUF0;
-  static constexpr int FIXED = PBUF * PB + RBUF * RB + TAIL;
+  static constexpr int FIXED = PBUF * PB + RBUF * RB + AREAS + TAIL;
   static constexpr int NS_FIT = (BUDGET - FIXED) / STAGE;
-  static constexpr int NS = NS_FIT > 4 ? 4 : NS_FIT;
+  static constexpr int NS_MAX = PS ? 6 : 4;  // stage barriers exist for six
+  static constexpr int NS = NS_FIT > NS_MAX ? NS_MAX : NS_FIT;
   static constexpr int SMEM = NS * STAGE + FIXED + 1024;
   // split operands at d_k = 256 leave room for one stage only (the units then run in turn)
   static constexpr bool FITS = NS >= (HL ? 1 : 2) && USED <= 512 && (DVS == 64 || DVS == 128) && (!RTM || DRBUF == 1) &&
@@ -691,22 +695,26 @@ struct Cfg3 {
 
 // Barrier slots of the pipelined kernel ([2] = indexed by buffer).
 enum : int {
-  Q_TMA_FULL = 0,      // [4] stage landed (TMA transaction count)
-  Q_CONV_FULL = 4,     // [4] stage converted (128 converters)
-  Q_STAGE_EMPTY = 8,   // [4] stage consumed (MMA commit)
-  Q_S_FULL = 12,       // [2] S'' of a unit in TMEM (commit)
-  Q_S_FREE = 14,       // [2] S read by the P group
-  Q_P_FULL = 16,       // [2] P in shared memory
-  Q_P_FREE = 18,       // [2] P consumed by the P V product (commit)
-  Q_DR_FULL = 20,      // [2] state increment Kz^T V in TMEM (commit)
-  Q_DR_FREE = 22,      // [2] increment read by the state group
-  Q_R16_FULL = 24,     // [2] fp16 chunk-start state written (state group)
-  Q_R16_FREE = 26,     // [2] every cross term of that chunk done (commit)
-  Q_O_FULL = 28,       // [2] O (and X) of a row block complete (commit)
-  Q_O_FREE = 30,       // [2] O/X read by the epilogue
-  Q_DRAIN = 32,
-  Q_TAB = 33,          // [2] rotation tables written (converters)
-  Q_XFULL = 35         // [2] FUSE: the row statistics of every CTA of the cluster have landed here
+  Q_TMA_FULL = 0,      // [6] stage landed (TMA transaction count)
+  Q_CONV_FULL = 6,     // [6] stage converted (128 converters)
+  Q_STAGE_EMPTY = 12,  // [6] stage consumed (MMA commit)
+  Q_S_FULL = 18,       // [2] S'' of a unit in TMEM (commit)
+  Q_S_FREE = 20,       // [2] S read by the P group
+  Q_P_FULL = 22,       // [2] P in shared memory
+  Q_P_FREE = 24,       // [2] P consumed by the P V product (commit)
+  Q_DR_FULL = 26,      // [2] state increment Kz^T V in TMEM (commit)
+  Q_DR_FREE = 28,      // [2] increment read by the state group
+  Q_R16_FULL = 30,     // [2] fp16 chunk-start state written (state group)
+  Q_R16_FREE = 32,     // [2] every cross term of that chunk done (commit)
+  Q_O_FULL = 34,       // [2] O (and X) of a row block complete (commit)
+  Q_O_FREE = 36,       // [2] O/X read by the epilogue
+  Q_DRAIN = 38,
+  Q_TAB = 39,          // [2] rotation tables written (converters)
+  Q_XFULL = 41,        // [2] FUSE: the row statistics of every CTA of the cluster have landed here
+  Q_QA_FULL = 43,      // [2] PS: Q tile of a row block in its area slot (TMA)
+  Q_QA_FREE = 45,      // [2] PS: that row block's cross term done (commit)
+  Q_KA_FULL = 47,      // [2] PS: K tile of a last-row unit in its area slot (TMA)
+  Q_KA_FREE = 49       // [2] PS: that unit's state increment done (commit)
 };
 
 __device__ __forceinline__ float2 cpow_mul(float2 base, float2 step, int n) {
@@ -1025,7 +1033,8 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL, PS>::THREADS, 
 
   const uint32_t sP0 = sbase + C::NS * C::STAGE;
   const uint32_t sR0 = sP0 + C::PBUF * C::PB;
-  const int tail_off = C::NS * C::STAGE + C::PBUF * C::PB + C::RBUF * C::RB;
+  const uint32_t sA0 = sR0 + C::RBUF * C::RB;  // PS: Q area slots, then K area slots
+  const int tail_off = C::NS * C::STAGE + C::PBUF * C::PB + C::RBUF * C::RB + C::AREAS;
   float2* tab = reinterpret_cast<float2*>(gbase + tail_off);
   uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + tail_off + C::TABBYTES);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::NBARS);
@@ -1038,22 +1047,30 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL, PS>::THREADS, 
   const int n_cl = a.dv / DVS;  // cluster size under FUSE: every d_v slice of the head
   auto sQ = [&](int s) { return sbase + s * C::STAGE; };
   auto sK = [&](int s) { return sbase + s * C::STAGE + C::QBYTES; };
-  auto sV = [&](int s) { return sbase + s * C::STAGE + 2 * C::QBYTES; };
+  auto sV = [&](int s) { return sbase + s * C::STAGE + (PS ? 0 : 2 * C::QBYTES); };
+  auto sQa = [&](int slot) { return sA0 + slot * C::QBYTES; };                 // PS
+  auto sKa = [&](int slot) { return sA0 + (C::QSLOTS + slot) * C::QBYTES; };   // PS
   // HL: lo parts of Q and K after V in the stage; P and the state copy keep their lo part
   // right after the hi part of the same buffer
   auto sQl = [&](int s) { return sbase + s * C::STAGE + 2 * C::QBYTES + C::VBYTES; };
   auto sKl = [&](int s) { return sbase + s * C::STAGE + 3 * C::QBYTES + C::VBYTES; };
-  auto sPs = [&](int s) { return sbase + s * C::STAGE + 2 * C::QBYTES + C::VBYTES; };  // PS: the unit's P tile
+  auto sPs = [&](int s) { return sbase + s * C::STAGE + C::VBYTES; };  // PS: the unit's P tile
   auto sP = [&](int k) { return sP0 + (k % C::PBUF) * C::PB; };
   auto sR = [&](int i) { return sR0 + (i % C::RBUF) * C::RB; };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 4; ++s) {
+    for (int s = 0; s < C::NS_MAX; ++s) {
       mbar_init(bar(Q_TMA_FULL + s), 1);
       if (!PRE) mbar_init(bar(Q_CONV_FULL + s), C::NCONV);
       mbar_init(bar(Q_STAGE_EMPTY + s), 1);
     }
     for (int k = 0; k < 2; ++k) {
+      if (PS) {
+        mbar_init(bar(Q_QA_FULL + k), 1);
+        mbar_init(bar(Q_QA_FREE + k), 1);
+        mbar_init(bar(Q_KA_FULL + k), 1);
+        mbar_init(bar(Q_KA_FREE + k), 1);
+      }
       mbar_init(bar(Q_S_FULL + k), 1);
       mbar_init(bar(Q_S_FREE + k), 128);
       mbar_init(bar(Q_P_FULL + k), 128);
@@ -1092,25 +1109,64 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL, PS>::THREADS, 
 
   if (warp == C::WARP_TMA) {
     // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    if (PS && lane == 0) {
+      // P tiles from the P pass: every unit's stage takes V_w and P_{u,w}; the first unit of a
+      // row block loads Q_u into a Q slot, a unit of the last row block K_w into a K slot.
+      int issued[C::NS_MAX] = {}, q_issued[2] = {0, 0}, k_issued[2] = {0, 0};
+      UnitIter<T, SM> it;
+      for (it.start(a.L, nb, c_first, c_lo, c_hi); it.valid(); it.next()) {
+        const int s = it.k % C::NS;
+        if (it.k >= C::NS && !mbar_wait(bar(Q_STAGE_EMPTY + s), ((it.k / C::NS) - 1) & 1)) break;
+        const int tq = it.t0() + it.u * T, tk = it.t0() + it.w * T;
+        mbar_arrive_expect_tx(bar(Q_TMA_FULL + s), C::VBYTES + C::PBYTES);
+#pragma unroll
+        for (int bx = 0; bx < C::NDV; ++bx)
+          tma_load_4d(sV(s) + bx * T * 128, &tm_v, bar(Q_TMA_FULL + s), dvb * DVS + 64 * bx, h, tk, b);
+        // the P tile of unit (u, w) of chunk i: ((b h) n_chunks + i) U + u (u + 1) / 2 + w
+        const int tile = ((b * a.heads + h) * a.n_chunks + it.i) * (nb * (nb + 1) / 2) + it.u * (it.u + 1) / 2 + it.w;
+        tma_load_4d(sPs(s), &tm_ql, bar(Q_TMA_FULL + s), 0, 0, tile, 0);
+        issued[s]++;
+        if (it.w == 0) {
+          const int qs = it.rb % 2;
+          if (it.rb >= 2 && !mbar_wait(bar(Q_QA_FREE + qs), ((it.rb / 2) - 1) & 1)) break;
+          mbar_arrive_expect_tx(bar(Q_QA_FULL + qs), C::QBYTES);
+#pragma unroll
+          for (int bx = 0; bx < DK / 64; ++bx)
+            tma_load_4d(sQa(qs) + bx * T * 128, &tm_q, bar(Q_QA_FULL + qs), bx * 64, h, tq, b);
+          q_issued[qs]++;
+        }
+        if (it.last_row()) {
+          const int ks = it.dr % 2;
+          if (it.dr >= 2 && !mbar_wait(bar(Q_KA_FREE + ks), ((it.dr / 2) - 1) & 1)) break;
+          mbar_arrive_expect_tx(bar(Q_KA_FULL + ks), C::QBYTES);
+#pragma unroll
+          for (int bx = 0; bx < DK / 64; ++bx)
+            tma_load_4d(sKa(ks) + bx * T * 128, &tm_k, bar(Q_KA_FULL + ks), bx * 64, h, tk, b);
+          k_issued[ks]++;
+        }
+      }
+      // Every load this thread issued must have landed before the CTA may exit.
+      for (int s = 0; s < C::NS; ++s)
+        if (issued[s] > 0) mbar_wait(bar(Q_TMA_FULL + s), (issued[s] - 1) & 1, kDrainBudget);
+      for (int j = 0; j < 2; ++j) {
+        if (q_issued[j] > 0) mbar_wait(bar(Q_QA_FULL + j), (q_issued[j] - 1) & 1, kDrainBudget);
+        if (k_issued[j] > 0) mbar_wait(bar(Q_KA_FULL + j), (k_issued[j] - 1) & 1, kDrainBudget);
+      }
+    } else if (lane == 0) {
       int issued[4] = {0, 0, 0, 0};
       UnitIter<T, SM> it;
       for (it.start(a.L, nb, c_first, c_lo, c_hi); it.valid(); it.next()) {
         const int s = it.k % C::NS;
         if (it.k >= C::NS && !mbar_wait(bar(Q_STAGE_EMPTY + s), ((it.k / C::NS) - 1) & 1)) break;
-        // Q unless state replay; with P tiles from the P pass (PS), Q only for the cross term (the
-        // first unit of a row block) and K only for the state increment (the last row block)
-        const bool with_q = !it.pre() && (!PS || it.w == 0);
-        const bool with_k = !PS || it.last_row();
-        // bytes that land: Q and K as needed, with their lo parts when pre-converted split
+        const bool with_q = !it.pre();  // state replay needs K and V only
+        // bytes that land: Q (unless replay) and K, with their lo parts when pre-converted split
         constexpr int QK_PARTS = (HL && PRE) ? 2 : 1;
-        mbar_arrive_expect_tx(bar(Q_TMA_FULL + s), ((with_q ? 1 : 0) + (with_k ? 1 : 0)) * C::QBYTES * QK_PARTS +
-                                                       C::VBYTES + (PS ? C::PBYTES : 0));
+        mbar_arrive_expect_tx(bar(Q_TMA_FULL + s), (with_q ? 2 : 1) * C::QBYTES * QK_PARTS + C::VBYTES);
         const int tq = it.t0() + it.u * T, tk = it.t0() + it.w * T;
 #pragma unroll
         for (int bx = 0; bx < DK / 64; ++bx) {
           if (with_q) tma_load_4d(sQ(s) + bx * T * 128, &tm_q, bar(Q_TMA_FULL + s), bx * 64, h, tq, b);
-          if (with_k) tma_load_4d(sK(s) + bx * T * 128, &tm_k, bar(Q_TMA_FULL + s), bx * 64, h, tk, b);
+          tma_load_4d(sK(s) + bx * T * 128, &tm_k, bar(Q_TMA_FULL + s), bx * 64, h, tk, b);
           if constexpr (HL && PRE) {
             if (with_q) tma_load_4d(sQl(s) + bx * T * 128, &tm_ql, bar(Q_TMA_FULL + s), bx * 64, h, tq, b);
             tma_load_4d(sKl(s) + bx * T * 128, &tm_kl, bar(Q_TMA_FULL + s), bx * 64, h, tk, b);
@@ -1119,10 +1175,6 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL, PS>::THREADS, 
 #pragma unroll
         for (int bx = 0; bx < C::NDV; ++bx)
           tma_load_4d(sV(s) + bx * T * 128, &tm_v, bar(Q_TMA_FULL + s), dvb * DVS + 64 * bx, h, tk, b);
-        if constexpr (PS) {  // the P tile of unit (u, w) of chunk i: ((b h) n_chunks + i) U + u (u + 1) / 2 + w
-          const int tile = ((b * a.heads + h) * a.n_chunks + it.i) * (nb * (nb + 1) / 2) + it.u * (it.u + 1) / 2 + it.w;
-          tma_load_4d(sPs(s), &tm_ql, bar(Q_TMA_FULL + s), 0, 0, tile, 0);
-        }
         issued[s]++;
       }
       // Every load this thread issued must have landed before the CTA may exit.
@@ -1145,6 +1197,8 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL, PS>::THREADS, 
       // unit never holds back the output (and the stage release) of an earlier one.
       auto f_ready = [&](const UnitIter<T, SM>& f) -> bool {
         if (!mbar_test(bar(Q_READY + f.k % C::NS), (f.k / C::NS) & 1)) return false;
+        // PS: the unit's K tile in its slot (state increment of the last row block)
+        if (PS && f.last_row() && !mbar_test(bar(Q_KA_FULL + f.dr % 2), (f.dr / 2) & 1)) return false;
         if (!PS && !f.pre() && f.kf() >= C::SBUF &&
             !mbar_test(bar(Q_S_FREE + (f.kf() % C::SBUF)), ((f.kf() - C::SBUF) / C::SBUF) & 1))
           return false;
@@ -1177,7 +1231,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL, PS>::THREADS, 
         }
         if (f.last_row()) {
           const uint32_t tD = tmem + C::COL_DR + (f.dr % C::DRBUF) * C::RBLK * DVS;
-          const uint64_t dkm = sdesc_sw128(sK(s), T * 128, 1024), dv = sdesc_sw128(sV(s), T * 128, 1024);
+          const uint64_t dkm = sdesc_sw128(PS ? sKa(f.dr % 2) : sK(s), T * 128, 1024), dv = sdesc_sw128(sV(s), T * 128, 1024);
 #pragma unroll
           for (int blk = 0; blk < C::RBLK; ++blk)
 #pragma unroll
@@ -1194,12 +1248,14 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL, PS>::THREADS, 
                            dv + static_cast<uint64_t>((ks * 2048) >> 4), ID_R, 1u);
           }
           mma_commit(bar(Q_DR_FULL + (f.dr % C::DRBUF)));
+          if (PS) mma_commit(bar(Q_KA_FREE + f.dr % 2));
         }
         if (f.pre()) mma_commit(bar(Q_STAGE_EMPTY + s));  // a replay unit has no P V
       };
       auto x_ready = [&](const UnitIter<T, SM>& q) -> bool {
         const int ri = q.i - c_lo;  // fp16 state copies are written for output chunks only
         if (!mbar_test(bar(Q_R16_FULL + (ri % C::RBUF)), (ri / C::RBUF) & 1)) return false;
+        if (PS && !mbar_test(bar(Q_QA_FULL + q.rb % 2), (q.rb / 2) & 1)) return false;  // the row block's Q
         return q.rb < 2 || mbar_test(bar(Q_O_FREE + (q.rb & 1)), ((q.rb - 2) >> 1) & 1);
       };
       auto x_issue = [&](const UnitIter<T, SM>& q) {
@@ -1208,7 +1264,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL, PS>::THREADS, 
         const uint32_t tO = tmem + C::COL_O + (q.rb & 1) * DVS;
         const uint32_t tX = (C::XBUF > 0 && nb > 1) ? tmem + C::COL_X + (q.rb & 1) * DVS : tO;
         const int ri = q.i - c_lo;
-        const uint64_t dq = sdesc_sw128(sQ(s), 16, 1024), dr = sdesc_sw128(sR(ri), DK * 128, 1024);
+        const uint64_t dq = sdesc_sw128(PS ? sQa(q.rb % 2) : sQ(s), 16, 1024), dr = sdesc_sw128(sR(ri), DK * 128, 1024);
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk)
           mma_f16_ss(tX, dq + kstep(kk), dr + static_cast<uint64_t>((kk * 2048) >> 4), ID_X, kk > 0);
@@ -1221,6 +1277,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL, PS>::THREADS, 
           for (int kk = 0; kk < DK / 16; ++kk)
             mma_f16_ss(tX, dq + kstep(kk), drl + static_cast<uint64_t>((kk * 2048) >> 4), ID_X, 1u);
         }
+        if (PS) mma_commit(bar(Q_QA_FREE + q.rb % 2));
         if (q.last_row()) mma_commit(bar(Q_R16_FREE + (ri % C::RBUF)));
       };
       auto p_ready = [&](const UnitIter<T, SM>& q) -> bool {
