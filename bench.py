@@ -343,7 +343,7 @@ def bench_backward(rn, device, stream, steps, peaks):
     tf = flops / secs / 1e12
     return {"workload": "backward_" + c["workload"], "us_per_step": secs * 1e6, "tokens_per_s": b * L / secs,
             "tflops": tf, "frac_bf16_peak": tf / peaks["bf16"],
-            "kernel": "tcgen05 (three chunkwise runs, hi|lo values)" if path == 1 else "fp32 CUDA cores",
+            "kernel": "tcgen05 (three chunkwise runs, fp16 value rows)" if path == 1 else "fp32 CUDA cores",
             "workspace_bytes": ws.numel(), "launches_per_step": launches, "gpu_launches": launches * steps}
 
 

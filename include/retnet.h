@@ -324,9 +324,10 @@ RETNET_API retnet_status_t retnet_msr_chunkwise(const void* q, const void* k, co
  * retnet_backward_workspace_size bytes run on the tensor cores: each gradient sum has the shape
  * of a retention output (dq: query dO, key v, value k~; dk: read backwards, query v, key dO,
  * value f q~; dv: backwards, query k, key q, value f dO), so three runs of the chunkwise kernel
- * compute them: k~, f q~ and f dO, which are not bf16 numbers, go in as two bf16 parts (hi +
- * lo) side by side in a value of twice the width (max|err|/rms <= 1e-2).  Every other call runs
- * on fp32 CUDA cores, O(seqlen^2) per (batch, head).
+ * compute them: k~, f q~ and f dO, which are not bf16 numbers, go in as fp16 value rows (one
+ * rounding to 11 significant bits; max|err|/rms <= 1e-2), counted by retnet_fp16_range_errors
+ * where they leave the fp16 range.  Every other call runs on fp32 CUDA cores, O(seqlen^2) per
+ * (batch, head).
  * d_k, d_v <= 256 and seqlen <= 524280, else RETNET_ERR_UNSUPPORTED; RETNET_F_NORM_R (R~, a
  * division by a function of q and k) is RETNET_ERR_UNSUPPORTED.  Outputs do not alias inputs.
  */
@@ -339,8 +340,9 @@ RETNET_API retnet_status_t retnet_retention_backward(const void* q, const void* 
 
 /*
  * Workspace bytes that let retnet_retention_backward take the tensor-core path where it
- * applies (bf16 operands of the three chunkwise runs, their fp32 outputs, S0^T and the runs'
- * segment states); at least 2 * 4 * batch * seqlen * heads * d_k, what the CUDA-core path needs.
+ * applies (bf16 and fp16 operands of the three chunkwise runs, their fp32 outputs, S0^T and the
+ * runs' segment states); at least 2 * 4 * batch * seqlen * heads * d_k, what the CUDA-core path
+ * needs.
  */
 RETNET_API retnet_status_t retnet_backward_workspace_size(retnet_dims_t dims, size_t* bytes);
 
@@ -416,7 +418,8 @@ RETNET_API retnet_status_t retnet_debug_set_wait_budget(long long cycles);
 /*
  * Count of device threads that, since the last clear, rounded a tensor-core operand outside
  * the fp16 range (a magnitude of 65520 or more becomes inf; a NaN counts too): the scaled,
- * rotated q and k, v, the masked scores or the fp16 state copy (see Precision).  A call whose
+ * rotated q and k, v, the masked scores or the fp16 state copy (see Precision), and the fp16
+ * value rows of the gradient's runs (retnet_retention_backward).  A call whose
  * bf16 inputs leave that range produces non-finite outputs on the tensor-core kernel and
  * raises this count; the fp32 CUDA-core kernel (fp32 inputs) has no such limit.  Synchronises
  * with the device; with clear != 0 the count is reset to 0.  Returns RETNET_OK or

@@ -59,6 +59,7 @@ struct TcArgs {
   uint32_t flags;
   int nb;     // sub-blocks of T rows per chunk (pipelined kernel)
   int batch;
+  int v_f16;  // value rows arrive as fp16 (the converters leave V alone)
   // Fused MSR epilogue: out = GroupNorm_h(o) * swish(gate), written to o's place.
   const void* gate;
   float eps;
@@ -801,6 +802,7 @@ struct UnitConverter {
   float2 W[4], Z[4];                  // e^{i r0 theta_j}, e^{i RS theta_j} for the thread's pairs
   float2 cur, stepT, stepB;           // table producer (lt < DK/2): chunk base, e^{iT theta}, e^{iB theta}
   int cs, r0, lt, cur_chunk;
+  bool conv_v;                        // V arrives as bf16 (converted here) rather than fp16
 
   __device__ void init(int lt_, int nb, const HeadParams& hp) {
     lt = lt_;
@@ -817,6 +819,7 @@ struct UnitConverter {
     }
     cur = stepT = stepB = make_float2(1.f, 0.f);
     cur_chunk = -1;
+    conv_v = true;
     if (lt < DK / 2) {
       float sn, c;
       xpos_sincos(T, hp.theta[lt], &sn, &c);
@@ -913,6 +916,7 @@ struct UnitConverter {
       }
     }
     // V: each 64-column box, slot lt % 8, rows lt / 8 + VR k.
+    if (!conv_v) return;
 #pragma unroll 1
     for (int kg = 0; kg < NDV * VP; kg += VG) {
       const uint32_t vb = sv + (kg / VP) * T * 128;
@@ -1366,6 +1370,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL, PS>::THREADS, 
     if constexpr (!PRE) {
     UnitConverter<DK, T, C::NCONV, C::NDV> cv;
     cv.init(threadIdx.x - 32 * C::WARP_CONV0, nb, hp);
+    cv.conv_v = a.v_f16 == 0;
     const bool xpos = (a.flags & RETNET_F_XPOS) != 0;
     bool ok = true;
     float mx = 0.f;  // largest magnitude rounded to fp16
@@ -2227,7 +2232,7 @@ PreCopies pre_copies(const RetentionCall& c) {
 // The pre-pass pays one extra read and write of q, k, v; it saves the (nb + 1) / 2-fold
 // reconversion of chunks of nb >= 2 sub-blocks.  Not combined with sequence segments.
 bool pre_convert_applies(const RetentionCall& c, int nb, int n_seg) {
-  return nb >= 2 && n_seg < 2 && c.ws && c.ws_bytes >= pre_copy_bytes(c.dims, c.precise);
+  return nb >= 2 && n_seg < 2 && !c.v_f16 && c.ws && c.ws_bytes >= pre_copy_bytes(c.dims, c.precise);
 }
 
 // P pass (d_k = 256, 64-row sub-blocks, chunks of several of them, single operands, no fused
@@ -2314,6 +2319,7 @@ TcArgs make_args(const RetentionCall& c, int n_chunks, int nb) {
   a.pos0 = c.pos0;
   a.flags = c.flags;
   a.nb = nb;
+  a.v_f16 = c.v_f16 ? 1 : 0;
   a.n_seg = 1;
   a.n_sub = 0;
   for (int s = 0; s < 4; ++s) a.seg_lo[s] = a.seg_hi[s] = a.sub_before[s] = 0;
@@ -2600,7 +2606,10 @@ bool tc_chunkwise_supported(const RetentionCall& c) {
   if (d.d_k != 64 && d.d_k != 128 && d.d_k != 256) return false;
   if (d.d_v % kDVS != 0) return false;
   if (c.chunk != 64 && c.chunk != 128 && c.chunk != 256 && c.chunk != 512) return false;
-  if (force_serial_kernel() && (c.chunk > 128 || c.precise)) return false;
+  if (force_serial_kernel() && (c.chunk > 128 || c.precise || c.v_f16)) return false;
+  // fp16 value rows: the pipelined kernel's converters only (no pre-pass, split operands or
+  // fused epilogue), values of 64 or 128 columns a CTA
+  if (c.v_f16 && (c.precise || c.gate || c.rden)) return false;
   if (d.seqlen < 1 || d.seqlen > (1LL << 30) || d.heads > 65535 || d.batch > 65535) return false;
   if (!aligned16(c.q) || !aligned16(c.k) || !aligned16(c.v) || !aligned16(c.o)) return false;
   if ((c.state_in && !aligned16(c.state_in)) || (c.state_out && !aligned16(c.state_out))) return false;

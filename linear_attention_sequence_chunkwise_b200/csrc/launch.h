@@ -39,6 +39,9 @@ struct RetentionCall {
   // Split fp16 operands (hi + lo) on the tensor-core kernel: RETNET_F_PRECISE, R~ and the fused
   // MSR epilogue, whose normalisations magnify the operand rounding of a single fp16 copy.
   bool precise = false;
+  // Value rows already in fp16 (in_dtype still describes q and k): the gradient's runs, whose
+  // values are not bf16 numbers.  The pipelined kernel's converters leave V as it is.
+  bool v_f16 = false;
 };
 
 // Sequence segments of the key-sum pass, at most; and the workspace bytes of the R~ factors
@@ -83,6 +86,7 @@ cudaError_t tc_set_wait_budget(long long cycles);
 // Reads (and optionally clears) the count of threads that rounded a tensor-core operand outside
 // the fp16 range.
 cudaError_t tc_fp16_overflows(unsigned int* count, bool clear);
+cudaError_t bwd_fp16_overflows(unsigned int* count, bool clear);  // the gradient's fp16 value rows
 
 struct StepCall {
   const void* q;

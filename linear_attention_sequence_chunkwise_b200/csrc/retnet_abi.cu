@@ -408,7 +408,12 @@ retnet_status_t retnet_debug_set_wait_budget(long long cycles) {
 retnet_status_t retnet_fp16_range_errors(unsigned int* count, int clear) {
   if (!count) return RETNET_ERR_NULL_PTR;
   if (cudaDeviceSynchronize() != cudaSuccess) return RETNET_ERR_CUDA;
-  return from_cuda(tc_fp16_overflows(count, clear != 0));
+  unsigned int bwd = 0;
+  const retnet_status_t st = from_cuda(tc_fp16_overflows(count, clear != 0));
+  if (st != RETNET_OK) return st;
+  const retnet_status_t sb = from_cuda(bwd_fp16_overflows(&bwd, clear != 0));
+  *count += bwd;
+  return sb;
 }
 
 retnet_status_t retnet_retention_step(const void* q, const void* k, const void* v, void* o, int64_t batch,

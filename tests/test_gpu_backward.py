@@ -3,7 +3,7 @@ gradient (pinned by finite differences in test_oracle_pins.py), on both paths.
 
 Bar: max|err|/rms(oracle) <= 1e-4 for every output on the fp32 CUDA-core path (fp32
 arithmetic; bf16 inputs are exact in both); <= 1e-2 on the tensor-core path (three runs of the
-bf16-input chunkwise kernel, with one bf16 rounding of the rotated / scaled operands).
+chunkwise kernel: fp16 operands, the rotated / scaled value rows rounded to fp16 once).
 """
 import numpy as np
 import pytest
@@ -91,3 +91,18 @@ def test_backward_cuda_core_path_with_small_workspace():
     rn.retnet_retention_backward(dev(q), dev(k), dev(v), dev(do), *outs, g, th, 0, FLAGS, workspace=small)
     torch.cuda.synchronize()
     assert max(err(outs[0], rq), err(outs[1], rk), err(outs[2], rv)) <= TOL_F32
+
+
+def test_backward_reports_fp16_value_range():
+    """A gradient whose scaled value rows (f dO here) leave the fp16 range is reported by
+    retnet_fp16_range_errors rather than returned as silent inf."""
+    b, L, h, dk, dv = 1, 64, 2, 64, 64
+    q, k, v = si.qkv(b, L, h, dk, dv, 91, "bf16")
+    do = si.randn((b, L, h, dv), 92, "bf16", std=3e6)
+    g, th = si.gamma_schedule(h), si.theta_schedule(dk)
+    ws = torch.empty(rn.retnet_backward_workspace_size((b, L, h, dk, dv)), dtype=torch.uint8, device="cuda")
+    assert rn.retnet_backward_kernel((b, L, h, dk), dv, rn.BF16, FLAGS, g, ws.numel()) == 1
+    outs = [torch.empty(b, L, h, d, device="cuda") for d in (dk, dk, dv)]
+    rn.retnet_retention_backward(dev(q), dev(k), dev(v), do.cuda(), *outs, g, th, 0, FLAGS, workspace=ws)
+    torch.cuda.synchronize()
+    assert rn.retnet_fp16_range_errors(clear=True) > 0
