@@ -85,7 +85,7 @@ enum : int {
   SEG_NONE = 0,     // one CTA walks the whole sequence of its slice
   SEG_REPLAY = 1,   // segment s replays the state over chunks [0, lo_s), then outputs [lo_s, hi_s)
   SEG_FROM_WS = 2,  // segment s starts from state_in and the states of segments < s (workspace)
-  SEG_STATE = 3     // pre-pass: segment s accumulates its own state (from zero) into the workspace
+  SEG_STATE = 3     // chunk walk of the segment-state pass (its own kernel): every chunk state-only
 };
 
 template <int DK, int T>
@@ -968,21 +968,11 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL, PS>::THREADS, 
   const float log2g = hp.log2g[h];
   const int nb = a.nb;
   // The CTA visits chunks [c_first, c_hi); those below c_lo only update the state (the replay
-  // of earlier segments, or the whole segment in the state pre-pass); outputs start at c_lo.
+  // of earlier segments); outputs start at c_lo.
   // Without segments the bounds are compile-time constants and every such branch folds away.
+  static_assert(SM != SEG_STATE, "the segment-state pass has its own kernel");
   int seg = 0, s_lo = 0, s_hi = 0x7fffffff;
-  if constexpr (SM == SEG_STATE) {  // seg = the pre-pass sub-segment
-    griddep_launch_dependents();    // the output pass may start on the SMs this grid leaves idle
-    seg = blockIdx.x / n_dvb;
-    s_lo = a.sub_lo[0];
-    s_hi = a.sub_hi[0];
-#pragma unroll
-    for (int i = 1; i < kMaxSub; ++i)
-      if (seg == i) {
-        s_lo = a.sub_lo[i];
-        s_hi = a.sub_hi[i];
-      }
-  } else if constexpr (SEG) {
+  if constexpr (SEG) {
     seg = (SM == SEG_FROM_WS) ? blockIdx.z / a.batch : blockIdx.x / n_dvb;
     s_lo = a.seg_lo[0];
     s_hi = a.seg_hi[0];
@@ -994,7 +984,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL, PS>::THREADS, 
       }
   }
   const int c_first = (SM == SEG_REPLAY) ? 0 : s_lo;
-  const int c_lo = (SM == SEG_STATE) ? s_hi : s_lo;
+  const int c_lo = s_lo;
   const int c_hi = s_hi;
   // Start state of a two-pass output segment: state_in carried over the earlier segments,
   // R = gamma^len_j R + W_j (row dk, columns [col, col + n) of the slice).
@@ -1307,27 +1297,6 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL, PS>::THREADS, 
         if (q.rb_done()) mma_commit(bar(Q_O_FULL + (q.rb & 1)));
         mma_commit(bar(Q_STAGE_EMPTY + s));
       };
-      if constexpr (SM == SEG_STATE) {
-        // State pre-pass: every increment Kz'^T V accumulates into one tensor-memory tile
-        // (Kz' carries the decay to the segment's end), committed once at the end.
-        UnitIter<T, SM> f;
-        bool first = true;
-        for (f.start(a.L, nb, c_first, c_lo, c_hi); f.valid(); f.next()) {
-          const int s = f.k % C::NS;
-          if (!mbar_wait(bar(Q_READY + s), (f.k / C::NS) & 1)) break;
-          tc_fence_after();
-          const uint64_t dkm = sdesc_sw128(sK(s), T * 128, 1024), dv = sdesc_sw128(sV(s), T * 128, 1024);
-#pragma unroll
-          for (int blk = 0; blk < C::RBLK; ++blk)
-#pragma unroll
-            for (int ks = 0; ks < T / 16; ++ks)
-              mma_f16_ss(tmem + C::COL_DR + blk * DVS, dkm + static_cast<uint64_t>((blk * 2 * T * 128 + ks * 2048) >> 4),
-                         dv + static_cast<uint64_t>((ks * 2048) >> 4), ID_R, (first && ks == 0) ? 0u : 1u);
-          first = false;
-          mma_commit(bar(Q_STAGE_EMPTY + s));
-        }
-        mma_commit(bar(Q_DR_FULL + 0));
-      }
       constexpr int LA = 2;  // F of unit f only while f <= q + LA (q = oldest unit with P pending)
       UnitIter<T, SM> f, q;
       f.start(a.L, nb, c_first, c_lo, c_hi);
@@ -1386,12 +1355,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL, PS>::THREADS, 
       ok = mbar_wait(bar(Q_TAB + (it.k & 1)), (it.k >> 1) & 1);
       if (ok) ok = mbar_wait(bar(Q_TMA_FULL + s), (it.k / C::NS) & 1);
       if (!ok) break;
-      if constexpr (SM == SEG_STATE) {
-        // K of column block w decays to the segment's end E: gamma^(E - 1 - t) in all
-        const int e_tok = min(c_hi * nb * T, a.L), blk_end = it.t0() + (it.w + 1) * T;
-        cv.template convert<false>(sQ(s), sK(s), sV(s), tq, tk, xpos, log2g, mx,
-                                   exp2f(static_cast<float>(e_tok - blk_end) * log2g));
-      } else if (SM == SEG_REPLAY && it.pre()) {
+      if (SM == SEG_REPLAY && it.pre()) {
         cv.template convert<false>(sQ(s), sK(s), sV(s), tq, tk, xpos, log2g, mx);
       } else {
         cv.template convert<true, HL>(sQ(s), sK(s), sV(s), tq, tk, xpos, log2g, mx, 1.f, sQl(s), sKl(s));
@@ -1403,36 +1367,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL, PS>::THREADS, 
     }
   } else if (warp >= C::WARP_S0 && warp < C::WARP_S0 + C::WARPS_S) {
     // ------------------------------------------------------------------ state group
-    if constexpr (SM == SEG_STATE) {
-      // State pre-pass: once the last increment has landed, the accumulated segment state
-      // (thread = one d_k row, all DVS columns) goes to the workspace.
-      const uint32_t lane_off = static_cast<uint32_t>(32 * (warp % 4)) << 16;
-      if (__all_sync(0xffffffffu, mbar_wait(bar(Q_DR_FULL + 0), 0))) {
-        tc_fence_after();
-        const size_t plane = static_cast<size_t>(a.batch) * a.heads * DK * a.dv;
-#pragma unroll 1
-        for (int bk = 0; bk < C::BPT; ++bk) {
-          const int blk = C::BPT > 1 ? bk : (warp - C::WARP_S0) / 4 % C::RBLK;
-          const int dk = (DK == 64) ? (lane < 16 ? 16 * (warp % 4) + lane : -1) : blk * 128 + 32 * (warp % 4) + lane;
-          float* dst = a.ws + seg * plane + (static_cast<size_t>(b) * a.heads + h) * DK * a.dv + dvb * DVS +
-                       static_cast<size_t>(dk < 0 ? 0 : dk) * a.dv;
-#pragma unroll 1
-          for (int grp = 0; grp < DVS / 32; ++grp) {
-            uint32_t u[2][16];
-            tmem_ld_wait(tmem + C::COL_DR + blk * DVS + 32 * grp + lane_off, u);
-            if (dk >= 0) {
-#pragma unroll
-              for (int c4 = 0; c4 < 8; ++c4)
-                *reinterpret_cast<float4*>(dst + 32 * grp + 4 * c4) =
-                    make_float4(__uint_as_float(u[(4 * c4) / 16][(4 * c4) % 16]),
-                                __uint_as_float(u[(4 * c4 + 1) / 16][(4 * c4 + 1) % 16]),
-                                __uint_as_float(u[(4 * c4 + 2) / 16][(4 * c4 + 2) % 16]),
-                                __uint_as_float(u[(4 * c4 + 3) / 16][(4 * c4 + 3) % 16]));
-            }
-          }
-        }
-      }
-    } else if constexpr (C::RTM) {
+    if constexpr (C::RTM) {
       // The fp32 state stays in tensor memory as a master M; thread = one TMEM lane, i.e. one
       // d_k row in each of its BPT 128-row blocks, all DVS columns.  Before every increment
       // Kz_w^T V_w (the column blocks w of a chunk's last row block) accumulates into M, the
@@ -1939,6 +1874,200 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL, PS>::THREADS, 
 }
 
 // ============================================================================================
+// Segment-state pass (two-pass sequence segments, and the state of a sequence shard): for each
+// sub-segment j of chunks [sub_lo[j], sub_hi[j]) with end token E, from a zero start,
+//   W_j = sum_t gamma^(E-1-t) k~_t^T v_t  ("阅读笔记：RetNet" §2.4: the chunk recurrence unrolled
+// over the sub-segment; it is associative, R <- gamma^len R + W, which the output pass uses).
+// The whole sub-segment is one contraction, so there is no per-chunk state update: the key rows
+// carry the decay to E, every increment Kz^T V accumulates into one tensor-memory tile, and the
+// CTA is bound by streaming and converting K and V.  Roles: eight converter warps (K rotated and
+// scaled, V to fp16; they also write W out at the end), a TMA warp, an MMA warp; stages hold K
+// and V only.  Output: ws fp32 [j][batch][heads][d_k][d_v] (slice columns of this CTA).
+template <int DK, int T, int DVS>
+struct CfgS {
+  static constexpr int NCW = 8;
+  static constexpr int NCONV = 32 * NCW;
+  static constexpr int WARP_TMA = NCW, WARP_MMA = NCW + 1;
+  static constexpr int THREADS = 32 * (NCW + 2);
+  static constexpr int NDV = DVS / 64;
+  static constexpr int RBLK = DK > 128 ? 2 : 1;  // 128-row blocks of the state
+  static constexpr int MR = DK >= 128 ? 128 : 64;
+  static constexpr int KBYTES = T * DK * 2, VBYTES = T * DVS * 2;
+  static constexpr int STAGE = KBYTES + VBYTES;
+  static constexpr int TABBYTES = 2 * 2 * (DK / 2) * 8;
+  static constexpr int NBARS = 3 * 6 + 2 + 2;
+  static constexpr int BUDGET = 227 * 1024 - 1024;
+  static constexpr int NS_FIT = (BUDGET - TABBYTES - NBARS * 8 - 16) / STAGE;
+  static constexpr int NS = NS_FIT > 6 ? 6 : NS_FIT;
+  static constexpr int SMEM = NS * STAGE + TABBYTES + NBARS * 8 + 16 + 1024;
+  static constexpr int TMEM_COLS = RBLK * DVS <= 128 ? 128 : 256;
+  static_assert(NS >= 2, "segment-state stages");
+};
+
+template <int DK, int T, int DVS>
+__global__ void __launch_bounds__(CfgS<DK, T, DVS>::THREADS, 1)
+    tc_segment_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                            TcArgs a, HeadParams hp) {
+  using C = CfgS<DK, T, DVS>;
+  enum : int { B_FULL = 0, B_CONV = 6, B_EMPTY = 12, B_TAB = 18, B_DONE = 20, B_DRAIN = 21 };
+  griddep_launch_dependents();  // the output pass may start on the SMs this grid leaves idle
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_addr(smem_raw);
+  const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (sbase - raw_addr);
+  float2* tab = reinterpret_cast<float2*>(gbase + C::NS * C::STAGE);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + C::NS * C::STAGE + C::TABBYTES);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::NBARS);
+  auto bar = [&](int i) { return smem_addr(bars + i); };
+  auto sK = [&](int st) { return sbase + st * C::STAGE; };
+  auto sV = [&](int st) { return sbase + st * C::STAGE + C::KBYTES; };
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int n_dvb = a.dv / DVS;
+  const int dvb = blockIdx.x % n_dvb, seg = blockIdx.x / n_dvb, h = blockIdx.y, b = blockIdx.z;
+  int s_lo = a.sub_lo[0], s_hi = a.sub_hi[0];
+#pragma unroll
+  for (int i = 1; i < kMaxSub; ++i)  // constant-index selects keep the kernel parameters in place
+    if (seg == i) {
+      s_lo = a.sub_lo[i];
+      s_hi = a.sub_hi[i];
+    }
+  const int nb = a.nb;
+  const float log2g = hp.log2g[h];
+
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < 6; ++st) {
+      mbar_init(bar(B_FULL + st), 1);
+      mbar_init(bar(B_CONV + st), C::NCONV);
+      mbar_init(bar(B_EMPTY + st), 1);
+    }
+    mbar_init(bar(B_TAB), C::NCONV);
+    mbar_init(bar(B_TAB + 1), C::NCONV);
+    mbar_init(bar(B_DONE), 1);
+    mbar_init(bar(B_DRAIN), 1);
+    fence_mbar_init();
+  }
+  if (warp == C::WARP_MMA) {
+    tmem_alloc(smem_addr(tmem_holder), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == C::WARP_TMA && lane == 0) {
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == C::WARP_TMA) {
+    if (lane == 0) {
+      int issued[6] = {0, 0, 0, 0, 0, 0};
+      UnitIter<T, SEG_STATE> it;
+      for (it.start(a.L, nb, s_lo, s_hi, s_hi); it.valid(); it.next()) {
+        const int st = it.k % C::NS;
+        if (it.k >= C::NS && !mbar_wait(bar(B_EMPTY + st), ((it.k / C::NS) - 1) & 1)) break;
+        mbar_arrive_expect_tx(bar(B_FULL + st), C::KBYTES + C::VBYTES);
+        const int tk = it.t0() + it.w * T;
+#pragma unroll
+        for (int bx = 0; bx < DK / 64; ++bx) tma_load_4d(sK(st) + bx * T * 128, &tm_k, bar(B_FULL + st), bx * 64, h, tk, b);
+#pragma unroll
+        for (int bx = 0; bx < C::NDV; ++bx)
+          tma_load_4d(sV(st) + bx * T * 128, &tm_v, bar(B_FULL + st), dvb * DVS + 64 * bx, h, tk, b);
+        issued[st]++;
+      }
+      // Every load this thread issued must have landed before the CTA may exit.
+      for (int st = 0; st < C::NS; ++st)
+        if (issued[st] > 0) mbar_wait(bar(B_FULL + st), (issued[st] - 1) & 1, kDrainBudget);
+    }
+  } else if (warp == C::WARP_MMA) {
+    if (lane == 0) {
+      constexpr uint32_t ID_R = idesc_f16_f32(C::MR, DVS, 1, 1);
+      UnitIter<T, SEG_STATE> f;
+      bool first = true;
+      for (f.start(a.L, nb, s_lo, s_hi, s_hi); f.valid(); f.next()) {
+        const int st = f.k % C::NS;
+        if (!mbar_wait(bar(B_CONV + st), (f.k / C::NS) & 1)) break;
+        tc_fence_after();
+        const uint64_t dkm = sdesc_sw128(sK(st), T * 128, 1024), dv = sdesc_sw128(sV(st), T * 128, 1024);
+#pragma unroll
+        for (int blk = 0; blk < C::RBLK; ++blk)
+#pragma unroll
+          for (int ks = 0; ks < T / 16; ++ks)
+            mma_f16_ss(tmem + blk * DVS, dkm + static_cast<uint64_t>((blk * 2 * T * 128 + ks * 2048) >> 4),
+                       dv + static_cast<uint64_t>((ks * 2048) >> 4), ID_R, (first && ks == 0) ? 0u : 1u);
+        first = false;
+        mma_commit(bar(B_EMPTY + st));
+      }
+      mma_commit(bar(B_DONE));
+      mma_commit(bar(B_DRAIN));
+      mbar_wait(bar(B_DRAIN), 0, kDrainBudget);
+    }
+  } else {
+    // ------------------------------------------------------------------ converters
+    UnitConverter<DK, T, C::NCONV, C::NDV> cv;
+    cv.init(threadIdx.x, nb, hp);
+    cv.conv_v = a.v_f16 == 0;
+    const bool xpos = (a.flags & RETNET_F_XPOS) != 0;
+    const int e_tok = min(s_hi * nb * T, a.L);  // the sub-segment's end E
+    bool ok = true;
+    float mx = 0.f;
+    UnitIter<T, SEG_STATE> it;
+    for (it.start(a.L, nb, s_lo, s_hi, s_hi); ok && it.valid(); it.next()) {
+      const int st = it.k % C::NS;
+      float2* tq = tab + (it.k & 1) * DK;
+      float2* tk = tq + DK / 2;
+      if (xpos) cv.put_bases(tq, tk, it.i, it.u, it.w, it.t0(), a.pos0, hp);
+      // table buffer (k & 1) complete once all converters arrived (as in the pipelined kernel)
+      mbar_arrive(bar(B_TAB + (it.k & 1)));
+      ok = mbar_wait(bar(B_TAB + (it.k & 1)), (it.k >> 1) & 1);
+      if (ok) ok = mbar_wait(bar(B_FULL + st), (it.k / C::NS) & 1);
+      if (!ok) break;
+      // K of column block w decays to E: gamma^(E - 1 - t) in all
+      const int blk_end = it.t0() + (it.w + 1) * T;
+      cv.template convert<false>(0, sK(st), sV(st), tq, tk, xpos, log2g, mx,
+                                 exp2f(static_cast<float>(e_tok - blk_end) * log2g));
+      fence_proxy_async_smem();
+      mbar_arrive(bar(B_CONV + st));
+    }
+    report_fp16_range(mx);
+    // W out: warp w reads TMEM lane quarter w % 4 (d_k rows), column half w / 4 of the slice.
+    if (__all_sync(0xffffffffu, mbar_wait(bar(B_DONE), 0))) {
+      tc_fence_after();
+      const uint32_t lane_off = static_cast<uint32_t>(32 * (warp % 4)) << 16;
+      const size_t plane = static_cast<size_t>(a.batch) * a.heads * DK * a.dv;
+      constexpr int HALF = DVS / 2;
+#pragma unroll 1
+      for (int blk = 0; blk < C::RBLK; ++blk) {
+        const int dk = (DK == 64) ? (lane < 16 ? 16 * (warp % 4) + lane : -1) : blk * 128 + 32 * (warp % 4) + lane;
+        const int col0 = (warp / 4) * HALF;
+        float* dst = a.ws + seg * plane + (static_cast<size_t>(b) * a.heads + h) * DK * a.dv + dvb * DVS + col0 +
+                     static_cast<size_t>(dk < 0 ? 0 : dk) * a.dv;
+#pragma unroll 1
+        for (int grp = 0; grp < HALF / 32; ++grp) {
+          uint32_t u[2][16];
+          tmem_ld_wait(tmem + blk * DVS + col0 + 32 * grp + lane_off, u);
+          if (dk >= 0) {
+#pragma unroll
+            for (int c4 = 0; c4 < 8; ++c4)
+              *reinterpret_cast<float4*>(dst + 32 * grp + 4 * c4) =
+                  make_float4(__uint_as_float(u[(4 * c4) / 16][(4 * c4) % 16]),
+                              __uint_as_float(u[(4 * c4 + 1) / 16][(4 * c4 + 1) % 16]),
+                              __uint_as_float(u[(4 * c4 + 2) / 16][(4 * c4 + 2) % 16]),
+                              __uint_as_float(u[(4 * c4 + 3) / 16][(4 * c4 + 3) % 16]));
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == C::WARP_MMA) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
 // Conversion pre-pass (chunks of several sub-blocks).  The pipelined kernel converts Q_u, K_w
 // and V_w for every unit (u, w), i.e. (nb + 1) / 2 times per token; this kernel writes fp16
 // copies that already carry its operand scaling, once per token, and the pipelined kernel then
@@ -2532,8 +2661,12 @@ cudaError_t launch_pipe(const RetentionCall& c, const HeadParams& hp, cudaStream
   }
   as.n_sub = j;
   as.ws = static_cast<float*>(c.ws);
-  cudaError_t e = run(tc_chunkwise_pipe_kernel<DK, T, DVS, SEG_STATE, false, false, Tout>, as.n_sub);
+  using CfS = CfgS<DK, T, DVS>;
+  auto kst = tc_segment_state_kernel<DK, T, DVS>;
+  cudaError_t e = cudaFuncSetAttribute(kst, cudaFuncAttributeMaxDynamicSharedMemorySize, CfS::SMEM);
   if (e != cudaSuccess) return e;
+  kst<<<dim3(grid.x * as.n_sub, grid.y, grid.z), CfS::THREADS, CfS::SMEM, s>>>(mk, mv, as, hp);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // Output pass, launched as a programmatic dependent of the pre-pass (segment-major grid):
   // its segment-0 CTAs run on the SMs the pre-pass leaves idle; later segments wait on the
   // device (griddepcontrol.wait) before they read the pre-pass states.
@@ -2661,7 +2794,7 @@ cudaError_t tc_wait_timeouts(unsigned int* count, bool clear) {
 namespace {
 template <int DK, int T, typename Tout>
 cudaError_t launch_segment_state_t(const RetentionCall& c, const HeadParams& hp, cudaStream_t s) {
-  using Cf = Cfg3<DK, T, 64>;
+  using Cf = CfgS<DK, T, 64>;
   CUtensorMap mq, mk, mv;
   // The state pass never loads Q: its map is built over K (a valid tensor of the same shape).
   RetentionCall cc = c;
@@ -2675,10 +2808,10 @@ cudaError_t launch_segment_state_t(const RetentionCall& c, const HeadParams& hp,
   a.sub_lo[0] = 0;
   a.sub_hi[0] = n_chunks;
   a.ws = c.state_out;  // sub-segment 0 of the workspace layout is [batch][heads][d_k][d_v]
-  auto kern = tc_chunkwise_pipe_kernel<DK, T, 64, SEG_STATE, false, false, Tout>;
+  auto kern = tc_segment_state_kernel<DK, T, 64>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<tc_grid(c.dims, 64), Cf::THREADS, Cf::SMEM, s>>>(mq, mk, mv, mq, mk, a, hp);
+  kern<<<tc_grid(c.dims, 64), Cf::THREADS, Cf::SMEM, s>>>(mk, mv, a, hp);
   return cudaGetLastError();
 }
 
