@@ -987,7 +987,10 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL, PS>::THREADS, 
   const int c_lo = s_lo;
   const int c_hi = s_hi;
   // Start state of a two-pass output segment: state_in carried over the earlier segments,
-  // R = gamma^len_j R + W_j (row dk, columns [col, col + n) of the slice).
+  // R = gamma^len_j R + W_j (row dk, columns [col, col + n) of the slice, n a multiple of 32).
+  // The states W_j are read two at a time with both loads in flight (they do not depend on the
+  // running sum), 32 columns at a time; a loop that read one state after the other paid one
+  // memory latency per state and column group.
   auto start_state = [&](int dk, int col, int n, float* R) {
     const int64_t bh = static_cast<int64_t>(b) * a.heads + h;
     for (int c = 0; c < n; ++c) R[c] = 0.f;
@@ -1004,21 +1007,42 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL, PS>::THREADS, 
       for (int t = 1; t < 4; ++t)  // constant-index selects, as above
         if (t == seg) n_before = a.sub_before[t];
       if (n_before > 0) griddep_wait();  // the pre-pass states are complete and visible
-      for (int j = 0; j < n_before; ++j) {
+      const size_t plane = static_cast<size_t>(a.batch) * a.heads * DK * a.dv;
+      const float* w0base = a.ws + static_cast<size_t>(bh) * DK * a.dv + col + static_cast<size_t>(dk) * a.dv;
+      auto factor = [&](int j) {  // gamma^len_j, len_j = the tokens of sub-segment j
         int chunks_j = 0;
 #pragma unroll
         for (int t = 0; t < kMaxSub; ++t)
           if (t == j) chunks_j = a.sub_hi[t] - a.sub_lo[t];
-        const int len_j = chunks_j * nb * T;
-        const float gl = exp2f(static_cast<float>(len_j) * log2g);
-        const size_t plane = static_cast<size_t>(a.batch) * a.heads * DK * a.dv;
-        const float* w = a.ws + j * plane + static_cast<size_t>(bh) * DK * a.dv + col + static_cast<size_t>(dk) * a.dv;
-        for (int c4 = 0; c4 < n / 4; ++c4) {
-          const float4 x = *reinterpret_cast<const float4*>(w + 4 * c4);
-          R[4 * c4] = fmaf(gl, R[4 * c4], x.x);
-          R[4 * c4 + 1] = fmaf(gl, R[4 * c4 + 1], x.y);
-          R[4 * c4 + 2] = fmaf(gl, R[4 * c4 + 2], x.z);
-          R[4 * c4 + 3] = fmaf(gl, R[4 * c4 + 3], x.w);
+        return exp2f(static_cast<float>(chunks_j * nb * T) * log2g);
+      };
+      for (int j = 0; j < n_before; j += 2) {
+        const bool two = j + 1 < n_before;
+        const int j1 = two ? j + 1 : j;  // a valid state either way; its terms count only if two
+        const float g0 = factor(j), g1 = factor(j1);
+        const float* w0 = w0base + j * plane;
+        const float* w1 = w0base + j1 * plane;
+        for (int c32 = 0; c32 < n; c32 += 32) {
+          float4 x0[8], x1[8];
+#pragma unroll
+          for (int c4 = 0; c4 < 8; ++c4) {
+            x0[c4] = *reinterpret_cast<const float4*>(w0 + c32 + 4 * c4);
+            x1[c4] = *reinterpret_cast<const float4*>(w1 + c32 + 4 * c4);
+          }
+#pragma unroll
+          for (int c4 = 0; c4 < 8; ++c4) {
+            float* r = R + c32 + 4 * c4;
+            r[0] = fmaf(g0, r[0], x0[c4].x);
+            r[1] = fmaf(g0, r[1], x0[c4].y);
+            r[2] = fmaf(g0, r[2], x0[c4].z);
+            r[3] = fmaf(g0, r[3], x0[c4].w);
+            if (two) {
+              r[0] = fmaf(g1, r[0], x1[c4].x);
+              r[1] = fmaf(g1, r[1], x1[c4].y);
+              r[2] = fmaf(g1, r[2], x1[c4].z);
+              r[3] = fmaf(g1, r[3], x1[c4].w);
+            }
+          }
         }
       }
     }
