@@ -55,39 +55,67 @@ __device__ __forceinline__ void row_factors(float* sf, int heads, int d_k, int64
   __syncthreads();
 }
 
+// Rotation (cos, sin) of every pair j at position p, into shared memory (identity without
+// xPos); one sincos a pair, shared by the heads.
+__device__ __forceinline__ void pair_rotations(float2* rot, int d_k, int64_t p, bool xpos, const HeadParams& hp) {
+  for (int j = threadIdx.x; j < d_k / 2; j += blockDim.x) {
+    float c = 1.f, s = 0.f;
+    if (xpos) xpos_sincos(p, hp.theta[j], &s, &c);
+    rot[j] = make_float2(c, s);
+  }
+  __syncthreads();
+}
+
+// bf16x2 word -> two floats (element 2i at the low half).
+__device__ __forceinline__ float2 bf2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+__device__ __forceinline__ uint32_t h2(float a, float b, float& mx) {
+  const __half2 x = __halves2half2(to_f16(a, mx), to_f16(b, mx));
+  return *reinterpret_cast<const uint32_t*>(&x);
+}
+
 // Token (b, t): k~ (forward order) and f q~ (reversed) as fp16 rows; q, k copied reversed.
+// Thread = (head, 16-byte group of 8 elements = 4 rotary pairs).
 __global__ void __launch_bounds__(128) bwd_tc_prep_qk(const __nv_bfloat16* __restrict__ q,
                                                       const __nv_bfloat16* __restrict__ k, __half* __restrict__ kt,
                                                       __nv_bfloat16* __restrict__ qR, __nv_bfloat16* __restrict__ kR,
                                                       __half* __restrict__ fqR, int L, int heads, int d_k, int64_t pos0,
                                                       uint32_t flags, HeadParams hp) {
   __shared__ float sf[RETNET_MAX_HEADS];
+  __shared__ float2 rot[kMaxPairs];
   const int64_t bt = blockIdx.x;
   const int t = static_cast<int>(bt % L);
   const int64_t rbt = bt - t + (L - 1 - t);  // the same b at t' = L-1-t
   row_factors(sf, heads, d_k, pos0 + t, flags, hp);
-  const bool xpos = (flags & RETNET_F_XPOS) != 0;
+  pair_rotations(rot, d_k, pos0 + t, (flags & RETNET_F_XPOS) != 0, hp);
+  const int groups = d_k / 8;
   float mx = 0.f;
-  for (int j = threadIdx.x; j < d_k / 2; j += blockDim.x) {
-    float c = 1.f, s = 0.f;
-    if (xpos) xpos_sincos(pos0 + t, hp.theta[j], &s, &c);
-    for (int h = 0; h < heads; ++h) {
-      const int64_t o = (bt * heads + h) * d_k + 2 * j, ro = (rbt * heads + h) * d_k + 2 * j;
-      const __nv_bfloat162 q2 = *reinterpret_cast<const __nv_bfloat162*>(q + o);
-      const __nv_bfloat162 k2 = *reinterpret_cast<const __nv_bfloat162*>(k + o);
-      const float2 qf = __bfloat1622float2(q2), kf = __bfloat1622float2(k2);
-      *reinterpret_cast<__nv_bfloat162*>(qR + ro) = q2;
-      *reinterpret_cast<__nv_bfloat162*>(kR + ro) = k2;
-      *reinterpret_cast<__half2*>(kt + o) = __halves2half2(to_f16(kf.x * c - kf.y * s, mx), to_f16(kf.x * s + kf.y * c, mx));
-      const float f = sf[h];
-      *reinterpret_cast<__half2*>(fqR + ro) =
-          __halves2half2(to_f16(f * (qf.x * c - qf.y * s), mx), to_f16(f * (qf.x * s + qf.y * c), mx));
+  for (int e = threadIdx.x; e < heads * groups; e += blockDim.x) {
+    const int h = e / groups, g = e % groups;
+    const int64_t o = (bt * heads + h) * d_k + 8 * g, ro = (rbt * heads + h) * d_k + 8 * g;
+    const uint4 q4 = *reinterpret_cast<const uint4*>(q + o);
+    const uint4 k4 = *reinterpret_cast<const uint4*>(k + o);
+    *reinterpret_cast<uint4*>(qR + ro) = q4;
+    *reinterpret_cast<uint4*>(kR + ro) = k4;
+    const uint32_t qw[4] = {q4.x, q4.y, q4.z, q4.w}, kw[4] = {k4.x, k4.y, k4.z, k4.w};
+    uint32_t ko[4], qo[4];
+    const float f = sf[h];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 cs = rot[4 * g + i];
+      const float2 kf = bf2(kw[i]), qf = bf2(qw[i]);
+      ko[i] = h2(kf.x * cs.x - kf.y * cs.y, kf.x * cs.y + kf.y * cs.x, mx);
+      qo[i] = h2(f * (qf.x * cs.x - qf.y * cs.y), f * (qf.x * cs.y + qf.y * cs.x), mx);
     }
+    *reinterpret_cast<uint4*>(kt + o) = make_uint4(ko[0], ko[1], ko[2], ko[3]);
+    *reinterpret_cast<uint4*>(fqR + ro) = make_uint4(qo[0], qo[1], qo[2], qo[3]);
   }
   report_range(mx);
 }
 
-// Token (b, t): v and dO copied reversed; f dO reversed as fp16 rows.
+// Token (b, t): v and dO copied reversed; f dO reversed as fp16 rows.  Thread = (head,
+// 16-byte group of 8 elements).
 __global__ void __launch_bounds__(128) bwd_tc_prep_v(const __nv_bfloat16* __restrict__ v,
                                                      const __nv_bfloat16* __restrict__ dout,
                                                      __nv_bfloat16* __restrict__ vR, __nv_bfloat16* __restrict__ doR,
@@ -98,17 +126,24 @@ __global__ void __launch_bounds__(128) bwd_tc_prep_v(const __nv_bfloat16* __rest
   const int t = static_cast<int>(bt % L);
   const int64_t rbt = bt - t + (L - 1 - t);
   row_factors(sf, heads, d_k, pos0 + t, flags, hp);
-  const int half = d_v / 2;
+  const int groups = d_v / 8;
   float mx = 0.f;
-  for (int e = threadIdx.x; e < heads * half; e += blockDim.x) {
-    const int h = e / half, j = 2 * (e % half);
-    const int64_t o = (bt * heads + h) * d_v + j, ro = (rbt * heads + h) * d_v + j;
-    const __nv_bfloat162 v2 = *reinterpret_cast<const __nv_bfloat162*>(v + o);
-    const __nv_bfloat162 d2 = *reinterpret_cast<const __nv_bfloat162*>(dout + o);
-    *reinterpret_cast<__nv_bfloat162*>(vR + ro) = v2;
-    *reinterpret_cast<__nv_bfloat162*>(doR + ro) = d2;
-    const float2 df = __bfloat1622float2(d2);
-    *reinterpret_cast<__half2*>(fdoR + ro) = __halves2half2(to_f16(sf[h] * df.x, mx), to_f16(sf[h] * df.y, mx));
+  for (int e = threadIdx.x; e < heads * groups; e += blockDim.x) {
+    const int h = e / groups, g = e % groups;
+    const int64_t o = (bt * heads + h) * d_v + 8 * g, ro = (rbt * heads + h) * d_v + 8 * g;
+    const uint4 v4 = *reinterpret_cast<const uint4*>(v + o);
+    const uint4 d4 = *reinterpret_cast<const uint4*>(dout + o);
+    *reinterpret_cast<uint4*>(vR + ro) = v4;
+    *reinterpret_cast<uint4*>(doR + ro) = d4;
+    const uint32_t dw[4] = {d4.x, d4.y, d4.z, d4.w};
+    uint32_t fo[4];
+    const float f = sf[h];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 df = bf2(dw[i]);
+      fo[i] = h2(f * df.x, f * df.y, mx);
+    }
+    *reinterpret_cast<uint4*>(fdoR + ro) = make_uint4(fo[0], fo[1], fo[2], fo[3]);
   }
   report_range(mx);
 }
@@ -252,7 +287,9 @@ bool backward_tc_applies(const BackwardCall& c, const HeadParams& hp) {
   if (!dim_ok(d.d_k) || !dim_ok(d.d_v) || d.seqlen < 1) return false;
   if (!c.ws || c.ws_bytes < backward_tc_workspace_bytes(d)) return false;
   auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
-  if (!al16(c.q) || !al16(c.k) || !al16(c.dq) || !al16(c.dk) || !al16(c.dv) || !al16(c.ws)) return false;
+  if (!al16(c.q) || !al16(c.k) || !al16(c.v) || !al16(c.dout) || !al16(c.dq) || !al16(c.dk) || !al16(c.dv) ||
+      !al16(c.ws))
+    return false;
   RetentionCall calls[kRuns];
   tc_calls(c, static_cast<char*>(c.ws), tc_layout(d), calls);
   for (int i = 0; i < kRuns; ++i)
