@@ -14,8 +14,9 @@
 // A prep kernel writes the operands (rotations, row factors, reversal): exact bf16 copies of q,
 // k, v, dO for the runs' queries and keys; k~, f q~ and f dO, which are not bf16 numbers, as
 // fp16 value rows (one rounding, 2^-11 relative: a bf16 rounding of the values, 2^-8, left
-// 1-2e-2 max|err|/rms in the gradient), which the runs' converters take as they are.  A post
-// kernel scales dq by f, turns dq and dk back (R^T) and undoes the reversal of dk and dv.
+// 1-2e-2 max|err|/rms in the gradient), which the runs' converters take as they are.  The dv
+// run writes its rows in forward order itself (reversed-output epilogue); a post kernel scales
+// dq by f, turns dq and dk back (R^T) and undoes the reversal of dk.
 #include <algorithm>
 
 #include "launch.h"
@@ -183,20 +184,6 @@ __global__ void __launch_bounds__(128) bwd_tc_post_qk(const float* __restrict__ 
   }
 }
 
-// Token (b, t): dv = the dv run's reversed row (float4 a thread).
-__global__ void __launch_bounds__(128) bwd_tc_post_v(const float* __restrict__ ovR, float* __restrict__ dv, int L,
-                                                     int heads, int d_v) {
-  const int64_t bt = blockIdx.x;
-  const int t = static_cast<int>(bt % L);
-  const int64_t rbt = bt - t + (L - 1 - t);
-  const int q4 = d_v / 4;
-  for (int e = threadIdx.x; e < heads * q4; e += blockDim.x) {
-    const int h = e / q4, j = 4 * (e % q4);
-    *reinterpret_cast<float4*>(dv + (bt * heads + h) * d_v + j) =
-        *reinterpret_cast<const float4*>(ovR + (rbt * heads + h) * d_v + j);
-  }
-}
-
 // dS0[i][j] = sum_t' g^(L-t') (f q~)R[t'][i] doR[t'][j]  (t' = L-1-n, so g^(n+1)):
 // CTA = (b * h, 32-row block of d_k), thread = (row i, columns j).
 __global__ void __launch_bounds__(256) bwd_tc_dstate(const __half* __restrict__ fqR,
@@ -222,7 +209,7 @@ constexpr int kBwdChunk = 64;
 size_t a256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct TcLayout {
-  size_t kt, qR, kR, fqR, vR, doR, fdoR, oq, okR, ovR, s0t, fwd, total;
+  size_t kt, qR, kR, fqR, vR, doR, fdoR, oq, okR, s0t, fwd, total;
 };
 TcLayout tc_layout(const Dims& d) {
   const size_t tok = static_cast<size_t>(d.batch * d.seqlen * d.heads);
@@ -238,7 +225,6 @@ TcLayout tc_layout(const Dims& d) {
   l.fdoR = off; off += a256(tok * dv * 2);
   l.oq = off; off += a256(tok * dk * 4);
   l.okR = off; off += a256(tok * dk * 4);
-  l.ovR = off; off += a256(tok * dv * 4);
   l.s0t = off; off += a256(static_cast<size_t>(d.batch * d.heads) * dv * dk * 4);
   l.fwd = off;
   // the forward runs' own workspace (two-pass segment states), shared by the three in turn
@@ -265,7 +251,8 @@ void tc_calls(const BackwardCall& c, char* ws, const TcLayout& l, RetentionCall 
   out[0] = base(c.dout, c.v, ws + l.kt, ws + l.oq, d1, 0u,
                 c.state_in ? reinterpret_cast<const float*>(ws + l.s0t) : nullptr);
   out[1] = base(ws + l.vR, ws + l.doR, ws + l.fqR, ws + l.okR, d1, 0u, nullptr);
-  out[2] = base(ws + l.kR, ws + l.qR, ws + l.fdoR, ws + l.ovR, d3, c.flags & RETNET_F_XPOS, nullptr);
+  out[2] = base(ws + l.kR, ws + l.qR, ws + l.fdoR, c.dv, d3, c.flags & RETNET_F_XPOS, nullptr);
+  out[2].o_rev = true;  // dv in forward order straight from the run
 }
 
 // Head parameters of each run: the kernels rotate by whatever theta they are given (a call
@@ -327,8 +314,6 @@ cudaError_t launch_backward_tc(const BackwardCall& c, const HeadParams& hp, cuda
     if ((e = launch_tc_chunkwise(calls[i], run_params(hp, i), s)) != cudaSuccess) return e;
   bwd_tc_post_qk<<<tokens, 128, 0, s>>>(fp(l.oq), fp(l.okR), c.dq, c.dk, L, H, dk, c.pos0, c.flags, hp);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  bwd_tc_post_v<<<tokens, 128, 0, s>>>(fp(l.ovR), c.dv, L, H, dv);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (c.dstate) {
     const dim3 gs(static_cast<unsigned>(d.batch * d.heads), static_cast<unsigned>((dk + 31) / 32));
     bwd_tc_dstate<<<gs, 256, 0, s>>>(hf(l.fqR), bf(l.doR), c.dstate, L, H, dk, dv, hp);
@@ -347,7 +332,7 @@ cudaError_t bwd_fp16_overflows(unsigned int* count, bool clear) {
 int backward_tc_launches(const BackwardCall& c) {
   RetentionCall calls[kRuns];
   tc_calls(c, static_cast<char*>(c.ws), tc_layout(c.dims), calls);
-  int n = 2 + 2 + (c.state_in ? 1 : 0) + (c.dstate ? 1 : 0);
+  int n = 2 + 1 + (c.state_in ? 1 : 0) + (c.dstate ? 1 : 0);
   for (int i = 0; i < kRuns; ++i) n += tc_chunkwise_launches(calls[i]);
   return n;
 }

@@ -60,6 +60,7 @@ struct TcArgs {
   int nb;     // sub-blocks of T rows per chunk (pipelined kernel)
   int batch;
   int v_f16;  // value rows arrive as fp16 (the converters leave V alone)
+  int o_rev;  // output row of token t written at token L - 1 - t (plain epilogue only)
   // Fused MSR epilogue: out = GroupNorm_h(o) * swish(gate), written to o's place.
   const void* gate;
   float eps;
@@ -1646,7 +1647,8 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL, PS>::THREADS, 
       float f = row_factor_f32(gam, sd, a.pos0 + t, a.flags) / sd;
       if (a.rden && my_row >= 0 && my_row < rows) f *= __ldg(a.rden + (static_cast<int64_t>(b) * a.L + t) * a.heads + h);
       const float gx = (nb > 1) ? exp2f(static_cast<float>(u * T) * log2g) : 0.f;
-      Tout* dst = static_cast<Tout*>(a.o) + ((static_cast<int64_t>(b) * a.L + t) * a.heads + h) * a.dv + dvb * DVS;
+      const int t_out = a.o_rev ? a.L - 1 - t : t;
+      Tout* dst = static_cast<Tout*>(a.o) + ((static_cast<int64_t>(b) * a.L + t_out) * a.heads + h) * a.dv + dvb * DVS;
       // O (and X) from TMEM, o = (O + gamma^(uT) X) * s / c_p, 16-byte stores of 16 columns.
       auto store16 = [&](int q, const float (&ov)[16]) {
         if constexpr (sizeof(Tout) == 2) {
@@ -2473,6 +2475,7 @@ TcArgs make_args(const RetentionCall& c, int n_chunks, int nb) {
   a.flags = c.flags;
   a.nb = nb;
   a.v_f16 = c.v_f16 ? 1 : 0;
+  a.o_rev = c.o_rev ? 1 : 0;
   a.n_seg = 1;
   a.n_sub = 0;
   for (int s = 0; s < 4; ++s) a.seg_lo[s] = a.seg_hi[s] = a.sub_before[s] = 0;
@@ -2767,6 +2770,8 @@ bool tc_chunkwise_supported(const RetentionCall& c) {
   // fp16 value rows: the pipelined kernel's converters only (no pre-pass, split operands or
   // fused epilogue), values of 64 or 128 columns a CTA
   if (c.v_f16 && (c.precise || c.gate || c.rden)) return false;
+  // reversed output rows: the pipelined kernel's plain epilogue only
+  if (c.o_rev && (c.gate || force_serial_kernel())) return false;
   if (d.seqlen < 1 || d.seqlen > (1LL << 30) || d.heads > 65535 || d.batch > 65535) return false;
   if (!aligned16(c.q) || !aligned16(c.k) || !aligned16(c.v) || !aligned16(c.o)) return false;
   if ((c.state_in && !aligned16(c.state_in)) || (c.state_out && !aligned16(c.state_out))) return false;

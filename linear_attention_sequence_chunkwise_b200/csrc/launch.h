@@ -42,6 +42,9 @@ struct RetentionCall {
   // Value rows already in fp16 (in_dtype still describes q and k): the gradient's runs, whose
   // values are not bf16 numbers.  The pipelined kernel's converters leave V as it is.
   bool v_f16 = false;
+  // Output row of token t written at token L - 1 - t (internal: the gradient's dv run, whose
+  // sequence is reversed, writes dv in forward order).
+  bool o_rev = false;
 };
 
 // Sequence segments of the key-sum pass, at most; and the workspace bytes of the R~ factors
