@@ -1612,12 +1612,18 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL, PS>::THREADS, 
     const int gwarp = is_epi ? warp - C::WARP_EPI0 : warp;
     const uint32_t lane_off = static_cast<uint32_t>(32 * gwarp) << 16;
     const int my_row = (T == 128) ? 32 * gwarp + lane : (lane < 16 ? 16 * gwarp + lane : -1);
+    // With T = 64 (rows in lanes 0-15) the scores and the plain epilogue take each row on two
+    // threads: lane l and l + 16 hold row 16 gwarp + (l mod 16), columns of half phalf.
+    constexpr bool HALVES = T == 64;
+    const int prow = HALVES ? 16 * gwarp + (lane & 15) : my_row;
+    const int phalf = HALVES ? (lane >> 4) : 0;
     const float gam = hp.gamma[h];
     // Epilogue of row block (chunk i, block u), O/X buffer rb & 1.
     auto epilogue = [&](int rb, int i, int u, int bl) -> bool {
       const int rows = min(T, bl - u * T);
-      const bool live = my_row >= 0 && my_row < rows;
-      const int t = i * nb * T + u * T + (my_row < 0 ? 0 : my_row);
+      const int row = FUSE ? my_row : prow;  // this thread's row (the fused epilogue keeps its own split)
+      const bool live = row >= 0 && row < rows;
+      const int t = i * nb * T + u * T + (row < 0 ? 0 : row);
       // FUSE output rows and columns of this lane.  With T = 64 the rows sit in lanes 0-15 of
       // each warp; lane l + 16 then writes the upper half of the columns of lane l's row.
       constexpr bool SPLIT = FUSE && T == 64;
@@ -1645,7 +1651,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL, PS>::THREADS, 
       if (!__all_sync(0xffffffffu, mbar_wait(bar(Q_O_FULL + (rb & 1)), (rb >> 1) & 1))) return false;
       tc_fence_after();
       float f = row_factor_f32(gam, sd, a.pos0 + t, a.flags) / sd;
-      if (a.rden && my_row >= 0 && my_row < rows) f *= __ldg(a.rden + (static_cast<int64_t>(b) * a.L + t) * a.heads + h);
+      if (a.rden && live) f *= __ldg(a.rden + (static_cast<int64_t>(b) * a.L + t) * a.heads + h);
       const float gx = (nb > 1) ? exp2f(static_cast<float>(u * T) * log2g) : 0.f;
       const int t_out = a.o_rev ? a.L - 1 - t : t;
       Tout* dst = static_cast<Tout*>(a.o) + ((static_cast<int64_t>(b) * a.L + t_out) * a.heads + h) * a.dv + dvb * DVS;
@@ -1780,7 +1786,34 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL, PS>::THREADS, 
         }
         return true;
       }
-      if (C::XBUF == 0 || nb == 1) {
+      if constexpr (HALVES) {
+        // Each thread: half phalf of its row's DVS columns, 32 at a time (O, and X with nb > 1).
+        constexpr int HC = DVS / 2;
+#pragma unroll 1
+        for (int grp = 0; grp < HC / 32; ++grp) {
+          uint32_t uo[2][16], ux[2][16];
+          if (C::XBUF > 0 && nb > 1) {
+            tmem_ld16x2_wait<HC>(tO + 32 * grp, uo, tX + 32 * grp, ux);
+          } else {
+            tmem_ld16x2_wait<HC>(tO + 32 * grp, uo);
+          }
+          if (grp == HC / 32 - 1) {
+            tc_fence_before();
+            mbar_arrive(bar(Q_O_FREE + (rb & 1)));
+          }
+          if (live) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              float ov[16];
+#pragma unroll
+              for (int c = 0; c < 16; ++c)
+                ov[c] = (C::XBUF > 0 && nb > 1) ? f * fmaf(gx, __uint_as_float(ux[e][c]), __uint_as_float(uo[e][c]))
+                                                : f * __uint_as_float(uo[e][c]);
+              store16((phalf * HC + 32 * grp) / 16 + e, ov);
+            }
+          }
+        }
+      } else if (C::XBUF == 0 || nb == 1) {
         // No cross accumulator: O alone, LDW columns per load.
 #pragma unroll
         for (int grp = 0; grp < DVS / C::LDW; ++grp) {
@@ -1844,8 +1877,35 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL, PS>::THREADS, 
       const float pf = exp2f(static_cast<float>((it.u - it.w - 1) * T) * log2g) * sd;
       const bool diag = (it.u == it.w);
       const uint32_t tS = tmem + C::COL_S + (k % C::SBUF) * T + lane_off;
+      if constexpr (HALVES) {
+        // row prow, columns [32 phalf, 32 phalf + 32) of the 64-column score tile
+        uint32_t u16[2][16];
+        tmem_ld16x2_wait<32>(tS, u16);
+        tc_fence_before();
+        mbar_arrive(bar(Q_S_FREE + (k % C::SBUF)));
 #pragma unroll
-      for (int grp = 0; grp < T / C::LDW; ++grp) {
+        for (int c8 = 0; c8 < 4; ++c8) {
+          const int col = 32 * phalf + 8 * c8;
+          uint32_t pk[4], pl[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c0 = col + 2 * e;
+            const float p0 = (!diag || c0 <= prow) ? __uint_as_float(u16[c8 / 2][(8 * c8 + 2 * e) % 16]) * pf : 0.f;
+            const float p1 = (!diag || c0 + 1 <= prow) ? __uint_as_float(u16[c8 / 2][(8 * c8 + 2 * e + 1) % 16]) * pf : 0.f;
+            pmx = absmax(absmax(pmx, p0), p1);
+            if (HL) {
+              split_f16x2(p0, p1, pk[e], pl[e]);
+            } else {
+              pk[e] = pack_f16x2(p0, p1);
+            }
+          }
+          const uint32_t poff = sw128(prow, col / 8);
+          st_shared_v4(sP(k) + poff, pk[0], pk[1], pk[2], pk[3]);
+          if (HL) st_shared_v4(sP(k) + C::PBYTES + poff, pl[0], pl[1], pl[2], pl[3]);
+        }
+      }
+#pragma unroll
+      for (int grp = 0; grp < (HALVES ? 0 : T / C::LDW); ++grp) {
         uint32_t u16[C::LDW / 16][16];
         tmem_ld_wait(tS + grp * C::LDW, u16);
         if (grp == T / C::LDW - 1) {

@@ -291,6 +291,29 @@ __device__ __forceinline__ void tmem_ld_wait(uint32_t taddr, uint32_t (&r)[2][16
       : "memory");
 }
 
+// M = 64 accumulator tiles keep their rows in lanes 0-15 of each lane quarter.  This load
+// gives every thread of the warp 32 columns of one of those rows: thread i < 16 row i, columns
+// [c, c + 32); thread i + 16 row i, columns [c + OFF, c + OFF + 32) (c = the address's column).
+template <int OFF>
+__device__ __forceinline__ void tmem_ld16x2_wait(uint32_t taddr, uint32_t (&r)[2][16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32], %33; tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0][0]), "=r"(r[0][1]), "=r"(r[0][2]), "=r"(r[0][3]), "=r"(r[0][4]), "=r"(r[0][5]), "=r"(r[0][6]), "=r"(r[0][7]), "=r"(r[0][8]), "=r"(r[0][9]), "=r"(r[0][10]), "=r"(r[0][11]), "=r"(r[0][12]), "=r"(r[0][13]), "=r"(r[0][14]), "=r"(r[0][15]), "=r"(r[1][0]), "=r"(r[1][1]), "=r"(r[1][2]), "=r"(r[1][3]), "=r"(r[1][4]), "=r"(r[1][5]), "=r"(r[1][6]), "=r"(r[1][7]), "=r"(r[1][8]), "=r"(r[1][9]), "=r"(r[1][10]), "=r"(r[1][11]), "=r"(r[1][12]), "=r"(r[1][13]), "=r"(r[1][14]), "=r"(r[1][15])
+      : "r"(taddr), "n"(OFF)
+      : "memory");
+}
+
+// The same from two addresses (two accumulators of the same layout), one wait.
+template <int OFF>
+__device__ __forceinline__ void tmem_ld16x2_wait(uint32_t ta, uint32_t (&ra)[2][16], uint32_t tb, uint32_t (&rb)[2][16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%64], %66; "
+      "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 {%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%65], %66; tcgen05.wait::ld.sync.aligned;"
+      : "=r"(ra[0][0]), "=r"(ra[0][1]), "=r"(ra[0][2]), "=r"(ra[0][3]), "=r"(ra[0][4]), "=r"(ra[0][5]), "=r"(ra[0][6]), "=r"(ra[0][7]), "=r"(ra[0][8]), "=r"(ra[0][9]), "=r"(ra[0][10]), "=r"(ra[0][11]), "=r"(ra[0][12]), "=r"(ra[0][13]), "=r"(ra[0][14]), "=r"(ra[0][15]), "=r"(ra[1][0]), "=r"(ra[1][1]), "=r"(ra[1][2]), "=r"(ra[1][3]), "=r"(ra[1][4]), "=r"(ra[1][5]), "=r"(ra[1][6]), "=r"(ra[1][7]), "=r"(ra[1][8]), "=r"(ra[1][9]), "=r"(ra[1][10]), "=r"(ra[1][11]), "=r"(ra[1][12]), "=r"(ra[1][13]), "=r"(ra[1][14]), "=r"(ra[1][15]), "=r"(rb[0][0]), "=r"(rb[0][1]), "=r"(rb[0][2]), "=r"(rb[0][3]), "=r"(rb[0][4]), "=r"(rb[0][5]), "=r"(rb[0][6]), "=r"(rb[0][7]), "=r"(rb[0][8]), "=r"(rb[0][9]), "=r"(rb[0][10]), "=r"(rb[0][11]), "=r"(rb[0][12]), "=r"(rb[0][13]), "=r"(rb[0][14]), "=r"(rb[0][15]), "=r"(rb[1][0]), "=r"(rb[1][1]), "=r"(rb[1][2]), "=r"(rb[1][3]), "=r"(rb[1][4]), "=r"(rb[1][5]), "=r"(rb[1][6]), "=r"(rb[1][7]), "=r"(rb[1][8]), "=r"(rb[1][9]), "=r"(rb[1][10]), "=r"(rb[1][11]), "=r"(rb[1][12]), "=r"(rb[1][13]), "=r"(rb[1][14]), "=r"(rb[1][15])
+      : "r"(ta), "r"(tb), "n"(OFF)
+      : "memory");
+}
+
 // 64 columns.
 __device__ __forceinline__ void tmem_ld_wait(uint32_t taddr, uint32_t (&r)[4][16]) {
   asm volatile(
