@@ -1621,7 +1621,8 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL, PS>::THREADS, 
     // Epilogue of row block (chunk i, block u), O/X buffer rb & 1.
     auto epilogue = [&](int rb, int i, int u, int bl) -> bool {
       const int rows = min(T, bl - u * T);
-      const int row = FUSE ? my_row : prow;  // this thread's row (the fused epilogue keeps its own split)
+      // this thread's row: with T = 64 lanes l and l + 16 share row 16 gwarp + (l mod 16)
+      const int row = prow;
       const bool live = row >= 0 && row < rows;
       const int t = i * nb * T + u * T + (row < 0 ? 0 : row);
       // FUSE output rows and columns of this lane.  With T = 64 the rows sit in lanes 0-15 of
@@ -1687,29 +1688,57 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL, PS>::THREADS, 
         // its writer has seen every CTA's statistics of row block rb + 1, which each CTA sends
         // after it has finished reading the slot for row block rb: two slots need no release
         // barrier.
-        float y[DVS];
-#pragma unroll
-        for (int grp = 0; grp < DVS / 32; ++grp) {
+        // yv: this lane's EC columns of its row (with T = 64 each lane loads its half directly
+        // and the row's sum and M2 combine across lanes l and l + 16)
+        float yv[EC];
+        float mean_i = 0.f, m2 = 0.f;
+        if constexpr (SPLIT) {
+          static_assert(EC == 32, "the split epilogue takes 64-column slices");
           uint32_t uo[2][16], ux[2][16];
           if (C::XBUF > 0 && nb > 1) {
-            tmem_ld_wait(tO + 32 * grp, uo, tX + 32 * grp, ux);
+            tmem_ld16x2_wait<32>(tO, uo, tX, ux);
           } else {
-            tmem_ld_wait(tO + 32 * grp, uo);
+            tmem_ld16x2_wait<32>(tO, uo);
           }
+          tc_fence_before();
+          mbar_arrive(bar(Q_O_FREE + (rb & 1)));
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
             const float ov = __uint_as_float(uo[c / 16][c % 16]);
-            y[32 * grp + c] = (C::XBUF > 0 && nb > 1) ? f * fmaf(gx, __uint_as_float(ux[c / 16][c % 16]), ov) : f * ov;
+            yv[c] = (C::XBUF > 0 && nb > 1) ? f * fmaf(gx, __uint_as_float(ux[c / 16][c % 16]), ov) : f * ov;
+            mean_i += yv[c];
           }
+          mean_i += __shfl_xor_sync(0xffffffffu, mean_i, 16);
+          mean_i *= 1.f / DVS;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) m2 = fmaf(yv[c] - mean_i, yv[c] - mean_i, m2);
+          m2 += __shfl_xor_sync(0xffffffffu, m2, 16);
+        } else {
+          float y[DVS];
+#pragma unroll
+          for (int grp = 0; grp < DVS / 32; ++grp) {
+            uint32_t uo[2][16], ux[2][16];
+            if (C::XBUF > 0 && nb > 1) {
+              tmem_ld_wait(tO + 32 * grp, uo, tX + 32 * grp, ux);
+            } else {
+              tmem_ld_wait(tO + 32 * grp, uo);
+            }
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              const float ov = __uint_as_float(uo[c / 16][c % 16]);
+              y[32 * grp + c] = (C::XBUF > 0 && nb > 1) ? f * fmaf(gx, __uint_as_float(ux[c / 16][c % 16]), ov) : f * ov;
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(bar(Q_O_FREE + (rb & 1)));
+#pragma unroll
+          for (int c = 0; c < DVS; ++c) mean_i += y[c];
+          mean_i *= 1.f / DVS;
+#pragma unroll
+          for (int c = 0; c < DVS; ++c) m2 = fmaf(y[c] - mean_i, y[c] - mean_i, m2);
+#pragma unroll
+          for (int c = 0; c < EC; ++c) yv[c] = y[c];
         }
-        tc_fence_before();
-        mbar_arrive(bar(Q_O_FREE + (rb & 1)));
-        float mean_i = 0.f, m2 = 0.f;
-#pragma unroll
-        for (int c = 0; c < DVS; ++c) mean_i += y[c];
-        mean_i *= 1.f / DVS;
-#pragma unroll
-        for (int c = 0; c < DVS; ++c) m2 = fmaf(y[c] - mean_i, y[c] - mean_i, m2);
         const int slot = rb & 1;
         const uint32_t me = cluster_ctarank();
         if (gwarp == 0 && lane == 0) mbar_arrive_expect_tx(bar(Q_XFULL + slot), static_cast<uint32_t>(n_cl * T * 8));
@@ -1719,17 +1748,6 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL, PS>::THREADS, 
                         map_shared_rank(bar(Q_XFULL + slot), pr));
         }
         if (!__all_sync(0xffffffffu, mbar_wait_cluster(bar(Q_XFULL + slot), (rb >> 1) & 1))) return false;
-        // this lane's EC columns of the row
-        float yv[EC];
-#pragma unroll
-        for (int c = 0; c < EC; ++c) {
-          if constexpr (SPLIT) {
-            const float up = __shfl_up_sync(0xffffffffu, y[EC + c], 16);
-            yv[c] = lane >= 16 ? up : y[c];
-          } else {
-            yv[c] = y[c];
-          }
-        }
         if (elive) {
           // gate loads in flight together where registers allow (half rows), else 16 columns at a time
           uint4 gv[SPLIT ? EC / 8 : 2];
