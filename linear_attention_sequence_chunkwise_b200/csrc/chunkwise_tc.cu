@@ -1351,7 +1351,7 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL, PS>::THREADS, 
         }
         if (progress) {
           idle_since = clock64();
-        } else if (clock64() - idle_since > *const_cast<volatile long long*>(&g_wait_budget)) {
+        } else if (clock64() - idle_since > g_wait_budget) {
           atomicAdd(&g_wait_timeouts, 1u);  // same bound and report as a blocking wait
           break;
         }

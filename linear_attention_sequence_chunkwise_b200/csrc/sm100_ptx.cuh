@@ -72,7 +72,10 @@ static __device__ unsigned int g_wait_timeouts = 0;
 // issued (TMA loads, MMAs) always take kDrainBudget, so a kernel that gave up never leaves with
 // copies or products in flight.
 constexpr long long kDrainBudget = 4000000000LL;
-static __device__ long long g_wait_budget = kDrainBudget;
+// In constant memory: every bounded wait (and the MMA issuer's polling loop) reads it, and a
+// global-memory read there put a memory latency into the wait for an mbarrier phase.  The host
+// changes it only between launches (retnet_debug_set_wait_budget synchronises first).
+static __constant__ long long g_wait_budget = kDrainBudget;
 // Threads that rounded a value outside the fp16 range (magnitude >= 65520 becomes inf, or NaN)
 // when forming a tensor-core operand: bf16 inputs span a far wider range than fp16 operands.
 static __device__ unsigned int g_fp16_overflows = 0;
@@ -136,7 +139,7 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
     return ok != 0;
   };
   if (probe()) return true;
-  if (budget < 0) budget = *const_cast<volatile long long*>(&g_wait_budget);
+  if (budget < 0) budget = g_wait_budget;
   const long long t0 = clock64();
   while (!probe()) {
     if (clock64() - t0 > budget) {
@@ -153,7 +156,7 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
 // if it gave up.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long long budget = -1) {
   if (mbar_try_wait(bar, parity)) return true;
-  if (budget < 0) budget = *const_cast<volatile long long*>(&g_wait_budget);
+  if (budget < 0) budget = g_wait_budget;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
     if (clock64() - t0 > budget) {
