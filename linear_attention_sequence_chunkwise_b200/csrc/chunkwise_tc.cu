@@ -2364,6 +2364,159 @@ __global__ void __launch_bounds__(160, 1) tc_p_kernel(const __grid_constant__ CU
   }
 }
 
+// P pass, one CTA a (chunk, batch x head): the same tiles as tc_p_kernel, computed in turn by a
+// pipeline that keeps its operands on chip -- Q_u in one of two slots for the units of row block
+// u, K_w through a ring of three -- so that the launch, the tensor-memory set-up and the first
+// loads' latency are paid once a chunk rather than once a tile.  Warp 4 loads (TMA), warp 5
+// issues the MMAs into one of two tensor-memory score buffers, warps 0-3 scale, mask and store
+// (two threads a row, each 32 columns).  Same arithmetic as tc_p_kernel: bit-identical tiles.
+constexpr int kPChunkK = 3;  // K tiles in flight (two Q slots, three K slots: 160 KB at d_k 256; five ran no faster)
+template <int DK, int T>
+__global__ void __launch_bounds__(192, 1) tc_p_chunk_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                                            const __grid_constant__ CUtensorMap tm_k,
+                                                            uint4* __restrict__ P, int L, int heads, int n_chunks,
+                                                            int nb, HeadParams hp) {
+  static_assert(T == 64, "P pass: 64-row sub-blocks");
+  constexpr int QB = T * DK * 2;
+  constexpr int NQ = 2, NK = kPChunkK;
+  enum : int { B_QF = 0, B_QE = 2, B_KF = 4, B_KE = 4 + NK, B_SF = 4 + 2 * NK, B_SE = 6 + 2 * NK, B_DR = 8 + 2 * NK,
+               NB_ = 9 + 2 * NK };
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_addr(smem_raw);
+  const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (sbase - raw_addr);
+  auto sQ = [&](int j) { return sbase + j * QB; };
+  auto sK = [&](int j) { return sbase + (NQ + j) * QB; };
+  uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + (NQ + NK) * QB);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + NB_);
+  auto bar = [&](int j) { return smem_addr(bars + j); };
+  const int U = nb * (nb + 1) / 2;
+  const int i = blockIdx.x, bh = blockIdx.y;
+  const int h = bh % heads, b = bh / heads;
+  const int t0 = i * nb * T;
+  const int nbw = min(nb, (L - t0 + T - 1) / T);  // row blocks of this chunk inside the sequence
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (threadIdx.x == 0) {
+    for (int j = 0; j < NB_; ++j) mbar_init(bar(j), (j == B_SE || j == B_SE + 1) ? 128 : 1);
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_addr(tmem_holder), 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const float log2g = hp.log2g[h];
+  if (warp == 4) {
+    if (lane == 0) {
+      prefetch_tensormap(&tm_q);
+      prefetch_tensormap(&tm_k);
+      int k = 0, q_issued[NQ] = {0, 0}, k_issued[NK] = {};
+      bool ok = true;
+      for (int u = 0; ok && u < nbw; ++u) {
+        const int qs = u % NQ;
+        if (u >= NQ && !mbar_wait(bar(B_QE + qs), ((u / NQ) - 1) & 1)) break;
+        mbar_arrive_expect_tx(bar(B_QF + qs), QB);
+#pragma unroll
+        for (int bx = 0; bx < DK / 64; ++bx) tma_load_4d(sQ(qs) + bx * T * 128, &tm_q, bar(B_QF + qs), bx * 64, h, t0 + u * T, b);
+        q_issued[qs]++;
+        for (int w = 0; w <= u; ++w, ++k) {
+          const int ks = k % NK;
+          if (k >= NK && !mbar_wait(bar(B_KE + ks), ((k / NK) - 1) & 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(B_KF + ks), QB);
+#pragma unroll
+          for (int bx = 0; bx < DK / 64; ++bx)
+            tma_load_4d(sK(ks) + bx * T * 128, &tm_k, bar(B_KF + ks), bx * 64, h, t0 + w * T, b);
+          k_issued[ks]++;
+        }
+      }
+      // every load this thread issued lands before the CTA may exit
+      for (int j = 0; j < NQ; ++j)
+        if (q_issued[j] > 0) mbar_wait(bar(B_QF + j), (q_issued[j] - 1) & 1, kDrainBudget);
+      for (int j = 0; j < NK; ++j)
+        if (k_issued[j] > 0) mbar_wait(bar(B_KF + j), (k_issued[j] - 1) & 1, kDrainBudget);
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      constexpr uint32_t ID_S = idesc_f16_f32(T, T, 0, 0);
+      int k = 0;
+      bool ok = true;
+      for (int u = 0; ok && u < nbw; ++u) {
+        const int qs = u % NQ;
+        if (!mbar_wait(bar(B_QF + qs), (u / NQ) & 1)) break;
+        for (int w = 0; w <= u; ++w, ++k) {
+          const int ks = k % NK, sb = k % 2;
+          ok = mbar_wait(bar(B_KF + ks), (k / NK) & 1);
+          if (ok && k >= 2) ok = mbar_wait(bar(B_SE + sb), ((k / 2) - 1) & 1);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t dq = sdesc_sw128(sQ(qs), 16, 1024), dk = sdesc_sw128(sK(ks), 16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < DK / 16; ++kk) {
+            const uint64_t kst = static_cast<uint64_t>(((kk / 4) * T * 128 + (kk % 4) * 32) >> 4);
+            mma_f16_ss(tmem + sb * T, dq + kst, dk + kst, ID_S, kk > 0);
+          }
+          mma_commit(bar(B_SF + sb));
+          mma_commit(bar(B_KE + ks));
+        }
+        mma_commit(bar(B_QE + qs));
+      }
+      mma_commit(bar(B_DR));
+      mbar_wait(bar(B_DR), 0, kDrainBudget);
+    }
+  } else {
+    // rows of the M = 64 score tile: lanes 0-15 of each warp's lane quarter; lanes l and l + 16
+    // take row 16 warp + (l mod 16), columns [32 (l / 16), 32 (l / 16) + 32)
+    const uint32_t lane_off = static_cast<uint32_t>(32 * warp) << 16;
+    const int prow = 16 * warp + (lane & 15), phalf = lane >> 4;
+    const float sdk = rsqrtf(static_cast<float>(DK));
+    float pmx = 0.f;
+    int k = 0;
+    bool ok = true;
+    for (int u = 0; ok && u < nbw; ++u) {
+      for (int w = 0; w <= u; ++w, ++k) {
+        const int sb = k % 2;
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SF + sb), (k / 2) & 1));
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t r[2][16];
+        tmem_ld16x2_wait<32>(tmem + sb * T + lane_off, r);
+        tc_fence_before();
+        mbar_arrive(bar(B_SE + sb));
+        const float pf = exp2f(static_cast<float>((u - w - 1) * T) * log2g) * sdk;
+        const bool diag = (u == w);
+        const int64_t tile = (static_cast<int64_t>(bh) * n_chunks + i) * U + u * (u + 1) / 2 + w;
+        uint4* dst = P + (tile * T + prow) * (T * 2 / 16) + 4 * phalf;
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = 8 * c8 + 2 * e, c0 = 32 * phalf + c;
+            const float p0 = (!diag || c0 <= prow) ? __uint_as_float(r[c / 16][c % 16]) * pf : 0.f;
+            const float p1 = (!diag || c0 + 1 <= prow) ? __uint_as_float(r[(c + 1) / 16][(c + 1) % 16]) * pf : 0.f;
+            pmx = absmax(absmax(pmx, p0), p1);
+            pk[e] = pack_f16x2(p0, p1);
+          }
+          dst[c8] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+      }
+    }
+    report_fp16_range(pmx);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
 // ---- host side -------------------------------------------------------------------------------
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -2476,6 +2629,11 @@ int64_t p_tiles(const Dims& d, int64_t chunk, int T) {
 }
 size_t p_tile_bytes(const Dims& d, int64_t chunk, int T) {
   return align256(static_cast<size_t>(p_tiles(d, chunk, T)) * T * T * 2);
+}
+// Which P-pass kernel: one CTA a chunk (its tiles pipelined) or one CTA a tile.
+bool use_p_chunk_kernel(int nb) {
+  const char* e = getenv("RETNET_P_TILE_KERNEL");  // testing aid: force the per-tile kernel
+  return !(e && e[0] == '1') && nb >= 4;  // chunk 128 (two sub-blocks): the per-tile kernel was faster
 }
 bool p_pass_applies(const RetentionCall& c, int T, int nb, int n_seg) {
   if (c.dims.d_k != 256 || T != 64 || nb < 2 || c.precise || c.gate || n_seg >= 2 || !c.ws) return false;
@@ -2724,13 +2882,23 @@ cudaError_t launch_pipe(const RetentionCall& c, const HeadParams& hp, cudaStream
             void* ptiles = static_cast<char*>(c.ws) + pre_copy_bytes(c.dims, false);
             const int64_t n_chunks = (c.dims.seqlen + c.chunk - 1) / c.chunk;
             const int U = nb * (nb + 1) / 2;
-            constexpr int PSMEM = 2 * T * DK * 2 + 1024 + 64;
-            e = cudaFuncSetAttribute(tc_p_kernel<DK, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, PSMEM);
-            if (e != cudaSuccess) return e;
-            tc_p_kernel<DK, T><<<dim3(U, static_cast<unsigned>(n_chunks), static_cast<unsigned>(c.dims.batch * c.dims.heads)),
-                                 160, PSMEM, s>>>(pm[0], pm[1], static_cast<uint4*>(ptiles),
-                                                  static_cast<int>(c.dims.seqlen), static_cast<int>(c.dims.heads),
-                                                  static_cast<int>(n_chunks), nb, hp);
+            if (use_p_chunk_kernel(nb)) {  // one CTA a chunk, operands pipelined on chip
+              constexpr int PCSMEM = (2 + kPChunkK) * T * DK * 2 + 1024 + (9 + 2 * kPChunkK) * 8 + 16;
+              e = cudaFuncSetAttribute(tc_p_chunk_kernel<DK, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, PCSMEM);
+              if (e != cudaSuccess) return e;
+              tc_p_chunk_kernel<DK, T><<<dim3(static_cast<unsigned>(n_chunks), static_cast<unsigned>(c.dims.batch * c.dims.heads)),
+                                         192, PCSMEM, s>>>(pm[0], pm[1], static_cast<uint4*>(ptiles),
+                                                           static_cast<int>(c.dims.seqlen), static_cast<int>(c.dims.heads),
+                                                           static_cast<int>(n_chunks), nb, hp);
+            } else {  // one CTA a tile
+              constexpr int PSMEM = 2 * T * DK * 2 + 1024 + 64;
+              e = cudaFuncSetAttribute(tc_p_kernel<DK, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, PSMEM);
+              if (e != cudaSuccess) return e;
+              tc_p_kernel<DK, T><<<dim3(U, static_cast<unsigned>(n_chunks), static_cast<unsigned>(c.dims.batch * c.dims.heads)),
+                                   160, PSMEM, s>>>(pm[0], pm[1], static_cast<uint4*>(ptiles),
+                                                    static_cast<int>(c.dims.seqlen), static_cast<int>(c.dims.heads),
+                                                    static_cast<int>(n_chunks), nb, hp);
+            }
             e = cudaGetLastError();
             if (e != cudaSuccess) return e;
             if (!make_map_p(&pm[3], ptiles, p_tiles(c.dims, c.chunk, T), T)) return cudaErrorInvalidValue;

@@ -4,6 +4,8 @@ Bar: max|err|/rms(oracle) <= 1e-2 on the raw output (the bf16-input tolerance); 
 state hand-off is held to the same bar.  Every case asserts first that the call takes
 the tensor-core kernel, and last that no bounded wait inside it gave up.
 """
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -432,7 +434,8 @@ def test_tc_p_pass_matches_oracle(dv, B, L, pos0, with_state):
     tile once per head into the workspace and the pipelined kernel loads them beside V (three
     launches: conversion pre-pass, P pass, kernel).  Against the oracle, and bit-identical to the
     same call with a workspace one byte too small for the P tiles (the kernel then forms P itself
-    from the same operands, in the same order)."""
+    from the same operands, in the same order) and to the same call with the one-CTA-a-tile P
+    kernel (RETNET_P_TILE_KERNEL=1) in place of the one-CTA-a-chunk kernel."""
     b, h, dk = 2, 3, 256
     q, k, v = si.qkv(b, L, h, dk, dv, 1800 + B + L, "bf16")
     g, th = si.gamma_schedule(h), si.theta_schedule(dk)
@@ -446,15 +449,21 @@ def test_tc_p_pass_matches_oracle(dv, B, L, pos0, with_state):
     assert rn.retnet_chunkwise_launches((b, L, h, dk), dv, rn.BF16, FLAGS, B, g, full) == 3
     assert rn.retnet_chunkwise_launches((b, L, h, dk), dv, rn.BF16, FLAGS, B, g, small) == 2
     outs = []
-    for nbytes in (full, small):
+    for nbytes, tile_kernel in ((full, False), (small, False), (full, True)):
         ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
         o = torch.empty(b, L, h, dv, device="cuda")
         so = torch.empty(b, h, dk, dv, device="cuda")
-        rn.retnet_retention_chunkwise_ws(dev(q), dev(k), dev(v), o, g, th, pos0, FLAGS, B,
-                                         None if S0 is None else dev(S0), so, workspace=ws)
-        torch.cuda.synchronize()
+        if tile_kernel:
+            os.environ["RETNET_P_TILE_KERNEL"] = "1"
+        try:
+            rn.retnet_retention_chunkwise_ws(dev(q), dev(k), dev(v), o, g, th, pos0, FLAGS, B,
+                                             None if S0 is None else dev(S0), so, workspace=ws)
+            torch.cuda.synchronize()
+        finally:
+            os.environ.pop("RETNET_P_TILE_KERNEL", None)
         outs.append((o, so))
     e, es = err(outs[0][0], ref), err(outs[0][1], Sref)
     print(f"P pass dv={dv} B={B} L={L}: out {e:.3e}, state {es:.3e}")
     assert e <= TOL_BF16 and es <= TOL_BF16
-    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+    for o2, s2 in outs[1:]:
+        assert torch.equal(outs[0][0], o2) and torch.equal(outs[0][1], s2)
