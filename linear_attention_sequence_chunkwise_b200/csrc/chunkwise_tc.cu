@@ -872,17 +872,20 @@ struct UnitConverter {
       Zq[jj] = make_float2(xstep * Z[jj].x, xstep * Z[jj].y);
       Zk[jj] = make_float2(zstep * Z[jj].x, zstep * Z[jj].y);
     }
+    // rows a load batch: split operands and 128-row units (more live values a row) ran faster
+    // with two (1.13x and 1.05x) and the plain 64-row path the same with two or four
+    constexpr int GB = (HL || T == 128) ? (NR < 2 ? NR : 2) : G;
 #pragma unroll 1
-    for (int kg = 0; kg < NR; kg += G) {
-      uint32_t q4[G][4], k4[G][4];
+    for (int kg = 0; kg < NR; kg += GB) {
+      uint32_t q4[GB][4], k4[GB][4];
 #pragma unroll
-      for (int k = 0; k < G; ++k) {
+      for (int k = 0; k < GB; ++k) {
         const uint32_t off = box + sw128(r0 + RS * (kg + k), chunk);
         if (WITH_Q) ld_shared_v4(sq + off, q4[k][0], q4[k][1], q4[k][2], q4[k][3]);
         ld_shared_v4(sk + off, k4[k][0], k4[k][1], k4[k][2], k4[k][3]);
       }
 #pragma unroll
-      for (int k = 0; k < G; ++k) {
+      for (int k = 0; k < GB; ++k) {
         uint32_t qo[4], ko[4], ql[4], kl[4];
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
