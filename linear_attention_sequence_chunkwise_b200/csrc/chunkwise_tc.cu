@@ -1990,7 +1990,11 @@ __global__ void __launch_bounds__(Cfg3<DK, T, DVS, PRE, FUSE, HL, PS>::THREADS, 
 // CTA is bound by streaming and converting K and V.  Roles: eight converter warps (K rotated and
 // scaled, V to fp16; they also write W out at the end), a TMA warp, an MMA warp; stages hold K
 // and V only.  Output: ws fp32 [j][batch][heads][d_k][d_v] (slice columns of this CTA).
-template <int DK, int T, int DVS>
+// TWO: half the shared memory, two CTAs an SM (the state of a whole sequence shard, one CTA a
+// (batch, head, slice): a second resident CTA hides the fixed cost; 1663 -> 1578 us on the
+// b2/L8192/h16/d256/512 shard).  The two-pass segments keep one CTA an SM, which leaves SMs to
+// the first output segment.
+template <int DK, int T, int DVS, bool TWO = false>
 struct CfgS {
   static constexpr int NCW = 8;
   static constexpr int NCONV = 32 * NCW;
@@ -2003,7 +2007,7 @@ struct CfgS {
   static constexpr int STAGE = KBYTES + VBYTES;
   static constexpr int TABBYTES = 2 * 2 * (DK / 2) * 8;
   static constexpr int NBARS = 3 * 6 + 2 + 2;
-  static constexpr int BUDGET = 227 * 1024 - 1024;
+  static constexpr int BUDGET = (TWO ? 113 : 227) * 1024 - 1024;
   static constexpr int NS_FIT = (BUDGET - TABBYTES - NBARS * 8 - 16) / STAGE;
   static constexpr int NS = NS_FIT > 6 ? 6 : NS_FIT;
   static constexpr int SMEM = NS * STAGE + TABBYTES + NBARS * 8 + 16 + 1024;
@@ -2011,11 +2015,11 @@ struct CfgS {
   static_assert(NS >= 2, "segment-state stages");
 };
 
-template <int DK, int T, int DVS>
-__global__ void __launch_bounds__(CfgS<DK, T, DVS>::THREADS, 1)
+template <int DK, int T, int DVS, bool TWO = false>
+__global__ void __launch_bounds__(CfgS<DK, T, DVS, TWO>::THREADS, TWO ? 2 : 1)
     tc_segment_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                             TcArgs a, HeadParams hp) {
-  using C = CfgS<DK, T, DVS>;
+  using C = CfgS<DK, T, DVS, TWO>;
   enum : int { B_FULL = 0, B_CONV = 6, B_EMPTY = 12, B_TAB = 18, B_DONE = 20, B_DRAIN = 21 };
   griddep_launch_dependents();  // the output pass may start on the SMs this grid leaves idle
   extern __shared__ uint8_t smem_raw[];
@@ -3072,7 +3076,7 @@ cudaError_t tc_wait_timeouts(unsigned int* count, bool clear) {
 namespace {
 template <int DK, int T, typename Tout>
 cudaError_t launch_segment_state_t(const RetentionCall& c, const HeadParams& hp, cudaStream_t s) {
-  using Cf = CfgS<DK, T, 64>;
+  using Cf = CfgS<DK, T, 64, true>;
   CUtensorMap mq, mk, mv;
   // The state pass never loads Q: its map is built over K (a valid tensor of the same shape).
   RetentionCall cc = c;
@@ -3086,7 +3090,7 @@ cudaError_t launch_segment_state_t(const RetentionCall& c, const HeadParams& hp,
   a.sub_lo[0] = 0;
   a.sub_hi[0] = n_chunks;
   a.ws = c.state_out;  // sub-segment 0 of the workspace layout is [batch][heads][d_k][d_v]
-  auto kern = tc_segment_state_kernel<DK, T, 64>;
+  auto kern = tc_segment_state_kernel<DK, T, 64, true>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM);
   if (e != cudaSuccess) return e;
   kern<<<tc_grid(c.dims, 64), Cf::THREADS, Cf::SMEM, s>>>(mk, mv, a, hp);
